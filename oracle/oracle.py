@@ -1,0 +1,145 @@
+"""Float64 CPU oracle: ctypes wrapper around ``ssm_oracle.c``.
+
+TEST INFRASTRUCTURE ONLY.  The tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline / reference arm are the only callers.  The CUDA
+library never imports, links or runs anything here, and nothing here imports
+the CUDA library.
+
+What it computes (float64, plain sequential recurrence, zero initial state):
+
+    Delta_t  = softplus(delta_t + bias_d)            (softplus may be off)
+    h_t,n    = exp(Delta_t * A_d,n) * h_{t-1},n + Delta_t * B_t,n * u_t
+    y_t      = sum_n C_t,n * h_t,n + D_d * u_t
+    out_t    = y_t * silu(z_t)                       (z optional)
+
+following "超越注意力：探索Mamba与状态空间模型" (sections 状态空间模型基础,
+选择性状态空间模型, 代码实现概览) and "Mamba 与状态空间模型" (section 由词元决定).
+The update is the same single step applied to a given state.
+
+Every input is converted to contiguous float64 first; bf16 and fp32 values
+convert exactly, so the oracle sees the same numbers the GPU sees.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from pathlib import Path
+
+import numpy as np
+
+HERE = Path(__file__).resolve().parent
+SOURCE = HERE / "ssm_oracle.c"
+BUILD_DIR = HERE / "_build"
+LIBRARY = BUILD_DIR / "libssm_oracle.so"
+
+
+def build(source: Path = SOURCE, output: Path = LIBRARY, force: bool = False) -> Path:
+    """Compile the C oracle with gcc (-O2, OpenMP, no fast-math)."""
+    source, output = Path(source), Path(output)
+    if not force and output.exists() and output.stat().st_mtime >= source.stat().st_mtime:
+        return output
+    output.parent.mkdir(parents=True, exist_ok=True)
+    tmp = output.with_suffix(f".{os.getpid()}.tmp.so")
+    cmd = ["gcc", "-O2", "-std=c99", "-fopenmp", "-fPIC", "-shared",
+           str(source), "-o", str(tmp), "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, output)
+    return output
+
+
+def _f64(a):
+    """Contiguous float64 numpy copy of an array-like (numpy or CPU torch)."""
+    if a is None:
+        return None
+    if hasattr(a, "detach"):  # torch tensor
+        a = a.detach().to("cpu").double().numpy()
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+class Oracle:
+    """Handle on one compiled oracle library (the default one, or a test build)."""
+
+    def __init__(self, library: Path | str | None = None):
+        path = Path(library) if library is not None else build()
+        self.path = path
+        self._lib = ctypes.CDLL(str(path))
+        dp = ctypes.POINTER(ctypes.c_double)
+        i64 = ctypes.c_int64
+        self._lib.oracle_selective_scan_f64.restype = ctypes.c_int
+        self._lib.oracle_selective_scan_f64.argtypes = [
+            i64, i64, i64, i64, dp, dp, dp, dp, dp, dp, dp, dp, ctypes.c_int, dp, dp]
+        self._lib.oracle_selective_state_update_f64.restype = ctypes.c_int
+        self._lib.oracle_selective_state_update_f64.argtypes = [
+            i64, i64, i64, dp, dp, dp, dp, dp, dp, dp, dp, dp, ctypes.c_int, dp, dp]
+        self._lib.oracle_num_threads.restype = ctypes.c_int
+        self._lib.oracle_num_threads.argtypes = []
+
+    def num_threads(self) -> int:
+        return int(self._lib.oracle_num_threads())
+
+    def selective_scan(self, u, delta, A, B, C, D=None, z=None, delta_bias=None,
+                       softplus=True):
+        """Return (out, last_state) as float64 arrays.
+
+        u, delta, z: (batch, dim, L); B, C: (batch, N, L); A: (dim, N);
+        D, delta_bias: (dim,).  out: (batch, dim, L); last_state: (batch, dim, N).
+        """
+        u, delta, A, B, C = map(_f64, (u, delta, A, B, C))
+        D, z, delta_bias = map(_f64, (D, z, delta_bias))
+        batch, dim, seqlen = u.shape
+        dstate = A.shape[1]
+        assert delta.shape == u.shape and A.shape == (dim, dstate)
+        assert B.shape == (batch, dstate, seqlen) and C.shape == B.shape
+        assert z is None or z.shape == u.shape
+        assert D is None or D.shape == (dim,)
+        assert delta_bias is None or delta_bias.shape == (dim,)
+        out = np.empty_like(u)
+        last_state = np.empty((batch, dim, dstate), dtype=np.float64)
+        rc = self._lib.oracle_selective_scan_f64(
+            batch, dim, dstate, seqlen, _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C),
+            _ptr(D), _ptr(z), _ptr(delta_bias), int(bool(softplus)), _ptr(out),
+            _ptr(last_state))
+        if rc != 0:
+            raise ValueError(f"oracle_selective_scan_f64 returned {rc}")
+        return out, last_state
+
+    def selective_state_update(self, state, x, dt, A, B, C, D=None, z=None, dt_bias=None,
+                               dt_softplus=True):
+        """Return (new_state, out) as float64 arrays; the input state is not modified.
+
+        state: (batch, dim, N); x, dt, z: (batch, dim); B, C: (batch, N);
+        A: (dim, N); D, dt_bias: (dim,).
+        """
+        state, x, dt, A, B, C = map(_f64, (state, x, dt, A, B, C))
+        D, z, dt_bias = map(_f64, (D, z, dt_bias))
+        batch, dim, dstate = state.shape
+        assert x.shape == (batch, dim) and dt.shape == x.shape
+        assert A.shape == (dim, dstate) and B.shape == (batch, dstate) and C.shape == B.shape
+        assert z is None or z.shape == x.shape
+        new_state = np.empty_like(state)
+        out = np.empty_like(x)
+        rc = self._lib.oracle_selective_state_update_f64(
+            batch, dim, dstate, _ptr(state), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C),
+            _ptr(D), _ptr(z), _ptr(dt_bias), int(bool(dt_softplus)), _ptr(new_state),
+            _ptr(out))
+        if rc != 0:
+            raise ValueError(f"oracle_selective_state_update_f64 returned {rc}")
+        return new_state, out
+
+
+_DEFAULT: Oracle | None = None
+
+
+def default() -> Oracle:
+    """The oracle built from ``ssm_oracle.c`` (compiled on first use)."""
+    global _DEFAULT
+    if _DEFAULT is None:
+        _DEFAULT = Oracle()
+    return _DEFAULT

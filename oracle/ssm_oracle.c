@@ -1,0 +1,166 @@
+/*
+ * Float64 CPU oracle for the Mamba selective-SSM scan and the single-token
+ * state update.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path links, loads or calls
+ * this file: only the tests, the package's smoke check and the benchmark's
+ * CPU-baseline / reference arm use it.  It shares no code, header, table or
+ * constant with the CUDA library.
+ *
+ * It is the plain definition, written out one step at a time in float64:
+ *
+ *   Delta_t   = softplus(delta_t + bias_d)   (or delta_t + bias_d, softplus off)
+ *   Abar_t,n  = exp(Delta_t * A_d,n)
+ *   h_t,n     = Abar_t,n * h_{t-1},n + Delta_t * B_t,n * u_t,   h_{-1} = 0
+ *   y_t       = sum_n C_t,n * h_t,n + D_d * u_t
+ *   out_t     = y_t * silu(z_t)              (when z is given, else y_t)
+ *
+ * Sources (page title, section):
+ *  - "超越注意力：探索Mamba与状态空间模型" (ai-lab.club), section
+ *    "状态空间模型基础": the discretised recurrence h_t = Abar h_{t-1} + Bbar x_t,
+ *    y_t = C h_t + D x_t with Abar = exp(Delta A).
+ *  - same page, section "选择性状态空间模型": Delta_t = softplus(W x_t + b),
+ *    B_t and C_t depend on the token.  Here the projection outputs are inputs
+ *    (delta, B, C); the bias b is delta_bias.
+ *  - same page, section "代码实现概览": the simplified forward uses the Euler
+ *    input matrix Bbar = Delta * B and starts from a zero state.  This oracle
+ *    follows that reading (the page's zero-order-hold Bbar is not used).
+ *  - "Mamba 与状态空间模型" (world.lapla.si), section "由词元决定": the amount
+ *    of old state kept is exp(Delta * A).
+ *  - The output gate y * silu(z) is the Mamba block's multiplicative gate; no
+ *    page prints it.  silu(z) = z / (1 + exp(-z)).
+ *
+ * Loops: chains (b, d) are independent; OpenMP splits them across threads.
+ * Within a chain, t runs forward one step at a time and n ascends; nothing is
+ * blocked, fused or reordered.
+ *
+ * Layouts (all row-major, contiguous):
+ *   scan:   u, delta, z, out (batch, dim, seqlen); B, C (batch, dstate, seqlen);
+ *           A (dim, dstate); D, delta_bias (dim); last_state (batch, dim, dstate)
+ *   update: state (batch, dim, dstate) read and returned in new_state;
+ *           x, dt, z, out (batch, dim); B, C (batch, dstate); A (dim, dstate);
+ *           D, dt_bias (dim)
+ * Optional pointers (D, z, bias, last_state) may be NULL.
+ * Return value: 0 on success, -1 on a bad size.
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_MAX_DSTATE 256
+
+/* softplus(s) = log(1 + e^s).  For s > 30 the same value is taken as
+ * s + log1p(e^-s), which avoids overflowing exp. */
+static double oracle_softplus(double s)
+{
+    if (s > 30.0)
+        return s + log1p(exp(-s));
+    return log1p(exp(s));
+}
+
+/* silu(z) = z * sigmoid(z) = z / (1 + e^-z). */
+static double oracle_silu(double z)
+{
+    return z / (1.0 + exp(-z));
+}
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+int oracle_selective_scan_f64(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
+                              const double *u, const double *delta, const double *A,
+                              const double *B, const double *C, const double *D,
+                              const double *z, const double *delta_bias, int softplus,
+                              double *out, double *last_state)
+{
+    if (batch < 0 || dim < 0 || seqlen < 0 || dstate < 1 || dstate > ORACLE_MAX_DSTATE)
+        return -1;
+
+    int64_t chains = batch * dim;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t chain = 0; chain < chains; ++chain) {
+        int64_t b = chain / dim;
+        int64_t d = chain % dim;
+        double h[ORACLE_MAX_DSTATE];
+        for (int64_t n = 0; n < dstate; ++n)
+            h[n] = 0.0;
+
+        const double *u_row = u + (b * dim + d) * seqlen;
+        const double *delta_row = delta + (b * dim + d) * seqlen;
+        const double *z_row = z ? z + (b * dim + d) * seqlen : NULL;
+        double *out_row = out + (b * dim + d) * seqlen;
+
+        for (int64_t t = 0; t < seqlen; ++t) {
+            double dt = delta_row[t];
+            if (delta_bias)
+                dt += delta_bias[d];
+            if (softplus)
+                dt = oracle_softplus(dt);
+            double x = u_row[t];
+
+            double y = 0.0;
+            for (int64_t n = 0; n < dstate; ++n) {
+                double a_bar = exp(dt * A[d * dstate + n]);
+                double b_tn = B[(b * dstate + n) * seqlen + t];
+                double c_tn = C[(b * dstate + n) * seqlen + t];
+                h[n] = a_bar * h[n] + dt * b_tn * x;
+                y += c_tn * h[n];
+            }
+            if (D)
+                y += D[d] * x;
+            if (z_row)
+                y *= oracle_silu(z_row[t]);
+            out_row[t] = y;
+        }
+        if (last_state)
+            for (int64_t n = 0; n < dstate; ++n)
+                last_state[(b * dim + d) * dstate + n] = h[n];
+    }
+    return 0;
+}
+
+int oracle_selective_state_update_f64(int64_t batch, int64_t dim, int64_t dstate,
+                                      const double *state, const double *x, const double *dt,
+                                      const double *A, const double *B, const double *C,
+                                      const double *D, const double *z, const double *dt_bias,
+                                      int dt_softplus, double *new_state, double *out)
+{
+    if (batch < 0 || dim < 0 || dstate < 1 || dstate > ORACLE_MAX_DSTATE)
+        return -1;
+
+    int64_t chains = batch * dim;
+#pragma omp parallel for schedule(static)
+    for (int64_t chain = 0; chain < chains; ++chain) {
+        int64_t b = chain / dim;
+        int64_t d = chain % dim;
+        double delta = dt[chain];
+        if (dt_bias)
+            delta += dt_bias[d];
+        if (dt_softplus)
+            delta = oracle_softplus(delta);
+        double xv = x[chain];
+
+        double y = 0.0;
+        for (int64_t n = 0; n < dstate; ++n) {
+            double a_bar = exp(delta * A[d * dstate + n]);
+            double h = a_bar * state[chain * dstate + n] + delta * B[b * dstate + n] * xv;
+            new_state[chain * dstate + n] = h;
+            y += C[b * dstate + n] * h;
+        }
+        if (D)
+            y += D[d] * xv;
+        if (z)
+            y *= oracle_silu(z[chain]);
+        out[chain] = y;
+    }
+    return 0;
+}

@@ -1,0 +1,318 @@
+"""Pins for the float64 oracle: checks against what the pages and mathematics fix.
+
+Each pin takes an ``oracle.oracle.Oracle`` handle and raises AssertionError when
+the handle disagrees with an independent statement of the result.  None of
+them re-evaluates the oracle's recurrence: they use the unrolled sum, the LTI
+convolution, the gated-RNN form, the limits of Delta, closed values and
+invariants.  The mutation test runs every pin against deliberately broken
+copies of the oracle to show that a plausible slip is caught by at least one.
+
+Sources (page title, section):
+  - "超越注意力：探索Mamba与状态空间模型", 状态空间模型基础: discretisation and
+    the recurrence; the LTI system is a convolution.
+  - "Mamba 与状态空间模型", 每一步都一样: a time-invariant SSM is a convolution
+    with a fixed kernel; A is initialised to -1 ... -16.
+  - same page, 由词元决定: large Delta resets the state to the current input,
+    small Delta holds it; with a one-number state the update is the gate
+    h <- (1 - g) h + g x (Theorem 1).
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+
+def _rel(got, want):
+    got, want = np.asarray(got, np.float64), np.asarray(want, np.float64)
+    scale = max(float(np.max(np.abs(want))) if want.size else 0.0, 1e-300)
+    return float(np.max(np.abs(got - want))) / scale if want.size else 0.0
+
+
+def _close(got, want, tol, what):
+    err = _rel(got, want)
+    assert err <= tol, f"{what}: relative error {err:.3e} > {tol:.1e}"
+
+
+def _random_problem(seed, batch=2, dim=3, dstate=4, seqlen=40):
+    rng = np.random.default_rng(seed)
+    return dict(
+        u=rng.standard_normal((batch, dim, seqlen)),
+        delta=rng.uniform(0.05, 0.6, (batch, dim, seqlen)),
+        A=-rng.uniform(0.2, 2.0, (dim, dstate)),
+        B=rng.standard_normal((batch, dstate, seqlen)),
+        C=rng.standard_normal((batch, dstate, seqlen)),
+        D=rng.standard_normal(dim),
+        delta_bias=rng.uniform(0.0, 0.1, dim),
+    )
+
+
+def pin_unrolled_sum(o):
+    """y_t = sum_{s<=t} C_t (prod_{s<r<=t} Abar_r) Delta_s B_s u_s + D u_t, brute force.
+
+    Softplus off so Delta = delta + bias is fixed by the inputs alone.  Also
+    checks last_state = the same sum at t = L-1 without the C_t factor.
+    """
+    p = _random_problem(11)
+    out, last = o.selective_scan(p["u"], p["delta"], p["A"], p["B"], p["C"], D=p["D"],
+                                 delta_bias=p["delta_bias"], softplus=False)
+    u, A, B, C, D = p["u"], p["A"], p["B"], p["C"], p["D"]
+    Delta = p["delta"] + p["delta_bias"][None, :, None]
+    batch, dim, L = u.shape
+    want = np.zeros_like(u)
+    want_last = np.zeros((batch, dim, A.shape[1]))
+    for b in range(batch):
+        for d in range(dim):
+            abar = np.exp(Delta[b, d][:, None] * A[d][None, :])        # (L, N)
+            for t in range(L):
+                acc = 0.0
+                for s in range(t + 1):
+                    decay = np.prod(abar[s + 1:t + 1], axis=0)          # (N,)
+                    acc += np.sum(C[b, :, t] * decay * Delta[b, d, s] * B[b, :, s]) * u[b, d, s]
+                want[b, d, t] = acc + D[d] * u[b, d, t]
+            for s in range(L):
+                decay = np.prod(abar[s + 1:L], axis=0)
+                want_last[b, d] += decay * Delta[b, d, s] * B[b, :, s] * u[b, d, s]
+    _close(out, want, 1e-12, "unrolled sum: out")
+    _close(last, want_last, 1e-12, "unrolled sum: last_state")
+
+
+def pin_gate_closed_values(o):
+    """out = y * silu(z) with silu at closed values: silu(0)=0, silu(+-ln 3)=(3/4)ln 3,
+    -(1/4)ln 3, silu(40) = 40 to 1e-16."""
+    p = _random_problem(12, batch=1, dim=2, seqlen=8)
+    y, _ = o.selective_scan(p["u"], p["delta"], p["A"], p["B"], p["C"], D=p["D"],
+                            delta_bias=p["delta_bias"], softplus=True)
+    ln3 = math.log(3.0)
+    zvals = np.array([0.0, ln3, -ln3, 40.0, 0.0, ln3, -ln3, 40.0])
+    silu = np.array([0.0, 0.75 * ln3, -0.25 * ln3, 40.0, 0.0, 0.75 * ln3, -0.25 * ln3, 40.0])
+    z = np.broadcast_to(zvals, p["u"].shape).copy()
+    out, _ = o.selective_scan(p["u"], p["delta"], p["A"], p["B"], p["C"], D=p["D"], z=z,
+                              delta_bias=p["delta_bias"], softplus=True)
+    _close(out, y * silu[None, None, :], 1e-14, "gate closed values")
+
+
+def pin_lti_convolution(o):
+    """Delta, B, C constant in t: y = u * K + D u with K_k = sum_n C_n Abar_n^k Delta B_n."""
+    rng = np.random.default_rng(13)
+    batch, dim, N, L = 2, 3, 4, 48
+    u = rng.standard_normal((batch, dim, L))
+    Dl = rng.uniform(0.05, 0.5, (batch, dim))
+    delta = np.broadcast_to(Dl[:, :, None], (batch, dim, L)).copy()
+    A = -rng.uniform(0.1, 1.5, (dim, N))
+    Bc = rng.standard_normal((batch, N))
+    Cc = rng.standard_normal((batch, N))
+    B = np.broadcast_to(Bc[:, :, None], (batch, N, L)).copy()
+    C = np.broadcast_to(Cc[:, :, None], (batch, N, L)).copy()
+    D = rng.standard_normal(dim)
+    out, _ = o.selective_scan(u, delta, A, B, C, D=D, softplus=False)
+    want = np.zeros_like(u)
+    k = np.arange(L)
+    for b in range(batch):
+        for d in range(dim):
+            abar = np.exp(Dl[b, d] * A[d])                                   # (N,)
+            K = np.sum(Cc[b][None, :] * np.power(abar[None, :], k[:, None])
+                       * Dl[b, d] * Bc[b][None, :], axis=1)                  # (L,)
+            want[b, d] = np.convolve(u[b, d], K)[:L] + D[d] * u[b, d]
+    _close(out, want, 1e-12, "LTI convolution")
+
+
+def pin_gated_rnn_theorem1(o):
+    """N=1, A=-1, softplus on, C=1: with B_t = g_t / Delta_t the scan is the gate
+    h_t = (1-g_t) h_{t-1} + g_t x_t, g = sigmoid(delta + bias), since
+    1 - exp(-softplus(s)) = sigmoid(s)."""
+    rng = np.random.default_rng(14)
+    batch, L = 3, 64
+    s_delta = rng.standard_normal((batch, 1, L)) * 2.0
+    bias = np.array([-0.7])
+    s = s_delta + bias[None, :, None]
+    g = 1.0 / (1.0 + np.exp(-s))
+    Delta = np.log1p(np.exp(s))
+    x = rng.standard_normal((batch, 1, L))
+    B = (g / Delta).reshape(batch, 1, L)
+    C = np.ones((batch, 1, L))
+    A = np.array([[-1.0]])
+    out, last = o.selective_scan(x, s_delta, A, B, C, delta_bias=bias, softplus=True)
+    want = np.zeros_like(x)
+    for b in range(batch):
+        h = 0.0
+        for t in range(L):
+            h = (1.0 - g[b, 0, t]) * h + g[b, 0, t] * x[b, 0, t]
+            want[b, 0, t] = h
+    _close(out, want, 1e-12, "gated RNN (Theorem 1)")
+    _close(last[:, :, 0], want[:, :, -1], 1e-12, "gated RNN last state")
+
+
+def pin_small_delta_holds(o):
+    """Delta -> 0 holds the state: write once with Delta = softplus(40), then Delta ~ e^-80."""
+    rng = np.random.default_rng(15)
+    batch, dim, N, L = 1, 2, 4, 32
+    u = rng.standard_normal((batch, dim, L))
+    delta = np.full((batch, dim, L), -80.0)
+    delta[:, :, 0] = 40.0
+    A = -np.tile(np.arange(1, N + 1, dtype=np.float64), (dim, 1))
+    B = rng.standard_normal((batch, N, L))
+    C = rng.standard_normal((batch, N, L))
+    D = rng.standard_normal(dim)
+    out, last = o.selective_scan(u, delta, A, B, C, D=D, softplus=True)
+    h0 = 40.0 * B[:, None, :, 0] * u[:, :, 0][:, :, None]                  # (b, d, N)
+    want = np.einsum("bdn,bnt->bdt", h0, C) + D[None, :, None] * u
+    _close(out, want, 1e-12, "small Delta holds the state")
+    _close(last, h0, 1e-12, "small Delta: last_state")
+
+
+def pin_large_delta_resets(o):
+    """Large Delta with A <= -1: Abar underflows to 0, h_t = Delta B_t u_t (no history)."""
+    rng = np.random.default_rng(16)
+    batch, dim, N, L = 2, 3, 4, 20
+    u = rng.standard_normal((batch, dim, L))
+    delta = np.full((batch, dim, L), 1000.0)
+    A = -rng.uniform(1.0, 3.0, (dim, N))
+    B = rng.standard_normal((batch, N, L))
+    C = rng.standard_normal((batch, N, L))
+    D = rng.standard_normal(dim)
+    out, last = o.selective_scan(u, delta, A, B, C, D=D, softplus=False)
+    want = 1000.0 * np.einsum("bnt,bnt->bt", C, B)[:, None, :] * u + D[None, :, None] * u
+    _close(out, want, 1e-13, "large Delta resets the state")
+    _close(last, 1000.0 * B[:, None, :, -1] * u[:, :, -1][:, :, None], 1e-13,
+           "large Delta: last_state")
+
+
+def pin_zero_A_cumulative_sum(o):
+    """A = 0 gives Abar = 1: h_t = cumulative sum of Delta_s B_s u_s."""
+    p = _random_problem(17, seqlen=33)
+    A = np.zeros_like(p["A"])
+    out, last = o.selective_scan(p["u"], p["delta"], A, p["B"], p["C"], D=p["D"],
+                                 delta_bias=p["delta_bias"], softplus=False)
+    Delta = p["delta"] + p["delta_bias"][None, :, None]
+    inc = Delta[:, :, None, :] * p["B"][:, None, :, :] * p["u"][:, :, None, :]   # b d n t
+    h = np.cumsum(inc, axis=-1)
+    want = np.einsum("bdnt,bnt->bdt", h, p["C"]) + p["D"][None, :, None] * p["u"]
+    _close(out, want, 1e-12, "A = 0 cumulative sum")
+    _close(last, h[..., -1], 1e-12, "A = 0 last_state")
+
+
+def pin_softplus_closed_values(o):
+    """With N=1, A=0, B=C=u=1, L=1 the output is Delta itself:
+    softplus(0) = ln 2, softplus(ln(e-1)) = 1, softplus(log(expm1(v))) = v,
+    softplus(50) = 50, softplus(-50) = e^-50 (to 1e-21 relative)."""
+    v = 0.037
+    s = np.array([0.0, math.log(math.e - 1.0), math.log(math.expm1(v)), 50.0, -50.0])
+    want = np.array([math.log(2.0), 1.0, v, 50.0, math.exp(-50.0)])
+    dim = s.size
+    ones = np.ones((1, dim, 1))
+    out, _ = o.selective_scan(ones, s.reshape(1, dim, 1), np.zeros((dim, 1)),
+                              np.ones((1, 1, 1)), np.ones((1, 1, 1)), softplus=True)
+    got = out.reshape(-1)
+    err = np.abs(got - want) / np.abs(want)
+    assert np.all(err <= 1e-14), f"softplus closed values: {got} vs {want}"
+    # split between delta and delta_bias: the bias is added before softplus
+    out2, _ = o.selective_scan(ones, (s - 0.25).reshape(1, dim, 1), np.zeros((dim, 1)),
+                               np.ones((1, 1, 1)), np.ones((1, 1, 1)),
+                               delta_bias=np.full(dim, 0.25), softplus=True)
+    _close(out2.reshape(-1), want, 1e-14, "softplus with bias")
+
+
+def pin_linearity_and_causality(o):
+    """Without the gate, out is linear in u (B, C, Delta fixed) and causal."""
+    p = _random_problem(18, seqlen=30)
+    rng = np.random.default_rng(19)
+    u2 = rng.standard_normal(p["u"].shape)
+    args = (p["A"], p["B"], p["C"])
+    kw = dict(D=p["D"], delta_bias=p["delta_bias"], softplus=True)
+    y1, _ = o.selective_scan(p["u"], p["delta"], *args, **kw)
+    y2, _ = o.selective_scan(u2, p["delta"], *args, **kw)
+    y12, _ = o.selective_scan(2.5 * p["u"] - 0.75 * u2, p["delta"], *args, **kw)
+    _close(y12, 2.5 * y1 - 0.75 * y2, 1e-12, "linearity in u")
+    s0 = 17
+    u3 = p["u"].copy()
+    u3[:, :, s0] += 1.0
+    y3, _ = o.selective_scan(u3, p["delta"], *args, **kw)
+    assert np.array_equal(y3[:, :, :s0], y1[:, :, :s0]), "causality: earlier outputs moved"
+    assert np.all(np.abs(y3[:, :, s0] - y1[:, :, s0]) > 0), "perturbation had no effect"
+
+
+def _decode_problem(seed, batch=2, dim=3, N=4, T=24):
+    rng = np.random.default_rng(seed)
+    return dict(
+        x=rng.standard_normal((batch, dim, T)),
+        dt=rng.standard_normal((batch, dim, T)),
+        z=rng.standard_normal((batch, dim, T)),
+        A=-rng.uniform(0.2, 2.0, (dim, N)),
+        B=rng.standard_normal((batch, N, T)) / 4,
+        C=rng.standard_normal((batch, N, T)) / 4,
+        D=rng.standard_normal(dim),
+        bias=rng.uniform(-1.0, 0.0, dim),
+    )
+
+
+def pin_update_steps_equal_scan(o):
+    """T single-token updates from the zero state reproduce the scan over the same T tokens."""
+    p = _decode_problem(21)
+    out_scan, last = o.selective_scan(p["x"], p["dt"], p["A"], p["B"], p["C"], D=p["D"],
+                                      z=p["z"], delta_bias=p["bias"], softplus=True)
+    batch, dim, T = p["x"].shape
+    state = np.zeros((batch, dim, p["A"].shape[1]))
+    outs = np.zeros_like(p["x"])
+    for t in range(T):
+        state, outs[:, :, t] = o.selective_state_update(
+            state, p["x"][:, :, t], p["dt"][:, :, t], p["A"], p["B"][:, :, t],
+            p["C"][:, :, t], D=p["D"], z=p["z"][:, :, t], dt_bias=p["bias"], dt_softplus=True)
+    _close(outs, out_scan, 1e-13, "update steps = scan: out")
+    _close(state, last, 1e-13, "update steps = scan: state")
+
+
+def pin_update_continues_scan(o):
+    """Updates started from the scan's last_state after T1 tokens continue it exactly."""
+    p = _decode_problem(22, T=30)
+    T1 = 18
+    out_full, last_full = o.selective_scan(p["x"], p["dt"], p["A"], p["B"], p["C"], D=p["D"],
+                                           z=p["z"], delta_bias=p["bias"], softplus=True)
+    _, state = o.selective_scan(p["x"][:, :, :T1], p["dt"][:, :, :T1], p["A"],
+                                p["B"][:, :, :T1], p["C"][:, :, :T1], D=p["D"],
+                                z=p["z"][:, :, :T1], delta_bias=p["bias"], softplus=True)
+    outs = []
+    for t in range(T1, p["x"].shape[2]):
+        state, y = o.selective_state_update(
+            state, p["x"][:, :, t], p["dt"][:, :, t], p["A"], p["B"][:, :, t],
+            p["C"][:, :, t], D=p["D"], z=p["z"][:, :, t], dt_bias=p["bias"], dt_softplus=True)
+        outs.append(y)
+    _close(np.stack(outs, axis=-1), out_full[:, :, T1:], 1e-13, "update continues scan: out")
+    _close(state, last_full, 1e-13, "update continues scan: state")
+
+
+def pin_update_limits(o):
+    """Update with large Delta resets the state to Delta B x; with tiny Delta it holds it."""
+    rng = np.random.default_rng(23)
+    batch, dim, N = 2, 3, 4
+    state = rng.standard_normal((batch, dim, N))
+    x = rng.standard_normal((batch, dim))
+    A = -rng.uniform(1.0, 2.0, (dim, N))
+    B = rng.standard_normal((batch, N))
+    C = rng.standard_normal((batch, N))
+    D = rng.standard_normal(dim)
+    new, out = o.selective_state_update(state, x, np.full((batch, dim), 1000.0), A, B, C,
+                                        D=D, dt_softplus=False)
+    reset = 1000.0 * B[:, None, :] * x[:, :, None]
+    _close(new, reset, 1e-13, "update reset: state")
+    _close(out, np.einsum("bdn,bn->bd", reset, C) + D[None, :] * x, 1e-13, "update reset: out")
+    new, out = o.selective_state_update(state, x, np.full((batch, dim), -80.0), A, B, C,
+                                        D=D, dt_softplus=True)
+    _close(new, state, 1e-13, "update hold: state")
+    _close(out, np.einsum("bdn,bn->bd", state, C) + D[None, :] * x, 1e-13, "update hold: out")
+
+
+PINS = {
+    "unrolled_sum": pin_unrolled_sum,
+    "gate_closed_values": pin_gate_closed_values,
+    "lti_convolution": pin_lti_convolution,
+    "gated_rnn_theorem1": pin_gated_rnn_theorem1,
+    "small_delta_holds": pin_small_delta_holds,
+    "large_delta_resets": pin_large_delta_resets,
+    "zero_A_cumulative_sum": pin_zero_A_cumulative_sum,
+    "softplus_closed_values": pin_softplus_closed_values,
+    "linearity_and_causality": pin_linearity_and_causality,
+    "update_steps_equal_scan": pin_update_steps_equal_scan,
+    "update_continues_scan": pin_update_continues_scan,
+    "update_limits": pin_update_limits,
+}

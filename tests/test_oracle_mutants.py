@@ -1,0 +1,81 @@
+"""Mutation check of the oracle's pins (CPU only).
+
+Each mutant is a copy of the C oracle with one plausible slip planted in it: a
+dropped term, a flipped sign, a wrong or transposed index, an operand swapped.
+The copy is compiled into a temporary directory and every pin is run against
+it; the test requires at least one pin to reject it.  The oracle's own source
+is never modified.  All mutants keep their memory accesses in bounds.
+"""
+import subprocess
+
+import pytest
+
+from oracle import oracle
+from oracle_pins import PINS
+
+# (name, exact snippet in ssm_oracle.c, replacement)
+MUTANTS = [
+    ("drop_D_term", "y += D[d] * x;", "y += 0.0 * x;"),
+    ("exp_sign_flipped", "exp(dt * A[d * dstate + n])", "exp(-dt * A[d * dstate + n])"),
+    ("B_read_from_C", "double b_tn = B[(b * dstate + n) * seqlen + t];",
+     "double b_tn = C[(b * dstate + n) * seqlen + t];"),
+    ("softplus_skipped", "if (softplus)\n                dt = oracle_softplus(dt);", ""),
+    ("softplus_is_identity", "return log1p(exp(s));", "return log(exp(s));"),
+    ("softplus_missing_one", "return log1p(exp(s));", "return log(exp(s) + 1e-3);"),
+    ("bias_dropped", "dt += delta_bias[d];", "dt += 0.0;"),
+    ("bias_after_softplus",
+     "if (delta_bias)\n                dt += delta_bias[d];\n            if (softplus)\n"
+     "                dt = oracle_softplus(dt);",
+     "if (softplus)\n                dt = oracle_softplus(dt);\n            if (delta_bias)\n"
+     "                dt += delta_bias[d];"),
+    ("gate_sign_flipped", "return z / (1.0 + exp(-z));", "return z / (1.0 + exp(z));"),
+    ("gate_is_sigmoid", "return z / (1.0 + exp(-z));", "return 1.0 / (1.0 + exp(-z));"),
+    ("bbar_without_delta", "h[n] = a_bar * h[n] + dt * b_tn * x;", "h[n] = a_bar * h[n] + b_tn * x;"),
+    ("state_not_decayed", "h[n] = a_bar * h[n] + dt * b_tn * x;", "h[n] = h[n] + dt * b_tn * x;"),
+    ("readout_before_update",
+     "h[n] = a_bar * h[n] + dt * b_tn * x;\n                y += c_tn * h[n];",
+     "y += c_tn * h[n];\n                h[n] = a_bar * h[n] + dt * b_tn * x;"),
+    ("B_time_shifted", "double b_tn = B[(b * dstate + n) * seqlen + t];",
+     "double b_tn = B[(b * dstate + n) * seqlen + (t > 0 ? t - 1 : t)];"),
+    ("C_batch_ignored", "double c_tn = C[(b * dstate + n) * seqlen + t];",
+     "double c_tn = C[(0 * dstate + n) * seqlen + t];"),
+    ("A_transposed", "exp(dt * A[d * dstate + n])", "exp(dt * A[n * dim + d])"),
+    ("u_time_shifted", "double x = u_row[t];", "double x = u_row[t > 0 ? t - 1 : 0];"),
+    ("last_state_zeroed", "last_state[(b * dim + d) * dstate + n] = h[n];",
+     "last_state[(b * dim + d) * dstate + n] = 0.0 * h[n];"),
+    ("update_state_not_decayed", "double h = a_bar * state[chain * dstate + n]",
+     "double h = state[chain * dstate + n]"),
+    ("update_bias_dropped", "delta += dt_bias[d];", "delta += 0.0;"),
+    ("update_gate_dropped", "y *= oracle_silu(z[chain]);", "y *= 1.0;"),
+    ("update_B_batch_ignored", "delta * B[b * dstate + n] * xv", "delta * B[n] * xv"),
+    ("update_C_from_B", "y += C[b * dstate + n] * h;", "y += B[b * dstate + n] * h;"),
+    ("update_D_dropped", "y += D[d] * xv;", "y += 0.0 * xv;"),
+    ("update_softplus_skipped", "if (dt_softplus)\n            delta = oracle_softplus(delta);", ""),
+]
+
+
+def test_mutant_snippets_present():
+    src = oracle.SOURCE.read_text()
+    for name, old, _ in MUTANTS:
+        assert old in src, f"mutant {name}: snippet not found in the oracle source"
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_mutant_is_caught(tmp_path, name, old, new):
+    src = oracle.SOURCE.read_text()
+    assert old in src
+    mutated = tmp_path / f"{name}.c"
+    mutated.write_text(src.replace(old, new, 1))
+    lib = tmp_path / f"lib{name}.so"
+    try:
+        oracle.build(mutated, lib, force=True)
+    except subprocess.CalledProcessError as e:  # pragma: no cover - a mutant must compile
+        pytest.fail(f"mutant {name} does not compile: {e}")
+    handle = oracle.Oracle(lib)
+    caught = []
+    for pin_name, pin in PINS.items():
+        try:
+            pin(handle)
+        except AssertionError:
+            caught.append(pin_name)
+    assert caught, f"mutant {name} passed every pin"
