@@ -1,0 +1,543 @@
+#!/usr/bin/env python
+"""Benchmark of the selective-SSM hot path on B200.
+
+One step = one pass of the whole path on synthetic data:
+  1. selective scan over the Mamba-2.8B-layer workload: batch 16, d_inner 5120,
+     N 16, L 2048, bf16 u/delta/z/out, fp32 state, last_state returned;
+  2. one generated token through 48 layers of selective_state_update at batch
+     128, d_inner 4096, N 16, each layer's fp32 state (33.5 MB) updated in place
+     (the 48 states, 1.6 GB, rotate so the state streams from HBM).
+
+Reported: scan elements (B*D*L) per second, as the metric's value, with its
+fraction of the MUFU roofline; the decode token-step in microseconds with its
+fraction of HBM bandwidth.  Both inputs exceed L2 (126 MB), so no L2 flush is
+needed between steps.  Timing uses CUDA events on the launching stream,
+bracketed by a barrier and device synchronisation, max over ranks.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (torchrun): every rank runs its own copy of the step on its own
+inputs (weak scaling, no data-path collective); the value is the job total.
+``--impl reference`` times the float64 CPU oracle on a bounded sample of the
+same workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+from pathlib import Path
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+import torch  # noqa: E402
+
+METRIC = ("selective-scan Gelem/s (B·D·L) and % of roofline; "
+          "decode-step µs at batch 128")
+SCAN_WORKLOAD = "mamba_2p8b_layer"
+PROFILES = ROOT / "profiles"
+HBM_FALLBACK_GBS = 6650.0
+SM_MAX_MHZ_FALLBACK = 1965.0
+
+
+# ----------------------------------------------------------------- helpers
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def measured_peaks() -> dict:
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        try:
+            d = json.loads(p.read_text())
+            return {"hbm_gbs": float(d["hbm_gbs"]), "sm_max_mhz": float(d.get("sm_max_mhz", SM_MAX_MHZ_FALLBACK)),
+                    "source": "measured"}
+        except Exception:  # noqa: BLE001
+            pass
+    return {"hbm_gbs": HBM_FALLBACK_GBS, "sm_max_mhz": SM_MAX_MHZ_FALLBACK, "source": "fallback"}
+
+
+def sources_digest() -> str:
+    h = hashlib.sha256()
+    csrc = ROOT / "selective_state_space_55_b200" / "csrc"
+    for p in sorted(csrc.glob("*")) + [ROOT / "include" / "mamba_ssm.h"]:
+        h.update(p.name.encode())
+        h.update(p.read_bytes())
+    return h.hexdigest()
+
+
+def recorded_traffic(kernel: str, digest: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    p = PROFILES / "ncu_traffic.json"
+    if not p.exists():
+        return None
+    try:
+        rec = json.loads(p.read_text()).get(kernel)
+    except Exception:  # noqa: BLE001
+        return None
+    if not rec or rec.get("sources_sha256") != digest:
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons of one GPU through NVML (falls
+    back to nvidia-smi) from a background thread."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, local_rank: int, period_s: float = 0.02):
+        self.period = period_s
+        self.samples: list[tuple[float, float, int]] = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self._handle = None
+        self._nvml = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+            idx = local_rank
+            parts = [p for p in vis.split(",") if p.strip()]
+            if parts and local_rank < len(parts) and parts[local_rank].strip().isdigit():
+                idx = int(parts[local_rank])
+            self._handle = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self._nvml = pynvml
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self._handle, pynvml.NVML_CLOCK_SM))
+        except Exception as e:  # noqa: BLE001
+            log(f"[bench] NVML unavailable ({e}); clocks via nvidia-smi")
+        self.local_rank = local_rank
+
+    def _poll(self):
+        while not self._stop.is_set():
+            t = time.time()
+            try:
+                if self._nvml is not None:
+                    mhz = float(self._nvml.nvmlDeviceGetClockInfo(self._handle, self._nvml.NVML_CLOCK_SM))
+                    reasons = int(self._nvml.nvmlDeviceGetCurrentClocksEventReasons(self._handle))
+                else:
+                    out = subprocess.run(
+                        ["nvidia-smi", f"--id={self.local_rank}",
+                         "--query-gpu=clocks.sm,clocks.max.sm,clocks_event_reasons.active",
+                         "--format=csv,noheader,nounits"],
+                        capture_output=True, text=True, timeout=5).stdout.strip().split(",")
+                    mhz, self.max_mhz = float(out[0]), float(out[1])
+                    reasons = int(out[2].strip(), 16)
+                self.samples.append((t, mhz, reasons))
+            except Exception:  # noqa: BLE001
+                pass
+            self._stop.wait(self.period)
+
+    def start(self):
+        self._thread = threading.Thread(target=self._poll, daemon=True)
+        self._thread.start()
+
+    def stop(self):
+        self._stop.set()
+        if self._thread:
+            self._thread.join(timeout=10)
+
+    def summary(self, t0: float, t1: float) -> dict:
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        window = "timed_region"
+        if not inside:
+            inside, window = self.samples, "whole_run"
+        reasons = set()
+        for _, _, r in inside:
+            for bit, name in self.REASONS.items():
+                if r & bit and name != "gpu_idle":
+                    reasons.add(name)
+        mhz = [s[1] for s in inside]
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(inside), "window": window}
+
+
+# ----------------------------------------------------------------- workloads
+
+class Workload:
+    """Device-resident inputs and outputs of one step, and the calls that run it."""
+
+    def __init__(self, rank: int, scan_batch: int | None = None, decode_layers: int | None = None,
+                 only: str | None = None):
+        from selective_state_space_55_b200 import inputs as I
+        from selective_state_space_55_b200 import ops
+
+        self.ops = ops
+        self.only = only
+        self.cfg = I.SCAN_CONFIGS[SCAN_WORKLOAD]
+        if scan_batch:
+            self.cfg = self.cfg.resized(batch=scan_batch)
+        self.dcfg = I.DECODE_CONFIG
+        if decode_layers:
+            self.dcfg = I.DecodeConfig(self.dcfg.name, self.dcfg.batch, self.dcfg.dim,
+                                       self.dcfg.dstate, decode_layers, self.dcfg.steps)
+        c = self.cfg
+        self.x = I.make_scan_inputs(c, "cuda", seed=1000 + rank)
+        self.out = torch.empty_like(self.x["u"])
+        self.last = torch.empty((c.batch, c.dim, c.dstate), dtype=torch.float32, device="cuda")
+        ws = ops.scan_workspace_bytes(c.batch, c.dim, c.dstate, c.seqlen, c.io_dtype, c.bc_dtype)
+        self.ws = torch.empty(ws, dtype=torch.uint8, device="cuda") if ws else None
+        self.plan = ops.scan_plan(c.batch, c.dim, c.dstate, c.seqlen, c.io_dtype, c.bc_dtype,
+                                  sm_count=torch.cuda.get_device_properties(0).multi_processor_count)
+        d = self.dcfg
+        nl = 0 if only == "scan" else d.layers
+        self.layers = [I.make_decode_layer(d, "cuda", seed=2000 + 100 * rank + i) for i in range(nl)]
+        self.toks = [I.make_decode_token(d, "cuda", seed=3000 + 100 * rank + i) for i in range(nl)]
+        self.douts = [torch.empty_like(t["x"]) for t in self.toks]
+        self.graph = None
+
+    def scan(self):
+        if self.only == "decode":
+            return
+        x = self.x
+        self.ops.selective_scan_fwd(x["u"], x["delta"], x["A"], x["B"], x["C"], D=x["D"], z=x["z"],
+                                    delta_bias=x["delta_bias"], softplus=True, out=self.out,
+                                    last_state=self.last, workspace=self.ws)
+
+    def decode_layers(self):
+        for lay, tok, out in zip(self.layers, self.toks, self.douts):
+            self.ops.selective_state_update(lay["state"], tok["x"], tok["dt"], lay["A"], tok["B"],
+                                            tok["C"], D=lay["D"], z=tok["z"],
+                                            dt_bias=lay["dt_bias"], out=out)
+
+    def capture_decode(self):
+        """Capture the 48 state-update launches of one token in a CUDA graph."""
+        if not self.layers:
+            return
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            self.decode_layers()          # warm the launch path outside capture
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self.decode_layers()
+        torch.cuda.synchronize()
+
+    def decode(self):
+        if self.graph is not None:
+            self.graph.replay()
+
+    @property
+    def launches_per_step(self) -> int:
+        return (0 if self.only == "decode" else self.plan["launches"]) + len(self.layers)
+
+
+def run_e2e(w: Workload, steps: int, warmup: int) -> dict:
+    """Scan metric end to end: pinned host inputs -> device -> scan -> host."""
+    x = w.x
+    names = ["u", "delta", "z", "B", "C"]
+    host = {k: torch.empty(x[k].shape, dtype=x[k].dtype, pin_memory=True) for k in names}
+    for k in names:
+        host[k].copy_(x[k])
+    out_h = torch.empty(w.out.shape, dtype=w.out.dtype, pin_memory=True)
+    last_h = torch.empty(w.last.shape, dtype=w.last.dtype, pin_memory=True)
+    h2d = sum(host[k].numel() * host[k].element_size() for k in names)
+    d2h = out_h.numel() * out_h.element_size() + last_h.numel() * last_h.element_size()
+
+    def step():
+        for k in names:
+            x[k].copy_(host[k], non_blocking=True)
+        w.scan()
+        out_h.copy_(w.out, non_blocking=True)
+        last_h.copy_(w.last, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        step()
+    e.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(s.elapsed_time(e))
+    return {"ms_total": ms, "steps": steps, "h2d": h2d, "d2h": d2h}
+
+
+def cpu_baseline(w: Workload, target_s: float) -> dict:
+    """The float64 oracle on the host cores over a contiguous block of chains
+    of the same workload (batch row 0, channels 0..S-1, all L steps)."""
+    from oracle import oracle
+    ref = oracle.default()
+    x = w.x
+    L = w.cfg.seqlen
+
+    def run(S):
+        sl = lambda t: None if t is None else t[0:1, :S].cpu()  # noqa: E731
+        args = (sl(x["u"]), sl(x["delta"]), x["A"][:S].cpu(), x["B"][0:1].cpu(), x["C"][0:1].cpu())
+        t0 = time.perf_counter()
+        ref.selective_scan(*args, D=x["D"][:S].cpu(), z=sl(x["z"]),
+                           delta_bias=x["delta_bias"][:S].cpu(), softplus=True)
+        return time.perf_counter() - t0
+
+    S = 32
+    t = run(S)
+    if t < target_s:
+        S = int(min(w.cfg.dim, max(S, S * target_s / max(t, 1e-6))))
+        t = run(S)
+    return {"value": S * L / t / 1e9, "unit": "Gelem/s", "cores": ref.num_threads(),
+            "kind": "oracle",
+            "sample": f"{S} chains (batch row 0, channels 0..{S - 1}) x L={L} of "
+                      f"{SCAN_WORKLOAD}: {S * L} elements in {t:.1f} s"}
+
+
+# ----------------------------------------------------------------- distributed
+
+_WORLD = 1
+
+
+def barrier():
+    if _WORLD > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(v: float) -> float:
+    if _WORLD == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------- arms
+
+def bench_ours(args, rank, world, local):
+    global _WORLD
+    _WORLD = world
+    from selective_state_space_55_b200 import build as cuda_build
+    from selective_state_space_55_b200 import roofline as R
+
+    if rank == 0:
+        cuda_build.build()
+    barrier()
+    torch.cuda.set_device(local)
+    partial = args.only is not None or args.scan_batch or args.decode_layers
+    w = Workload(rank, args.scan_batch, args.decode_layers, args.only)
+    c, d = w.cfg, w.dcfg
+    w.capture_decode()
+    for _ in range(args.warmup):
+        w.scan()
+        w.decode()
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    start.record()
+    for e0, e1, e2 in ev:
+        e0.record()
+        w.scan()
+        e1.record()
+        w.decode()
+        e2.record()
+    end.record()
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    barrier()
+    sampler.stop()
+
+    total_ms = max_over_ranks(start.elapsed_time(end))
+    scan_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b, _ in ev))
+    decode_ms = max_over_ranks(sum(b.elapsed_time(cc) for _, b, cc in ev))
+    K = args.steps
+    elems = c.elements
+    value = world * elems * K / (scan_ms * 1e-3) / 1e9          # Gelem/s, whole job
+    scan_launch_ms = scan_ms / K
+    decode_step_us = decode_ms / K * 1e3
+
+    peaks = measured_peaks()
+    clocks = sampler.summary(t_wall0, t_wall1)
+    mufu = R.scan_mufu_per_element(c.dstate, has_z=True, softplus=True)
+    peak_elems = R.mufu_peak_elements_per_s(torch.cuda.get_device_properties(local).multi_processor_count,
+                                            peaks["sm_max_mhz"], mufu) / 1e9
+    achieved = elems / (scan_launch_ms * 1e-3) / 1e9               # per launch, this rank
+    scan_bytes = R.scan_bytes(c.batch, c.dim, c.dstate, c.seqlen, 2, 2, True, True)
+    upd_bytes = R.update_bytes(d.batch, d.dim, d.dstate, 2, 2, True)
+    decode_gbs = upd_bytes * d.layers / (decode_ms / K * 1e-3) / 1e9
+    digest = sources_digest()
+    roof = {
+        "bound": "alu", "pipe": "MUFU (16 ops/clk/SM; 20 per element)",
+        "kernel": "selective_scan_fwd_kernel",
+        "achieved": round(achieved, 2), "peak": round(peak_elems, 2), "unit": "Gelem/s",
+        "frac": round(achieved / peak_elems, 4),
+        "peak_basis": f"148 SMs x 16 MUFU/clk x {peaks['sm_max_mhz']:.0f} MHz / {mufu} per element",
+        "frac_at_measured_clock": (round(achieved / (peak_elems * clocks["sm_mhz"] / peaks["sm_max_mhz"]), 4)
+                                   if clocks.get("sm_mhz") else None),
+        "algorithmic_bytes_per_launch": scan_bytes,
+        "hbm_gbs": round(scan_bytes / (scan_launch_ms * 1e-3) / 1e9, 1),
+        "traffic": recorded_traffic("selective_scan_fwd_kernel", digest),
+    }
+    decode = {
+        "workload": f"decode_b128: {d.layers} layers x state ({d.batch}, {d.dim}, {d.dstate}) fp32, "
+                    "bf16 x/dt/z/B/C/out, one CUDA graph per token",
+        "us_per_token_step": round(decode_step_us, 2),
+        "us_per_layer": round(decode_step_us / d.layers, 3),
+        "roofline": {"bound": "hbm", "kernel": "state_update_n16_kernel",
+                     "achieved": round(decode_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(decode_gbs / peaks["hbm_gbs"], 4),
+                     "peak_source": peaks["source"],
+                     "algorithmic_bytes_per_launch": upd_bytes,
+                     "traffic": recorded_traffic("state_update_n16_kernel", digest)},
+        "tokens_per_s": round(world * d.batch / (decode_step_us * 1e-6), 1),
+    }
+
+    e2e = None
+    if not args.no_e2e and args.only != "decode":
+        r = run_e2e(w, max(1, min(K, args.e2e_steps)), 2)
+        e2e = {"value": round(world * elems * r["steps"] / (r["ms_total"] * 1e-3) / 1e9, 3),
+               "unit": "Gelem/s", "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
+               "steps": r["steps"],
+               "path": "pinned host u/delta/z/B/C -> device -> mamba_selective_scan_fwd -> "
+                       "out/last_state to pinned host, one stream"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.only != "decode":
+        cpu = cpu_baseline(w, args.cpu_seconds)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 3), "unit": "Gelem/s", "n_gpus": world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": round(total_ms / K, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (seeded; shapes and distributions of the pages' workloads)",
+            "config": {
+                "workload": f"{SCAN_WORKLOAD} scan ({c.batch}x{c.dim}, N={c.dstate}, L={c.seqlen}, "
+                            "bf16 in/out, fp32 state, last_state) + decode_b128 token step "
+                            f"({d.layers} layers, batch {d.batch}, d_inner {d.dim}, N {d.dstate})",
+                "io_dtype": "bf16", "state_dtype": "f32", "global_batch": world * c.batch,
+                "seq_len": c.seqlen, "parallelism": f"replicas{world}" if world > 1 else "single",
+                "l2": "inputs larger than L2 (1.0 GB scan inputs, 1.6 GB rotating decode state)",
+                "scan_plan": w.plan,
+            },
+            "scan_ms_per_step": round(scan_ms / K, 4),
+            "roofline": roof,
+            "decode": decode,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": K * w.launches_per_step,
+            "clocks": clocks,
+            "sources_sha256": digest[:16],
+        }
+        if partial:
+            line["partial_case"] = {"only": args.only, "scan_batch": args.scan_batch,
+                                    "decode_layers": args.decode_layers,
+                                    "note": "profiling case, not the benchmark workload"}
+        print(json.dumps(line), flush=True)
+
+
+def bench_reference(args, rank, world):
+    """The float64 CPU oracle, on the same workload's metric, a bounded sample
+    per step (rank 0 only)."""
+    if rank != 0:
+        return
+    import numpy as np  # noqa: F401
+    from oracle import oracle
+    from selective_state_space_55_b200 import inputs as I
+
+    ref = oracle.default()
+    cfg = I.SCAN_CONFIGS[SCAN_WORKLOAD]
+    L = cfg.seqlen
+    small = cfg.resized(batch=1, dim=min(cfg.dim, 4096))
+    x = I.make_scan_inputs(small, "cpu", seed=1000)
+
+    def run(S):
+        sl = lambda t: None if t is None else t[0:1, :S]  # noqa: E731
+        t0 = time.perf_counter()
+        ref.selective_scan(sl(x["u"]), sl(x["delta"]), x["A"][:S], x["B"][0:1], x["C"][0:1],
+                           D=x["D"][:S], z=sl(x["z"]), delta_bias=x["delta_bias"][:S], softplus=True)
+        return time.perf_counter() - t0
+
+    budget_s = args.reference_seconds
+    t1 = run(8) / 8
+    per_step = budget_s / max(1, args.steps + args.warmup)
+    S = int(max(1, min(small.dim, per_step / max(t1, 1e-9))))
+    for _ in range(args.warmup):
+        run(S)
+    times = [run(S) for _ in range(args.steps)]
+    total = sum(times)
+    value = S * L * args.steps / total / 1e9
+    sample = (f"{S} chains (batch row 0, channels 0..{S - 1}) x L={L} of {SCAN_WORKLOAD} per step")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "Gelem/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{SCAN_WORKLOAD} scan, sampled chains (float64 CPU oracle)",
+                   "seq_len": L},
+        "cpu_baseline": {"value": value, "unit": "Gelem/s", "cores": ref.num_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "Gelem/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=600)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--reference-seconds", type=float, default=120.0,
+                    help="budget of the whole --impl reference run")
+    ap.add_argument("--only", choices=["scan", "decode"], default=None,
+                    help="profiling case: run one half of the step")
+    ap.add_argument("--scan-batch", type=int, default=None,
+                    help="profiling case: smaller scan batch")
+    ap.add_argument("--decode-layers", type=int, default=None,
+                    help="profiling case: fewer decode layers")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        log("[bench] warm-up raised to 3 steps (minimum)")
+        args.warmup = 3
+
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    if world != args.gpus:
+        log(f"[bench] note: --gpus {args.gpus} but WORLD_SIZE={world}; using WORLD_SIZE")
+
+    if args.impl == "reference":
+        bench_reference(args, rank, world)
+        return
+
+    if world > 1:
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group(
+            "nccl", timeout=datetime.timedelta(seconds=300),
+            device_id=torch.device("cuda", local))
+    try:
+        bench_ours(args, rank, world, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,213 @@
+/*
+ * mamba_ssm.h — C ABI of the B200 (sm_100a) selective-SSM library.
+ *
+ * Two operations, both from the Mamba selective state space model:
+ *
+ *   mamba_selective_scan_fwd      the selective scan over a whole sequence
+ *   mamba_selective_state_update  one token of generation (recurrent mode)
+ *
+ * Definition (per batch b, channel d, state index n, time t):
+ *
+ *   Delta_t  = softplus(delta_t + delta_bias_d)      (or without softplus)
+ *   Abar     = exp(Delta_t * A_d,n)
+ *   h_t,n    = Abar * h_{t-1},n + Delta_t * B_t,n * u_t        h_{-1} = 0
+ *   y_t      = sum_n C_t,n * h_t,n + D_d * u_t
+ *   out_t    = y_t * silu(z_t)                                   (z optional)
+ *
+ * Sources: "超越注意力：探索Mamba与状态空间模型" (ai-lab.club), section
+ * 状态空间模型基础 (zero-order-hold Abar = exp(Delta A), recurrence and
+ * readout) and section 选择性状态空间模型 (Delta = softplus(W x + b), B and C
+ * per token); its section 代码实现概览 uses the Euler input term
+ * Bbar = Delta * B, which this library follows.  "Mamba 与状态空间模型"
+ * (world.lapla.si), section 由词元决定 (exp(Delta A) decides how much old state
+ * is kept) and section 在芯片上扫过去 (the scan never writes the full state to
+ * HBM).  The silu(z) gate is the Mamba block's output gate (not printed on the
+ * pages).  The update is the same step applied once to a stored state
+ * ("Mamba: Linear-Time Sequence Modeling with Selective State Spaces"
+ * (mentras.net), table 复杂度对比: constant work per generated token).
+ *
+ * Conventions shared by every entry point
+ *  - Pointers named in the signatures are DEVICE pointers owned by the caller;
+ *    the dims struct is a HOST pointer.  The library keeps no per-call state
+ *    and performs no device allocation.  Work is enqueued on `stream`
+ *    (asynchronous); pass 0 for the legacy default stream.
+ *  - All tensors are dense, row-major, contiguous, without padding.
+ *  - Floating-point arithmetic is fp32; the state is fp32.  u/delta/z/out
+ *    (x/dt/z/out) and B/C may each be fp32 or bf16 (see mamba_dtype_t).
+ *    A, D and the delta/dt bias are fp32.
+ *  - Return value: MAMBA_OK, or a negative mamba_status_t.  Argument errors
+ *    are detected before anything is launched.  MAMBA_ERR_CUDA reports a
+ *    launch failure (cudaGetLastError after the launch).  Faults that happen
+ *    later on the device surface at the next synchronising CUDA call;
+ *    mamba_device_status() reports the library's own device-side checks.
+ *  - Outputs must not alias inputs (except the in-place state of the update).
+ */
+#ifndef MAMBA_SSM_H
+#define MAMBA_SSM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(_WIN32)
+#define MAMBA_API __declspec(dllexport)
+#else
+#define MAMBA_API __attribute__((visibility("default")))
+#endif
+
+typedef enum {
+    MAMBA_OK = 0,
+    MAMBA_ERR_INVALID_ARG = -1,   /* null required pointer, negative size, ... */
+    MAMBA_ERR_UNSUPPORTED = -2,   /* dtype code, or dstate outside 1..16 */
+    MAMBA_ERR_ALIGN = -3,         /* a pointer is not aligned to its element size */
+    MAMBA_ERR_WORKSPACE = -4,     /* workspace missing or smaller than required */
+    MAMBA_ERR_CUDA = -5,          /* a CUDA runtime call failed */
+    MAMBA_ERR_TIMEOUT = -6        /* a bounded device-side wait gave up */
+} mamba_status_t;
+
+typedef enum {
+    MAMBA_F32 = 0,
+    MAMBA_BF16 = 1
+} mamba_dtype_t;
+
+/* Flags (mamba_dims_t.flags). */
+#define MAMBA_FLAG_NO_TMA 0x1          /* stage tiles with plain loads instead of TMA */
+#define MAMBA_FLAG_PARALLEL_CHUNKS 0x2 /* with num_chunks >= 1: parallel (recompute) mode */
+
+#define MAMBA_MAX_DSTATE 16
+
+/*
+ * Sizes and options of one call.
+ *   batch, dim, dstate   B, D (channels) and N (state size, 1..16)
+ *   seqlen               L for the scan; ignored by the update
+ *   io_dtype             dtype of u, delta, z, out (update: x, dt, z, out)
+ *   bc_dtype             dtype of B and C
+ *   dt_softplus          update only: apply softplus to dt + dt_bias (0/1)
+ *   num_chunks           scan only: 0 = automatic; k >= 1 forces the sequence
+ *                        to be split into k segments (k = 1: one segment)
+ *   flags                MAMBA_FLAG_*
+ *   workspace            scan only: device scratch of at least
+ *                        mamba_selective_scan_workspace_bytes() bytes, 256-byte
+ *                        aligned, owned by the caller.  The call zeroes a few KB
+ *                        at its start (counters, flags) on `stream`; concurrent
+ *                        calls need separate workspaces.
+ */
+typedef struct {
+    int64_t batch;
+    int64_t dim;
+    int64_t dstate;
+    int64_t seqlen;
+    int32_t io_dtype;
+    int32_t bc_dtype;
+    int32_t dt_softplus;
+    int32_t num_chunks;
+    int32_t flags;
+    int32_t reserved;
+    void *workspace;
+    size_t workspace_bytes;
+} mamba_dims_t;
+
+/*
+ * How a scan call will run (host-side planning; no CUDA call is made).
+ * The channels form groups of 32 (one warp each); the sequence is cut into
+ * nchunks segments of chunk_len steps (the last may be shorter).  A persistent
+ * grid of warps pulls (segment, group) work items from a counter.
+ *   mode 0 (chained): one launch.  Segment k of a group starts from the state
+ *     segment k-1 left in the workspace; no work is repeated.  Used when there
+ *     are enough groups to occupy the GPU; nchunks only balances the load.
+ *   mode 1 (parallel): two launches, for few channels and long sequences.
+ *     Pass A runs segments 0..nchunks-2 at once: segment 0 writes its outputs
+ *     and end state, the others only their end state from a zero start and
+ *     the sum of Delta.  Pass B runs segments 1..nchunks-1 at once, each
+ *     folding the earlier segments' (exp(A sum Delta), end state) pairs into
+ *     its true start state before recomputing its outputs.
+ */
+typedef struct {
+    int32_t nchunks;           /* segments per sequence */
+    int32_t tile_len;          /* time steps staged per pipeline stage */
+    int64_t chunk_len;         /* time steps per segment (multiple of tile_len) */
+    int64_t groups;            /* batch * ceil(dim / 32) */
+    int64_t units_pass_a;      /* work items of the first launch */
+    int64_t units_pass_b;      /* work items of the second launch (0 in mode 0) */
+    int32_t warps_per_cta;
+    int32_t launches;          /* kernel launches per call (plus one memset) */
+    int32_t tma_capable;       /* strides allow TMA staging */
+    int32_t mode;              /* 0 chained, 1 parallel */
+    size_t workspace_bytes;
+} mamba_scan_plan_t;
+
+/*
+ * Plan a scan for `dims` on a GPU with `sm_count` SMs.  Pure host function.
+ * Returns MAMBA_ERR_INVALID_ARG / MAMBA_ERR_UNSUPPORTED for bad dims.
+ */
+MAMBA_API mamba_status_t mamba_selective_scan_plan(const mamba_dims_t *dims, int sm_count,
+                                                   mamba_scan_plan_t *plan);
+
+/*
+ * Scratch bytes mamba_selective_scan_fwd needs for `dims` on the current
+ * device: a few KB of counters and flags plus the segment carry (64 bytes per
+ * chain in mode 0, 68 bytes per chain and segment in mode 1).  0 for empty
+ * problems.  Returns (size_t)-1 on bad dims or when the current device cannot
+ * be queried.
+ */
+MAMBA_API size_t mamba_selective_scan_workspace_bytes(const mamba_dims_t *dims);
+
+/*
+ * Selective scan forward.
+ *   u, delta, z, out   (batch, dim, seqlen), io_dtype; z may be NULL (no gate)
+ *   A                  (dim, dstate) fp32
+ *   B, C               (batch, dstate, seqlen), bc_dtype, shared by all channels
+ *   D, delta_bias      (dim,) fp32; may be NULL (treated as 0)
+ *   softplus           nonzero: Delta = softplus(delta + delta_bias)
+ *   last_state         (batch, dim, dstate) fp32 = h at t = seqlen-1; may be NULL
+ *   dims->workspace    required (see mamba_selective_scan_workspace_bytes)
+ * seqlen == 0 writes no output; last_state (if given) is set to zero.
+ * Returns MAMBA_ERR_WORKSPACE if the workspace is missing or too small.
+ */
+MAMBA_API mamba_status_t mamba_selective_scan_fwd(const void *u, const void *delta, const float *A,
+                                                  const void *B, const void *C, const float *D,
+                                                  const void *z, const float *delta_bias,
+                                                  int softplus, void *out, float *last_state,
+                                                  const mamba_dims_t *dims, cudaStream_t stream);
+
+/*
+ * Single-token state update (generation).  The state is read and written in
+ * place.
+ *   state              (batch, dim, dstate) fp32, updated in place
+ *   x, dt, z, out      (batch, dim), io_dtype; z may be NULL
+ *   A                  (dim, dstate) fp32
+ *   B, C               (batch, dstate), bc_dtype
+ *   D, dt_bias         (dim,) fp32; may be NULL
+ *   dims->dt_softplus  nonzero: Delta = softplus(dt + dt_bias)
+ * dims->seqlen, num_chunks and workspace are ignored.
+ */
+MAMBA_API mamba_status_t mamba_selective_state_update(float *state, const void *x, const void *dt,
+                                                      const float *A, const void *B, const void *C,
+                                                      const float *D, const void *z,
+                                                      const float *dt_bias, void *out,
+                                                      const mamba_dims_t *dims,
+                                                      cudaStream_t stream);
+
+/*
+ * Read and clear the library's device-side status word on the current device
+ * (synchronises the device).  Returns MAMBA_OK, or the first device-side
+ * error recorded since the last call (e.g. MAMBA_ERR_TIMEOUT).
+ */
+MAMBA_API mamba_status_t mamba_device_status(void);
+
+/* Static, human-readable name of a status code. */
+MAMBA_API const char *mamba_status_string(mamba_status_t status);
+
+/* Library version as "major.minor.patch". */
+MAMBA_API const char *mamba_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MAMBA_SSM_H */

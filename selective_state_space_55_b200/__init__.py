@@ -1,0 +1,16 @@
+"""Selective-SSM scan and single-token state update for NVIDIA B200 (sm_100a).
+
+The computation lives in ``libmamba_ssm.so`` (hand-written CUDA behind the C
+ABI of ``include/mamba_ssm.h``); ``ops`` is its ctypes binding and ``inputs``
+the seeded synthetic workloads.
+"""
+from . import inputs  # noqa: F401
+from .ops import (  # noqa: F401
+    MambaError, device_status, scan_plan, scan_workspace_bytes, selective_scan_fwd,
+    selective_state_update, status_string, version,
+)
+
+__all__ = [
+    "inputs", "MambaError", "device_status", "scan_plan", "scan_workspace_bytes",
+    "selective_scan_fwd", "selective_state_update", "status_string", "version",
+]

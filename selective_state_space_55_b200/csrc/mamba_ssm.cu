@@ -1,0 +1,459 @@
+// C ABI of the selective-SSM library: argument validation, planning, TMA
+// descriptor set-up and kernel dispatch.  One translation unit holds every
+// kernel so that device globals need no separate device link.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+
+#include "mamba_ssm.h"
+#include "selective_scan.cuh"
+#include "state_update.cuh"
+
+namespace mamba {
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+int dtype_bytes(int32_t dt) { return dt == MAMBA_BF16 ? 2 : 4; }
+bool dtype_ok(int32_t dt) { return dt == MAMBA_F32 || dt == MAMBA_BF16; }
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+mamba_status_t check_dims(const mamba_dims_t* dims, bool scan) {
+    if (dims == nullptr) return MAMBA_ERR_INVALID_ARG;
+    if (dims->batch < 0 || dims->dim < 0 || dims->dstate < 0) return MAMBA_ERR_INVALID_ARG;
+    if (scan && dims->seqlen < 0) return MAMBA_ERR_INVALID_ARG;
+    if (scan && dims->num_chunks < 0) return MAMBA_ERR_INVALID_ARG;
+    if (dims->dstate < 1 || dims->dstate > MAMBA_MAX_DSTATE) return MAMBA_ERR_UNSUPPORTED;
+    if (!dtype_ok(dims->io_dtype) || !dtype_ok(dims->bc_dtype)) return MAMBA_ERR_UNSUPPORTED;
+    // Index arithmetic inside the kernels is 64-bit; TMA coordinates are
+    // 32-bit, so keep every extent below 2^31.
+    const int64_t lim = (int64_t)1 << 31;
+    if (dims->batch >= lim || dims->dim >= lim || (scan && dims->seqlen >= lim))
+        return MAMBA_ERR_INVALID_ARG;
+    return MAMBA_OK;
+}
+
+// SM count of the current device, cached per device.
+int current_sm_count(int* device_out) {
+    static int cached[kMaxDevices] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    if (device_out) *device_out = dev;
+    if (dev >= 0 && dev < kMaxDevices && cached[dev] > 0) return cached[dev];
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+    if (dev >= 0 && dev < kMaxDevices) cached[dev] = sms;
+    return sms;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// 3-D map over a row-major (d2, d1, d0) tensor, d0 innermost, box (box0, box1, 1).
+bool encode_map_3d(CUtensorMap* map, const void* base, int esize, uint64_t d0, uint64_t d1,
+                   uint64_t d2, uint32_t box0, uint32_t box1, CUtensorMapSwizzle swizzle) {
+    auto encode = tensor_map_encoder();
+    if (encode == nullptr) return false;
+    const cuuint64_t dims[3] = {d0, d1, d2};
+    const cuuint64_t strides[2] = {d0 * esize, d0 * d1 * esize};
+    const cuuint32_t box[3] = {box0, box1, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUtensorMapDataType dt =
+        esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    const CUresult r = encode(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <typename Kernel>
+cudaError_t ensure_smem_attr(Kernel kernel, int bytes, bool* done_per_device, int dev) {
+    if (dev >= 0 && dev < kMaxDevices && done_per_device[dev]) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && dev >= 0 && dev < kMaxDevices) done_per_device[dev] = true;
+    return e;
+}
+
+template <typename IoT, bool kHasZ, bool kSoftplus>
+cudaError_t launch_scan(const ScanParams& prm, const CUtensorMap* maps, int dev, int sms,
+                        cudaStream_t stream) {
+    static bool attr_done[kMaxDevices] = {false};
+    static int resident[kMaxDevices] = {0};
+    auto kernel = selective_scan_fwd_kernel<IoT, kHasZ, kSoftplus>;
+    cudaError_t e = ensure_smem_attr(kernel, kScanSmemBytes, attr_done, dev);
+    if (e != cudaSuccess) return e;
+    int per_sm = (dev >= 0 && dev < kMaxDevices) ? resident[dev] : 0;
+    if (per_sm <= 0) {
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kScanWarps * 32,
+                                                          kScanSmemBytes);
+        if (e != cudaSuccess) return e;
+        if (per_sm <= 0) return cudaErrorInvalidConfiguration;
+        if (dev >= 0 && dev < kMaxDevices) resident[dev] = per_sm;
+    }
+    // Persistent grid: every warp keeps pulling work items until none are left.
+    const int64_t want = (prm.items + kScanWarps - 1) / kScanWarps;
+    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)per_sm * sms));
+    kernel<<<(unsigned)grid, kScanWarps * 32, kScanSmemBytes, stream>>>(prm, maps[0], maps[1],
+                                                                          maps[2], maps[3], maps[4]);
+    return cudaGetLastError();
+}
+
+template <typename IoT>
+cudaError_t dispatch_scan(const ScanParams& prm, const CUtensorMap* maps, bool has_z, bool sp,
+                          int dev, int sms, cudaStream_t stream) {
+    if (has_z)
+        return sp ? launch_scan<IoT, true, true>(prm, maps, dev, sms, stream)
+                  : launch_scan<IoT, true, false>(prm, maps, dev, sms, stream);
+    return sp ? launch_scan<IoT, false, true>(prm, maps, dev, sms, stream)
+              : launch_scan<IoT, false, false>(prm, maps, dev, sms, stream);
+}
+
+template <typename IoT, typename BcT>
+cudaError_t dispatch_update_bc(const UpdateParams& prm, bool fast, bool has_z,
+                               cudaStream_t stream) {
+    if (fast) {
+        // x covers channels (kUpdateChainsPerCta per CTA), y covers batch rows.
+        const dim3 grid((unsigned)((prm.dim + kUpdateChainsPerCta - 1) / kUpdateChainsPerCta),
+                        (unsigned)std::min<int64_t>(prm.batch, 65535));
+        if (has_z)
+            state_update_n16_kernel<IoT, BcT, true><<<grid, kUpdateThreads, 0, stream>>>(prm);
+        else
+            state_update_n16_kernel<IoT, BcT, false><<<grid, kUpdateThreads, 0, stream>>>(prm);
+    } else {
+        const unsigned grid = (unsigned)((prm.chains + kUpdateThreads - 1) / kUpdateThreads);
+        if (has_z)
+            state_update_generic_kernel<IoT, BcT, true><<<grid, kUpdateThreads, 0, stream>>>(prm);
+        else
+            state_update_generic_kernel<IoT, BcT, false><<<grid, kUpdateThreads, 0, stream>>>(prm);
+    }
+    return cudaGetLastError();
+}
+
+template <typename IoT>
+cudaError_t dispatch_update(const UpdateParams& prm, bool bc_bf16, bool fast, bool has_z,
+                            cudaStream_t stream) {
+    return bc_bf16 ? dispatch_update_bc<IoT, __nv_bfloat16>(prm, fast, has_z, stream)
+                   : dispatch_update_bc<IoT, float>(prm, fast, has_z, stream);
+}
+
+}  // namespace
+
+// Scratch layout of one scan call (offsets in bytes).
+struct ScanWorkspace {
+    size_t zeroed;      // prefix cleared before every call: counters and flags
+    size_t carry;       // chained mode: [chains][16] fp32
+    size_t ws_h;        // parallel mode: [K-1][chains][16] fp32
+    size_t ws_sdt;      // parallel mode: [K-1][chains] fp32
+    size_t total;
+};
+
+ScanWorkspace scan_workspace_layout(const mamba_dims_t* dims, int64_t groups, int64_t K, int mode) {
+    ScanWorkspace w{};
+    const size_t chains = (size_t)dims->batch * (size_t)dims->dim;
+    w.zeroed = kWsFlags + align256((size_t)groups * sizeof(unsigned int));
+    size_t off = w.zeroed;
+    if (mode == 0 && K > 1) {
+        w.carry = off;
+        off += align256(chains * kNPad * sizeof(float));
+    }
+    if (mode == 1) {
+        w.ws_h = off;
+        off += align256((size_t)(K - 1) * chains * kNPad * sizeof(float));
+        w.ws_sdt = off;
+        off += align256((size_t)(K - 1) * chains * sizeof(float));
+    }
+    w.total = off;
+    return w;
+}
+
+// Planning rules (pure host logic, see mamba_selective_scan_plan).
+//  - W = resident warps on the GPU (16 per SM), G = channel groups of 32.
+//  - G >= W: chained mode, K segments so that G*K is about 8 W work items
+//    (even load across SMs), segments at least 256 steps long.
+//  - W/4 <= G < W: one segment per group (every chain stays on one warp).
+//  - G < W/4: parallel mode, K-1 = W/G segments per pass (every resident
+//    warp busy), segments at least 16 tiles and 512 steps long.
+//  - num_chunks >= 1 forces K; MAMBA_FLAG_PARALLEL_CHUNKS forces the parallel
+//    mode for a forced K.
+mamba_status_t plan_scan(const mamba_dims_t* dims, int sm_count, mamba_scan_plan_t* plan) {
+    mamba_status_t st = check_dims(dims, true);
+    if (st != MAMBA_OK) return st;
+    if (plan == nullptr || sm_count <= 0) return MAMBA_ERR_INVALID_ARG;
+    *plan = mamba_scan_plan_t{};
+    const int io_es = dtype_bytes(dims->io_dtype);
+    const int bc_es = dtype_bytes(dims->bc_dtype);
+    const int64_t T = kRowBytes / io_es;
+    const int64_t L = dims->seqlen;
+    const int64_t gpb = (dims->dim + kGroupRows - 1) / kGroupRows;
+    const int64_t groups = dims->batch * gpb;
+    const int64_t W = (int64_t)sm_count * kScanWarpsPerSm;
+    plan->tile_len = (int32_t)T;
+    plan->groups = groups;
+    plan->warps_per_cta = kScanWarps;
+    plan->tma_capable = (L > 0 && (L * io_es) % 16 == 0 && (L * bc_es) % 16 == 0) ? 1 : 0;
+
+    int64_t K = 1;
+    int mode = 0;
+    if (dims->num_chunks >= 1) {
+        K = dims->num_chunks;
+        mode = (dims->flags & MAMBA_FLAG_PARALLEL_CHUNKS) ? 1 : 0;
+    } else if (groups > 0 && L > 0) {
+        if (groups >= W) {
+            const int64_t want = (8 * W + groups - 1) / groups;
+            K = std::max<int64_t>(1, std::min<int64_t>(want, L / 256));
+        } else if (groups * 4 >= W) {
+            K = 1;
+        } else {
+            mode = 1;
+            K = std::max<int64_t>(
+                1, std::min<int64_t>(W / groups + 1, L / std::max<int64_t>(16 * T, 512)));
+        }
+    }
+    int64_t seg_len = L;
+    if (K > 1 && L > 0) {
+        seg_len = ((L + K - 1) / K + T - 1) / T * T;
+        K = (L + seg_len - 1) / seg_len;
+    }
+    if (K <= 1) {
+        K = 1;
+        seg_len = L;
+        mode = 0;
+    }
+    const int64_t items = mode == 0 ? groups * K : groups * (K - 1);
+    if (items >= ((int64_t)1 << 31)) return MAMBA_ERR_UNSUPPORTED;
+    plan->nchunks = (int32_t)K;
+    plan->chunk_len = seg_len;
+    plan->mode = mode;
+    plan->units_pass_a = items;
+    plan->units_pass_b = mode == 0 ? 0 : items;
+    plan->launches = (groups > 0 && L > 0) ? (mode == 0 ? 1 : 2) : 0;
+    plan->workspace_bytes =
+        (groups > 0 && L > 0) ? scan_workspace_layout(dims, groups, K, mode).total : 0;
+    return MAMBA_OK;
+}
+
+}  // namespace mamba
+
+using namespace mamba;
+
+extern "C" {
+
+MAMBA_API mamba_status_t mamba_selective_scan_plan(const mamba_dims_t* dims, int sm_count,
+                                                   mamba_scan_plan_t* plan) {
+    return plan_scan(dims, sm_count, plan);
+}
+
+MAMBA_API size_t mamba_selective_scan_workspace_bytes(const mamba_dims_t* dims) {
+    const int sms = current_sm_count(nullptr);
+    if (sms <= 0) return static_cast<size_t>(-1);
+    mamba_scan_plan_t plan;
+    if (plan_scan(dims, sms, &plan) != MAMBA_OK) return static_cast<size_t>(-1);
+    return plan.workspace_bytes;
+}
+
+MAMBA_API mamba_status_t mamba_selective_scan_fwd(const void* u, const void* delta, const float* A,
+                                                  const void* B, const void* C, const float* D,
+                                                  const void* z, const float* delta_bias,
+                                                  int softplus, void* out, float* last_state,
+                                                  const mamba_dims_t* dims, cudaStream_t stream) {
+    mamba_status_t st = check_dims(dims, true);
+    if (st != MAMBA_OK) return st;
+    // Empty problems first: tensors without elements may have null pointers.
+    const int64_t chains = dims->batch * dims->dim;
+    if (chains == 0) return MAMBA_OK;
+    if (dims->seqlen == 0) {
+        if (last_state == nullptr) return MAMBA_OK;
+        if (!aligned(last_state, 4)) return MAMBA_ERR_ALIGN;
+        const cudaError_t e = cudaMemsetAsync(last_state, 0,
+                                              (size_t)chains * dims->dstate * sizeof(float), stream);
+        return e == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
+    }
+    if (u == nullptr || delta == nullptr || A == nullptr || B == nullptr || C == nullptr ||
+        out == nullptr)
+        return MAMBA_ERR_INVALID_ARG;
+    const int io_es = dtype_bytes(dims->io_dtype);
+    const int bc_es = dtype_bytes(dims->bc_dtype);
+    if (!aligned(u, io_es) || !aligned(delta, io_es) || !aligned(out, io_es) ||
+        (z && !aligned(z, io_es)) || !aligned(B, bc_es) || !aligned(C, bc_es) || !aligned(A, 4) ||
+        (D && !aligned(D, 4)) || (delta_bias && !aligned(delta_bias, 4)) ||
+        (last_state && !aligned(last_state, 4)))
+        return MAMBA_ERR_ALIGN;
+
+    int dev = 0;
+    const int sms = current_sm_count(&dev);
+    if (sms <= 0) return MAMBA_ERR_CUDA;
+    mamba_scan_plan_t plan;
+    st = plan_scan(dims, sms, &plan);
+    if (st != MAMBA_OK) return st;
+    if (dims->workspace == nullptr || dims->workspace_bytes < plan.workspace_bytes)
+        return MAMBA_ERR_WORKSPACE;
+    if (!aligned(dims->workspace, 256)) return MAMBA_ERR_ALIGN;
+
+    ScanParams prm{};
+    prm.u = u;
+    prm.delta = delta;
+    prm.z = z;
+    prm.A = A;
+    prm.B = B;
+    prm.C = C;
+    prm.D = D;
+    prm.delta_bias = delta_bias;
+    prm.out = out;
+    prm.last_state = last_state;
+    prm.batch = dims->batch;
+    prm.dim = dims->dim;
+    prm.seqlen = dims->seqlen;
+    prm.groups_per_batch = (dims->dim + kGroupRows - 1) / kGroupRows;
+    prm.groups = plan.groups;
+    prm.chains = chains;
+    prm.seg_len = plan.chunk_len;
+    prm.dstate = (int)dims->dstate;
+    prm.nseg = plan.nchunks;
+    prm.bc_bf16 = dims->bc_dtype == MAMBA_BF16;
+    prm.vec_out = ((dims->seqlen * io_es) % 16 == 0) && aligned(out, 16);
+    uint8_t* ws = static_cast<uint8_t*>(dims->workspace);
+    const ScanWorkspace lay = scan_workspace_layout(dims, plan.groups, plan.nchunks, plan.mode);
+    unsigned int* counters = reinterpret_cast<unsigned int*>(ws + kWsCounters);
+    prm.flags = reinterpret_cast<unsigned int*>(ws + kWsFlags);
+    if (lay.carry) prm.carry = reinterpret_cast<float*>(ws + lay.carry);
+    if (lay.ws_h) prm.ws_h = reinterpret_cast<float*>(ws + lay.ws_h);
+    if (lay.ws_sdt) prm.ws_sdt = reinterpret_cast<float*>(ws + lay.ws_sdt);
+
+    const bool use_tma = plan.tma_capable && !(dims->flags & MAMBA_FLAG_NO_TMA) &&
+                         aligned(u, 16) && aligned(delta, 16) && (!z || aligned(z, 16)) &&
+                         aligned(B, 16) && aligned(C, 16) && tensor_map_encoder() != nullptr;
+    prm.use_tma = use_tma ? 1 : 0;
+    CUtensorMap maps[5];
+    std::memset(maps, 0, sizeof(maps));
+    if (use_tma) {
+        const uint32_t T = (uint32_t)plan.tile_len;
+        const uint64_t L = (uint64_t)dims->seqlen;
+        const uint64_t Dm = (uint64_t)dims->dim, Bt = (uint64_t)dims->batch;
+        const uint64_t N = (uint64_t)dims->dstate;
+        bool ok = encode_map_3d(&maps[0], u, io_es, L, Dm, Bt, T, kGroupRows,
+                                CU_TENSOR_MAP_SWIZZLE_32B) &&
+                  encode_map_3d(&maps[1], delta, io_es, L, Dm, Bt, T, kGroupRows,
+                                CU_TENSOR_MAP_SWIZZLE_32B) &&
+                  encode_map_3d(&maps[2], z ? z : u, io_es, L, Dm, Bt, T, kGroupRows,
+                                CU_TENSOR_MAP_SWIZZLE_32B) &&
+                  encode_map_3d(&maps[3], B, bc_es, L, N, Bt, T, (uint32_t)N,
+                                CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                  encode_map_3d(&maps[4], C, bc_es, L, N, Bt, T, (uint32_t)N,
+                                CU_TENSOR_MAP_SWIZZLE_NONE);
+        if (!ok) {
+            prm.use_tma = 0;
+            std::memset(maps, 0, sizeof(maps));
+        }
+    }
+
+    // Counters and flags start at zero on every call.
+    if (cudaMemsetAsync(ws, 0, lay.zeroed, stream) != cudaSuccess) return MAMBA_ERR_CUDA;
+    const bool has_z = z != nullptr;
+    const bool sp = softplus != 0;
+    auto run = [&](int mode, unsigned int* counter, int64_t items) -> cudaError_t {
+        prm.mode = mode;
+        prm.counter = counter;
+        prm.items = items;
+        if (items == 0) return cudaSuccess;
+        return dims->io_dtype == MAMBA_BF16
+                   ? dispatch_scan<__nv_bfloat16>(prm, maps, has_z, sp, dev, sms, stream)
+                   : dispatch_scan<float>(prm, maps, has_z, sp, dev, sms, stream);
+    };
+    cudaError_t e;
+    if (plan.mode == 0) {
+        e = run(kModeChained, counters, plan.units_pass_a);
+    } else {
+        e = run(kModePassA, counters, plan.units_pass_a);
+        if (e == cudaSuccess) e = run(kModePassB, counters + 1, plan.units_pass_b);
+    }
+    return e == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
+}
+
+MAMBA_API mamba_status_t mamba_selective_state_update(float* state, const void* x, const void* dt,
+                                                      const float* A, const void* B, const void* C,
+                                                      const float* D, const void* z,
+                                                      const float* dt_bias, void* out,
+                                                      const mamba_dims_t* dims,
+                                                      cudaStream_t stream) {
+    mamba_status_t st = check_dims(dims, false);
+    if (st != MAMBA_OK) return st;
+    const int64_t chains = dims->batch * dims->dim;
+    if (chains == 0) return MAMBA_OK;
+    if (state == nullptr || x == nullptr || dt == nullptr || A == nullptr || B == nullptr ||
+        C == nullptr || out == nullptr)
+        return MAMBA_ERR_INVALID_ARG;
+    const int io_es = dtype_bytes(dims->io_dtype);
+    const int bc_es = dtype_bytes(dims->bc_dtype);
+    if (!aligned(state, 4) || !aligned(x, io_es) || !aligned(dt, io_es) || !aligned(out, io_es) ||
+        (z && !aligned(z, io_es)) || !aligned(B, bc_es) || !aligned(C, bc_es) || !aligned(A, 4) ||
+        (D && !aligned(D, 4)) || (dt_bias && !aligned(dt_bias, 4)))
+        return MAMBA_ERR_ALIGN;
+
+    UpdateParams prm{};
+    prm.state = state;
+    prm.x = x;
+    prm.dt = dt;
+    prm.A = A;
+    prm.B = B;
+    prm.C = C;
+    prm.D = D;
+    prm.z = z;
+    prm.dt_bias = dt_bias;
+    prm.out = out;
+    prm.batch = dims->batch;
+    prm.dim = dims->dim;
+    prm.chains = chains;
+    prm.dstate = (int)dims->dstate;
+    prm.dt_softplus = dims->dt_softplus != 0;
+    const bool fast = dims->dstate == 16 && aligned(state, 16) && aligned(A, 16) &&
+                      aligned(B, 4 * bc_es) && aligned(C, 4 * bc_es);
+    const bool has_z = z != nullptr;
+    const bool bc_bf16 = dims->bc_dtype == MAMBA_BF16;
+    const cudaError_t e = dims->io_dtype == MAMBA_BF16
+                              ? dispatch_update<__nv_bfloat16>(prm, bc_bf16, fast, has_z, stream)
+                              : dispatch_update<float>(prm, bc_bf16, fast, has_z, stream);
+    return e == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
+}
+
+MAMBA_API mamba_status_t mamba_device_status(void) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return MAMBA_ERR_CUDA;
+    int code = 0;
+    if (cudaMemcpyFromSymbol(&code, g_device_status, sizeof(int)) != cudaSuccess)
+        return MAMBA_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess)
+        return MAMBA_ERR_CUDA;
+    return static_cast<mamba_status_t>(code);
+}
+
+MAMBA_API const char* mamba_status_string(mamba_status_t status) {
+    switch (status) {
+        case MAMBA_OK: return "MAMBA_OK";
+        case MAMBA_ERR_INVALID_ARG: return "MAMBA_ERR_INVALID_ARG";
+        case MAMBA_ERR_UNSUPPORTED: return "MAMBA_ERR_UNSUPPORTED";
+        case MAMBA_ERR_ALIGN: return "MAMBA_ERR_ALIGN";
+        case MAMBA_ERR_WORKSPACE: return "MAMBA_ERR_WORKSPACE";
+        case MAMBA_ERR_CUDA: return "MAMBA_ERR_CUDA";
+        case MAMBA_ERR_TIMEOUT: return "MAMBA_ERR_TIMEOUT";
+    }
+    return "MAMBA_ERR_UNKNOWN";
+}
+
+MAMBA_API const char* mamba_version(void) { return "0.1.0"; }
+
+}  // extern "C"

@@ -1,0 +1,232 @@
+"""Python binding of the C ABI in ``include/mamba_ssm.h`` (ctypes).
+
+Argument marshalling only: tensors are checked for device, dtype and layout,
+their data pointers and sizes are packed into ``mamba_dims_t`` and the call
+goes to ``libmamba_ssm.so``.  Every step of the computation runs in the
+library's CUDA kernels; PyTorch only supplies device memory (including the
+scan's scratch workspace) and the current stream.  There is no fallback: if
+the library cannot be loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+from pathlib import Path
+
+import torch
+
+PKG = Path(__file__).resolve().parent
+LIBRARY_PATH = PKG / "libmamba_ssm.so"
+
+MAMBA_OK = 0
+STATUS_NAMES = {
+    0: "MAMBA_OK", -1: "MAMBA_ERR_INVALID_ARG", -2: "MAMBA_ERR_UNSUPPORTED",
+    -3: "MAMBA_ERR_ALIGN", -4: "MAMBA_ERR_WORKSPACE", -5: "MAMBA_ERR_CUDA",
+    -6: "MAMBA_ERR_TIMEOUT",
+}
+MAMBA_F32, MAMBA_BF16 = 0, 1
+MAMBA_FLAG_NO_TMA = 0x1
+MAMBA_FLAG_PARALLEL_CHUNKS = 0x2
+
+_DTYPE_CODE = {torch.float32: MAMBA_F32, torch.bfloat16: MAMBA_BF16}
+
+
+class MambaDims(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int64), ("dim", ctypes.c_int64), ("dstate", ctypes.c_int64),
+        ("seqlen", ctypes.c_int64), ("io_dtype", ctypes.c_int32), ("bc_dtype", ctypes.c_int32),
+        ("dt_softplus", ctypes.c_int32), ("num_chunks", ctypes.c_int32),
+        ("flags", ctypes.c_int32), ("reserved", ctypes.c_int32),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+
+class ScanPlan(ctypes.Structure):
+    _fields_ = [
+        ("nchunks", ctypes.c_int32), ("tile_len", ctypes.c_int32),
+        ("chunk_len", ctypes.c_int64), ("groups", ctypes.c_int64),
+        ("units_pass_a", ctypes.c_int64), ("units_pass_b", ctypes.c_int64),
+        ("warps_per_cta", ctypes.c_int32), ("launches", ctypes.c_int32),
+        ("tma_capable", ctypes.c_int32), ("mode", ctypes.c_int32),
+        ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+    def as_dict(self) -> dict:
+        return {name: getattr(self, name) for name, _ in self._fields_}
+
+
+class MambaError(RuntimeError):
+    def __init__(self, call: str, status: int):
+        self.status = status
+        super().__init__(f"{call} failed: {STATUS_NAMES.get(status, status)}")
+
+
+_LIB = None
+
+
+def library(path: Path | str | None = None) -> ctypes.CDLL:
+    """Load (once) and return the CUDA library; raises if it is missing."""
+    global _LIB
+    if _LIB is not None and path is None:
+        return _LIB
+    p = Path(path) if path is not None else LIBRARY_PATH
+    if not p.exists():
+        raise RuntimeError(
+            f"{p} is missing: build it with `python -m selective_state_space_55_b200.build` "
+            "(there is no CPU fallback)")
+    lib = ctypes.CDLL(str(p))
+    vp, i32 = ctypes.c_void_p, ctypes.c_int
+    dims_p = ctypes.POINTER(MambaDims)
+    lib.mamba_selective_scan_plan.restype = i32
+    lib.mamba_selective_scan_plan.argtypes = [dims_p, i32, ctypes.POINTER(ScanPlan)]
+    lib.mamba_selective_scan_workspace_bytes.restype = ctypes.c_size_t
+    lib.mamba_selective_scan_workspace_bytes.argtypes = [dims_p]
+    lib.mamba_selective_scan_fwd.restype = i32
+    lib.mamba_selective_scan_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, dims_p, vp]
+    lib.mamba_selective_state_update.restype = i32
+    lib.mamba_selective_state_update.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, dims_p, vp]
+    lib.mamba_device_status.restype = i32
+    lib.mamba_device_status.argtypes = []
+    lib.mamba_status_string.restype = ctypes.c_char_p
+    lib.mamba_status_string.argtypes = [i32]
+    lib.mamba_version.restype = ctypes.c_char_p
+    lib.mamba_version.argtypes = []
+    if path is None:
+        _LIB = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return library().mamba_status_string(status).decode()
+
+
+def version() -> str:
+    return library().mamba_version().decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _check_cuda(name, t, dtypes, shape):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name}: dtype {t.dtype} not in {dtypes}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)} != {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _stream_handle(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def make_scan_dims(batch, dim, dstate, seqlen, io_dtype, bc_dtype, num_chunks=0, flags=0,
+                   workspace=None) -> MambaDims:
+    return MambaDims(batch=batch, dim=dim, dstate=dstate, seqlen=seqlen,
+                     io_dtype=_DTYPE_CODE[io_dtype], bc_dtype=_DTYPE_CODE[bc_dtype],
+                     dt_softplus=0, num_chunks=num_chunks, flags=flags, reserved=0,
+                     workspace=None if workspace is None else workspace.data_ptr(),
+                     workspace_bytes=0 if workspace is None else workspace.numel())
+
+
+def scan_plan(batch, dim, dstate, seqlen, io_dtype=torch.bfloat16, bc_dtype=torch.bfloat16,
+              num_chunks=0, sm_count=148, flags=0) -> dict:
+    """The library's plan for a scan of these sizes on a GPU with ``sm_count`` SMs."""
+    dims = make_scan_dims(batch, dim, dstate, seqlen, io_dtype, bc_dtype, num_chunks, flags)
+    plan = ScanPlan()
+    rc = library().mamba_selective_scan_plan(ctypes.byref(dims), sm_count, ctypes.byref(plan))
+    if rc != MAMBA_OK:
+        raise MambaError("mamba_selective_scan_plan", rc)
+    return plan.as_dict()
+
+
+def scan_workspace_bytes(batch, dim, dstate, seqlen, io_dtype=torch.bfloat16,
+                         bc_dtype=torch.bfloat16, num_chunks=0, flags=0) -> int:
+    """Scratch bytes the scan needs on the current device."""
+    dims = make_scan_dims(batch, dim, dstate, seqlen, io_dtype, bc_dtype, num_chunks, flags)
+    n = library().mamba_selective_scan_workspace_bytes(ctypes.byref(dims))
+    if n == ctypes.c_size_t(-1).value:
+        raise MambaError("mamba_selective_scan_workspace_bytes", -1)
+    return int(n)
+
+
+def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
+                       out=None, last_state=None, return_last_state=False, num_chunks=0,
+                       flags=0, workspace=None, stream=None):
+    """Selective scan forward through ``mamba_selective_scan_fwd``.
+
+    u, delta, z: (batch, dim, L) fp32 or bf16 (one dtype); B, C: (batch, N, L)
+    fp32 or bf16; A: (dim, N) fp32; D, delta_bias: (dim,) fp32 or None.
+    Returns ``out`` (batch, dim, L) in u's dtype, and the fp32 last state
+    (batch, dim, N) too when ``return_last_state`` or ``last_state`` is given.
+    """
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    io, bc = u.dtype, B.dtype
+    _check_cuda("u", u, (torch.float32, torch.bfloat16), (batch, dim, L))
+    _check_cuda("delta", delta, (io,), (batch, dim, L))
+    _check_cuda("z", z, (io,), (batch, dim, L))
+    _check_cuda("A", A, (torch.float32,), (dim, N))
+    _check_cuda("B", B, (torch.float32, torch.bfloat16), (batch, N, L))
+    _check_cuda("C", C, (bc,), (batch, N, L))
+    _check_cuda("D", D, (torch.float32,), (dim,))
+    _check_cuda("delta_bias", delta_bias, (torch.float32,), (dim,))
+    if out is None:
+        out = torch.empty_like(u)
+    _check_cuda("out", out, (io,), (batch, dim, L))
+    if last_state is None and return_last_state:
+        last_state = torch.empty((batch, dim, N), dtype=torch.float32, device=u.device)
+    _check_cuda("last_state", last_state, (torch.float32,), (batch, dim, N))
+    if workspace is None:
+        need = scan_workspace_bytes(batch, dim, N, L, io, bc, num_chunks, flags)
+        if need > 0:
+            workspace = torch.empty(need, dtype=torch.uint8, device=u.device)
+    dims = make_scan_dims(batch, dim, N, L, io, bc, num_chunks, flags, workspace)
+    rc = library().mamba_selective_scan_fwd(
+        _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
+        int(bool(softplus)), _ptr(out), _ptr(last_state), ctypes.byref(dims),
+        _stream_handle(stream))
+    if rc != MAMBA_OK:
+        raise MambaError("mamba_selective_scan_fwd", rc)
+    if last_state is not None:
+        return out, last_state
+    return out
+
+
+def selective_state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=None,
+                           dt_softplus=True, out=None, stream=None):
+    """One generation step through ``mamba_selective_state_update``; ``state`` is
+    updated in place.  Returns ``out`` (batch, dim) in x's dtype."""
+    batch, dim, N = state.shape
+    io, bc = x.dtype, B.dtype
+    _check_cuda("state", state, (torch.float32,), (batch, dim, N))
+    _check_cuda("x", x, (torch.float32, torch.bfloat16), (batch, dim))
+    _check_cuda("dt", dt, (io,), (batch, dim))
+    _check_cuda("z", z, (io,), (batch, dim))
+    _check_cuda("A", A, (torch.float32,), (dim, N))
+    _check_cuda("B", B, (torch.float32, torch.bfloat16), (batch, N))
+    _check_cuda("C", C, (bc,), (batch, N))
+    _check_cuda("D", D, (torch.float32,), (dim,))
+    _check_cuda("dt_bias", dt_bias, (torch.float32,), (dim,))
+    if out is None:
+        out = torch.empty_like(x)
+    _check_cuda("out", out, (io,), (batch, dim))
+    dims = MambaDims(batch=batch, dim=dim, dstate=N, seqlen=0, io_dtype=_DTYPE_CODE[io],
+                     bc_dtype=_DTYPE_CODE[bc], dt_softplus=int(bool(dt_softplus)),
+                     num_chunks=0, flags=0, reserved=0, workspace=None, workspace_bytes=0)
+    rc = library().mamba_selective_state_update(
+        _ptr(state), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+        _ptr(dt_bias), _ptr(out), ctypes.byref(dims), _stream_handle(stream))
+    if rc != MAMBA_OK:
+        raise MambaError("mamba_selective_state_update", rc)
+    return out
+
+
+def device_status() -> int:
+    """Read and clear the library's device-side status word (synchronises)."""
+    return int(library().mamba_device_status())

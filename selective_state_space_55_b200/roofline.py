@@ -1,0 +1,69 @@
+"""Algorithmic work of the scan and the update, and the B200 ceilings they meet.
+
+Scan, per element (b, d, t):
+  MUFU-class operations: 16 ex2 for Abar (one per state entry) + 2 for
+  softplus (ex2 and a reciprocal) + 2 for the silu gate (ex2 and a
+  reciprocal) = 20.  At 16 per clock per SM this is the binding pipe; the
+  bytes (u, delta, z read, out written, plus each batch row's B and C shared
+  by all channels) are about 8 per element in bf16, far below what HBM moves
+  in the same time.
+Update, per layer: the fp32 state is read and written once (2 x 64 bytes per
+  chain at N = 16) next to a few bytes of token inputs, so HBM bandwidth
+  bounds it.
+
+The state-size arithmetic of "Mamba 与状态空间模型" (section 固定大小的状态) and
+the KV-cache arithmetic of its section 越读越长的缓存 are reproduced by
+``state_numbers`` and ``kv_cache_bytes_per_token`` (the tests pin both to the
+page's printed figures).
+"""
+from __future__ import annotations
+
+MUFU_PER_SM_PER_CLOCK = 16
+EXP_PER_STATE = 1
+SOFTPLUS_MUFU = 2
+SILU_MUFU = 2
+
+
+def scan_mufu_per_element(dstate: int = 16, has_z: bool = True, softplus: bool = True) -> int:
+    return dstate * EXP_PER_STATE + (SOFTPLUS_MUFU if softplus else 0) + (SILU_MUFU if has_z else 0)
+
+
+def scan_bytes(batch: int, dim: int, dstate: int, seqlen: int, io_bytes: int = 2,
+               bc_bytes: int = 2, has_z: bool = True, last_state: bool = False) -> int:
+    """HBM bytes one scan must move: u, delta, (z) read, out written, B and C
+    read once per batch row, A/D/bias once, last_state written."""
+    elems = batch * dim * seqlen
+    io = elems * io_bytes * (3 + (1 if has_z else 0))
+    bc = 2 * batch * dstate * seqlen * bc_bytes
+    params = dim * dstate * 4 + 2 * dim * 4
+    tail = batch * dim * dstate * 4 if last_state else 0
+    return io + bc + params + tail
+
+
+def mufu_peak_elements_per_s(sm_count: int, sm_mhz: float, mufu_per_element: int) -> float:
+    """Elements per second if every SM's MUFU pipe issued every clock."""
+    return sm_count * MUFU_PER_SM_PER_CLOCK * sm_mhz * 1e6 / mufu_per_element
+
+
+def update_bytes(batch: int, dim: int, dstate: int, io_bytes: int = 2, bc_bytes: int = 2,
+                 has_z: bool = True) -> int:
+    """HBM bytes of one state update: state read + written, x, dt, (z) read,
+    out written, B and C, and the per-channel parameters."""
+    chains = batch * dim
+    state = 2 * chains * dstate * 4
+    tok = chains * io_bytes * (3 + (1 if has_z else 0))
+    bc = 2 * batch * dstate * bc_bytes
+    params = dim * dstate * 4 + 2 * dim * 4
+    return state + tok + bc + params
+
+
+def state_numbers(layers: int, channels: int, dstate: int, conv_taps: int) -> int:
+    """Numbers in a model's recurrent state: per layer and channel, dstate SSM
+    entries plus the short convolution's last conv_taps inputs."""
+    return layers * channels * (dstate + conv_taps)
+
+
+def kv_cache_bytes_per_token(layers: int, width: int, bytes_per_number: int) -> int:
+    """A Transformer's KV cache per token: a key and a value of `width`
+    numbers in every layer."""
+    return 2 * layers * width * bytes_per_number

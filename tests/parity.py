@@ -1,0 +1,35 @@
+"""Error metric and tolerances for comparing the CUDA path with the oracle.
+
+err = max_i |got_i - want_i| / max(|want_i|, rms(want)).  The denominator is
+the element's own magnitude, floored at the RMS of the reference so that
+elements near zero (an output gated by silu(z) ~ 0) do not divide by ~0.
+
+Tolerances: 1e-5 for fp32 inputs and outputs; 2e-2 for bf16 inputs/outputs
+with the fp32 state (the bf16 rounding of the output alone is up to 2^-9).
+"""
+import numpy as np
+import torch
+
+FP32_TOL = 1e-5
+BF16_TOL = 2e-2
+
+
+def as_f64(t):
+    if isinstance(t, torch.Tensor):
+        return t.detach().to("cpu").double().numpy()
+    return np.asarray(t, dtype=np.float64)
+
+
+def max_rel_err(got, want) -> float:
+    got, want = as_f64(got), as_f64(want)
+    assert got.shape == want.shape, (got.shape, want.shape)
+    if want.size == 0:
+        return 0.0
+    rms = float(np.sqrt(np.mean(want * want)))
+    denom = np.maximum(np.abs(want), rms)
+    denom = np.where(denom > 0, denom, 1.0)
+    return float(np.max(np.abs(got - want) / denom))
+
+
+def tol_for(dtype) -> float:
+    return FP32_TOL if dtype == torch.float32 else BF16_TOL

@@ -1,0 +1,169 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every symbol the header declares, plans scans as documented and rejects bad
+arguments before touching the device."""
+import ctypes
+import re
+from pathlib import Path
+
+import pytest
+import torch
+
+from selective_state_space_55_b200 import build, ops
+from selective_state_space_55_b200.inputs import SCAN_CONFIGS
+
+ROOT = Path(__file__).resolve().parent.parent
+HEADER = ROOT / "include" / "mamba_ssm.h"
+FAKE = ctypes.c_void_p(0x10000)        # never dereferenced: validation fails first
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return ops.library()
+
+
+def declared_symbols():
+    text = HEADER.read_text()
+    return re.findall(r"MAMBA_API\s+[\w\s\*]+?\b(mamba_\w+)\s*\(", text)
+
+
+def test_header_declares_entry_points():
+    syms = declared_symbols()
+    for name in ("mamba_selective_scan_fwd", "mamba_selective_state_update",
+                 "mamba_selective_scan_workspace_bytes", "mamba_selective_scan_plan",
+                 "mamba_status_string", "mamba_device_status", "mamba_version"):
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), f"{name} not exported"
+
+
+def test_status_strings(lib):
+    for code, name in ops.STATUS_NAMES.items():
+        assert ops.status_string(code) == name
+    assert ops.status_string(-99) == "MAMBA_ERR_UNKNOWN"
+
+
+def _dims(**kw):
+    base = dict(batch=2, dim=64, dstate=16, seqlen=128, io_dtype=torch.bfloat16,
+                bc_dtype=torch.bfloat16)
+    base.update(kw)
+    return ops.make_scan_dims(**base)
+
+
+def _scan(lib, dims, u=FAKE, delta=FAKE, A=FAKE, B=FAKE, C=FAKE, out=FAKE, D=None, z=None,
+          bias=None, last=None):
+    return lib.mamba_selective_scan_fwd(u, delta, A, B, C, D, z, bias, 1, out, last,
+                                        ctypes.byref(dims) if dims is not None else None, None)
+
+
+def test_scan_rejects_bad_arguments(lib):
+    assert _scan(lib, None) == -1
+    assert _scan(lib, _dims(batch=-1)) == -1
+    assert _scan(lib, _dims(seqlen=-5)) == -1
+    assert _scan(lib, _dims(dstate=0)) == -2
+    assert _scan(lib, _dims(dstate=17)) == -2
+    d = _dims(); d.io_dtype = 7
+    assert _scan(lib, d) == -2
+    d = _dims(); d.num_chunks = -1
+    assert _scan(lib, d) == -1
+    assert _scan(lib, _dims(), u=None) == -1
+    assert _scan(lib, _dims(), out=None) == -1
+    assert _scan(lib, _dims(), A=None) == -1
+    assert _scan(lib, _dims(), C=None) == -1
+    # bf16 tensors must be 2-byte aligned, fp32 tensors 4-byte aligned
+    assert _scan(lib, _dims(), u=ctypes.c_void_p(0x10001)) == -3
+    assert _scan(lib, _dims(), A=ctypes.c_void_p(0x10002)) == -3
+    assert _scan(lib, _dims(io_dtype=torch.float32), out=ctypes.c_void_p(0x10002)) == -3
+
+
+def test_scan_empty_batch_is_a_no_op(lib):
+    assert _scan(lib, _dims(batch=0)) == 0
+    assert _scan(lib, _dims(dim=0)) == 0
+
+
+def test_update_rejects_bad_arguments(lib):
+    def call(dims, state=FAKE, x=FAKE, out=FAKE):
+        return lib.mamba_selective_state_update(state, x, FAKE, FAKE, FAKE, FAKE, None, None,
+                                                None, out, ctypes.byref(dims), None)
+    good = ops.MambaDims(batch=4, dim=8, dstate=16, io_dtype=1, bc_dtype=1, dt_softplus=1)
+    assert call(ops.MambaDims(batch=4, dim=8, dstate=0, io_dtype=1, bc_dtype=1)) == -2
+    assert call(ops.MambaDims(batch=-4, dim=8, dstate=16, io_dtype=1, bc_dtype=1)) == -1
+    assert call(good, state=None) == -1
+    assert call(good, out=None) == -1
+    assert call(good, state=ctypes.c_void_p(0x10002)) == -3
+    assert call(ops.MambaDims(batch=0, dim=8, dstate=16, io_dtype=1, bc_dtype=1)) == 0
+
+
+def test_plan_layer_shapes(lib):
+    # 2.8B layer: 2560 groups >= 148 x 16 resident warps -> chained 256-step segments
+    c = SCAN_CONFIGS["mamba_2p8b_layer"]
+    p = ops.scan_plan(c.batch, c.dim, c.dstate, c.seqlen, c.io_dtype, c.bc_dtype)
+    assert p["mode"] == 0 and p["launches"] == 1
+    assert p["groups"] == c.batch * c.dim // 32
+    assert p["tile_len"] == 16 and p["tma_capable"] == 1
+    assert p["nchunks"] == 8 and p["chunk_len"] == 256
+    assert p["units_pass_a"] == p["groups"] * 8 and p["units_pass_b"] == 0
+    chains = c.batch * c.dim
+    flags = (p["groups"] * 4 + 255) // 256 * 256
+    assert p["workspace_bytes"] == 256 + flags + chains * 64
+    # 1.4B layer: 1024 groups, between a quarter and all of the resident warps -> one segment
+    c = SCAN_CONFIGS["mamba_1p4b_layer"]
+    p = ops.scan_plan(c.batch, c.dim, c.dstate, c.seqlen, c.io_dtype, c.bc_dtype)
+    assert p["mode"] == 0 and p["nchunks"] == 1 and p["units_pass_a"] == 1024
+    assert p["workspace_bytes"] == 256 + 4096
+
+
+def test_plan_parallel_for_the_million_token_sequence(lib):
+    c = SCAN_CONFIGS["long_dna_1m"]
+    p = ops.scan_plan(c.batch, c.dim, c.dstate, c.seqlen, c.io_dtype, c.bc_dtype, sm_count=148)
+    K = p["nchunks"]
+    assert p["mode"] == 1 and p["launches"] == 2
+    assert K - 1 == (148 * 16) // p["groups"]           # one item per resident warp and pass
+    assert p["chunk_len"] % p["tile_len"] == 0
+    assert (K - 1) * p["chunk_len"] < c.seqlen <= K * p["chunk_len"]
+    assert p["units_pass_a"] == p["units_pass_b"] == p["groups"] * (K - 1)
+    chains = c.batch * c.dim
+    expect = 256 + 256 + ((K - 1) * chains * 64 + 255) // 256 * 256 + \
+        ((K - 1) * chains * 4 + 255) // 256 * 256
+    assert p["workspace_bytes"] == expect
+
+
+def test_plan_tiny_is_one_segment(lib):
+    c = SCAN_CONFIGS["tiny_fp32"]
+    p = ops.scan_plan(c.batch, c.dim, c.dstate, c.seqlen, c.io_dtype, c.bc_dtype)
+    assert p["nchunks"] == 1 and p["mode"] == 0 and p["tile_len"] == 8
+    assert p["workspace_bytes"] == 512
+
+
+@pytest.mark.parametrize("L,K,want_k,want_len", [
+    (100, 5, 4, 32),        # segment length rounds up to the 16-step tile
+    (1000, 3, 3, 336),
+    (64, 8, 4, 16),
+    (31, 4, 2, 16),
+    (15, 4, 1, 15),         # shorter than a tile: one segment
+])
+def test_plan_forced_chunk_counts(lib, L, K, want_k, want_len):
+    p = ops.scan_plan(1, 32, 16, L, torch.bfloat16, torch.bfloat16, num_chunks=K)
+    assert p["nchunks"] == want_k and p["chunk_len"] == want_len
+    assert p["mode"] == 0
+    q = ops.scan_plan(1, 32, 16, L, torch.bfloat16, torch.bfloat16, num_chunks=K,
+                      flags=ops.MAMBA_FLAG_PARALLEL_CHUNKS)
+    assert q["nchunks"] == want_k and q["mode"] == (1 if want_k > 1 else 0)
+
+
+def test_plan_tma_capability_follows_strides(lib):
+    assert ops.scan_plan(1, 32, 16, 40, torch.bfloat16, torch.bfloat16)["tma_capable"] == 1
+    assert ops.scan_plan(1, 32, 16, 37, torch.bfloat16, torch.bfloat16)["tma_capable"] == 0
+    assert ops.scan_plan(1, 32, 16, 44, torch.float32, torch.float32)["tma_capable"] == 1
+    assert ops.scan_plan(1, 32, 16, 42, torch.float32, torch.float32)["tma_capable"] == 0
+    assert ops.scan_plan(1, 32, 16, 44, torch.float32, torch.bfloat16)["tma_capable"] == 0
+
+
+def test_plan_rejects_bad_dims(lib):
+    with pytest.raises(ops.MambaError):
+        ops.scan_plan(1, 32, 17, 64)
+    with pytest.raises(ops.MambaError):
+        ops.scan_plan(-1, 32, 16, 64)
