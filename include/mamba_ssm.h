@@ -78,6 +78,10 @@ typedef enum {
 /* Flags (mamba_dims_t.flags). */
 #define MAMBA_FLAG_NO_TMA 0x1          /* stage tiles with plain loads instead of TMA */
 #define MAMBA_FLAG_PARALLEL_CHUNKS 0x2 /* with num_chunks >= 1: parallel (recompute) mode */
+/* Test only: in mode 0, segments never hand their state on, so every wait for
+ * a predecessor runs out (after ~0.3 s) and the call reports MAMBA_ERR_TIMEOUT
+ * through mamba_device_status().  Outputs are then undefined. */
+#define MAMBA_FLAG_TEST_WITHHOLD_HANDOFF 0x4
 
 #define MAMBA_MAX_DSTATE 16
 

@@ -326,6 +326,14 @@ MAMBA_API mamba_status_t mamba_selective_scan_fwd(const void* u, const void* del
     prm.nseg = plan.nchunks;
     prm.bc_bf16 = dims->bc_dtype == MAMBA_BF16;
     prm.vec_out = ((dims->seqlen * io_es) % 16 == 0) && aligned(out, 16);
+    // A predecessor segment legitimately takes well under 64 us per step even
+    // on a crowded GPU; wait that long (at least ~1 s) before reporting a stall.
+    prm.withhold_handoff = (dims->flags & MAMBA_FLAG_TEST_WITHHOLD_HANDOFF) ? 1 : 0;
+    prm.flag_poll_limit =
+        prm.withhold_handoff
+            ? (1u << 18)
+            : (unsigned int)std::min<int64_t>(std::max<int64_t>(plan.chunk_len * 64, 1 << 20),
+                                              (int64_t)1 << 31);
     uint8_t* ws = static_cast<uint8_t*>(dims->workspace);
     const ScanWorkspace lay = scan_workspace_layout(dims, plan.groups, plan.nchunks, plan.mode);
     unsigned int* counters = reinterpret_cast<unsigned int*>(ws + kWsCounters);

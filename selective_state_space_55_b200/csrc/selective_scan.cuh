@@ -102,6 +102,8 @@ struct ScanParams {
     int use_tma;
     int bc_bf16;
     int vec_out;             // 16-byte output stores are aligned
+    unsigned int flag_poll_limit;   // chained mode: polls (~1 us each) before a wait gives up
+    int withhold_handoff;    // test only: segments never publish their state (waits time out)
 };
 
 // Byte offset of (row r, byte x of the row) in a 32-byte-row tile written by
@@ -397,9 +399,6 @@ __device__ __forceinline__ void st_release_gpu(unsigned int* p, unsigned int v) 
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-// Upper bound on polls of a predecessor's flag (each poll sleeps ~1 us).
-constexpr uint32_t kMaxFlagPolls = 1u << 22;
-
 template <typename IoT, bool kHasZ, bool kSoftplus>
 __global__ void __launch_bounds__(kScanWarps * 32, kScanMinBlocks)
     selective_scan_fwd_kernel(const __grid_constant__ ScanParams p,
@@ -459,7 +458,7 @@ __global__ void __launch_bounds__(kScanWarps * 32, kScanMinBlocks)
             bool ok = true;
             if (lane == 0) {
                 ok = false;
-                for (uint32_t i = 0; i < kMaxFlagPolls; ++i) {
+                for (uint32_t i = 0; i < p.flag_poll_limit; ++i) {
                     if (ld_acquire_gpu(p.flags + g) >= (unsigned int)k) {
                         ok = true;
                         break;
@@ -507,7 +506,8 @@ __global__ void __launch_bounds__(kScanWarps * 32, kScanMinBlocks)
                 if (valid) store16(p.carry + chain * kNPad, h);
                 __threadfence();
                 __syncwarp();
-                if (lane == 0) st_release_gpu(p.flags + g, (unsigned int)(k + 1));
+                if (lane == 0 && !p.withhold_handoff)
+                    st_release_gpu(p.flags + g, (unsigned int)(k + 1));
             }
         } else if (p.mode == kModePassA && valid) {
             store16(p.ws_h + (k * p.chains + chain) * kNPad, h);

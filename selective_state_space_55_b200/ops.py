@@ -26,6 +26,7 @@ STATUS_NAMES = {
 MAMBA_F32, MAMBA_BF16 = 0, 1
 MAMBA_FLAG_NO_TMA = 0x1
 MAMBA_FLAG_PARALLEL_CHUNKS = 0x2
+MAMBA_FLAG_TEST_WITHHOLD_HANDOFF = 0x4
 
 _DTYPE_CODE = {torch.float32: MAMBA_F32, torch.bfloat16: MAMBA_BF16}
 

@@ -307,3 +307,16 @@ def test_workspace_reuse_across_calls():
     torch.cuda.synchronize()
     assert ops.device_status() == 0
     assert torch.equal(a, b)
+
+
+def test_bounded_wait_reports_timeout():
+    """A predecessor that never hands its state on: the waits give up, the
+    status word says MAMBA_ERR_TIMEOUT, and the context stays usable."""
+    x = layer_inputs(1, 64, 1024, seed=33)
+    ops.selective_scan_fwd(x["u"], x["delta"], x["A"], x["B"], x["C"], num_chunks=4,
+                           flags=ops.MAMBA_FLAG_TEST_WITHHOLD_HANDOFF)
+    torch.cuda.synchronize()
+    assert ops.device_status() == -6
+    assert ops.device_status() == 0          # reading clears it
+    out, last = run_gpu(x, num_chunks=4)     # a normal call afterwards is fine
+    assert torch.isfinite(out.float()).all()
