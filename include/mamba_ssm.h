@@ -67,7 +67,8 @@ typedef enum {
     MAMBA_ERR_ALIGN = -3,         /* a pointer is not aligned to its element size */
     MAMBA_ERR_WORKSPACE = -4,     /* workspace missing or smaller than required */
     MAMBA_ERR_CUDA = -5,          /* a CUDA runtime call failed */
-    MAMBA_ERR_TIMEOUT = -6        /* a bounded device-side wait gave up */
+    MAMBA_ERR_TIMEOUT = -6,       /* a bounded device-side wait gave up */
+    MAMBA_ERR_TOO_LARGE = -7      /* needs more scratch than the built-in array holds */
 } mamba_status_t;
 
 typedef enum {
@@ -178,6 +179,42 @@ MAMBA_API mamba_status_t mamba_selective_scan_fwd(const void *u, const void *del
                                                   const void *z, const float *delta_bias,
                                                   int softplus, void *out, float *last_state,
                                                   const mamba_dims_t *dims, cudaStream_t stream);
+
+/*
+ * Selective scan forward that allocates nothing and takes no workspace.
+ *
+ * The paper has no counterpart to this entry point; it is a deployment aid.
+ * Some callers cannot allocate device memory: a host program whose device
+ * memory is owned by another allocator (a framework's caching allocator, a
+ * fixed arena) that forbids outside cudaMalloc calls, or latency-critical
+ * code that cannot pay for cudaMalloc/cudaFree and the device
+ * synchronisation they may imply.  This variant runs the same kernel as
+ * mamba_selective_scan_fwd with its scratch in a static device array of
+ * MAMBA_NOALLOC_SCRATCH_BYTES (8 MiB) that every GPU which loads the library
+ * holds until the process exits.  The caller still provides every input and
+ * output buffer; dims->workspace and dims->workspace_bytes are ignored.
+ *
+ *  - Arguments, layouts and results are those of mamba_selective_scan_fwd.
+ *  - Problems whose plan needs more than MAMBA_NOALLOC_SCRATCH_BYTES of
+ *    scratch are refused with MAMBA_ERR_TOO_LARGE before anything is
+ *    launched.  8 MiB covers, for example, chained segments of up to
+ *    131,000 (batch x channel) chains, which includes the Mamba-2.8B layer
+ *    shape (81,920 chains).
+ *  - The first call on each device looks up the array's device address with
+ *    cudaGetSymbolAddress, with that device current.  Make that first call
+ *    before any stream capture.
+ *  - Every call, on every stream, shares the one array per device.  Each call
+ *    clears the part that must start at zero, but calls whose executions
+ *    overlap on the GPU race on the array: run them in one stream or otherwise
+ *    one after another.
+ *  - Never calls cudaMalloc, cudaFree or any allocating library routine.
+ */
+#define MAMBA_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+
+MAMBA_API mamba_status_t mamba_selective_scan_fwd_noalloc(
+    const void *u, const void *delta, const float *A, const void *B, const void *C,
+    const float *D, const void *z, const float *delta_bias, int softplus, void *out,
+    float *last_state, const mamba_dims_t *dims, cudaStream_t stream);
 
 /*
  * Single-token state update (generation).  The state is read and written in

@@ -438,6 +438,70 @@ MAMBA_API mamba_status_t mamba_selective_state_update(float* state, const void* 
     return e == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Scan without a caller workspace (mamba_selective_scan_fwd_noalloc).
+//
+// For callers that may not allocate device memory, the scan's scratch lives
+// in this file-scope device array.  In host code `g_noalloc_scratch` names a
+// host-side stand-in, not a device address: its device address is looked up
+// per device with cudaGetSymbolAddress and passed to the kernels.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[MAMBA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+std::mutex g_noalloc_mutex;
+void* g_noalloc_address[kMaxDevices] = {nullptr};
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device (with that device current) and cached.
+mamba_status_t noalloc_scratch_address(void** address) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MAMBA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (dev >= 0 && dev < kMaxDevices && g_noalloc_address[dev] != nullptr) {
+        *address = g_noalloc_address[dev];
+        return MAMBA_OK;
+    }
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr)
+        return MAMBA_ERR_CUDA;
+    if (dev >= 0 && dev < kMaxDevices) g_noalloc_address[dev] = ptr;
+    *address = ptr;
+    return MAMBA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+MAMBA_API mamba_status_t mamba_selective_scan_fwd_noalloc(
+    const void* u, const void* delta, const float* A, const void* B, const void* C,
+    const float* D, const void* z, const float* delta_bias, int softplus, void* out,
+    float* last_state, const mamba_dims_t* dims, cudaStream_t stream) {
+    mamba_status_t st = check_dims(dims, true);
+    if (st != MAMBA_OK) return st;
+    mamba_dims_t local = *dims;
+    local.workspace = nullptr;
+    local.workspace_bytes = 0;
+    if (local.batch * local.dim > 0 && local.seqlen > 0) {
+        const int sms = current_sm_count(nullptr);
+        if (sms <= 0) return MAMBA_ERR_CUDA;
+        mamba_scan_plan_t plan;
+        st = plan_scan(&local, sms, &plan);
+        if (st != MAMBA_OK) return st;
+        if (plan.workspace_bytes > MAMBA_NOALLOC_SCRATCH_BYTES) return MAMBA_ERR_TOO_LARGE;
+        void* scratch = nullptr;
+        st = noalloc_scratch_address(&scratch);
+        if (st != MAMBA_OK) return st;
+        local.workspace = scratch;
+        local.workspace_bytes = MAMBA_NOALLOC_SCRATCH_BYTES;
+    }
+    return mamba_selective_scan_fwd(u, delta, A, B, C, D, z, delta_bias, softplus, out, last_state,
+                                    &local, stream);
+}
+
 MAMBA_API mamba_status_t mamba_device_status(void) {
     if (cudaDeviceSynchronize() != cudaSuccess) return MAMBA_ERR_CUDA;
     int code = 0;
@@ -458,6 +522,7 @@ MAMBA_API const char* mamba_status_string(mamba_status_t status) {
         case MAMBA_ERR_WORKSPACE: return "MAMBA_ERR_WORKSPACE";
         case MAMBA_ERR_CUDA: return "MAMBA_ERR_CUDA";
         case MAMBA_ERR_TIMEOUT: return "MAMBA_ERR_TIMEOUT";
+        case MAMBA_ERR_TOO_LARGE: return "MAMBA_ERR_TOO_LARGE";
     }
     return "MAMBA_ERR_UNKNOWN";
 }
