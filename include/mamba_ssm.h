@@ -119,7 +119,8 @@ typedef struct {
 
 /*
  * How a scan call will run (host-side planning; no CUDA call is made).
- * The channels form groups of 32 (one warp each); the sequence is cut into
+ * The channels form groups of 32 or 64 (one warp each, with one or two
+ * channels per lane); the sequence is cut into
  * nchunks segments of chunk_len steps (the last may be shorter).  A persistent
  * grid of warps pulls (segment, group) work items from a counter.
  *   mode 0 (chained): one launch.  Segment k of a group starts from the state
@@ -143,6 +144,9 @@ typedef struct {
     int32_t launches;          /* kernel launches per call (plus one memset) */
     int32_t tma_capable;       /* strides allow TMA staging */
     int32_t mode;              /* 0 chained, 1 parallel */
+    int32_t channels_per_lane; /* 1 or 2: a group is 32 x this many channels */
+    int32_t reserved;
+    int64_t max_warps;         /* warps the persistent grid uses at most */
     size_t workspace_bytes;
 } mamba_scan_plan_t;
 

@@ -89,38 +89,46 @@ cudaError_t ensure_smem_attr(Kernel kernel, int bytes, bool* done_per_device, in
     return e;
 }
 
-template <typename IoT, bool kHasZ, bool kSoftplus>
-cudaError_t launch_scan(const ScanParams& prm, const CUtensorMap* maps, int dev, int sms,
-                        cudaStream_t stream) {
+template <typename IoT, int kCpl, bool kHasZ, bool kSoftplus>
+cudaError_t launch_scan(const ScanParams& prm, const CUtensorMap* maps, int64_t want_warps,
+                        int dev, int sms, cudaStream_t stream) {
+    using Lay = ScanLayout<kCpl>;
     static bool attr_done[kMaxDevices] = {false};
     static int resident[kMaxDevices] = {0};
-    auto kernel = selective_scan_fwd_kernel<IoT, kHasZ, kSoftplus>;
-    cudaError_t e = ensure_smem_attr(kernel, kScanSmemBytes, attr_done, dev);
+    auto kernel = selective_scan_fwd_kernel<IoT, kCpl, kHasZ, kSoftplus>;
+    cudaError_t e = ensure_smem_attr(kernel, Lay::kCtaSmem, attr_done, dev);
     if (e != cudaSuccess) return e;
     int per_sm = (dev >= 0 && dev < kMaxDevices) ? resident[dev] : 0;
     if (per_sm <= 0) {
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kScanWarps * 32,
-                                                          kScanSmemBytes);
+                                                          Lay::kCtaSmem);
         if (e != cudaSuccess) return e;
         if (per_sm <= 0) return cudaErrorInvalidConfiguration;
         if (dev >= 0 && dev < kMaxDevices) resident[dev] = per_sm;
     }
     // Persistent grid: every warp keeps pulling work items until none are left.
-    const int64_t want = (prm.items + kScanWarps - 1) / kScanWarps;
+    const int64_t want = (want_warps + kScanWarps - 1) / kScanWarps;
     const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)per_sm * sms));
-    kernel<<<(unsigned)grid, kScanWarps * 32, kScanSmemBytes, stream>>>(prm, maps[0], maps[1],
-                                                                          maps[2], maps[3], maps[4]);
+    kernel<<<(unsigned)grid, kScanWarps * 32, Lay::kCtaSmem, stream>>>(prm, maps[0], maps[1],
+                                                                         maps[2], maps[3], maps[4]);
     return cudaGetLastError();
 }
 
-template <typename IoT>
-cudaError_t dispatch_scan(const ScanParams& prm, const CUtensorMap* maps, bool has_z, bool sp,
-                          int dev, int sms, cudaStream_t stream) {
+template <typename IoT, int kCpl>
+cudaError_t dispatch_scan_cpl(const ScanParams& prm, const CUtensorMap* maps, bool has_z, bool sp,
+                              int64_t want_warps, int dev, int sms, cudaStream_t stream) {
     if (has_z)
-        return sp ? launch_scan<IoT, true, true>(prm, maps, dev, sms, stream)
-                  : launch_scan<IoT, true, false>(prm, maps, dev, sms, stream);
-    return sp ? launch_scan<IoT, false, true>(prm, maps, dev, sms, stream)
-              : launch_scan<IoT, false, false>(prm, maps, dev, sms, stream);
+        return sp ? launch_scan<IoT, kCpl, true, true>(prm, maps, want_warps, dev, sms, stream)
+                  : launch_scan<IoT, kCpl, true, false>(prm, maps, want_warps, dev, sms, stream);
+    return sp ? launch_scan<IoT, kCpl, false, true>(prm, maps, want_warps, dev, sms, stream)
+              : launch_scan<IoT, kCpl, false, false>(prm, maps, want_warps, dev, sms, stream);
+}
+
+template <typename IoT>
+cudaError_t dispatch_scan(const ScanParams& prm, const CUtensorMap* maps, int cpl, bool has_z,
+                          bool sp, int64_t want_warps, int dev, int sms, cudaStream_t stream) {
+    if (cpl != 1) return cudaErrorInvalidValue;
+    return dispatch_scan_cpl<IoT, 1>(prm, maps, has_z, sp, want_warps, dev, sms, stream);
 }
 
 template <typename IoT, typename BcT>
@@ -182,10 +190,12 @@ ScanWorkspace scan_workspace_layout(const mamba_dims_t* dims, int64_t groups, in
 }
 
 // Planning rules (pure host logic, see mamba_selective_scan_plan).
-//  - W = resident warps on the GPU (16 per SM), G = channel groups of 32.
-//  - G >= W: chained mode, K segments so that G*K is about 8 W work items
-//    (even load across SMs), segments at least 256 steps long.
-//  - W/4 <= G < W: one segment per group (every chain stays on one warp).
+//  - One channel per lane (32-channel groups).
+//  - W = resident warps on the GPU (16 per SM), G = channel groups.
+//  - G >= W/4: chained mode, K segments so that G*K is about 8 W work items
+//    (even load across SMs), segments at least 256 steps long.  At most G
+//    warps run, so a warp rarely picks up a segment whose predecessor has not
+//    finished.
 //  - G < W/4: parallel mode, K-1 = W/G segments per pass (every resident
 //    warp busy), segments at least 16 tiles and 512 steps long.
 //  - num_chunks >= 1 forces K; MAMBA_FLAG_PARALLEL_CHUNKS forces the parallel
@@ -199,12 +209,22 @@ mamba_status_t plan_scan(const mamba_dims_t* dims, int sm_count, mamba_scan_plan
     const int bc_es = dtype_bytes(dims->bc_dtype);
     const int64_t T = kRowBytes / io_es;
     const int64_t L = dims->seqlen;
-    const int64_t gpb = (dims->dim + kGroupRows - 1) / kGroupRows;
-    const int64_t groups = dims->batch * gpb;
-    const int64_t W = (int64_t)sm_count * kScanWarpsPerSm;
+    const int64_t g1 = dims->batch * ((dims->dim + 31) / 32);
+    const int64_t g2 = dims->batch * ((dims->dim + 63) / 64);
+    const int64_t w1 = (int64_t)sm_count * ScanLayout<1>::kWarpsPerSm;
+    const int64_t w2 = (int64_t)sm_count * ScanLayout<2>::kWarpsPerSm;
+    // One channel per lane: measured faster than two on every workload shape
+    // (16 resident warps per SM against 12; the packed fp32x2 step already
+    // leaves issue slots to spare).
+    const int cpl = 1;
+    (void)g2;
+    (void)w2;
+    const int64_t groups = g1;
+    const int64_t W = w1;
     plan->tile_len = (int32_t)T;
     plan->groups = groups;
     plan->warps_per_cta = kScanWarps;
+    plan->channels_per_lane = cpl;
     plan->tma_capable = (L > 0 && (L * io_es) % 16 == 0 && (L * bc_es) % 16 == 0) ? 1 : 0;
 
     int64_t K = 1;
@@ -213,11 +233,9 @@ mamba_status_t plan_scan(const mamba_dims_t* dims, int sm_count, mamba_scan_plan
         K = dims->num_chunks;
         mode = (dims->flags & MAMBA_FLAG_PARALLEL_CHUNKS) ? 1 : 0;
     } else if (groups > 0 && L > 0) {
-        if (groups >= W) {
+        if (4 * groups >= W) {
             const int64_t want = (8 * W + groups - 1) / groups;
             K = std::max<int64_t>(1, std::min<int64_t>(want, L / 256));
-        } else if (groups * 4 >= W) {
-            K = 1;
         } else {
             mode = 1;
             K = std::max<int64_t>(
@@ -241,6 +259,7 @@ mamba_status_t plan_scan(const mamba_dims_t* dims, int sm_count, mamba_scan_plan
     plan->mode = mode;
     plan->units_pass_a = items;
     plan->units_pass_b = mode == 0 ? 0 : items;
+    plan->max_warps = mode == 0 && K > 1 ? std::min<int64_t>(groups, W) : std::min<int64_t>(items, W);
     plan->launches = (groups > 0 && L > 0) ? (mode == 0 ? 1 : 2) : 0;
     plan->workspace_bytes =
         (groups > 0 && L > 0) ? scan_workspace_layout(dims, groups, K, mode).total : 0;
@@ -318,7 +337,7 @@ MAMBA_API mamba_status_t mamba_selective_scan_fwd(const void* u, const void* del
     prm.batch = dims->batch;
     prm.dim = dims->dim;
     prm.seqlen = dims->seqlen;
-    prm.groups_per_batch = (dims->dim + kGroupRows - 1) / kGroupRows;
+    prm.groups_per_batch = (dims->dim + 32 * plan.channels_per_lane - 1) / (32 * plan.channels_per_lane);
     prm.groups = plan.groups;
     prm.chains = chains;
     prm.seg_len = plan.chunk_len;
@@ -353,11 +372,12 @@ MAMBA_API mamba_status_t mamba_selective_scan_fwd(const void* u, const void* del
         const uint64_t L = (uint64_t)dims->seqlen;
         const uint64_t Dm = (uint64_t)dims->dim, Bt = (uint64_t)dims->batch;
         const uint64_t N = (uint64_t)dims->dstate;
-        bool ok = encode_map_3d(&maps[0], u, io_es, L, Dm, Bt, T, kGroupRows,
+        const uint32_t rows = 32u * (uint32_t)plan.channels_per_lane;
+        bool ok = encode_map_3d(&maps[0], u, io_es, L, Dm, Bt, T, rows,
                                 CU_TENSOR_MAP_SWIZZLE_32B) &&
-                  encode_map_3d(&maps[1], delta, io_es, L, Dm, Bt, T, kGroupRows,
+                  encode_map_3d(&maps[1], delta, io_es, L, Dm, Bt, T, rows,
                                 CU_TENSOR_MAP_SWIZZLE_32B) &&
-                  encode_map_3d(&maps[2], z ? z : u, io_es, L, Dm, Bt, T, kGroupRows,
+                  encode_map_3d(&maps[2], z ? z : u, io_es, L, Dm, Bt, T, rows,
                                 CU_TENSOR_MAP_SWIZZLE_32B) &&
                   encode_map_3d(&maps[3], B, bc_es, L, N, Bt, T, (uint32_t)N,
                                 CU_TENSOR_MAP_SWIZZLE_NONE) &&
@@ -379,8 +399,10 @@ MAMBA_API mamba_status_t mamba_selective_scan_fwd(const void* u, const void* del
         prm.items = items;
         if (items == 0) return cudaSuccess;
         return dims->io_dtype == MAMBA_BF16
-                   ? dispatch_scan<__nv_bfloat16>(prm, maps, has_z, sp, dev, sms, stream)
-                   : dispatch_scan<float>(prm, maps, has_z, sp, dev, sms, stream);
+                   ? dispatch_scan<__nv_bfloat16>(prm, maps, plan.channels_per_lane, has_z, sp,
+                                                  plan.max_warps, dev, sms, stream)
+                   : dispatch_scan<float>(prm, maps, plan.channels_per_lane, has_z, sp,
+                                          plan.max_warps, dev, sms, stream);
     };
     cudaError_t e;
     if (plan.mode == 0) {

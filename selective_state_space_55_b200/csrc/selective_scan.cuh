@@ -1,13 +1,16 @@
 // Selective-scan forward kernel (sm_100a).
 //
-// Work decomposition.  One warp owns 32 consecutive channels of one batch row
-// (a "group") for one contiguous range of time steps (a "segment").  Lane l
-// owns channel d = d0 + l: its 16 state values h_n and the 16 factors
-// A_d,n * log2(e) live in registers for the whole segment, so the state never
-// touches HBM ("Mamba 与状态空间模型", section 在芯片上扫过去: discretise and recur
-// on chip, write only the output).  Each time step costs 16 MUFU ex2 for
-// Abar = 2^(Delta * A log2 e), four fp32 operations per state entry, and the
-// softplus / silu of the step.
+// Work decomposition.  One warp owns 32 x kCpl consecutive channels of one
+// batch row (a "group") for one contiguous range of time steps (a
+// "segment").  Lane l owns channels d0 + l + 32 c for c < kCpl: their 16
+// state values h_n and 16 factors A_d,n log2(e) live in registers for the
+// whole segment, so the state never touches HBM ("Mamba 与状态空间模型",
+// section 在芯片上扫过去: discretise and recur on chip, write only the output).
+// Each time step costs 16 MUFU ex2 per channel for Abar = 2^(Delta A log2 e),
+// four fp32 operations per state entry, and the softplus / silu of the step.
+// With kCpl = 2 every read of a step's B and C coefficients serves two
+// channels, which halves the shared-memory traffic per element and gives each
+// warp two independent recurrences to interleave.
 //
 // Scheduling.  The grid is persistent (as many CTAs as stay resident) and
 // every warp pulls (segment k, group g) work items from a global counter in
@@ -31,15 +34,14 @@
 //    section 硬件效率; "Mamba 与状态空间模型", section 在芯片上扫过去).
 //
 // Staging.  Per warp, a two-stage ring in shared memory holds tiles of
-// T = 32 bytes / sizeof(io) time steps of the warp's 32 channel rows of u,
-// delta and z (TMA 3-D tiles with 32-byte swizzle, so each lane's 16-byte reads
-// of its own row are conflict free; L2 promotion fetches whole 128-byte lines
+// T = 32 bytes / sizeof(io) time steps of the warp's channel rows of u, delta
+// and z (TMA 3-D tiles with 32-byte swizzle, so each lane's 16-byte reads of
+// its own rows are conflict free; L2 promotion fetches whole 128-byte lines
 // so the next tiles of a row hit L2) and the B and C rows of the batch (TMA).
 // Once a tile lands the warp converts B and C to an fp32 table
 // bcf[t][B0..15 C0..15] that every lane reads with broadcast 16-byte loads.
 // Without TMA (odd strides or MAMBA_FLAG_NO_TMA) plain loads fill the same
-// tiles.  About 12 KB of shared memory and at most 128 registers per warp let
-// 16 warps share an SM.
+// tiles.
 #pragma once
 
 #include "ssm_device.cuh"
@@ -47,28 +49,31 @@
 namespace mamba {
 
 constexpr int kScanWarps = 4;              // warps per CTA (each an independent worker)
-#ifndef MAMBA_SCAN_MIN_BLOCKS
-#define MAMBA_SCAN_MIN_BLOCKS 4
-#endif
-constexpr int kScanMinBlocks = MAMBA_SCAN_MIN_BLOCKS;   // CTAs per SM the kernel is compiled for
 constexpr int kScanStages = 2;             // tiles in flight per warp
 constexpr int kRowBytes = 32;              // bytes of one channel row in a tile
-constexpr int kGroupRows = 32;             // channels per warp
 constexpr int kNPad = 16;                  // compiled state size (smaller N is zero-padded)
 constexpr int kMaxTile = kRowBytes / 2;    // time steps per tile for 2-byte inputs
-constexpr int kIoTileBytes = kGroupRows * kRowBytes;        // 1024
-constexpr int kBcRawBytes = kNPad * kMaxTile * 4;           // 16 rows of up to 64 bytes
-constexpr int kOffU = 0;
-constexpr int kOffDelta = kIoTileBytes;
-constexpr int kOffZ = 2 * kIoTileBytes;
-constexpr int kOffB = 3 * kIoTileBytes;
-constexpr int kOffC = 3 * kIoTileBytes + kBcRawBytes;
-constexpr int kStageBytes = 3 * kIoTileBytes + 2 * kBcRawBytes;   // 5120
-constexpr int kBcfBytes = kMaxTile * 32 * 4;                      // [T][32] fp32
-constexpr int kBarOffset = kScanStages * kStageBytes + kBcfBytes;
-constexpr int kWarpSmemBytes = ((kBarOffset + 64 + 255) / 256) * 256;
-constexpr int kScanSmemBytes = kScanWarps * kWarpSmemBytes + 1024;  // + base alignment slack
-constexpr int kScanWarpsPerSm = kScanWarps * kScanMinBlocks;
+constexpr int kBcRawBytes = kNPad * kMaxTile * 4;   // 16 rows of up to 64 bytes
+constexpr int kBcfBytes = kMaxTile * 32 * 4;        // [T][32] fp32
+
+// Shared-memory layout and residency of the kernel with kCpl channels per lane.
+template <int kCpl>
+struct ScanLayout {
+    static constexpr int kRows = 32 * kCpl;                       // channels per group
+    static constexpr int kIoTile = kRows * kRowBytes;             // one tensor's tile
+    static constexpr int kOffU = 0;
+    static constexpr int kOffDelta = kIoTile;
+    static constexpr int kOffZ = 2 * kIoTile;
+    static constexpr int kOffB = 3 * kIoTile;
+    static constexpr int kOffC = 3 * kIoTile + kBcRawBytes;
+    static constexpr int kStage = 3 * kIoTile + 2 * kBcRawBytes;
+    static constexpr int kOffBcf = kScanStages * kStage;
+    static constexpr int kOffBar = kOffBcf + kBcfBytes;
+    static constexpr int kWarpSmem = ((kOffBar + 64 + 255) / 256) * 256;
+    static constexpr int kCtaSmem = kScanWarps * kWarpSmem + 1024;   // + base alignment slack
+    static constexpr int kMinBlocks = kCpl == 1 ? 4 : 3;            // CTAs per SM
+    static constexpr int kWarpsPerSm = kScanWarps * kMinBlocks;
+};
 
 // Workspace layout (bytes from the start).
 constexpr size_t kWsCounters = 0;          // uint32 [2] dequeue counters
@@ -120,36 +125,6 @@ __device__ __forceinline__ void kahan_add(float& sum, float& comp, float v) {
     sum = t;
 }
 
-// One time step for one lane: advance the 16 states, return y (kOut).
-// kExact selects exp2_near_one_exact for Abar (fp32 input/output path).
-template <bool kOut, bool kExact>
-__device__ __forceinline__ float scan_step(const float* bc_row, float dt, float du,
-                                           float (&h)[kNPad], const float (&a2)[kNPad]) {
-    const float4* bc = reinterpret_cast<const float4*>(bc_row);
-    float yq[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const float4 Bq = bc[q];
-        const float b4[4] = {Bq.x, Bq.y, Bq.z, Bq.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int n = 4 * q + i;
-            const float x = dt * a2[n];
-            const float abar = kExact ? exp2_near_one_exact(x) : ex2_approx(x);
-            h[n] = fmaf(abar, h[n], du * b4[i]);
-        }
-        if (kOut) {
-            const float4 Cq = bc[4 + q];
-            float y = Cq.x * h[4 * q];
-            y = fmaf(Cq.y, h[4 * q + 1], y);
-            y = fmaf(Cq.z, h[4 * q + 2], y);
-            y = fmaf(Cq.w, h[4 * q + 3], y);
-            yq[q] = y;
-        }
-    }
-    return kOut ? (yq[0] + yq[1]) + (yq[2] + yq[3]) : 0.0f;
-}
-
 // Element j of a 16-byte vector holding 8 bf16 or 4 fp32 values, as fp32.
 template <typename IoT>
 __device__ __forceinline__ float vec_elem(const uint4& v, int j);
@@ -180,88 +155,177 @@ template <> struct OutPack<float> {
     __device__ __forceinline__ uint4 vec() const { return make_uint4(w[0], w[1], w[2], w[3]); }
 };
 
+// Per-lane state of one work item: kCpl channels.  State entries and A log2 e
+// factors are kept as pairs (n, n+1) so the recurrence and the readout run on
+// Blackwell's packed fp32x2 FMA/FMUL, two state entries per instruction.
+template <int kCpl>
+struct LaneChains {
+    float2 h[kCpl][kNPad / 2];
+    float2 a2[kCpl][kNPad / 2];
+    float bias[kCpl];
+    float Dd[kCpl];
+};
+
+// 2^x for both halves of x: MUFU ex2, or exp2_near_one_exact (fp32 path).
+template <bool kExact>
+__device__ __forceinline__ float2 exp2_pair(float2 x) {
+    if (kExact) return make_float2(exp2_near_one_exact(x.x), exp2_near_one_exact(x.y));
+    return make_float2(ex2_approx(x.x), ex2_approx(x.y));
+}
+
+// One time step for one lane: advance the kCpl x 16 states, return y per
+// channel (kOut).  kExact selects exp2_near_one_exact for Abar (fp32 path).
+template <int kCpl, bool kOut, bool kExact>
+__device__ __forceinline__ void scan_step(const float* bc_row, const float (&dt)[kCpl],
+                                          const float (&du)[kCpl], LaneChains<kCpl>& lc,
+                                          float (&y)[kCpl]) {
+    const float4* bc = reinterpret_cast<const float4*>(bc_row);
+    float2 ya[kCpl], yb[kCpl];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const float4 Bq = bc[q];
+        const float2 bq[2] = {make_float2(Bq.x, Bq.y), make_float2(Bq.z, Bq.w)};
+#pragma unroll
+        for (int c = 0; c < kCpl; ++c) {
+            const float2 dt2 = make_float2(dt[c], dt[c]);
+            const float2 du2 = make_float2(du[c], du[c]);
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const int pi = 2 * q + half;
+                const float2 abar = exp2_pair<kExact>(__fmul2_rn(dt2, lc.a2[c][pi]));
+                lc.h[c][pi] = __ffma2_rn(abar, lc.h[c][pi], __fmul2_rn(du2, bq[half]));
+            }
+        }
+        if (kOut) {
+            const float4 Cq = bc[4 + q];
+            const float2 c01 = make_float2(Cq.x, Cq.y);
+            const float2 c23 = make_float2(Cq.z, Cq.w);
+#pragma unroll
+            for (int c = 0; c < kCpl; ++c) {
+                if (q == 0) {
+                    ya[c] = __fmul2_rn(c01, lc.h[c][0]);
+                    yb[c] = __fmul2_rn(c23, lc.h[c][1]);
+                } else {
+                    ya[c] = __ffma2_rn(c01, lc.h[c][2 * q], ya[c]);
+                    yb[c] = __ffma2_rn(c23, lc.h[c][2 * q + 1], yb[c]);
+                }
+            }
+        }
+    }
+    if (kOut) {
+#pragma unroll
+        for (int c = 0; c < kCpl; ++c) y[c] = (ya[c].x + ya[c].y) + (yb[c].x + yb[c].y);
+    }
+}
+
 // Process the `nsteps` (<= T) valid time steps of one staged tile.  The
 // 16-byte vectors of u, delta and z stay packed and are unpacked step by
-// step, which keeps the kernel within 128 registers.
-template <typename IoT, bool kHasZ, bool kSoftplus, bool kOut>
+// step to save registers.
+template <typename IoT, int kCpl, bool kHasZ, bool kSoftplus, bool kOut>
 __device__ __forceinline__ void compute_tile(const uint8_t* st, const float* bcf, int lane,
-                                             int nsteps, float (&h)[kNPad],
-                                             const float (&a2)[kNPad], float bias, float Dd,
-                                             IoT* out_row, bool vec_out, float& sdt,
-                                             float& sdt_c) {
+                                             int nsteps, LaneChains<kCpl>& lc,
+                                             IoT* const (&out_row)[kCpl], bool vec_out,
+                                             float (&sdt)[kCpl], float (&sdt_c)[kCpl]) {
+    using Lay = ScanLayout<kCpl>;
     constexpr int V = 16 / (int)sizeof(IoT);          // steps per 16-byte vector
     constexpr int T = kRowBytes / (int)sizeof(IoT);   // steps per tile
     constexpr bool kExact = sizeof(IoT) == 4;
 #pragma unroll 1
-    for (int c = 0; c < T / V; ++c) {
-        const int base = c * V;
+    for (int cv = 0; cv < T / V; ++cv) {
+        const int base = cv * V;
         if (base >= nsteps) break;
-        const uint32_t so = swz32(lane, 16u * c);
-        const uint4 ur = *reinterpret_cast<const uint4*>(st + kOffU + so);
-        const uint4 dr = *reinterpret_cast<const uint4*>(st + kOffDelta + so);
-        uint4 zr = make_uint4(0u, 0u, 0u, 0u);
-        if (kHasZ && kOut) zr = *reinterpret_cast<const uint4*>(st + kOffZ + so);
+        uint4 ur[kCpl], dr[kCpl], zr[kCpl];
+#pragma unroll
+        for (int c = 0; c < kCpl; ++c) {
+            const uint32_t so = swz32(lane + 32 * c, 16u * cv);
+            ur[c] = *reinterpret_cast<const uint4*>(st + Lay::kOffU + so);
+            dr[c] = *reinterpret_cast<const uint4*>(st + Lay::kOffDelta + so);
+            zr[c] = make_uint4(0u, 0u, 0u, 0u);
+            if (kHasZ && kOut) zr[c] = *reinterpret_cast<const uint4*>(st + Lay::kOffZ + so);
+        }
         const int steps = min(V, nsteps - base);
-        const bool whole = steps == V && vec_out && out_row != nullptr;
-        OutPack<IoT> pk;
+        bool whole[kCpl];
+#pragma unroll
+        for (int c = 0; c < kCpl; ++c) whole[c] = steps == V && vec_out && out_row[c] != nullptr;
+        OutPack<IoT> pk[kCpl];
 #pragma unroll
         for (int j = 0; j < V; ++j) {
             if (steps == V || j < steps) {
-                const float uj = vec_elem<IoT>(ur, j);
-                const float s = vec_elem<IoT>(dr, j) + bias;
-                const float dt = kSoftplus ? softplus_f32(s) : s;
-                const float y = scan_step<kOut, kExact>(bcf + (base + j) * 32, dt, dt * uj, h, a2);
-                if (kOut) {
-                    float yo = fmaf(Dd, uj, y);
-                    if (kHasZ) yo *= silu_f32(vec_elem<IoT>(zr, j));
-                    if (whole)
-                        pk.put(j, yo);
-                    else if (out_row != nullptr)
-                        DType<IoT>::store(out_row + base + j, yo);
-                } else {
-                    kahan_add(sdt, sdt_c, dt);
+                float uj[kCpl], dt[kCpl], du[kCpl], y[kCpl];
+#pragma unroll
+                for (int c = 0; c < kCpl; ++c) {
+                    uj[c] = vec_elem<IoT>(ur[c], j);
+                    const float s = vec_elem<IoT>(dr[c], j) + lc.bias[c];
+                    dt[c] = kSoftplus ? softplus_f32(s) : s;
+                    du[c] = dt[c] * uj[c];
+                }
+                scan_step<kCpl, kOut, kExact>(bcf + (base + j) * 32, dt, du, lc, y);
+#pragma unroll
+                for (int c = 0; c < kCpl; ++c) {
+                    if (kOut) {
+                        float yo = fmaf(lc.Dd[c], uj[c], y[c]);
+                        if (kHasZ) yo *= silu_f32(vec_elem<IoT>(zr[c], j));
+                        if (whole[c])
+                            pk[c].put(j, yo);
+                        else if (out_row[c] != nullptr)
+                            DType<IoT>::store(out_row[c] + base + j, yo);
+                    } else {
+                        kahan_add(sdt[c], sdt_c[c], dt[c]);
+                    }
                 }
             }
         }
-        if (kOut && whole) *reinterpret_cast<uint4*>(out_row + base) = pk.vec();
+        if (kOut) {
+#pragma unroll
+            for (int c = 0; c < kCpl; ++c)
+                if (whole[c]) *reinterpret_cast<uint4*>(out_row[c] + base) = pk[c].vec();
+        }
     }
 }
 
 // Convert the raw B (and C) rows of a TMA-staged tile into the fp32 table
-// bcf[t][32] = (B_0..B_15, C_0..C_15) of each step.  Lane l handles row
-// l & 15 of B (l < 16) or C; rows n >= dstate read as zero.
-template <int T, bool kNeedC>
+// bcf[t][32] = (B_0..B_15, C_0..C_15) of each step.  Lane l converts row l & 15
+// of B (l < 16) or C with 16-byte reads; rows n >= dstate become zero.
+template <int kCpl, int T, bool kNeedC>
 __device__ __forceinline__ void convert_bc(const uint8_t* st, float* bcf, int lane, int dstate,
                                            bool bc_bf16) {
+    using Lay = ScanLayout<kCpl>;
     const int which = lane >> 4;
     const int n = lane & 15;
     const bool live = n < dstate && (which == 0 || kNeedC);
-    const uint8_t* raw = st + (which ? kOffC : kOffB);
+    const uint8_t* raw = st + (which ? Lay::kOffC : Lay::kOffB);
+    if (bc_bf16) {
+        // T bf16 values = T/8 16-byte vectors
+        const uint4* row = reinterpret_cast<const uint4*>(raw + n * T * 2);
 #pragma unroll
-    for (int k = 0; k < T; ++k) {
-        const int j = (k + lane) & (T - 1);
-        float v = 0.0f;
-        if (live) {
-            if (bc_bf16)
-                v = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(raw)[n * T + j]);
-            else
-                v = reinterpret_cast<const float*>(raw)[n * T + j];
+        for (int v = 0; v < T / 8; ++v) {
+            const uint4 r = live ? row[v] : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) bcf[(8 * v + j) * 32 + lane] = vec_elem<__nv_bfloat16>(r, j);
         }
-        bcf[j * 32 + lane] = v;
+    } else {
+        const uint4* row = reinterpret_cast<const uint4*>(raw + n * T * 4);
+#pragma unroll
+        for (int v = 0; v < T / 4; ++v) {
+            const uint4 r = live ? row[v] : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) bcf[(4 * v + j) * 32 + lane] = vec_elem<float>(r, j);
+        }
     }
 }
 
 // Fill one stage with plain loads (any stride or alignment).  Rows beyond
 // dim and steps beyond seqlen read as zero, as TMA's out-of-bounds fill does.
-template <typename IoT, bool kNeedZ, bool kNeedC>
+template <typename IoT, int kCpl, bool kNeedZ, bool kNeedC>
 __device__ __forceinline__ void portable_stage(const ScanParams& p, uint8_t* st, float* bcf,
                                                int lane, int64_t b, int64_t d0, int64_t t0) {
+    using Lay = ScanLayout<kCpl>;
     constexpr int ES = (int)sizeof(IoT);
     constexpr int T = kRowBytes / ES;
     const IoT* u = static_cast<const IoT*>(p.u);
     const IoT* dl = static_cast<const IoT*>(p.delta);
     const IoT* zz = static_cast<const IoT*>(p.z);
-    for (int idx = lane; idx < kGroupRows * T; idx += 32) {
+    for (int idx = lane; idx < Lay::kRows * T; idx += 32) {
         const int r = idx / T;
         const int j = idx % T;
         const int64_t d = d0 + r;
@@ -270,9 +334,9 @@ __device__ __forceinline__ void portable_stage(const ScanParams& p, uint8_t* st,
         const int64_t off = (b * p.dim + d) * p.seqlen + t;
         const uint32_t so = swz32(r, j * ES);
         const IoT zero = IoT(0.0f);
-        *reinterpret_cast<IoT*>(st + kOffU + so) = in ? u[off] : zero;
-        *reinterpret_cast<IoT*>(st + kOffDelta + so) = in ? dl[off] : zero;
-        if (kNeedZ) *reinterpret_cast<IoT*>(st + kOffZ + so) = in ? zz[off] : zero;
+        *reinterpret_cast<IoT*>(st + Lay::kOffU + so) = in ? u[off] : zero;
+        *reinterpret_cast<IoT*>(st + Lay::kOffDelta + so) = in ? dl[off] : zero;
+        if (kNeedZ) *reinterpret_cast<IoT*>(st + Lay::kOffZ + so) = in ? zz[off] : zero;
     }
     const int which = lane >> 4;
     const int n = lane & 15;
@@ -299,39 +363,42 @@ struct TmaMaps {
     const CUtensorMap* C;
 };
 
-// Run time steps [t_begin, t_end) of one group, starting from h.  `seq`
+// Run time steps [t_begin, t_end) of one group, starting from lc.h.  `seq`
 // counts the tiles this warp has consumed (it fixes each tile's stage and
 // mbarrier parity across items).  Returns false if a staged tile never
 // arrived (the warp has then waited, bounded, for its copies in flight).
-template <typename IoT, bool kHasZ, bool kSoftplus, bool kOut>
+template <typename IoT, int kCpl, bool kHasZ, bool kSoftplus, bool kOut>
 __device__ __forceinline__ bool run_segment(const ScanParams& p, const TmaMaps& maps, uint8_t* wsm,
                                             int lane, int64_t b, int64_t d0, int64_t t_begin,
-                                            int64_t t_end, float (&h)[kNPad],
-                                            const float (&a2)[kNPad], float bias, float Dd,
-                                            IoT* out_row, uint32_t& seq, float& sdt) {
+                                            int64_t t_end, LaneChains<kCpl>& lc,
+                                            IoT* const (&out_row)[kCpl], uint32_t& seq,
+                                            float (&sdt)[kCpl]) {
+    using Lay = ScanLayout<kCpl>;
     constexpr int T = kRowBytes / (int)sizeof(IoT);
     constexpr bool kNeedZ = kHasZ && kOut;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(wsm + kBarOffset);
-    float* bcf = reinterpret_cast<float*>(wsm + kScanStages * kStageBytes);
-    float sdt_c = 0.0f;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(wsm + Lay::kOffBar);
+    float* bcf = reinterpret_cast<float*>(wsm + Lay::kOffBcf);
+    float sdt_c[kCpl];
+#pragma unroll
+    for (int c = 0; c < kCpl; ++c) sdt_c[c] = 0.0f;
 
     const int ntiles = (int)((t_end - t_begin + T - 1) / T);
     const uint32_t bc_bytes = (uint32_t)(p.dstate * T * (p.bc_bf16 ? 2 : 4));
     const uint32_t stage_tx =
-        (uint32_t)((kNeedZ ? 3 : 2) * kIoTileBytes) + (kOut ? 2u : 1u) * bc_bytes;
+        (uint32_t)((kNeedZ ? 3 : 2) * Lay::kIoTile) + (kOut ? 2u : 1u) * bc_bytes;
 
     auto issue = [&](int i) {
         const uint32_t s = (seq + (uint32_t)i) % kScanStages;
-        uint8_t* st = wsm + s * kStageBytes;
+        uint8_t* st = wsm + s * Lay::kStage;
         const int t0 = (int)(t_begin + (int64_t)i * T);
         const uint32_t bar = smem_u32(&bars[s]);
         fence_proxy_async_smem();
         mbar_arrive_expect_tx(bar, stage_tx);
-        tma_load_3d(smem_u32(st + kOffU), maps.u, t0, (int)d0, (int)b, bar);
-        tma_load_3d(smem_u32(st + kOffDelta), maps.delta, t0, (int)d0, (int)b, bar);
-        if (kNeedZ) tma_load_3d(smem_u32(st + kOffZ), maps.z, t0, (int)d0, (int)b, bar);
-        tma_load_3d(smem_u32(st + kOffB), maps.B, t0, 0, (int)b, bar);
-        if (kOut) tma_load_3d(smem_u32(st + kOffC), maps.C, t0, 0, (int)b, bar);
+        tma_load_3d(smem_u32(st + Lay::kOffU), maps.u, t0, (int)d0, (int)b, bar);
+        tma_load_3d(smem_u32(st + Lay::kOffDelta), maps.delta, t0, (int)d0, (int)b, bar);
+        if (kNeedZ) tma_load_3d(smem_u32(st + Lay::kOffZ), maps.z, t0, (int)d0, (int)b, bar);
+        tma_load_3d(smem_u32(st + Lay::kOffB), maps.B, t0, 0, (int)b, bar);
+        if (kOut) tma_load_3d(smem_u32(st + Lay::kOffC), maps.C, t0, 0, (int)b, bar);
     };
 
     if (p.use_tma && lane == 0)
@@ -340,7 +407,7 @@ __device__ __forceinline__ bool run_segment(const ScanParams& p, const TmaMaps& 
 
     for (int i = 0; i < ntiles; ++i) {
         const uint32_t sq = seq + (uint32_t)i;
-        uint8_t* st = wsm + (sq % kScanStages) * kStageBytes;
+        uint8_t* st = wsm + (sq % kScanStages) * Lay::kStage;
         const int64_t t0 = t_begin + (int64_t)i * T;
         const int nsteps = (int)min((int64_t)T, t_end - t0);
         if (p.use_tma) {
@@ -358,14 +425,16 @@ __device__ __forceinline__ bool run_segment(const ScanParams& p, const TmaMaps& 
                 __syncwarp();
                 return false;
             }
-            convert_bc<T, kOut>(st, bcf, lane, p.dstate, p.bc_bf16 != 0);
+            convert_bc<kCpl, T, kOut>(st, bcf, lane, p.dstate, p.bc_bf16 != 0);
         } else {
-            portable_stage<IoT, kNeedZ, kOut>(p, st, bcf, lane, b, d0, t0);
+            portable_stage<IoT, kCpl, kNeedZ, kOut>(p, st, bcf, lane, b, d0, t0);
         }
         __syncwarp();
-        compute_tile<IoT, kHasZ, kSoftplus, kOut>(st, bcf, lane, nsteps, h, a2, bias, Dd,
-                                                  out_row ? out_row + (t0 - t_begin) : nullptr,
-                                                  p.vec_out != 0, sdt, sdt_c);
+        IoT* rows[kCpl];
+#pragma unroll
+        for (int c = 0; c < kCpl; ++c) rows[c] = out_row[c] ? out_row[c] + (t0 - t_begin) : nullptr;
+        compute_tile<IoT, kCpl, kHasZ, kSoftplus, kOut>(st, bcf, lane, nsteps, lc, rows,
+                                                        p.vec_out != 0, sdt, sdt_c);
         __syncwarp();
         if (p.use_tma && lane == 0 && i + kScanStages < ntiles) issue(i + kScanStages);
     }
@@ -373,19 +442,20 @@ __device__ __forceinline__ bool run_segment(const ScanParams& p, const TmaMaps& 
     return true;
 }
 
-__device__ __forceinline__ void store16(float* dst, const float (&h)[kNPad]) {
+__device__ __forceinline__ void store16(float* dst, const float2 (&h)[kNPad / 2]) {
     float4* d4 = reinterpret_cast<float4*>(dst);
 #pragma unroll
     for (int q = 0; q < 4; ++q)
-        __stcg(d4 + q, make_float4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]));
+        __stcg(d4 + q, make_float4(h[2 * q].x, h[2 * q].y, h[2 * q + 1].x, h[2 * q + 1].y));
 }
 
-__device__ __forceinline__ void load16(const float* src, float (&h)[kNPad]) {
+__device__ __forceinline__ void load16(const float* src, float2 (&h)[kNPad / 2]) {
     const float4* s4 = reinterpret_cast<const float4*>(src);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         const float4 v = __ldcg(s4 + q);
-        h[4 * q] = v.x; h[4 * q + 1] = v.y; h[4 * q + 2] = v.z; h[4 * q + 3] = v.w;
+        h[2 * q] = make_float2(v.x, v.y);
+        h[2 * q + 1] = make_float2(v.z, v.w);
     }
 }
 
@@ -399,24 +469,25 @@ __device__ __forceinline__ void st_release_gpu(unsigned int* p, unsigned int v) 
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-template <typename IoT, bool kHasZ, bool kSoftplus>
-__global__ void __launch_bounds__(kScanWarps * 32, kScanMinBlocks)
+template <typename IoT, int kCpl, bool kHasZ, bool kSoftplus>
+__global__ void __launch_bounds__(kScanWarps * 32, ScanLayout<kCpl>::kMinBlocks)
     selective_scan_fwd_kernel(const __grid_constant__ ScanParams p,
                               const __grid_constant__ CUtensorMap tm_u,
                               const __grid_constant__ CUtensorMap tm_delta,
                               const __grid_constant__ CUtensorMap tm_z,
                               const __grid_constant__ CUtensorMap tm_B,
                               const __grid_constant__ CUtensorMap tm_C) {
+    using Lay = ScanLayout<kCpl>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    uint8_t* wsm = smem + warp * kWarpSmemBytes;
+    uint8_t* wsm = smem + warp * Lay::kWarpSmem;
     const TmaMaps maps{&tm_u, &tm_delta, &tm_z, &tm_B, &tm_C};
 
     if (p.use_tma && lane == 0) {
-        uint64_t* bars = reinterpret_cast<uint64_t*>(wsm + kBarOffset);
+        uint64_t* bars = reinterpret_cast<uint64_t*>(wsm + Lay::kOffBar);
         for (int s = 0; s < kScanStages; ++s) mbar_init(smem_u32(&bars[s]), 1);
         fence_mbar_init();
         prefetch_tensormap(&tm_u);
@@ -435,23 +506,29 @@ __global__ void __launch_bounds__(kScanWarps * 32, kScanMinBlocks)
         const int64_t g = item % p.groups;
         const int64_t k = (p.mode == kModePassB ? 1 : 0) + item / p.groups;
         const int64_t b = g / p.groups_per_batch;
-        const int64_t d0 = (g % p.groups_per_batch) * kGroupRows;
-        const int64_t d = d0 + lane;
-        const bool valid = d < p.dim;
-        const int64_t chain = b * p.dim + d;
+        const int64_t d0 = (g % p.groups_per_batch) * Lay::kRows;
         const int64_t t_begin = k * p.seg_len;
         const int64_t t_end = min(t_begin + p.seg_len, p.seqlen);
 
-        float a2[kNPad];
+        LaneChains<kCpl> lc;
+        bool valid[kCpl];
+        int64_t chain[kCpl];
 #pragma unroll
-        for (int n = 0; n < kNPad; ++n)
-            a2[n] = (valid && n < p.dstate) ? p.A[d * p.dstate + n] * kLog2e : 0.0f;
-        const float bias = (valid && p.delta_bias != nullptr) ? p.delta_bias[d] : 0.0f;
-        const float Dd = (valid && p.D != nullptr) ? p.D[d] : 0.0f;
-
-        float h[kNPad];
+        for (int c = 0; c < kCpl; ++c) {
+            const int64_t d = d0 + lane + 32 * c;
+            valid[c] = d < p.dim;
+            chain[c] = b * p.dim + d;
 #pragma unroll
-        for (int n = 0; n < kNPad; ++n) h[n] = 0.0f;
+            for (int pi = 0; pi < kNPad / 2; ++pi) {
+                const int n = 2 * pi;
+                lc.a2[c][pi] = make_float2(
+                    (valid[c] && n < p.dstate) ? p.A[d * p.dstate + n] * kLog2e : 0.0f,
+                    (valid[c] && n + 1 < p.dstate) ? p.A[d * p.dstate + n + 1] * kLog2e : 0.0f);
+                lc.h[c][pi] = make_float2(0.0f, 0.0f);
+            }
+            lc.bias[c] = (valid[c] && p.delta_bias != nullptr) ? p.delta_bias[d] : 0.0f;
+            lc.Dd[c] = (valid[c] && p.D != nullptr) ? p.D[d] : 0.0f;
+        }
 
         if (p.mode == kModeChained && k > 0) {
             // Wait for segment k-1 of this group, then take over its state.
@@ -472,52 +549,76 @@ __global__ void __launch_bounds__(kScanWarps * 32, kScanMinBlocks)
                 break;
             }
             (void)ld_acquire_gpu(p.flags + g);
-            if (valid) load16(p.carry + chain * kNPad, h);
-        } else if (p.mode == kModePassB && valid) {
-            // True start state of segment k: fold the end states of 0..k-1.
-            load16(p.ws_h + chain * kNPad, h);
-            for (int64_t j = 1; j < k; ++j) {
-                const float sj = __ldcg(p.ws_sdt + j * p.chains + chain);
-                float hj[kNPad];
-                load16(p.ws_h + (j * p.chains + chain) * kNPad, hj);
 #pragma unroll
-                for (int n = 0; n < kNPad; ++n) {
-                    const float x = a2[n] * sj;
-                    const float decay = sizeof(IoT) == 4 ? exp2_near_one_exact(x) : ex2_approx(x);
-                    h[n] = fmaf(decay, h[n], hj[n]);
+            for (int c = 0; c < kCpl; ++c)
+                if (valid[c]) load16(p.carry + chain[c] * kNPad, lc.h[c]);
+        } else if (p.mode == kModePassB) {
+            // True start state of segment k: fold the end states of 0..k-1.
+#pragma unroll
+            for (int c = 0; c < kCpl; ++c) {
+                if (!valid[c]) continue;
+                load16(p.ws_h + chain[c] * kNPad, lc.h[c]);
+                for (int64_t j = 1; j < k; ++j) {
+                    const float sj = __ldcg(p.ws_sdt + j * p.chains + chain[c]);
+                    const float2 s2 = make_float2(sj, sj);
+                    float2 hj[kNPad / 2];
+                    load16(p.ws_h + (j * p.chains + chain[c]) * kNPad, hj);
+#pragma unroll
+                    for (int pi = 0; pi < kNPad / 2; ++pi) {
+                        const float2 decay =
+                            exp2_pair<sizeof(IoT) == 4>(__fmul2_rn(lc.a2[c][pi], s2));
+                        lc.h[c][pi] = __ffma2_rn(decay, lc.h[c][pi], hj[pi]);
+                    }
                 }
             }
         }
 
-        IoT* out_row = valid ? static_cast<IoT*>(p.out) + chain * p.seqlen + t_begin : nullptr;
-        float sdt = 0.0f;
+        IoT* out_row[kCpl];
+        float sdt[kCpl];
+#pragma unroll
+        for (int c = 0; c < kCpl; ++c) {
+            out_row[c] = valid[c] ? static_cast<IoT*>(p.out) + chain[c] * p.seqlen + t_begin : nullptr;
+            sdt[c] = 0.0f;
+        }
         bool ok;
         if (p.mode == kModePassA && k > 0)
-            ok = run_segment<IoT, kHasZ, kSoftplus, false>(p, maps, wsm, lane, b, d0, t_begin, t_end,
-                                                           h, a2, bias, Dd, nullptr, seq, sdt);
+            ok = run_segment<IoT, kCpl, kHasZ, kSoftplus, false>(p, maps, wsm, lane, b, d0, t_begin,
+                                                                 t_end, lc, out_row, seq, sdt);
         else
-            ok = run_segment<IoT, kHasZ, kSoftplus, true>(p, maps, wsm, lane, b, d0, t_begin, t_end,
-                                                          h, a2, bias, Dd, out_row, seq, sdt);
+            ok = run_segment<IoT, kCpl, kHasZ, kSoftplus, true>(p, maps, wsm, lane, b, d0, t_begin,
+                                                                t_end, lc, out_row, seq, sdt);
         if (!ok) break;
 
         const bool last_seg = k == p.nseg - 1;
         if (p.mode == kModeChained) {
             if (!last_seg) {
-                if (valid) store16(p.carry + chain * kNPad, h);
+#pragma unroll
+                for (int c = 0; c < kCpl; ++c)
+                    if (valid[c]) store16(p.carry + chain[c] * kNPad, lc.h[c]);
                 __threadfence();
                 __syncwarp();
                 if (lane == 0 && !p.withhold_handoff)
                     st_release_gpu(p.flags + g, (unsigned int)(k + 1));
             }
-        } else if (p.mode == kModePassA && valid) {
-            store16(p.ws_h + (k * p.chains + chain) * kNPad, h);
-            if (k >= 1) __stcg(p.ws_sdt + k * p.chains + chain, sdt);
-        }
-        if (last_seg && p.mode != kModePassA && valid && p.last_state != nullptr) {
-            float* ls = p.last_state + chain * p.dstate;
+        } else if (p.mode == kModePassA) {
 #pragma unroll
-            for (int n = 0; n < kNPad; ++n)
-                if (n < p.dstate) ls[n] = h[n];
+            for (int c = 0; c < kCpl; ++c) {
+                if (!valid[c]) continue;
+                store16(p.ws_h + (k * p.chains + chain[c]) * kNPad, lc.h[c]);
+                if (k >= 1) __stcg(p.ws_sdt + k * p.chains + chain[c], sdt[c]);
+            }
+        }
+        if (last_seg && p.mode != kModePassA && p.last_state != nullptr) {
+#pragma unroll
+            for (int c = 0; c < kCpl; ++c) {
+                if (!valid[c]) continue;
+                float* ls = p.last_state + chain[c] * p.dstate;
+#pragma unroll
+                for (int pi = 0; pi < kNPad / 2; ++pi) {
+                    if (2 * pi < p.dstate) ls[2 * pi] = lc.h[c][pi].x;
+                    if (2 * pi + 1 < p.dstate) ls[2 * pi + 1] = lc.h[c][pi].y;
+                }
+            }
         }
     }
 }

@@ -48,11 +48,12 @@ class ScanPlan(ctypes.Structure):
         ("units_pass_a", ctypes.c_int64), ("units_pass_b", ctypes.c_int64),
         ("warps_per_cta", ctypes.c_int32), ("launches", ctypes.c_int32),
         ("tma_capable", ctypes.c_int32), ("mode", ctypes.c_int32),
-        ("workspace_bytes", ctypes.c_size_t),
+        ("channels_per_lane", ctypes.c_int32), ("reserved", ctypes.c_int32),
+        ("max_warps", ctypes.c_int64), ("workspace_bytes", ctypes.c_size_t),
     ]
 
     def as_dict(self) -> dict:
-        return {name: getattr(self, name) for name, _ in self._fields_}
+        return {name: getattr(self, name) for name, _ in self._fields_ if name != "reserved"}
 
 
 class MambaError(RuntimeError):

@@ -98,29 +98,33 @@ def test_update_rejects_bad_arguments(lib):
 
 
 def test_plan_layer_shapes(lib):
-    # 2.8B layer: 2560 groups >= 148 x 16 resident warps -> chained 256-step segments
+    # 2.8B layer: 2560 groups of 32 channels, chained 256-step segments,
+    # at most one warp per group
     c = SCAN_CONFIGS["mamba_2p8b_layer"]
     p = ops.scan_plan(c.batch, c.dim, c.dstate, c.seqlen, c.io_dtype, c.bc_dtype)
-    assert p["mode"] == 0 and p["launches"] == 1
+    assert p["mode"] == 0 and p["launches"] == 1 and p["channels_per_lane"] == 1
     assert p["groups"] == c.batch * c.dim // 32
     assert p["tile_len"] == 16 and p["tma_capable"] == 1
     assert p["nchunks"] == 8 and p["chunk_len"] == 256
     assert p["units_pass_a"] == p["groups"] * 8 and p["units_pass_b"] == 0
+    assert p["max_warps"] == min(p["groups"], 148 * 16)
     chains = c.batch * c.dim
     flags = (p["groups"] * 4 + 255) // 256 * 256
     assert p["workspace_bytes"] == 256 + flags + chains * 64
-    # 1.4B layer: 1024 groups, between a quarter and all of the resident warps -> one segment
+    # 1.4B layer: 1024 groups, chained the same way with one warp per group
     c = SCAN_CONFIGS["mamba_1p4b_layer"]
     p = ops.scan_plan(c.batch, c.dim, c.dstate, c.seqlen, c.io_dtype, c.bc_dtype)
-    assert p["mode"] == 0 and p["nchunks"] == 1 and p["units_pass_a"] == 1024
-    assert p["workspace_bytes"] == 256 + 4096
+    assert p["mode"] == 0 and p["channels_per_lane"] == 1 and p["groups"] == 1024
+    assert p["nchunks"] == 8 and p["max_warps"] == 1024
+    assert p["workspace_bytes"] == 256 + 4096 + 8 * 4096 * 64
 
 
 def test_plan_parallel_for_the_million_token_sequence(lib):
     c = SCAN_CONFIGS["long_dna_1m"]
     p = ops.scan_plan(c.batch, c.dim, c.dstate, c.seqlen, c.io_dtype, c.bc_dtype, sm_count=148)
     K = p["nchunks"]
-    assert p["mode"] == 1 and p["launches"] == 2
+    assert p["mode"] == 1 and p["launches"] == 2 and p["channels_per_lane"] == 1
+    assert p["groups"] == 1536 // 32
     assert K - 1 == (148 * 16) // p["groups"]           # one item per resident warp and pass
     assert p["chunk_len"] % p["tile_len"] == 0
     assert (K - 1) * p["chunk_len"] < c.seqlen <= K * p["chunk_len"]
@@ -129,6 +133,7 @@ def test_plan_parallel_for_the_million_token_sequence(lib):
     expect = 256 + 256 + ((K - 1) * chains * 64 + 255) // 256 * 256 + \
         ((K - 1) * chains * 4 + 255) // 256 * 256
     assert p["workspace_bytes"] == expect
+    assert p["workspace_bytes"] <= 8 << 20
 
 
 def test_plan_tiny_is_one_segment(lib):
