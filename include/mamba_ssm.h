@@ -77,7 +77,8 @@ typedef enum {
 } mamba_dtype_t;
 
 /* Flags (mamba_dims_t.flags). */
-#define MAMBA_FLAG_NO_TMA 0x1          /* stage tiles with plain loads instead of TMA */
+#define MAMBA_FLAG_NO_TMA 0x1          /* plain loads instead of TMA (scan tiles; the
+                                          * update's bulk streaming path) */
 #define MAMBA_FLAG_PARALLEL_CHUNKS 0x2 /* with num_chunks >= 1: parallel (recompute) mode */
 /* Test only: in mode 0, segments never hand their state on, so every wait for
  * a predecessor runs out (after ~0.3 s) and the call reports MAMBA_ERR_TIMEOUT
@@ -230,6 +231,9 @@ MAMBA_API mamba_status_t mamba_selective_scan_fwd_noalloc(
  *   D, dt_bias         (dim,) fp32; may be NULL
  *   dims->dt_softplus  nonzero: Delta = softplus(dt + dt_bias)
  * dims->seqlen, num_chunks and workspace are ignored.
+ * Paths: for dstate == 16, dim % 8 == 0 and 16-byte aligned buffers the state
+ * streams through shared memory by bulk TMA (MAMBA_FLAG_NO_TMA turns that
+ * off); otherwise plain vectorised loads (dstate == 16) or a scalar path.
  */
 MAMBA_API mamba_status_t mamba_selective_state_update(float *state, const void *x, const void *dt,
                                                       const float *A, const void *B, const void *C,

@@ -131,9 +131,40 @@ cudaError_t dispatch_scan(const ScanParams& prm, const CUtensorMap* maps, int cp
     return dispatch_scan_cpl<IoT, 1>(prm, maps, has_z, sp, want_warps, dev, sms, stream);
 }
 
+template <typename IoT, typename BcT, bool kHasZ>
+cudaError_t launch_update_bulk(const UpdateParams& prm, int dev, int sms, cudaStream_t stream) {
+    static bool attr_done[kMaxDevices] = {false};
+    static int resident[kMaxDevices] = {0};
+    auto kernel = state_update_bulk_kernel<IoT, BcT, kHasZ>;
+    cudaError_t e = ensure_smem_attr(kernel, kBulkSmemBytes, attr_done, dev);
+    if (e != cudaSuccess) return e;
+    int per_sm = (dev >= 0 && dev < kMaxDevices) ? resident[dev] : 0;
+    if (per_sm <= 0) {
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kBulkThreads,
+                                                          kBulkSmemBytes);
+        if (e != cudaSuccess) return e;
+        if (per_sm <= 0) return cudaErrorInvalidConfiguration;
+        if (dev >= 0 && dev < kMaxDevices) resident[dev] = per_sm;
+    }
+    // Each CTA owns one channel block and every J-th batch row: J copies of the
+    // nblk blocks fill the resident CTAs.  Among J <= resident / nblk pick the
+    // one whose slowest CTA has the fewest rows, then the smallest such J.
+    const int64_t nblk = (prm.dim + kBulkTile - 1) / kBulkTile;
+    const int64_t jmax = std::max<int64_t>(1, std::min<int64_t>(prm.batch, ((int64_t)per_sm * sms) / nblk));
+    int64_t J = jmax;
+    for (int64_t j = jmax; j >= 1 && j * 2 >= jmax; --j)
+        if ((prm.batch + j - 1) / j <= (prm.batch + J - 1) / J) J = j;
+    const int64_t grid = nblk * J;
+    kernel<<<(unsigned)grid, kBulkThreads, kBulkSmemBytes, stream>>>(prm);
+    return cudaGetLastError();
+}
+
 template <typename IoT, typename BcT>
-cudaError_t dispatch_update_bc(const UpdateParams& prm, bool fast, bool has_z,
-                               cudaStream_t stream) {
+cudaError_t dispatch_update_bc(const UpdateParams& prm, bool fast, bool bulk, bool has_z,
+                               int dev, int sms, cudaStream_t stream) {
+    if (bulk)
+        return has_z ? launch_update_bulk<IoT, BcT, true>(prm, dev, sms, stream)
+                     : launch_update_bulk<IoT, BcT, false>(prm, dev, sms, stream);
     if (fast) {
         // x covers channels (kUpdateChainsPerCta per CTA), y covers batch rows.
         const dim3 grid((unsigned)((prm.dim + kUpdateChainsPerCta - 1) / kUpdateChainsPerCta),
@@ -153,10 +184,11 @@ cudaError_t dispatch_update_bc(const UpdateParams& prm, bool fast, bool has_z,
 }
 
 template <typename IoT>
-cudaError_t dispatch_update(const UpdateParams& prm, bool bc_bf16, bool fast, bool has_z,
-                            cudaStream_t stream) {
-    return bc_bf16 ? dispatch_update_bc<IoT, __nv_bfloat16>(prm, fast, has_z, stream)
-                   : dispatch_update_bc<IoT, float>(prm, fast, has_z, stream);
+cudaError_t dispatch_update(const UpdateParams& prm, bool bc_bf16, bool fast, bool bulk,
+                            bool has_z, int dev, int sms, cudaStream_t stream) {
+    return bc_bf16
+               ? dispatch_update_bc<IoT, __nv_bfloat16>(prm, fast, bulk, has_z, dev, sms, stream)
+               : dispatch_update_bc<IoT, float>(prm, fast, bulk, has_z, dev, sms, stream);
 }
 
 }  // namespace
@@ -452,11 +484,23 @@ MAMBA_API mamba_status_t mamba_selective_state_update(float* state, const void* 
     prm.dt_softplus = dims->dt_softplus != 0;
     const bool fast = dims->dstate == 16 && aligned(state, 16) && aligned(A, 16) &&
                       aligned(B, 4 * bc_es) && aligned(C, 4 * bc_es);
+    // Streaming (bulk TMA) path: every bulk copy needs 16-byte aligned ends.
+    const bool bulk = fast && !(dims->flags & MAMBA_FLAG_NO_TMA) && dims->dim % 8 == 0 &&
+                      aligned(x, 16) && aligned(dt, 16) && aligned(out, 16) &&
+                      (!z || aligned(z, 16)) && (!D || aligned(D, 16)) &&
+                      (!dt_bias || aligned(dt_bias, 16)) && aligned(B, 16) && aligned(C, 16);
     const bool has_z = z != nullptr;
     const bool bc_bf16 = dims->bc_dtype == MAMBA_BF16;
-    const cudaError_t e = dims->io_dtype == MAMBA_BF16
-                              ? dispatch_update<__nv_bfloat16>(prm, bc_bf16, fast, has_z, stream)
-                              : dispatch_update<float>(prm, bc_bf16, fast, has_z, stream);
+    int dev = 0;
+    int sms = 1;
+    if (bulk) {
+        sms = current_sm_count(&dev);
+        if (sms <= 0) return MAMBA_ERR_CUDA;
+    }
+    const cudaError_t e =
+        dims->io_dtype == MAMBA_BF16
+            ? dispatch_update<__nv_bfloat16>(prm, bc_bf16, fast, bulk, has_z, dev, sms, stream)
+            : dispatch_update<float>(prm, bc_bf16, fast, bulk, has_z, dev, sms, stream);
     return e == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
 }
 

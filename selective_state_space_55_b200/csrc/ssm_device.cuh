@@ -53,6 +53,18 @@ __device__ __forceinline__ float exp2_near_one_exact(float x) {
     return fabsf(x) < 0.0625f ? series : hw;
 }
 
+// exp2_near_one_exact on both halves of x, the series in packed fp32x2.
+__device__ __forceinline__ float2 exp2_near_one_exact2(float2 x) {
+    const float2 c1 = make_float2(0.6931471805599453f, 0.6931471805599453f);
+    const float2 c2 = make_float2(0.2402265069591007f, 0.2402265069591007f);
+    const float2 c3 = make_float2(0.05550410866482158f, 0.05550410866482158f);
+    const float2 c4 = make_float2(0.009618129107628477f, 0.009618129107628477f);
+    const float2 one = make_float2(1.0f, 1.0f);
+    const float2 series = __ffma2_rn(x, __ffma2_rn(x, __ffma2_rn(x, __ffma2_rn(x, c4, c3), c2), c1), one);
+    return make_float2(fabsf(x.x) < 0.0625f ? series.x : ex2_approx(x.x),
+                       fabsf(x.y) < 0.0625f ? series.y : ex2_approx(x.y));
+}
+
 // softplus(s) = log(1 + e^s) = max(s, 0) + log1p(e^-|s|).
 // log1p(w) for w = e^-|s| in (0, 1] is evaluated as 2 atanh(r) with
 // r = w / (2 + w) in (0, 1/3]:  2 atanh(r) = 2 r (1 + r^2/3 + r^4/5 + ...).
@@ -137,6 +149,10 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                  : "memory");
@@ -175,6 +191,39 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
         " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
         : "memory");
+}
+
+// 1-D bulk copy global -> this CTA's shared memory, completing on `bar`.
+// Addresses 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
+// 1-D bulk copy shared -> global, tracked by the issuing thread's bulk groups.
+__device__ __forceinline__ void bulk_store(void* dst, uint32_t src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+                 ::"l"(reinterpret_cast<uint64_t>(dst)), "r"(src), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Wait until at most N of this thread's committed bulk stores still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+// Wait until at most N of this thread's committed bulk stores are incomplete.
+template <int N>
+__device__ __forceinline__ void bulk_wait() {
+    asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
 }
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {

@@ -123,6 +123,200 @@ __global__ void __launch_bounds__(kUpdateThreads)
     }
 }
 
+// ----------------------------------------------------------------------------
+// Streaming path (N = 16, dim % 8 == 0, 16-byte aligned buffers).
+//
+// Each CTA owns one block of kBulkTile channels and walks batch rows; the
+// block's A rows, D and dt_bias stay in registers.  A producer warp keeps a
+// kBulkStages-deep ring of tiles loading by 1-D bulk TMA (the tile's fp32
+// state, x, dt, z and the batch row's B and C).  Four consumer warps each own
+// 32 channels of the tile: they update the state in place in shared memory,
+// write the outputs beside it, bulk-store their slice back, and release the
+// stage through an mbarrier once the store has read it.  No CTA-wide barrier
+// sits on the path, so the ring keeps several tiles in flight per CTA.  Four
+// lanes share a chain (a float4 of state each); softplus and silu run once per
+// chain, spread over the four lanes, and are exchanged by shuffles.  Abar is
+// MUFU ex2 for bf16 inputs and exp2_near_one_exact for fp32 inputs, as in the
+// scan.
+constexpr int kBulkConsumers = 4;
+constexpr int kBulkThreads = 32 * (kBulkConsumers + 1);
+constexpr int kBulkTile = 32 * kBulkConsumers;       // channels per tile
+constexpr int kBulkStages = 4;
+constexpr int kBOffState = 0;                        // kBulkTile x 64 B
+constexpr int kBOffX = kBulkTile * 64;               // kBulkTile x up to 4 B each:
+constexpr int kBOffDt = kBOffX + kBulkTile * 4;
+constexpr int kBOffZ = kBOffDt + kBulkTile * 4;
+constexpr int kBOffOut = kBOffZ + kBulkTile * 4;
+constexpr int kBOffB = kBOffOut + kBulkTile * 4;     // 16 x up to 4 B
+constexpr int kBOffC = kBOffB + 64;
+constexpr int kBStage = ((kBOffC + 64 + 127) / 128) * 128;
+constexpr int kBulkSmemBytes = kBulkStages * kBStage + 2 * kBulkStages * 8 + 1024;
+
+template <typename IoT, typename BcT, bool kHasZ>
+__global__ void __launch_bounds__(kBulkThreads)
+    state_update_bulk_kernel(const __grid_constant__ UpdateParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBulkStages * kBStage);
+    uint64_t* empty = full + kBulkStages;
+    constexpr int ES = (int)sizeof(IoT);
+    constexpr int BS = (int)sizeof(BcT);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // This CTA: channel block `blk`, batch rows b0, b0 + bstep, ...
+    const int nblk = (int)((p.dim + kBulkTile - 1) / kBulkTile);
+    const int blk = (int)(blockIdx.x % nblk);
+    const int64_t b0 = blockIdx.x / nblk;
+    const int64_t bstep = max(1u, gridDim.x / (unsigned)nblk);
+    const int64_t d0 = (int64_t)blk * kBulkTile;
+    const int nch = (int)min((int64_t)kBulkTile, p.dim - d0);
+    const int64_t mine = b0 < p.batch ? (p.batch - b0 + bstep - 1) / bstep : 0;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kBulkStages; ++s) {
+            mbar_init(smem_u32(&full[s]), 1);
+            mbar_init(smem_u32(&empty[s]), kBulkConsumers);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    if (warp == kBulkConsumers) {
+        // ---------------- producer ----------------
+        if (lane != 0) return;
+        const uint32_t tok = (uint32_t)nch * ES;
+        const uint32_t bytes = (uint32_t)nch * 64 + (kHasZ ? 3u : 2u) * tok + 2u * 16u * BS;
+        int64_t k = 0;
+        for (; k < mine; ++k) {
+            const int s = (int)(k % kBulkStages);
+            if (k >= kBulkStages &&
+                !mbar_wait_bounded(smem_u32(&empty[s]), (uint32_t)((k / kBulkStages - 1) & 1))) {
+                record_device_error(MAMBA_ERR_TIMEOUT);
+                break;
+            }
+            const int64_t b = b0 + k * bstep;
+            const int64_t c0 = b * p.dim + d0;
+            uint8_t* st = smem + s * kBStage;
+            const uint32_t bar = smem_u32(&full[s]);
+            fence_proxy_async_smem();
+            mbar_arrive_expect_tx(bar, bytes);
+            bulk_load(smem_u32(st + kBOffState), p.state + c0 * 16, (uint32_t)nch * 64, bar);
+            bulk_load(smem_u32(st + kBOffX), static_cast<const IoT*>(p.x) + c0, tok, bar);
+            bulk_load(smem_u32(st + kBOffDt), static_cast<const IoT*>(p.dt) + c0, tok, bar);
+            if (kHasZ) bulk_load(smem_u32(st + kBOffZ), static_cast<const IoT*>(p.z) + c0, tok, bar);
+            bulk_load(smem_u32(st + kBOffB), static_cast<const BcT*>(p.B) + b * 16, 16 * BS, bar);
+            bulk_load(smem_u32(st + kBOffC), static_cast<const BcT*>(p.C) + b * 16, 16 * BS, bar);
+        }
+        // Loads still in flight must land before the CTA's shared memory goes away.
+        for (int64_t j = max((int64_t)0, k - kBulkStages); j < k; ++j)
+            (void)mbar_wait_bounded(smem_u32(&full[j % kBulkStages]), (uint32_t)((j / kBulkStages) & 1));
+        return;
+    }
+
+    // ---------------- consumers ----------------
+    // Lane l of warp w holds quarter q = l & 3 of chain 32 w + 8 it + (l >> 2)
+    // for items it = 0..3.  The four lanes of a quad also split the per-chain
+    // scalar work: lane q computes softplus and silu for item q.
+    constexpr bool kExact = sizeof(IoT) == 4;
+    const int q = lane & 3;
+    const int quad = lane & ~3;
+    constexpr int kItems = 4;
+    float2 a01[kItems], a23[kItems];
+    int ch[kItems];
+#pragma unroll
+    for (int it = 0; it < kItems; ++it) {
+        ch[it] = 32 * warp + 8 * it + (lane >> 2);
+        const int64_t d = d0 + (ch[it] < nch ? ch[it] : 0);
+        const float4 av = *(reinterpret_cast<const float4*>(p.A + d * 16) + q);
+        a01[it] = __fmul2_rn(make_float2(av.x, av.y), make_float2(kLog2e, kLog2e));
+        a23[it] = __fmul2_rn(make_float2(av.z, av.w), make_float2(kLog2e, kLog2e));
+    }
+    // Per-chain parameters of item q (this lane's scalar duty).
+    const int my_ch = 32 * warp + 8 * q + (lane >> 2);   // chain of item q
+    const bool my_live = my_ch < nch;
+    const int64_t my_d = d0 + (my_live ? my_ch : 0);
+    const float my_D = p.D != nullptr ? p.D[my_d] : 0.0f;
+    const float my_bias = p.dt_bias != nullptr ? p.dt_bias[my_d] : 0.0f;
+    const int nw = max(0, min(32, nch - 32 * warp));   // this warp's chains in a tile
+
+    for (int64_t k = 0; k < mine; ++k) {
+        const int s = (int)(k % kBulkStages);
+        uint8_t* st = smem + s * kBStage;
+        bool ok = mbar_wait_bounded(smem_u32(&full[s]), (uint32_t)((k / kBulkStages) & 1));
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) {
+            if (lane == 0) record_device_error(MAMBA_ERR_TIMEOUT);
+            break;
+        }
+        const IoT* xs = reinterpret_cast<const IoT*>(st + kBOffX);
+        const BcT* Bs = reinterpret_cast<const BcT*>(st + kBOffB) + 4 * q;
+        const BcT* Cs = reinterpret_cast<const BcT*>(st + kBOffC) + 4 * q;
+        const float2 b01 = make_float2(DType<BcT>::load(Bs), DType<BcT>::load(Bs + 1));
+        const float2 b23 = make_float2(DType<BcT>::load(Bs + 2), DType<BcT>::load(Bs + 3));
+        const float2 c01 = make_float2(DType<BcT>::load(Cs), DType<BcT>::load(Cs + 1));
+        const float2 c23 = make_float2(DType<BcT>::load(Cs + 2), DType<BcT>::load(Cs + 3));
+        // Delta of item q's chain, computed by this lane.
+        const int mc = my_live ? my_ch : 0;
+        const float my_s = DType<IoT>::load(reinterpret_cast<const IoT*>(st + kBOffDt) + mc) + my_bias;
+        const float my_delta = p.dt_softplus ? softplus_f32(my_s) : my_s;
+        float y_item[kItems];
+#pragma unroll
+        for (int it = 0; it < kItems; ++it) {
+            const int c = ch[it] < nch ? ch[it] : 0;
+            const float4 hs = reinterpret_cast<const float4*>(st + kBOffState)[4 * c + q];
+            const float x = DType<IoT>::load(xs + c);
+            const float delta = __shfl_sync(0xffffffffu, my_delta, quad | it);
+            const float dx = delta * x;
+            const float2 d2 = make_float2(delta, delta);
+            const float2 dx2 = make_float2(dx, dx);
+            const float2 x01 = __fmul2_rn(d2, a01[it]);
+            const float2 x23 = __fmul2_rn(d2, a23[it]);
+            const float2 e01 = kExact ? exp2_near_one_exact2(x01)
+                                      : make_float2(ex2_approx(x01.x), ex2_approx(x01.y));
+            const float2 e23 = kExact ? exp2_near_one_exact2(x23)
+                                      : make_float2(ex2_approx(x23.x), ex2_approx(x23.y));
+            const float2 h01 = __ffma2_rn(e01, make_float2(hs.x, hs.y), __fmul2_rn(dx2, b01));
+            const float2 h23 = __ffma2_rn(e23, make_float2(hs.z, hs.w), __fmul2_rn(dx2, b23));
+            const float2 yy = __ffma2_rn(c23, h23, __fmul2_rn(c01, h01));
+            float y = yy.x + yy.y;
+            y += __shfl_xor_sync(0xffffffffu, y, 1);
+            y += __shfl_xor_sync(0xffffffffu, y, 2);
+            y_item[it] = y;
+            if (ch[it] < nch)
+                reinterpret_cast<float4*>(st + kBOffState)[4 * c + q] =
+                    make_float4(h01.x, h01.y, h23.x, h23.y);
+        }
+        // Output of item q's chain, by this lane.
+        float y = y_item[0];
+#pragma unroll
+        for (int it = 1; it < kItems; ++it)
+            if (q == it) y = y_item[it];
+        if (my_live) {
+            y = fmaf(my_D, DType<IoT>::load(xs + my_ch), y);
+            if (kHasZ) y *= silu_f32(DType<IoT>::load(reinterpret_cast<const IoT*>(st + kBOffZ) + my_ch));
+            DType<IoT>::store(reinterpret_cast<IoT*>(st + kBOffOut) + my_ch, y);
+        }
+        // Store this warp's slice, then hand the stage back to the producer.
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            if (nw > 0) {
+                const int64_t c0 = (b0 + k * bstep) * p.dim + d0 + 32 * warp;
+                bulk_store(p.state + c0 * 16, smem_u32(st + kBOffState + 32 * warp * 64),
+                           (uint32_t)nw * 64);
+                bulk_store(static_cast<IoT*>(p.out) + c0, smem_u32(st + kBOffOut + 32 * warp * ES),
+                           (uint32_t)nw * ES);
+                bulk_commit();
+                bulk_wait_read<0>();
+            }
+            mbar_arrive(smem_u32(&empty[s]));
+        }
+    }
+    if (lane == 0) bulk_wait<0>();
+}
+
 template <typename IoT, typename BcT, bool kHasZ>
 __global__ void __launch_bounds__(kUpdateThreads)
     state_update_generic_kernel(const __grid_constant__ UpdateParams p) {

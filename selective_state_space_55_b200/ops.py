@@ -201,7 +201,7 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softp
 
 
 def selective_state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=None,
-                           dt_softplus=True, out=None, stream=None):
+                           dt_softplus=True, out=None, flags=0, stream=None):
     """One generation step through ``mamba_selective_state_update``; ``state`` is
     updated in place.  Returns ``out`` (batch, dim) in x's dtype."""
     batch, dim, N = state.shape
@@ -220,7 +220,7 @@ def selective_state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=None,
     _check_cuda("out", out, (io,), (batch, dim))
     dims = MambaDims(batch=batch, dim=dim, dstate=N, seqlen=0, io_dtype=_DTYPE_CODE[io],
                      bc_dtype=_DTYPE_CODE[bc], dt_softplus=int(bool(dt_softplus)),
-                     num_chunks=0, flags=0, reserved=0, workspace=None, workspace_bytes=0)
+                     num_chunks=0, flags=flags, reserved=0, workspace=None, workspace_bytes=0)
     rc = library().mamba_selective_state_update(
         _ptr(state), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
         _ptr(dt_bias), _ptr(out), ctypes.byref(dims), _stream_handle(stream))

@@ -157,3 +157,29 @@ def test_decode_48_layers_rotating(ref):
                                                     dt_bias=c(l["dt_bias"]))
         assert max_rel_err(l["state"], o_state) <= FP32_TOL
         assert max_rel_err(outs[i], o_out) <= BF16_TOL
+
+
+@pytest.mark.parametrize("dim", [1024, 136, 8])
+def test_decode_streaming_and_plain_paths_agree(ref, dim):
+    """The bulk-TMA streaming path (dim % 8 == 0, with a partial last tile of the
+    128-channel tiles) and the plain-load path both match the oracle."""
+    cfg = decode_cfg(6, dim)
+    layer = I.make_decode_layer(cfg, DEV, seed=dim)
+    tok = I.make_decode_token(cfg, DEV, seed=dim + 1)
+    results = []
+    for flags in (0, ops.MAMBA_FLAG_NO_TMA):
+        state = layer["state"].clone()
+        out = ops.selective_state_update(state, tok["x"], tok["dt"], layer["A"], tok["B"],
+                                         tok["C"], D=layer["D"], z=tok["z"],
+                                         dt_bias=layer["dt_bias"], flags=flags)
+        torch.cuda.synchronize()
+        assert ops.device_status() == 0
+        results.append((state, out))
+    c = lambda t: t.cpu()  # noqa: E731
+    o_state, o_out = ref.selective_state_update(
+        c(layer["state"]), c(tok["x"]), c(tok["dt"]), c(layer["A"]), c(tok["B"]), c(tok["C"]),
+        D=c(layer["D"]), z=c(tok["z"]), dt_bias=c(layer["dt_bias"]))
+    for state, out in results:
+        assert max_rel_err(state, o_state) <= FP32_TOL
+        assert max_rel_err(out, o_out) <= BF16_TOL
+    assert max_rel_err(results[0][0], results[1][0].double()) <= FP32_TOL
