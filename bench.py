@@ -186,7 +186,7 @@ class Workload:
             self.dcfg = I.DecodeConfig(self.dcfg.name, self.dcfg.batch, self.dcfg.dim,
                                        self.dcfg.dstate, decode_layers, self.dcfg.steps)
         c = self.cfg
-        self.x = I.make_scan_inputs(c, "cuda", seed=1000 + rank)
+        self.x = I.make_scan_inputs(c, "cuda", seed=rank_seed(rank))
         self.out = torch.empty_like(self.x["u"])
         self.last = torch.empty((c.batch, c.dim, c.dstate), dtype=torch.float32, device="cuda")
         ws = ops.scan_workspace_bytes(c.batch, c.dim, c.dstate, c.seqlen, c.io_dtype, c.bc_dtype)
@@ -304,6 +304,7 @@ def cpu_baseline(w: Workload, target_s: float) -> dict:
 # ----------------------------------------------------------------- distributed
 
 _WORLD = 1
+_REDUCE_DEVICE = "cuda"
 
 
 def barrier():
@@ -312,11 +313,22 @@ def barrier():
 
 
 def max_over_ranks(v: float) -> float:
+    """Largest value of `v` over all ranks (each rank's device time)."""
     if _WORLD == 1:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=_REDUCE_DEVICE)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(rank: int) -> int:
+    """Seed of a rank's own synthetic inputs (every rank scans its own batch)."""
+    return 1000 + rank
+
+
+def job_gelem_per_s(world: int, elements_per_rank: int, steps: int, max_ms: float) -> float:
+    """Whole-job throughput: every rank's elements over the slowest rank's time."""
+    return world * elements_per_rank * steps / (max_ms * 1e-3) / 1e9
 
 
 # ----------------------------------------------------------------- arms
@@ -366,7 +378,7 @@ def bench_ours(args, rank, world, local):
     decode_ms = max_over_ranks(sum(b.elapsed_time(cc) for _, b, cc in ev))
     K = args.steps
     elems = c.elements
-    value = world * elems * K / (scan_ms * 1e-3) / 1e9          # Gelem/s, whole job
+    value = job_gelem_per_s(world, elems, K, scan_ms)            # Gelem/s, whole job
     scan_launch_ms = scan_ms / K
     decode_step_us = decode_ms / K * 1e3
 
@@ -416,7 +428,7 @@ def bench_ours(args, rank, world, local):
     e2e = None
     if not args.no_e2e and args.only != "decode":
         r = run_e2e(w, max(1, min(K, args.e2e_steps)), 2)
-        e2e = {"value": round(world * elems * r["steps"] / (r["ms_total"] * 1e-3) / 1e9, 3),
+        e2e = {"value": round(job_gelem_per_s(world, elems, r["steps"], r["ms_total"]), 3),
                "unit": "Gelem/s", "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
                "steps": r["steps"],
                "path": "pinned host u/delta/z/B/C -> device -> mamba_selective_scan_fwd -> "
