@@ -5,16 +5,22 @@ benchmark's CPU-baseline / reference arm are the only callers.  The CUDA
 library never imports, links or runs anything here, and nothing here imports
 the CUDA library.
 
-What it computes (float64, plain sequential recurrence, zero initial state):
+What it computes (float64, plain sequential recurrence):
 
     Delta_t  = softplus(delta_t + bias_d)            (softplus may be off)
     h_t,n    = exp(Delta_t * A_d,n) * h_{t-1},n + Delta_t * B_t,n * u_t
     y_t      = sum_n C_t,n * h_t,n + D_d * u_t
     out_t    = y_t * silu(z_t)                       (z optional)
 
-following "超越注意力：探索Mamba与状态空间模型" (sections 状态空间模型基础,
-选择性状态空间模型, 代码实现概览) and "Mamba 与状态空间模型" (section 由词元决定).
-The update is the same single step applied to a given state.
+from h_{-1} = 0, or from a given ``initial_state``.  With ``zoh=True`` the input
+term is the zero-order-hold one, expm1(Delta_t A_d,n) / A_d,n * B_t,n * u_t
+(Delta_t B_t,n u_t where A_d,n = 0), i.e. Bbar = (Delta A)^-1 (exp(Delta A) - I)
+Delta B for the diagonal A.
+
+Following "超越注意力：探索Mamba与状态空间模型" (sections 状态空间模型基础 for
+the zero-order hold, 选择性状态空间模型, 代码实现概览 for the Euler default) and
+"Mamba 与状态空间模型" (section 由词元决定).  The update is the same single step
+applied to a given state.
 
 Every input is converted to contiguous float64 first; bf16 and fp32 values
 convert exactly, so the oracle sees the same numbers the GPU sees.
@@ -72,12 +78,13 @@ class Oracle:
         self._lib = ctypes.CDLL(str(path))
         dp = ctypes.POINTER(ctypes.c_double)
         i64 = ctypes.c_int64
-        self._lib.oracle_selective_scan_f64.restype = ctypes.c_int
-        self._lib.oracle_selective_scan_f64.argtypes = [
-            i64, i64, i64, i64, dp, dp, dp, dp, dp, dp, dp, dp, ctypes.c_int, dp, dp]
-        self._lib.oracle_selective_state_update_f64.restype = ctypes.c_int
-        self._lib.oracle_selective_state_update_f64.argtypes = [
-            i64, i64, i64, dp, dp, dp, dp, dp, dp, dp, dp, dp, ctypes.c_int, dp, dp]
+        ci = ctypes.c_int
+        self._lib.oracle_selective_scan_ex_f64.restype = ctypes.c_int
+        self._lib.oracle_selective_scan_ex_f64.argtypes = [
+            i64, i64, i64, i64, dp, dp, dp, dp, dp, dp, dp, dp, ci, ci, dp, dp, dp]
+        self._lib.oracle_selective_state_update_ex_f64.restype = ctypes.c_int
+        self._lib.oracle_selective_state_update_ex_f64.argtypes = [
+            i64, i64, i64, dp, dp, dp, dp, dp, dp, dp, dp, dp, ci, ci, dp, dp]
         self._lib.oracle_num_threads.restype = ctypes.c_int
         self._lib.oracle_num_threads.argtypes = []
 
@@ -85,14 +92,15 @@ class Oracle:
         return int(self._lib.oracle_num_threads())
 
     def selective_scan(self, u, delta, A, B, C, D=None, z=None, delta_bias=None,
-                       softplus=True):
+                       softplus=True, zoh=False, initial_state=None):
         """Return (out, last_state) as float64 arrays.
 
         u, delta, z: (batch, dim, L); B, C: (batch, N, L); A: (dim, N);
-        D, delta_bias: (dim,).  out: (batch, dim, L); last_state: (batch, dim, N).
+        D, delta_bias: (dim,); initial_state: (batch, dim, N) or None (zeros).
+        out: (batch, dim, L); last_state: (batch, dim, N).
         """
         u, delta, A, B, C = map(_f64, (u, delta, A, B, C))
-        D, z, delta_bias = map(_f64, (D, z, delta_bias))
+        D, z, delta_bias, initial_state = map(_f64, (D, z, delta_bias, initial_state))
         batch, dim, seqlen = u.shape
         dstate = A.shape[1]
         assert delta.shape == u.shape and A.shape == (dim, dstate)
@@ -100,19 +108,21 @@ class Oracle:
         assert z is None or z.shape == u.shape
         assert D is None or D.shape == (dim,)
         assert delta_bias is None or delta_bias.shape == (dim,)
+        assert initial_state is None or initial_state.shape == (batch, dim, dstate)
         out = np.empty_like(u)
         last_state = np.empty((batch, dim, dstate), dtype=np.float64)
-        rc = self._lib.oracle_selective_scan_f64(
+        rc = self._lib.oracle_selective_scan_ex_f64(
             batch, dim, dstate, seqlen, _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C),
-            _ptr(D), _ptr(z), _ptr(delta_bias), int(bool(softplus)), _ptr(out),
-            _ptr(last_state))
+            _ptr(D), _ptr(z), _ptr(delta_bias), int(bool(softplus)), int(bool(zoh)),
+            _ptr(initial_state), _ptr(out), _ptr(last_state))
         if rc != 0:
             raise ValueError(f"oracle_selective_scan_f64 returned {rc}")
         return out, last_state
 
     def selective_state_update(self, state, x, dt, A, B, C, D=None, z=None, dt_bias=None,
-                               dt_softplus=True):
+                               dt_softplus=True, zoh=False):
         """Return (new_state, out) as float64 arrays; the input state is not modified.
+        ``zoh`` selects the zero-order-hold input term, as in ``selective_scan``.
 
         state: (batch, dim, N); x, dt, z: (batch, dim); B, C: (batch, N);
         A: (dim, N); D, dt_bias: (dim,).
@@ -125,10 +135,10 @@ class Oracle:
         assert z is None or z.shape == x.shape
         new_state = np.empty_like(state)
         out = np.empty_like(x)
-        rc = self._lib.oracle_selective_state_update_f64(
+        rc = self._lib.oracle_selective_state_update_ex_f64(
             batch, dim, dstate, _ptr(state), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C),
-            _ptr(D), _ptr(z), _ptr(dt_bias), int(bool(dt_softplus)), _ptr(new_state),
-            _ptr(out))
+            _ptr(D), _ptr(z), _ptr(dt_bias), int(bool(dt_softplus)), int(bool(zoh)),
+            _ptr(new_state), _ptr(out))
         if rc != 0:
             raise ValueError(f"oracle_selective_state_update_f64 returned {rc}")
         return new_state, out

@@ -15,6 +15,12 @@
  *   y_t       = sum_n C_t,n * h_t,n + D_d * u_t
  *   out_t     = y_t * silu(z_t)              (when z is given, else y_t)
  *
+ * Two options (the *_ex entry points; the plain ones are Euler, zero start):
+ *  - zero-order hold: the input term uses the exact discretisation
+ *    Bbar = (Delta A)^-1 (exp(Delta A) - I) Delta B, which for the diagonal A
+ *    is expm1(Delta A_d,n) / A_d,n * B_t,n (Delta * B_t,n when A_d,n = 0);
+ *  - an initial state h_{-1} given per (b, d, n) instead of zero.
+ *
  * Sources (page title, section):
  *  - "超越注意力：探索Mamba与状态空间模型" (ai-lab.club), section
  *    "状态空间模型基础": the discretised recurrence h_t = Abar h_{t-1} + Bbar x_t,
@@ -23,8 +29,9 @@
  *    B_t and C_t depend on the token.  Here the projection outputs are inputs
  *    (delta, B, C); the bias b is delta_bias.
  *  - same page, section "代码实现概览": the simplified forward uses the Euler
- *    input matrix Bbar = Delta * B and starts from a zero state.  This oracle
- *    follows that reading (the page's zero-order-hold Bbar is not used).
+ *    input matrix Bbar = Delta * B and starts from a zero state.  That is the
+ *    default here; the section "状态空间模型基础" zero-order-hold Bbar and a
+ *    given start state are the options above.
  *  - "Mamba 与状态空间模型" (world.lapla.si), section "由词元决定": the amount
  *    of old state kept is exp(Delta * A).
  *  - The output gate y * silu(z) is the Mamba block's multiplicative gate; no
@@ -36,11 +43,12 @@
  *
  * Layouts (all row-major, contiguous):
  *   scan:   u, delta, z, out (batch, dim, seqlen); B, C (batch, dstate, seqlen);
- *           A (dim, dstate); D, delta_bias (dim); last_state (batch, dim, dstate)
+ *           A (dim, dstate); D, delta_bias (dim); initial_state and
+ *           last_state (batch, dim, dstate)
  *   update: state (batch, dim, dstate) read and returned in new_state;
  *           x, dt, z, out (batch, dim); B, C (batch, dstate); A (dim, dstate);
  *           D, dt_bias (dim)
- * Optional pointers (D, z, bias, last_state) may be NULL.
+ * Optional pointers (D, z, bias, initial_state, last_state) may be NULL.
  * Return value: 0 on success, -1 on a bad size.
  */
 #include <math.h>
@@ -67,6 +75,16 @@ static double oracle_silu(double z)
     return z / (1.0 + exp(-z));
 }
 
+/* Zero-order-hold input gain of one diagonal entry a of A:
+ * (Delta a)^-1 (exp(Delta a) - 1) Delta = expm1(Delta a) / a, and Delta in the
+ * limit a = 0.  expm1 keeps the digits that exp(Delta a) - 1 would cancel. */
+static double oracle_zoh_gain(double dt, double a)
+{
+    if (a == 0.0)
+        return dt;
+    return expm1(dt * a) / a;
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP
@@ -76,11 +94,12 @@ int oracle_num_threads(void)
 #endif
 }
 
-int oracle_selective_scan_f64(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
-                              const double *u, const double *delta, const double *A,
-                              const double *B, const double *C, const double *D,
-                              const double *z, const double *delta_bias, int softplus,
-                              double *out, double *last_state)
+int oracle_selective_scan_ex_f64(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
+                                 const double *u, const double *delta, const double *A,
+                                 const double *B, const double *C, const double *D,
+                                 const double *z, const double *delta_bias, int softplus,
+                                 int zoh, const double *initial_state, double *out,
+                                 double *last_state)
 {
     if (batch < 0 || dim < 0 || seqlen < 0 || dstate < 1 || dstate > ORACLE_MAX_DSTATE)
         return -1;
@@ -92,7 +111,7 @@ int oracle_selective_scan_f64(int64_t batch, int64_t dim, int64_t dstate, int64_
         int64_t d = chain % dim;
         double h[ORACLE_MAX_DSTATE];
         for (int64_t n = 0; n < dstate; ++n)
-            h[n] = 0.0;
+            h[n] = initial_state ? initial_state[(b * dim + d) * dstate + n] : 0.0;
 
         const double *u_row = u + (b * dim + d) * seqlen;
         const double *delta_row = delta + (b * dim + d) * seqlen;
@@ -109,10 +128,12 @@ int oracle_selective_scan_f64(int64_t batch, int64_t dim, int64_t dstate, int64_
 
             double y = 0.0;
             for (int64_t n = 0; n < dstate; ++n) {
-                double a_bar = exp(dt * A[d * dstate + n]);
+                double a_dn = A[d * dstate + n];
+                double a_bar = exp(dt * a_dn);
+                double gain = zoh ? oracle_zoh_gain(dt, a_dn) : dt;
                 double b_tn = B[(b * dstate + n) * seqlen + t];
                 double c_tn = C[(b * dstate + n) * seqlen + t];
-                h[n] = a_bar * h[n] + dt * b_tn * x;
+                h[n] = a_bar * h[n] + gain * b_tn * x;
                 y += c_tn * h[n];
             }
             if (D)
@@ -128,11 +149,21 @@ int oracle_selective_scan_f64(int64_t batch, int64_t dim, int64_t dstate, int64_
     return 0;
 }
 
-int oracle_selective_state_update_f64(int64_t batch, int64_t dim, int64_t dstate,
-                                      const double *state, const double *x, const double *dt,
-                                      const double *A, const double *B, const double *C,
-                                      const double *D, const double *z, const double *dt_bias,
-                                      int dt_softplus, double *new_state, double *out)
+int oracle_selective_scan_f64(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
+                              const double *u, const double *delta, const double *A,
+                              const double *B, const double *C, const double *D,
+                              const double *z, const double *delta_bias, int softplus,
+                              double *out, double *last_state)
+{
+    return oracle_selective_scan_ex_f64(batch, dim, dstate, seqlen, u, delta, A, B, C, D, z,
+                                        delta_bias, softplus, 0, NULL, out, last_state);
+}
+
+int oracle_selective_state_update_ex_f64(int64_t batch, int64_t dim, int64_t dstate,
+                                         const double *state, const double *x, const double *dt,
+                                         const double *A, const double *B, const double *C,
+                                         const double *D, const double *z, const double *dt_bias,
+                                         int dt_softplus, int zoh, double *new_state, double *out)
 {
     if (batch < 0 || dim < 0 || dstate < 1 || dstate > ORACLE_MAX_DSTATE)
         return -1;
@@ -151,8 +182,10 @@ int oracle_selective_state_update_f64(int64_t batch, int64_t dim, int64_t dstate
 
         double y = 0.0;
         for (int64_t n = 0; n < dstate; ++n) {
-            double a_bar = exp(delta * A[d * dstate + n]);
-            double h = a_bar * state[chain * dstate + n] + delta * B[b * dstate + n] * xv;
+            double a_dn = A[d * dstate + n];
+            double a_bar = exp(delta * a_dn);
+            double gain = zoh ? oracle_zoh_gain(delta, a_dn) : delta;
+            double h = a_bar * state[chain * dstate + n] + gain * B[b * dstate + n] * xv;
             new_state[chain * dstate + n] = h;
             y += C[b * dstate + n] * h;
         }
@@ -163,4 +196,14 @@ int oracle_selective_state_update_f64(int64_t batch, int64_t dim, int64_t dstate
         out[chain] = y;
     }
     return 0;
+}
+
+int oracle_selective_state_update_f64(int64_t batch, int64_t dim, int64_t dstate,
+                                      const double *state, const double *x, const double *dt,
+                                      const double *A, const double *B, const double *C,
+                                      const double *D, const double *z, const double *dt_bias,
+                                      int dt_softplus, double *new_state, double *out)
+{
+    return oracle_selective_state_update_ex_f64(batch, dim, dstate, state, x, dt, A, B, C, D, z,
+                                                dt_bias, dt_softplus, 0, new_state, out);
 }

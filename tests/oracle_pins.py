@@ -15,6 +15,10 @@ Sources (page title, section):
   - same page, 由词元决定: large Delta resets the state to the current input,
     small Delta holds it; with a one-number state the update is the gate
     h <- (1 - g) h + g x (Theorem 1).
+  - "超越注意力：探索Mamba与状态空间模型", 状态空间模型基础: the zero-order-hold
+    input matrix Bbar = (Delta A)^-1 (exp(Delta A) - I) Delta B.  Under it the
+    Theorem-1 gate holds with B = 1 and no rescaling, and a constant input has
+    the fixed point h* = -B u / A for every Delta.
 """
 from __future__ import annotations
 
@@ -302,6 +306,167 @@ def pin_update_limits(o):
     _close(out, np.einsum("bdn,bn->bd", state, C) + D[None, :] * x, 1e-13, "update hold: out")
 
 
+def pin_zoh_gated_rnn_exact(o):
+    """Zero-order hold, N=1, A=-1, B=C=1, softplus on: Bbar = 1 - exp(-Delta) = g with
+    g = sigmoid(delta + bias), so the scan is exactly h_t = (1-g_t) h_{t-1} + g_t x_t."""
+    rng = np.random.default_rng(31)
+    batch, L = 2, 64
+    s_delta = rng.standard_normal((batch, 1, L)) * 2.0
+    bias = np.array([0.3])
+    g = 1.0 / (1.0 + np.exp(-(s_delta + bias[None, :, None])))
+    x = rng.standard_normal((batch, 1, L))
+    ones = np.ones((batch, 1, L))
+    out, last = o.selective_scan(x, s_delta, np.array([[-1.0]]), ones, ones, delta_bias=bias,
+                                 softplus=True, zoh=True)
+    want = np.zeros_like(x)
+    for b in range(batch):
+        h = 0.0
+        for t in range(L):
+            h = (1.0 - g[b, 0, t]) * h + g[b, 0, t] * x[b, 0, t]
+            want[b, 0, t] = h
+    _close(out, want, 1e-12, "zero-order hold gate (Theorem 1)")
+    _close(last[:, :, 0], want[:, :, -1], 1e-12, "zero-order hold gate: last state")
+
+
+def pin_zoh_fixed_point(o):
+    """Zero-order hold with u and B constant in time: h* = -B u / A is a fixed point for
+    any Delta sequence, so starting there the state never moves and y_t = C_t h* + D u."""
+    rng = np.random.default_rng(32)
+    batch, dim, N, L = 2, 3, 4, 40
+    A = -rng.uniform(0.2, 2.0, (dim, N))
+    ubd = rng.standard_normal((batch, dim))
+    Bbn = rng.standard_normal((batch, N))
+    u = np.broadcast_to(ubd[:, :, None], (batch, dim, L)).copy()
+    B = np.broadcast_to(Bbn[:, :, None], (batch, N, L)).copy()
+    C = rng.standard_normal((batch, N, L))
+    D = rng.standard_normal(dim)
+    delta = rng.uniform(0.01, 2.0, (batch, dim, L))
+    h_star = -Bbn[:, None, :] * ubd[:, :, None] / A[None, :, :]          # (b, d, N)
+    out, last = o.selective_scan(u, delta, A, B, C, D=D, softplus=False, zoh=True,
+                                 initial_state=h_star)
+    want = np.einsum("bdn,bnt->bdt", h_star, C) + D[None, :, None] * u
+    _close(out, want, 1e-12, "zero-order hold fixed point: out")
+    _close(last, h_star, 1e-12, "zero-order hold fixed point: last_state")
+
+
+def pin_zoh_zero_A_is_cumulative_sum(o):
+    """Zero-order hold at A = 0: the gain's limit is Delta, so h_t = sum_s Delta_s B_s u_s."""
+    p = _random_problem(33, seqlen=29)
+    A = np.zeros_like(p["A"])
+    out, last = o.selective_scan(p["u"], p["delta"], A, p["B"], p["C"], D=p["D"],
+                                 delta_bias=p["delta_bias"], softplus=False, zoh=True)
+    Delta = p["delta"] + p["delta_bias"][None, :, None]
+    h = np.cumsum(Delta[:, :, None, :] * p["B"][:, None, :, :] * p["u"][:, :, None, :], axis=-1)
+    want = np.einsum("bdnt,bnt->bdt", h, p["C"]) + p["D"][None, :, None] * p["u"]
+    _close(out, want, 1e-12, "zero-order hold, A = 0: out")
+    _close(last, h[..., -1], 1e-12, "zero-order hold, A = 0: last_state")
+
+
+def pin_zoh_unrolled_sum(o):
+    """Zero-order hold, brute force: y_t = sum_{s<=t} C_t (prod_{s<r<=t} Abar_r)
+    (Abar_s - 1) / A B_s u_s + D u_t."""
+    p = _random_problem(34, seqlen=24)
+    out, last = o.selective_scan(p["u"], p["delta"], p["A"], p["B"], p["C"], D=p["D"],
+                                 delta_bias=p["delta_bias"], softplus=False, zoh=True)
+    u, A, B, C, D = p["u"], p["A"], p["B"], p["C"], p["D"]
+    Delta = p["delta"] + p["delta_bias"][None, :, None]
+    batch, dim, L = u.shape
+    want = np.zeros_like(u)
+    want_last = np.zeros((batch, dim, A.shape[1]))
+    for b in range(batch):
+        for d in range(dim):
+            abar = np.exp(Delta[b, d][:, None] * A[d][None, :])        # (L, N)
+            bbar = (abar - 1.0) / A[d][None, :]                          # (L, N) per unit B
+            for t in range(L):
+                acc = 0.0
+                for s in range(t + 1):
+                    decay = np.prod(abar[s + 1:t + 1], axis=0)
+                    acc += np.sum(C[b, :, t] * decay * bbar[s] * B[b, :, s]) * u[b, d, s]
+                want[b, d, t] = acc + D[d] * u[b, d, t]
+            for s in range(L):
+                want_last[b, d] += np.prod(abar[s + 1:L], axis=0) * bbar[s] * B[b, :, s] * u[b, d, s]
+    _close(out, want, 1e-11, "zero-order hold unrolled sum: out")
+    _close(last, want_last, 1e-11, "zero-order hold unrolled sum: last_state")
+
+
+def pin_initial_state_free_decay(o):
+    """u = 0 leaves only the start state: h_t,n = exp(A_n S_t) h0_n with S_t the running
+    sum of Delta = softplus(delta + bias), so y_t = sum_n C_t,n exp(A_n S_t) h0_n."""
+    rng = np.random.default_rng(35)
+    batch, dim, N, L = 2, 3, 4, 30
+    A = -rng.uniform(0.2, 2.0, (dim, N))
+    h0 = rng.standard_normal((batch, dim, N))
+    delta = rng.standard_normal((batch, dim, L))
+    bias = rng.uniform(-1.0, 0.0, dim)
+    C = rng.standard_normal((batch, N, L))
+    B = rng.standard_normal((batch, N, L))
+    D = rng.standard_normal(dim)
+    u = np.zeros((batch, dim, L))
+    S = np.cumsum(np.logaddexp(0.0, delta + bias[None, :, None]), axis=-1)   # (b, d, L)
+    h = np.exp(A[None, :, :, None] * S[:, :, None, :]) * h0[..., None]        # (b, d, N, L)
+    want = np.einsum("bdnt,bnt->bdt", h, C)
+    for zoh in (False, True):
+        out, last = o.selective_scan(u, delta, A, B, C, D=D, delta_bias=bias, softplus=True,
+                                     zoh=zoh, initial_state=h0)
+        _close(out, want, 1e-12, f"free decay from the start state (zoh={zoh}): out")
+        _close(last, h[..., -1], 1e-12, f"free decay from the start state (zoh={zoh}): last")
+
+
+def pin_initial_state_split(o):
+    """A scan over L steps equals a scan over the first L1 steps followed by a scan over
+    the rest that starts from the first part's last_state (both discretisations)."""
+    p = _random_problem(36, seqlen=37)
+    rng = np.random.default_rng(37)
+    h0 = rng.standard_normal((2, 3, 4))
+    z = rng.standard_normal(p["u"].shape)
+    L1 = 15
+    for zoh in (False, True):
+        kw = dict(D=p["D"], delta_bias=p["delta_bias"], softplus=True, zoh=zoh)
+        out, last = o.selective_scan(p["u"], p["delta"], p["A"], p["B"], p["C"], z=z,
+                                     initial_state=h0, **kw)
+        part = lambda a, sl: a[:, :, sl]
+        o1, l1 = o.selective_scan(part(p["u"], slice(0, L1)), part(p["delta"], slice(0, L1)),
+                                  p["A"], part(p["B"], slice(0, L1)), part(p["C"], slice(0, L1)),
+                                  z=part(z, slice(0, L1)), initial_state=h0, **kw)
+        o2, l2 = o.selective_scan(part(p["u"], slice(L1, None)), part(p["delta"], slice(L1, None)),
+                                  p["A"], part(p["B"], slice(L1, None)),
+                                  part(p["C"], slice(L1, None)), z=part(z, slice(L1, None)),
+                                  initial_state=l1, **kw)
+        _close(np.concatenate([o1, o2], axis=-1), out, 1e-13, f"split scan (zoh={zoh}): out")
+        _close(l2, last, 1e-13, f"split scan (zoh={zoh}): last_state")
+
+
+def pin_update_zoh(o):
+    """Update with the zero-order hold: the Theorem-1 gate for N=1, A=-1, B=C=1, and
+    T updates from a start state reproduce the zero-order-hold scan from that state."""
+    rng = np.random.default_rng(38)
+    batch, dim = 2, 5
+    state = rng.standard_normal((batch, dim, 1))
+    x = rng.standard_normal((batch, dim))
+    dt = rng.standard_normal((batch, dim))
+    bias = rng.uniform(-1.0, 1.0, dim)
+    g = 1.0 / (1.0 + np.exp(-(dt + bias[None, :])))
+    new, out = o.selective_state_update(state, x, dt, -np.ones((dim, 1)), np.ones((batch, 1)),
+                                        np.ones((batch, 1)), dt_bias=bias, dt_softplus=True,
+                                        zoh=True)
+    gate = (1.0 - g) * state[:, :, 0] + g * x
+    _close(new[:, :, 0], gate, 1e-13, "update zero-order hold gate: state")
+    _close(out, gate, 1e-13, "update zero-order hold gate: out")
+    p = _decode_problem(39)
+    h0 = rng.standard_normal((2, 3, 4))
+    out_scan, last = o.selective_scan(p["x"], p["dt"], p["A"], p["B"], p["C"], D=p["D"],
+                                      z=p["z"], delta_bias=p["bias"], softplus=True, zoh=True,
+                                      initial_state=h0)
+    st = h0.copy()
+    outs = np.zeros_like(p["x"])
+    for t in range(p["x"].shape[2]):
+        st, outs[:, :, t] = o.selective_state_update(
+            st, p["x"][:, :, t], p["dt"][:, :, t], p["A"], p["B"][:, :, t], p["C"][:, :, t],
+            D=p["D"], z=p["z"][:, :, t], dt_bias=p["bias"], dt_softplus=True, zoh=True)
+    _close(outs, out_scan, 1e-13, "zero-order-hold updates = scan: out")
+    _close(st, last, 1e-13, "zero-order-hold updates = scan: state")
+
+
 PINS = {
     "unrolled_sum": pin_unrolled_sum,
     "gate_closed_values": pin_gate_closed_values,
@@ -315,4 +480,11 @@ PINS = {
     "update_steps_equal_scan": pin_update_steps_equal_scan,
     "update_continues_scan": pin_update_continues_scan,
     "update_limits": pin_update_limits,
+    "zoh_gated_rnn_exact": pin_zoh_gated_rnn_exact,
+    "zoh_fixed_point": pin_zoh_fixed_point,
+    "zoh_zero_A_is_cumulative_sum": pin_zoh_zero_A_is_cumulative_sum,
+    "zoh_unrolled_sum": pin_zoh_unrolled_sum,
+    "initial_state_free_decay": pin_initial_state_free_decay,
+    "initial_state_split": pin_initial_state_split,
+    "update_zoh": pin_update_zoh,
 }

@@ -16,7 +16,7 @@ from oracle_pins import PINS
 # (name, exact snippet in ssm_oracle.c, replacement)
 MUTANTS = [
     ("drop_D_term", "y += D[d] * x;", "y += 0.0 * x;"),
-    ("exp_sign_flipped", "exp(dt * A[d * dstate + n])", "exp(-dt * A[d * dstate + n])"),
+    ("exp_sign_flipped", "double a_bar = exp(dt * a_dn);", "double a_bar = exp(-dt * a_dn);"),
     ("B_read_from_C", "double b_tn = B[(b * dstate + n) * seqlen + t];",
      "double b_tn = C[(b * dstate + n) * seqlen + t];"),
     ("softplus_skipped", "if (softplus)\n                dt = oracle_softplus(dt);", ""),
@@ -30,16 +30,19 @@ MUTANTS = [
      "                dt += delta_bias[d];"),
     ("gate_sign_flipped", "return z / (1.0 + exp(-z));", "return z / (1.0 + exp(z));"),
     ("gate_is_sigmoid", "return z / (1.0 + exp(-z));", "return 1.0 / (1.0 + exp(-z));"),
-    ("bbar_without_delta", "h[n] = a_bar * h[n] + dt * b_tn * x;", "h[n] = a_bar * h[n] + b_tn * x;"),
-    ("state_not_decayed", "h[n] = a_bar * h[n] + dt * b_tn * x;", "h[n] = h[n] + dt * b_tn * x;"),
+    ("bbar_without_delta", "h[n] = a_bar * h[n] + gain * b_tn * x;",
+     "h[n] = a_bar * h[n] + b_tn * x;"),
+    ("state_not_decayed", "h[n] = a_bar * h[n] + gain * b_tn * x;",
+     "h[n] = h[n] + gain * b_tn * x;"),
     ("readout_before_update",
-     "h[n] = a_bar * h[n] + dt * b_tn * x;\n                y += c_tn * h[n];",
-     "y += c_tn * h[n];\n                h[n] = a_bar * h[n] + dt * b_tn * x;"),
+     "h[n] = a_bar * h[n] + gain * b_tn * x;\n                y += c_tn * h[n];",
+     "y += c_tn * h[n];\n                h[n] = a_bar * h[n] + gain * b_tn * x;"),
     ("B_time_shifted", "double b_tn = B[(b * dstate + n) * seqlen + t];",
      "double b_tn = B[(b * dstate + n) * seqlen + (t > 0 ? t - 1 : t)];"),
     ("C_batch_ignored", "double c_tn = C[(b * dstate + n) * seqlen + t];",
      "double c_tn = C[(0 * dstate + n) * seqlen + t];"),
-    ("A_transposed", "exp(dt * A[d * dstate + n])", "exp(dt * A[n * dim + d])"),
+    ("A_transposed", "double a_dn = A[d * dstate + n];\n                double a_bar",
+     "double a_dn = A[n * dim + d];\n                double a_bar"),
     ("u_time_shifted", "double x = u_row[t];", "double x = u_row[t > 0 ? t - 1 : 0];"),
     ("last_state_zeroed", "last_state[(b * dim + d) * dstate + n] = h[n];",
      "last_state[(b * dim + d) * dstate + n] = 0.0 * h[n];"),
@@ -47,10 +50,23 @@ MUTANTS = [
      "double h = state[chain * dstate + n]"),
     ("update_bias_dropped", "delta += dt_bias[d];", "delta += 0.0;"),
     ("update_gate_dropped", "y *= oracle_silu(z[chain]);", "y *= 1.0;"),
-    ("update_B_batch_ignored", "delta * B[b * dstate + n] * xv", "delta * B[n] * xv"),
+    ("update_B_batch_ignored", "gain * B[b * dstate + n] * xv", "gain * B[n] * xv"),
     ("update_C_from_B", "y += C[b * dstate + n] * h;", "y += B[b * dstate + n] * h;"),
     ("update_D_dropped", "y += D[d] * xv;", "y += 0.0 * xv;"),
     ("update_softplus_skipped", "if (dt_softplus)\n            delta = oracle_softplus(delta);", ""),
+    # zero-order hold and the start state
+    ("zoh_gain_sign_flipped", "return expm1(dt * a) / a;", "return expm1(-dt * a) / a;"),
+    ("zoh_gain_not_divided", "return expm1(dt * a) / a;", "return expm1(dt * a);"),
+    ("zoh_gain_limit_dropped", "        return dt;\n    return expm1", "        return 0.0;\n    return expm1"),
+    ("zoh_gain_uses_exp", "return expm1(dt * a) / a;", "return exp(dt * a) / a;"),
+    ("zoh_ignored_in_scan", "double gain = zoh ? oracle_zoh_gain(dt, a_dn) : dt;",
+     "double gain = dt;"),
+    ("zoh_ignored_in_update", "double gain = zoh ? oracle_zoh_gain(delta, a_dn) : delta;",
+     "double gain = delta;"),
+    ("initial_state_ignored",
+     "h[n] = initial_state ? initial_state[(b * dim + d) * dstate + n] : 0.0;", "h[n] = 0.0;"),
+    ("initial_state_transposed", "initial_state[(b * dim + d) * dstate + n]",
+     "initial_state[(d * batch + b) * dstate + n]"),
 ]
 
 
