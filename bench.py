@@ -43,6 +43,7 @@ import torch  # noqa: E402
 METRIC = ("selective-scan Gelem/s (B·D·L) and % of roofline; "
           "decode-step µs at batch 128")
 SCAN_WORKLOAD = "mamba_2p8b_layer"
+SCAN_VARIANTS = ("euler", "zoh", "start_state")
 PROFILES = ROOT / "profiles"
 HBM_FALLBACK_GBS = 6650.0
 SM_MAX_MHZ_FALLBACK = 1965.0
@@ -172,13 +173,15 @@ class Workload:
     """Device-resident inputs and outputs of one step, and the calls that run it."""
 
     def __init__(self, rank: int, scan_batch: int | None = None, decode_layers: int | None = None,
-                 only: str | None = None):
+                 only: str | None = None, scan_workload: str = SCAN_WORKLOAD,
+                 scan_variant: str = "euler"):
         from selective_state_space_55_b200 import inputs as I
         from selective_state_space_55_b200 import ops
 
         self.ops = ops
         self.only = only
-        self.cfg = I.SCAN_CONFIGS[SCAN_WORKLOAD]
+        self.variant = scan_variant
+        self.cfg = I.SCAN_CONFIGS[scan_workload]
         if scan_batch:
             self.cfg = self.cfg.resized(batch=scan_batch)
         self.dcfg = I.DECODE_CONFIG
@@ -189,6 +192,11 @@ class Workload:
         self.x = I.make_scan_inputs(c, "cuda", seed=rank_seed(rank))
         self.out = torch.empty_like(self.x["u"])
         self.last = torch.empty((c.batch, c.dim, c.dstate), dtype=torch.float32, device="cuda")
+        self.h0 = None
+        if scan_variant == "start_state":
+            g = torch.Generator(device="cuda")
+            g.manual_seed(rank_seed(rank) + 7)
+            self.h0 = torch.randn((c.batch, c.dim, c.dstate), generator=g, device="cuda")
         ws = ops.scan_workspace_bytes(c.batch, c.dim, c.dstate, c.seqlen, c.io_dtype, c.bc_dtype)
         self.ws = torch.empty(ws, dtype=torch.uint8, device="cuda") if ws else None
         self.plan = ops.scan_plan(c.batch, c.dim, c.dstate, c.seqlen, c.io_dtype, c.bc_dtype,
@@ -200,13 +208,16 @@ class Workload:
         self.douts = [torch.empty_like(t["x"]) for t in self.toks]
         self.graph = None
 
+    def scan_kwargs(self) -> dict:
+        return {"zoh": self.variant == "zoh", "initial_state": self.h0}
+
     def scan(self):
         if self.only == "decode":
             return
         x = self.x
         self.ops.selective_scan_fwd(x["u"], x["delta"], x["A"], x["B"], x["C"], D=x["D"], z=x["z"],
                                     delta_bias=x["delta_bias"], softplus=True, out=self.out,
-                                    last_state=self.last, workspace=self.ws)
+                                    last_state=self.last, workspace=self.ws, **self.scan_kwargs())
 
     def decode_layers(self):
         for lay, tok, out in zip(self.layers, self.toks, self.douts):
@@ -247,12 +258,19 @@ def run_e2e(w: Workload, steps: int, warmup: int) -> dict:
         host[k].copy_(x[k])
     out_h = torch.empty(w.out.shape, dtype=w.out.dtype, pin_memory=True)
     last_h = torch.empty(w.last.shape, dtype=w.last.dtype, pin_memory=True)
+    h0_h = None
+    if w.h0 is not None:
+        h0_h = torch.empty(w.h0.shape, dtype=w.h0.dtype, pin_memory=True)
+        h0_h.copy_(w.h0)
     h2d = sum(host[k].numel() * host[k].element_size() for k in names)
+    h2d += 0 if h0_h is None else h0_h.numel() * h0_h.element_size()
     d2h = out_h.numel() * out_h.element_size() + last_h.numel() * last_h.element_size()
 
     def step():
         for k in names:
             x[k].copy_(host[k], non_blocking=True)
+        if h0_h is not None:
+            w.h0.copy_(h0_h, non_blocking=True)
         w.scan()
         out_h.copy_(w.out, non_blocking=True)
         last_h.copy_(w.last, non_blocking=True)
@@ -282,13 +300,15 @@ def cpu_baseline(w: Workload, target_s: float) -> dict:
     for b in range(c.batch):
         sl = lambda t: None if t is None else t[b:b + 1].cpu()  # noqa: E731
         rows.append((sl(x["u"]), sl(x["delta"]), sl(x["z"]), x["B"][b:b + 1].cpu(),
-                     x["C"][b:b + 1].cpu()))
+                     x["C"][b:b + 1].cpu(), sl(w.h0)))
     A, D, bias = x["A"].cpu(), x["D"].cpu(), x["delta_bias"].cpu()
+    zoh = w.variant == "zoh"
     done, t_total, passes = 0, 0.0, 0
     while True:                      # whole passes over the workload
-        for u, delta, z, B, C in rows:
+        for u, delta, z, B, C, h0 in rows:
             t0 = time.perf_counter()
-            ref.selective_scan(u, delta, A, B, C, D=D, z=z, delta_bias=bias, softplus=True)
+            ref.selective_scan(u, delta, A, B, C, D=D, z=z, delta_bias=bias, softplus=True,
+                               zoh=zoh, initial_state=h0)
             t_total += time.perf_counter() - t0
             done += c.dim * c.seqlen
         passes += 1
@@ -296,7 +316,7 @@ def cpu_baseline(w: Workload, target_s: float) -> dict:
             break
     return {"value": done / t_total / 1e9, "unit": "Gelem/s", "cores": ref.num_threads(),
             "kind": "oracle",
-            "sample": f"{passes} full pass(es) over {SCAN_WORKLOAD} ({c.batch} batch rows x "
+            "sample": f"{passes} full pass(es) over {c.name} ({c.batch} batch rows x "
                       f"{c.dim} channels x L={c.seqlen}; {done} elements) in {t_total:.1f} s "
                       "of oracle time"}
 
@@ -343,8 +363,10 @@ def bench_ours(args, rank, world, local):
         cuda_build.build()
     barrier()
     torch.cuda.set_device(local)
-    partial = args.only is not None or args.scan_batch or args.decode_layers
-    w = Workload(rank, args.scan_batch, args.decode_layers, args.only)
+    partial = (args.only is not None or args.scan_batch or args.decode_layers
+               or args.scan_workload != SCAN_WORKLOAD or args.scan_variant != "euler")
+    w = Workload(rank, args.scan_batch, args.decode_layers, args.only, args.scan_workload,
+                 args.scan_variant)
     c, d = w.cfg, w.dcfg
     w.capture_decode()
     for _ in range(args.warmup):
@@ -384,16 +406,18 @@ def bench_ours(args, rank, world, local):
 
     peaks = measured_peaks()
     clocks = sampler.summary(t_wall0, t_wall1)
-    mufu = R.scan_mufu_per_element(c.dstate, has_z=True, softplus=True)
+    mufu = R.scan_mufu_per_element(c.dstate, has_z=True, softplus=True,
+                                   zoh=args.scan_variant == "zoh")
     peak_elems = R.mufu_peak_elements_per_s(torch.cuda.get_device_properties(local).multi_processor_count,
                                             peaks["sm_max_mhz"], mufu) / 1e9
     achieved = elems / (scan_launch_ms * 1e-3) / 1e9               # per launch, this rank
-    scan_bytes = R.scan_bytes(c.batch, c.dim, c.dstate, c.seqlen, 2, 2, True, True)
+    scan_bytes = R.scan_bytes(c.batch, c.dim, c.dstate, c.seqlen, 2, 2, True, True,
+                              start_state=w.h0 is not None)
     upd_bytes = R.update_bytes(d.batch, d.dim, d.dstate, 2, 2, True)
     decode_gbs = upd_bytes * d.layers / (decode_ms / K * 1e-3) / 1e9
     digest = sources_digest()
     scan_roof = {
-        "bound": "alu", "pipe": "MUFU (16 ops/clk/SM; 20 per element)",
+        "bound": "alu", "pipe": f"MUFU (16 ops/clk/SM; {mufu} per element)",
         "kernel": "selective_scan_fwd_kernel",
         "achieved": round(achieved, 2), "peak": round(peak_elems, 2), "unit": "Gelem/s",
         "frac": round(achieved / peak_elems, 4),
@@ -445,8 +469,10 @@ def bench_ours(args, rank, world, local):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic (seeded; shapes and distributions of the pages' workloads)",
             "config": {
-                "workload": f"{SCAN_WORKLOAD} scan ({c.batch}x{c.dim}, N={c.dstate}, L={c.seqlen}, "
-                            "bf16 in/out, fp32 state, last_state) + decode_b128 token step "
+                "workload": f"{c.name} scan ({c.batch}x{c.dim}, N={c.dstate}, L={c.seqlen}, "
+                            "bf16 in/out, fp32 state, last_state"
+                            + ("" if w.variant == "euler" else f"; variant {w.variant}")
+                            + ") + decode_b128 token step "
                             f"({d.layers} layers, batch {d.batch}, d_inner {d.dim}, N {d.dstate})",
                 "io_dtype": "bf16", "state_dtype": "f32", "global_batch": world * c.batch,
                 "seq_len": c.seqlen, "parallelism": f"replicas{world}" if world > 1 else "single",
@@ -466,6 +492,8 @@ def bench_ours(args, rank, world, local):
         if partial:
             line["partial_case"] = {"only": args.only, "scan_batch": args.scan_batch,
                                     "decode_layers": args.decode_layers,
+                                    "scan_workload": args.scan_workload,
+                                    "scan_variant": args.scan_variant,
                                     "note": "profiling case, not the benchmark workload"}
         print(json.dumps(line), flush=True)
 
@@ -535,6 +563,11 @@ def main():
                     help="profiling case: smaller scan batch")
     ap.add_argument("--decode-layers", type=int, default=None,
                     help="profiling case: fewer decode layers")
+    ap.add_argument("--scan-workload", default=SCAN_WORKLOAD,
+                    choices=["mamba_1p4b_layer", "mamba_2p8b_layer", "long_dna_1m"],
+                    help="measurement case: another scan workload")
+    ap.add_argument("--scan-variant", default="euler", choices=SCAN_VARIANTS,
+                    help="measurement case: zero-order-hold input term, or a start state")
     args = ap.parse_args()
     if args.warmup < 3:
         log("[bench] warm-up raised to 3 steps (minimum)")

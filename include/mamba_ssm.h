@@ -14,11 +14,17 @@
  *   y_t      = sum_n C_t,n * h_t,n + D_d * u_t
  *   out_t    = y_t * silu(z_t)                                   (z optional)
  *
+ * Options: MAMBA_FLAG_ZOH replaces the Euler input term Delta_t B_t,n u_t by
+ * the zero-order-hold one, expm1(Delta_t A_d,n) / A_d,n * B_t,n * u_t
+ * (Delta_t B_t,n u_t where A_d,n = 0); mamba_selective_scan_fwd_with_state
+ * starts from a given h_{-1} instead of zero.
+ *
  * Sources: "超越注意力：探索Mamba与状态空间模型" (ai-lab.club), section
  * 状态空间模型基础 (zero-order-hold Abar = exp(Delta A), recurrence and
- * readout) and section 选择性状态空间模型 (Delta = softplus(W x + b), B and C
- * per token); its section 代码实现概览 uses the Euler input term
- * Bbar = Delta * B, which this library follows.  "Mamba 与状态空间模型"
+ * readout, and the zero-order-hold Bbar = (Delta A)^-1 (exp(Delta A) - I) Delta B
+ * of MAMBA_FLAG_ZOH) and section 选择性状态空间模型 (Delta = softplus(W x + b),
+ * B and C per token); its section 代码实现概览 uses the Euler input term
+ * Bbar = Delta * B, the default here.  "Mamba 与状态空间模型"
  * (world.lapla.si), section 由词元决定 (exp(Delta A) decides how much old state
  * is kept) and section 在芯片上扫过去 (the scan never writes the full state to
  * HBM).  The silu(z) gate is the Mamba block's output gate (not printed on the
@@ -84,6 +90,11 @@ typedef enum {
  * a predecessor runs out (after ~0.3 s) and the call reports MAMBA_ERR_TIMEOUT
  * through mamba_device_status().  Outputs are then undefined. */
 #define MAMBA_FLAG_TEST_WITHHOLD_HANDOFF 0x4
+/* Scan and update: zero-order-hold input term expm1(Delta A) / A * B * u
+ * instead of the Euler Delta * B * u (Abar = exp(Delta A) either way).  The scan
+ * then runs a kernel instance with 1/A held in registers (fewer resident
+ * warps); results follow the same tolerance as the Euler path. */
+#define MAMBA_FLAG_ZOH 0x8
 
 #define MAMBA_MAX_DSTATE 16
 
@@ -186,6 +197,29 @@ MAMBA_API mamba_status_t mamba_selective_scan_fwd(const void *u, const void *del
                                                   const mamba_dims_t *dims, cudaStream_t stream);
 
 /*
+ * Selective scan forward from a given start state.
+ *
+ * Same as mamba_selective_scan_fwd, except that the recurrence starts from
+ *   initial_state      (batch, dim, dstate) fp32 device buffer = h_{-1}, or NULL
+ *                      for the zero state (then identical to
+ *                      mamba_selective_scan_fwd).
+ * A sequence can thus be scanned in pieces: the last_state of one call is the
+ * initial_state of the next, and the outputs equal those of one call over the
+ * whole sequence up to rounding.  initial_state may be the same buffer as
+ * last_state (it is read before last_state is written); a partial overlap of
+ * the two returns MAMBA_ERR_INVALID_ARG.  With seqlen == 0, last_state (if
+ * given) receives a copy of initial_state (zero if NULL).
+ * Source: the recurrence of "超越注意力：探索Mamba与状态空间模型", section
+ * 状态空间模型基础, from an arbitrary h_{t-1}; "Mamba 与状态空间模型", section
+ * 固定大小的状态 (the fixed-size state carries everything the model keeps).
+ */
+MAMBA_API mamba_status_t mamba_selective_scan_fwd_with_state(
+    const void *u, const void *delta, const float *A, const void *B, const void *C,
+    const float *D, const void *z, const float *delta_bias, int softplus,
+    const float *initial_state, void *out, float *last_state, const mamba_dims_t *dims,
+    cudaStream_t stream);
+
+/*
  * Selective scan forward that allocates nothing and takes no workspace.
  *
  * The paper has no counterpart to this entry point; it is a deployment aid.
@@ -230,6 +264,7 @@ MAMBA_API mamba_status_t mamba_selective_scan_fwd_noalloc(
  *   B, C               (batch, dstate), bc_dtype
  *   D, dt_bias         (dim,) fp32; may be NULL
  *   dims->dt_softplus  nonzero: Delta = softplus(dt + dt_bias)
+ *   dims->flags        MAMBA_FLAG_ZOH: zero-order-hold input term
  * dims->seqlen, num_chunks and workspace are ignored.
  * Paths: for dstate == 16, dim % 8 == 0 and 16-byte aligned buffers the state
  * streams through shared memory by bulk TMA (MAMBA_FLAG_NO_TMA turns that

@@ -89,13 +89,13 @@ cudaError_t ensure_smem_attr(Kernel kernel, int bytes, bool* done_per_device, in
     return e;
 }
 
-template <typename IoT, int kCpl, bool kHasZ, bool kSoftplus>
+template <typename IoT, int kCpl, bool kHasZ, bool kSoftplus, bool kZoh>
 cudaError_t launch_scan(const ScanParams& prm, const CUtensorMap* maps, int64_t want_warps,
                         int dev, int sms, cudaStream_t stream) {
     using Lay = ScanLayout<kCpl>;
     static bool attr_done[kMaxDevices] = {false};
     static int resident[kMaxDevices] = {0};
-    auto kernel = selective_scan_fwd_kernel<IoT, kCpl, kHasZ, kSoftplus>;
+    auto kernel = selective_scan_fwd_kernel<IoT, kCpl, kHasZ, kSoftplus, kZoh>;
     cudaError_t e = ensure_smem_attr(kernel, Lay::kCtaSmem, attr_done, dev);
     if (e != cudaSuccess) return e;
     int per_sm = (dev >= 0 && dev < kMaxDevices) ? resident[dev] : 0;
@@ -114,28 +114,30 @@ cudaError_t launch_scan(const ScanParams& prm, const CUtensorMap* maps, int64_t 
     return cudaGetLastError();
 }
 
-template <typename IoT, int kCpl>
+template <typename IoT, int kCpl, bool kZoh>
 cudaError_t dispatch_scan_cpl(const ScanParams& prm, const CUtensorMap* maps, bool has_z, bool sp,
                               int64_t want_warps, int dev, int sms, cudaStream_t stream) {
     if (has_z)
-        return sp ? launch_scan<IoT, kCpl, true, true>(prm, maps, want_warps, dev, sms, stream)
-                  : launch_scan<IoT, kCpl, true, false>(prm, maps, want_warps, dev, sms, stream);
-    return sp ? launch_scan<IoT, kCpl, false, true>(prm, maps, want_warps, dev, sms, stream)
-              : launch_scan<IoT, kCpl, false, false>(prm, maps, want_warps, dev, sms, stream);
+        return sp ? launch_scan<IoT, kCpl, true, true, kZoh>(prm, maps, want_warps, dev, sms, stream)
+                  : launch_scan<IoT, kCpl, true, false, kZoh>(prm, maps, want_warps, dev, sms, stream);
+    return sp ? launch_scan<IoT, kCpl, false, true, kZoh>(prm, maps, want_warps, dev, sms, stream)
+              : launch_scan<IoT, kCpl, false, false, kZoh>(prm, maps, want_warps, dev, sms, stream);
 }
 
 template <typename IoT>
 cudaError_t dispatch_scan(const ScanParams& prm, const CUtensorMap* maps, int cpl, bool has_z,
-                          bool sp, int64_t want_warps, int dev, int sms, cudaStream_t stream) {
+                          bool sp, bool zoh, int64_t want_warps, int dev, int sms,
+                          cudaStream_t stream) {
     if (cpl != 1) return cudaErrorInvalidValue;
-    return dispatch_scan_cpl<IoT, 1>(prm, maps, has_z, sp, want_warps, dev, sms, stream);
+    return zoh ? dispatch_scan_cpl<IoT, 1, true>(prm, maps, has_z, sp, want_warps, dev, sms, stream)
+               : dispatch_scan_cpl<IoT, 1, false>(prm, maps, has_z, sp, want_warps, dev, sms, stream);
 }
 
-template <typename IoT, typename BcT, bool kHasZ>
+template <typename IoT, typename BcT, bool kHasZ, bool kZoh>
 cudaError_t launch_update_bulk(const UpdateParams& prm, int dev, int sms, cudaStream_t stream) {
     static bool attr_done[kMaxDevices] = {false};
     static int resident[kMaxDevices] = {0};
-    auto kernel = state_update_bulk_kernel<IoT, BcT, kHasZ>;
+    auto kernel = state_update_bulk_kernel<IoT, BcT, kHasZ, kZoh>;
     cudaError_t e = ensure_smem_attr(kernel, kBulkSmemBytes, attr_done, dev);
     if (e != cudaSuccess) return e;
     int per_sm = (dev >= 0 && dev < kMaxDevices) ? resident[dev] : 0;
@@ -162,9 +164,13 @@ cudaError_t launch_update_bulk(const UpdateParams& prm, int dev, int sms, cudaSt
 template <typename IoT, typename BcT>
 cudaError_t dispatch_update_bc(const UpdateParams& prm, bool fast, bool bulk, bool has_z,
                                int dev, int sms, cudaStream_t stream) {
-    if (bulk)
-        return has_z ? launch_update_bulk<IoT, BcT, true>(prm, dev, sms, stream)
-                     : launch_update_bulk<IoT, BcT, false>(prm, dev, sms, stream);
+    if (bulk) {
+        if (prm.zoh)
+            return has_z ? launch_update_bulk<IoT, BcT, true, true>(prm, dev, sms, stream)
+                         : launch_update_bulk<IoT, BcT, false, true>(prm, dev, sms, stream);
+        return has_z ? launch_update_bulk<IoT, BcT, true, false>(prm, dev, sms, stream)
+                     : launch_update_bulk<IoT, BcT, false, false>(prm, dev, sms, stream);
+    }
     if (fast) {
         // x covers channels (kUpdateChainsPerCta per CTA), y covers batch rows.
         const dim3 grid((unsigned)((prm.dim + kUpdateChainsPerCta - 1) / kUpdateChainsPerCta),
@@ -322,16 +328,38 @@ MAMBA_API mamba_status_t mamba_selective_scan_fwd(const void* u, const void* del
                                                   const void* z, const float* delta_bias,
                                                   int softplus, void* out, float* last_state,
                                                   const mamba_dims_t* dims, cudaStream_t stream) {
+    return mamba_selective_scan_fwd_with_state(u, delta, A, B, C, D, z, delta_bias, softplus,
+                                               nullptr, out, last_state, dims, stream);
+}
+
+MAMBA_API mamba_status_t mamba_selective_scan_fwd_with_state(
+    const void* u, const void* delta, const float* A, const void* B, const void* C,
+    const float* D, const void* z, const float* delta_bias, int softplus,
+    const float* initial_state, void* out, float* last_state, const mamba_dims_t* dims,
+    cudaStream_t stream) {
     mamba_status_t st = check_dims(dims, true);
     if (st != MAMBA_OK) return st;
     // Empty problems first: tensors without elements may have null pointers.
     const int64_t chains = dims->batch * dims->dim;
     if (chains == 0) return MAMBA_OK;
+    const size_t state_bytes = (size_t)chains * dims->dstate * sizeof(float);
+    if (initial_state != nullptr && !aligned(initial_state, 4)) return MAMBA_ERR_ALIGN;
+    // The start state may be the last_state buffer itself (in-place
+    // continuation), but must not partly overlap it.
+    if (initial_state != nullptr && last_state != nullptr && initial_state != last_state) {
+        const uintptr_t a = reinterpret_cast<uintptr_t>(initial_state);
+        const uintptr_t b = reinterpret_cast<uintptr_t>(last_state);
+        if (a < b + state_bytes && b < a + state_bytes) return MAMBA_ERR_INVALID_ARG;
+    }
     if (dims->seqlen == 0) {
         if (last_state == nullptr) return MAMBA_OK;
         if (!aligned(last_state, 4)) return MAMBA_ERR_ALIGN;
-        const cudaError_t e = cudaMemsetAsync(last_state, 0,
-                                              (size_t)chains * dims->dstate * sizeof(float), stream);
+        cudaError_t e = cudaSuccess;
+        if (initial_state == nullptr)
+            e = cudaMemsetAsync(last_state, 0, state_bytes, stream);
+        else if (initial_state != last_state)
+            e = cudaMemcpyAsync(last_state, initial_state, state_bytes, cudaMemcpyDeviceToDevice,
+                                stream);
         return e == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
     }
     if (u == nullptr || delta == nullptr || A == nullptr || B == nullptr || C == nullptr ||
@@ -366,6 +394,7 @@ MAMBA_API mamba_status_t mamba_selective_scan_fwd(const void* u, const void* del
     prm.delta_bias = delta_bias;
     prm.out = out;
     prm.last_state = last_state;
+    prm.h0 = initial_state;
     prm.batch = dims->batch;
     prm.dim = dims->dim;
     prm.seqlen = dims->seqlen;
@@ -425,6 +454,7 @@ MAMBA_API mamba_status_t mamba_selective_scan_fwd(const void* u, const void* del
     if (cudaMemsetAsync(ws, 0, lay.zeroed, stream) != cudaSuccess) return MAMBA_ERR_CUDA;
     const bool has_z = z != nullptr;
     const bool sp = softplus != 0;
+    const bool zoh = (dims->flags & MAMBA_FLAG_ZOH) != 0;
     auto run = [&](int mode, unsigned int* counter, int64_t items) -> cudaError_t {
         prm.mode = mode;
         prm.counter = counter;
@@ -432,8 +462,8 @@ MAMBA_API mamba_status_t mamba_selective_scan_fwd(const void* u, const void* del
         if (items == 0) return cudaSuccess;
         return dims->io_dtype == MAMBA_BF16
                    ? dispatch_scan<__nv_bfloat16>(prm, maps, plan.channels_per_lane, has_z, sp,
-                                                  plan.max_warps, dev, sms, stream)
-                   : dispatch_scan<float>(prm, maps, plan.channels_per_lane, has_z, sp,
+                                                  zoh, plan.max_warps, dev, sms, stream)
+                   : dispatch_scan<float>(prm, maps, plan.channels_per_lane, has_z, sp, zoh,
                                           plan.max_warps, dev, sms, stream);
     };
     cudaError_t e;
@@ -482,6 +512,7 @@ MAMBA_API mamba_status_t mamba_selective_state_update(float* state, const void* 
     prm.chains = chains;
     prm.dstate = (int)dims->dstate;
     prm.dt_softplus = dims->dt_softplus != 0;
+    prm.zoh = (dims->flags & MAMBA_FLAG_ZOH) != 0;
     const bool fast = dims->dstate == 16 && aligned(state, 16) && aligned(A, 16) &&
                       aligned(B, 4 * bc_es) && aligned(C, 4 * bc_es);
     // Streaming (bulk TMA) path: every bulk copy needs 16-byte aligned ends.

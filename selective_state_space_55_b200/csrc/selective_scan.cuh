@@ -109,6 +109,7 @@ struct ScanParams {
     int vec_out;             // 16-byte output stores are aligned
     unsigned int flag_poll_limit;   // chained mode: polls (~1 us each) before a wait gives up
     int withhold_handoff;    // test only: segments never publish their state (waits time out)
+    const float* h0;         // (batch, dim, dstate) start state of segment 0, or null (zero)
 };
 
 // Byte offset of (row r, byte x of the row) in a 32-byte-row tile written by
@@ -162,6 +163,7 @@ template <int kCpl>
 struct LaneChains {
     float2 h[kCpl][kNPad / 2];
     float2 a2[kCpl][kNPad / 2];
+    float2 inva[kCpl][kNPad / 2];   // 1 / A_d,n (zero-order hold only)
     float bias[kCpl];
     float Dd[kCpl];
 };
@@ -175,12 +177,18 @@ __device__ __forceinline__ float2 exp2_pair(float2 x) {
 
 // One time step for one lane: advance the kCpl x 16 states, return y per
 // channel (kOut).  kExact selects exp2_near_one_exact for Abar (fp32 path).
-template <int kCpl, bool kOut, bool kExact>
+// kZoh takes the zero-order-hold input term Delta phi(Delta A) B u instead of
+// the Euler term Delta B u; phi = (Abar - 1) / (Delta A) is formed from
+// 1 / Delta (per step) and 1 / A (per channel), or from its series near 0.
+template <int kCpl, bool kOut, bool kExact, bool kZoh>
 __device__ __forceinline__ void scan_step(const float* bc_row, const float (&dt)[kCpl],
                                           const float (&du)[kCpl], LaneChains<kCpl>& lc,
                                           float (&y)[kCpl]) {
     const float4* bc = reinterpret_cast<const float4*>(bc_row);
     float2 ya[kCpl], yb[kCpl];
+    float rdt[kCpl];
+#pragma unroll
+    for (int c = 0; c < kCpl; ++c) rdt[c] = kZoh ? __fdividef(1.0f, dt[c]) : 0.0f;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         const float4 Bq = bc[q];
@@ -192,8 +200,18 @@ __device__ __forceinline__ void scan_step(const float* bc_row, const float (&dt)
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 const int pi = 2 * q + half;
-                const float2 abar = exp2_pair<kExact>(__fmul2_rn(dt2, lc.a2[c][pi]));
-                lc.h[c][pi] = __ffma2_rn(abar, lc.h[c][pi], __fmul2_rn(du2, bq[half]));
+                const float2 x2 = __fmul2_rn(dt2, lc.a2[c][pi]);
+                const float2 abar = exp2_pair<kExact>(x2);
+                float2 in = __fmul2_rn(du2, bq[half]);
+                if (kZoh) {
+                    const float2 big = __fmul2_rn(__fadd2_rn(abar, make_float2(-1.0f, -1.0f)),
+                                                  __fmul2_rn(make_float2(rdt[c], rdt[c]),
+                                                             lc.inva[c][pi]));
+                    const float2 ser = zoh_phi_series2(x2);
+                    in = __fmul2_rn(in, make_float2(fabsf(x2.x) < kZohSmall ? ser.x : big.x,
+                                                    fabsf(x2.y) < kZohSmall ? ser.y : big.y));
+                }
+                lc.h[c][pi] = __ffma2_rn(abar, lc.h[c][pi], in);
             }
         }
         if (kOut) {
@@ -218,10 +236,12 @@ __device__ __forceinline__ void scan_step(const float* bc_row, const float (&dt)
     }
 }
 
-// Process the `nsteps` (<= T) valid time steps of one staged tile.  The
-// 16-byte vectors of u, delta and z stay packed and are unpacked step by
-// step to save registers.
-template <typename IoT, int kCpl, bool kHasZ, bool kSoftplus, bool kOut>
+// Process the `nsteps` (<= T) valid time steps of one staged tile, one
+// 16-byte vector of u, delta and z (V steps) at a time.  Delta and Delta u of
+// all V steps are formed first: their softplus chains are independent of the
+// state, so computing them together lets their latency overlap.  The vectors
+// stay packed and are unpacked element by element to save registers.
+template <typename IoT, int kCpl, bool kHasZ, bool kSoftplus, bool kZoh, bool kOut>
 __device__ __forceinline__ void compute_tile(const uint8_t* st, const float* bcf, int lane,
                                              int nsteps, LaneChains<kCpl>& lc,
                                              IoT* const (&out_row)[kCpl], bool vec_out,
@@ -248,22 +268,27 @@ __device__ __forceinline__ void compute_tile(const uint8_t* st, const float* bcf
 #pragma unroll
         for (int c = 0; c < kCpl; ++c) whole[c] = steps == V && vec_out && out_row[c] != nullptr;
         OutPack<IoT> pk[kCpl];
+        float dtv[kCpl][V], duv[kCpl][V];
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+#pragma unroll
+            for (int c = 0; c < kCpl; ++c) {
+                const float s = vec_elem<IoT>(dr[c], j) + lc.bias[c];
+                dtv[c][j] = kSoftplus ? softplus_f32(s) : s;
+                duv[c][j] = dtv[c][j] * vec_elem<IoT>(ur[c], j);
+            }
+        }
 #pragma unroll
         for (int j = 0; j < V; ++j) {
             if (steps == V || j < steps) {
-                float uj[kCpl], dt[kCpl], du[kCpl], y[kCpl];
+                float dt[kCpl], du[kCpl], y[kCpl];
 #pragma unroll
-                for (int c = 0; c < kCpl; ++c) {
-                    uj[c] = vec_elem<IoT>(ur[c], j);
-                    const float s = vec_elem<IoT>(dr[c], j) + lc.bias[c];
-                    dt[c] = kSoftplus ? softplus_f32(s) : s;
-                    du[c] = dt[c] * uj[c];
-                }
-                scan_step<kCpl, kOut, kExact>(bcf + (base + j) * 32, dt, du, lc, y);
+                for (int c = 0; c < kCpl; ++c) { dt[c] = dtv[c][j]; du[c] = duv[c][j]; }
+                scan_step<kCpl, kOut, kExact, kZoh>(bcf + (base + j) * 32, dt, du, lc, y);
 #pragma unroll
                 for (int c = 0; c < kCpl; ++c) {
                     if (kOut) {
-                        float yo = fmaf(lc.Dd[c], uj[c], y[c]);
+                        float yo = fmaf(lc.Dd[c], vec_elem<IoT>(ur[c], j), y[c]);
                         if (kHasZ) yo *= silu_f32(vec_elem<IoT>(zr[c], j));
                         if (whole[c])
                             pk[c].put(j, yo);
@@ -367,7 +392,7 @@ struct TmaMaps {
 // counts the tiles this warp has consumed (it fixes each tile's stage and
 // mbarrier parity across items).  Returns false if a staged tile never
 // arrived (the warp has then waited, bounded, for its copies in flight).
-template <typename IoT, int kCpl, bool kHasZ, bool kSoftplus, bool kOut>
+template <typename IoT, int kCpl, bool kHasZ, bool kSoftplus, bool kZoh, bool kOut>
 __device__ __forceinline__ bool run_segment(const ScanParams& p, const TmaMaps& maps, uint8_t* wsm,
                                             int lane, int64_t b, int64_t d0, int64_t t_begin,
                                             int64_t t_end, LaneChains<kCpl>& lc,
@@ -433,8 +458,8 @@ __device__ __forceinline__ bool run_segment(const ScanParams& p, const TmaMaps& 
         IoT* rows[kCpl];
 #pragma unroll
         for (int c = 0; c < kCpl; ++c) rows[c] = out_row[c] ? out_row[c] + (t0 - t_begin) : nullptr;
-        compute_tile<IoT, kCpl, kHasZ, kSoftplus, kOut>(st, bcf, lane, nsteps, lc, rows,
-                                                        p.vec_out != 0, sdt, sdt_c);
+        compute_tile<IoT, kCpl, kHasZ, kSoftplus, kZoh, kOut>(st, bcf, lane, nsteps, lc, rows,
+                                                              p.vec_out != 0, sdt, sdt_c);
         __syncwarp();
         if (p.use_tma && lane == 0 && i + kScanStages < ntiles) issue(i + kScanStages);
     }
@@ -469,8 +494,10 @@ __device__ __forceinline__ void st_release_gpu(unsigned int* p, unsigned int v) 
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-template <typename IoT, int kCpl, bool kHasZ, bool kSoftplus>
-__global__ void __launch_bounds__(kScanWarps * 32, ScanLayout<kCpl>::kMinBlocks)
+// kZoh keeps 1 / A in 16 more registers per channel, so its instances are
+// compiled for one CTA per SM fewer.
+template <typename IoT, int kCpl, bool kHasZ, bool kSoftplus, bool kZoh>
+__global__ void __launch_bounds__(kScanWarps * 32, ScanLayout<kCpl>::kMinBlocks - (kZoh ? 1 : 0))
     selective_scan_fwd_kernel(const __grid_constant__ ScanParams p,
                               const __grid_constant__ CUtensorMap tm_u,
                               const __grid_constant__ CUtensorMap tm_delta,
@@ -521,10 +548,16 @@ __global__ void __launch_bounds__(kScanWarps * 32, ScanLayout<kCpl>::kMinBlocks)
 #pragma unroll
             for (int pi = 0; pi < kNPad / 2; ++pi) {
                 const int n = 2 * pi;
-                lc.a2[c][pi] = make_float2(
-                    (valid[c] && n < p.dstate) ? p.A[d * p.dstate + n] * kLog2e : 0.0f,
-                    (valid[c] && n + 1 < p.dstate) ? p.A[d * p.dstate + n + 1] * kLog2e : 0.0f);
-                lc.h[c][pi] = make_float2(0.0f, 0.0f);
+                const bool in0 = valid[c] && n < p.dstate;
+                const bool in1 = valid[c] && n + 1 < p.dstate;
+                const float a0 = in0 ? p.A[d * p.dstate + n] : 0.0f;
+                const float a1 = in1 ? p.A[d * p.dstate + n + 1] : 0.0f;
+                lc.a2[c][pi] = make_float2(a0 * kLog2e, a1 * kLog2e);
+                if (kZoh) lc.inva[c][pi] = make_float2(in0 ? 1.0f / a0 : 0.0f, in1 ? 1.0f / a1 : 0.0f);
+                // Segment 0 starts from the given state (chained mode and pass A).
+                const float* h0 = (k == 0 && p.h0 != nullptr) ? p.h0 + chain[c] * p.dstate : nullptr;
+                lc.h[c][pi] = make_float2((h0 != nullptr && in0) ? h0[n] : 0.0f,
+                                          (h0 != nullptr && in1) ? h0[n + 1] : 0.0f);
             }
             lc.bias[c] = (valid[c] && p.delta_bias != nullptr) ? p.delta_bias[d] : 0.0f;
             lc.Dd[c] = (valid[c] && p.D != nullptr) ? p.D[d] : 0.0f;
@@ -582,11 +615,11 @@ __global__ void __launch_bounds__(kScanWarps * 32, ScanLayout<kCpl>::kMinBlocks)
         }
         bool ok;
         if (p.mode == kModePassA && k > 0)
-            ok = run_segment<IoT, kCpl, kHasZ, kSoftplus, false>(p, maps, wsm, lane, b, d0, t_begin,
-                                                                 t_end, lc, out_row, seq, sdt);
+            ok = run_segment<IoT, kCpl, kHasZ, kSoftplus, kZoh, false>(
+                p, maps, wsm, lane, b, d0, t_begin, t_end, lc, out_row, seq, sdt);
         else
-            ok = run_segment<IoT, kCpl, kHasZ, kSoftplus, true>(p, maps, wsm, lane, b, d0, t_begin,
-                                                                t_end, lc, out_row, seq, sdt);
+            ok = run_segment<IoT, kCpl, kHasZ, kSoftplus, kZoh, true>(
+                p, maps, wsm, lane, b, d0, t_begin, t_end, lc, out_row, seq, sdt);
         if (!ok) break;
 
         const bool last_seg = k == p.nseg - 1;

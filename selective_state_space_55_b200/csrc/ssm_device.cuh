@@ -65,6 +65,38 @@ __device__ __forceinline__ float2 exp2_near_one_exact2(float2 x) {
                        fabsf(x.y) < 0.0625f ? series.y : ex2_approx(x.y));
 }
 
+// Zero-order-hold input gain.  For the diagonal A the exact discretisation
+// Bbar = (Delta A)^-1 (exp(Delta A) - I) Delta B gives, per state entry,
+// Bbar_n = Delta phi(Delta A_n) B_n with phi(x) = (e^x - 1) / x, phi(0) = 1.
+// Written in x2 = x log2(e) (the exponent the scan already forms for Abar):
+// near 0, phi = 1 + x/2 + x^2/6 + x^3/24 + x^4/120 (truncation below 2.3e-10
+// for |x2| < 1/16), which avoids the cancellation in e^x - 1; elsewhere
+// phi = (Abar - 1) / x.
+constexpr float kZohSmall = 0.0625f;   // |x2| below which the series is used
+
+__device__ __forceinline__ float zoh_phi_series(float x2) {
+    constexpr float k1 = 0.34657359027997264f;     // ln2 / 2
+    constexpr float k2 = 0.08007550231970023f;     // ln2^2 / 6
+    constexpr float k3 = 0.013876027166205394f;    // ln2^3 / 24
+    constexpr float k4 = 0.0019236258215256953f;   // ln2^4 / 120
+    return fmaf(x2, fmaf(x2, fmaf(x2, fmaf(x2, k4, k3), k2), k1), 1.0f);
+}
+
+// zoh_phi_series on both halves, in packed fp32x2.
+__device__ __forceinline__ float2 zoh_phi_series2(float2 x2) {
+    const float2 k1 = make_float2(0.34657359027997264f, 0.34657359027997264f);
+    const float2 k2 = make_float2(0.08007550231970023f, 0.08007550231970023f);
+    const float2 k3 = make_float2(0.013876027166205394f, 0.013876027166205394f);
+    const float2 k4 = make_float2(0.0019236258215256953f, 0.0019236258215256953f);
+    const float2 one = make_float2(1.0f, 1.0f);
+    return __ffma2_rn(x2, __ffma2_rn(x2, __ffma2_rn(x2, __ffma2_rn(x2, k4, k3), k2), k1), one);
+}
+
+// phi for one entry given x2 = Delta A log2(e) and Abar = 2^x2 (scalar path).
+__device__ __forceinline__ float zoh_phi(float x2, float abar) {
+    return fabsf(x2) < kZohSmall ? zoh_phi_series(x2) : (abar - 1.0f) / (x2 * kLn2);
+}
+
 // softplus(s) = log(1 + e^s) = max(s, 0) + log1p(e^-|s|).
 // log1p(w) for w = e^-|s| in (0, 1] is evaluated as 2 atanh(r) with
 // r = w / (2 + w) in (0, 1/3]:  2 atanh(r) = 2 r (1 + r^2/3 + r^4/5 + ...).

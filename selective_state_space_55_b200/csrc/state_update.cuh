@@ -14,7 +14,9 @@
 // in flight.  The generic path (any N <= 16, any alignment) uses one thread
 // per chain.  Abar uses exp2_near_one_exact: the state persists across calls,
 // so an unbiased decay matters over many generated tokens, and this
-// memory-bound kernel has ALU time to spare.
+// memory-bound kernel has ALU time to spare.  With MAMBA_FLAG_ZOH every path
+// multiplies the input term by the zero-order-hold gain zoh_phi ("超越注意力：
+// 探索Mamba与状态空间模型", section 状态空间模型基础).
 #pragma once
 
 #include "ssm_device.cuh"
@@ -35,6 +37,7 @@ struct UpdateParams {
     int64_t batch, dim, chains;
     int dstate;
     int dt_softplus;
+    int zoh;             // zero-order-hold input term Delta phi(Delta A) B x
 };
 
 constexpr int kUpdateThreads = 256;
@@ -105,8 +108,10 @@ __global__ void __launch_bounds__(kUpdateThreads)
         float y = 0.0f;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const float abar = exp2_near_one_exact(delta * (a[i] * kLog2e));
-            h[i] = fmaf(abar, h[i], dx * Bv[i]);
+            const float x2 = delta * (a[i] * kLog2e);
+            const float abar = exp2_near_one_exact(x2);
+            const float gx = p.zoh ? dx * zoh_phi(x2, abar) : dx;
+            h[i] = fmaf(abar, h[i], gx * Bv[i]);
             y = fmaf(Cv[i], h[i], y);
         }
         y += __shfl_xor_sync(0xffffffffu, y, 1);
@@ -137,7 +142,8 @@ __global__ void __launch_bounds__(kUpdateThreads)
 // lanes share a chain (a float4 of state each); softplus and silu run once per
 // chain, spread over the four lanes, and are exchanged by shuffles.  Abar is
 // MUFU ex2 for bf16 inputs and exp2_near_one_exact for fp32 inputs, as in the
-// scan.
+// scan.  kZoh, the zero-order-hold gain zoh_phi, is a separate instance so
+// that the Euler one keeps its register count (72) and 5 CTAs per SM.
 constexpr int kBulkConsumers = 4;
 constexpr int kBulkThreads = 32 * (kBulkConsumers + 1);
 constexpr int kBulkTile = 32 * kBulkConsumers;       // channels per tile
@@ -152,7 +158,7 @@ constexpr int kBOffC = kBOffB + 64;
 constexpr int kBStage = ((kBOffC + 64 + 127) / 128) * 128;
 constexpr int kBulkSmemBytes = kBulkStages * kBStage + 2 * kBulkStages * 8 + 1024;
 
-template <typename IoT, typename BcT, bool kHasZ>
+template <typename IoT, typename BcT, bool kHasZ, bool kZoh>
 __global__ void __launch_bounds__(kBulkThreads)
     state_update_bulk_kernel(const __grid_constant__ UpdateParams p) {
     extern __shared__ uint8_t smem_raw[];
@@ -277,8 +283,14 @@ __global__ void __launch_bounds__(kBulkThreads)
                                       : make_float2(ex2_approx(x01.x), ex2_approx(x01.y));
             const float2 e23 = kExact ? exp2_near_one_exact2(x23)
                                       : make_float2(ex2_approx(x23.x), ex2_approx(x23.y));
-            const float2 h01 = __ffma2_rn(e01, make_float2(hs.x, hs.y), __fmul2_rn(dx2, b01));
-            const float2 h23 = __ffma2_rn(e23, make_float2(hs.z, hs.w), __fmul2_rn(dx2, b23));
+            float2 in01 = __fmul2_rn(dx2, b01);
+            float2 in23 = __fmul2_rn(dx2, b23);
+            if (kZoh) {
+                in01 = __fmul2_rn(in01, make_float2(zoh_phi(x01.x, e01.x), zoh_phi(x01.y, e01.y)));
+                in23 = __fmul2_rn(in23, make_float2(zoh_phi(x23.x, e23.x), zoh_phi(x23.y, e23.y)));
+            }
+            const float2 h01 = __ffma2_rn(e01, make_float2(hs.x, hs.y), in01);
+            const float2 h23 = __ffma2_rn(e23, make_float2(hs.z, hs.w), in23);
             const float2 yy = __ffma2_rn(c23, h23, __fmul2_rn(c01, h01));
             float y = yy.x + yy.y;
             y += __shfl_xor_sync(0xffffffffu, y, 1);
@@ -331,9 +343,11 @@ __global__ void __launch_bounds__(kUpdateThreads)
     const float dx = delta * x;
     float y = 0.0f;
     for (int n = 0; n < p.dstate; ++n) {
-        const float abar = exp2_near_one_exact(delta * (p.A[d * p.dstate + n] * kLog2e));
+        const float x2 = delta * (p.A[d * p.dstate + n] * kLog2e);
+        const float abar = exp2_near_one_exact(x2);
+        const float gx = p.zoh ? dx * zoh_phi(x2, abar) : dx;
         float* hp = p.state + chain * p.dstate + n;
-        const float h = fmaf(abar, *hp, dx * load_as_float<BcT>(p.B, b * p.dstate + n));
+        const float h = fmaf(abar, *hp, gx * load_as_float<BcT>(p.B, b * p.dstate + n));
         *hp = h;
         y = fmaf(load_as_float<BcT>(p.C, b * p.dstate + n), h, y);
     }

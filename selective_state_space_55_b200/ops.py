@@ -21,12 +21,13 @@ MAMBA_OK = 0
 STATUS_NAMES = {
     0: "MAMBA_OK", -1: "MAMBA_ERR_INVALID_ARG", -2: "MAMBA_ERR_UNSUPPORTED",
     -3: "MAMBA_ERR_ALIGN", -4: "MAMBA_ERR_WORKSPACE", -5: "MAMBA_ERR_CUDA",
-    -6: "MAMBA_ERR_TIMEOUT",
+    -6: "MAMBA_ERR_TIMEOUT", -7: "MAMBA_ERR_TOO_LARGE",
 }
 MAMBA_F32, MAMBA_BF16 = 0, 1
 MAMBA_FLAG_NO_TMA = 0x1
 MAMBA_FLAG_PARALLEL_CHUNKS = 0x2
 MAMBA_FLAG_TEST_WITHHOLD_HANDOFF = 0x4
+MAMBA_FLAG_ZOH = 0x8
 
 _DTYPE_CODE = {torch.float32: MAMBA_F32, torch.bfloat16: MAMBA_BF16}
 
@@ -84,6 +85,9 @@ def library(path: Path | str | None = None) -> ctypes.CDLL:
     lib.mamba_selective_scan_workspace_bytes.argtypes = [dims_p]
     lib.mamba_selective_scan_fwd.restype = i32
     lib.mamba_selective_scan_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, dims_p, vp]
+    lib.mamba_selective_scan_fwd_with_state.restype = i32
+    lib.mamba_selective_scan_fwd_with_state.argtypes = [
+        vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, dims_p, vp]
     lib.mamba_selective_state_update.restype = i32
     lib.mamba_selective_state_update.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, dims_p, vp]
     lib.mamba_device_status.restype = i32
@@ -159,11 +163,14 @@ def scan_workspace_bytes(batch, dim, dstate, seqlen, io_dtype=torch.bfloat16,
 
 def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
                        out=None, last_state=None, return_last_state=False, num_chunks=0,
-                       flags=0, workspace=None, stream=None):
-    """Selective scan forward through ``mamba_selective_scan_fwd``.
+                       flags=0, workspace=None, stream=None, initial_state=None, zoh=False):
+    """Selective scan forward through ``mamba_selective_scan_fwd`` (or
+    ``mamba_selective_scan_fwd_with_state`` when ``initial_state`` is given).
 
     u, delta, z: (batch, dim, L) fp32 or bf16 (one dtype); B, C: (batch, N, L)
-    fp32 or bf16; A: (dim, N) fp32; D, delta_bias: (dim,) fp32 or None.
+    fp32 or bf16; A: (dim, N) fp32; D, delta_bias: (dim,) fp32 or None;
+    initial_state: (batch, dim, N) fp32 start state or None (zero).  ``zoh``
+    sets MAMBA_FLAG_ZOH (zero-order-hold input term).
     Returns ``out`` (batch, dim, L) in u's dtype, and the fp32 last state
     (batch, dim, N) too when ``return_last_state`` or ``last_state`` is given.
     """
@@ -184,26 +191,40 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softp
     if last_state is None and return_last_state:
         last_state = torch.empty((batch, dim, N), dtype=torch.float32, device=u.device)
     _check_cuda("last_state", last_state, (torch.float32,), (batch, dim, N))
+    _check_cuda("initial_state", initial_state, (torch.float32,), (batch, dim, N))
+    if zoh:
+        flags |= MAMBA_FLAG_ZOH
     if workspace is None:
         need = scan_workspace_bytes(batch, dim, N, L, io, bc, num_chunks, flags)
         if need > 0:
             workspace = torch.empty(need, dtype=torch.uint8, device=u.device)
     dims = make_scan_dims(batch, dim, N, L, io, bc, num_chunks, flags, workspace)
-    rc = library().mamba_selective_scan_fwd(
-        _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
-        int(bool(softplus)), _ptr(out), _ptr(last_state), ctypes.byref(dims),
-        _stream_handle(stream))
+    if initial_state is None:
+        name = "mamba_selective_scan_fwd"
+        rc = library().mamba_selective_scan_fwd(
+            _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
+            int(bool(softplus)), _ptr(out), _ptr(last_state), ctypes.byref(dims),
+            _stream_handle(stream))
+    else:
+        name = "mamba_selective_scan_fwd_with_state"
+        rc = library().mamba_selective_scan_fwd_with_state(
+            _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
+            int(bool(softplus)), _ptr(initial_state), _ptr(out), _ptr(last_state),
+            ctypes.byref(dims), _stream_handle(stream))
     if rc != MAMBA_OK:
-        raise MambaError("mamba_selective_scan_fwd", rc)
+        raise MambaError(name, rc)
     if last_state is not None:
         return out, last_state
     return out
 
 
 def selective_state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=None,
-                           dt_softplus=True, out=None, flags=0, stream=None):
+                           dt_softplus=True, out=None, flags=0, stream=None, zoh=False):
     """One generation step through ``mamba_selective_state_update``; ``state`` is
-    updated in place.  Returns ``out`` (batch, dim) in x's dtype."""
+    updated in place.  ``zoh`` sets MAMBA_FLAG_ZOH.  Returns ``out`` (batch, dim) in
+    x's dtype."""
+    if zoh:
+        flags |= MAMBA_FLAG_ZOH
     batch, dim, N = state.shape
     io, bc = x.dtype, B.dtype
     _check_cuda("state", state, (torch.float32,), (batch, dim, N))

@@ -3,7 +3,8 @@
 Scan, per element (b, d, t):
   MUFU-class operations: 16 ex2 for Abar (one per state entry) + 2 for
   softplus (ex2 and a reciprocal) + 2 for the silu gate (ex2 and a
-  reciprocal) = 20.  At 16 per clock per SM this is the binding pipe; the
+  reciprocal) = 20, plus one reciprocal of Delta with the zero-order hold.
+  At 16 per clock per SM this is the binding pipe; the
   bytes (u, delta, z read, out written, plus each batch row's B and C shared
   by all channels) are about 8 per element in bf16, far below what HBM moves
   in the same time.
@@ -22,22 +23,28 @@ MUFU_PER_SM_PER_CLOCK = 16
 EXP_PER_STATE = 1
 SOFTPLUS_MUFU = 2
 SILU_MUFU = 2
+ZOH_MUFU = 1          # zero-order hold: 1 / Delta once per element
 
 
-def scan_mufu_per_element(dstate: int = 16, has_z: bool = True, softplus: bool = True) -> int:
-    return dstate * EXP_PER_STATE + (SOFTPLUS_MUFU if softplus else 0) + (SILU_MUFU if has_z else 0)
+def scan_mufu_per_element(dstate: int = 16, has_z: bool = True, softplus: bool = True,
+                          zoh: bool = False) -> int:
+    return (dstate * EXP_PER_STATE + (SOFTPLUS_MUFU if softplus else 0)
+            + (SILU_MUFU if has_z else 0) + (ZOH_MUFU if zoh else 0))
 
 
 def scan_bytes(batch: int, dim: int, dstate: int, seqlen: int, io_bytes: int = 2,
-               bc_bytes: int = 2, has_z: bool = True, last_state: bool = False) -> int:
+               bc_bytes: int = 2, has_z: bool = True, last_state: bool = False,
+               start_state: bool = False) -> int:
     """HBM bytes one scan must move: u, delta, (z) read, out written, B and C
-    read once per batch row, A/D/bias once, last_state written."""
+    read once per batch row, A/D/bias once, last_state written, the start
+    state read."""
     elems = batch * dim * seqlen
     io = elems * io_bytes * (3 + (1 if has_z else 0))
     bc = 2 * batch * dstate * seqlen * bc_bytes
     params = dim * dstate * 4 + 2 * dim * 4
     tail = batch * dim * dstate * 4 if last_state else 0
-    return io + bc + params + tail
+    head = batch * dim * dstate * 4 if start_state else 0
+    return io + bc + params + tail + head
 
 
 def mufu_peak_elements_per_s(sm_count: int, sm_mhz: float, mufu_per_element: int) -> float:

@@ -30,6 +30,7 @@ def declared_symbols():
 def test_header_declares_entry_points():
     syms = declared_symbols()
     for name in ("mamba_selective_scan_fwd", "mamba_selective_state_update",
+                 "mamba_selective_scan_fwd_with_state", "mamba_selective_scan_fwd_noalloc",
                  "mamba_selective_scan_workspace_bytes", "mamba_selective_scan_plan",
                  "mamba_status_string", "mamba_device_status", "mamba_version"):
         assert name in syms
@@ -77,6 +78,29 @@ def test_scan_rejects_bad_arguments(lib):
     assert _scan(lib, _dims(), u=ctypes.c_void_p(0x10001)) == -3
     assert _scan(lib, _dims(), A=ctypes.c_void_p(0x10002)) == -3
     assert _scan(lib, _dims(io_dtype=torch.float32), out=ctypes.c_void_p(0x10002)) == -3
+
+
+def _scan_h0(lib, dims, h0, last, u=FAKE):
+    return lib.mamba_selective_scan_fwd_with_state(u, FAKE, FAKE, FAKE, FAKE, None, None, None, 1,
+                                                   h0, FAKE, last, ctypes.byref(dims), None)
+
+
+def test_scan_with_state_rejects_bad_start_state(lib):
+    d = _dims(batch=2, dim=64, dstate=16)            # 2 * 64 * 16 fp32 = 8 KiB of state
+    nbytes = 2 * 64 * 16 * 4
+    base = 0x100000
+    # misaligned start state
+    assert _scan_h0(lib, d, ctypes.c_void_p(base + 2), ctypes.c_void_p(base + 0x10000)) == -3
+    # partial overlap with last_state, either way round, by one element or by most of it
+    for shift in (4, nbytes - 4, -4, -(nbytes - 4)):
+        assert _scan_h0(lib, d, ctypes.c_void_p(base), ctypes.c_void_p(base + shift)) == -1
+    # the same buffer (in-place continuation) passes these checks and then fails on
+    # the null input pointer, still before any device work
+    assert _scan_h0(lib, d, ctypes.c_void_p(base), ctypes.c_void_p(base), u=None) == -1
+    # disjoint buffers likewise
+    assert _scan_h0(lib, d, ctypes.c_void_p(base), ctypes.c_void_p(base + nbytes), u=None) == -1
+    # the start-state entry point validates dims like the plain one
+    assert _scan_h0(lib, _dims(dstate=17), ctypes.c_void_p(base), None) == -2
 
 
 def test_scan_empty_batch_is_a_no_op(lib):

@@ -1,0 +1,249 @@
+"""Scan and update options: the zero-order-hold input term (MAMBA_FLAG_ZOH) and
+a given start state (mamba_selective_scan_fwd_with_state).  CUDA path through
+the C ABI vs the float64 oracle, plus closed forms the pages fix: the Theorem-1
+gate is exact under the zero-order hold, and a constant input has the fixed
+point -B u / A whatever Delta does."""
+import pytest
+import torch
+
+from oracle import oracle
+from parity import BF16_TOL, FP32_TOL, max_rel_err, tol_for
+from selective_state_space_55_b200 import inputs as I
+from selective_state_space_55_b200 import ops
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+PAR = ops.MAMBA_FLAG_PARALLEL_CHUNKS
+
+
+@pytest.fixture(scope="module")
+def ref():
+    return oracle.default()
+
+
+def layer_inputs(batch, dim, L, dtype=torch.bfloat16, seed=0, N=16):
+    cfg = I.SCAN_CONFIGS["mamba_1p4b_layer"].resized(batch=batch, dim=dim, seqlen=L, dstate=N,
+                                                       io_dtype=dtype, bc_dtype=dtype,
+                                                       recipe="layer")
+    return I.make_scan_inputs(cfg, DEV, seed)
+
+
+def start_state(batch, dim, N, seed, scale=1.0):
+    g = torch.Generator(device=DEV)
+    g.manual_seed(seed)
+    return torch.randn(batch, dim, N, generator=g, device=DEV) * scale
+
+
+def gpu_scan(x, **kw):
+    out, last = ops.selective_scan_fwd(x["u"], x["delta"], x["A"], x["B"], x["C"], D=x["D"],
+                                       z=x["z"], delta_bias=x["delta_bias"],
+                                       return_last_state=True, **kw)
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    return out, last
+
+
+def oracle_scan(ref, x, zoh=False, initial_state=None, softplus=True):
+    c = lambda t: None if t is None else t.cpu()  # noqa: E731
+    return ref.selective_scan(c(x["u"]), c(x["delta"]), c(x["A"]), c(x["B"]), c(x["C"]),
+                              D=c(x["D"]), z=c(x["z"]), delta_bias=c(x["delta_bias"]),
+                              softplus=softplus, zoh=zoh, initial_state=c(initial_state))
+
+
+def compare(ref, x, tol, zoh=False, h0=None, **kw):
+    o_out, o_last = oracle_scan(ref, x, zoh=zoh, initial_state=h0)
+    out, last = gpu_scan(x, zoh=zoh, initial_state=h0, **kw)
+    e_out, e_last = max_rel_err(out, o_out), max_rel_err(last, o_last)
+    assert e_out <= tol, f"out error {e_out:.3e} > {tol:.1e}"
+    assert e_last <= tol, f"last_state error {e_last:.3e} > {tol:.1e}"
+    return out, last
+
+
+# ------------------------------------------------------------ zero-order hold
+
+def test_zoh_tiny_fp32(ref):
+    x = I.make_scan_inputs(I.SCAN_CONFIGS["tiny_fp32"], DEV, seed=0)
+    compare(ref, x, FP32_TOL, zoh=True)
+
+
+@pytest.mark.parametrize("dtype,shape", [(torch.bfloat16, (2, 256, 2048)),
+                                         (torch.float32, (2, 96, 1024))])
+def test_zoh_layer_recipe(ref, dtype, shape):
+    """The layer recipe's Delta (1e-4 .. 0.7) times A (-1 .. -16) takes both the
+    series and the (Abar - 1) / (Delta A) branch of the gain."""
+    x = layer_inputs(*shape, dtype=dtype, seed=5)
+    compare(ref, x, tol_for(dtype), zoh=True)
+
+
+@pytest.mark.parametrize("flags", [0, PAR], ids=["chained", "parallel"])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_zoh_segments_long_memory(ref, dtype, flags):
+    x = layer_inputs(1, 64, 4096, dtype=dtype, seed=7)
+    x["delta_bias"] = torch.full_like(x["delta_bias"], -9.0)   # Delta ~ 1e-4
+    compare(ref, x, tol_for(dtype), zoh=True, num_chunks=3, flags=flags)
+
+
+def test_zoh_zero_A_is_euler(ref):
+    """A = 0: the gain's limit is Delta (no 0/0 from 1/A or 1/Delta)."""
+    x = layer_inputs(2, 40, 300, dtype=torch.float32, seed=9)
+    x["A"] = torch.zeros_like(x["A"])
+    out, last = compare(ref, x, FP32_TOL, zoh=True)
+    e_out, e_last = gpu_scan(x)
+    assert max_rel_err(out, e_out.double()) <= FP32_TOL
+    assert max_rel_err(last, e_last.double()) <= FP32_TOL
+
+
+def test_zoh_gated_rnn_theorem1_on_gpu():
+    """N=1, A=-1, B=C=1, D=0, softplus on: h_t = (1-g_t) h_{t-1} + g_t x_t exactly,
+    g = sigmoid(delta + bias) (no B = g / Delta rescaling needed)."""
+    g_ = torch.Generator(device=DEV)
+    g_.manual_seed(21)
+    batch, dim, L = 2, 33, 200
+    s = torch.randn(batch, dim, L, generator=g_, device=DEV) * 2
+    xin = torch.randn(batch, dim, L, generator=g_, device=DEV)
+    bias = torch.rand(dim, generator=g_, device=DEV) - 0.5
+    ones = torch.ones(batch, 1, L, device=DEV)
+    out, last = ops.selective_scan_fwd(xin, s, -torch.ones(dim, 1, device=DEV), ones, ones,
+                                       delta_bias=bias, return_last_state=True, zoh=True)
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    g = torch.sigmoid((s + bias[None, :, None]).double().cpu())
+    xd = xin.double().cpu()
+    h = torch.zeros(batch, dim, dtype=torch.float64)
+    want = torch.zeros(batch, dim, L, dtype=torch.float64)
+    for t in range(L):
+        h = (1 - g[:, :, t]) * h + g[:, :, t] * xd[:, :, t]
+        want[:, :, t] = h
+    assert max_rel_err(out, want) <= FP32_TOL
+    assert max_rel_err(last[:, :, 0], want[:, :, -1]) <= FP32_TOL
+
+
+def test_zoh_fixed_point_from_start_state():
+    """u and B constant in time, start state h* = -B u / A: the state never moves and
+    y_t = sum_n C_t,n h*_n + D u for any Delta sequence."""
+    x = layer_inputs(2, 48, 512, dtype=torch.float32, seed=23)
+    x["u"] = x["u"][:, :, :1].expand_as(x["u"]).contiguous()
+    x["B"] = x["B"][:, :, :1].expand_as(x["B"]).contiguous()
+    x["z"] = None
+    h_star = (-x["B"][:, None, :, 0] * x["u"][:, :, :1] / x["A"][None, :, :]).contiguous()
+    out, last = gpu_scan(x, zoh=True, initial_state=h_star, num_chunks=2)
+    want = torch.einsum("bdn,bnt->bdt", h_star.double(), x["C"].double()) + \
+        x["D"].double()[None, :, None] * x["u"].double()
+    assert max_rel_err(out, want.cpu()) <= FP32_TOL
+    assert max_rel_err(last, h_star.double().cpu()) <= FP32_TOL
+
+
+# ------------------------------------------------------------ start state
+
+@pytest.mark.parametrize("K,flags", [(0, 0), (1, 0), (3, 0), (3, PAR)],
+                         ids=["auto", "one_segment", "chained3", "parallel3"])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_start_state(ref, dtype, K, flags):
+    x = layer_inputs(2, 80, 1536, dtype=dtype, seed=31)
+    h0 = start_state(2, 80, 16, seed=32)
+    compare(ref, x, tol_for(dtype), h0=h0, num_chunks=K, flags=flags)
+
+
+@pytest.mark.parametrize("N", [1, 5, 16])
+def test_start_state_sizes(ref, N):
+    x = layer_inputs(1, 40, 300, dtype=torch.float32, seed=33 + N, N=N)
+    compare(ref, x, FP32_TOL, h0=start_state(1, 40, N, seed=34 + N))
+
+
+def test_start_state_with_zoh_layer(ref):
+    x = layer_inputs(2, 256, 2048, seed=35)
+    compare(ref, x, BF16_TOL, zoh=True, h0=start_state(2, 256, 16, seed=36))
+
+
+@pytest.mark.parametrize("L1", [384, 377])
+def test_split_scan_equals_whole(ref, L1):
+    """Scanning [0, L1) and then [L1, L) from the first part's last_state gives the
+    whole scan's outputs and end state."""
+    x = layer_inputs(2, 64, 1000, dtype=torch.float32, seed=37)
+    out, last = compare(ref, x, FP32_TOL)
+    part = lambda t, sl: None if t is None else t[:, :, sl].contiguous()  # noqa: E731
+    keys = ("u", "delta", "z", "B", "C")
+    x1 = dict(x, **{k: part(x[k], slice(0, L1)) for k in keys})
+    x2 = dict(x, **{k: part(x[k], slice(L1, None)) for k in keys})
+    o1, l1 = gpu_scan(x1)
+    o2, l2 = gpu_scan(x2, initial_state=l1)
+    assert max_rel_err(torch.cat([o1, o2], dim=-1), out.double()) <= FP32_TOL
+    assert max_rel_err(l2, last.double()) <= FP32_TOL
+
+
+def test_start_state_in_place(ref):
+    """initial_state and last_state may be one buffer: read first, then overwritten."""
+    x = layer_inputs(2, 64, 700, dtype=torch.float32, seed=39)
+    h = start_state(2, 64, 16, seed=40)
+    o_out, o_last = oracle_scan(ref, x, initial_state=h)
+    out = ops.selective_scan_fwd(x["u"], x["delta"], x["A"], x["B"], x["C"], D=x["D"], z=x["z"],
+                                 delta_bias=x["delta_bias"], initial_state=h, last_state=h,
+                                 num_chunks=3)[0]
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    assert max_rel_err(out, o_out) <= FP32_TOL
+    assert max_rel_err(h, o_last) <= FP32_TOL
+
+
+def test_start_state_empty_sequence():
+    """seqlen 0: last_state becomes a copy of the start state."""
+    x = layer_inputs(2, 24, 0, dtype=torch.float32, seed=41)
+    h0 = start_state(2, 24, 16, seed=42)
+    last = torch.full_like(h0, float("nan"))
+    ops.selective_scan_fwd(x["u"], x["delta"], x["A"], x["B"], x["C"], initial_state=h0,
+                           last_state=last)
+    torch.cuda.synchronize()
+    assert torch.equal(last, h0)
+    same = h0.clone()
+    ops.selective_scan_fwd(x["u"], x["delta"], x["A"], x["B"], x["C"], initial_state=same,
+                           last_state=same)
+    torch.cuda.synchronize()
+    assert torch.equal(same, h0)
+
+
+# ------------------------------------------------------------ update
+
+def decode_cfg(batch, dim, N=16, io=torch.bfloat16, bc=torch.bfloat16):
+    return I.DecodeConfig("t", batch=batch, dim=dim, dstate=N, layers=1, steps=1, io_dtype=io,
+                          bc_dtype=bc)
+
+
+@pytest.mark.parametrize("dim,N,flags", [(1024, 16, 0), (1024, 16, ops.MAMBA_FLAG_NO_TMA),
+                                         (320, 5, 0)], ids=["streaming", "plain", "generic"])
+@pytest.mark.parametrize("io", [torch.bfloat16, torch.float32])
+def test_zoh_update_paths(ref, dim, N, flags, io):
+    cfg = decode_cfg(8, dim, N, io=io, bc=io)
+    layer = I.make_decode_layer(cfg, DEV, seed=dim + N)
+    tok = I.make_decode_token(cfg, DEV, seed=dim + N + 1)
+    state = layer["state"].clone()
+    out = ops.selective_state_update(state, tok["x"], tok["dt"], layer["A"], tok["B"], tok["C"],
+                                     D=layer["D"], z=tok["z"], dt_bias=layer["dt_bias"],
+                                     flags=flags, zoh=True)
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    c = lambda t: t.cpu()  # noqa: E731
+    o_state, o_out = ref.selective_state_update(
+        c(layer["state"]), c(tok["x"]), c(tok["dt"]), c(layer["A"]), c(tok["B"]), c(tok["C"]),
+        D=c(layer["D"]), z=c(tok["z"]), dt_bias=c(layer["dt_bias"]), zoh=True)
+    assert max_rel_err(state, o_state) <= FP32_TOL
+    assert max_rel_err(out, o_out) <= tol_for(io)
+
+
+def test_zoh_updates_continue_zoh_scan():
+    """T zero-order-hold updates from a start state equal the zero-order-hold scan
+    over the same T tokens from that state."""
+    x = layer_inputs(4, 256, 24, dtype=torch.float32, seed=43)
+    h0 = start_state(4, 256, 16, seed=44)
+    out, last = gpu_scan(x, zoh=True, initial_state=h0)
+    state = h0.clone()
+    outs = []
+    for t in range(24):
+        col = lambda k: x[k][:, :, t].contiguous()  # noqa: E731
+        outs.append(ops.selective_state_update(state, col("u"), col("delta"), x["A"], col("B"),
+                                               col("C"), D=x["D"], z=col("z"),
+                                               dt_bias=x["delta_bias"], zoh=True))
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    assert max_rel_err(torch.stack(outs, dim=-1), out.double()) <= FP32_TOL
+    assert max_rel_err(state, last.double()) <= FP32_TOL
