@@ -407,7 +407,8 @@ def bench_ours(args, rank, world, local):
     peaks = measured_peaks()
     clocks = sampler.summary(t_wall0, t_wall1)
     mufu = R.scan_mufu_per_element(c.dstate, has_z=True, softplus=True,
-                                   zoh=args.scan_variant == "zoh")
+                                   zoh=args.scan_variant == "zoh",
+                                   io_bytes=c.io_dtype.itemsize)
     peak_elems = R.mufu_peak_elements_per_s(torch.cuda.get_device_properties(local).multi_processor_count,
                                             peaks["sm_max_mhz"], mufu) / 1e9
     achieved = elems / (scan_launch_ms * 1e-3) / 1e9               # per launch, this rank
@@ -421,7 +422,8 @@ def bench_ours(args, rank, world, local):
         "kernel": "selective_scan_fwd_kernel",
         "achieved": round(achieved, 2), "peak": round(peak_elems, 2), "unit": "Gelem/s",
         "frac": round(achieved / peak_elems, 4),
-        "peak_basis": f"148 SMs x 16 MUFU/clk x {peaks['sm_max_mhz']:.0f} MHz / {mufu} per element",
+        "peak_basis": f"148 SMs x 16 MUFU/clk x {peaks['sm_max_mhz']:.0f} MHz / {mufu} MUFU ops "
+                      "the kernel issues per element",
         "frac_at_measured_clock": (round(achieved / (peak_elems * clocks["sm_mhz"] / peaks["sm_max_mhz"]), 4)
                                    if clocks.get("sm_mhz") else None),
         "algorithmic_bytes_per_launch": scan_bytes,

@@ -232,12 +232,16 @@ __device__ __forceinline__ void scan_step(const float* bc_row, const float (&dt)
     }
     if (kOut) {
 #pragma unroll
-        for (int c = 0; c < kCpl; ++c) y[c] = (ya[c].x + ya[c].y) + (yb[c].x + yb[c].y);
+        for (int c = 0; c < kCpl; ++c) {
+            const float2 t = __fadd2_rn(ya[c], yb[c]);
+            y[c] = t.x + t.y;
+        }
     }
 }
 
 // Process the `nsteps` (<= T) valid time steps of one staged tile, one
-// 16-byte vector of u, delta and z (V steps) at a time.  Delta and Delta u of
+// 16-byte vector of u, delta and z (V steps) at a time.  bf16 inputs take the
+// shorter softplus_lg2 / silu_tanh, fp32 inputs softplus_f32 / silu_f32.  Delta and Delta u of
 // all V steps are formed first: their softplus chains are independent of the
 // state, so computing them together lets their latency overlap.  The vectors
 // stay packed and are unpacked element by element to save registers.
@@ -274,7 +278,7 @@ __device__ __forceinline__ void compute_tile(const uint8_t* st, const float* bcf
 #pragma unroll
             for (int c = 0; c < kCpl; ++c) {
                 const float s = vec_elem<IoT>(dr[c], j) + lc.bias[c];
-                dtv[c][j] = kSoftplus ? softplus_f32(s) : s;
+                dtv[c][j] = kSoftplus ? (kExact ? softplus_f32(s) : softplus_lg2(s)) : s;
                 duv[c][j] = dtv[c][j] * vec_elem<IoT>(ur[c], j);
             }
         }
@@ -289,7 +293,10 @@ __device__ __forceinline__ void compute_tile(const uint8_t* st, const float* bcf
                 for (int c = 0; c < kCpl; ++c) {
                     if (kOut) {
                         float yo = fmaf(lc.Dd[c], vec_elem<IoT>(ur[c], j), y[c]);
-                        if (kHasZ) yo *= silu_f32(vec_elem<IoT>(zr[c], j));
+                        if (kHasZ) {
+                            const float zj = vec_elem<IoT>(zr[c], j);
+                            yo *= kExact ? silu_f32(zj) : silu_tanh(zj);
+                        }
                         if (whole[c])
                             pk[c].put(j, yo);
                         else if (out_row[c] != nullptr)

@@ -123,6 +123,39 @@ __device__ __forceinline__ float silu_f32(float z) {
     return __fdividef(z, 1.0f + ex2_approx(-z * kLog2e));
 }
 
+// ---- shorter forms for bf16 inputs and outputs ----------------------------
+// The scan is bounded by instruction issue and the MUFU pipe, not by memory,
+// so each instruction per step counts.  With bf16 inputs the inputs already
+// carry a relative rounding of 2^-9 (for delta near -9 that alone moves Delta
+// by about 2%), so these forms trade digits that bf16 cannot hold:
+//  - softplus_lg2: log1p(w) = log2(1 + w) ln 2 on MUFU lg2.  1 + w rounds
+//    to fp32 and lg2.approx has an absolute error near 2^-22, so Delta is off
+//    by at most ~3e-7 absolute (relative ~3e-3 at the smallest Delta ~1e-4 of
+//    the layer workloads), against ~16 instructions and an rcp for softplus_f32.
+//  - silu_tanh: sigmoid(z) = (1 + tanh(z/2)) / 2, one MUFU tanh (relative
+//    error 2^-11) instead of ex2 and rcp; silu is off by at most ~2.5e-4 |z|.
+__device__ __forceinline__ float lg2_approx(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ float tanh_approx(float x) {
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ float softplus_lg2(float s) {
+    const float w = ex2_approx(-fabsf(s) * kLog2e);
+    return fmaf(lg2_approx(1.0f + w), kLn2, fmaxf(s, 0.0f));
+}
+
+__device__ __forceinline__ float silu_tanh(float z) {
+    const float hz = 0.5f * z;
+    return fmaf(hz, tanh_approx(hz), hz);
+}
+
 // ------------------------------------------------------------------- dtypes
 
 template <typename T> struct DType;

@@ -2,8 +2,9 @@
 
 Scan, per element (b, d, t):
   MUFU-class operations: 16 ex2 for Abar (one per state entry) + 2 for
-  softplus (ex2 and a reciprocal) + 2 for the silu gate (ex2 and a
-  reciprocal) = 20, plus one reciprocal of Delta with the zero-order hold.
+  softplus (ex2 and a reciprocal, or ex2 and lg2 for bf16 inputs) + the silu
+  gate (ex2 and a reciprocal, or one tanh for bf16 inputs) = 20 (fp32) or 19
+  (bf16), plus one reciprocal of Delta with the zero-order hold.
   At 16 per clock per SM this is the binding pipe; the
   bytes (u, delta, z read, out written, plus each batch row's B and C shared
   by all channels) are about 8 per element in bf16, far below what HBM moves
@@ -26,10 +27,17 @@ SILU_MUFU = 2
 ZOH_MUFU = 1          # zero-order hold: 1 / Delta once per element
 
 
+SILU_MUFU_BF16 = 1    # bf16 path: one tanh
+
+
 def scan_mufu_per_element(dstate: int = 16, has_z: bool = True, softplus: bool = True,
-                          zoh: bool = False) -> int:
-    return (dstate * EXP_PER_STATE + (SOFTPLUS_MUFU if softplus else 0)
-            + (SILU_MUFU if has_z else 0) + (ZOH_MUFU if zoh else 0))
+                          zoh: bool = False, io_bytes: int = 4) -> int:
+    """MUFU operations the scan kernel issues per element: one ex2 per state
+    entry, softplus (ex2 + rcp for fp32 inputs, ex2 + lg2 for bf16), the gate
+    (ex2 + rcp for fp32, one tanh for bf16) and 1/Delta with the zero-order hold."""
+    silu = (SILU_MUFU_BF16 if io_bytes == 2 else SILU_MUFU) if has_z else 0
+    return (dstate * EXP_PER_STATE + (SOFTPLUS_MUFU if softplus else 0) + silu
+            + (ZOH_MUFU if zoh else 0))
 
 
 def scan_bytes(batch: int, dim: int, dstate: int, seqlen: int, io_bytes: int = 2,

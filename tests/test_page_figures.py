@@ -40,6 +40,8 @@ def test_update_bytes_decode_shape():
 def test_scan_mufu_model():
     assert R.scan_mufu_per_element(16) == 20
     assert R.scan_mufu_per_element(16, has_z=False, softplus=False) == 16
+    assert R.scan_mufu_per_element(16, io_bytes=2) == 19          # bf16: lg2 softplus, tanh gate
+    assert R.scan_mufu_per_element(16, io_bytes=2, zoh=True) == 20  # + 1/Delta
     peak = R.mufu_peak_elements_per_s(148, 1965.0, 20)
     assert abs(peak / 1e9 - 232.7) < 0.1
 
