@@ -249,31 +249,33 @@ class Workload:
         return (0 if self.only == "decode" else self.plan["launches"]) + len(self.layers)
 
 
-def run_e2e(w: Workload, steps: int, warmup: int) -> dict:
-    """Scan metric end to end: pinned host inputs -> device -> scan -> host."""
+def run_e2e(w: Workload, steps: int, warmup: int, rows: int = 0) -> dict:
+    """Scan metric end to end through mamba_selective_scan_fwd_host: every step
+    reads its inputs from pinned host memory and writes out / last_state back
+    to pinned host memory; the library pipelines the copies by chunks of batch
+    rows against the scans."""
+    ops = w.ops
     x = w.x
-    names = ["u", "delta", "z", "B", "C"]
-    host = {k: torch.empty(x[k].shape, dtype=x[k].dtype, pin_memory=True) for k in names}
-    for k in names:
-        host[k].copy_(x[k])
+    c = w.cfg
+    names = ["u", "delta", "z", "B", "C", "A", "D", "delta_bias"]
+    host = {k: (None if x[k] is None else x[k].cpu().pin_memory()) for k in names}
+    h0_h = None if w.h0 is None else w.h0.cpu().pin_memory()
     out_h = torch.empty(w.out.shape, dtype=w.out.dtype, pin_memory=True)
     last_h = torch.empty(w.last.shape, dtype=w.last.dtype, pin_memory=True)
-    h0_h = None
-    if w.h0 is not None:
-        h0_h = torch.empty(w.h0.shape, dtype=w.h0.dtype, pin_memory=True)
-        h0_h.copy_(w.h0)
-    h2d = sum(host[k].numel() * host[k].element_size() for k in names)
+    zoh = w.variant == "zoh"
+    flags = ops.MAMBA_FLAG_ZOH if zoh else 0
+    need = ops.scan_host_workspace_bytes(c.batch, c.dim, c.dstate, c.seqlen, c.io_dtype,
+                                         c.bc_dtype, rows=rows, flags=flags)
+    ws = torch.empty(max(need, 1), dtype=torch.uint8, device="cuda")
+    h2d = sum(t.numel() * t.element_size() for t in host.values() if t is not None)
     h2d += 0 if h0_h is None else h0_h.numel() * h0_h.element_size()
     d2h = out_h.numel() * out_h.element_size() + last_h.numel() * last_h.element_size()
 
     def step():
-        for k in names:
-            x[k].copy_(host[k], non_blocking=True)
-        if h0_h is not None:
-            w.h0.copy_(h0_h, non_blocking=True)
-        w.scan()
-        out_h.copy_(w.out, non_blocking=True)
-        last_h.copy_(w.last, non_blocking=True)
+        ops.selective_scan_fwd_host(host["u"], host["delta"], host["A"], host["B"], host["C"],
+                                    D=host["D"], z=host["z"], delta_bias=host["delta_bias"],
+                                    softplus=True, out=out_h, last_state=last_h, rows=rows,
+                                    workspace=ws, initial_state=h0_h, zoh=zoh)
 
     for _ in range(warmup):
         step()
@@ -286,7 +288,8 @@ def run_e2e(w: Workload, steps: int, warmup: int) -> dict:
     e.record()
     torch.cuda.synchronize()
     ms = max_over_ranks(s.elapsed_time(e))
-    return {"ms_total": ms, "steps": steps, "h2d": h2d, "d2h": d2h}
+    chunk_rows = rows if rows > 0 else max(1, (c.batch + 7) // 8)
+    return {"ms_total": ms, "steps": steps, "h2d": h2d, "d2h": d2h, "rows": chunk_rows}
 
 
 def cpu_baseline(w: Workload, target_s: float) -> dict:
@@ -453,12 +456,13 @@ def bench_ours(args, rank, world, local):
 
     e2e = None
     if not args.no_e2e and args.only != "decode":
-        r = run_e2e(w, max(1, min(K, args.e2e_steps)), 2)
+        r = run_e2e(w, max(1, min(K, args.e2e_steps)), 2, args.e2e_rows)
         e2e = {"value": round(job_gelem_per_s(world, elems, r["steps"], r["ms_total"]), 3),
                "unit": "Gelem/s", "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
                "steps": r["steps"],
-               "path": "pinned host u/delta/z/B/C -> device -> mamba_selective_scan_fwd -> "
-                       "out/last_state to pinned host, one stream"}
+               "path": "mamba_selective_scan_fwd_host: pinned host u/delta/z/B/C/A/D/bias -> "
+                       f"device in chunks of {r['rows']} batch rows, scans overlapped with the "
+                       "copies in and out -> out/last_state in pinned host memory"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.only != "decode":
@@ -553,6 +557,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--e2e-rows", type=int, default=0,
+                    help="batch rows per chunk of the host-buffer call (0: automatic)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,

@@ -220,6 +220,46 @@ MAMBA_API mamba_status_t mamba_selective_scan_fwd_with_state(
     cudaStream_t stream);
 
 /*
+ * Selective scan forward over HOST buffers, with the copies pipelined.
+ *
+ * For callers whose activations live in host memory: the batch is cut into
+ * chunks of `rows` batch rows; while chunk c is scanned, chunk c+1 is being
+ * copied in and chunk c-1 copied out, on two internal streams, so that the
+ * host-to-device and device-to-host transfers (the bound for this use) run at
+ * the same time and hide the scan.  Each chunk is one scan over its rows,
+ * identical in definition to mamba_selective_scan_fwd_with_state.
+ *   u, delta, z, B, C, A, D, delta_bias, initial_state     HOST pointers (read)
+ *   out, last_state                                        HOST pointers (written)
+ *     Same shapes, dtypes, optional (NULL) arguments and meaning as in
+ *     mamba_selective_scan_fwd_with_state.  Page-locked (pinned) host memory
+ *     is needed for the copies to overlap; pageable memory gives the same
+ *     results, without the overlap.
+ *   rows               batch rows per chunk; 0 = automatic (about 8 chunks)
+ *   dims->workspace    DEVICE scratch of at least
+ *                      mamba_selective_scan_host_workspace_bytes(dims, rows)
+ *                      bytes, 256-byte aligned: three chunk stages (their
+ *                      inputs, outputs and scan scratch) and A, D, delta_bias.
+ *   stream             the scans run on it; the call is ordered after earlier
+ *                      work on `stream`, and later work on `stream` is ordered
+ *                      after the last copy back to the host.  The call returns
+ *                      once everything is enqueued; host results are complete
+ *                      when `stream` has been synchronised.
+ * The two copy streams and their events are created on first use per device
+ * and kept; enqueueing is serialised by a lock, so calls from several host
+ * threads are safe but do not overlap each other's copies.
+ * Returns MAMBA_ERR_INVALID_ARG for rows < 0 or missing required pointers,
+ * MAMBA_ERR_WORKSPACE if the workspace is missing or too small.
+ * The paper has no counterpart; it is the host side of the same scan.
+ */
+MAMBA_API size_t mamba_selective_scan_host_workspace_bytes(const mamba_dims_t *dims, int64_t rows);
+
+MAMBA_API mamba_status_t mamba_selective_scan_fwd_host(
+    const void *u, const void *delta, const float *A, const void *B, const void *C,
+    const float *D, const void *z, const float *delta_bias, int softplus,
+    const float *initial_state, void *out, float *last_state, int64_t rows,
+    const mamba_dims_t *dims, cudaStream_t stream);
+
+/*
  * Selective scan forward that allocates nothing and takes no workspace.
  *
  * The paper has no counterpart to this entry point; it is a deployment aid.

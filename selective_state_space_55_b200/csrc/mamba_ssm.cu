@@ -599,6 +599,234 @@ MAMBA_API mamba_status_t mamba_selective_scan_fwd_noalloc(
                                     &local, stream);
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Scan over host buffers (mamba_selective_scan_fwd_host): chunks of batch rows
+// flow through three device stages; copies in run on one internal stream,
+// scans on the caller's stream, copies out on a second internal stream.
+
+namespace {
+
+constexpr int kHostStages = 3;
+
+// Device scratch of the host pipeline (offsets in bytes).
+struct HostLayout {
+    size_t a, d, bias;                                   // parameters, copied once
+    size_t stage0, stage_bytes;                          // first stage, stage stride
+    size_t u, delta, z, out, B, C, h0, last, scan;       // offsets inside a stage
+    size_t scan_bytes;
+    size_t total;
+    int64_t rows, nchunks;
+};
+
+int64_t host_chunk_rows(const mamba_dims_t* dims, int64_t rows) {
+    if (rows > 0) return std::min<int64_t>(rows, std::max<int64_t>(dims->batch, 1));
+    return std::max<int64_t>(1, (dims->batch + 7) / 8);   // about 8 chunks
+}
+
+mamba_status_t host_layout(const mamba_dims_t* dims, int64_t rows_req, int sms, HostLayout* L) {
+    *L = HostLayout{};
+    const int64_t rows = host_chunk_rows(dims, rows_req);
+    const size_t io = (size_t)dtype_bytes(dims->io_dtype), bc = (size_t)dtype_bytes(dims->bc_dtype);
+    const size_t Dm = (size_t)dims->dim, N = (size_t)dims->dstate, Ls = (size_t)dims->seqlen;
+    const size_t R = (size_t)rows;
+    size_t off = 0;
+    L->a = off;    off += align256(Dm * N * sizeof(float));
+    L->d = off;    off += align256(Dm * sizeof(float));
+    L->bias = off; off += align256(Dm * sizeof(float));
+    L->stage0 = off;
+    size_t s = 0;
+    const size_t act = R * Dm * Ls * io;
+    L->u = s;     s += align256(act);
+    L->delta = s; s += align256(act);
+    L->z = s;     s += align256(act);
+    L->out = s;   s += align256(act);
+    L->B = s;     s += align256(R * N * Ls * bc);
+    L->C = s;     s += align256(R * N * Ls * bc);
+    L->h0 = s;    s += align256(R * Dm * N * sizeof(float));
+    L->last = s;  s += align256(R * Dm * N * sizeof(float));
+    // Scan scratch: the larger of a full chunk's plan and the last chunk's.
+    size_t scan = 0;
+    const int64_t sizes[2] = {rows, dims->batch % rows};
+    for (int64_t r : sizes) {
+        if (r <= 0) continue;
+        mamba_dims_t cd = *dims;
+        cd.batch = r;
+        mamba_scan_plan_t plan;
+        const mamba_status_t st = plan_scan(&cd, sms, &plan);
+        if (st != MAMBA_OK) return st;
+        scan = std::max(scan, plan.workspace_bytes);
+    }
+    L->scan = s;
+    s += align256(scan);
+    L->scan_bytes = scan;
+    L->stage_bytes = s;
+    L->total = off + kHostStages * s;
+    L->rows = rows;
+    L->nchunks = (dims->batch + rows - 1) / rows;
+    return MAMBA_OK;
+}
+
+// Copy streams and events of the host pipeline, created once per device.
+struct HostPipe {
+    cudaStream_t h2d = nullptr;
+    cudaStream_t d2h = nullptr;
+    cudaEvent_t start = nullptr;
+    cudaEvent_t h2d_done[kHostStages] = {};
+    cudaEvent_t comp_done[kHostStages] = {};
+    cudaEvent_t d2h_done[kHostStages] = {};
+    bool ready = false;
+};
+
+std::mutex g_host_mutex;          // held while a call enqueues its work
+HostPipe g_host_pipe[kMaxDevices];
+
+// Called with g_host_mutex held and the device current.
+mamba_status_t host_pipe(int dev, HostPipe** out) {
+    if (dev < 0 || dev >= kMaxDevices) return MAMBA_ERR_CUDA;
+    HostPipe& p = g_host_pipe[dev];
+    if (!p.ready) {
+        HostPipe q;
+        bool ok = cudaStreamCreateWithFlags(&q.h2d, cudaStreamNonBlocking) == cudaSuccess &&
+                  cudaStreamCreateWithFlags(&q.d2h, cudaStreamNonBlocking) == cudaSuccess &&
+                  cudaEventCreateWithFlags(&q.start, cudaEventDisableTiming) == cudaSuccess;
+        for (int i = 0; ok && i < kHostStages; ++i)
+            ok = cudaEventCreateWithFlags(&q.h2d_done[i], cudaEventDisableTiming) == cudaSuccess &&
+                 cudaEventCreateWithFlags(&q.comp_done[i], cudaEventDisableTiming) == cudaSuccess &&
+                 cudaEventCreateWithFlags(&q.d2h_done[i], cudaEventDisableTiming) == cudaSuccess;
+        if (!ok) return MAMBA_ERR_CUDA;   // handles made so far are kept by the runtime until exit
+        q.ready = true;
+        p = q;
+    }
+    *out = &p;
+    return MAMBA_OK;
+}
+
+cudaError_t copy_async(void* dst, const void* src, size_t bytes, cudaMemcpyKind kind,
+                       cudaStream_t stream) {
+    if (bytes == 0 || src == nullptr || dst == nullptr) return cudaSuccess;
+    return cudaMemcpyAsync(dst, src, bytes, kind, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+MAMBA_API size_t mamba_selective_scan_host_workspace_bytes(const mamba_dims_t* dims, int64_t rows) {
+    if (check_dims(dims, true) != MAMBA_OK || rows < 0) return static_cast<size_t>(-1);
+    if (dims->batch * dims->dim == 0) return 0;
+    const int sms = current_sm_count(nullptr);
+    if (sms <= 0) return static_cast<size_t>(-1);
+    HostLayout L;
+    if (host_layout(dims, rows, sms, &L) != MAMBA_OK) return static_cast<size_t>(-1);
+    return L.total;
+}
+
+MAMBA_API mamba_status_t mamba_selective_scan_fwd_host(
+    const void* u, const void* delta, const float* A, const void* B, const void* C,
+    const float* D, const void* z, const float* delta_bias, int softplus,
+    const float* initial_state, void* out, float* last_state, int64_t rows,
+    const mamba_dims_t* dims, cudaStream_t stream) {
+    mamba_status_t st = check_dims(dims, true);
+    if (st != MAMBA_OK) return st;
+    if (rows < 0) return MAMBA_ERR_INVALID_ARG;
+    const int64_t chains = dims->batch * dims->dim;
+    if (chains == 0) return MAMBA_OK;
+    if (A == nullptr) return MAMBA_ERR_INVALID_ARG;
+    if (dims->seqlen > 0 &&
+        (u == nullptr || delta == nullptr || B == nullptr || C == nullptr || out == nullptr))
+        return MAMBA_ERR_INVALID_ARG;
+    const size_t state_bytes = (size_t)chains * dims->dstate * sizeof(float);
+    if (initial_state != nullptr && last_state != nullptr && initial_state != last_state) {
+        const uintptr_t a = reinterpret_cast<uintptr_t>(initial_state);
+        const uintptr_t b = reinterpret_cast<uintptr_t>(last_state);
+        if (a < b + state_bytes && b < a + state_bytes) return MAMBA_ERR_INVALID_ARG;
+    }
+    int dev = 0;
+    const int sms = current_sm_count(&dev);
+    if (sms <= 0) return MAMBA_ERR_CUDA;
+    HostLayout L;
+    st = host_layout(dims, rows, sms, &L);
+    if (st != MAMBA_OK) return st;
+    if (dims->workspace == nullptr || dims->workspace_bytes < L.total) return MAMBA_ERR_WORKSPACE;
+    if (!aligned(dims->workspace, 256)) return MAMBA_ERR_ALIGN;
+
+    std::lock_guard<std::mutex> lock(g_host_mutex);
+    HostPipe* pp = nullptr;
+    st = host_pipe(dev, &pp);
+    if (st != MAMBA_OK) return st;
+    uint8_t* ws = static_cast<uint8_t*>(dims->workspace);
+    const size_t io = (size_t)dtype_bytes(dims->io_dtype), bc = (size_t)dtype_bytes(dims->bc_dtype);
+    const size_t Dm = (size_t)dims->dim, N = (size_t)dims->dstate, Ls = (size_t)dims->seqlen;
+    float* dA = reinterpret_cast<float*>(ws + L.a);
+    float* dD = D ? reinterpret_cast<float*>(ws + L.d) : nullptr;
+    float* dbias = delta_bias ? reinterpret_cast<float*>(ws + L.bias) : nullptr;
+    auto fail = [](cudaError_t e) { return e == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA; };
+
+    // Parameters, on the scan stream ahead of every chunk.
+    cudaError_t e = copy_async(dA, A, Dm * N * sizeof(float), cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess) e = copy_async(dD, D, Dm * sizeof(float), cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess)
+        e = copy_async(dbias, delta_bias, Dm * sizeof(float), cudaMemcpyHostToDevice, stream);
+    // Both copy streams start after the earlier work on `stream`.
+    if (e == cudaSuccess) e = cudaEventRecord(pp->start, stream);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(pp->h2d, pp->start, 0);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(pp->d2h, pp->start, 0);
+    if (e != cudaSuccess) return MAMBA_ERR_CUDA;
+
+    const uint8_t* hu = static_cast<const uint8_t*>(u);
+    const uint8_t* hdelta = static_cast<const uint8_t*>(delta);
+    const uint8_t* hz = static_cast<const uint8_t*>(z);
+    const uint8_t* hB = static_cast<const uint8_t*>(B);
+    const uint8_t* hC = static_cast<const uint8_t*>(C);
+    uint8_t* hout = static_cast<uint8_t*>(out);
+    for (int64_t c = 0; c < L.nchunks; ++c) {
+        const int s = (int)(c % kHostStages);
+        const size_t b0 = (size_t)(c * L.rows);
+        const size_t r = (size_t)std::min<int64_t>(L.rows, dims->batch - (int64_t)b0);
+        uint8_t* stg = ws + L.stage0 + (size_t)s * L.stage_bytes;
+        const size_t act = r * Dm * Ls * io, act0 = b0 * Dm * Ls * io;
+        const size_t bcb = r * N * Ls * bc, bc0 = b0 * N * Ls * bc;
+        const size_t sb = r * Dm * N * sizeof(float), s0 = b0 * Dm * N;
+        // in: stage s is free once the scan of chunk c - 3 has read it
+        if (c >= kHostStages) e = cudaStreamWaitEvent(pp->h2d, pp->comp_done[s], 0);
+        if (e == cudaSuccess) e = copy_async(stg + L.u, hu ? hu + act0 : nullptr, act, cudaMemcpyHostToDevice, pp->h2d);
+        if (e == cudaSuccess) e = copy_async(stg + L.delta, hdelta ? hdelta + act0 : nullptr, act, cudaMemcpyHostToDevice, pp->h2d);
+        if (e == cudaSuccess) e = copy_async(stg + L.z, hz ? hz + act0 : nullptr, act, cudaMemcpyHostToDevice, pp->h2d);
+        if (e == cudaSuccess) e = copy_async(stg + L.B, hB ? hB + bc0 : nullptr, bcb, cudaMemcpyHostToDevice, pp->h2d);
+        if (e == cudaSuccess) e = copy_async(stg + L.C, hC ? hC + bc0 : nullptr, bcb, cudaMemcpyHostToDevice, pp->h2d);
+        if (e == cudaSuccess)
+            e = copy_async(stg + L.h0, initial_state ? initial_state + s0 : nullptr, sb, cudaMemcpyHostToDevice, pp->h2d);
+        if (e == cudaSuccess) e = cudaEventRecord(pp->h2d_done[s], pp->h2d);
+        // scan: after its inputs, and after chunk c - 3's outputs left stage s
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, pp->h2d_done[s], 0);
+        if (e == cudaSuccess && c >= kHostStages) e = cudaStreamWaitEvent(stream, pp->d2h_done[s], 0);
+        if (e != cudaSuccess) return MAMBA_ERR_CUDA;
+        mamba_dims_t cd = *dims;
+        cd.batch = (int64_t)r;
+        cd.workspace = stg + L.scan;
+        cd.workspace_bytes = L.scan_bytes;
+        st = mamba_selective_scan_fwd_with_state(
+            stg + L.u, stg + L.delta, dA, stg + L.B, stg + L.C, dD, z ? stg + L.z : nullptr, dbias,
+            softplus, initial_state ? reinterpret_cast<float*>(stg + L.h0) : nullptr, stg + L.out,
+            last_state ? reinterpret_cast<float*>(stg + L.last) : nullptr, &cd, stream);
+        if (st != MAMBA_OK) return st;
+        e = cudaEventRecord(pp->comp_done[s], stream);
+        // out: after the scan of chunk c
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(pp->d2h, pp->comp_done[s], 0);
+        if (e == cudaSuccess) e = copy_async(hout ? hout + act0 : nullptr, stg + L.out, act, cudaMemcpyDeviceToHost, pp->d2h);
+        if (e == cudaSuccess)
+            e = copy_async(last_state ? last_state + s0 : nullptr, stg + L.last, last_state ? sb : 0,
+                           cudaMemcpyDeviceToHost, pp->d2h);
+        if (e == cudaSuccess) e = cudaEventRecord(pp->d2h_done[s], pp->d2h);
+        if (e != cudaSuccess) return MAMBA_ERR_CUDA;
+    }
+    // Later work on `stream` follows the last copy back (the copy-in stream
+    // already joined it through the scans' waits).
+    return fail(cudaStreamWaitEvent(stream, pp->d2h_done[(L.nchunks - 1) % kHostStages], 0));
+}
+
 MAMBA_API mamba_status_t mamba_device_status(void) {
     if (cudaDeviceSynchronize() != cudaSuccess) return MAMBA_ERR_CUDA;
     int code = 0;

@@ -88,6 +88,11 @@ def library(path: Path | str | None = None) -> ctypes.CDLL:
     lib.mamba_selective_scan_fwd_with_state.restype = i32
     lib.mamba_selective_scan_fwd_with_state.argtypes = [
         vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, dims_p, vp]
+    lib.mamba_selective_scan_host_workspace_bytes.restype = ctypes.c_size_t
+    lib.mamba_selective_scan_host_workspace_bytes.argtypes = [dims_p, ctypes.c_int64]
+    lib.mamba_selective_scan_fwd_host.restype = i32
+    lib.mamba_selective_scan_fwd_host.argtypes = [
+        vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, ctypes.c_int64, dims_p, vp]
     lib.mamba_selective_state_update.restype = i32
     lib.mamba_selective_state_update.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, dims_p, vp]
     lib.mamba_device_status.restype = i32
@@ -118,6 +123,19 @@ def _check_cuda(name, t, dtypes, shape):
         return
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name}: dtype {t.dtype} not in {dtypes}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)} != {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _check_host(name, t, dtypes, shape):
+    if t is None:
+        return
+    if t.device.type != "cpu":
+        raise ValueError(f"{name} must be a host (CPU) tensor")
     if t.dtype not in dtypes:
         raise ValueError(f"{name}: dtype {t.dtype} not in {dtypes}")
     if tuple(t.shape) != tuple(shape):
@@ -213,6 +231,68 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softp
             ctypes.byref(dims), _stream_handle(stream))
     if rc != MAMBA_OK:
         raise MambaError(name, rc)
+    if last_state is not None:
+        return out, last_state
+    return out
+
+
+def scan_host_workspace_bytes(batch, dim, dstate, seqlen, io_dtype=torch.bfloat16,
+                              bc_dtype=torch.bfloat16, rows=0, num_chunks=0, flags=0) -> int:
+    """Device scratch bytes of ``selective_scan_fwd_host`` on the current device."""
+    dims = make_scan_dims(batch, dim, dstate, seqlen, io_dtype, bc_dtype, num_chunks, flags)
+    n = library().mamba_selective_scan_host_workspace_bytes(ctypes.byref(dims), rows)
+    if n == ctypes.c_size_t(-1).value:
+        raise MambaError("mamba_selective_scan_host_workspace_bytes", -1)
+    return int(n)
+
+
+def selective_scan_fwd_host(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
+                            out=None, last_state=None, return_last_state=False, rows=0,
+                            num_chunks=0, flags=0, workspace=None, stream=None,
+                            initial_state=None, zoh=False, device=None):
+    """Selective scan over HOST tensors through ``mamba_selective_scan_fwd_host``.
+
+    Every tensor argument is a contiguous CPU tensor (page-locked for the copies
+    to overlap the scans), with the shapes and dtypes of ``selective_scan_fwd``.
+    ``rows`` batch rows go through the device per chunk (0: automatic).
+    ``workspace`` is a device uint8 tensor of at least ``scan_host_workspace_bytes``
+    (allocated on ``device``, default the current CUDA device, when None).
+    The call returns once the work is enqueued on ``stream``; synchronise it
+    before reading ``out`` / ``last_state``.  Returns ``out`` (and the last
+    state, as ``selective_scan_fwd`` does).
+    """
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    io, bc = u.dtype, B.dtype
+    _check_host("u", u, (torch.float32, torch.bfloat16), (batch, dim, L))
+    _check_host("delta", delta, (io,), (batch, dim, L))
+    _check_host("z", z, (io,), (batch, dim, L))
+    _check_host("A", A, (torch.float32,), (dim, N))
+    _check_host("B", B, (torch.float32, torch.bfloat16), (batch, N, L))
+    _check_host("C", C, (bc,), (batch, N, L))
+    _check_host("D", D, (torch.float32,), (dim,))
+    _check_host("delta_bias", delta_bias, (torch.float32,), (dim,))
+    _check_host("initial_state", initial_state, (torch.float32,), (batch, dim, N))
+    pin = torch.cuda.is_available()
+    if out is None:
+        out = torch.empty(u.shape, dtype=io, pin_memory=pin)
+    _check_host("out", out, (io,), (batch, dim, L))
+    if last_state is None and return_last_state:
+        last_state = torch.empty((batch, dim, N), dtype=torch.float32, pin_memory=pin)
+    _check_host("last_state", last_state, (torch.float32,), (batch, dim, N))
+    if zoh:
+        flags |= MAMBA_FLAG_ZOH
+    if workspace is None:
+        need = scan_host_workspace_bytes(batch, dim, N, L, io, bc, rows, num_chunks, flags)
+        dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    dims = make_scan_dims(batch, dim, N, L, io, bc, num_chunks, flags, workspace)
+    rc = library().mamba_selective_scan_fwd_host(
+        _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
+        int(bool(softplus)), _ptr(initial_state), _ptr(out), _ptr(last_state), rows,
+        ctypes.byref(dims), _stream_handle(stream))
+    if rc != MAMBA_OK:
+        raise MambaError("mamba_selective_scan_fwd_host", rc)
     if last_state is not None:
         return out, last_state
     return out

@@ -103,6 +103,22 @@ def test_scan_with_state_rejects_bad_start_state(lib):
     assert _scan_h0(lib, _dims(dstate=17), ctypes.c_void_p(base), None) == -2
 
 
+def test_host_scan_rejects_bad_arguments(lib):
+    d = _dims()
+    call = lambda dims, rows, u=FAKE, A=FAKE, out=FAKE: lib.mamba_selective_scan_fwd_host(  # noqa: E731
+        u, FAKE, A, FAKE, FAKE, None, None, None, 1, None, out, None, rows,
+        ctypes.byref(dims) if dims is not None else None, None)
+    assert call(None, 0) == -1
+    assert call(d, -1) == -1                      # negative chunk size
+    assert call(d, 0, u=None) == -1               # missing input
+    assert call(d, 0, A=None) == -1
+    assert call(d, 0, out=None) == -1
+    assert call(_dims(dstate=17), 0) == -2
+    assert call(_dims(batch=0), 0) == 0           # empty problem: nothing to do
+    assert lib.mamba_selective_scan_host_workspace_bytes(ctypes.byref(d), -1) == \
+        ctypes.c_size_t(-1).value
+
+
 def test_scan_empty_batch_is_a_no_op(lib):
     assert _scan(lib, _dims(batch=0)) == 0
     assert _scan(lib, _dims(dim=0)) == 0
