@@ -17,6 +17,11 @@ term is the zero-order-hold one, expm1(Delta_t A_d,n) / A_d,n * B_t,n * u_t
 (Delta_t B_t,n u_t where A_d,n = 0), i.e. Bbar = (Delta A)^-1 (exp(Delta A) - I)
 Delta B for the diagonal A.
 
+The block's short causal convolution (depthwise, W taps, optional silu) and
+its single-token update are the plain weighted sums over the window ("Mamba 与
+状态空间模型", section 固定大小的状态: a short convolution keeps the 4 most
+recent inputs of each channel).
+
 Following "超越注意力：探索Mamba与状态空间模型" (sections 状态空间模型基础 for
 the zero-order hold, 选择性状态空间模型, 代码实现概览 for the Euler default) and
 "Mamba 与状态空间模型" (section 由词元决定).  The update is the same single step
@@ -85,6 +90,12 @@ class Oracle:
         self._lib.oracle_selective_state_update_ex_f64.restype = ctypes.c_int
         self._lib.oracle_selective_state_update_ex_f64.argtypes = [
             i64, i64, i64, dp, dp, dp, dp, dp, dp, dp, dp, dp, ci, ci, dp, dp]
+        self._lib.oracle_causal_conv1d_f64.restype = ctypes.c_int
+        self._lib.oracle_causal_conv1d_f64.argtypes = [
+            i64, i64, i64, i64, dp, dp, dp, dp, ci, dp, dp]
+        self._lib.oracle_causal_conv1d_update_f64.restype = ctypes.c_int
+        self._lib.oracle_causal_conv1d_update_f64.argtypes = [
+            i64, i64, i64, dp, dp, dp, dp, ci, dp, dp]
         self._lib.oracle_num_threads.restype = ctypes.c_int
         self._lib.oracle_num_threads.argtypes = []
 
@@ -142,6 +153,44 @@ class Oracle:
         if rc != 0:
             raise ValueError(f"oracle_selective_state_update_f64 returned {rc}")
         return new_state, out
+
+    def causal_conv1d(self, x, weight, bias=None, initial_conv_state=None, silu=True):
+        """Return (out, final_conv_state) as float64 arrays.
+
+        x: (batch, dim, L); weight: (dim, W); bias: (dim,); initial_conv_state:
+        (batch, dim, W), the W inputs before t = 0, oldest first (None: zeros).
+        final_conv_state: (batch, dim, W), the last W inputs.
+        """
+        x, weight = _f64(x), _f64(weight)
+        bias, init = _f64(bias), _f64(initial_conv_state)
+        batch, dim, seqlen = x.shape
+        width = weight.shape[1]
+        assert weight.shape == (dim, width)
+        assert bias is None or bias.shape == (dim,)
+        assert init is None or init.shape == (batch, dim, width)
+        out = np.empty_like(x)
+        final = np.empty((batch, dim, width), dtype=np.float64)
+        rc = self._lib.oracle_causal_conv1d_f64(batch, dim, seqlen, width, _ptr(x), _ptr(weight),
+                                                _ptr(bias), _ptr(init), int(bool(silu)),
+                                                _ptr(out), _ptr(final))
+        if rc != 0:
+            raise ValueError(f"oracle_causal_conv1d_f64 returned {rc}")
+        return out, final
+
+    def causal_conv1d_update(self, conv_state, x, weight, bias=None, silu=True):
+        """Return (new_conv_state, out) as float64 arrays; conv_state: (batch, dim, W)
+        is not modified; x: (batch, dim)."""
+        conv_state, x, weight, bias = _f64(conv_state), _f64(x), _f64(weight), _f64(bias)
+        batch, dim, width = conv_state.shape
+        assert x.shape == (batch, dim) and weight.shape == (dim, width)
+        new = np.empty_like(conv_state)
+        out = np.empty_like(x)
+        rc = self._lib.oracle_causal_conv1d_update_f64(batch, dim, width, _ptr(conv_state), _ptr(x),
+                                                       _ptr(weight), _ptr(bias), int(bool(silu)),
+                                                       _ptr(new), _ptr(out))
+        if rc != 0:
+            raise ValueError(f"oracle_causal_conv1d_update_f64 returned {rc}")
+        return new, out
 
 
 _DEFAULT: Oracle | None = None

@@ -37,6 +37,15 @@
  *  - The output gate y * silu(z) is the Mamba block's multiplicative gate; no
  *    page prints it.  silu(z) = z / (1 + exp(-z)).
  *
+ * The short causal convolution of the Mamba block ("Mamba 与状态空间模型",
+ * section 固定大小的状态: besides its 16 state numbers each channel keeps a
+ * short convolution over the 4 most recent inputs) is here too, as the plain
+ * weighted sum over a depthwise window of W taps:
+ *   out_t = act(bias_d + sum_{k<W} w_d,k x_{t-W+1+k}),  act = silu or identity,
+ * where x at negative times comes from a conv state holding the W most recent
+ * inputs, oldest first (zero when none is given).  The decode step shifts that
+ * state by one, appends x_t and applies the same sum.
+ *
  * Loops: chains (b, d) are independent; OpenMP splits them across threads.
  * Within a chain, t runs forward one step at a time and n ascends; nothing is
  * blocked, fused or reordered.
@@ -206,4 +215,70 @@ int oracle_selective_state_update_f64(int64_t batch, int64_t dim, int64_t dstate
 {
     return oracle_selective_state_update_ex_f64(batch, dim, dstate, state, x, dt, A, B, C, D, z,
                                                 dt_bias, dt_softplus, 0, new_state, out);
+}
+
+/* Input x_s of the conv window for chain `chain`: s >= 0 reads the sequence,
+ * s in [-W, -1] the initial conv state (index W + s), zero without one. */
+static double oracle_conv_input(const double *x_row, const double *state, int64_t chain,
+                                int64_t width, int64_t s)
+{
+    if (s >= 0)
+        return x_row[s];
+    return state ? state[chain * width + (width + s)] : 0.0;
+}
+
+int oracle_causal_conv1d_f64(int64_t batch, int64_t dim, int64_t seqlen, int64_t width,
+                             const double *x, const double *weight, const double *bias,
+                             const double *initial_conv_state, int silu, double *out,
+                             double *final_conv_state)
+{
+    if (batch < 0 || dim < 0 || seqlen < 0 || width < 1)
+        return -1;
+
+    int64_t chains = batch * dim;
+#pragma omp parallel for schedule(static)
+    for (int64_t chain = 0; chain < chains; ++chain) {
+        int64_t d = chain % dim;
+        const double *x_row = x + chain * seqlen;
+        double *out_row = out + chain * seqlen;
+        for (int64_t t = 0; t < seqlen; ++t) {
+            double acc = bias ? bias[d] : 0.0;
+            for (int64_t k = 0; k < width; ++k) {
+                int64_t s = t - (width - 1) + k;
+                acc += weight[d * width + k] *
+                       oracle_conv_input(x_row, initial_conv_state, chain, width, s);
+            }
+            out_row[t] = silu ? oracle_silu(acc) : acc;
+        }
+        if (final_conv_state)
+            for (int64_t j = 0; j < width; ++j)
+                final_conv_state[chain * width + j] =
+                    oracle_conv_input(x_row, initial_conv_state, chain, width, seqlen - width + j);
+    }
+    return 0;
+}
+
+int oracle_causal_conv1d_update_f64(int64_t batch, int64_t dim, int64_t width,
+                                    const double *conv_state, const double *x,
+                                    const double *weight, const double *bias, int silu,
+                                    double *new_conv_state, double *out)
+{
+    if (batch < 0 || dim < 0 || width < 1)
+        return -1;
+
+    int64_t chains = batch * dim;
+#pragma omp parallel for schedule(static)
+    for (int64_t chain = 0; chain < chains; ++chain) {
+        int64_t d = chain % dim;
+        const double *old = conv_state + chain * width;
+        double *cur = new_conv_state + chain * width;
+        for (int64_t j = 0; j + 1 < width; ++j)
+            cur[j] = old[j + 1];
+        cur[width - 1] = x[chain];
+        double acc = bias ? bias[d] : 0.0;
+        for (int64_t k = 0; k < width; ++k)
+            acc += weight[d * width + k] * cur[k];
+        out[chain] = silu ? oracle_silu(acc) : acc;
+    }
+    return 0;
 }

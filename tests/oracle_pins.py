@@ -467,6 +467,90 @@ def pin_update_zoh(o):
     _close(st, last, 1e-13, "zero-order-hold updates = scan: state")
 
 
+# ------------------------------------------------------------ short causal convolution
+# "Mamba 与状态空间模型", 固定大小的状态: each channel keeps a short convolution
+# over its 4 most recent inputs.  Conv state = the W most recent inputs, oldest first.
+
+def _silu(v):
+    return v / (1.0 + np.exp(-v))
+
+
+def pin_conv_one_hot_is_a_delay(o):
+    """A one-hot weight at tap k delays the input by W-1-k steps (zero before t = 0,
+    the initial conv state when one is given)."""
+    rng = np.random.default_rng(41)
+    for W in (2, 3, 4):
+        x = rng.standard_normal((2, 3, 11))
+        init = rng.standard_normal((2, 3, W))
+        for k in range(W):
+            w = np.zeros((3, W))
+            w[:, k] = 1.0
+            lag = W - 1 - k
+            out, _ = o.causal_conv1d(x, w, silu=False)
+            want = np.concatenate([np.zeros((2, 3, lag)), x[:, :, :x.shape[2] - lag]], axis=2)
+            _close(out, want, 0.0, f"conv delay W={W} k={k}")
+            out, _ = o.causal_conv1d(x, w, initial_conv_state=init, silu=False)
+            want = np.concatenate([init[:, :, W - lag:], x[:, :, :x.shape[2] - lag]], axis=2)
+            _close(out, want, 0.0, f"conv delay from state W={W} k={k}")
+
+
+def pin_conv_is_a_library_correlation(o):
+    """out = silu(bias + correlate(state[1:] ++ x, w, 'valid')) per channel (numpy's
+    correlation), and the final state is the last W inputs of state ++ x."""
+    rng = np.random.default_rng(42)
+    batch, dim, L, W = 2, 5, 23, 4
+    x = rng.standard_normal((batch, dim, L))
+    w = rng.standard_normal((dim, W))
+    bias = rng.standard_normal(dim)
+    init = rng.standard_normal((batch, dim, W))
+    out, final = o.causal_conv1d(x, w, bias=bias, initial_conv_state=init, silu=True)
+    want = np.zeros_like(x)
+    want_final = np.zeros((batch, dim, W))
+    for b in range(batch):
+        for d in range(dim):
+            xx = np.concatenate([init[b, d, 1:], x[b, d]])
+            want[b, d] = _silu(np.correlate(xx, w[d], mode="valid") + bias[d])
+            want_final[b, d] = np.concatenate([init[b, d], x[b, d]])[-W:]
+    _close(out, want, 1e-13, "conv = library correlation")
+    _close(final, want_final, 0.0, "conv final state")
+    short, final_short = o.causal_conv1d(x[:, :, :2], w, initial_conv_state=init, silu=False)
+    _close(final_short, np.concatenate([init, x[:, :, :2]], axis=2)[:, :, -W:], 0.0,
+           "conv final state, L < W")
+
+
+def pin_conv_silu_closed_values(o):
+    """Identity tap, no bias: out = silu(x) at silu(0) = 0, silu(+-ln 3) = 3/4 ln 3,
+    -1/4 ln 3, silu(40) = 40."""
+    ln3 = math.log(3.0)
+    x = np.array([0.0, ln3, -ln3, 40.0]).reshape(1, 1, 4)
+    out, _ = o.causal_conv1d(x, np.array([[0.0, 0.0, 0.0, 1.0]]), silu=True)
+    _close(out.reshape(-1), np.array([0.0, 0.75 * ln3, -0.25 * ln3, 40.0]), 1e-15,
+           "conv silu closed values")
+
+
+def pin_conv_updates_equal_prefill(o):
+    """T single-token updates from a conv state reproduce the prefill convolution over
+    the same T tokens from that state, outputs and final state; a prefill split in two
+    equals the whole."""
+    rng = np.random.default_rng(43)
+    batch, dim, T, W = 3, 4, 9, 4
+    x = rng.standard_normal((batch, dim, T))
+    w = rng.standard_normal((dim, W))
+    bias = rng.standard_normal(dim)
+    init = rng.standard_normal((batch, dim, W))
+    out, final = o.causal_conv1d(x, w, bias=bias, initial_conv_state=init, silu=True)
+    st = init.copy()
+    outs = np.zeros_like(x)
+    for t in range(T):
+        st, outs[:, :, t] = o.causal_conv1d_update(st, x[:, :, t], w, bias=bias, silu=True)
+    _close(outs, out, 1e-14, "conv updates = prefill: out")
+    _close(st, final, 0.0, "conv updates = prefill: state")
+    o1, f1 = o.causal_conv1d(x[:, :, :4], w, bias=bias, initial_conv_state=init, silu=True)
+    o2, f2 = o.causal_conv1d(x[:, :, 4:], w, bias=bias, initial_conv_state=f1, silu=True)
+    _close(np.concatenate([o1, o2], axis=2), out, 1e-14, "conv split prefill: out")
+    _close(f2, final, 0.0, "conv split prefill: state")
+
+
 PINS = {
     "unrolled_sum": pin_unrolled_sum,
     "gate_closed_values": pin_gate_closed_values,
@@ -487,4 +571,8 @@ PINS = {
     "initial_state_free_decay": pin_initial_state_free_decay,
     "initial_state_split": pin_initial_state_split,
     "update_zoh": pin_update_zoh,
+    "conv_one_hot_is_a_delay": pin_conv_one_hot_is_a_delay,
+    "conv_is_a_library_correlation": pin_conv_is_a_library_correlation,
+    "conv_silu_closed_values": pin_conv_silu_closed_values,
+    "conv_updates_equal_prefill": pin_conv_updates_equal_prefill,
 }

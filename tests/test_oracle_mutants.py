@@ -67,6 +67,20 @@ MUTANTS = [
      "h[n] = initial_state ? initial_state[(b * dim + d) * dstate + n] : 0.0;", "h[n] = 0.0;"),
     ("initial_state_transposed", "initial_state[(b * dim + d) * dstate + n]",
      "initial_state[(d * batch + b) * dstate + n]"),
+    # short causal convolution
+    ("conv_tap_off_by_one", "int64_t s = t - (width - 1) + k;", "int64_t s = t - width + k;"),
+    ("conv_state_index_shifted", "return state ? state[chain * width + (width + s)] : 0.0;",
+     "return state ? state[chain * width + (width + s + 1) % width] : 0.0;"),
+    ("conv_bias_dropped", "double acc = bias ? bias[d] : 0.0;\n            for",
+     "double acc = 0.0;\n            for"),
+    ("conv_silu_skipped", "out_row[t] = silu ? oracle_silu(acc) : acc;", "out_row[t] = acc;"),
+    ("conv_weight_transposed", "acc += weight[d * width + k] *\n", "acc += weight[k * dim + d] *\n"),
+    ("conv_final_state_reversed", "final_conv_state[chain * width + j] =",
+     "final_conv_state[chain * width + (width - 1 - j)] ="),
+    ("conv_update_not_shifted", "cur[j] = old[j + 1];", "cur[j] = old[j];"),
+    ("conv_update_x_not_appended", "cur[width - 1] = x[chain];", "cur[width - 1] = old[width - 1];"),
+    ("conv_update_bias_dropped", "double acc = bias ? bias[d] : 0.0;\n        for",
+     "double acc = 0.0;\n        for"),
 ]
 
 
