@@ -46,7 +46,22 @@
  * inputs, oldest first (zero when none is given).  The decode step shifts that
  * state by one, appends x_t and applies the same sum.
  *
- * Loops: chains (b, d) are independent; OpenMP splits them across threads.
+ * The backward pass (gradients of the scan) is the adjoint of the same
+ * recurrence, taken in reverse time ("Mamba 与状态空间模型", section
+ * 在芯片上扫过去: the intermediate states the backward pass needs are not kept
+ * but computed again).  With lambda_t = dLoss/dh_t (all paths through later
+ * steps included):
+ *   lambda_t,n = C_t,n dy_t + Abar_t+1,n lambda_t+1,n   (lambda_L-1 from dlast_state)
+ *   dC_t,n = dy_t h_t,n,  dB_t,n = lambda_t,n Delta_t u_t,
+ *   dDelta_t = sum_n lambda_t,n (B_t,n u_t + A_n Abar_t,n h_t-1,n),
+ *   dA_n = sum_t lambda_t,n Delta_t Abar_t,n h_t-1,n,
+ *   du_t = D dy_t + sum_n lambda_t,n Delta_t B_t,n,   dh_-1 = Abar_0 lambda_0,
+ * with dy = dout silu(z) and dz = dout y silu'(z) when gated, and the softplus
+ * derivative sigmoid(delta + bias) applied to dDelta.
+ *
+ * Loops: chains (b, d) are independent; OpenMP splits them across threads
+ * (the backward runs them in order, since its gradients of A, B, C, D and the
+ * bias sum over chains).
  * Within a chain, t runs forward one step at a time and n ascends; nothing is
  * blocked, fused or reordered.
  *
@@ -63,6 +78,7 @@
 #include <math.h>
 #include <stddef.h>
 #include <stdint.h>
+#include <stdlib.h>
 #ifdef _OPENMP
 #include <omp.h>
 #endif
@@ -280,5 +296,126 @@ int oracle_causal_conv1d_update_f64(int64_t batch, int64_t dim, int64_t width,
             acc += weight[d * width + k] * cur[k];
         out[chain] = silu ? oracle_silu(acc) : acc;
     }
+    return 0;
+}
+
+/* d silu / dz = sigmoid(z) (1 + z (1 - sigmoid(z))). */
+static double oracle_silu_grad(double z)
+{
+    double sg = 1.0 / (1.0 + exp(-z));
+    return sg * (1.0 + z * (1.0 - sg));
+}
+
+/* d softplus / ds = sigmoid(s). */
+static double oracle_softplus_grad(double s)
+{
+    return 1.0 / (1.0 + exp(-s));
+}
+
+/* Gradients of sum_t dout_t out_t + sum_n dlast_n last_state_n with respect to
+ * every input of oracle_selective_scan_ex_f64 (Euler input term).  Gradient
+ * outputs for NULL inputs may be NULL; all others are overwritten.  Returns
+ * -1 on a bad size, -2 if the scratch cannot be allocated. */
+int oracle_selective_scan_bwd_f64(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
+                                  const double *u, const double *delta, const double *A,
+                                  const double *B, const double *C, const double *D,
+                                  const double *z, const double *delta_bias, int softplus,
+                                  const double *initial_state, const double *dout,
+                                  const double *dlast_state, double *du, double *ddelta,
+                                  double *dA, double *dB, double *dC, double *dD, double *dz,
+                                  double *ddelta_bias, double *dinitial_state)
+{
+    if (batch < 0 || dim < 0 || seqlen < 0 || dstate < 1 || dstate > ORACLE_MAX_DSTATE)
+        return -1;
+    for (int64_t i = 0; i < dim * dstate; ++i)
+        dA[i] = 0.0;
+    for (int64_t i = 0; i < batch * dstate * seqlen; ++i) {
+        dB[i] = 0.0;
+        dC[i] = 0.0;
+    }
+    if (dD)
+        for (int64_t d = 0; d < dim; ++d)
+            dD[d] = 0.0;
+    if (ddelta_bias)
+        for (int64_t d = 0; d < dim; ++d)
+            ddelta_bias[d] = 0.0;
+    /* states h_t of one chain, t = -1 .. L-1 */
+    double *hs = malloc(sizeof(double) * (size_t)(seqlen + 1) * (size_t)dstate);
+    double *dts = malloc(sizeof(double) * (size_t)(seqlen > 0 ? seqlen : 1));
+    double *ys = malloc(sizeof(double) * (size_t)(seqlen > 0 ? seqlen : 1));
+    if (!hs || !dts || !ys) {
+        free(hs);
+        free(dts);
+        free(ys);
+        return -2;
+    }
+    for (int64_t chain = 0; chain < batch * dim; ++chain) {
+        int64_t b = chain / dim;
+        int64_t d = chain % dim;
+        const double *u_row = u + chain * seqlen;
+        const double *delta_row = delta + chain * seqlen;
+        /* forward, keeping every state */
+        for (int64_t n = 0; n < dstate; ++n)
+            hs[n] = initial_state ? initial_state[chain * dstate + n] : 0.0;
+        for (int64_t t = 0; t < seqlen; ++t) {
+            double s = delta_row[t] + (delta_bias ? delta_bias[d] : 0.0);
+            double dt = softplus ? oracle_softplus(s) : s;
+            dts[t] = dt;
+            double y = 0.0;
+            for (int64_t n = 0; n < dstate; ++n) {
+                double a_bar = exp(dt * A[d * dstate + n]);
+                double h = a_bar * hs[t * dstate + n] + dt * B[(b * dstate + n) * seqlen + t] * u_row[t];
+                hs[(t + 1) * dstate + n] = h;
+                y += C[(b * dstate + n) * seqlen + t] * h;
+            }
+            ys[t] = y + (D ? D[d] * u_row[t] : 0.0);
+        }
+        /* reverse */
+        double lam[ORACLE_MAX_DSTATE];
+        for (int64_t n = 0; n < dstate; ++n)
+            lam[n] = dlast_state ? dlast_state[chain * dstate + n] : 0.0;
+        for (int64_t t = seqlen - 1; t >= 0; --t) {
+            double g = dout[chain * seqlen + t];
+            double dy = g;
+            if (z) {
+                double zt = z[chain * seqlen + t];
+                dy = g * oracle_silu(zt);
+                if (dz)
+                    dz[chain * seqlen + t] = g * ys[t] * oracle_silu_grad(zt);
+            }
+            double x = u_row[t];
+            double dt = dts[t];
+            double dut = D ? dy * D[d] : 0.0;
+            if (dD)
+                dD[d] += dy * x;
+            double ddt = 0.0;
+            for (int64_t n = 0; n < dstate; ++n) {
+                double b_tn = B[(b * dstate + n) * seqlen + t];
+                double c_tn = C[(b * dstate + n) * seqlen + t];
+                double a_dn = A[d * dstate + n];
+                double a_bar = exp(dt * a_dn);
+                double h_prev = hs[t * dstate + n];
+                lam[n] += c_tn * dy;
+                dC[(b * dstate + n) * seqlen + t] += dy * hs[(t + 1) * dstate + n];
+                dB[(b * dstate + n) * seqlen + t] += lam[n] * dt * x;
+                ddt += lam[n] * (b_tn * x + a_dn * a_bar * h_prev);
+                dA[d * dstate + n] += lam[n] * dt * a_bar * h_prev;
+                dut += lam[n] * dt * b_tn;
+                lam[n] *= a_bar;
+            }
+            du[chain * seqlen + t] = dut;
+            double s = delta_row[t] + (delta_bias ? delta_bias[d] : 0.0);
+            double ds = softplus ? ddt * oracle_softplus_grad(s) : ddt;
+            ddelta[chain * seqlen + t] = ds;
+            if (ddelta_bias)
+                ddelta_bias[d] += ds;
+        }
+        if (dinitial_state)
+            for (int64_t n = 0; n < dstate; ++n)
+                dinitial_state[chain * dstate + n] = lam[n];
+    }
+    free(hs);
+    free(dts);
+    free(ys);
     return 0;
 }

@@ -551,6 +551,75 @@ def pin_conv_updates_equal_prefill(o):
     _close(f2, final, 0.0, "conv split prefill: state")
 
 
+# ------------------------------------------------------------ backward pass
+# "Mamba 与状态空间模型", 在芯片上扫过去: training back-propagates through the
+# scan (recomputing the states).  The gradients are pinned to central finite
+# differences of the forward oracle, which its own pins fix.
+
+def _bwd_problem(seed, gated=True):
+    rng = np.random.default_rng(seed)
+    batch, dim, N, L = 2, 3, 3, 10
+    p = dict(
+        u=rng.standard_normal((batch, dim, L)),
+        delta=rng.standard_normal((batch, dim, L)) * 0.7,
+        A=-rng.uniform(0.3, 1.5, (dim, N)),
+        B=rng.standard_normal((batch, N, L)) * 0.5,
+        C=rng.standard_normal((batch, N, L)) * 0.5,
+    )
+    if gated:
+        p.update(D=rng.standard_normal(dim), z=rng.standard_normal((batch, dim, L)),
+                 delta_bias=rng.uniform(-0.5, 0.5, dim),
+                 initial_state=rng.standard_normal((batch, dim, N)))
+    dout = rng.standard_normal((batch, dim, L))
+    dlast = rng.standard_normal((batch, dim, N)) if gated else None
+    return p, dout, dlast
+
+
+def _fd_check(o, p, dout, dlast, softplus, what):
+    def loss(q):
+        out, last = o.selective_scan(q["u"], q["delta"], q["A"], q["B"], q["C"], D=q.get("D"),
+                                     z=q.get("z"), delta_bias=q.get("delta_bias"),
+                                     softplus=softplus, initial_state=q.get("initial_state"))
+        val = float(np.sum(dout * out))
+        if dlast is not None:
+            val += float(np.sum(dlast * last))
+        return val
+
+    g = o.selective_scan_bwd(p["u"], p["delta"], p["A"], p["B"], p["C"], dout, D=p.get("D"),
+                             z=p.get("z"), delta_bias=p.get("delta_bias"), softplus=softplus,
+                             initial_state=p.get("initial_state"), dlast_state=dlast)
+    names = {"u": "du", "delta": "ddelta", "A": "dA", "B": "dB", "C": "dC", "D": "dD",
+             "z": "dz", "delta_bias": "ddelta_bias", "initial_state": "dinitial_state"}
+    for key, gname in names.items():
+        if key not in p:
+            assert gname not in g
+            continue
+        want = np.zeros_like(p[key])
+        for idx in np.ndindex(p[key].shape):
+            x0 = p[key][idx]
+            eps = 1e-6 * max(1.0, abs(x0))
+            q = {k: v.copy() for k, v in p.items()}
+            q[key][idx] = x0 + eps
+            lp = loss(q)
+            q[key][idx] = x0 - eps
+            lm = loss(q)
+            want[idx] = (lp - lm) / (2 * eps)
+        _close(g[gname], want, 2e-6, f"{what}: {gname} vs finite differences")
+
+
+def pin_bwd_finite_differences_gated(o):
+    """Every gradient (u, delta, A, B, C, D, z, bias, start state) with the gate,
+    softplus, a start state and a last-state term, against central differences."""
+    p, dout, dlast = _bwd_problem(51, gated=True)
+    _fd_check(o, p, dout, dlast, True, "gated backward")
+
+
+def pin_bwd_finite_differences_plain(o):
+    """The same without gate, D, bias, start state or last-state term, softplus off."""
+    p, dout, dlast = _bwd_problem(52, gated=False)
+    _fd_check(o, p, dout, dlast, False, "plain backward")
+
+
 PINS = {
     "unrolled_sum": pin_unrolled_sum,
     "gate_closed_values": pin_gate_closed_values,
@@ -575,4 +644,6 @@ PINS = {
     "conv_is_a_library_correlation": pin_conv_is_a_library_correlation,
     "conv_silu_closed_values": pin_conv_silu_closed_values,
     "conv_updates_equal_prefill": pin_conv_updates_equal_prefill,
+    "bwd_finite_differences_gated": pin_bwd_finite_differences_gated,
+    "bwd_finite_differences_plain": pin_bwd_finite_differences_plain,
 }

@@ -81,6 +81,24 @@ MUTANTS = [
     ("conv_update_x_not_appended", "cur[width - 1] = x[chain];", "cur[width - 1] = old[width - 1];"),
     ("conv_update_bias_dropped", "double acc = bias ? bias[d] : 0.0;\n        for",
      "double acc = 0.0;\n        for"),
+    # backward pass
+    ("bwd_lambda_not_propagated", "lam[n] *= a_bar;", "lam[n] *= 1.0;"),
+    ("bwd_dC_uses_previous_state", "+= dy * hs[(t + 1) * dstate + n];", "+= dy * hs[t * dstate + n];"),
+    ("bwd_dA_missing_delta", "dA[d * dstate + n] += lam[n] * dt * a_bar * h_prev;",
+     "dA[d * dstate + n] += lam[n] * a_bar * h_prev;"),
+    ("bwd_softplus_grad_skipped", "double ds = softplus ? ddt * oracle_softplus_grad(s) : ddt;",
+     "double ds = ddt;"),
+    ("bwd_silu_grad_is_sigmoid", "return sg * (1.0 + z * (1.0 - sg));", "return sg;"),
+    ("bwd_ddelta_A_term_sign", "ddt += lam[n] * (b_tn * x + a_dn * a_bar * h_prev);",
+     "ddt += lam[n] * (b_tn * x - a_dn * a_bar * h_prev);"),
+    ("bwd_du_missing_D", "double dut = D ? dy * D[d] : 0.0;", "double dut = 0.0;"),
+    ("bwd_dB_missing_u", "+= lam[n] * dt * x;", "+= lam[n] * dt;"),
+    ("bwd_dlast_ignored", "lam[n] = dlast_state ? dlast_state[chain * dstate + n] : 0.0;",
+     "lam[n] = 0.0;"),
+    ("bwd_readout_grad_ungated", "dy = g * oracle_silu(zt);", "dy = g;"),
+    ("bwd_dD_uses_dout", "dD[d] += dy * x;", "dD[d] += g * x;"),
+    ("bwd_dh0_one_step_late", "dinitial_state[chain * dstate + n] = lam[n];",
+     "dinitial_state[chain * dstate + n] = lam[n] * exp(dts[0] * A[d * dstate + n]);"),
 ]
 
 
