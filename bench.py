@@ -220,10 +220,13 @@ class Workload:
                                     last_state=self.last, workspace=self.ws, **self.scan_kwargs())
 
     def decode_layers(self):
+        # Each layer updates its own state, so a layer's launch may overlap the
+        # previous layer's (programmatic dependent launch, MAMBA_FLAG_PDL).
         for lay, tok, out in zip(self.layers, self.toks, self.douts):
             self.ops.selective_state_update(lay["state"], tok["x"], tok["dt"], lay["A"], tok["B"],
                                             tok["C"], D=lay["D"], z=tok["z"],
-                                            dt_bias=lay["dt_bias"], out=out)
+                                            dt_bias=lay["dt_bias"], out=out,
+                                            flags=self.ops.MAMBA_FLAG_PDL)
 
     def capture_decode(self):
         """Capture the 48 state-update launches of one token in a CUDA graph."""
@@ -441,7 +444,8 @@ def bench_ours(args, rank, world, local):
                    "traffic": recorded_traffic("state_update_bulk_kernel", digest)}
     decode = {
         "workload": f"decode_b128: {d.layers} layers x state ({d.batch}, {d.dim}, {d.dstate}) fp32, "
-                    "bf16 x/dt/z/B/C/out, one CUDA graph per token",
+                    "bf16 x/dt/z/B/C/out, one CUDA graph per token, each layer's launch a "
+                    "programmatic dependent launch (MAMBA_FLAG_PDL: distinct states per layer)",
         "us_per_token_step": round(decode_step_us, 2),
         "us_per_layer": round(decode_step_us / d.layers, 3),
         "roofline": decode_roof,
@@ -501,6 +505,97 @@ def bench_ours(args, rank, world, local):
                                     "scan_workload": args.scan_workload,
                                     "scan_variant": args.scan_variant,
                                     "note": "profiling case, not the benchmark workload"}
+        print(json.dumps(line), flush=True)
+
+
+def bench_conv(args, rank, world, local):
+    """Measurement case: the block's short causal convolution (W = 4, bf16) on the
+    Mamba-2.8B layer shape (prefill) and 48 decode layers of batch 128 x 4096
+    (one CUDA graph per token), each against the HBM roofline."""
+    global _WORLD
+    _WORLD = world
+    from selective_state_space_55_b200 import build as cuda_build
+    from selective_state_space_55_b200 import inputs as I
+    from selective_state_space_55_b200 import ops
+
+    if rank == 0:
+        cuda_build.build()
+    barrier()
+    torch.cuda.set_device(local)
+    c, d, W, bf = I.SCAN_CONFIGS[SCAN_WORKLOAD], I.DECODE_CONFIG, 4, torch.bfloat16
+    g = torch.Generator(device="cuda")
+    g.manual_seed(rank_seed(rank) + 11)
+    x = torch.randn(c.batch, c.dim, c.seqlen, generator=g, device="cuda").to(bf)
+    w = torch.randn(c.dim, W, generator=g, device="cuda") / W
+    bias = torch.randn(c.dim, generator=g, device="cuda")
+    out = torch.empty_like(x)
+    fin = torch.empty(c.batch, c.dim, W, dtype=bf, device="cuda")
+    lay = [dict(st=torch.randn(d.batch, d.dim, W, generator=g, device="cuda").to(bf),
+                x=torch.randn(d.batch, d.dim, generator=g, device="cuda").to(bf),
+                w=torch.randn(d.dim, W, generator=g, device="cuda") / W,
+                b=torch.randn(d.dim, generator=g, device="cuda"),
+                out=torch.empty(d.batch, d.dim, dtype=bf, device="cuda")) for _ in range(d.layers)]
+
+    def prefill():
+        ops.causal_conv1d_fwd(x, w, bias=bias, out=out, final_conv_state=fin)
+
+    def decode():
+        for ly in lay:
+            ops.causal_conv1d_update(ly["st"], ly["x"], ly["w"], bias=ly["b"], out=ly["out"])
+
+    decode()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        decode()
+    for _ in range(args.warmup):
+        prefill()
+        graph.replay()
+    torch.cuda.synchronize()
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    sampler = ClockSampler(local)
+    sampler.start()
+    barrier()
+    torch.cuda.synchronize()
+    t0 = time.time()
+    for e0, e1, e2 in ev:
+        e0.record()
+        prefill()
+        e1.record()
+        graph.replay()
+        e2.record()
+    torch.cuda.synchronize()
+    t1 = time.time()
+    barrier()
+    sampler.stop()
+    pre_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b, _ in ev)) / K
+    dec_ms = max_over_ranks(sum(b.elapsed_time(e) for _, b, e in ev)) / K
+    chains_p, chains_d = c.batch * c.dim, d.batch * d.dim
+    pre_bytes = c.elements * 2 * 2 + chains_p * W * 2 + c.dim * (W + 1) * 4
+    dec_bytes = chains_d * (2 * W * 2 + 2 * 2) + d.dim * (W + 1) * 4        # per layer
+    peaks = measured_peaks()
+    pre_gbs = pre_bytes / (pre_ms * 1e-3) / 1e9
+    dec_gbs = dec_bytes * d.layers / (dec_ms * 1e-3) / 1e9
+    if rank == 0:
+        line = {
+            "metric": "causal conv1d GB/s (prefill, Mamba-2.8B layer shape)", "value": round(world * pre_gbs, 1),
+            "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": round(pre_ms + dec_ms, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded)",
+            "config": {"workload": f"causal conv1d W={W} bf16: prefill ({c.batch}x{c.dim}x{c.seqlen}) "
+                                   f"+ decode update ({d.layers} layers x {d.batch}x{d.dim}, CUDA graph)"},
+            "prefill": {"ms": round(pre_ms, 4), "bytes": pre_bytes,
+                        "roofline": {"bound": "hbm", "achieved": round(pre_gbs, 1), "peak": peaks["hbm_gbs"],
+                                     "unit": "GB/s", "frac": round(pre_gbs / peaks["hbm_gbs"], 4)}},
+            "decode": {"us_per_layer": round(dec_ms * 1e3 / d.layers, 3), "bytes_per_layer": dec_bytes,
+                       "roofline": {"bound": "hbm", "achieved": round(dec_gbs, 1), "peak": peaks["hbm_gbs"],
+                                    "unit": "GB/s", "frac": round(dec_gbs / peaks["hbm_gbs"], 4)}},
+            "gpu_launches": K * (1 + 1 + d.layers),
+            "clocks": sampler.summary(t0, t1),
+            "partial_case": {"only": "conv", "note": "measurement of the short convolution, not the benchmark workload"},
+        }
         print(json.dumps(line), flush=True)
 
 
@@ -565,8 +660,8 @@ def main():
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--reference-seconds", type=float, default=120.0,
                     help="budget of the whole --impl reference run")
-    ap.add_argument("--only", choices=["scan", "decode"], default=None,
-                    help="profiling case: run one half of the step")
+    ap.add_argument("--only", choices=["scan", "decode", "conv"], default=None,
+                    help="profiling case: one half of the step; conv: the short convolution")
     ap.add_argument("--scan-batch", type=int, default=None,
                     help="profiling case: smaller scan batch")
     ap.add_argument("--decode-layers", type=int, default=None,
@@ -597,7 +692,10 @@ def main():
             "nccl", timeout=datetime.timedelta(seconds=300),
             device_id=torch.device("cuda", local))
     try:
-        bench_ours(args, rank, world, local)
+        if args.only == "conv":
+            bench_conv(args, rank, world, local)
+        else:
+            bench_ours(args, rank, world, local)
     finally:
         if world > 1:
             torch.distributed.destroy_process_group()

@@ -6,6 +6,9 @@
  *   mamba_selective_scan_fwd      the selective scan over a whole sequence
  *   mamba_selective_state_update  one token of generation (recurrent mode)
  *
+ * and, next to them, the block's short causal convolution (prefill and decode
+ * update) that produces the scan's input.
+ *
  * Definition (per batch b, channel d, state index n, time t):
  *
  *   Delta_t  = softplus(delta_t + delta_bias_d)      (or without softplus)
@@ -95,6 +98,14 @@ typedef enum {
  * then runs a kernel instance with 1/A held in registers (fewer resident
  * warps); results follow the same tolerance as the Euler path. */
 #define MAMBA_FLAG_ZOH 0x8
+/* Update only: launch the streaming kernel as a programmatic dependent launch,
+ * so that it may start while the previous kernel on the stream finishes.  It
+ * reads its own state before waiting for that kernel, and x, dt, z, B, C after
+ * it completes.  Set it only when the previous kernel on the stream does not
+ * write this call's state, as when consecutive calls update the states of
+ * different layers; then results are identical with and without the flag.
+ * Paths other than the streaming one ignore it. */
+#define MAMBA_FLAG_PDL 0x10
 
 #define MAMBA_MAX_DSTATE 16
 
@@ -316,6 +327,52 @@ MAMBA_API mamba_status_t mamba_selective_state_update(float *state, const void *
                                                       const float *dt_bias, void *out,
                                                       const mamba_dims_t *dims,
                                                       cudaStream_t stream);
+
+/*
+ * Short causal convolution of the Mamba block.
+ *
+ * Besides its 16 state numbers, each channel keeps a short convolution over
+ * its most recent inputs ("Mamba 与状态空间模型", section 固定大小的状态: 4 of
+ * them in Mamba-2.8B).  Per channel d, with W = width taps:
+ *
+ *   out_t = act(bias_d + sum_{k<W} weight_d,k * x_{t-W+1+k}),   act = silu or identity
+ *
+ * where x at negative times comes from a conv state holding the W most recent
+ * inputs, oldest first (zero when no state is given).  In the block the conv
+ * output feeds the projections that produce Delta, B and C, so it runs before
+ * the scan (prefill) or the state update (decode), not inside them.
+ *
+ * mamba_causal_conv1d_fwd (prefill over a sequence)
+ *   x, out              (batch, dim, seqlen), io_dtype; out must not alias x
+ *   weight              (dim, width) fp32;  bias (dim,) fp32 or NULL
+ *   initial_conv_state  (batch, dim, width), io_dtype, or NULL (zeros)
+ *   final_conv_state    (batch, dim, width), io_dtype, or NULL: the last
+ *                       width inputs of (initial state ++ x); may be the
+ *                       initial_conv_state buffer itself (partial overlap:
+ *                       MAMBA_ERR_INVALID_ARG)
+ *   silu                nonzero: act = silu
+ * mamba_causal_conv1d_update (one token of generation)
+ *   conv_state          (batch, dim, width), io_dtype, updated in place: shifted
+ *                       by one with x appended, then used for the sum
+ *   x, out              (batch, dim), io_dtype
+ * dims: batch, dim, seqlen (prefill) and io_dtype are read; dstate, bc_dtype
+ * and the workspace are ignored.  width must be 1..MAMBA_MAX_CONV_WIDTH
+ * (MAMBA_ERR_UNSUPPORTED otherwise).  Both calls are asynchronous on `stream`
+ * and allocate nothing.
+ */
+#define MAMBA_MAX_CONV_WIDTH 4
+
+MAMBA_API mamba_status_t mamba_causal_conv1d_fwd(const void *x, const float *weight,
+                                                 const float *bias,
+                                                 const void *initial_conv_state, int width,
+                                                 int silu, void *out, void *final_conv_state,
+                                                 const mamba_dims_t *dims, cudaStream_t stream);
+
+MAMBA_API mamba_status_t mamba_causal_conv1d_update(void *conv_state, const void *x,
+                                                    const float *weight, const float *bias,
+                                                    int width, int silu, void *out,
+                                                    const mamba_dims_t *dims,
+                                                    cudaStream_t stream);
 
 /*
  * Read and clear the library's device-side status word on the current device

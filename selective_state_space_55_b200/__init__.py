@@ -2,15 +2,18 @@
 
 The computation lives in ``libmamba_ssm.so`` (hand-written CUDA behind the C
 ABI of ``include/mamba_ssm.h``); ``ops`` is its ctypes binding and ``inputs``
-the seeded synthetic workloads.
+the seeded synthetic workloads.  Besides the scan and the update, the library
+holds the scan over host buffers and the block's short causal convolution.
 """
 from . import inputs  # noqa: F401
 from .ops import (  # noqa: F401
-    MambaError, device_status, scan_plan, scan_workspace_bytes, selective_scan_fwd,
+    MambaError, causal_conv1d_fwd, causal_conv1d_update, device_status, scan_host_workspace_bytes,
+    scan_plan, scan_workspace_bytes, selective_scan_fwd, selective_scan_fwd_host,
     selective_state_update, status_string, version,
 )
 
 __all__ = [
-    "inputs", "MambaError", "device_status", "scan_plan", "scan_workspace_bytes",
-    "selective_scan_fwd", "selective_state_update", "status_string", "version",
+    "inputs", "MambaError", "causal_conv1d_fwd", "causal_conv1d_update", "device_status",
+    "scan_host_workspace_bytes", "scan_plan", "scan_workspace_bytes", "selective_scan_fwd",
+    "selective_scan_fwd_host", "selective_state_update", "status_string", "version",
 ]

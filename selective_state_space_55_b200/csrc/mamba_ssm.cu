@@ -10,6 +10,7 @@
 #include "mamba_ssm.h"
 #include "selective_scan.cuh"
 #include "state_update.cuh"
+#include "conv1d.cuh"
 
 namespace mamba {
 
@@ -134,19 +135,25 @@ cudaError_t dispatch_scan(const ScanParams& prm, const CUtensorMap* maps, int cp
 }
 
 template <typename IoT, typename BcT, bool kHasZ, bool kZoh>
-cudaError_t launch_update_bulk(const UpdateParams& prm, int dev, int sms, cudaStream_t stream) {
+cudaError_t launch_update_bulk(const UpdateParams& prm, int dev, int sms, bool pdl,
+                               cudaStream_t stream) {
     static bool attr_done[kMaxDevices] = {false};
     static int resident[kMaxDevices] = {0};
-    auto kernel = state_update_bulk_kernel<IoT, BcT, kHasZ, kZoh>;
-    cudaError_t e = ensure_smem_attr(kernel, kBulkSmemBytes, attr_done, dev);
+    auto kernel = pdl ? state_update_bulk_kernel<IoT, BcT, kHasZ, kZoh, true>
+                      : state_update_bulk_kernel<IoT, BcT, kHasZ, kZoh, false>;
+    static bool attr_done_pdl[kMaxDevices] = {false};
+    static int resident_pdl[kMaxDevices] = {0};
+    bool* done = pdl ? attr_done_pdl : attr_done;
+    int* res = pdl ? resident_pdl : resident;
+    cudaError_t e = ensure_smem_attr(kernel, kBulkSmemBytes, done, dev);
     if (e != cudaSuccess) return e;
-    int per_sm = (dev >= 0 && dev < kMaxDevices) ? resident[dev] : 0;
+    int per_sm = (dev >= 0 && dev < kMaxDevices) ? res[dev] : 0;
     if (per_sm <= 0) {
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kBulkThreads,
                                                           kBulkSmemBytes);
         if (e != cudaSuccess) return e;
         if (per_sm <= 0) return cudaErrorInvalidConfiguration;
-        if (dev >= 0 && dev < kMaxDevices) resident[dev] = per_sm;
+        if (dev >= 0 && dev < kMaxDevices) res[dev] = per_sm;
     }
     // Each CTA owns one channel block and every J-th batch row: J copies of the
     // nblk blocks fill the resident CTAs.  Among J <= resident / nblk pick the
@@ -157,19 +164,30 @@ cudaError_t launch_update_bulk(const UpdateParams& prm, int dev, int sms, cudaSt
     for (int64_t j = jmax; j >= 1 && j * 2 >= jmax; --j)
         if ((prm.batch + j - 1) / j <= (prm.batch + J - 1) / J) J = j;
     const int64_t grid = nblk * J;
-    kernel<<<(unsigned)grid, kBulkThreads, kBulkSmemBytes, stream>>>(prm);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kBulkThreads);
+    cfg.dynamicSmemBytes = kBulkSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    e = cudaLaunchKernelEx(&cfg, kernel, prm);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
 template <typename IoT, typename BcT>
 cudaError_t dispatch_update_bc(const UpdateParams& prm, bool fast, bool bulk, bool has_z,
-                               int dev, int sms, cudaStream_t stream) {
+                               int dev, int sms, bool pdl, cudaStream_t stream) {
     if (bulk) {
         if (prm.zoh)
-            return has_z ? launch_update_bulk<IoT, BcT, true, true>(prm, dev, sms, stream)
-                         : launch_update_bulk<IoT, BcT, false, true>(prm, dev, sms, stream);
-        return has_z ? launch_update_bulk<IoT, BcT, true, false>(prm, dev, sms, stream)
-                     : launch_update_bulk<IoT, BcT, false, false>(prm, dev, sms, stream);
+            return has_z ? launch_update_bulk<IoT, BcT, true, true>(prm, dev, sms, pdl, stream)
+                         : launch_update_bulk<IoT, BcT, false, true>(prm, dev, sms, pdl, stream);
+        return has_z ? launch_update_bulk<IoT, BcT, true, false>(prm, dev, sms, pdl, stream)
+                     : launch_update_bulk<IoT, BcT, false, false>(prm, dev, sms, pdl, stream);
     }
     if (fast) {
         // x covers channels (kUpdateChainsPerCta per CTA), y covers batch rows.
@@ -191,10 +209,10 @@ cudaError_t dispatch_update_bc(const UpdateParams& prm, bool fast, bool bulk, bo
 
 template <typename IoT>
 cudaError_t dispatch_update(const UpdateParams& prm, bool bc_bf16, bool fast, bool bulk,
-                            bool has_z, int dev, int sms, cudaStream_t stream) {
+                            bool has_z, int dev, int sms, bool pdl, cudaStream_t stream) {
     return bc_bf16
-               ? dispatch_update_bc<IoT, __nv_bfloat16>(prm, fast, bulk, has_z, dev, sms, stream)
-               : dispatch_update_bc<IoT, float>(prm, fast, bulk, has_z, dev, sms, stream);
+               ? dispatch_update_bc<IoT, __nv_bfloat16>(prm, fast, bulk, has_z, dev, sms, pdl, stream)
+               : dispatch_update_bc<IoT, float>(prm, fast, bulk, has_z, dev, sms, pdl, stream);
 }
 
 }  // namespace
@@ -528,10 +546,11 @@ MAMBA_API mamba_status_t mamba_selective_state_update(float* state, const void* 
         sms = current_sm_count(&dev);
         if (sms <= 0) return MAMBA_ERR_CUDA;
     }
+    const bool pdl = (dims->flags & MAMBA_FLAG_PDL) != 0;
     const cudaError_t e =
         dims->io_dtype == MAMBA_BF16
-            ? dispatch_update<__nv_bfloat16>(prm, bc_bf16, fast, bulk, has_z, dev, sms, stream)
-            : dispatch_update<float>(prm, bc_bf16, fast, bulk, has_z, dev, sms, stream);
+            ? dispatch_update<__nv_bfloat16>(prm, bc_bf16, fast, bulk, has_z, dev, sms, pdl, stream)
+            : dispatch_update<float>(prm, bc_bf16, fast, bulk, has_z, dev, sms, pdl, stream);
     return e == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
 }
 
@@ -825,6 +844,150 @@ MAMBA_API mamba_status_t mamba_selective_scan_fwd_host(
     // Later work on `stream` follows the last copy back (the copy-in stream
     // already joined it through the scans' waits).
     return fail(cudaStreamWaitEvent(stream, pp->d2h_done[(L.nchunks - 1) % kHostStages], 0));
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Short causal convolution (prefill and decode update).
+
+namespace {
+
+mamba_status_t check_conv(const mamba_dims_t* dims, int width, bool seq) {
+    if (dims == nullptr) return MAMBA_ERR_INVALID_ARG;
+    if (dims->batch < 0 || dims->dim < 0 || (seq && dims->seqlen < 0)) return MAMBA_ERR_INVALID_ARG;
+    if (width < 1 || width > MAMBA_MAX_CONV_WIDTH) return MAMBA_ERR_UNSUPPORTED;
+    if (!dtype_ok(dims->io_dtype)) return MAMBA_ERR_UNSUPPORTED;
+    const int64_t lim = (int64_t)1 << 40;
+    if (dims->batch >= lim || dims->dim >= lim || (seq && dims->seqlen >= lim))
+        return MAMBA_ERR_INVALID_ARG;
+    return MAMBA_OK;
+}
+
+bool partly_overlap(const void* a, const void* b, size_t bytes) {
+    if (a == nullptr || b == nullptr || a == b) return false;
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + bytes && y < x + bytes;
+}
+
+unsigned int blocks_for(int64_t threads) {
+    return (unsigned int)((threads + kConvThreads - 1) / kConvThreads);
+}
+
+template <typename IoT>
+cudaError_t launch_conv_fwd(const ConvParams& prm, bool vec, cudaStream_t stream) {
+    if (prm.seqlen > 0) {
+        if (vec) {
+            const int64_t warps = prm.chains * ((prm.vec_per_row + 32 * kConvVecs - 1) / (32 * kConvVecs));
+            const unsigned int grid = blocks_for(warps * 32);
+            switch (prm.width) {
+                case 1: causal_conv1d_vec_kernel<IoT, 1><<<grid, kConvThreads, 0, stream>>>(prm); break;
+                case 2: causal_conv1d_vec_kernel<IoT, 2><<<grid, kConvThreads, 0, stream>>>(prm); break;
+                case 3: causal_conv1d_vec_kernel<IoT, 3><<<grid, kConvThreads, 0, stream>>>(prm); break;
+                default: causal_conv1d_vec_kernel<IoT, 4><<<grid, kConvThreads, 0, stream>>>(prm); break;
+            }
+        } else {
+            causal_conv1d_generic_kernel<IoT><<<blocks_for(prm.chains * prm.seqlen), kConvThreads, 0,
+                                               stream>>>(prm);
+        }
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    if (prm.final_state != nullptr)
+        causal_conv1d_final_state_kernel<IoT><<<blocks_for(prm.chains), kConvThreads, 0, stream>>>(prm);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+extern "C" {
+
+MAMBA_API mamba_status_t mamba_causal_conv1d_fwd(const void* x, const float* weight,
+                                                 const float* bias, const void* initial_conv_state,
+                                                 int width, int silu, void* out,
+                                                 void* final_conv_state, const mamba_dims_t* dims,
+                                                 cudaStream_t stream) {
+    mamba_status_t st = check_conv(dims, width, true);
+    if (st != MAMBA_OK) return st;
+    const int64_t chains = dims->batch * dims->dim;
+    if (chains == 0) return MAMBA_OK;
+    if (weight == nullptr) return MAMBA_ERR_INVALID_ARG;
+    if (dims->seqlen > 0 && (x == nullptr || out == nullptr)) return MAMBA_ERR_INVALID_ARG;
+    const int es = dtype_bytes(dims->io_dtype);
+    if ((x && !aligned(x, es)) || (out && !aligned(out, es)) || !aligned(weight, 4) ||
+        (bias && !aligned(bias, 4)) || (initial_conv_state && !aligned(initial_conv_state, es)) ||
+        (final_conv_state && !aligned(final_conv_state, es)))
+        return MAMBA_ERR_ALIGN;
+    if (partly_overlap(initial_conv_state, final_conv_state, (size_t)chains * width * es))
+        return MAMBA_ERR_INVALID_ARG;
+    if (dims->seqlen > 0 && x == out) return MAMBA_ERR_INVALID_ARG;
+    if (chains * std::max<int64_t>(dims->seqlen, 1) / kConvThreads >= ((int64_t)1 << 31))
+        return MAMBA_ERR_UNSUPPORTED;
+    ConvParams prm{};
+    prm.x = x;
+    prm.weight = weight;
+    prm.bias = bias;
+    prm.init = initial_conv_state;
+    prm.out = out;
+    prm.final_state = final_conv_state;
+    prm.batch = dims->batch;
+    prm.dim = dims->dim;
+    prm.seqlen = dims->seqlen;
+    prm.chains = chains;
+    prm.width = width;
+    prm.silu = silu != 0;
+    const bool vec = (dims->seqlen * es) % 16 == 0 && aligned(x, 16) && aligned(out, 16);
+    prm.vec_per_row = vec ? dims->seqlen * es / 16 : 0;
+    const cudaError_t e = dims->io_dtype == MAMBA_BF16
+                              ? launch_conv_fwd<__nv_bfloat16>(prm, vec, stream)
+                              : launch_conv_fwd<float>(prm, vec, stream);
+    return e == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
+}
+
+MAMBA_API mamba_status_t mamba_causal_conv1d_update(void* conv_state, const void* x,
+                                                    const float* weight, const float* bias,
+                                                    int width, int silu, void* out,
+                                                    const mamba_dims_t* dims,
+                                                    cudaStream_t stream) {
+    mamba_status_t st = check_conv(dims, width, false);
+    if (st != MAMBA_OK) return st;
+    const int64_t chains = dims->batch * dims->dim;
+    if (chains == 0) return MAMBA_OK;
+    if (conv_state == nullptr || x == nullptr || weight == nullptr || out == nullptr)
+        return MAMBA_ERR_INVALID_ARG;
+    const int es = dtype_bytes(dims->io_dtype);
+    if (!aligned(conv_state, es) || !aligned(x, es) || !aligned(out, es) || !aligned(weight, 4) ||
+        (bias && !aligned(bias, 4)))
+        return MAMBA_ERR_ALIGN;
+    if (chains / kConvThreads >= ((int64_t)1 << 31)) return MAMBA_ERR_UNSUPPORTED;
+    ConvParams prm{};
+    prm.x = x;
+    prm.weight = weight;
+    prm.bias = bias;
+    prm.state = conv_state;
+    prm.out = out;
+    prm.batch = dims->batch;
+    prm.dim = dims->dim;
+    prm.chains = chains;
+    prm.width = width;
+    prm.silu = silu != 0;
+    // W = 4: kConvUpdateChains chains per thread when the state is aligned to its
+    // vector and x/out to that many elements, else one chain per thread.
+    constexpr int kC = kConvUpdateChains;
+    const bool w4xn = width == 4 && aligned(conv_state, 4 * es) && aligned(x, kC * es) &&
+                      aligned(out, kC * es) && aligned(weight, 16);
+    const bool w4 = width == 4 && aligned(conv_state, 4 * es) && aligned(weight, 16);
+    const unsigned int grid = blocks_for(w4xn ? (chains + kC - 1) / kC : chains);
+    if (dims->io_dtype == MAMBA_BF16) {
+        if (w4xn) causal_conv1d_update_w4xn_kernel<__nv_bfloat16, kC><<<grid, kConvThreads, 0, stream>>>(prm);
+        else if (w4) causal_conv1d_update_w4_kernel<__nv_bfloat16><<<grid, kConvThreads, 0, stream>>>(prm);
+        else causal_conv1d_update_kernel<__nv_bfloat16><<<grid, kConvThreads, 0, stream>>>(prm);
+    } else {
+        if (w4xn) causal_conv1d_update_w4xn_kernel<float, kC><<<grid, kConvThreads, 0, stream>>>(prm);
+        else if (w4) causal_conv1d_update_w4_kernel<float><<<grid, kConvThreads, 0, stream>>>(prm);
+        else causal_conv1d_update_kernel<float><<<grid, kConvThreads, 0, stream>>>(prm);
+    }
+    return cudaGetLastError() == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
 }
 
 MAMBA_API mamba_status_t mamba_device_status(void) {

@@ -142,8 +142,14 @@ __global__ void __launch_bounds__(kUpdateThreads)
 // lanes share a chain (a float4 of state each); softplus and silu run once per
 // chain, spread over the four lanes, and are exchanged by shuffles.  Abar is
 // MUFU ex2 for bf16 inputs and exp2_near_one_exact for fp32 inputs, as in the
-// scan.  kZoh, the zero-order-hold gain zoh_phi, is a separate instance so
-// that the Euler one keeps its register count (72) and 5 CTAs per SM.
+// scan.  kZoh, the zero-order-hold gain zoh_phi, is a separate instance (4
+// CTAs per SM) so that the Euler one keeps 5 CTAs per SM.
+// kPdl is the instance for a programmatic dependent launch (MAMBA_FLAG_PDL):
+// the grid may start while the previous kernel on the stream finishes, so the
+// producer first requests the state of its first tiles, then waits for that
+// kernel before the token inputs, and lets the next launch start once its last
+// loads are issued.  That instance runs 4 CTAs per SM, which leaves room for
+// the next launch's CTAs to start early; the plain instance runs 5.
 constexpr int kBulkConsumers = 4;
 constexpr int kBulkThreads = 32 * (kBulkConsumers + 1);
 constexpr int kBulkTile = 32 * kBulkConsumers;       // channels per tile
@@ -158,7 +164,7 @@ constexpr int kBOffC = kBOffB + 64;
 constexpr int kBStage = ((kBOffC + 64 + 127) / 128) * 128;
 constexpr int kBulkSmemBytes = kBulkStages * kBStage + 2 * kBulkStages * 8 + 1024;
 
-template <typename IoT, typename BcT, bool kHasZ, bool kZoh>
+template <typename IoT, typename BcT, bool kHasZ, bool kZoh, bool kPdl>
 __global__ void __launch_bounds__(kBulkThreads)
     state_update_bulk_kernel(const __grid_constant__ UpdateParams p) {
     extern __shared__ uint8_t smem_raw[];
@@ -194,7 +200,36 @@ __global__ void __launch_bounds__(kBulkThreads)
         if (lane != 0) return;
         const uint32_t tok = (uint32_t)nch * ES;
         const uint32_t bytes = (uint32_t)nch * 64 + (kHasZ ? 3u : 2u) * tok + 2u * 16u * BS;
-        int64_t k = 0;
+        auto load_state = [&](int64_t k) {
+            const int s = (int)(k % kBulkStages);
+            const int64_t c0 = (b0 + k * bstep) * p.dim + d0;
+            const uint32_t bar = smem_u32(&full[s]);
+            fence_proxy_async_smem();
+            mbar_arrive_expect_tx(bar, bytes);
+            bulk_load(smem_u32(smem + s * kBStage + kBOffState), p.state + c0 * 16, (uint32_t)nch * 64, bar);
+        };
+        auto load_tokens = [&](int64_t k) {
+            const int s = (int)(k % kBulkStages);
+            const int64_t b = b0 + k * bstep;
+            const int64_t c0 = b * p.dim + d0;
+            uint8_t* st = smem + s * kBStage;
+            const uint32_t bar = smem_u32(&full[s]);
+            bulk_load(smem_u32(st + kBOffX), static_cast<const IoT*>(p.x) + c0, tok, bar);
+            bulk_load(smem_u32(st + kBOffDt), static_cast<const IoT*>(p.dt) + c0, tok, bar);
+            if (kHasZ) bulk_load(smem_u32(st + kBOffZ), static_cast<const IoT*>(p.z) + c0, tok, bar);
+            bulk_load(smem_u32(st + kBOffB), static_cast<const BcT*>(p.B) + b * 16, 16 * BS, bar);
+            bulk_load(smem_u32(st + kBOffC), static_cast<const BcT*>(p.C) + b * 16, 16 * BS, bar);
+        };
+        // The state belongs to this call alone, so the first tiles' state is
+        // requested before waiting for the kernel this one may overlap with
+        // (programmatic dependent launch); the token inputs may come from it.
+        const int64_t pre = kPdl ? (mine < kBulkStages ? mine : kBulkStages) : 0;
+        if constexpr (kPdl) {
+            for (int64_t k = 0; k < pre; ++k) load_state(k);
+            grid_dependency_wait();
+            for (int64_t k = 0; k < pre; ++k) load_tokens(k);
+        }
+        int64_t k = pre;
         for (; k < mine; ++k) {
             const int s = (int)(k % kBulkStages);
             if (k >= kBulkStages &&
@@ -202,19 +237,10 @@ __global__ void __launch_bounds__(kBulkThreads)
                 record_device_error(MAMBA_ERR_TIMEOUT);
                 break;
             }
-            const int64_t b = b0 + k * bstep;
-            const int64_t c0 = b * p.dim + d0;
-            uint8_t* st = smem + s * kBStage;
-            const uint32_t bar = smem_u32(&full[s]);
-            fence_proxy_async_smem();
-            mbar_arrive_expect_tx(bar, bytes);
-            bulk_load(smem_u32(st + kBOffState), p.state + c0 * 16, (uint32_t)nch * 64, bar);
-            bulk_load(smem_u32(st + kBOffX), static_cast<const IoT*>(p.x) + c0, tok, bar);
-            bulk_load(smem_u32(st + kBOffDt), static_cast<const IoT*>(p.dt) + c0, tok, bar);
-            if (kHasZ) bulk_load(smem_u32(st + kBOffZ), static_cast<const IoT*>(p.z) + c0, tok, bar);
-            bulk_load(smem_u32(st + kBOffB), static_cast<const BcT*>(p.B) + b * 16, 16 * BS, bar);
-            bulk_load(smem_u32(st + kBOffC), static_cast<const BcT*>(p.C) + b * 16, 16 * BS, bar);
+            load_state(k);
+            load_tokens(k);
         }
+        if constexpr (kPdl) grid_launch_dependents();
         // Loads still in flight must land before the CTA's shared memory goes away.
         for (int64_t j = max((int64_t)0, k - kBulkStages); j < k; ++j)
             (void)mbar_wait_bounded(smem_u32(&full[j % kBulkStages]), (uint32_t)((j / kBulkStages) & 1));

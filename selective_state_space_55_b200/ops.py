@@ -28,6 +28,7 @@ MAMBA_FLAG_NO_TMA = 0x1
 MAMBA_FLAG_PARALLEL_CHUNKS = 0x2
 MAMBA_FLAG_TEST_WITHHOLD_HANDOFF = 0x4
 MAMBA_FLAG_ZOH = 0x8
+MAMBA_FLAG_PDL = 0x10
 
 _DTYPE_CODE = {torch.float32: MAMBA_F32, torch.bfloat16: MAMBA_BF16}
 
@@ -93,6 +94,10 @@ def library(path: Path | str | None = None) -> ctypes.CDLL:
     lib.mamba_selective_scan_fwd_host.restype = i32
     lib.mamba_selective_scan_fwd_host.argtypes = [
         vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, ctypes.c_int64, dims_p, vp]
+    lib.mamba_causal_conv1d_fwd.restype = i32
+    lib.mamba_causal_conv1d_fwd.argtypes = [vp, vp, vp, vp, i32, i32, vp, vp, dims_p, vp]
+    lib.mamba_causal_conv1d_update.restype = i32
+    lib.mamba_causal_conv1d_update.argtypes = [vp, vp, vp, vp, i32, i32, vp, dims_p, vp]
     lib.mamba_selective_state_update.restype = i32
     lib.mamba_selective_state_update.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, dims_p, vp]
     lib.mamba_device_status.restype = i32
@@ -327,6 +332,65 @@ def selective_state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=None,
         _ptr(dt_bias), _ptr(out), ctypes.byref(dims), _stream_handle(stream))
     if rc != MAMBA_OK:
         raise MambaError("mamba_selective_state_update", rc)
+    return out
+
+
+def _conv_dims(batch, dim, seqlen, io_dtype) -> MambaDims:
+    return MambaDims(batch=batch, dim=dim, dstate=1, seqlen=seqlen, io_dtype=_DTYPE_CODE[io_dtype],
+                     bc_dtype=_DTYPE_CODE[io_dtype], dt_softplus=0, num_chunks=0, flags=0,
+                     reserved=0, workspace=None, workspace_bytes=0)
+
+
+def causal_conv1d_fwd(x, weight, bias=None, initial_conv_state=None, silu=True, out=None,
+                      final_conv_state=None, return_final_state=False, stream=None):
+    """Short causal convolution over a sequence through ``mamba_causal_conv1d_fwd``.
+
+    x: (batch, dim, L) fp32 or bf16; weight: (dim, W) fp32, W <= 4; bias: (dim,)
+    fp32 or None; initial_conv_state: (batch, dim, W) in x's dtype or None.
+    Returns ``out`` (and the final conv state when asked for or given).
+    """
+    batch, dim, L = x.shape
+    W = weight.shape[1]
+    io = x.dtype
+    _check_cuda("x", x, (torch.float32, torch.bfloat16), (batch, dim, L))
+    _check_cuda("weight", weight, (torch.float32,), (dim, W))
+    _check_cuda("bias", bias, (torch.float32,), (dim,))
+    _check_cuda("initial_conv_state", initial_conv_state, (io,), (batch, dim, W))
+    if out is None:
+        out = torch.empty_like(x)
+    _check_cuda("out", out, (io,), (batch, dim, L))
+    if final_conv_state is None and return_final_state:
+        final_conv_state = torch.empty((batch, dim, W), dtype=io, device=x.device)
+    _check_cuda("final_conv_state", final_conv_state, (io,), (batch, dim, W))
+    dims = _conv_dims(batch, dim, L, io)
+    rc = library().mamba_causal_conv1d_fwd(
+        _ptr(x), _ptr(weight), _ptr(bias), _ptr(initial_conv_state), W, int(bool(silu)),
+        _ptr(out), _ptr(final_conv_state), ctypes.byref(dims), _stream_handle(stream))
+    if rc != MAMBA_OK:
+        raise MambaError("mamba_causal_conv1d_fwd", rc)
+    if final_conv_state is not None:
+        return out, final_conv_state
+    return out
+
+
+def causal_conv1d_update(conv_state, x, weight, bias=None, silu=True, out=None, stream=None):
+    """One token of the short convolution through ``mamba_causal_conv1d_update``;
+    ``conv_state`` (batch, dim, W) is shifted in place.  Returns ``out`` (batch, dim)."""
+    batch, dim, W = conv_state.shape
+    io = x.dtype
+    _check_cuda("conv_state", conv_state, (io,), (batch, dim, W))
+    _check_cuda("x", x, (torch.float32, torch.bfloat16), (batch, dim))
+    _check_cuda("weight", weight, (torch.float32,), (dim, W))
+    _check_cuda("bias", bias, (torch.float32,), (dim,))
+    if out is None:
+        out = torch.empty_like(x)
+    _check_cuda("out", out, (io,), (batch, dim))
+    dims = _conv_dims(batch, dim, 0, io)
+    rc = library().mamba_causal_conv1d_update(
+        _ptr(conv_state), _ptr(x), _ptr(weight), _ptr(bias), W, int(bool(silu)), _ptr(out),
+        ctypes.byref(dims), _stream_handle(stream))
+    if rc != MAMBA_OK:
+        raise MambaError("mamba_causal_conv1d_update", rc)
     return out
 
 

@@ -119,6 +119,28 @@ def test_host_scan_rejects_bad_arguments(lib):
         ctypes.c_size_t(-1).value
 
 
+def test_conv_rejects_bad_arguments(lib):
+    d = _dims()
+    fwd = lambda dims, W, x=FAKE, w=FAKE, out=FAKE, init=None, fin=None: lib.mamba_causal_conv1d_fwd(  # noqa: E731
+        x, w, None, init, W, 1, out, fin, ctypes.byref(dims) if dims is not None else None, None)
+    upd = lambda dims, W, st=FAKE, x=FAKE, w=FAKE, out=FAKE: lib.mamba_causal_conv1d_update(  # noqa: E731
+        st, x, w, None, W, 1, out, ctypes.byref(dims) if dims is not None else None, None)
+    assert fwd(None, 4) == -1
+    assert fwd(d, 0) == -2 and fwd(d, 5) == -2          # width outside 1..4
+    assert fwd(d, 4, x=None) == -1 and fwd(d, 4, w=None) == -1 and fwd(d, 4, out=None) == -1
+    assert fwd(d, 4, x=ctypes.c_void_p(0x10001)) == -3   # bf16 needs 2-byte alignment
+    assert fwd(d, 4, out=FAKE, x=FAKE) == -1            # out aliases x
+    base = 0x200000
+    assert fwd(d, 4, x=ctypes.c_void_p(0x400000), init=ctypes.c_void_p(base),
+               fin=ctypes.c_void_p(base + 2)) == -1     # states partly overlap
+    bad = _dims(); bad.io_dtype = 9
+    assert fwd(bad, 4) == -2
+    assert fwd(_dims(batch=0), 4) == 0
+    assert upd(None, 4) == -1 and upd(d, 7) == -2
+    assert upd(d, 4, st=None) == -1 and upd(d, 4, w=None) == -1
+    assert upd(d, 4, w=ctypes.c_void_p(0x10002)) == -3  # fp32 weights need 4-byte alignment
+
+
 def test_scan_empty_batch_is_a_no_op(lib):
     assert _scan(lib, _dims(batch=0)) == 0
     assert _scan(lib, _dims(dim=0)) == 0
