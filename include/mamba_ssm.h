@@ -329,6 +329,47 @@ MAMBA_API mamba_status_t mamba_selective_state_update(float *state, const void *
                                                       cudaStream_t stream);
 
 /*
+ * Backward pass of the selective scan (training).
+ *
+ * Gradients of a scalar loss, given dout = dLoss/dout (and optionally
+ * dlast_state = dLoss/dlast_state), with respect to every input of
+ * mamba_selective_scan_fwd_with_state, Euler input term.  As in the pages'
+ * description of the hardware-aware scan ("Mamba 与状态空间模型", section
+ * 在芯片上扫过去), the per-step states are not stored by the forward: a
+ * checkpoint pass keeps the state every 8 steps in the workspace, and the
+ * backward recomputes the states in between from it.  With
+ * lambda_t = dLoss/dh_t the adjoint runs backwards in time:
+ *   lambda_t = C_t dy_t + Abar_t+1 lambda_t+1,   dy = dout * silu(z)
+ *   dC_t,n = dy_t h_t,n;  dB_t,n = lambda_t,n Delta_t u_t
+ *   dDelta_t = sum_n lambda_t,n (B_t,n u_t + A_n Abar_t,n h_t-1,n)  (then * softplus')
+ *   dA_n = sum_t lambda_t,n Delta_t Abar_t,n h_t-1,n;  du_t = D dy_t + Delta_t sum_n lambda_t,n B_t,n
+ * Inputs (device): the forward's inputs (u, delta, A, B, C, D, z, delta_bias,
+ *   softplus, initial_state: same shapes, dtypes and NULL rules), dout
+ *   (batch, dim, seqlen) io_dtype, dlast_state (batch, dim, dstate) fp32 or NULL.
+ * Outputs (device, overwritten): du, ddelta, dz (batch, dim, seqlen) io_dtype;
+ *   dA (dim, dstate), dB and dC (batch, dstate, seqlen), dD and ddelta_bias
+ *   (dim,), dinitial_state (batch, dim, dstate), all fp32.  dz, dD,
+ *   ddelta_bias and dinitial_state may be NULL (not computed); dz needs z.
+ *   dA, dB, dC, dD and ddelta_bias are sums over many channels and time
+ *   steps, accumulated with atomic adds: their rounding order (not their
+ *   value) varies from run to run.
+ * dims->workspace: at least mamba_selective_scan_bwd_workspace_bytes(dims)
+ *   bytes, 256-byte aligned (64 bytes per chain and 8 steps for the
+ *   checkpoints, plus the segment handoffs).
+ * MAMBA_FLAG_ZOH is not supported here (MAMBA_ERR_UNSUPPORTED).  Segments of a
+ * sequence are processed one after another (chained), so sequences much longer
+ * than the batch x channel count can keep busy run with little parallelism.
+ */
+MAMBA_API size_t mamba_selective_scan_bwd_workspace_bytes(const mamba_dims_t *dims);
+
+MAMBA_API mamba_status_t mamba_selective_scan_bwd(
+    const void *u, const void *delta, const float *A, const void *B, const void *C,
+    const float *D, const void *z, const float *delta_bias, int softplus,
+    const float *initial_state, const void *dout, const float *dlast_state, void *du,
+    void *ddelta, float *dA, float *dB, float *dC, float *dD, void *dz, float *ddelta_bias,
+    float *dinitial_state, const mamba_dims_t *dims, cudaStream_t stream);
+
+/*
  * Short causal convolution of the Mamba block.
  *
  * Besides its 16 state numbers, each channel keeps a short convolution over

@@ -11,6 +11,7 @@
 #include "selective_scan.cuh"
 #include "state_update.cuh"
 #include "conv1d.cuh"
+#include "scan_backward.cuh"
 
 namespace mamba {
 
@@ -326,6 +327,13 @@ mamba_status_t plan_scan(const mamba_dims_t* dims, int sm_count, mamba_scan_plan
 
 using namespace mamba;
 
+mamba_status_t scan_fwd_internal(const void* u, const void* delta, const float* A, const void* B,
+                                 const void* C, const float* D, const void* z,
+                                 const float* delta_bias, int softplus,
+                                 const float* initial_state, void* out, float* last_state,
+                                 const mamba_dims_t* dims, cudaStream_t stream, float* ckpt,
+                                 int64_t ckpt_tiles);
+
 extern "C" {
 
 MAMBA_API mamba_status_t mamba_selective_scan_plan(const mamba_dims_t* dims, int sm_count,
@@ -355,6 +363,21 @@ MAMBA_API mamba_status_t mamba_selective_scan_fwd_with_state(
     const float* D, const void* z, const float* delta_bias, int softplus,
     const float* initial_state, void* out, float* last_state, const mamba_dims_t* dims,
     cudaStream_t stream) {
+    return scan_fwd_internal(u, delta, A, B, C, D, z, delta_bias, softplus, initial_state, out,
+                             last_state, dims, stream, nullptr, 0);
+}
+
+}  // extern "C"
+
+// The forward scan.  With `ckpt` set it is the backward's checkpoint pass: no
+// output, the state before every kCkptSteps steps stored to
+// ckpt[chain][ckpt_tiles][16] instead.
+mamba_status_t scan_fwd_internal(const void* u, const void* delta, const float* A, const void* B,
+                                 const void* C, const float* D, const void* z,
+                                 const float* delta_bias, int softplus,
+                                 const float* initial_state, void* out, float* last_state,
+                                 const mamba_dims_t* dims, cudaStream_t stream, float* ckpt,
+                                 int64_t ckpt_tiles) {
     mamba_status_t st = check_dims(dims, true);
     if (st != MAMBA_OK) return st;
     // Empty problems first: tensors without elements may have null pointers.
@@ -381,11 +404,11 @@ MAMBA_API mamba_status_t mamba_selective_scan_fwd_with_state(
         return e == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
     }
     if (u == nullptr || delta == nullptr || A == nullptr || B == nullptr || C == nullptr ||
-        out == nullptr)
+        (out == nullptr && ckpt == nullptr))
         return MAMBA_ERR_INVALID_ARG;
     const int io_es = dtype_bytes(dims->io_dtype);
     const int bc_es = dtype_bytes(dims->bc_dtype);
-    if (!aligned(u, io_es) || !aligned(delta, io_es) || !aligned(out, io_es) ||
+    if (!aligned(u, io_es) || !aligned(delta, io_es) || (out && !aligned(out, io_es)) ||
         (z && !aligned(z, io_es)) || !aligned(B, bc_es) || !aligned(C, bc_es) || !aligned(A, 4) ||
         (D && !aligned(D, 4)) || (delta_bias && !aligned(delta_bias, 4)) ||
         (last_state && !aligned(last_state, 4)))
@@ -413,6 +436,8 @@ MAMBA_API mamba_status_t mamba_selective_scan_fwd_with_state(
     prm.out = out;
     prm.last_state = last_state;
     prm.h0 = initial_state;
+    prm.ckpt = ckpt;
+    prm.ckpt_tiles = ckpt_tiles;
     prm.batch = dims->batch;
     prm.dim = dims->dim;
     prm.seqlen = dims->seqlen;
@@ -423,7 +448,7 @@ MAMBA_API mamba_status_t mamba_selective_scan_fwd_with_state(
     prm.dstate = (int)dims->dstate;
     prm.nseg = plan.nchunks;
     prm.bc_bf16 = dims->bc_dtype == MAMBA_BF16;
-    prm.vec_out = ((dims->seqlen * io_es) % 16 == 0) && aligned(out, 16);
+    prm.vec_out = out != nullptr && ((dims->seqlen * io_es) % 16 == 0) && aligned(out, 16);
     // A predecessor segment legitimately takes well under 64 us per step even
     // on a crowded GPU; wait that long (at least ~1 s) before reporting a stall.
     prm.withhold_handoff = (dims->flags & MAMBA_FLAG_TEST_WITHHOLD_HANDOFF) ? 1 : 0;
@@ -493,6 +518,8 @@ MAMBA_API mamba_status_t mamba_selective_scan_fwd_with_state(
     }
     return e == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
 }
+
+extern "C" {
 
 MAMBA_API mamba_status_t mamba_selective_state_update(float* state, const void* x, const void* dt,
                                                       const float* A, const void* B, const void* C,
@@ -988,6 +1015,225 @@ MAMBA_API mamba_status_t mamba_causal_conv1d_update(void* conv_state, const void
         else causal_conv1d_update_kernel<float><<<grid, kConvThreads, 0, stream>>>(prm);
     }
     return cudaGetLastError() == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Backward pass of the scan.
+
+namespace {
+
+// Scratch of one backward call (offsets in bytes).
+struct BwdWorkspace {
+    size_t fwd_zeroed;      // checkpoint pass: counters + flags, cleared
+    size_t fwd_bytes;       // checkpoint pass scratch (zeroed part + carry)
+    size_t bwd;             // backward: counter at +0, flags at +kWsFlags
+    size_t bwd_zeroed;
+    size_t bwd_carry;       // [chains][16] lambda handoff
+    size_t ckpt;            // [chains][tiles][16] fp32
+    size_t total;
+    int64_t K, seg_len, groups, tiles;
+};
+
+// Segments of the backward (chained, in reverse): the chained rule of the
+// forward planner, K = min(ceil(8 W / G), L / 256), at least 1.
+mamba_status_t bwd_layout(const mamba_dims_t* dims, int sms, BwdWorkspace* w) {
+    *w = BwdWorkspace{};
+    const int io_es = dtype_bytes(dims->io_dtype);
+    const int64_t T = kRowBytes / io_es;                   // forward tile, a multiple of 8
+    const int64_t L = dims->seqlen;
+    const int64_t groups = dims->batch * ((dims->dim + 31) / 32);
+    const int64_t W = (int64_t)sms * ScanLayout<1>::kWarpsPerSm;
+    int64_t K = 1;
+    if (groups > 0 && L > 0) K = std::max<int64_t>(1, std::min<int64_t>((8 * W + groups - 1) / groups, L / 256));
+    int64_t seg = L;
+    if (K > 1) {
+        seg = ((L + K - 1) / K + T - 1) / T * T;
+        K = (L + seg - 1) / seg;
+    }
+    if (K <= 1) { K = 1; seg = L; }
+    if (groups * K >= ((int64_t)1 << 31)) return MAMBA_ERR_UNSUPPORTED;
+    const size_t chains = (size_t)dims->batch * (size_t)dims->dim;
+    const int64_t tiles = (L + kCkptSteps - 1) / kCkptSteps;
+    size_t off = 0;
+    w->fwd_zeroed = kWsFlags + align256((size_t)groups * sizeof(unsigned int));
+    off = w->fwd_zeroed + (K > 1 ? align256(chains * kNPad * sizeof(float)) : 0);
+    w->fwd_bytes = off;
+    w->bwd = off;
+    w->bwd_zeroed = kWsFlags + align256((size_t)groups * sizeof(unsigned int));
+    off += w->bwd_zeroed;
+    w->bwd_carry = off;
+    off += align256(chains * kNPad * sizeof(float));
+    w->ckpt = off;
+    off += align256(chains * (size_t)tiles * kNPad * sizeof(float));
+    w->total = off;
+    w->K = K;
+    w->seg_len = seg;
+    w->groups = groups;
+    w->tiles = tiles;
+    return MAMBA_OK;
+}
+
+template <typename IoT, typename BcT, bool kHasZ>
+cudaError_t launch_bwd(const BwdParams& prm, int dev, int sms, cudaStream_t stream) {
+    static int resident[kMaxDevices] = {0};
+    auto kernel = selective_scan_bwd_kernel<IoT, BcT, kHasZ>;
+    int per_sm = (dev >= 0 && dev < kMaxDevices) ? resident[dev] : 0;
+    if (per_sm <= 0) {
+        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kBwdWarps * 32, 0);
+        if (e != cudaSuccess) return e;
+        if (per_sm <= 0) return cudaErrorInvalidConfiguration;
+        if (dev >= 0 && dev < kMaxDevices) resident[dev] = per_sm;
+    }
+    const int64_t want = (std::min<int64_t>(prm.items, prm.groups) + kBwdWarps - 1) / kBwdWarps;
+    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)per_sm * sms));
+    kernel<<<(unsigned)grid, kBwdWarps * 32, 0, stream>>>(prm);
+    return cudaGetLastError();
+}
+
+template <typename IoT>
+cudaError_t dispatch_bwd(const BwdParams& prm, bool has_z, int dev, int sms, cudaStream_t stream) {
+    if (prm.bc_bf16)
+        return has_z ? launch_bwd<IoT, __nv_bfloat16, true>(prm, dev, sms, stream)
+                     : launch_bwd<IoT, __nv_bfloat16, false>(prm, dev, sms, stream);
+    return has_z ? launch_bwd<IoT, float, true>(prm, dev, sms, stream)
+                 : launch_bwd<IoT, float, false>(prm, dev, sms, stream);
+}
+
+cudaError_t zero_async(void* p, size_t bytes, cudaStream_t stream) {
+    return (p == nullptr || bytes == 0) ? cudaSuccess : cudaMemsetAsync(p, 0, bytes, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+MAMBA_API size_t mamba_selective_scan_bwd_workspace_bytes(const mamba_dims_t* dims) {
+    if (check_dims(dims, true) != MAMBA_OK) return static_cast<size_t>(-1);
+    if (dims->batch * dims->dim == 0 || dims->seqlen == 0) return 0;
+    const int sms = current_sm_count(nullptr);
+    if (sms <= 0) return static_cast<size_t>(-1);
+    BwdWorkspace w;
+    if (bwd_layout(dims, sms, &w) != MAMBA_OK) return static_cast<size_t>(-1);
+    return w.total;
+}
+
+MAMBA_API mamba_status_t mamba_selective_scan_bwd(
+    const void* u, const void* delta, const float* A, const void* B, const void* C,
+    const float* D, const void* z, const float* delta_bias, int softplus,
+    const float* initial_state, const void* dout, const float* dlast_state, void* du,
+    void* ddelta, float* dA, float* dB, float* dC, float* dD, void* dz, float* ddelta_bias,
+    float* dinitial_state, const mamba_dims_t* dims, cudaStream_t stream) {
+    mamba_status_t st = check_dims(dims, true);
+    if (st != MAMBA_OK) return st;
+    if (dims->flags & MAMBA_FLAG_ZOH) return MAMBA_ERR_UNSUPPORTED;
+    const int64_t chains = dims->batch * dims->dim;
+    if (chains == 0) return MAMBA_OK;
+    const int64_t L = dims->seqlen, N = dims->dstate;
+    if (A == nullptr || dA == nullptr) return MAMBA_ERR_INVALID_ARG;
+    if (L > 0 && (u == nullptr || delta == nullptr || B == nullptr || C == nullptr ||
+                  dout == nullptr || du == nullptr || ddelta == nullptr || dB == nullptr ||
+                  dC == nullptr))
+        return MAMBA_ERR_INVALID_ARG;
+    const int io_es = dtype_bytes(dims->io_dtype);
+    const int bc_es = dtype_bytes(dims->bc_dtype);
+    const void* io_ptrs[7] = {u, delta, z, dout, du, ddelta, dz};
+    for (const void* q : io_ptrs)
+        if (q && !aligned(q, io_es)) return MAMBA_ERR_ALIGN;
+    const void* f32_ptrs[10] = {A, D, delta_bias, initial_state, dlast_state, dA, dD,
+                                ddelta_bias, dinitial_state, nullptr};
+    for (const void* q : f32_ptrs)
+        if (q && !aligned(q, 4)) return MAMBA_ERR_ALIGN;
+    if ((B && !aligned(B, bc_es)) || (C && !aligned(C, bc_es)) || (dB && !aligned(dB, 4)) ||
+        (dC && !aligned(dC, 4)))
+        return MAMBA_ERR_ALIGN;
+    cudaError_t e = cudaSuccess;
+    // gradients that are sums start from zero
+    e = zero_async(dA, (size_t)dims->dim * N * sizeof(float), stream);
+    if (e == cudaSuccess) e = zero_async(dD, (size_t)dims->dim * sizeof(float), stream);
+    if (e == cudaSuccess) e = zero_async(ddelta_bias, (size_t)dims->dim * sizeof(float), stream);
+    if (e != cudaSuccess) return MAMBA_ERR_CUDA;
+    if (L == 0) {       // nothing to scan: the start state's gradient is dlast_state
+        const size_t sb = (size_t)chains * N * sizeof(float);
+        if (dinitial_state == nullptr) return MAMBA_OK;
+        e = dlast_state ? cudaMemcpyAsync(dinitial_state, dlast_state, sb, cudaMemcpyDeviceToDevice, stream)
+                        : cudaMemsetAsync(dinitial_state, 0, sb, stream);
+        return e == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
+    }
+    int dev = 0;
+    const int sms = current_sm_count(&dev);
+    if (sms <= 0) return MAMBA_ERR_CUDA;
+    BwdWorkspace w;
+    st = bwd_layout(dims, sms, &w);
+    if (st != MAMBA_OK) return st;
+    if (dims->workspace == nullptr || dims->workspace_bytes < w.total) return MAMBA_ERR_WORKSPACE;
+    if (!aligned(dims->workspace, 256)) return MAMBA_ERR_ALIGN;
+    uint8_t* ws = static_cast<uint8_t*>(dims->workspace);
+    e = zero_async(dB, (size_t)dims->batch * N * L * sizeof(float), stream);
+    if (e == cudaSuccess) e = zero_async(dC, (size_t)dims->batch * N * L * sizeof(float), stream);
+    if (e == cudaSuccess) e = zero_async(ws + w.bwd, w.bwd_zeroed, stream);
+    if (e != cudaSuccess) return MAMBA_ERR_CUDA;
+
+    // 1. checkpoint pass: the forward, chained in w.K segments, states only
+    mamba_dims_t fd = *dims;
+    fd.num_chunks = (int32_t)w.K;
+    fd.flags = dims->flags & MAMBA_FLAG_NO_TMA;
+    fd.workspace = ws;
+    fd.workspace_bytes = w.fwd_bytes;
+    float* ckpt = reinterpret_cast<float*>(ws + w.ckpt);
+    st = scan_fwd_internal(u, delta, A, B, C, nullptr, nullptr, delta_bias, softplus,
+                           initial_state, nullptr, nullptr, &fd, stream, ckpt, w.tiles);
+    if (st != MAMBA_OK) return st;
+
+    // 2. the adjoint, segments in reverse
+    BwdParams prm{};
+    prm.u = u;
+    prm.delta = delta;
+    prm.z = z;
+    prm.dout = dout;
+    prm.A = A;
+    prm.B = B;
+    prm.C = C;
+    prm.D = D;
+    prm.delta_bias = delta_bias;
+    prm.dlast = dlast_state;
+    prm.ckpt = ckpt;
+    prm.du = du;
+    prm.ddelta = ddelta;
+    prm.dz = dz;
+    prm.dA = dA;
+    prm.dB = dB;
+    prm.dC = dC;
+    prm.dD = dD;
+    prm.dbias = ddelta_bias;
+    prm.dh0 = dinitial_state;
+    prm.counter = reinterpret_cast<unsigned int*>(ws + w.bwd + kWsCounters);
+    prm.flags = reinterpret_cast<unsigned int*>(ws + w.bwd + kWsFlags);
+    prm.carry = reinterpret_cast<float*>(ws + w.bwd_carry);
+    prm.batch = dims->batch;
+    prm.dim = dims->dim;
+    prm.seqlen = L;
+    prm.groups_per_batch = (dims->dim + 31) / 32;
+    prm.groups = w.groups;
+    prm.chains = chains;
+    prm.seg_len = w.seg_len;
+    prm.items = w.groups * w.K;
+    prm.ckpt_tiles = w.tiles;
+    prm.dstate = (int)N;
+    prm.nseg = (int)w.K;
+    prm.softplus = softplus != 0;
+    prm.bc_bf16 = dims->bc_dtype == MAMBA_BF16;
+    bool vec = true;
+    for (const void* q : io_ptrs)
+        if (q && !aligned(q, 16)) vec = false;
+    prm.vec_ok = vec ? 1 : 0;
+    prm.bc_vec = ((L * bc_es) % 16 == 0 && aligned(B, 16) && aligned(C, 16)) ? 1 : 0;
+    prm.flag_poll_limit =
+        (unsigned int)std::min<int64_t>(std::max<int64_t>(w.seg_len * 256, 1 << 20), (int64_t)1 << 31);
+    e = dims->io_dtype == MAMBA_BF16 ? dispatch_bwd<__nv_bfloat16>(prm, z != nullptr, dev, sms, stream)
+                                     : dispatch_bwd<float>(prm, z != nullptr, dev, sms, stream);
+    return e == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
 }
 
 MAMBA_API mamba_status_t mamba_device_status(void) {

@@ -1,0 +1,382 @@
+// Backward pass of the selective scan (sm_100a).
+//
+// Training back-propagates through the scan without keeping its per-step
+// states: they are computed again from checkpoints ("Mamba 与状态空间模型",
+// section 在芯片上扫过去).  With lambda_t = dLoss/dh_t, the adjoint runs in
+// reverse time:
+//
+//   lambda_t   = C_t dy_t + Abar_t+1 lambda_t+1        (lambda_L-1 from dlast_state)
+//   dC_t,n     = dy_t h_t,n          dB_t,n = lambda_t,n Delta_t u_t
+//   dDelta_t   = sum_n lambda_t,n (B_t,n u_t + A_n Abar_t,n h_t-1,n)
+//   dA_n      += lambda_t,n Delta_t Abar_t,n h_t-1,n
+//   du_t       = D dy_t + Delta_t sum_n lambda_t,n B_t,n
+//   dh_-1      = Abar_0 lambda_0
+//
+// with dy = dout silu(z), dz = dout y silu'(z) and the softplus derivative
+// sigmoid(delta + bias) applied to dDelta.
+//
+// Layout of the work.  A first launch (the forward kernel in its checkpoint
+// mode) stores the state before every block of kCkptSteps = 8 steps.  Then one
+// warp owns 32 channels of one batch row for one segment, as in the forward,
+// and walks the segment's 8-step blocks from the last to the first.  Segments
+// run in reverse order: a segment starts from the lambda the later segment
+// left in an L2-resident carry buffer (release/acquire flag, bounded wait).
+// Within a block, for each quarter of the state (4 of the 16 entries) the lane
+// recomputes the block's 8 states from the checkpoint into registers, then
+// runs the adjoint backwards over them; Abar is computed again on the way
+// back rather than kept, and Abar_t h_t-1 is taken as h_t - Delta_t B_t u_t.  dB and dC sum over the channels of a batch row: the
+// warp reduces its 32 channels with shuffles (8 values per lane and step) and
+// one lane per value adds the sum to global memory atomically.  dA, dD and
+// the bias gradient are summed per lane over the segment and added once.
+#pragma once
+
+#include "selective_scan.cuh"
+
+namespace mamba {
+
+constexpr int kBwdWarps = 4;
+constexpr int kBwdSteps = kCkptSteps;      // steps per block (one checkpoint each)
+
+struct BwdParams {
+    const void* u;
+    const void* delta;
+    const void* z;
+    const void* dout;
+    const float* A;
+    const void* B;
+    const void* C;
+    const float* D;
+    const float* delta_bias;
+    const float* dlast;        // (batch, dim, dstate) or null
+    const float* ckpt;         // [chains][ckpt_tiles][16]
+    void* du;
+    void* ddelta;
+    void* dz;
+    float* dA;                 // (dim, dstate), accumulated
+    float* dB;                 // (batch, dstate, seqlen), accumulated
+    float* dC;
+    float* dD;                 // (dim) or null, accumulated
+    float* dbias;              // (dim) or null, accumulated
+    float* dh0;                // (batch, dim, dstate) or null
+    unsigned int* counter;
+    unsigned int* flags;       // [groups] segments finished, counted from the end
+    float* carry;              // [chains][16] lambda handed to the earlier segment
+    int64_t batch, dim, seqlen, groups_per_batch, groups, chains, seg_len, items, ckpt_tiles;
+    int dstate;
+    int nseg;
+    int softplus;
+    int bc_bf16;
+    int vec_ok;                // u, delta, z, dout, du, ddelta, dz all 16-byte aligned
+    int bc_vec;                // B and C rows 16-byte aligned
+    unsigned int flag_poll_limit;
+};
+
+// kBwdSteps consecutive elements t0.. of a row as fp32 (zero past `n`); one
+// 16-byte load when the row is 16-byte aligned at t0 and the block is whole.
+template <typename T>
+__device__ __forceinline__ void load_block(const T* row, int64_t t0, int n, bool vec,
+                                           float (&v)[kBwdSteps]) {
+    if (vec && n == kBwdSteps) {
+        if constexpr (sizeof(T) == 2) {
+            unpack16(*reinterpret_cast<const uint4*>(row + t0), v);
+        } else {
+            float a[4], b[4];
+            unpack16(*reinterpret_cast<const uint4*>(row + t0), a);
+            unpack16(*reinterpret_cast<const uint4*>(row + t0 + 4), b);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) { v[i] = a[i]; v[4 + i] = b[i]; }
+        }
+        return;
+    }
+#pragma unroll
+    for (int i = 0; i < kBwdSteps; ++i) v[i] = i < n ? DType<T>::load(row + t0 + i) : 0.0f;
+}
+
+template <typename T>
+__device__ __forceinline__ void store_block(T* row, int64_t t0, int n, bool vec,
+                                            const float (&v)[kBwdSteps]) {
+    if (vec && n == kBwdSteps) {
+        if constexpr (sizeof(T) == 2) {
+            *reinterpret_cast<uint4*>(row + t0) = pack16(v);
+        } else {
+            const float a[4] = {v[0], v[1], v[2], v[3]}, b[4] = {v[4], v[5], v[6], v[7]};
+            *reinterpret_cast<uint4*>(row + t0) = pack16(a);
+            *reinterpret_cast<uint4*>(row + t0 + 4) = pack16(b);
+        }
+        return;
+    }
+#pragma unroll
+    for (int i = 0; i < kBwdSteps; ++i)
+        if (i < n) DType<T>::store(row + t0 + i, v[i]);
+}
+
+// Sum of v[j] over the warp's 32 lanes for j < 8.  Three halving exchanges
+// leave lane l with the partial sum of value (l >> 2) over 8 lanes; two
+// butterflies complete it on all four lanes of the quad.
+__device__ __forceinline__ float warp_reduce8(float (&v)[8], int lane) {
+#pragma unroll
+    for (int lvl = 0; lvl < 3; ++lvl) {
+        const int off = 16 >> lvl;               // 16, 8, 4
+        const int half = 4 >> lvl;               // values kept: 4, 2, 1
+        const bool upper = (lane & off) != 0;
+#pragma unroll
+        for (int i = 0; i < half; ++i) {
+            const float send = upper ? v[i] : v[i + half];
+            const float keep = upper ? v[i + half] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+    }
+    float r = v[0];
+    r += __shfl_xor_sync(0xffffffffu, r, 2);
+    r += __shfl_xor_sync(0xffffffffu, r, 1);
+    return r;                                    // total of value (lane >> 2)
+}
+
+__device__ __forceinline__ float sigmoid_f32(float x) {
+    return __fdividef(1.0f, 1.0f + ex2_approx(-x * kLog2e));
+}
+
+// Abar and Delta as the forward computes them (MUFU ex2 and the lg2 softplus
+// for bf16 inputs, the unbiased forms for fp32), so that the recomputed states
+// follow the forward's arithmetic.
+template <bool kExact>
+__device__ __forceinline__ float bwd_exp2(float x) {
+    return kExact ? exp2_near_one_exact(x) : ex2_approx(x);
+}
+
+template <typename IoT, typename BcT, bool kHasZ>
+__global__ void __launch_bounds__(kBwdWarps * 32, 3)
+    selective_scan_bwd_kernel(const __grid_constant__ BwdParams p) {
+    constexpr bool kExact = sizeof(IoT) == 4;
+    __shared__ __align__(16) float bcf_all[kBwdWarps][kBwdSteps][32];
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    float (*bcf)[32] = bcf_all[warp];
+
+    for (;;) {
+        unsigned int item = 0;
+        if (lane == 0) item = atomicAdd(p.counter, 1u);
+        item = __shfl_sync(0xffffffffu, item, 0);
+        if ((int64_t)item >= p.items) break;
+        const int64_t g = item % p.groups;
+        const int64_t kr = item / p.groups;                  // segments done after this one
+        const int64_t k = p.nseg - 1 - kr;
+        const int64_t b = g / p.groups_per_batch;
+        const int64_t d0 = (g % p.groups_per_batch) * 32;
+        const int64_t d = d0 + lane;
+        const bool valid = d < p.dim;
+        const int64_t chain = b * p.dim + (valid ? d : 0);
+        const int64_t t_begin = k * p.seg_len;
+        const int64_t t_end = min(t_begin + p.seg_len, p.seqlen);
+
+        float a2[kNPad];
+#pragma unroll
+        for (int n = 0; n < kNPad; ++n)
+            a2[n] = (valid && n < p.dstate) ? p.A[d * p.dstate + n] * kLog2e : 0.0f;
+        const float bias = (valid && p.delta_bias != nullptr) ? p.delta_bias[d] : 0.0f;
+        const float Dd = (valid && p.D != nullptr) ? p.D[d] : 0.0f;
+
+        float lam[kNPad];
+        if (kr == 0) {
+#pragma unroll
+            for (int n = 0; n < kNPad; ++n)
+                lam[n] = (valid && p.dlast != nullptr && n < p.dstate)
+                             ? p.dlast[chain * p.dstate + n] : 0.0f;
+        } else {
+            bool ok = true;
+            if (lane == 0) {
+                ok = false;
+                for (uint32_t i = 0; i < p.flag_poll_limit; ++i) {
+                    if (ld_acquire_gpu(p.flags + g) >= (unsigned int)kr) {
+                        ok = true;
+                        break;
+                    }
+                    __nanosleep(1000);
+                }
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) {
+                if (lane == 0) record_device_error(MAMBA_ERR_TIMEOUT);
+                break;
+            }
+            (void)ld_acquire_gpu(p.flags + g);
+            float2 c2[kNPad / 2];
+            load16(p.carry + chain * kNPad, c2);
+#pragma unroll
+            for (int i = 0; i < kNPad / 2; ++i) {
+                lam[2 * i] = valid ? c2[i].x : 0.0f;
+                lam[2 * i + 1] = valid ? c2[i].y : 0.0f;
+            }
+        }
+        float dA_acc[kNPad];
+#pragma unroll
+        for (int n = 0; n < kNPad; ++n) dA_acc[n] = 0.0f;
+        float dD_acc = 0.0f, dbias_acc = 0.0f;
+
+        const IoT* urow = static_cast<const IoT*>(p.u) + chain * p.seqlen;
+        const IoT* drow = static_cast<const IoT*>(p.delta) + chain * p.seqlen;
+        const IoT* zrow = kHasZ ? static_cast<const IoT*>(p.z) + chain * p.seqlen : nullptr;
+        const IoT* grow = static_cast<const IoT*>(p.dout) + chain * p.seqlen;
+        const bool vec = p.vec_ok && (p.seqlen * (int64_t)sizeof(IoT)) % 16 == 0 && valid;
+        const int nblk = (int)((t_end - t_begin + kBwdSteps - 1) / kBwdSteps);
+
+        for (int j = nblk - 1; j >= 0; --j) {
+            const int64_t t0 = t_begin + (int64_t)j * kBwdSteps;
+            const int ns = (int)min((int64_t)kBwdSteps, t_end - t0);
+            // ---- inputs of this block: the lane's own channel, and the B/C table
+            float uu[kBwdSteps], dt[kBwdSteps], dy[kBwdSteps], aux[kBwdSteps];
+            if (valid) {
+                load_block(urow, t0, ns, vec, uu);
+                load_block(drow, t0, ns, vec, dt);       // delta, turned into Delta below
+                load_block(grow, t0, ns, vec, dy);       // dout, turned into dy below
+                if (kHasZ) load_block(zrow, t0, ns, vec, aux);
+            } else {
+#pragma unroll
+                for (int i = 0; i < kBwdSteps; ++i) uu[i] = dt[i] = dy[i] = aux[i] = 0.0f;
+            }
+            {
+                const int n = lane & 15;
+                const BcT* src = static_cast<const BcT*>(lane < 16 ? p.B : p.C) +
+                                 (b * p.dstate + (n < p.dstate ? n : 0)) * p.seqlen;
+                float row[kBwdSteps];
+                if (n < p.dstate) {
+                    load_block(src, t0, ns, p.bc_vec != 0, row);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < kBwdSteps; ++i) row[i] = 0.0f;
+                }
+                __syncwarp();
+#pragma unroll
+                for (int i = 0; i < kBwdSteps; ++i) bcf[i][lane] = row[i];
+                __syncwarp();
+            }
+            // Delta, the softplus derivative (kept in dt / sp), dy and the gate factor.
+            float sp[kBwdSteps];
+#pragma unroll
+            for (int i = 0; i < kBwdSteps; ++i) {
+                const float s = dt[i] + bias;
+                dt[i] = p.softplus ? (kExact ? softplus_f32(s) : softplus_lg2(s)) : s;
+                sp[i] = p.softplus ? sigmoid_f32(s) : 1.0f;
+                if (kHasZ) {
+                    const float zv = aux[i];
+                    const float sg = sigmoid_f32(zv);
+                    const float g = dy[i];
+                    dy[i] = g * zv * sg;                              // dout * silu(z)
+                    aux[i] = g * sg * fmaf(zv, 1.0f - sg, 1.0f);      // dout * silu'(z)
+                }
+            }
+            float y[kBwdSteps], ddt[kBwdSteps], dlb[kBwdSteps];
+#pragma unroll
+            for (int i = 0; i < kBwdSteps; ++i) y[i] = ddt[i] = dlb[i] = 0.0f;
+            const float* ck = p.ckpt + (chain * p.ckpt_tiles + t0 / kBwdSteps) * kNPad;
+
+#pragma unroll
+            for (int q = 0; q < kNPad / 4; ++q) {
+                const int n0 = 4 * q;
+                // forward: the block's 8 states of entries n0..n0+3
+                const float4 hs4 = valid ? __ldcg(reinterpret_cast<const float4*>(ck + n0))
+                                         : make_float4(0.f, 0.f, 0.f, 0.f);
+                float hq[kBwdSteps][4];
+                float h[4] = {hs4.x, hs4.y, hs4.z, hs4.w};
+#pragma unroll
+                for (int t = 0; t < kBwdSteps; ++t) {
+                    if (t < ns) {
+                        const float4 Bq = *reinterpret_cast<const float4*>(&bcf[t][n0]);
+                        const float4 Cq = *reinterpret_cast<const float4*>(&bcf[t][16 + n0]);
+                        const float bq[4] = {Bq.x, Bq.y, Bq.z, Bq.w};
+                        const float cq[4] = {Cq.x, Cq.y, Cq.z, Cq.w};
+                        const float du = dt[t] * uu[t];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const float ab = bwd_exp2<kExact>(dt[t] * a2[n0 + i]);
+                            h[i] = fmaf(ab, h[i], du * bq[i]);
+                            hq[t][i] = h[i];
+                            y[t] = fmaf(cq[i], h[i], y[t]);
+                        }
+                    }
+                }
+                // reverse: the adjoint of entries n0..n0+3 over the block
+                float l4[4] = {lam[n0], lam[n0 + 1], lam[n0 + 2], lam[n0 + 3]};
+#pragma unroll
+                for (int t = kBwdSteps - 1; t >= 0; --t) {
+                    if (t < ns) {
+                        const float4 Bq = *reinterpret_cast<const float4*>(&bcf[t][n0]);
+                        const float4 Cq = *reinterpret_cast<const float4*>(&bcf[t][16 + n0]);
+                        const float bq[4] = {Bq.x, Bq.y, Bq.z, Bq.w};
+                        const float cq[4] = {Cq.x, Cq.y, Cq.z, Cq.w};
+                        const float du = dt[t] * uu[t];
+                        float red[8];
+                        float s_dt = 0.0f, s_b = 0.0f;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            l4[i] = fmaf(cq[i], dy[t], l4[i]);                 // lambda_t
+                            const float ab = bwd_exp2<kExact>(dt[t] * a2[n0 + i]);
+                            const float abh = fmaf(-du, bq[i], hq[t][i]);      // Abar_t h_t-1 = h_t - b_t
+                            red[i] = l4[i] * du;                                // dB
+                            red[4 + i] = dy[t] * hq[t][i];                      // dC
+                            s_dt = fmaf(l4[i], fmaf(a2[n0 + i] * kLn2, abh, bq[i] * uu[t]), s_dt);
+                            s_b = fmaf(l4[i], bq[i], s_b);
+                            dA_acc[n0 + i] = fmaf(l4[i] * dt[t], abh, dA_acc[n0 + i]);
+                            l4[i] *= ab;                                        // to h_t-1
+                        }
+                        ddt[t] += s_dt;
+                        dlb[t] += s_b;
+                        const float tot = warp_reduce8(red, lane);
+                        const int idx = lane >> 2;                              // 0..7
+                        const int n = n0 + (idx & 3);
+                        if ((lane & 3) == 0 && n < p.dstate) {
+                            float* dst = (idx < 4 ? p.dB : p.dC) + (b * p.dstate + n) * p.seqlen + t0 + t;
+                            atomicAdd(dst, tot);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) lam[n0 + i] = l4[i];
+            }
+            // per-step outputs of the block
+            float o_du[kBwdSteps], o_dd[kBwdSteps], o_dz[kBwdSteps];
+#pragma unroll
+            for (int t = 0; t < kBwdSteps; ++t) {
+                const bool in = t < ns;
+                o_du[t] = fmaf(Dd, dy[t], dt[t] * dlb[t]);
+                const float ds = ddt[t] * sp[t];
+                o_dd[t] = ds;
+                if (in) {
+                    dbias_acc += ds;
+                    dD_acc = fmaf(dy[t], uu[t], dD_acc);
+                }
+                o_dz[t] = kHasZ ? aux[t] * fmaf(Dd, uu[t], y[t]) : 0.0f;
+            }
+            if (valid) {
+                store_block(static_cast<IoT*>(p.du) + chain * p.seqlen, t0, ns, vec, o_du);
+                store_block(static_cast<IoT*>(p.ddelta) + chain * p.seqlen, t0, ns, vec, o_dd);
+                if (kHasZ && p.dz != nullptr)
+                    store_block(static_cast<IoT*>(p.dz) + chain * p.seqlen, t0, ns, vec, o_dz);
+            }
+        }
+
+        // hand lambda to the earlier segment, or it is the start state's gradient
+        if (k > 0) {
+            float2 c2[kNPad / 2];
+#pragma unroll
+            for (int i = 0; i < kNPad / 2; ++i) c2[i] = make_float2(lam[2 * i], lam[2 * i + 1]);
+            if (valid) store16(p.carry + chain * kNPad, c2);
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) st_release_gpu(p.flags + g, (unsigned int)(kr + 1));
+        } else if (valid && p.dh0 != nullptr) {
+#pragma unroll
+            for (int n = 0; n < kNPad; ++n)
+                if (n < p.dstate) p.dh0[chain * p.dstate + n] = lam[n];
+        }
+        if (valid) {
+#pragma unroll
+            for (int n = 0; n < kNPad; ++n)
+                if (n < p.dstate) atomicAdd(p.dA + d * p.dstate + n, dA_acc[n]);
+            if (p.dD != nullptr) atomicAdd(p.dD + d, dD_acc);
+            if (p.dbias != nullptr) atomicAdd(p.dbias + d, dbias_acc);
+        }
+    }
+}
+
+}  // namespace mamba

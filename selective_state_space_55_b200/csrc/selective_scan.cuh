@@ -55,6 +55,7 @@ constexpr int kNPad = 16;                  // compiled state size (smaller N is 
 constexpr int kMaxTile = kRowBytes / 2;    // time steps per tile for 2-byte inputs
 constexpr int kBcRawBytes = kNPad * kMaxTile * 4;   // 16 rows of up to 64 bytes
 constexpr int kBcfBytes = kMaxTile * 32 * 4;        // [T][32] fp32
+constexpr int kCkptSteps = 8;                         // backward checkpoint spacing (steps)
 
 // Shared-memory layout and residency of the kernel with kCpl channels per lane.
 template <int kCpl>
@@ -110,7 +111,10 @@ struct ScanParams {
     unsigned int flag_poll_limit;   // chained mode: polls (~1 us each) before a wait gives up
     int withhold_handoff;    // test only: segments never publish their state (waits time out)
     const float* h0;         // (batch, dim, dstate) start state of segment 0, or null (zero)
+    float* ckpt;             // backward's checkpoint pass: [chains][ckpt_tiles][16], or null
+    int64_t ckpt_tiles;      // ceil(seqlen / kCkptSteps)
 };
+
 
 // Byte offset of (row r, byte x of the row) in a 32-byte-row tile written by
 // TMA with 32-byte swizzle: address bit 4 is XORed with bit 7.
@@ -167,6 +171,24 @@ struct LaneChains {
     float bias[kCpl];
     float Dd[kCpl];
 };
+
+// 16 fp32 state values <-> 64 bytes of memory (L2-cached, no L1 allocation).
+__device__ __forceinline__ void store16(float* dst, const float2 (&h)[kNPad / 2]) {
+    float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        __stcg(d4 + q, make_float4(h[2 * q].x, h[2 * q].y, h[2 * q + 1].x, h[2 * q + 1].y));
+}
+
+__device__ __forceinline__ void load16(const float* src, float2 (&h)[kNPad / 2]) {
+    const float4* s4 = reinterpret_cast<const float4*>(src);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const float4 v = __ldcg(s4 + q);
+        h[2 * q] = make_float2(v.x, v.y);
+        h[2 * q + 1] = make_float2(v.z, v.w);
+    }
+}
 
 // 2^x for both halves of x: MUFU ex2, or exp2_near_one_exact (fp32 path).
 template <bool kExact>
@@ -245,11 +267,12 @@ __device__ __forceinline__ void scan_step(const float* bc_row, const float (&dt)
 // all V steps are formed first: their softplus chains are independent of the
 // state, so computing them together lets their latency overlap.  The vectors
 // stay packed and are unpacked element by element to save registers.
-template <typename IoT, int kCpl, bool kHasZ, bool kSoftplus, bool kZoh, bool kOut>
+template <typename IoT, int kCpl, bool kHasZ, bool kSoftplus, bool kZoh, bool kOut, bool kCkpt>
 __device__ __forceinline__ void compute_tile(const uint8_t* st, const float* bcf, int lane,
                                              int nsteps, LaneChains<kCpl>& lc,
                                              IoT* const (&out_row)[kCpl], bool vec_out,
-                                             float (&sdt)[kCpl], float (&sdt_c)[kCpl]) {
+                                             float (&sdt)[kCpl], float (&sdt_c)[kCpl],
+                                             float* const (&ck)[kCpl]) {
     using Lay = ScanLayout<kCpl>;
     constexpr int V = 16 / (int)sizeof(IoT);          // steps per 16-byte vector
     constexpr int T = kRowBytes / (int)sizeof(IoT);   // steps per tile
@@ -268,6 +291,11 @@ __device__ __forceinline__ void compute_tile(const uint8_t* st, const float* bcf
             if (kHasZ && kOut) zr[c] = *reinterpret_cast<const uint4*>(st + Lay::kOffZ + so);
         }
         const int steps = min(V, nsteps - base);
+        if (kCkpt && base % kCkptSteps == 0) {
+#pragma unroll
+            for (int c = 0; c < kCpl; ++c)
+                if (ck[c] != nullptr) store16(ck[c] + (base / kCkptSteps) * kNPad, lc.h[c]);
+        }
         bool whole[kCpl];
 #pragma unroll
         for (int c = 0; c < kCpl; ++c) whole[c] = steps == V && vec_out && out_row[c] != nullptr;
@@ -399,12 +427,12 @@ struct TmaMaps {
 // counts the tiles this warp has consumed (it fixes each tile's stage and
 // mbarrier parity across items).  Returns false if a staged tile never
 // arrived (the warp has then waited, bounded, for its copies in flight).
-template <typename IoT, int kCpl, bool kHasZ, bool kSoftplus, bool kZoh, bool kOut>
+template <typename IoT, int kCpl, bool kHasZ, bool kSoftplus, bool kZoh, bool kOut, bool kCkpt>
 __device__ __forceinline__ bool run_segment(const ScanParams& p, const TmaMaps& maps, uint8_t* wsm,
                                             int lane, int64_t b, int64_t d0, int64_t t_begin,
                                             int64_t t_end, LaneChains<kCpl>& lc,
                                             IoT* const (&out_row)[kCpl], uint32_t& seq,
-                                            float (&sdt)[kCpl]) {
+                                            float (&sdt)[kCpl], float* const (&ckpt_row)[kCpl]) {
     using Lay = ScanLayout<kCpl>;
     constexpr int T = kRowBytes / (int)sizeof(IoT);
     constexpr bool kNeedZ = kHasZ && kOut;
@@ -463,32 +491,20 @@ __device__ __forceinline__ bool run_segment(const ScanParams& p, const TmaMaps& 
         }
         __syncwarp();
         IoT* rows[kCpl];
+        float* cks[kCpl];
 #pragma unroll
-        for (int c = 0; c < kCpl; ++c) rows[c] = out_row[c] ? out_row[c] + (t0 - t_begin) : nullptr;
-        compute_tile<IoT, kCpl, kHasZ, kSoftplus, kZoh, kOut>(st, bcf, lane, nsteps, lc, rows,
-                                                              p.vec_out != 0, sdt, sdt_c);
+        for (int c = 0; c < kCpl; ++c) {
+            rows[c] = out_row[c] ? out_row[c] + (t0 - t_begin) : nullptr;
+            cks[c] = (kCkpt && ckpt_row[c]) ? ckpt_row[c] + ((t0 - t_begin) / kCkptSteps) * kNPad
+                                            : nullptr;
+        }
+        compute_tile<IoT, kCpl, kHasZ, kSoftplus, kZoh, kOut, kCkpt>(
+            st, bcf, lane, nsteps, lc, rows, p.vec_out != 0, sdt, sdt_c, cks);
         __syncwarp();
         if (p.use_tma && lane == 0 && i + kScanStages < ntiles) issue(i + kScanStages);
     }
     seq += (uint32_t)ntiles;
     return true;
-}
-
-__device__ __forceinline__ void store16(float* dst, const float2 (&h)[kNPad / 2]) {
-    float4* d4 = reinterpret_cast<float4*>(dst);
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-        __stcg(d4 + q, make_float4(h[2 * q].x, h[2 * q].y, h[2 * q + 1].x, h[2 * q + 1].y));
-}
-
-__device__ __forceinline__ void load16(const float* src, float2 (&h)[kNPad / 2]) {
-    const float4* s4 = reinterpret_cast<const float4*>(src);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const float4 v = __ldcg(s4 + q);
-        h[2 * q] = make_float2(v.x, v.y);
-        h[2 * q + 1] = make_float2(v.z, v.w);
-    }
 }
 
 __device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int* p) {
@@ -614,19 +630,27 @@ __global__ void __launch_bounds__(kScanWarps * 32, ScanLayout<kCpl>::kMinBlocks 
         }
 
         IoT* out_row[kCpl];
+        float* ckpt_row[kCpl];
         float sdt[kCpl];
 #pragma unroll
         for (int c = 0; c < kCpl; ++c) {
-            out_row[c] = valid[c] ? static_cast<IoT*>(p.out) + chain[c] * p.seqlen + t_begin : nullptr;
+            out_row[c] = (valid[c] && p.out != nullptr)
+                             ? static_cast<IoT*>(p.out) + chain[c] * p.seqlen + t_begin : nullptr;
+            ckpt_row[c] = (valid[c] && p.ckpt != nullptr)
+                              ? p.ckpt + (chain[c] * p.ckpt_tiles + t_begin / kCkptSteps) * kNPad
+                              : nullptr;
             sdt[c] = 0.0f;
         }
         bool ok;
-        if (p.mode == kModePassA && k > 0)
-            ok = run_segment<IoT, kCpl, kHasZ, kSoftplus, kZoh, false>(
-                p, maps, wsm, lane, b, d0, t_begin, t_end, lc, out_row, seq, sdt);
+        if (p.ckpt != nullptr)           // checkpoint pass of the backward: states only
+            ok = run_segment<IoT, kCpl, kHasZ, kSoftplus, kZoh, false, true>(
+                p, maps, wsm, lane, b, d0, t_begin, t_end, lc, out_row, seq, sdt, ckpt_row);
+        else if (p.mode == kModePassA && k > 0)
+            ok = run_segment<IoT, kCpl, kHasZ, kSoftplus, kZoh, false, false>(
+                p, maps, wsm, lane, b, d0, t_begin, t_end, lc, out_row, seq, sdt, ckpt_row);
         else
-            ok = run_segment<IoT, kCpl, kHasZ, kSoftplus, kZoh, true>(
-                p, maps, wsm, lane, b, d0, t_begin, t_end, lc, out_row, seq, sdt);
+            ok = run_segment<IoT, kCpl, kHasZ, kSoftplus, kZoh, true, false>(
+                p, maps, wsm, lane, b, d0, t_begin, t_end, lc, out_row, seq, sdt, ckpt_row);
         if (!ok) break;
 
         const bool last_seg = k == p.nseg - 1;

@@ -94,6 +94,10 @@ def library(path: Path | str | None = None) -> ctypes.CDLL:
     lib.mamba_selective_scan_fwd_host.restype = i32
     lib.mamba_selective_scan_fwd_host.argtypes = [
         vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, ctypes.c_int64, dims_p, vp]
+    lib.mamba_selective_scan_bwd_workspace_bytes.restype = ctypes.c_size_t
+    lib.mamba_selective_scan_bwd_workspace_bytes.argtypes = [dims_p]
+    lib.mamba_selective_scan_bwd.restype = i32
+    lib.mamba_selective_scan_bwd.argtypes = [vp] * 8 + [i32] + [vp] * 12 + [dims_p, vp]
     lib.mamba_causal_conv1d_fwd.restype = i32
     lib.mamba_causal_conv1d_fwd.argtypes = [vp, vp, vp, vp, i32, i32, vp, vp, dims_p, vp]
     lib.mamba_causal_conv1d_update.restype = i32
@@ -333,6 +337,67 @@ def selective_state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=None,
     if rc != MAMBA_OK:
         raise MambaError("mamba_selective_state_update", rc)
     return out
+
+
+def scan_bwd_workspace_bytes(batch, dim, dstate, seqlen, io_dtype=torch.bfloat16,
+                             bc_dtype=torch.bfloat16) -> int:
+    """Scratch bytes of ``selective_scan_bwd`` on the current device."""
+    dims = make_scan_dims(batch, dim, dstate, seqlen, io_dtype, bc_dtype)
+    n = library().mamba_selective_scan_bwd_workspace_bytes(ctypes.byref(dims))
+    if n == ctypes.c_size_t(-1).value:
+        raise MambaError("mamba_selective_scan_bwd_workspace_bytes", -1)
+    return int(n)
+
+
+def selective_scan_bwd(u, delta, A, B, C, dout, D=None, z=None, delta_bias=None, softplus=True,
+                       initial_state=None, dlast_state=None, flags=0, workspace=None,
+                       stream=None):
+    """Gradients of the scan through ``mamba_selective_scan_bwd``.
+
+    Same inputs as ``selective_scan_fwd`` (Euler term) plus dout (batch, dim, L)
+    in u's dtype and dlast_state (batch, dim, N) fp32 or None.  Returns a dict:
+    du, ddelta (and dz when z is given) in u's dtype; dA, dB, dC (and dD,
+    ddelta_bias, dinitial_state for the optional inputs given) in fp32.
+    """
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    io, bc = u.dtype, B.dtype
+    dev = u.device
+    _check_cuda("u", u, (torch.float32, torch.bfloat16), (batch, dim, L))
+    for name, t in (("delta", delta), ("z", z), ("dout", dout)):
+        _check_cuda(name, t, (io,), (batch, dim, L))
+    _check_cuda("A", A, (torch.float32,), (dim, N))
+    _check_cuda("B", B, (torch.float32, torch.bfloat16), (batch, N, L))
+    _check_cuda("C", C, (bc,), (batch, N, L))
+    _check_cuda("D", D, (torch.float32,), (dim,))
+    _check_cuda("delta_bias", delta_bias, (torch.float32,), (dim,))
+    _check_cuda("initial_state", initial_state, (torch.float32,), (batch, dim, N))
+    _check_cuda("dlast_state", dlast_state, (torch.float32,), (batch, dim, N))
+    g = {"du": torch.empty_like(u), "ddelta": torch.empty_like(u),
+         "dA": torch.empty((dim, N), dtype=torch.float32, device=dev),
+         "dB": torch.empty((batch, N, L), dtype=torch.float32, device=dev),
+         "dC": torch.empty((batch, N, L), dtype=torch.float32, device=dev)}
+    if z is not None:
+        g["dz"] = torch.empty_like(u)
+    if D is not None:
+        g["dD"] = torch.empty((dim,), dtype=torch.float32, device=dev)
+    if delta_bias is not None:
+        g["ddelta_bias"] = torch.empty((dim,), dtype=torch.float32, device=dev)
+    if initial_state is not None:
+        g["dinitial_state"] = torch.empty((batch, dim, N), dtype=torch.float32, device=dev)
+    if workspace is None:
+        need = scan_bwd_workspace_bytes(batch, dim, N, L, io, bc)
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    dims = make_scan_dims(batch, dim, N, L, io, bc, 0, flags, workspace)
+    rc = library().mamba_selective_scan_bwd(
+        _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
+        int(bool(softplus)), _ptr(initial_state), _ptr(dout), _ptr(dlast_state), _ptr(g["du"]),
+        _ptr(g["ddelta"]), _ptr(g["dA"]), _ptr(g["dB"]), _ptr(g["dC"]), _ptr(g.get("dD")),
+        _ptr(g.get("dz")), _ptr(g.get("ddelta_bias")), _ptr(g.get("dinitial_state")),
+        ctypes.byref(dims), _stream_handle(stream))
+    if rc != MAMBA_OK:
+        raise MambaError("mamba_selective_scan_bwd", rc)
+    return g
 
 
 def _conv_dims(batch, dim, seqlen, io_dtype) -> MambaDims:

@@ -21,10 +21,14 @@ def as_f64(t):
 
 
 def max_rel_err(got, want) -> float:
+    """The error metric above; infinity when either side holds a non-finite
+    value, so that a NaN can never pass a tolerance."""
     got, want = as_f64(got), as_f64(want)
     assert got.shape == want.shape, (got.shape, want.shape)
     if want.size == 0:
         return 0.0
+    if not (np.all(np.isfinite(got)) and np.all(np.isfinite(want))):
+        return float("inf")
     rms = float(np.sqrt(np.mean(want * want)))
     denom = np.maximum(np.abs(want), rms)
     denom = np.where(denom > 0, denom, 1.0)

@@ -141,6 +141,21 @@ def test_conv_rejects_bad_arguments(lib):
     assert upd(d, 4, w=ctypes.c_void_p(0x10002)) == -3  # fp32 weights need 4-byte alignment
 
 
+def test_backward_rejects_bad_arguments(lib):
+    d = _dims()
+    call = lambda dims, u=FAKE, A=FAKE, dout=FAKE, du=FAKE, dA=FAKE: lib.mamba_selective_scan_bwd(  # noqa: E731
+        u, FAKE, A, FAKE, FAKE, None, None, None, 1, None, dout, None, du, FAKE, dA, FAKE, FAKE,
+        None, None, None, None, ctypes.byref(dims) if dims is not None else None, None)
+    assert call(None) == -1
+    assert call(_dims(dstate=17)) == -2
+    zoh = _dims(); zoh.flags = ops.MAMBA_FLAG_ZOH
+    assert call(zoh) == -2                             # zero-order hold: forward only
+    assert call(d, u=None) == -1 and call(d, dout=None) == -1 and call(d, du=None) == -1
+    assert call(d, A=None) == -1 and call(d, dA=None) == -1
+    assert call(d, u=ctypes.c_void_p(0x10001)) == -3
+    assert call(_dims(batch=0)) == 0
+
+
 def test_scan_empty_batch_is_a_no_op(lib):
     assert _scan(lib, _dims(batch=0)) == 0
     assert _scan(lib, _dims(dim=0)) == 0

@@ -1,0 +1,102 @@
+"""Backward pass of the scan (mamba_selective_scan_bwd): every gradient against
+the float64 oracle's adjoint, which finite differences of the forward oracle
+pin.  fp32 and bf16, with and without gate / D / bias / softplus / start
+state / last-state gradient, state sizes below 16, ragged lengths and channel
+counts, and sequences cut into many chained segments."""
+import pytest
+import torch
+
+from oracle import oracle
+from parity import BF16_TOL, FP32_TOL, max_rel_err, tol_for
+from selective_state_space_55_b200 import inputs as I
+from selective_state_space_55_b200 import ops
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module")
+def ref():
+    return oracle.default()
+
+
+def problem(batch, dim, L, dtype=torch.float32, N=16, seed=0, gated=True):
+    cfg = I.SCAN_CONFIGS["mamba_1p4b_layer"].resized(batch=batch, dim=dim, seqlen=L, dstate=N,
+                                                       io_dtype=dtype, bc_dtype=dtype)
+    x = I.make_scan_inputs(cfg, DEV, seed)
+    g = torch.Generator(device=DEV)
+    g.manual_seed(seed + 99)
+    x["dout"] = torch.randn(batch, dim, L, generator=g, device=DEV).to(dtype)
+    x["h0"] = torch.randn(batch, dim, N, generator=g, device=DEV) if gated else None
+    x["dlast"] = torch.randn(batch, dim, N, generator=g, device=DEV) if gated else None
+    if not gated:
+        x["z"] = x["D"] = x["delta_bias"] = None
+    return x
+
+
+def check(ref, x, tol, softplus=True, **kw):
+    g = ops.selective_scan_bwd(x["u"], x["delta"], x["A"], x["B"], x["C"], x["dout"], D=x["D"],
+                               z=x["z"], delta_bias=x["delta_bias"], softplus=softplus,
+                               initial_state=x["h0"], dlast_state=x["dlast"], **kw)
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    c = lambda t: None if t is None else t.cpu()  # noqa: E731
+    o = ref.selective_scan_bwd(c(x["u"]), c(x["delta"]), c(x["A"]), c(x["B"]), c(x["C"]),
+                               c(x["dout"]), D=c(x["D"]), z=c(x["z"]), delta_bias=c(x["delta_bias"]),
+                               softplus=softplus, initial_state=c(x["h0"]), dlast_state=c(x["dlast"]))
+    assert set(g) == set(o), (set(g), set(o))
+    errs = {k: max_rel_err(g[k], o[k]) for k in o}
+    bad = {k: e for k, e in errs.items() if e > tol}
+    assert not bad, f"gradients beyond {tol:.0e}: {bad}"
+    return errs
+
+
+def test_fp32_all_gradients(ref):
+    check(ref, problem(2, 70, 300, seed=1), FP32_TOL)
+
+
+def test_fp32_plain(ref):
+    """No gate, D, bias, start state or last-state gradient; softplus off (Delta =
+    delta itself, drawn positive so that the state decays)."""
+    x = problem(2, 40, 200, seed=2, gated=False)
+    x["delta"] = x["delta"].abs() * 0.1
+    check(ref, x, FP32_TOL, softplus=False)
+
+
+@pytest.mark.parametrize("N", [1, 5, 8])
+def test_state_sizes(ref, N):
+    check(ref, problem(1, 33, 130, N=N, seed=3 + N), FP32_TOL)
+
+
+@pytest.mark.parametrize("L", [1, 7, 8, 9, 257])
+def test_ragged_lengths(ref, L):
+    check(ref, problem(2, 32, L, seed=10 + L), FP32_TOL)
+
+
+def test_many_segments(ref):
+    """Few chains and a long sequence: 16 chained segments hand lambda backwards."""
+    check(ref, problem(1, 64, 4096, seed=20), FP32_TOL)
+
+
+def test_bf16_layer_recipe(ref):
+    check(ref, problem(2, 256, 2048, dtype=torch.bfloat16, seed=21), BF16_TOL)
+
+
+def test_last_state_gradient_only(ref):
+    """dout = 0: every gradient flows from dlast_state through the adjoint alone."""
+    x = problem(2, 48, 333, seed=22)
+    x["dout"] = torch.zeros_like(x["dout"])
+    check(ref, x, FP32_TOL)
+
+
+def test_unaligned_rows_take_scalar_path(ref):
+    """A length whose rows are not 16-byte aligned (L * 4 % 16 != 0)."""
+    check(ref, problem(2, 36, 301, seed=23), FP32_TOL)
+
+
+def test_zoh_is_rejected():
+    x = problem(1, 32, 64, seed=24)
+    with pytest.raises(ops.MambaError, match="UNSUPPORTED"):
+        ops.selective_scan_bwd(x["u"], x["delta"], x["A"], x["B"], x["C"], x["dout"],
+                               flags=ops.MAMBA_FLAG_ZOH)
