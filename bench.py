@@ -599,6 +599,82 @@ def bench_conv(args, rank, world, local):
         print(json.dumps(line), flush=True)
 
 
+def bench_bwd(args, rank, world, local):
+    """Measurement case: the backward pass of the scan (checkpoint pass + adjoint)
+    on the Mamba-2.8B layer shape, gate, D and bias on, dout random."""
+    global _WORLD
+    _WORLD = world
+    from selective_state_space_55_b200 import build as cuda_build
+    from selective_state_space_55_b200 import inputs as I
+    from selective_state_space_55_b200 import ops
+    from selective_state_space_55_b200 import roofline as R
+
+    if rank == 0:
+        cuda_build.build()
+    barrier()
+    torch.cuda.set_device(local)
+    c = I.SCAN_CONFIGS[SCAN_WORKLOAD]
+    if args.scan_batch:
+        c = c.resized(batch=args.scan_batch)
+    x = I.make_scan_inputs(c, "cuda", seed=rank_seed(rank))
+    g = torch.Generator(device="cuda")
+    g.manual_seed(rank_seed(rank) + 13)
+    dout = torch.randn(c.batch, c.dim, c.seqlen, generator=g, device="cuda").to(c.io_dtype)
+    ws = torch.empty(ops.scan_bwd_workspace_bytes(c.batch, c.dim, c.dstate, c.seqlen, c.io_dtype,
+                                                  c.bc_dtype), dtype=torch.uint8, device="cuda")
+
+    def step():
+        return ops.selective_scan_bwd(x["u"], x["delta"], x["A"], x["B"], x["C"], dout, D=x["D"],
+                                      z=x["z"], delta_bias=x["delta_bias"], workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    K = args.steps
+    sampler = ClockSampler(local)
+    sampler.start()
+    barrier()
+    torch.cuda.synchronize()
+    t0 = time.time()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(K):
+        step()
+    e.record()
+    torch.cuda.synchronize()
+    t1 = time.time()
+    barrier()
+    sampler.stop()
+    ms = max_over_ranks(s.elapsed_time(e)) / K
+    peaks = measured_peaks()
+    # MUFU ops per element over both launches.  Checkpoint pass: 16 ex2 + the
+    # softplus (2).  Adjoint: 16 ex2 recomputing the states, 16 for Abar on the
+    # way back, the softplus again (2), its derivative sigmoid (2) and the
+    # gate's sigmoid (2).
+    mufu = (16 + 2) + (16 + 16 + 2 + 2 + 2)
+    peak = R.mufu_peak_elements_per_s(torch.cuda.get_device_properties(local).multi_processor_count,
+                                      peaks["sm_max_mhz"], mufu) / 1e9
+    value = world * c.elements / (ms * 1e-3) / 1e9
+    if rank == 0:
+        line = {
+            "metric": "selective-scan backward Gelem/s (Mamba-2.8B layer shape)", "value": round(value, 3),
+            "unit": "Gelem/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded)",
+            "config": {"workload": f"{c.name} backward ({c.batch}x{c.dim}, N={c.dstate}, L={c.seqlen}, "
+                                   "bf16, gate/D/bias, checkpoint pass + adjoint)",
+                       "checkpoint_bytes": ws.numel()},
+            "roofline": {"bound": "alu", "pipe": f"MUFU ({mufu} per element, both launches)",
+                         "achieved": round(value / world, 2), "peak": round(peak, 2), "unit": "Gelem/s",
+                         "frac": round(value / world / peak, 4), "traffic": None},
+            "gpu_launches": K * 2,
+            "clocks": sampler.summary(t0, t1),
+            "partial_case": {"only": "bwd", "scan_batch": args.scan_batch,
+                             "note": "measurement of the backward pass, not the benchmark workload"},
+        }
+        print(json.dumps(line), flush=True)
+
+
 def bench_reference(args, rank, world):
     """The float64 CPU oracle, on the same workload's metric, a bounded sample
     per step (rank 0 only)."""
@@ -660,8 +736,8 @@ def main():
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--reference-seconds", type=float, default=120.0,
                     help="budget of the whole --impl reference run")
-    ap.add_argument("--only", choices=["scan", "decode", "conv"], default=None,
-                    help="profiling case: one half of the step; conv: the short convolution")
+    ap.add_argument("--only", choices=["scan", "decode", "conv", "bwd"], default=None,
+                    help="profiling case: one half of the step; conv: the short convolution; bwd: the backward pass")
     ap.add_argument("--scan-batch", type=int, default=None,
                     help="profiling case: smaller scan batch")
     ap.add_argument("--decode-layers", type=int, default=None,
@@ -694,6 +770,8 @@ def main():
     try:
         if args.only == "conv":
             bench_conv(args, rank, world, local)
+        elif args.only == "bwd":
+            bench_bwd(args, rank, world, local)
         else:
             bench_ours(args, rank, world, local)
     finally:

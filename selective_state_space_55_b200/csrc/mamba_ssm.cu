@@ -1077,18 +1077,23 @@ mamba_status_t bwd_layout(const mamba_dims_t* dims, int sms, BwdWorkspace* w) {
 
 template <typename IoT, typename BcT, bool kHasZ>
 cudaError_t launch_bwd(const BwdParams& prm, int dev, int sms, cudaStream_t stream) {
+    static bool attr_done[kMaxDevices] = {false};
     static int resident[kMaxDevices] = {0};
     auto kernel = selective_scan_bwd_kernel<IoT, BcT, kHasZ>;
+    constexpr int smem = kBwdWarps * bwd_warp_smem<IoT, BcT>();
+    cudaError_t e = ensure_smem_attr(kernel, smem, attr_done, dev);
+    if (e != cudaSuccess) return e;
     int per_sm = (dev >= 0 && dev < kMaxDevices) ? resident[dev] : 0;
     if (per_sm <= 0) {
-        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kBwdWarps * 32, 0);
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kBwdWarps * 32, smem);
         if (e != cudaSuccess) return e;
         if (per_sm <= 0) return cudaErrorInvalidConfiguration;
         if (dev >= 0 && dev < kMaxDevices) resident[dev] = per_sm;
     }
+    // At most one segment per group can run at a time (the chain of segments).
     const int64_t want = (std::min<int64_t>(prm.items, prm.groups) + kBwdWarps - 1) / kBwdWarps;
     const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)per_sm * sms));
-    kernel<<<(unsigned)grid, kBwdWarps * 32, 0, stream>>>(prm);
+    kernel<<<(unsigned)grid, kBwdWarps * 32, smem, stream>>>(prm);
     return cudaGetLastError();
 }
 

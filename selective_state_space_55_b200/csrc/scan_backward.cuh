@@ -132,6 +132,63 @@ __device__ __forceinline__ float warp_reduce8(float (&v)[8], int lane) {
     return r;                                    // total of value (lane >> 2)
 }
 
+// 16-byte asynchronous copy global -> shared (L2 only), and its groups.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)),
+                 "l"(reinterpret_cast<uint64_t>(gmem_src))
+                 : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// One lane's inputs of one 8-step block, staged by cp.async: its rows of u,
+// delta, z and dout, its row of B (lanes 0..15) or C (16..31), and the
+// checkpointed state.  Each lane reads back only what it copied.
+template <typename IoT, typename BcT>
+struct BwdStage {
+    static constexpr int kIoRow = kBwdSteps * (int)sizeof(IoT);    // 16 or 32 bytes
+    static constexpr int kBcRow = kBwdSteps * (int)sizeof(BcT);
+    uint4 io[4][32][kIoRow / 16];
+    uint4 bc[32][kBcRow / 16];
+    uint4 ck[32][4];
+};
+
+template <typename IoT, typename BcT>
+__host__ __device__ constexpr int bwd_warp_smem() {
+    return 2 * (int)sizeof(BwdStage<IoT, BcT>) + kBwdSteps * 32 * (int)sizeof(float);
+}
+
+template <int kVecs>
+__device__ __forceinline__ void unpack_rows(const uint4 (&r)[kVecs], float (&v)[kBwdSteps]) {
+    if constexpr (kVecs == 1) {
+        unpack16(r[0], v);
+    } else {
+        float a[4], b[4];
+        unpack16(r[0], a);
+        unpack16(r[1], b);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) { v[i] = a[i]; v[4 + i] = b[i]; }
+    }
+}
+
+// Move entries 4..15 down by four and 0..3 to the top (four calls restore the order).
+__device__ __forceinline__ void rotate_quarter(float (&v)[kNPad]) {
+    const float t0 = v[0], t1 = v[1], t2 = v[2], t3 = v[3];
+#pragma unroll
+    for (int i = 0; i < kNPad - 4; ++i) v[i] = v[i + 4];
+    v[kNPad - 4] = t0;
+    v[kNPad - 3] = t1;
+    v[kNPad - 2] = t2;
+    v[kNPad - 1] = t3;
+}
+
 __device__ __forceinline__ float sigmoid_f32(float x) {
     return __fdividef(1.0f, 1.0f + ex2_approx(-x * kLog2e));
 }
@@ -145,13 +202,17 @@ __device__ __forceinline__ float bwd_exp2(float x) {
 }
 
 template <typename IoT, typename BcT, bool kHasZ>
-__global__ void __launch_bounds__(kBwdWarps * 32, 3)
+__global__ void __launch_bounds__(kBwdWarps * 32)
     selective_scan_bwd_kernel(const __grid_constant__ BwdParams p) {
     constexpr bool kExact = sizeof(IoT) == 4;
-    __shared__ __align__(16) float bcf_all[kBwdWarps][kBwdSteps][32];
+    using Stage = BwdStage<IoT, BcT>;
+    constexpr int kIoVecs = Stage::kIoRow / 16, kBcVecs = Stage::kBcRow / 16;
+    extern __shared__ __align__(16) uint8_t bwd_smem[];
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    float (*bcf)[32] = bcf_all[warp];
+    uint8_t* wbase = bwd_smem + warp * bwd_warp_smem<IoT, BcT>();
+    Stage* stages = reinterpret_cast<Stage*>(wbase);
+    float (*bcf)[32] = reinterpret_cast<float (*)[32]>(wbase + 2 * sizeof(Stage));
 
     for (;;) {
         unsigned int item = 0;
@@ -219,31 +280,88 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 3)
         const IoT* grow = static_cast<const IoT*>(p.dout) + chain * p.seqlen;
         const bool vec = p.vec_ok && (p.seqlen * (int64_t)sizeof(IoT)) % 16 == 0 && valid;
         const int nblk = (int)((t_end - t_begin + kBwdSteps - 1) / kBwdSteps);
+        const int nbc = lane & 15;
+        const BcT* bcrow = static_cast<const BcT*>(lane < 16 ? p.B : p.C) +
+                           (b * p.dstate + (nbc < p.dstate ? nbc : 0)) * p.seqlen;
+        // Blocks are staged one ahead by cp.async when every row is 16-byte
+        // aligned; a block shorter than 8 steps (the sequence's last) is read
+        // directly.
+        const bool pipe = p.vec_ok && p.bc_vec && (p.seqlen * (int64_t)sizeof(IoT)) % 16 == 0;
+        auto issue = [&](int jj) {
+            const int64_t tt = t_begin + (int64_t)jj * kBwdSteps;
+            if (pipe && t_end - tt >= kBwdSteps) {
+                Stage& S = stages[jj & 1];
+                if (valid) {
+#pragma unroll
+                    for (int v = 0; v < kIoVecs; ++v) {
+                        cp_async16(&S.io[0][lane][v], urow + tt + v * (16 / (int)sizeof(IoT)));
+                        cp_async16(&S.io[1][lane][v], drow + tt + v * (16 / (int)sizeof(IoT)));
+                        if (kHasZ) cp_async16(&S.io[2][lane][v], zrow + tt + v * (16 / (int)sizeof(IoT)));
+                        cp_async16(&S.io[3][lane][v], grow + tt + v * (16 / (int)sizeof(IoT)));
+                    }
+                    const float* ckq = p.ckpt + (chain * p.ckpt_tiles + tt / kBwdSteps) * kNPad;
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) cp_async16(&S.ck[lane][v], ckq + 4 * v);
+                }
+                if (nbc < p.dstate) {
+#pragma unroll
+                    for (int v = 0; v < kBcVecs; ++v)
+                        cp_async16(&S.bc[lane][v], bcrow + tt + v * (16 / (int)sizeof(BcT)));
+                }
+            }
+            cp_async_commit();                   // possibly empty: one group per block
+        };
+        issue(nblk - 1);
 
         for (int j = nblk - 1; j >= 0; --j) {
             const int64_t t0 = t_begin + (int64_t)j * kBwdSteps;
             const int ns = (int)min((int64_t)kBwdSteps, t_end - t0);
+            if (j > 0) {
+                issue(j - 1);
+                cp_async_wait<1>();
+            } else {
+                cp_async_wait<0>();
+            }
+            const bool staged = pipe && ns == kBwdSteps;
+            const Stage& S = stages[j & 1];
             // ---- inputs of this block: the lane's own channel, and the B/C table
             float uu[kBwdSteps], dt[kBwdSteps], dy[kBwdSteps], aux[kBwdSteps];
-            if (valid) {
+            float4 ckv[4];
+            if (valid && staged) {
+                unpack_rows<kIoVecs>(S.io[0][lane], uu);
+                unpack_rows<kIoVecs>(S.io[1][lane], dt);   // delta, turned into Delta below
+                unpack_rows<kIoVecs>(S.io[3][lane], dy);   // dout, turned into dy below
+                if (kHasZ) unpack_rows<kIoVecs>(S.io[2][lane], aux);
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    const uint4 r = S.ck[lane][v];
+                    ckv[v] = make_float4(__uint_as_float(r.x), __uint_as_float(r.y),
+                                         __uint_as_float(r.z), __uint_as_float(r.w));
+                }
+            } else if (valid) {
                 load_block(urow, t0, ns, vec, uu);
-                load_block(drow, t0, ns, vec, dt);       // delta, turned into Delta below
-                load_block(grow, t0, ns, vec, dy);       // dout, turned into dy below
+                load_block(drow, t0, ns, vec, dt);
+                load_block(grow, t0, ns, vec, dy);
                 if (kHasZ) load_block(zrow, t0, ns, vec, aux);
+                const float4* ck4 = reinterpret_cast<const float4*>(
+                    p.ckpt + (chain * p.ckpt_tiles + t0 / kBwdSteps) * kNPad);
+#pragma unroll
+                for (int v = 0; v < 4; ++v) ckv[v] = __ldcg(ck4 + v);
             } else {
 #pragma unroll
                 for (int i = 0; i < kBwdSteps; ++i) uu[i] = dt[i] = dy[i] = aux[i] = 0.0f;
+#pragma unroll
+                for (int v = 0; v < 4; ++v) ckv[v] = make_float4(0.f, 0.f, 0.f, 0.f);
             }
             {
-                const int n = lane & 15;
-                const BcT* src = static_cast<const BcT*>(lane < 16 ? p.B : p.C) +
-                                 (b * p.dstate + (n < p.dstate ? n : 0)) * p.seqlen;
                 float row[kBwdSteps];
-                if (n < p.dstate) {
-                    load_block(src, t0, ns, p.bc_vec != 0, row);
-                } else {
+                if (nbc >= p.dstate) {
 #pragma unroll
                     for (int i = 0; i < kBwdSteps; ++i) row[i] = 0.0f;
+                } else if (staged) {
+                    unpack_rows<kBcVecs>(S.bc[lane], row);
+                } else {
+                    load_block(bcrow, t0, ns, p.bc_vec != 0, row);
                 }
                 __syncwarp();
 #pragma unroll
@@ -268,16 +386,16 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 3)
             float y[kBwdSteps], ddt[kBwdSteps], dlb[kBwdSteps];
 #pragma unroll
             for (int i = 0; i < kBwdSteps; ++i) y[i] = ddt[i] = dlb[i] = 0.0f;
-            const float* ck = p.ckpt + (chain * p.ckpt_tiles + t0 / kBwdSteps) * kNPad;
 
-#pragma unroll
+            // One state quarter per pass; the per-entry arrays (a2, lam, dA_acc)
+            // and the checkpoint rotate by one quarter after each pass, so the
+            // loop body indexes them statically and is emitted once.
+#pragma unroll 1
             for (int q = 0; q < kNPad / 4; ++q) {
                 const int n0 = 4 * q;
                 // forward: the block's 8 states of entries n0..n0+3
-                const float4 hs4 = valid ? __ldcg(reinterpret_cast<const float4*>(ck + n0))
-                                         : make_float4(0.f, 0.f, 0.f, 0.f);
                 float hq[kBwdSteps][4];
-                float h[4] = {hs4.x, hs4.y, hs4.z, hs4.w};
+                float h[4] = {ckv[0].x, ckv[0].y, ckv[0].z, ckv[0].w};
 #pragma unroll
                 for (int t = 0; t < kBwdSteps; ++t) {
                     if (t < ns) {
@@ -288,7 +406,7 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 3)
                         const float du = dt[t] * uu[t];
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
-                            const float ab = bwd_exp2<kExact>(dt[t] * a2[n0 + i]);
+                            const float ab = bwd_exp2<kExact>(dt[t] * a2[i]);
                             h[i] = fmaf(ab, h[i], du * bq[i]);
                             hq[t][i] = h[i];
                             y[t] = fmaf(cq[i], h[i], y[t]);
@@ -296,7 +414,7 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 3)
                     }
                 }
                 // reverse: the adjoint of entries n0..n0+3 over the block
-                float l4[4] = {lam[n0], lam[n0 + 1], lam[n0 + 2], lam[n0 + 3]};
+                float l4[4] = {lam[0], lam[1], lam[2], lam[3]};
 #pragma unroll
                 for (int t = kBwdSteps - 1; t >= 0; --t) {
                     if (t < ns) {
@@ -310,13 +428,13 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 3)
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
                             l4[i] = fmaf(cq[i], dy[t], l4[i]);                 // lambda_t
-                            const float ab = bwd_exp2<kExact>(dt[t] * a2[n0 + i]);
+                            const float ab = bwd_exp2<kExact>(dt[t] * a2[i]);
                             const float abh = fmaf(-du, bq[i], hq[t][i]);      // Abar_t h_t-1 = h_t - b_t
                             red[i] = l4[i] * du;                                // dB
                             red[4 + i] = dy[t] * hq[t][i];                      // dC
-                            s_dt = fmaf(l4[i], fmaf(a2[n0 + i] * kLn2, abh, bq[i] * uu[t]), s_dt);
+                            s_dt = fmaf(l4[i], fmaf(a2[i] * kLn2, abh, bq[i] * uu[t]), s_dt);
                             s_b = fmaf(l4[i], bq[i], s_b);
-                            dA_acc[n0 + i] = fmaf(l4[i] * dt[t], abh, dA_acc[n0 + i]);
+                            dA_acc[i] = fmaf(l4[i] * dt[t], abh, dA_acc[i]);
                             l4[i] *= ab;                                        // to h_t-1
                         }
                         ddt[t] += s_dt;
@@ -331,7 +449,15 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 3)
                     }
                 }
 #pragma unroll
-                for (int i = 0; i < 4; ++i) lam[n0 + i] = l4[i];
+                for (int i = 0; i < 4; ++i) lam[i] = l4[i];
+                rotate_quarter(a2);
+                rotate_quarter(lam);
+                rotate_quarter(dA_acc);
+                const float4 c0 = ckv[0];
+                ckv[0] = ckv[1];
+                ckv[1] = ckv[2];
+                ckv[2] = ckv[3];
+                ckv[3] = c0;
             }
             // per-step outputs of the block
             float o_du[kBwdSteps], o_dd[kBwdSteps], o_dz[kBwdSteps];
@@ -347,6 +473,7 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 3)
                 }
                 o_dz[t] = kHasZ ? aux[t] * fmaf(Dd, uu[t], y[t]) : 0.0f;
             }
+            __syncwarp();
             if (valid) {
                 store_block(static_cast<IoT*>(p.du) + chain * p.seqlen, t0, ns, vec, o_du);
                 store_block(static_cast<IoT*>(p.ddelta) + chain * p.seqlen, t0, ns, vec, o_dd);
