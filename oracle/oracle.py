@@ -21,6 +21,12 @@ The backward pass of the (Euler) scan is the adjoint recurrence in reverse
 time; ``selective_scan_bwd`` returns the gradients of a linear functional of
 out and last_state.
 
+``ssd_scan`` is the Mamba-2 layer ("Mamba 与状态空间模型", section
+"Mamba-2：两种算法"): A is a scalar per head, the state of a head is a
+(headdim x dstate) matrix, B and C are shared by the heads of a group, and the
+recurrence S_t = exp(Delta_t A_h) S_{t-1} + Delta_t x_t B_t^T, y_t = S_t C_t
++ D_h x_t is run one step at a time.
+
 The block's short causal convolution (depthwise, W taps, optional silu) and
 its single-token update are the plain weighted sums over the window ("Mamba 与
 状态空间模型", section 固定大小的状态: a short convolution keeps the 4 most
@@ -104,6 +110,9 @@ class Oracle:
         self._lib.oracle_causal_conv1d_update_f64.restype = ctypes.c_int
         self._lib.oracle_causal_conv1d_update_f64.argtypes = [
             i64, i64, i64, dp, dp, dp, dp, ci, dp, dp]
+        self._lib.oracle_ssd_scan_f64.restype = ctypes.c_int
+        self._lib.oracle_ssd_scan_f64.argtypes = [
+            i64, i64, i64, i64, i64, i64, dp, dp, dp, dp, dp, dp, dp, dp, ci, dp, dp, dp]
         self._lib.oracle_num_threads.restype = ctypes.c_int
         self._lib.oracle_num_threads.argtypes = []
 
@@ -231,6 +240,33 @@ class Oracle:
         if rc != 0:
             raise ValueError(f"oracle_causal_conv1d_update_f64 returned {rc}")
         return new, out
+
+    def ssd_scan(self, x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_softplus=True,
+                 initial_state=None):
+        """Mamba-2 layer with a scalar A per head, as the plain recurrence.
+
+        x, z: (batch, L, nheads, headdim); dt: (batch, L, nheads); A, D, dt_bias:
+        (nheads,); B, C: (batch, L, ngroups, dstate); initial_state: (batch,
+        nheads, headdim, dstate).  Returns (out, final_state) as float64 arrays,
+        out shaped like x and final_state (batch, nheads, headdim, dstate).
+        """
+        x, dt, A, B, C = map(_f64, (x, dt, A, B, C))
+        D, z, dt_bias, init = map(_f64, (D, z, dt_bias, initial_state))
+        batch, seqlen, nheads, headdim = x.shape
+        ngroups, dstate = B.shape[2], B.shape[3]
+        assert dt.shape == (batch, seqlen, nheads) and A.shape == (nheads,)
+        assert B.shape == (batch, seqlen, ngroups, dstate) and C.shape == B.shape
+        assert z is None or z.shape == x.shape
+        assert init is None or init.shape == (batch, nheads, headdim, dstate)
+        out = np.empty_like(x)
+        final = np.empty((batch, nheads, headdim, dstate), dtype=np.float64)
+        rc = self._lib.oracle_ssd_scan_f64(batch, seqlen, nheads, headdim, ngroups, dstate,
+                                           _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                           _ptr(z), _ptr(dt_bias), int(bool(dt_softplus)),
+                                           _ptr(init), _ptr(out), _ptr(final))
+        if rc != 0:
+            raise ValueError(f"oracle_ssd_scan_f64 returned {rc}")
+        return out, final
 
 
 _DEFAULT: Oracle | None = None

@@ -1,6 +1,6 @@
 /*
- * Float64 CPU oracle for the Mamba selective-SSM scan and the single-token
- * state update.
+ * Float64 CPU oracle for the Mamba selective-SSM scan, the single-token
+ * state update, the short convolution, the backward pass and the Mamba-2 layer.
  *
  * TEST INFRASTRUCTURE ONLY.  Nothing on the product path links, loads or calls
  * this file: only the tests, the package's smoke check and the benchmark's
@@ -58,6 +58,11 @@
  *   du_t = D dy_t + sum_n lambda_t,n Delta_t B_t,n,   dh_-1 = Abar_0 lambda_0,
  * with dy = dout silu(z) and dz = dout y silu'(z) when gated, and the softplus
  * derivative sigmoid(delta + bias) applied to dDelta.
+ *
+ * The Mamba-2 layer (scalar A per head, a (headdim x dstate) state per head,
+ * B and C shared by a group of heads) is the last function, as its plain
+ * recurrence; the tests pin it to the lower-triangular matrix the same layer
+ * applies ("Mamba 与状态空间模型", section "Mamba-2：两种算法").
  *
  * Loops: chains (b, d) are independent; OpenMP splits them across threads
  * (the backward runs them in order, since its gradients of A, B, C, D and the
@@ -418,4 +423,86 @@ int oracle_selective_scan_bwd_f64(int64_t batch, int64_t dim, int64_t dstate, in
     free(dts);
     free(ys);
     return 0;
+}
+
+/*
+ * Mamba-2 state-space layer with a scalar A per head ("Mamba 与状态空间模型",
+ * section "Mamba-2：两种算法": A is one number times the identity, and the layer
+ * is one lower-triangular matrix applied to the whole input).  This is the
+ * recurrence form of that matrix, step by step in float64.  For every
+ * (b, head h) the state S is a (headdim x dstate) matrix:
+ *
+ *   Delta_t  = softplus(dt_t,h + dt_bias_h)          (or dt + bias, softplus off)
+ *   S_t      = exp(Delta_t A_h) S_{t-1} + Delta_t x_t,h B_t,g^T   (S_{-1} = S0 or 0)
+ *   y_t,h,p  = sum_n C_t,g,n S_t[p][n] + D_h x_t,h,p
+ *   out      = y * silu(z)                            (when z is given)
+ *
+ * where the head's group is g = h / (nheads / ngroups): B and C are shared by
+ * the heads of one group.  The input term is Delta_t x_t B_t (Euler), the same
+ * discretisation as the diagonal scan above.
+ *
+ * Layouts (row-major, contiguous): x, z, out (batch, seqlen, nheads, headdim);
+ * dt (batch, seqlen, nheads); A, D, dt_bias (nheads); B, C (batch, seqlen,
+ * ngroups, dstate); initial_state, final_state (batch, nheads, headdim,
+ * dstate).  D, z, dt_bias, initial_state and final_state may be NULL.
+ * Returns 0, or -1 on a bad size (ngroups must divide nheads).
+ */
+int oracle_ssd_scan_f64(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,
+                        int64_t ngroups, int64_t dstate, const double *x, const double *dt,
+                        const double *A, const double *B, const double *C, const double *D,
+                        const double *z, const double *dt_bias, int dt_softplus,
+                        const double *initial_state, double *out, double *final_state)
+{
+    if (batch < 0 || seqlen < 0 || nheads < 1 || headdim < 1 || dstate < 1 || ngroups < 1 ||
+        nheads % ngroups != 0)
+        return -1;
+    int64_t heads_per_group = nheads / ngroups;
+    int64_t chains = batch * nheads;
+    int failed = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t chain = 0; chain < chains; ++chain) {
+        int64_t b = chain / nheads;
+        int64_t h = chain % nheads;
+        int64_t g = h / heads_per_group;
+        double *S = (double *)malloc(sizeof(double) * headdim * dstate);
+        if (!S) {
+#pragma omp atomic write
+            failed = 1;
+            continue;
+        }
+        for (int64_t i = 0; i < headdim * dstate; ++i)
+            S[i] = initial_state ? initial_state[chain * headdim * dstate + i] : 0.0;
+
+        for (int64_t t = 0; t < seqlen; ++t) {
+            double delta = dt[(b * seqlen + t) * nheads + h];
+            if (dt_bias)
+                delta += dt_bias[h];
+            if (dt_softplus)
+                delta = oracle_softplus(delta);
+            double decay = exp(delta * A[h]);
+            const double *x_t = x + ((b * seqlen + t) * nheads + h) * headdim;
+            const double *B_t = B + ((b * seqlen + t) * ngroups + g) * dstate;
+            const double *C_t = C + ((b * seqlen + t) * ngroups + g) * dstate;
+            double *out_t = out + ((b * seqlen + t) * nheads + h) * headdim;
+            const double *z_t = z ? z + ((b * seqlen + t) * nheads + h) * headdim : NULL;
+            for (int64_t p = 0; p < headdim; ++p) {
+                double *S_p = S + p * dstate;
+                double y = 0.0;
+                for (int64_t n = 0; n < dstate; ++n) {
+                    S_p[n] = decay * S_p[n] + delta * x_t[p] * B_t[n];
+                    y += C_t[n] * S_p[n];
+                }
+                if (D)
+                    y += D[h] * x_t[p];
+                if (z_t)
+                    y *= oracle_silu(z_t[p]);
+                out_t[p] = y;
+            }
+        }
+        if (final_state)
+            for (int64_t i = 0; i < headdim * dstate; ++i)
+                final_state[chain * headdim * dstate + i] = S[i];
+        free(S);
+    }
+    return failed ? -1 : 0;
 }

@@ -19,6 +19,9 @@ Sources (page title, section):
     input matrix Bbar = (Delta A)^-1 (exp(Delta A) - I) Delta B.  Under it the
     Theorem-1 gate holds with B = 1 and no rescaling, and a constant input has
     the fixed point h* = -B u / A for every Delta.
+  - "Mamba 与状态空间模型", Mamba-2：两种算法: with A a scalar per head the layer
+    is a lower-triangular matrix (C at step i, B at step j, the decay between);
+    a sequence can be cut into pieces that pass only the state on.
 """
 from __future__ import annotations
 
@@ -620,6 +623,114 @@ def pin_bwd_finite_differences_plain(o):
     _fd_check(o, p, dout, dlast, False, "plain backward")
 
 
+# --- Mamba-2 layer (scalar A per head) ------------------------------------------------------
+# "Mamba 与状态空间模型", section "Mamba-2：两种算法": with A a scalar times the identity,
+# the layer is one lower-triangular matrix: entry (i, j) is C at step i dotted with B at
+# step j, times all the decay between the two steps.  The pins below build that matrix
+# (and the chunked / tied-diagonal readings of it) without stepping the recurrence.
+
+
+def _ssd_problem(seed, batch=2, seqlen=23, nheads=4, headdim=3, ngroups=2, dstate=5,
+                 with_state=True):
+    rng = np.random.default_rng(seed)
+    return dict(
+        x=rng.standard_normal((batch, seqlen, nheads, headdim)),
+        dt=rng.standard_normal((batch, seqlen, nheads)) * 0.5,
+        A=-rng.uniform(0.3, 2.0, nheads),
+        B=rng.standard_normal((batch, seqlen, ngroups, dstate)),
+        C=rng.standard_normal((batch, seqlen, ngroups, dstate)),
+        D=rng.standard_normal(nheads),
+        z=rng.standard_normal((batch, seqlen, nheads, headdim)),
+        dt_bias=rng.uniform(-1.0, 0.5, nheads),
+        initial_state=(rng.standard_normal((batch, nheads, headdim, dstate))
+                       if with_state else None),
+    )
+
+
+def _softplus(v):
+    return np.log1p(np.exp(v))
+
+
+def pin_ssd_lower_triangular_matrix(o):
+    """out = (M x + start-state term + D x) * silu(z), M_ij = C_i.B_j exp(sum_{j<r<=i} Delta_r A) Delta_j."""
+    p = _ssd_problem(41)
+    out, final = o.ssd_scan(**p)
+    batch, L, H, P = p["x"].shape
+    G, N = p["B"].shape[2], p["B"].shape[3]
+    delta = _softplus(p["dt"] + p["dt_bias"])             # (batch, L, H)
+    for b in range(batch):
+        for h in range(H):
+            g = h // (H // G)
+            a = delta[b, :, h] * p["A"][h]                    # log-decay of each step
+            Bm, Cm = p["B"][b, :, g, :], p["C"][b, :, g, :]   # (L, N)
+            M = np.zeros((L, L))
+            for i in range(L):
+                for j in range(i + 1):
+                    M[i, j] = Cm[i] @ Bm[j] * math.exp(a[j + 1:i + 1].sum()) * delta[b, j, h]
+            S0 = p["initial_state"][b, h]                     # (P, N)
+            carry = np.array([math.exp(a[:i + 1].sum()) for i in range(L)])
+            xs = p["x"][b, :, h, :]                           # (L, P)
+            y = M @ xs + carry[:, None] * (Cm @ S0.T) + p["D"][h] * xs
+            y = y * _silu(p["z"][b, :, h, :])
+            _close(out[b, :, h, :], y, 1e-12, "SSD output vs the lower-triangular matrix")
+            w = np.array([math.exp(a[j + 1:].sum()) * delta[b, j, h] for j in range(L)])
+            S = math.exp(a.sum()) * S0 + (w[:, None] * xs).T @ Bm
+            _close(final[b, h], S, 1e-12, "SSD final state vs the sum over steps")
+
+
+def pin_ssd_is_tied_diagonal_scan(o):
+    """One group: every (head, p) channel is a diagonal scan whose A row is A_h repeated."""
+    p = _ssd_problem(42, ngroups=1, with_state=True)
+    out, final = o.ssd_scan(**p)
+    batch, L, H, P = p["x"].shape
+    N = p["B"].shape[3]
+    u = p["x"].transpose(0, 2, 3, 1).reshape(batch, H * P, L)
+    z = p["z"].transpose(0, 2, 3, 1).reshape(batch, H * P, L)
+    delta = np.repeat(p["dt"].transpose(0, 2, 1), P, axis=1)   # (batch, H*P, L)
+    A = np.repeat(p["A"], P)[:, None] * np.ones((1, N))
+    Bs = p["B"][:, :, 0, :].transpose(0, 2, 1)                # (batch, N, L)
+    Cs = p["C"][:, :, 0, :].transpose(0, 2, 1)
+    h0 = p["initial_state"].reshape(batch, H * P, N)
+    ref_out, ref_last = o.selective_scan(u, delta, A, Bs, Cs, D=np.repeat(p["D"], P), z=z,
+                                         delta_bias=np.repeat(p["dt_bias"], P),
+                                         initial_state=h0)
+    _close(out.transpose(0, 2, 3, 1).reshape(batch, H * P, L), ref_out, 1e-12,
+           "SSD output vs the diagonal scan")
+    _close(final.reshape(batch, H * P, N), ref_last, 1e-12, "SSD final state vs the diagonal scan")
+
+
+def pin_ssd_split_equals_whole(o):
+    """Scanning [0, k) then [k, L) from the first part's final state equals one scan."""
+    p = _ssd_problem(43)
+    out, final = o.ssd_scan(**p)
+    k = 9
+    first = {n: (v[:, :k] if n in ("x", "dt", "B", "C", "z") else v) for n, v in p.items()}
+    second = {n: (v[:, k:] if n in ("x", "dt", "B", "C", "z") else v) for n, v in p.items()}
+    out1, mid = o.ssd_scan(**first)
+    second["initial_state"] = mid
+    out2, final2 = o.ssd_scan(**second)
+    _close(np.concatenate([out1, out2], axis=1), out, 1e-12, "SSD split output")
+    _close(final2, final, 1e-12, "SSD split final state")
+
+
+def pin_ssd_zero_A_is_cumulative_sum(o):
+    """A = 0, softplus off, no gate, no D: S_t = S0 + sum_{j<=t} dt_j x_j B_j^T and y_t = S_t C_t."""
+    p = _ssd_problem(44)
+    p.update(A=np.zeros_like(p["A"]), dt=np.abs(p["dt"]), D=None, z=None, dt_bias=None)
+    out, final = o.ssd_scan(**p, dt_softplus=False)
+    batch, L, H, P = p["x"].shape
+    G = p["B"].shape[2]
+    for b in range(batch):
+        for h in range(H):
+            g = h // (H // G)
+            terms = p["dt"][b, :, h, None, None] * np.einsum(
+                "tp,tn->tpn", p["x"][b, :, h, :], p["B"][b, :, g, :])
+            S = p["initial_state"][b, h][None] + np.cumsum(terms, axis=0)   # (L, P, N)
+            y = np.einsum("tpn,tn->tp", S, p["C"][b, :, g, :])
+            _close(out[b, :, h, :], y, 1e-12, "SSD with A = 0 vs the cumulative sum")
+            _close(final[b, h], S[-1], 1e-12, "SSD with A = 0, final state")
+
+
 PINS = {
     "unrolled_sum": pin_unrolled_sum,
     "gate_closed_values": pin_gate_closed_values,
@@ -646,4 +757,8 @@ PINS = {
     "conv_updates_equal_prefill": pin_conv_updates_equal_prefill,
     "bwd_finite_differences_gated": pin_bwd_finite_differences_gated,
     "bwd_finite_differences_plain": pin_bwd_finite_differences_plain,
+    "ssd_lower_triangular_matrix": pin_ssd_lower_triangular_matrix,
+    "ssd_is_tied_diagonal_scan": pin_ssd_is_tied_diagonal_scan,
+    "ssd_split_equals_whole": pin_ssd_split_equals_whole,
+    "ssd_zero_A_is_cumulative_sum": pin_ssd_zero_A_is_cumulative_sum,
 }

@@ -99,6 +99,27 @@ MUTANTS = [
     ("bwd_dD_uses_dout", "dD[d] += dy * x;", "dD[d] += g * x;"),
     ("bwd_dh0_one_step_late", "dinitial_state[chain * dstate + n] = lam[n];",
      "dinitial_state[chain * dstate + n] = lam[n] * exp(dts[0] * A[d * dstate + n]);"),
+    # Mamba-2 layer (scalar A per head)
+    ("ssd_group_interleaved", "int64_t g = h / heads_per_group;", "int64_t g = h % ngroups;"),
+    ("ssd_decay_sign_flipped", "double decay = exp(delta * A[h]);",
+     "double decay = exp(-delta * A[h]);"),
+    ("ssd_input_without_delta", "S_p[n] = decay * S_p[n] + delta * x_t[p] * B_t[n];",
+     "S_p[n] = decay * S_p[n] + x_t[p] * B_t[n];"),
+    ("ssd_readout_before_update",
+     "S_p[n] = decay * S_p[n] + delta * x_t[p] * B_t[n];\n                    y += C_t[n] * S_p[n];",
+     "y += C_t[n] * S_p[n];\n                    S_p[n] = decay * S_p[n] + delta * x_t[p] * B_t[n];"),
+    ("ssd_C_read_from_B", "y += C_t[n] * S_p[n];", "y += B_t[n] * S_p[n];"),
+    ("ssd_D_dropped", "y += D[h] * x_t[p];", "y += 0.0 * x_t[p];"),
+    ("ssd_gate_dropped", "y *= oracle_silu(z_t[p]);", "y *= 1.0;"),
+    ("ssd_bias_dropped", "delta += dt_bias[h];", "delta += 0.0;"),
+    ("ssd_softplus_skipped", "if (dt_softplus)\n                delta = oracle_softplus(delta);", ""),
+    ("ssd_initial_state_ignored",
+     "S[i] = initial_state ? initial_state[chain * headdim * dstate + i] : 0.0;", "S[i] = 0.0;"),
+    ("ssd_final_state_stale", "final_state[chain * headdim * dstate + i] = S[i];",
+     "final_state[chain * headdim * dstate + i] = initial_state ? initial_state[chain * headdim * dstate + i] : 0.0;"),
+    ("ssd_headdim_reversed", "y += D[h] * x_t[p];", "y += D[h] * x_t[headdim - 1 - p];"),
+    ("ssd_dt_time_shifted", "double delta = dt[(b * seqlen + t) * nheads + h];",
+     "double delta = dt[(b * seqlen + (t > 0 ? t - 1 : 0)) * nheads + h];"),
 ]
 
 
