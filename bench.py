@@ -47,6 +47,7 @@ SCAN_VARIANTS = ("euler", "zoh", "start_state")
 PROFILES = ROOT / "profiles"
 HBM_FALLBACK_GBS = 6650.0
 SM_MAX_MHZ_FALLBACK = 1965.0
+BF16_TFLOPS_FALLBACK = 1590.0
 
 
 # ----------------------------------------------------------------- helpers
@@ -61,10 +62,12 @@ def measured_peaks() -> dict:
         try:
             d = json.loads(p.read_text())
             return {"hbm_gbs": float(d["hbm_gbs"]), "sm_max_mhz": float(d.get("sm_max_mhz", SM_MAX_MHZ_FALLBACK)),
+                    "bf16_tflops": float(d.get("bf16_tflops", BF16_TFLOPS_FALLBACK)),
                     "source": "measured"}
         except Exception:  # noqa: BLE001
             pass
-    return {"hbm_gbs": HBM_FALLBACK_GBS, "sm_max_mhz": SM_MAX_MHZ_FALLBACK, "source": "fallback"}
+    return {"hbm_gbs": HBM_FALLBACK_GBS, "sm_max_mhz": SM_MAX_MHZ_FALLBACK,
+            "bf16_tflops": BF16_TFLOPS_FALLBACK, "source": "fallback"}
 
 
 def sources_digest() -> str:
@@ -675,6 +678,80 @@ def bench_bwd(args, rank, world, local):
         print(json.dumps(line), flush=True)
 
 
+def bench_ssd(args, rank, world, local):
+    """Measurement case: the Mamba-2 layer (scalar A per head) on the tensor
+    cores, Mamba-2 2.7B layer shape (batch 16, L 2048, 80 heads x 64, state
+    128, one group), gate, D and bias on, final state returned."""
+    global _WORLD
+    _WORLD = world
+    from selective_state_space_55_b200 import build as cuda_build
+    from selective_state_space_55_b200 import inputs as I
+    from selective_state_space_55_b200 import ops
+    from selective_state_space_55_b200 import roofline as R
+
+    if rank == 0:
+        cuda_build.build()
+    barrier()
+    torch.cuda.set_device(local)
+    c = I.SSD_CONFIGS["mamba2_2p7b_layer"]
+    if args.scan_batch:
+        c = c.resized(batch=args.scan_batch)
+    x = I.make_ssd_inputs(c, "cuda", seed=rank_seed(rank))
+    out = torch.empty_like(x["x"])
+    final = torch.empty(c.batch, c.nheads, c.headdim, c.dstate, dtype=torch.float32, device="cuda")
+
+    def step():
+        ops.ssd_chunk_scan_fwd(x["x"], x["dt"], x["A"], x["B"], x["C"], D=x["D"], z=x["z"],
+                               dt_bias=x["dt_bias"], out=out, final_state=final)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    K = args.steps
+    sampler = ClockSampler(local)
+    sampler.start()
+    barrier()
+    torch.cuda.synchronize()
+    t0 = time.time()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(K):
+        step()
+    e.record()
+    torch.cuda.synchronize()
+    t1 = time.time()
+    barrier()
+    sampler.stop()
+    ms = max_over_ranks(s.elapsed_time(e)) / K
+    peaks = measured_peaks()
+    nbytes = R.ssd_bytes(c.batch, c.seqlen, c.nheads, c.headdim, c.ngroups, c.dstate, c.has_z)
+    flops = R.ssd_chunk_flops(c.batch, c.seqlen, c.nheads, c.headdim, c.dstate)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    tfs = flops / (ms * 1e-3) / 1e12
+    value = world * c.elements / (ms * 1e-3) / 1e9
+    if rank == 0:
+        line = {
+            "metric": "Mamba-2 layer Gelem/s (B·L·heads·headdim)", "value": round(value, 3),
+            "unit": "Gelem/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded)",
+            "config": {"workload": f"{c.name} ({c.batch}x{c.seqlen}, {c.nheads} heads x {c.headdim}, "
+                                   f"N={c.dstate}, groups={c.ngroups}, chunk 128, bf16, gate/D/bias, "
+                                   "final state)",
+                       "inputs_exceed_l2": nbytes > 126e6},
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
+                         "traffic": None, "bytes_per_step": nbytes},
+            "tensor": {"issued_tflops": round(tfs, 1), "peak": peaks["bf16_tflops"],
+                       "frac": round(tfs / peaks["bf16_tflops"], 4), "flops_per_step": flops},
+            "gpu_launches": K,
+            "clocks": sampler.summary(t0, t1),
+            "partial_case": {"only": "ssd", "scan_batch": args.scan_batch,
+                             "note": "measurement of the Mamba-2 layer, not the benchmark workload"},
+        }
+        print(json.dumps(line), flush=True)
+
+
 def bench_reference(args, rank, world):
     """The float64 CPU oracle, on the same workload's metric, a bounded sample
     per step (rank 0 only)."""
@@ -736,8 +813,9 @@ def main():
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--reference-seconds", type=float, default=120.0,
                     help="budget of the whole --impl reference run")
-    ap.add_argument("--only", choices=["scan", "decode", "conv", "bwd"], default=None,
-                    help="profiling case: one half of the step; conv: the short convolution; bwd: the backward pass")
+    ap.add_argument("--only", choices=["scan", "decode", "conv", "bwd", "ssd"], default=None,
+                    help="profiling case: one half of the step; conv: the short convolution; "
+                         "bwd: the backward pass; ssd: the Mamba-2 layer")
     ap.add_argument("--scan-batch", type=int, default=None,
                     help="profiling case: smaller scan batch")
     ap.add_argument("--decode-layers", type=int, default=None,
@@ -772,6 +850,8 @@ def main():
             bench_conv(args, rank, world, local)
         elif args.only == "bwd":
             bench_bwd(args, rank, world, local)
+        elif args.only == "ssd":
+            bench_ssd(args, rank, world, local)
         else:
             bench_ours(args, rank, world, local)
     finally:

@@ -416,6 +416,58 @@ MAMBA_API mamba_status_t mamba_causal_conv1d_update(void *conv_state, const void
                                                     cudaStream_t stream);
 
 /*
+ * Mamba-2 layer: the selective state space with a scalar A per head
+ * ("Mamba 与状态空间模型", section "Mamba-2：两种算法": A is one number times
+ * the identity, the layer applies one lower-triangular matrix whose entry
+ * (i, j) is C_i . B_j times the decay between the steps, and a chunked
+ * algorithm does dense products inside chunks and passes only the state
+ * between them).  For each batch b and head h, with group g = h / (nheads /
+ * ngroups) and the state S a (headdim x dstate) matrix:
+ *
+ *   Delta_t = softplus(dt_t,h + dt_bias_h)     (dt + dt_bias if dt_softplus == 0)
+ *   S_t     = exp(Delta_t A_h) S_{t-1} + Delta_t x_t,h B_t,g^T,   S_{-1} = initial_state or 0
+ *   out_t,h = (S_t C_t,g + D_h x_t,h) * silu(z_t,h)            (no gate when z == NULL)
+ *
+ * Arguments (all device pointers, caller-owned, contiguous row-major):
+ *   x, z, out      (batch, seqlen, nheads, headdim) bf16; z may be NULL;
+ *                  out must not alias an input
+ *   dt             (batch, seqlen, nheads) bf16
+ *   A              (nheads,) fp32, expected <= 0
+ *   B, C           (batch, seqlen, ngroups, dstate) bf16
+ *   D, dt_bias     (nheads,) fp32 or NULL
+ *   initial_state  (batch, nheads, headdim, dstate) fp32 or NULL (zeros)
+ *   final_state    (batch, nheads, headdim, dstate) fp32 or NULL: S at the
+ *                  last step (initial_state, or zeros, when seqlen == 0)
+ * Delta must not be negative: with dt_softplus == 0 the caller guarantees
+ * dt + dt_bias >= 0 (a negative Delta gives undefined output).
+ *
+ * Supported shape: headdim == 64 and dstate == 128 (the published Mamba-2
+ * models' head and state sizes), io_dtype MAMBA_BF16, ngroups dividing
+ * nheads; anything else returns MAMBA_ERR_UNSUPPORTED (or
+ * MAMBA_ERR_INVALID_ARG for negative sizes, missing required pointers or
+ * ngroups not dividing nheads) before anything is launched.  x, z, out, B and
+ * C must be 16-byte aligned, the fp32 arrays 4-byte aligned and dt 2-byte
+ * aligned (MAMBA_ERR_ALIGN).  Products run on the tensor cores with bf16
+ * operands (the intra-chunk matrix and the state copy used for the output
+ * are rounded to bf16) and fp32 accumulation; the carried state stays fp32.
+ * Asynchronous on `stream`; allocates nothing; a device-side wait that gives
+ * up is reported by mamba_device_status() as MAMBA_ERR_TIMEOUT.
+ */
+typedef struct {
+    int64_t batch, seqlen, nheads, headdim, ngroups, dstate;
+    mamba_dtype_t io_dtype;   /* x, dt, z, out, B, C */
+    int32_t dt_softplus;      /* nonzero: Delta = softplus(dt + dt_bias) */
+} mamba_ssd_dims_t;
+
+MAMBA_API mamba_status_t mamba_ssd_chunk_scan_fwd(const void *x, const void *dt, const float *A,
+                                                  const void *B, const void *C, const float *D,
+                                                  const void *z, const float *dt_bias,
+                                                  const float *initial_state, void *out,
+                                                  float *final_state,
+                                                  const mamba_ssd_dims_t *dims,
+                                                  cudaStream_t stream);
+
+/*
  * Read and clear the library's device-side status word on the current device
  * (synchronises the device).  Returns MAMBA_OK, or the first device-side
  * error recorded since the last call (e.g. MAMBA_ERR_TIMEOUT).

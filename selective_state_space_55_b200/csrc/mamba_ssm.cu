@@ -12,6 +12,7 @@
 #include "state_update.cuh"
 #include "conv1d.cuh"
 #include "scan_backward.cuh"
+#include "ssd_chunk_scan.cuh"
 
 namespace mamba {
 
@@ -1111,6 +1112,79 @@ cudaError_t zero_async(void* p, size_t bytes, cudaStream_t stream) {
 }
 
 }  // namespace
+
+namespace {
+
+// Argument checks of the Mamba-2 layer; MAMBA_OK when a launch may follow.
+mamba_status_t check_ssd(const void* x, const void* dt, const float* A, const void* B,
+                         const void* C, const float* D, const void* z, const float* dt_bias,
+                         const float* initial_state, const void* out, const float* final_state,
+                         const mamba_ssd_dims_t* d) {
+    if (d == nullptr) return MAMBA_ERR_INVALID_ARG;
+    if (d->batch < 0 || d->seqlen < 0 || d->nheads < 1 || d->ngroups < 1 || d->headdim < 1 ||
+        d->dstate < 1)
+        return MAMBA_ERR_INVALID_ARG;
+    if (d->nheads % d->ngroups != 0) return MAMBA_ERR_INVALID_ARG;
+    if (d->headdim != kSsdP || d->dstate != kSsdN || d->io_dtype != MAMBA_BF16)
+        return MAMBA_ERR_UNSUPPORTED;
+    const int64_t lim = (int64_t)1 << 31;
+    if (d->batch * d->nheads >= lim || d->seqlen >= lim) return MAMBA_ERR_INVALID_ARG;
+    if (A == nullptr) return MAMBA_ERR_INVALID_ARG;
+    if (d->batch > 0 && d->seqlen > 0 &&
+        (x == nullptr || dt == nullptr || B == nullptr || C == nullptr || out == nullptr))
+        return MAMBA_ERR_INVALID_ARG;
+    if ((x && !aligned(x, 16)) || (z && !aligned(z, 16)) || (out && !aligned(out, 16)) ||
+        (B && !aligned(B, 16)) || (C && !aligned(C, 16)) || (dt && !aligned(dt, 2)) ||
+        !aligned(A, 4) || (D && !aligned(D, 4)) || (dt_bias && !aligned(dt_bias, 4)) ||
+        (initial_state && !aligned(initial_state, 4)) || (final_state && !aligned(final_state, 4)))
+        return MAMBA_ERR_ALIGN;
+    return MAMBA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+MAMBA_API mamba_status_t mamba_ssd_chunk_scan_fwd(const void* x, const void* dt, const float* A,
+                                                  const void* B, const void* C, const float* D,
+                                                  const void* z, const float* dt_bias,
+                                                  const float* initial_state, void* out,
+                                                  float* final_state,
+                                                  const mamba_ssd_dims_t* dims,
+                                                  cudaStream_t stream) {
+    const mamba_status_t st = check_ssd(x, dt, A, B, C, D, z, dt_bias, initial_state, out,
+                                        final_state, dims);
+    if (st != MAMBA_OK) return st;
+    if (dims->batch == 0) return MAMBA_OK;
+    if (dims->seqlen == 0 && final_state == nullptr) return MAMBA_OK;
+    int dev = 0;
+    if (current_sm_count(&dev) <= 0) return MAMBA_ERR_CUDA;
+    static bool attr_done[kMaxDevices] = {false};
+    cudaError_t e = ensure_smem_attr(ssd_chunk_scan_kernel, kSsdSmemBytes, attr_done, dev);
+    if (e != cudaSuccess) return MAMBA_ERR_CUDA;
+    SsdParams prm;
+    prm.x = static_cast<const __nv_bfloat16*>(x);
+    prm.dt = static_cast<const __nv_bfloat16*>(dt);
+    prm.A = A;
+    prm.B = static_cast<const __nv_bfloat16*>(B);
+    prm.C = static_cast<const __nv_bfloat16*>(C);
+    prm.D = D;
+    prm.z = static_cast<const __nv_bfloat16*>(z);
+    prm.dt_bias = dt_bias;
+    prm.h0 = initial_state;
+    prm.out = static_cast<__nv_bfloat16*>(out);
+    prm.hT = final_state;
+    prm.seqlen = dims->seqlen;
+    prm.nheads = (int)dims->nheads;
+    prm.ngroups = (int)dims->ngroups;
+    prm.softplus = dims->dt_softplus != 0;
+    const unsigned grid = (unsigned)(dims->batch * dims->nheads);
+    ssd_chunk_scan_kernel<<<grid, kSsdThreads, kSsdSmemBytes, stream>>>(prm);
+    e = cudaGetLastError();
+    return e == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
+}
+
+}  // extern "C"
 
 extern "C" {
 

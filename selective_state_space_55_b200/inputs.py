@@ -24,6 +24,17 @@ Workloads (sizes from the pages' model shapes; all values synthetic):
 
 A is the S4D-real initialisation A_d,n = -(n+1), i.e. -1 ... -16 for N = 16
 ("Mamba 与状态空间模型", section 每一步都一样).
+
+Mamba-2 layer workloads (scalar A per head, head dim 64, state 128 per
+channel as in "Mamba 与状态空间模型", section "Mamba-2：两种算法"; layout
+(batch, L, heads, headdim)):
+
+  ssd_small          batch 2, L 300 (three chunks of 128, the last ragged),
+                     4 heads in 2 groups, with a start state.
+  mamba2_2p7b_layer  batch 16, L 2048, 80 heads x 64 (d_inner 5120), 1 group.
+                     Both: x, z, dt ~ N(0,1) bf16; dt_bias as the layer shapes;
+                     A_h = -U(1, 16); B, C ~ N(0,1)/4 bf16; D = 1; start state
+                     ~ N(0,1)/4 fp32 where used.
 """
 from __future__ import annotations
 
@@ -78,6 +89,61 @@ SCAN_CONFIGS = {
     "long_dna_1m": ScanConfig("long_dna_1m", 1, 1536, 16, 1 << 20, torch.bfloat16,
                               torch.bfloat16, "dna", last_state=True),
 }
+
+@dataclass(frozen=True)
+class SsdConfig:
+    name: str
+    batch: int
+    seqlen: int
+    nheads: int
+    headdim: int = 64
+    ngroups: int = 1
+    dstate: int = 128
+    has_z: bool = True
+    has_D: bool = True
+    has_bias: bool = True
+    initial_state: bool = False
+
+    @property
+    def elements(self) -> int:
+        return self.batch * self.seqlen * self.nheads * self.headdim
+
+    def resized(self, **kw) -> "SsdConfig":
+        return replace(self, **kw)
+
+
+SSD_CONFIGS = {
+    "ssd_small": SsdConfig("ssd_small", batch=2, seqlen=300, nheads=4, ngroups=2,
+                           initial_state=True),
+    "mamba2_2p7b_layer": SsdConfig("mamba2_2p7b_layer", batch=16, seqlen=2048, nheads=80),
+}
+
+
+def make_ssd_inputs(cfg: SsdConfig, device="cpu", seed: int = 0) -> dict:
+    """All Mamba-2 layer inputs for ``cfg`` as contiguous tensors on ``device``.
+
+    Keys: x, dt, A, B, C, D, z, dt_bias, initial_state (None where absent).
+    """
+    g = _gen(device, seed)
+    bsz, L, H, P, G, N = cfg.batch, cfg.seqlen, cfg.nheads, cfg.headdim, cfg.ngroups, cfg.dstate
+    bf = torch.bfloat16
+    x = _normal((bsz, L, H, P), g, device, dtype=bf)
+    z = _normal((bsz, L, H, P), g, device, dtype=bf)
+    dt = _normal((bsz, L, H), g, device, dtype=bf)
+    bias = layer_delta_bias(H, g, device)
+    A = (-_uniform((H,), 1.0, 16.0, g, device)).to(torch.float32)
+    B = _normal((bsz, L, G, N), g, device, scale=0.25, dtype=bf)
+    C = _normal((bsz, L, G, N), g, device, scale=0.25, dtype=bf)
+    h0 = _normal((bsz, H, P, N), g, device, scale=0.25)
+    return dict(
+        x=x.contiguous(), dt=dt.contiguous(), A=A.contiguous(), B=B.contiguous(),
+        C=C.contiguous(),
+        D=torch.ones(H, dtype=torch.float32, device=device) if cfg.has_D else None,
+        z=z.contiguous() if cfg.has_z else None,
+        dt_bias=bias.contiguous() if cfg.has_bias else None,
+        initial_state=h0.contiguous() if cfg.initial_state else None,
+    )
+
 
 DECODE_CONFIG = DecodeConfig("decode_b128", batch=128, dim=4096, dstate=16, layers=48, steps=128)
 
@@ -220,5 +286,5 @@ def gather_chains(inputs: dict, chains: list[tuple[int, int]]) -> dict:
 __all__ = [
     "ScanConfig", "DecodeConfig", "SCAN_CONFIGS", "DECODE_CONFIG", "s4d_real_A",
     "make_scan_inputs", "make_decode_layer", "make_decode_token", "sample_chains",
-    "gather_chains", "layer_delta_bias",
+    "gather_chains", "layer_delta_bias", "SsdConfig", "SSD_CONFIGS", "make_ssd_inputs",
 ]

@@ -43,6 +43,14 @@ class MambaDims(ctypes.Structure):
     ]
 
 
+class SsdDims(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64), ("nheads", ctypes.c_int64),
+        ("headdim", ctypes.c_int64), ("ngroups", ctypes.c_int64), ("dstate", ctypes.c_int64),
+        ("io_dtype", ctypes.c_int32), ("dt_softplus", ctypes.c_int32),
+    ]
+
+
 class ScanPlan(ctypes.Structure):
     _fields_ = [
         ("nchunks", ctypes.c_int32), ("tile_len", ctypes.c_int32),
@@ -104,6 +112,8 @@ def library(path: Path | str | None = None) -> ctypes.CDLL:
     lib.mamba_causal_conv1d_update.argtypes = [vp, vp, vp, vp, i32, i32, vp, dims_p, vp]
     lib.mamba_selective_state_update.restype = i32
     lib.mamba_selective_state_update.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, dims_p, vp]
+    lib.mamba_ssd_chunk_scan_fwd.restype = i32
+    lib.mamba_ssd_chunk_scan_fwd.argtypes = [vp] * 11 + [ctypes.POINTER(SsdDims), vp]
     lib.mamba_device_status.restype = i32
     lib.mamba_device_status.argtypes = []
     lib.mamba_status_string.restype = ctypes.c_char_p
@@ -456,6 +466,48 @@ def causal_conv1d_update(conv_state, x, weight, bias=None, silu=True, out=None, 
         ctypes.byref(dims), _stream_handle(stream))
     if rc != MAMBA_OK:
         raise MambaError("mamba_causal_conv1d_update", rc)
+    return out
+
+
+def ssd_chunk_scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_softplus=True,
+                       initial_state=None, out=None, final_state=None,
+                       return_final_state=False, stream=None):
+    """Mamba-2 layer (scalar A per head) through ``mamba_ssd_chunk_scan_fwd``.
+
+    x, z: (batch, L, nheads, 64) bf16; dt: (batch, L, nheads) bf16; A, D,
+    dt_bias: (nheads,) fp32; B, C: (batch, L, ngroups, 128) bf16;
+    initial_state: (batch, nheads, 64, 128) fp32 or None.  Returns out (like
+    x), or (out, final_state) when ``return_final_state``.
+    """
+    batch, L, nheads, headdim = x.shape
+    ngroups, dstate = B.shape[2], B.shape[3]
+    bf = (torch.bfloat16,)
+    _check_cuda("x", x, bf, (batch, L, nheads, headdim))
+    _check_cuda("dt", dt, bf, (batch, L, nheads))
+    _check_cuda("A", A, (torch.float32,), (nheads,))
+    _check_cuda("B", B, bf, (batch, L, ngroups, dstate))
+    _check_cuda("C", C, bf, (batch, L, ngroups, dstate))
+    _check_cuda("D", D, (torch.float32,), (nheads,))
+    _check_cuda("z", z, bf, (batch, L, nheads, headdim))
+    _check_cuda("dt_bias", dt_bias, (torch.float32,), (nheads,))
+    st_shape = (batch, nheads, headdim, dstate)
+    _check_cuda("initial_state", initial_state, (torch.float32,), st_shape)
+    if out is None:
+        out = torch.empty_like(x)
+    _check_cuda("out", out, bf, tuple(x.shape))
+    if final_state is None and return_final_state:
+        final_state = torch.empty(st_shape, dtype=torch.float32, device=x.device)
+    _check_cuda("final_state", final_state, (torch.float32,), st_shape)
+    dims = SsdDims(batch=batch, seqlen=L, nheads=nheads, headdim=headdim, ngroups=ngroups,
+                   dstate=dstate, io_dtype=MAMBA_BF16, dt_softplus=int(bool(dt_softplus)))
+    rc = library().mamba_ssd_chunk_scan_fwd(
+        _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(dt_bias),
+        _ptr(initial_state), _ptr(out), _ptr(final_state), ctypes.byref(dims),
+        _stream_handle(stream))
+    if rc != MAMBA_OK:
+        raise MambaError("mamba_ssd_chunk_scan_fwd", rc)
+    if return_final_state or final_state is not None:
+        return out, final_state
     return out
 
 

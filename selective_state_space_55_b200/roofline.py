@@ -82,3 +82,29 @@ def kv_cache_bytes_per_token(layers: int, width: int, bytes_per_number: int) -> 
     """A Transformer's KV cache per token: a key and a value of `width`
     numbers in every layer."""
     return 2 * layers * width * bytes_per_number
+
+
+def ssd_bytes(batch: int, seqlen: int, nheads: int, headdim: int = 64, ngroups: int = 1,
+              dstate: int = 128, has_z: bool = True, initial_state: bool = False,
+              final_state: bool = True) -> int:
+    """HBM bytes of one Mamba-2 layer pass in bf16: x, (z), dt read and out
+    written per (token, head); B and C once per (token, group); the fp32
+    state read (start state) and written (final state) once per head."""
+    tokens = batch * seqlen
+    per_head = (2 + 2 + (2 if has_z else 0)) * headdim + 2
+    state = batch * nheads * headdim * dstate * 4
+    return (tokens * nheads * per_head + tokens * ngroups * dstate * 2 * 2 +
+            state * (int(initial_state) + int(final_state)))
+
+
+def ssd_chunk_flops(batch: int, seqlen: int, nheads: int, headdim: int = 64,
+                    dstate: int = 128, chunk: int = 128) -> int:
+    """Dense tensor-core FLOPs the chunked algorithm issues per pass: per chunk
+    and head, C B^T (chunk x chunk x dstate), the masked matrix times x
+    (chunk x chunk x headdim), the chunk's state B^T x (dstate x chunk x
+    headdim) and the entering state's read-out C H^T (chunk x dstate x
+    headdim), 2 FLOPs per multiply-add.  Chunks are counted whole (a ragged
+    last chunk is padded)."""
+    chunks = -(-seqlen // chunk)
+    per = 2 * (chunk * chunk * dstate + chunk * chunk * headdim + 2 * dstate * chunk * headdim)
+    return batch * nheads * chunks * per

@@ -249,3 +249,31 @@ def test_plan_rejects_bad_dims(lib):
         ops.scan_plan(1, 32, 17, 64)
     with pytest.raises(ops.MambaError):
         ops.scan_plan(-1, 32, 16, 64)
+
+
+def _ssd(lib, dims, x=FAKE, dt=FAKE, A=FAKE, B=FAKE, C=FAKE, out=FAKE):
+    return lib.mamba_ssd_chunk_scan_fwd(x, dt, A, B, C, None, None, None, None, out, None,
+                                        ctypes.byref(dims) if dims is not None else None, None)
+
+
+def _ssd_dims(**kw):
+    base = dict(batch=2, seqlen=256, nheads=8, headdim=64, ngroups=1, dstate=128,
+                io_dtype=ops.MAMBA_BF16, dt_softplus=1)
+    base.update(kw)
+    return ops.SsdDims(**base)
+
+
+def test_ssd_rejects_bad_arguments_before_launch(lib):
+    assert _ssd(lib, None) == -1
+    assert _ssd(lib, _ssd_dims(batch=-1)) == -1
+    assert _ssd(lib, _ssd_dims(seqlen=-1)) == -1
+    assert _ssd(lib, _ssd_dims(nheads=6, ngroups=4)) == -1          # groups must divide heads
+    assert _ssd(lib, _ssd_dims(headdim=32)) == -2
+    assert _ssd(lib, _ssd_dims(dstate=64)) == -2
+    assert _ssd(lib, _ssd_dims(io_dtype=ops.MAMBA_F32)) == -2
+    assert _ssd(lib, _ssd_dims(), x=None) == -1
+    assert _ssd(lib, _ssd_dims(), A=None) == -1
+    assert _ssd(lib, _ssd_dims(), out=None) == -1
+    assert _ssd(lib, _ssd_dims(), x=ctypes.c_void_p(0x10008)) == -3  # 16-byte rows
+    assert _ssd(lib, _ssd_dims(), dt=ctypes.c_void_p(0x10001)) == -3
+    assert _ssd(lib, _ssd_dims(batch=0)) == 0                         # nothing to do
