@@ -1115,6 +1115,23 @@ cudaError_t zero_async(void* p, size_t bytes, cudaStream_t stream) {
 
 namespace {
 
+// 4-D map over a row-major bf16 (d3, d2, d1, d0) tensor with the box
+// (8, 1, 128, 1): one 2048-byte operand slab of the Mamba-2 layer kernel.
+bool encode_map_ssd(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                    uint64_t d3) {
+    auto encode = tensor_map_encoder();
+    if (encode == nullptr) return false;
+    const cuuint64_t dims[4] = {d0, d1, d2, d3};
+    const cuuint64_t strides[3] = {d0 * 2, d0 * d1 * 2, d0 * d1 * d2 * 2};
+    const cuuint32_t box[4] = {8, 1, (cuuint32_t)kSsdQ, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base),
+                              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // Argument checks of the Mamba-2 layer; MAMBA_OK when a launch may follow.
 mamba_status_t check_ssd(const void* x, const void* dt, const float* A, const void* B,
                          const void* C, const float* D, const void* z, const float* dt_bias,
@@ -1178,8 +1195,23 @@ MAMBA_API mamba_status_t mamba_ssd_chunk_scan_fwd(const void* x, const void* dt,
     prm.nheads = (int)dims->nheads;
     prm.ngroups = (int)dims->ngroups;
     prm.softplus = dims->dt_softplus != 0;
+    // TMA maps over x, z, out (batch, L, nheads, 64) and B, C (batch, L, ngroups,
+    // 128).  With L == 0 no chunk runs and the maps are never read.
+    CUtensorMap maps[5];
+    std::memset(maps, 0, sizeof(maps));
+    if (dims->seqlen > 0) {
+        const uint64_t Bt = (uint64_t)dims->batch, L = (uint64_t)dims->seqlen;
+        const uint64_t H = (uint64_t)dims->nheads, G = (uint64_t)dims->ngroups;
+        const bool ok = encode_map_ssd(&maps[0], x, kSsdP, H, L, Bt) &&
+                        encode_map_ssd(&maps[1], z ? z : x, kSsdP, H, L, Bt) &&
+                        encode_map_ssd(&maps[2], B, kSsdN, G, L, Bt) &&
+                        encode_map_ssd(&maps[3], C, kSsdN, G, L, Bt) &&
+                        encode_map_ssd(&maps[4], out, kSsdP, H, L, Bt);
+        if (!ok) return MAMBA_ERR_CUDA;
+    }
     const unsigned grid = (unsigned)(dims->batch * dims->nheads);
-    ssd_chunk_scan_kernel<<<grid, kSsdThreads, kSsdSmemBytes, stream>>>(prm);
+    ssd_chunk_scan_kernel<<<grid, kSsdThreads, kSsdSmemBytes, stream>>>(prm, maps[0], maps[1],
+                                                                        maps[2], maps[3], maps[4]);
     e = cudaGetLastError();
     return e == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
 }

@@ -47,8 +47,10 @@ constexpr int kSsdOffX = 65536;      // 128 x 64 bf16: x (rows j, k = p)
 constexpr int kSsdOffXw = 81920;     // 128 x 64 bf16: Xw (rows j, k = p)
 constexpr int kSsdOffH = 98304;      // 128 x 64 bf16: H (rows n, k = p)
 constexpr int kSsdOffE = 114688;     // 128 fp32: e_j = c_j - log2(Delta_j)
-constexpr int kSsdOffMisc = 115200;  // two mbarriers (+8, +16), the TMEM address (+24)
-constexpr int kSsdSmemBytes = 115232;
+constexpr int kSsdOffMisc = 115200;  // mbarriers (+0 products 1/3/4, +8 product 2, +16 tiles,
+                                     // +24 gate), the TMEM address (+32), warp totals (+48)
+constexpr int kSsdSmemBytes = 115264;
+constexpr uint32_t kSsdTileBytes = 2 * 32768 + 16384;   // C, B and x of one chunk
 
 struct SsdParams {
     const __nv_bfloat16* x;      // (batch, L, nheads, 64)
@@ -140,17 +142,44 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(r[k]);
 }
 
-__device__ __forceinline__ void cp_async_wait_all_copies() {
-    asm volatile("cp.async.wait_all;" ::: "memory");
+// 4-D tiled TMA copies.  Every map here is (inner 8 elements, 1, 128 rows, 1):
+// one 2048-byte slab of the operand layout, rows 16 bytes apart.  Rows past
+// the tensor's end are filled with zeros on load and dropped on store.
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
+                                            int c2, int c3, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
+        : "memory");
 }
 
-// 16-byte cp.async that fills zeros instead of reading when `valid` is false.
-__device__ __forceinline__ void cp_async16_or_zero(uint32_t dst, const void* src, bool valid) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst),
-                 "l"(reinterpret_cast<uint64_t>(src)), "r"(valid ? 16 : 0)
-                 : "memory");
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, uint32_t src, int c0, int c1,
+                                             int c2, int c3) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];"
+        ::"l"(reinterpret_cast<uint64_t>(map)), "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
 }
 
+// Two 32-column loads of this thread's TMEM lane and one wait: both arrays
+// are valid when the statement ends.
+__device__ __forceinline__ void tmem_ld32x2(uint32_t ta, uint32_t tb, float (&a)[32],
+                                            float (&b)[32]) {
+    uint32_t ra[32], rb[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%64];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(ra[0]), "=r"(ra[1]), "=r"(ra[2]), "=r"(ra[3]), "=r"(ra[4]), "=r"(ra[5]), "=r"(ra[6]), "=r"(ra[7]), "=r"(ra[8]), "=r"(ra[9]), "=r"(ra[10]), "=r"(ra[11]), "=r"(ra[12]), "=r"(ra[13]), "=r"(ra[14]), "=r"(ra[15]), "=r"(ra[16]), "=r"(ra[17]), "=r"(ra[18]), "=r"(ra[19]), "=r"(ra[20]), "=r"(ra[21]), "=r"(ra[22]), "=r"(ra[23]), "=r"(ra[24]), "=r"(ra[25]), "=r"(ra[26]), "=r"(ra[27]), "=r"(ra[28]), "=r"(ra[29]), "=r"(ra[30]), "=r"(ra[31]), "=r"(rb[0]), "=r"(rb[1]), "=r"(rb[2]), "=r"(rb[3]), "=r"(rb[4]), "=r"(rb[5]), "=r"(rb[6]), "=r"(rb[7]), "=r"(rb[8]), "=r"(rb[9]), "=r"(rb[10]), "=r"(rb[11]), "=r"(rb[12]), "=r"(rb[13]), "=r"(rb[14]), "=r"(rb[15]), "=r"(rb[16]), "=r"(rb[17]), "=r"(rb[18]), "=r"(rb[19]), "=r"(rb[20]), "=r"(rb[21]), "=r"(rb[22]), "=r"(rb[23]), "=r"(rb[24]), "=r"(rb[25]), "=r"(rb[26]), "=r"(rb[27]), "=r"(rb[28]), "=r"(rb[29]), "=r"(rb[30]), "=r"(rb[31])
+        : "r"(ta), "r"(tb)
+        : "memory");
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+        a[k] = __uint_as_float(ra[k]);
+        b[k] = __uint_as_float(rb[k]);
+    }
+}
 
 // The state H of this thread's row n as bf16 into sH: offset (p / 8) * 2048 + n * 16.
 __device__ __forceinline__ void ssd_store_state(unsigned char* smem, int n, const float (&H)[kSsdP]) {
@@ -172,23 +201,33 @@ __device__ __forceinline__ bool ssd_wait_failed(uint32_t bar, uint32_t parity) {
     return failed;
 }
 
-__global__ void __launch_bounds__(kSsdThreads, 2) ssd_chunk_scan_kernel(const SsdParams p) {
+__global__ void __launch_bounds__(kSsdThreads, 2)
+    ssd_chunk_scan_kernel(const __grid_constant__ SsdParams p,
+                          const __grid_constant__ CUtensorMap tm_x,
+                          const __grid_constant__ CUtensorMap tm_z,
+                          const __grid_constant__ CUtensorMap tm_B,
+                          const __grid_constant__ CUtensorMap tm_C,
+                          const __grid_constant__ CUtensorMap tm_out) {
     extern __shared__ __align__(1024) unsigned char smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int chain = blockIdx.x;                           // b * nheads + h
     const int h = chain % p.nheads;
-    const int64_t b = chain / p.nheads;
+    const int b = chain / p.nheads;
     const int g = h / (p.nheads / p.ngroups);
     const int64_t L = p.seqlen;
     const uint32_t s0 = smem_u32(smem);
     float* sE = reinterpret_cast<float*>(smem + kSsdOffE);
-    const uint32_t bar1 = s0 + kSsdOffMisc + 8, bar2 = s0 + kSsdOffMisc + 16;
-    const uint32_t* tslot = reinterpret_cast<const uint32_t*>(smem + kSsdOffMisc + 24);
+    float* sTot = reinterpret_cast<float*>(smem + kSsdOffMisc + 48);
+    const uint32_t bar1 = s0 + kSsdOffMisc, bar2 = bar1 + 8, bar_ld = bar1 + 16, bar_z = bar1 + 24;
+    const uint32_t* tslot = reinterpret_cast<const uint32_t*>(smem + kSsdOffMisc + 32);
+    const bool has_z = p.z != nullptr;
 
-    if (warp == 0) tmem_alloc(s0 + kSsdOffMisc + 24, kSsdTmemCols);
+    if (warp == 0) tmem_alloc(s0 + kSsdOffMisc + 32, kSsdTmemCols);
     if (tid == 0) {
         mbar_init(bar1, 1);
         mbar_init(bar2, 1);
+        mbar_init(bar_ld, 1);
+        mbar_init(bar_z, 1);
         fence_mbar_init();
     }
     tc_fence_before();
@@ -208,56 +247,47 @@ __global__ void __launch_bounds__(kSsdThreads, 2) ssd_chunk_scan_kernel(const Ss
     for (int q = 0; q < kSsdP; ++q) H[q] = p.h0 ? p.h0[hoff + (size_t)q * kSsdN] : 0.0f;
     ssd_store_state(smem, tid, H);
 
-    const int64_t xs = (int64_t)p.nheads * kSsdP;   // token stride of x, z, out
-    const int64_t bcs = (int64_t)p.ngroups * kSsdN; // token stride of B, C
     const int64_t nchunks = (L + kSsdQ - 1) / kSsdQ;
     bool failed = false;
+    // dt of this thread's token in the next chunk, loaded one chunk ahead.
+    auto load_dt = [&](int64_t l) -> float {
+        return l < L ? __bfloat162float(p.dt[((int64_t)b * L + l) * p.nheads + h]) : 0.0f;
+    };
+    float dt_next = load_dt(tid);
 
     for (int64_t c = 0; c < nchunks; ++c) {
-        const int64_t l0 = c * kSsdQ;
-        const int valid = (int)(L - l0 < kSsdQ ? L - l0 : kSsdQ);
+        const int l0 = (int)(c * kSsdQ);
         const uint32_t parity = (uint32_t)(c & 1);
 
-        // ---- operands: C, B (128 x 128) and x (128 x 64) by cp.async, zero rows
-        // past the end.  A warp copies 8 rows x 4 pieces of 16 bytes per step:
-        // 64 contiguous bytes of each row, four 128-byte runs of shared memory.
-        const __nv_bfloat16* Cg = p.C + ((b * L + l0) * p.ngroups + g) * kSsdN;
-        const __nv_bfloat16* Bg = p.B + ((b * L + l0) * p.ngroups + g) * kSsdN;
-        const __nv_bfloat16* Xg = p.x + ((b * L + l0) * p.nheads + h) * kSsdP;
-#pragma unroll
-        for (int it = 0; it < 16; ++it) {
-            const int q = tid + kSsdThreads * it;
-            const int r = (((q >> 5) & 15) << 3) | (q & 7);
-            const int kb = ((q >> 9) << 2) | ((q >> 3) & 3);
-            const uint32_t off = (uint32_t)(kb * 2048 + r * 16);
-            const bool ok = r < valid;
-            const int64_t src = ok ? (int64_t)r * bcs + kb * 8 : 0;
-            cp_async16_or_zero(s0 + kSsdOffC + off, Cg + src, ok);
-            cp_async16_or_zero(s0 + kSsdOffB + off, Bg + src, ok);
-        }
-#pragma unroll
-        for (int it = 0; it < 8; ++it) {
-            const int q = tid + kSsdThreads * it;
-            const int r = (((q >> 5) & 15) << 3) | (q & 7);
-            const int pb = ((q >> 9) << 2) | ((q >> 3) & 3);
-            const bool ok = r < valid;
-            cp_async16_or_zero(s0 + kSsdOffX + (uint32_t)(pb * 2048 + r * 16),
-                               Xg + (ok ? (int64_t)r * xs + pb * 8 : 0), ok);
+        // ---- C, B (128 x 128) and x (128 x 64) by TMA, one 2048-byte slab per
+        // 8 columns; rows past the end arrive as zeros.  The previous chunk's
+        // output store must have read the staging tile before it is reused.
+        if (tid == 0) {
+            bulk_wait_read<0>();
+            mbar_arrive_expect_tx(bar_ld, kSsdTileBytes);
+#pragma unroll 1
+            for (int kb = 0; kb < kSsdN / 8; ++kb) {
+                tma_load_4d(s0 + kSsdOffC + kb * 2048, &tm_C, kb * 8, g, l0, b, bar_ld);
+                tma_load_4d(s0 + kSsdOffB + kb * 2048, &tm_B, kb * 8, g, l0, b, bar_ld);
+            }
+#pragma unroll 1
+            for (int pb = 0; pb < kSsdP / 8; ++pb)
+                tma_load_4d(s0 + kSsdOffX + pb * 2048, &tm_x, pb * 8, h, l0, b, bar_ld);
         }
 
         // ---- Delta, the running log2-decay c_i and e_i = c_i - log2(Delta_i).
         float delta = 0.0f;
-        if (tid < valid) {
-            const float s = __bfloat162float(p.dt[(b * L + l0 + tid) * p.nheads + h]) + bias;
-            delta = p.softplus ? softplus_f32(s) : s;
+        if (l0 + tid < L) {
+            const float sarg = dt_next + bias;
+            delta = p.softplus ? softplus_f32(sarg) : sarg;
         }
+        dt_next = load_dt((int64_t)l0 + kSsdQ + tid);
         float a = delta * A2;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const float v = __shfl_up_sync(0xffffffffu, a, o);
             if (lane >= o) a += v;
         }
-        float* sTot = reinterpret_cast<float*>(smem + kSsdOffXw);   // Xw is free until below
         if (lane == 31) sTot[warp] = a;
         __syncthreads();
         float pre = 0.0f;
@@ -265,8 +295,10 @@ __global__ void __launch_bounds__(kSsdThreads, 2) ssd_chunk_scan_kernel(const Ss
         const float ci = a + pre;
         const float cQ = (sTot[0] + sTot[1]) + (sTot[2] + sTot[3]);
         sE[tid] = ci - lg2_approx(delta);   // +inf for Delta = 0
-        cp_async_wait_all_copies();
-        __syncthreads();
+        if (ssd_wait_failed(bar_ld, parity)) {   // tiles landed; sE published
+            failed = true;
+            break;
+        }
 
         // ---- Xw_j = 2^(c_Q - e_j) x_j = 2^(c_Q - c_j) Delta_j x_j (row j = tid).
         {
@@ -309,33 +341,71 @@ __global__ void __launch_bounds__(kSsdThreads, 2) ssd_chunk_scan_kernel(const Ss
             break;
         }
 
+        // ---- the gate tile z (128 x 64) by TMA into the Xw buffer, which MMA 4
+        // no longer reads; it lands while the masked matrix and MMA 2 run.
+        if (tid == 0 && has_z) {
+            mbar_arrive_expect_tx(bar_z, 16384);
+#pragma unroll 1
+            for (int pb = 0; pb < kSsdP / 8; ++pb)
+                tma_load_4d(s0 + kSsdOffXw + pb * 2048, &tm_z, pb * 8, h, l0, b, bar_z);
+        }
+
         // ---- state: H = 2^(c_Q) H + S (row n = tid), then its bf16 copy for
         // the next chunk's MMA 3.
         {
             const float dq = ex2_approx(cQ);
-            float sv[32];
+            float s_lo[32], s_hi[32];
+            tmem_ld32x2(tlane + 192, tlane + 224, s_lo, s_hi);
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                tmem_ld32(tlane + 192 + half * 32, sv);
-#pragma unroll
-                for (int k = 0; k < 32; ++k) H[half * 32 + k] = fmaf(dq, H[half * 32 + k], sv[k]);
+            for (int k = 0; k < 32; ++k) {
+                H[k] = fmaf(dq, H[k], s_lo[k]);
+                H[32 + k] = fmaf(dq, H[32 + k], s_hi[k]);
             }
             ssd_store_state(smem, tid, H);
         }
 
         // ---- Gm_ij = G_ij 2^(c_i - e_j) for j <= i (row i = tid), over C's tile.
+        // Warp w holds rows [32w, 32w + 32): quarters of columns below w are
+        // entirely at or below the diagonal, quarter w straddles it, and the
+        // quarters above are zero (no TMEM read, no exponentials).  Quarters
+        // are read from TMEM two at a time.
 #pragma unroll
-        for (int quarter = 0; quarter < 4; ++quarter) {
-            float gv[32];
-            tmem_ld32(tlane + quarter * 32, gv);
+        for (int pair = 0; pair < 2; ++pair) {
+            const int qa = 2 * pair, qb = 2 * pair + 1;
+            if (qa > warp) {
+                const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int j0 = quarter * 32 + q * 8;
-                float f[8];
+                for (int q = 0; q < 8; ++q)
+                    *reinterpret_cast<uint4*>(smem + kSsdOffC + (qa * 4 + q) * 2048 + tid * 16) = zero;
+                continue;
+            }
+            float gv[2][32];
+            tmem_ld32x2(tlane + qa * 32, tlane + qb * 32, gv[0], gv[1]);
 #pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    f[k] = (j0 + k <= tid) ? gv[q * 8 + k] * ex2_approx(ci - sE[j0 + k]) : 0.0f;
-                *reinterpret_cast<uint4*>(smem + kSsdOffC + (j0 / 8) * 2048 + tid * 16) = pack16(f);
+            for (int half = 0; half < 2; ++half) {
+                const int quarter = qa + half;
+                if (quarter > warp) {
+                    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        *reinterpret_cast<uint4*>(smem + kSsdOffC + (quarter * 4 + q) * 2048 + tid * 16) = zero;
+                    continue;
+                }
+                const bool diag = quarter == warp;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int j0 = quarter * 32 + q * 8;
+                    const float4 e0 = *reinterpret_cast<const float4*>(sE + j0);
+                    const float4 e1 = *reinterpret_cast<const float4*>(sE + j0 + 4);
+                    const float ej[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
+                    float f[8];
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const float v = gv[half][q * 8 + k] * ex2_approx(ci - ej[k]);
+                        f[k] = (!diag || j0 + k <= tid) ? v : 0.0f;
+                    }
+                    *reinterpret_cast<uint4*>(smem + kSsdOffC + (j0 / 8) * 2048 + tid * 16) = pack16(f);
+                }
             }
         }
         fence_proxy_async_smem();
@@ -352,49 +422,54 @@ __global__ void __launch_bounds__(kSsdThreads, 2) ssd_chunk_scan_kernel(const Ss
                           umma_sdesc(s0 + kSsdOffX + k * 256, 128, 2048), id_y, k);
             umma_commit(bar2);
         }
-        if (ssd_wait_failed(bar2, parity)) {
+        if (ssd_wait_failed(bar2, parity) || (has_z && ssd_wait_failed(bar_z, parity))) {
             failed = true;
             break;
         }
 
-        // ---- y_i = Ydiag_i + 2^(c_i) Yoff_i + D x_i, gated, stored (row i = tid).
+        // ---- y_i = Ydiag_i + 2^(c_i) Yoff_i + D x_i, gated (row i = tid), written
+        // as bf16 over the gate tile, then stored by TMA (rows past the end dropped).
         {
             const float sc = ex2_approx(ci);
-            const int64_t row = ((b * L + l0 + tid) * p.nheads + h) * kSsdP;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 float yd[32], yo[32];
-                tmem_ld32(tlane + half * 32, yd);
-                tmem_ld32(tlane + 128 + half * 32, yo);
-                if (tid < valid) {
+                tmem_ld32x2(tlane + half * 32, tlane + 128 + half * 32, yd, yo);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int p0 = half * 32 + q * 8;
-                        float xv[8], f[8];
-                        unpack16(*reinterpret_cast<const uint4*>(smem + kSsdOffX + (p0 / 8) * 2048 +
-                                                                 tid * 16), xv);
+                for (int q = 0; q < 4; ++q) {
+                    const int pb = half * 4 + q;
+                    const uint32_t off = (uint32_t)(pb * 2048 + tid * 16);
+                    float xv[8], f[8];
+                    unpack16(*reinterpret_cast<const uint4*>(smem + kSsdOffX + off), xv);
 #pragma unroll
-                        for (int k = 0; k < 8; ++k)
-                            f[k] = fmaf(Dh, xv[k], fmaf(sc, yo[q * 8 + k], yd[q * 8 + k]));
-                        if (p.z) {
-                            float zv[8];
-                            unpack16(*reinterpret_cast<const uint4*>(p.z + row + p0), zv);
+                    for (int k = 0; k < 8; ++k)
+                        f[k] = fmaf(Dh, xv[k], fmaf(sc, yo[q * 8 + k], yd[q * 8 + k]));
+                    if (has_z) {
+                        float zv[8];
+                        unpack16(*reinterpret_cast<const uint4*>(smem + kSsdOffXw + off), zv);
 #pragma unroll
-                            for (int k = 0; k < 8; ++k) f[k] *= silu_f32(zv[k]);
-                        }
-                        *reinterpret_cast<uint4*>(p.out + row + p0) = pack16(f);
+                        for (int k = 0; k < 8; ++k) f[k] *= silu_f32(zv[k]);
                     }
+                    *reinterpret_cast<uint4*>(smem + kSsdOffXw + off) = pack16(f);
                 }
             }
         }
+        fence_proxy_async_smem();
         tc_fence_before();
-        __syncthreads();   // the next chunk rewrites the tiles and the TMEM columns
+        __syncthreads();   // the output tile is complete; the next chunk rewrites the rest
+        if (tid == 0) {
+#pragma unroll 1
+            for (int pb = 0; pb < kSsdP / 8; ++pb)
+                tma_store_4d(&tm_out, s0 + kSsdOffXw + pb * 2048, pb * 8, h, l0, b);
+            bulk_commit();
+        }
     }
 
     if (!failed && p.hT) {
 #pragma unroll
         for (int q = 0; q < kSsdP; ++q) p.hT[hoff + (size_t)q * kSsdN] = H[q];
     }
+    if (tid == 0) bulk_wait<0>();   // output stores done before the CTA's shared memory goes
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
