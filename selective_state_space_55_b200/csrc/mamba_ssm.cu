@@ -1115,17 +1115,21 @@ cudaError_t zero_async(void* p, size_t bytes, cudaStream_t stream) {
 
 namespace {
 
-// 4-D map over a row-major bf16 (d3, d2, d1, d0) tensor with the box
-// (8, 1, 128, 1): one 2048-byte operand slab of the Mamba-2 layer kernel.
-bool encode_map_ssd(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
-                    uint64_t d3) {
+// Map over a row-major bf16 (batch, L, heads_or_groups, width) tensor whose one
+// box is a whole 128-row operand tile of the Mamba-2 layer kernel in its
+// shared-memory layout: dimensions (8 elements, L, width / 8 column blocks,
+// heads_or_groups, batch), box (8, 128, width / 8, 1, 1), so that shared
+// memory receives block kb of row r at kb * 2048 + r * 16.
+bool encode_map_ssd(CUtensorMap* map, const void* base, uint64_t width, uint64_t heads,
+                    uint64_t L, uint64_t batch) {
     auto encode = tensor_map_encoder();
     if (encode == nullptr) return false;
-    const cuuint64_t dims[4] = {d0, d1, d2, d3};
-    const cuuint64_t strides[3] = {d0 * 2, d0 * d1 * 2, d0 * d1 * d2 * 2};
-    const cuuint32_t box[4] = {8, 1, (cuuint32_t)kSsdQ, 1};
-    const cuuint32_t estr[4] = {1, 1, 1, 1};
-    const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base),
+    const uint64_t row = heads * width * 2;                 // bytes between tokens
+    const cuuint64_t dims[5] = {8, L, width / 8, heads, batch};
+    const cuuint64_t strides[4] = {row, 16, width * 2, row * L};
+    const cuuint32_t box[5] = {8, (cuuint32_t)kSsdQ, (cuuint32_t)(width / 8), 1, 1};
+    const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base),
                               dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -1207,6 +1211,7 @@ MAMBA_API mamba_status_t mamba_ssd_chunk_scan_fwd(const void* x, const void* dt,
                         encode_map_ssd(&maps[2], B, kSsdN, G, L, Bt) &&
                         encode_map_ssd(&maps[3], C, kSsdN, G, L, Bt) &&
                         encode_map_ssd(&maps[4], out, kSsdP, H, L, Bt);
+        // (each map: one box per 128-row tile)
         if (!ok) return MAMBA_ERR_CUDA;
     }
     const unsigned grid = (unsigned)(dims->batch * dims->nheads);

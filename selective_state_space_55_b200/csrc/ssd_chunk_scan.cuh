@@ -15,16 +15,19 @@
 //   G     = C B^T                       (Q x Q,  K = dstate)        MMA 1
 //   Yoff  = C H^T                       (Q x P,  K = dstate)        MMA 3
 //   S^T   = B^T Xw, Xw_j = 2^(c_Q - c_j) Delta_j x_j   (N x P, K = Q) MMA 4
-//   Gm_ij = G_ij 2^(c_i - c_j) Delta_j  for j <= i, else 0  (CUDA cores)
-//   Ydiag = Gm X                        (Q x P,  K = Q)             MMA 2
-//   y_i   = Ydiag_i + 2^(c_i) Yoff_i + D_h x_i,  out = y silu(z)
+//   Gm_ij = G_ij 2^(c_i - c_j) Delta_j  for j <= i, else 0,
+//           plus D_h on the diagonal    (CUDA cores)
+//   Ydiag = Gm X  (= intra-chunk part + D_h x)  (Q x P, K = Q)      MMA 2
+//   y_i   = Ydiag_i + 2^(c_i) Yoff_i,  out = y silu(z)
 //   H     = 2^(c_Q) H + S               (fp32, in registers)
 //
 // Operands are bf16 in shared memory in the no-swizzle canonical layout
 // ("core matrices" of 8 rows x 16 bytes); the products accumulate in fp32 in
 // tensor memory and are read back with tcgen05.ld.  One elected thread
 // issues the tcgen05.mma instructions and commits them to an mbarrier that
-// the CTA waits on (bounded).  Delta_j enters only through
+// the CTA waits on (bounded).  Operand tiles arrive by TMA, one box per
+// tile, and the next chunk's tiles are requested as soon as this chunk's
+// products are done with each buffer.  Delta_j enters only through
 // e_j = c_j - log2(Delta_j), so that 2^(c_i - e_j) = 2^(c_i - c_j) Delta_j
 // and padded tokens (Delta = 0, e = +inf) drop out by themselves.
 #pragma once
@@ -142,23 +145,25 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(r[k]);
 }
 
-// 4-D tiled TMA copies.  Every map here is (inner 8 elements, 1, 128 rows, 1):
-// one 2048-byte slab of the operand layout, rows 16 bytes apart.  Rows past
-// the tensor's end are filled with zeros on load and dropped on store.
-__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
-                                            int c2, int c3, uint32_t bar) {
+// 5-D tiled TMA copies of one whole operand tile.  Each map is (8 elements,
+// L, column blocks, heads or groups, batch) with the box (8, 128, all
+// blocks, 1, 1): shared memory gets column block kb of row r at
+// kb * 2048 + r * 16.  Rows past the end of the sequence are filled with
+// zeros on load and dropped on store.
+__device__ __forceinline__ void tma_load_tile(uint32_t dst, const CUtensorMap* map, int l0,
+                                              int head, int batch, uint32_t bar) {
     asm volatile(
-        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
+        "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %2, %4, %5}], [%6];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(l0), "r"(head), "r"(batch), "r"(bar)
         : "memory");
 }
 
-__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, uint32_t src, int c0, int c1,
-                                             int c2, int c3) {
+__device__ __forceinline__ void tma_store_tile(const CUtensorMap* map, uint32_t src, int l0,
+                                               int head, int batch) {
     asm volatile(
-        "cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];"
-        ::"l"(reinterpret_cast<uint64_t>(map)), "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        "cp.async.bulk.tensor.5d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %2, %4, %5}], [%1];"
+        ::"l"(reinterpret_cast<uint64_t>(map)), "r"(src), "r"(0), "r"(l0), "r"(head), "r"(batch)
         : "memory");
 }
 
@@ -224,6 +229,11 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
 
     if (warp == 0) tmem_alloc(s0 + kSsdOffMisc + 32, kSsdTmemCols);
     if (tid == 0) {
+        prefetch_tensormap(&tm_x);
+        prefetch_tensormap(&tm_z);
+        prefetch_tensormap(&tm_B);
+        prefetch_tensormap(&tm_C);
+        prefetch_tensormap(&tm_out);
         mbar_init(bar1, 1);
         mbar_init(bar2, 1);
         mbar_init(bar_ld, 1);
@@ -255,25 +265,24 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
     };
     float dt_next = load_dt(tid);
 
+    // Tiles of chunk c + 1 are requested while chunk c still computes: B once
+    // MMA 1 and 4 are done with it, C and x once MMA 2 is.  All three complete
+    // on bar_ld, whose expected byte count is set with the first of them.
+    if (tid == 0 && nchunks > 0) {
+        mbar_arrive_expect_tx(bar_ld, kSsdTileBytes);
+        tma_load_tile(s0 + kSsdOffB, &tm_B, 0, g, b, bar_ld);
+        tma_load_tile(s0 + kSsdOffC, &tm_C, 0, g, b, bar_ld);
+        tma_load_tile(s0 + kSsdOffX, &tm_x, 0, h, b, bar_ld);
+    }
+
     for (int64_t c = 0; c < nchunks; ++c) {
         const int l0 = (int)(c * kSsdQ);
         const uint32_t parity = (uint32_t)(c & 1);
 
-        // ---- C, B (128 x 128) and x (128 x 64) by TMA, one 2048-byte slab per
-        // 8 columns; rows past the end arrive as zeros.  The previous chunk's
-        // output store must have read the staging tile before it is reused.
-        if (tid == 0) {
-            bulk_wait_read<0>();
-            mbar_arrive_expect_tx(bar_ld, kSsdTileBytes);
-#pragma unroll 1
-            for (int kb = 0; kb < kSsdN / 8; ++kb) {
-                tma_load_4d(s0 + kSsdOffC + kb * 2048, &tm_C, kb * 8, g, l0, b, bar_ld);
-                tma_load_4d(s0 + kSsdOffB + kb * 2048, &tm_B, kb * 8, g, l0, b, bar_ld);
-            }
-#pragma unroll 1
-            for (int pb = 0; pb < kSsdP / 8; ++pb)
-                tma_load_4d(s0 + kSsdOffX + pb * 2048, &tm_x, pb * 8, h, l0, b, bar_ld);
-        }
+        const bool more = c + 1 < nchunks;
+        // The previous chunk's output store must have read the staging tile
+        // (Xw below) before it is rewritten.
+        if (tid == 0) bulk_wait_read<0>();
 
         // ---- Delta, the running log2-decay c_i and e_i = c_i - log2(Delta_i).
         float delta = 0.0f;
@@ -341,13 +350,16 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
             break;
         }
 
-        // ---- the gate tile z (128 x 64) by TMA into the Xw buffer, which MMA 4
-        // no longer reads; it lands while the masked matrix and MMA 2 run.
+        // ---- next chunk's B; then the gate tile z (128 x 64) by TMA into the Xw
+        // buffer, which MMA 4 no longer reads; both land while the masked
+        // matrix and MMA 2 run.
+        if (tid == 0 && more) {
+            mbar_arrive_expect_tx(bar_ld, kSsdTileBytes);
+            tma_load_tile(s0 + kSsdOffB, &tm_B, l0 + kSsdQ, g, b, bar_ld);
+        }
         if (tid == 0 && has_z) {
             mbar_arrive_expect_tx(bar_z, 16384);
-#pragma unroll 1
-            for (int pb = 0; pb < kSsdP / 8; ++pb)
-                tma_load_4d(s0 + kSsdOffXw + pb * 2048, &tm_z, pb * 8, h, l0, b, bar_z);
+            tma_load_tile(s0 + kSsdOffXw, &tm_z, l0, h, b, bar_z);
         }
 
         // ---- state: H = 2^(c_Q) H + S (row n = tid), then its bf16 copy for
@@ -391,7 +403,7 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
                         *reinterpret_cast<uint4*>(smem + kSsdOffC + (quarter * 4 + q) * 2048 + tid * 16) = zero;
                     continue;
                 }
-                const bool diag = quarter == warp;
+                const bool diag = quarter == warp;   // D_h x_i enters as Gm_ii += D_h
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     const int j0 = quarter * 32 + q * 8;
@@ -402,7 +414,7 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
                         const float v = gv[half][q * 8 + k] * ex2_approx(ci - ej[k]);
-                        f[k] = (!diag || j0 + k <= tid) ? v : 0.0f;
+                        f[k] = (!diag || j0 + k < tid) ? v : (j0 + k == tid ? v + Dh : 0.0f);
                     }
                     *reinterpret_cast<uint4*>(smem + kSsdOffC + (j0 / 8) * 2048 + tid * 16) = pack16(f);
                 }
@@ -422,13 +434,22 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
                           umma_sdesc(s0 + kSsdOffX + k * 256, 128, 2048), id_y, k);
             umma_commit(bar2);
         }
-        if (ssd_wait_failed(bar2, parity) || (has_z && ssd_wait_failed(bar_z, parity))) {
+        if (ssd_wait_failed(bar2, parity)) {
+            failed = true;
+            break;
+        }
+        if (tid == 0 && more) {   // Gm and x are no longer read
+            tma_load_tile(s0 + kSsdOffC, &tm_C, l0 + kSsdQ, g, b, bar_ld);
+            tma_load_tile(s0 + kSsdOffX, &tm_x, l0 + kSsdQ, h, b, bar_ld);
+        }
+        if (has_z && ssd_wait_failed(bar_z, parity)) {
             failed = true;
             break;
         }
 
-        // ---- y_i = Ydiag_i + 2^(c_i) Yoff_i + D x_i, gated (row i = tid), written
-        // as bf16 over the gate tile, then stored by TMA (rows past the end dropped).
+        // ---- y_i = Ydiag_i + 2^(c_i) Yoff_i (D x_i is inside Ydiag), gated (row
+        // i = tid), written as bf16 over the gate tile, then stored by TMA (rows
+        // past the end dropped).
         {
             const float sc = ex2_approx(ci);
 #pragma unroll
@@ -439,11 +460,9 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
                 for (int q = 0; q < 4; ++q) {
                     const int pb = half * 4 + q;
                     const uint32_t off = (uint32_t)(pb * 2048 + tid * 16);
-                    float xv[8], f[8];
-                    unpack16(*reinterpret_cast<const uint4*>(smem + kSsdOffX + off), xv);
+                    float f[8];
 #pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        f[k] = fmaf(Dh, xv[k], fmaf(sc, yo[q * 8 + k], yd[q * 8 + k]));
+                    for (int k = 0; k < 8; ++k) f[k] = fmaf(sc, yo[q * 8 + k], yd[q * 8 + k]);
                     if (has_z) {
                         float zv[8];
                         unpack16(*reinterpret_cast<const uint4*>(smem + kSsdOffXw + off), zv);
@@ -458,9 +477,7 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
         tc_fence_before();
         __syncthreads();   // the output tile is complete; the next chunk rewrites the rest
         if (tid == 0) {
-#pragma unroll 1
-            for (int pb = 0; pb < kSsdP / 8; ++pb)
-                tma_store_4d(&tm_out, s0 + kSsdOffXw + pb * 2048, pb * 8, h, l0, b);
+            tma_store_tile(&tm_out, s0 + kSsdOffXw, l0, h, b);
             bulk_commit();
         }
     }
