@@ -50,8 +50,9 @@ constexpr int kSsdOffX = 65536;      // 128 x 64 bf16: x (rows j, k = p)
 constexpr int kSsdOffXw = 81920;     // 128 x 64 bf16: Xw (rows j, k = p)
 constexpr int kSsdOffH = 98304;      // 128 x 64 bf16: H (rows n, k = p)
 constexpr int kSsdOffE = 114688;     // 128 fp32: e_j = c_j - log2(Delta_j)
-constexpr int kSsdOffMisc = 115200;  // mbarriers (+0 products 1/3/4, +8 product 2, +16 tiles,
-                                     // +24 gate), the TMEM address (+32), warp totals (+48)
+constexpr int kSsdOffMisc = 115200;  // mbarriers (+0 products 1/3, +8 product 2, +16 tiles,
+                                     // +24 gate, +40 product 4), the TMEM address (+32),
+                                     // warp totals (+48)
 constexpr int kSsdSmemBytes = 115264;
 constexpr uint32_t kSsdTileBytes = 2 * 32768 + 16384;   // C, B and x of one chunk
 
@@ -224,6 +225,7 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
     float* sE = reinterpret_cast<float*>(smem + kSsdOffE);
     float* sTot = reinterpret_cast<float*>(smem + kSsdOffMisc + 48);
     const uint32_t bar1 = s0 + kSsdOffMisc, bar2 = bar1 + 8, bar_ld = bar1 + 16, bar_z = bar1 + 24;
+    const uint32_t bar_s = bar1 + 40;
     const uint32_t* tslot = reinterpret_cast<const uint32_t*>(smem + kSsdOffMisc + 32);
     const bool has_z = p.z != nullptr;
 
@@ -238,6 +240,7 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
         mbar_init(bar2, 1);
         mbar_init(bar_ld, 1);
         mbar_init(bar_z, 1);
+        mbar_init(bar_s, 1);
         fence_mbar_init();
     }
     tc_fence_before();
@@ -280,9 +283,6 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
         const uint32_t parity = (uint32_t)(c & 1);
 
         const bool more = c + 1 < nchunks;
-        // The previous chunk's output store must have read the staging tile
-        // (Xw below) before it is rewritten.
-        if (tid == 0) bulk_wait_read<0>();
 
         // ---- Delta, the running log2-decay c_i and e_i = c_i - log2(Delta_i).
         float delta = 0.0f;
@@ -304,6 +304,9 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
         const float ci = a + pre;
         const float cQ = (sTot[0] + sTot[1]) + (sTot[2] + sTot[3]);
         sE[tid] = ci - lg2_approx(delta);   // +inf for Delta = 0
+        // The previous chunk's output store must have read the staging tile
+        // (rewritten by the Xw pass below).
+        if (tid == 0) bulk_wait_read<0>();
         if (ssd_wait_failed(bar_ld, parity)) {   // tiles landed; sE published
             failed = true;
             break;
@@ -325,45 +328,40 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
         fence_proxy_async_smem();
         __syncthreads();
 
-        // ---- MMA 1 (G = C B^T), 3 (Yoff = C H^T), 4 (S^T = B^T Xw).
+        // ---- MMA 4 (S^T = B^T Xw), committed alone, then 3 (Yoff = C H^T) and
+        // 1 (G = C B^T).
         if (tid == 0) {
             tc_fence_after();
             constexpr uint32_t id_g = umma_idesc_bf16(128, 128, false, false);
             constexpr uint32_t id_off = umma_idesc_bf16(128, 64, false, true);
             constexpr uint32_t id_s = umma_idesc_bf16(128, 64, true, true);
 #pragma unroll
-            for (int k = 0; k < kSsdN / 16; ++k)
-                umma_bf16(tmem, umma_sdesc(s0 + kSsdOffC + k * 4096, 2048, 128),
-                          umma_sdesc(s0 + kSsdOffB + k * 4096, 2048, 128), id_g, k);
+            for (int k = 0; k < kSsdQ / 16; ++k)
+                umma_bf16(tmem + 192, umma_sdesc(s0 + kSsdOffB + k * 256, 128, 2048),
+                          umma_sdesc(s0 + kSsdOffXw + k * 256, 128, 2048), id_s, k);
+            umma_commit(bar_s);
 #pragma unroll
             for (int k = 0; k < kSsdN / 16; ++k)
                 umma_bf16(tmem + 128, umma_sdesc(s0 + kSsdOffC + k * 4096, 2048, 128),
                           umma_sdesc(s0 + kSsdOffH + k * 256, 128, 2048), id_off, k);
 #pragma unroll
-            for (int k = 0; k < kSsdQ / 16; ++k)
-                umma_bf16(tmem + 192, umma_sdesc(s0 + kSsdOffB + k * 256, 128, 2048),
-                          umma_sdesc(s0 + kSsdOffXw + k * 256, 128, 2048), id_s, k);
+            for (int k = 0; k < kSsdN / 16; ++k)
+                umma_bf16(tmem, umma_sdesc(s0 + kSsdOffC + k * 4096, 2048, 128),
+                          umma_sdesc(s0 + kSsdOffB + k * 4096, 2048, 128), id_g, k);
             umma_commit(bar1);
         }
-        if (ssd_wait_failed(bar1, parity)) {
+        if (ssd_wait_failed(bar_s, parity)) {
             failed = true;
             break;
         }
-
-        // ---- next chunk's B; then the gate tile z (128 x 64) by TMA into the Xw
-        // buffer, which MMA 4 no longer reads; both land while the masked
-        // matrix and MMA 2 run.
-        if (tid == 0 && more) {
-            mbar_arrive_expect_tx(bar_ld, kSsdTileBytes);
-            tma_load_tile(s0 + kSsdOffB, &tm_B, l0 + kSsdQ, g, b, bar_ld);
-        }
+        // ---- the gate tile z (128 x 64) by TMA into the Xw buffer, which MMA 4
+        // no longer reads; it lands while the masked matrix and MMA 2 run.
         if (tid == 0 && has_z) {
             mbar_arrive_expect_tx(bar_z, 16384);
             tma_load_tile(s0 + kSsdOffXw, &tm_z, l0, h, b, bar_z);
         }
-
-        // ---- state: H = 2^(c_Q) H + S (row n = tid), then its bf16 copy for
-        // the next chunk's MMA 3.
+        // ---- state: H = 2^(c_Q) H + S (row n = tid), in registers while MMA 3
+        // and 1 run; its bf16 copy for the next chunk's MMA 3 waits for them.
         {
             const float dq = ex2_approx(cQ);
             float s_lo[32], s_hi[32];
@@ -373,8 +371,18 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
                 H[k] = fmaf(dq, H[k], s_lo[k]);
                 H[32 + k] = fmaf(dq, H[32 + k], s_hi[k]);
             }
-            ssd_store_state(smem, tid, H);
         }
+        if (ssd_wait_failed(bar1, parity)) {
+            failed = true;
+            break;
+        }
+
+        // ---- next chunk's B (MMA 1 and 4 are done with it); the state's bf16 copy.
+        if (tid == 0 && more) {
+            mbar_arrive_expect_tx(bar_ld, kSsdTileBytes);
+            tma_load_tile(s0 + kSsdOffB, &tm_B, l0 + kSsdQ, g, b, bar_ld);
+        }
+        ssd_store_state(smem, tid, H);
 
         // ---- Gm_ij = G_ij 2^(c_i - e_j) for j <= i (row i = tid), over C's tile.
         // Warp w holds rows [32w, 32w + 32): quarters of columns below w are
