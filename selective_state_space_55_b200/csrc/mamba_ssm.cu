@@ -1117,21 +1117,22 @@ namespace {
 
 // Map over a row-major bf16 (batch, L, heads_or_groups, width) tensor whose one
 // box is a whole 128-row operand tile of the Mamba-2 layer kernel in its
-// shared-memory layout: dimensions (8 elements, L, width / 8 column blocks,
-// heads_or_groups, batch), box (8, 128, width / 8, 1, 1), so that shared
-// memory receives block kb of row r at kb * 2048 + r * 16.
+// shared-memory layout: dimensions (64 elements, L, width / 64 column halves,
+// heads_or_groups, batch), box (64, 128, width / 64, 1, 1), 128-byte swizzle,
+// so that shared memory receives each 64-column half as 128 rows of 128 bytes
+// in 1024-byte swizzle atoms, halves 16 KB apart.
 bool encode_map_ssd(CUtensorMap* map, const void* base, uint64_t width, uint64_t heads,
                     uint64_t L, uint64_t batch) {
     auto encode = tensor_map_encoder();
     if (encode == nullptr) return false;
     const uint64_t row = heads * width * 2;                 // bytes between tokens
-    const cuuint64_t dims[5] = {8, L, width / 8, heads, batch};
-    const cuuint64_t strides[4] = {row, 16, width * 2, row * L};
-    const cuuint32_t box[5] = {8, (cuuint32_t)kSsdQ, (cuuint32_t)(width / 8), 1, 1};
+    const cuuint64_t dims[5] = {64, L, width / 64, heads, batch};
+    const cuuint64_t strides[4] = {row, 128, width * 2, row * L};
+    const cuuint32_t box[5] = {64, (cuuint32_t)kSsdQ, (cuuint32_t)(width / 64), 1, 1};
     const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
     const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base),
                               dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }

@@ -42,8 +42,11 @@ constexpr int kSsdQ = 128;         // chunk length
 constexpr int kSsdThreads = 128;   // one thread per TMEM lane
 constexpr int kSsdTmemCols = 256;  // G [0,128) (then Ydiag [0,64)), Yoff [128,192), S [192,256)
 
-// Shared-memory map (bytes).  sC holds C and later Gm; all operand tiles use
-// offset(row, k) = (k / 8) * 2048 + row * 16 + (k % 8) * 2 for 128 rows.
+// Shared-memory map (bytes).  sC holds C and later Gm.  Every operand tile is
+// 128 rows in the 128-byte-swizzle layout of the tensor cores: each group of
+// 64 columns ("half") is 128 rows of 128 bytes, 8 rows to a 1024-byte atom,
+// and the 16-byte chunk c of row r sits at chunk position c ^ (r % 8); halves
+// are 16 KB apart.  ssd_sw128 gives the byte offset.
 constexpr int kSsdOffC = 0;          // 128 x 128 bf16: C (rows i, k = n), then Gm (rows i, k = j)
 constexpr int kSsdOffB = 32768;      // 128 x 128 bf16: B (rows j, k = n)
 constexpr int kSsdOffX = 65536;      // 128 x 64 bf16: x (rows j, k = p)
@@ -88,6 +91,21 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N, bool a_mn, 
 __device__ __forceinline__ uint64_t umma_sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
     return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
            ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+
+// The same with the 128-byte swizzle (layout type 2).  K-major: rows 128 bytes
+// of K, 8-row groups `sbo` = 1024 bytes apart, `lbo` unused (16).  MN-major:
+// 64 M/N elements per 128-byte row, K rows in 8-row groups `sbo` apart, the
+// next 64 M/N elements `lbo` apart.
+__device__ __forceinline__ uint64_t umma_sdesc_sw128(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+    return umma_sdesc(addr, lbo, sbo) | (2ull << 61);
+}
+
+// Byte offset of 16-byte chunk `chunk` (0..15 over both halves) of row `row`
+// in a 128-row swizzled tile.
+__device__ __forceinline__ uint32_t ssd_sw128(int row, int chunk) {
+    return (uint32_t)((chunk >> 3) * 16384 + (row >> 3) * 1024 + (row & 7) * 128 +
+                      (((chunk & 7) ^ (row & 7)) << 4));
 }
 
 __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
@@ -146,11 +164,11 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(r[k]);
 }
 
-// 5-D tiled TMA copies of one whole operand tile.  Each map is (8 elements,
-// L, column blocks, heads or groups, batch) with the box (8, 128, all
-// blocks, 1, 1): shared memory gets column block kb of row r at
-// kb * 2048 + r * 16.  Rows past the end of the sequence are filled with
-// zeros on load and dropped on store.
+// 5-D tiled TMA copies of one whole operand tile.  Each map is (64 elements,
+// L, column halves, heads or groups, batch) with the box (64, 128, all
+// halves, 1, 1) and the 128-byte swizzle, which writes the tile in exactly
+// the layout ssd_sw128 describes.  Rows past the end of the sequence are
+// filled with zeros on load and dropped on store.
 __device__ __forceinline__ void tma_load_tile(uint32_t dst, const CUtensorMap* map, int l0,
                                               int head, int batch, uint32_t bar) {
     asm volatile(
@@ -187,14 +205,14 @@ __device__ __forceinline__ void tmem_ld32x2(uint32_t ta, uint32_t tb, float (&a)
     }
 }
 
-// The state H of this thread's row n as bf16 into sH: offset (p / 8) * 2048 + n * 16.
+// The state H of this thread's row n as bf16 into sH (row n, 64 columns p).
 __device__ __forceinline__ void ssd_store_state(unsigned char* smem, int n, const float (&H)[kSsdP]) {
 #pragma unroll
     for (int q = 0; q < kSsdP / 8; ++q) {
         float f[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) f[k] = H[q * 8 + k];
-        *reinterpret_cast<uint4*>(smem + kSsdOffH + q * 2048 + n * 16) = pack16(f);
+        *reinterpret_cast<uint4*>(smem + kSsdOffH + ssd_sw128(n, q)) = pack16(f);
     }
 }
 
@@ -262,6 +280,9 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
 
     const int64_t nchunks = (L + kSsdQ - 1) / kSsdQ;
     bool failed = false;
+    // K-major operand, K step k of 16 columns: 32 bytes along the swizzled
+    // 128-byte rows, the second 64 columns one half (16 KB) further.
+    auto kmaj = [](int k) -> uint32_t { return (uint32_t)((k >> 2) * 16384 + (k & 3) * 32); };
     // dt of this thread's token in the next chunk, loaded one chunk ahead.
     auto load_dt = [&](int64_t l) -> float {
         return l < L ? __bfloat162float(p.dt[((int64_t)b * L + l) * p.nheads + h]) : 0.0f;
@@ -317,7 +338,7 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
             const float w = ex2_approx(cQ - sE[tid]);
 #pragma unroll
             for (int pb = 0; pb < kSsdP / 8; ++pb) {
-                const uint32_t off = (uint32_t)(pb * 2048 + tid * 16);
+                const uint32_t off = ssd_sw128(tid, pb);
                 float f[8];
                 unpack16(*reinterpret_cast<const uint4*>(smem + kSsdOffX + off), f);
 #pragma unroll
@@ -337,17 +358,17 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
             constexpr uint32_t id_s = umma_idesc_bf16(128, 64, true, true);
 #pragma unroll
             for (int k = 0; k < kSsdQ / 16; ++k)
-                umma_bf16(tmem + 192, umma_sdesc(s0 + kSsdOffB + k * 256, 128, 2048),
-                          umma_sdesc(s0 + kSsdOffXw + k * 256, 128, 2048), id_s, k);
+                umma_bf16(tmem + 192, umma_sdesc_sw128(s0 + kSsdOffB + k * 2048, 16384, 1024),
+                          umma_sdesc_sw128(s0 + kSsdOffXw + k * 2048, 16384, 1024), id_s, k);
             umma_commit(bar_s);
 #pragma unroll
             for (int k = 0; k < kSsdN / 16; ++k)
-                umma_bf16(tmem + 128, umma_sdesc(s0 + kSsdOffC + k * 4096, 2048, 128),
-                          umma_sdesc(s0 + kSsdOffH + k * 256, 128, 2048), id_off, k);
+                umma_bf16(tmem + 128, umma_sdesc_sw128(s0 + kSsdOffC + kmaj(k), 16, 1024),
+                          umma_sdesc_sw128(s0 + kSsdOffH + k * 2048, 16384, 1024), id_off, k);
 #pragma unroll
             for (int k = 0; k < kSsdN / 16; ++k)
-                umma_bf16(tmem, umma_sdesc(s0 + kSsdOffC + k * 4096, 2048, 128),
-                          umma_sdesc(s0 + kSsdOffB + k * 4096, 2048, 128), id_g, k);
+                umma_bf16(tmem, umma_sdesc_sw128(s0 + kSsdOffC + kmaj(k), 16, 1024),
+                          umma_sdesc_sw128(s0 + kSsdOffB + kmaj(k), 16, 1024), id_g, k);
             umma_commit(bar1);
         }
         if (ssd_wait_failed(bar_s, parity)) {
@@ -396,7 +417,7 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
                 const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
                 for (int q = 0; q < 8; ++q)
-                    *reinterpret_cast<uint4*>(smem + kSsdOffC + (qa * 4 + q) * 2048 + tid * 16) = zero;
+                    *reinterpret_cast<uint4*>(smem + kSsdOffC + ssd_sw128(tid, qa * 4 + q)) = zero;
                 continue;
             }
             float gv[2][32];
@@ -408,7 +429,7 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
                     const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
-                        *reinterpret_cast<uint4*>(smem + kSsdOffC + (quarter * 4 + q) * 2048 + tid * 16) = zero;
+                        *reinterpret_cast<uint4*>(smem + kSsdOffC + ssd_sw128(tid, quarter * 4 + q)) = zero;
                     continue;
                 }
                 const bool diag = quarter == warp;   // D_h x_i enters as Gm_ii += D_h
@@ -424,7 +445,7 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
                         const float v = gv[half][q * 8 + k] * ex2_approx(ci - ej[k]);
                         f[k] = (!diag || j0 + k < tid) ? v : (j0 + k == tid ? v + Dh : 0.0f);
                     }
-                    *reinterpret_cast<uint4*>(smem + kSsdOffC + (j0 / 8) * 2048 + tid * 16) = pack16(f);
+                    *reinterpret_cast<uint4*>(smem + kSsdOffC + ssd_sw128(tid, j0 / 8)) = pack16(f);
                 }
             }
         }
@@ -438,8 +459,8 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
             constexpr uint32_t id_y = umma_idesc_bf16(128, 64, false, true);
 #pragma unroll
             for (int k = 0; k < kSsdQ / 16; ++k)
-                umma_bf16(tmem, umma_sdesc(s0 + kSsdOffC + k * 4096, 2048, 128),
-                          umma_sdesc(s0 + kSsdOffX + k * 256, 128, 2048), id_y, k);
+                umma_bf16(tmem, umma_sdesc_sw128(s0 + kSsdOffC + kmaj(k), 16, 1024),
+                          umma_sdesc_sw128(s0 + kSsdOffX + k * 2048, 16384, 1024), id_y, k);
             umma_commit(bar2);
         }
         if (ssd_wait_failed(bar2, parity)) {
@@ -467,7 +488,7 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     const int pb = half * 4 + q;
-                    const uint32_t off = (uint32_t)(pb * 2048 + tid * 16);
+                    const uint32_t off = ssd_sw128(tid, pb);
                     float f[8];
 #pragma unroll
                     for (int k = 0; k < 8; ++k) f[k] = fmaf(sc, yo[q * 8 + k], yd[q * 8 + k]);
