@@ -728,6 +728,7 @@ def bench_ssd(args, rank, world, local):
     flops = R.ssd_chunk_flops(c.batch, c.seqlen, c.nheads, c.headdim, c.dstate)
     gbs = nbytes / (ms * 1e-3) / 1e9
     tfs = flops / (ms * 1e-3) / 1e12
+    traffic = recorded_traffic("ssd_chunk_scan_kernel", sources_digest())
     value = world * c.elements / (ms * 1e-3) / 1e9
     if rank == 0:
         line = {
@@ -739,9 +740,11 @@ def bench_ssd(args, rank, world, local):
                                    f"N={c.dstate}, groups={c.ngroups}, chunk 128, bf16, gate/D/bias, "
                                    "final state)",
                        "inputs_exceed_l2": nbytes > 126e6},
-            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
-                         "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
-                         "traffic": None, "bytes_per_step": nbytes},
+            "roofline": {"bound": "hbm", "kernel": "ssd_chunk_scan_kernel", "achieved": round(gbs, 1),
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(gbs / peaks["hbm_gbs"], 4),
+                         "traffic": traffic if c.batch == 16 else None,
+                         "bytes_per_step": nbytes},
             "tensor": {"issued_tflops": round(tfs, 1), "peak": peaks["bf16_tflops"],
                        "frac": round(tfs / peaks["bf16_tflops"], 4), "flops_per_step": flops},
             "gpu_launches": K,
