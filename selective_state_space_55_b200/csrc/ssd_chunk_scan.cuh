@@ -205,6 +205,13 @@ __device__ __forceinline__ void tmem_ld32x2(uint32_t ta, uint32_t tb, float (&a)
     }
 }
 
+// 1/x on the MUFU pipe (rcp.approx, flush-to-zero); 0 for x = +inf.
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // The state H of this thread's row n as bf16 into sH (row n, 64 columns p).
 __device__ __forceinline__ void ssd_store_state(unsigned char* smem, int n, const float (&H)[kSsdP]) {
 #pragma unroll
@@ -324,7 +331,8 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
         for (int w = 0; w < warp; ++w) pre += sTot[w];
         const float ci = a + pre;
         const float cQ = (sTot[0] + sTot[1]) + (sTot[2] + sTot[3]);
-        sE[tid] = ci - lg2_approx(delta);   // +inf for Delta = 0
+        const float e_own = ci - lg2_approx(delta);   // +inf for Delta = 0
+        sE[tid] = -e_own;                              // stored negated: c_i - e_j is an add
         // The previous chunk's output store must have read the staging tile
         // (rewritten by the Xw pass below).
         if (tid == 0) bulk_wait_read<0>();
@@ -335,14 +343,19 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
 
         // ---- Xw_j = 2^(c_Q - e_j) x_j = 2^(c_Q - c_j) Delta_j x_j (row j = tid).
         {
-            const float w = ex2_approx(cQ - sE[tid]);
+            const float w = ex2_approx(cQ - e_own);
+            const float2 w2 = make_float2(w, w);
 #pragma unroll
             for (int pb = 0; pb < kSsdP / 8; ++pb) {
                 const uint32_t off = ssd_sw128(tid, pb);
                 float f[8];
                 unpack16(*reinterpret_cast<const uint4*>(smem + kSsdOffX + off), f);
 #pragma unroll
-                for (int k = 0; k < 8; ++k) f[k] *= w;
+                for (int k = 0; k < 8; k += 2) {
+                    const float2 r = __fmul2_rn(make_float2(f[k], f[k + 1]), w2);
+                    f[k] = r.x;
+                    f[k + 1] = r.y;
+                }
                 *reinterpret_cast<uint4*>(smem + kSsdOffXw + off) = pack16(f);
             }
         }
@@ -387,10 +400,16 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
             const float dq = ex2_approx(cQ);
             float s_lo[32], s_hi[32];
             tmem_ld32x2(tlane + 192, tlane + 224, s_lo, s_hi);
+            const float2 dq2 = make_float2(dq, dq);
 #pragma unroll
-            for (int k = 0; k < 32; ++k) {
-                H[k] = fmaf(dq, H[k], s_lo[k]);
-                H[32 + k] = fmaf(dq, H[32 + k], s_hi[k]);
+            for (int k = 0; k < 32; k += 2) {
+                const float2 lo = __ffma2_rn(dq2, make_float2(H[k], H[k + 1]), make_float2(s_lo[k], s_lo[k + 1]));
+                const float2 hi = __ffma2_rn(dq2, make_float2(H[32 + k], H[33 + k]),
+                                             make_float2(s_hi[k], s_hi[k + 1]));
+                H[k] = lo.x;
+                H[k + 1] = lo.y;
+                H[32 + k] = hi.x;
+                H[33 + k] = hi.y;
             }
         }
         if (ssd_wait_failed(bar1, parity)) {
@@ -405,6 +424,7 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
         }
         ssd_store_state(smem, tid, H);
 
+        const float2 ci2 = make_float2(ci, ci);
         // ---- Gm_ij = G_ij 2^(c_i - e_j) for j <= i (row i = tid), over C's tile.
         // Warp w holds rows [32w, 32w + 32): quarters of columns below w are
         // entirely at or below the diagonal, quarter w straddles it, and the
@@ -438,12 +458,22 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
                     const int j0 = quarter * 32 + q * 8;
                     const float4 e0 = *reinterpret_cast<const float4*>(sE + j0);
                     const float4 e1 = *reinterpret_cast<const float4*>(sE + j0 + 4);
-                    const float ej[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
+                    const float2 ne[4] = {make_float2(e0.x, e0.y), make_float2(e0.z, e0.w),
+                                          make_float2(e1.x, e1.y), make_float2(e1.z, e1.w)};
                     float f[8];
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const float v = gv[half][q * 8 + k] * ex2_approx(ci - ej[k]);
-                        f[k] = (!diag || j0 + k < tid) ? v : (j0 + k == tid ? v + Dh : 0.0f);
+                    for (int k = 0; k < 8; k += 2) {
+                        const float2 arg = __fadd2_rn(ci2, ne[k / 2]);
+                        const float2 v = __fmul2_rn(
+                            make_float2(gv[half][q * 8 + k], gv[half][q * 8 + k + 1]),
+                            make_float2(ex2_approx(arg.x), ex2_approx(arg.y)));
+                        f[k] = v.x;
+                        f[k + 1] = v.y;
+                    }
+                    if (diag) {
+#pragma unroll
+                        for (int k = 0; k < 8; ++k)
+                            f[k] = j0 + k < tid ? f[k] : (j0 + k == tid ? f[k] + Dh : 0.0f);
                     }
                     *reinterpret_cast<uint4*>(smem + kSsdOffC + ssd_sw128(tid, j0 / 8)) = pack16(f);
                 }
@@ -481,6 +511,7 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
         // past the end dropped).
         {
             const float sc = ex2_approx(ci);
+            const float2 sc2 = make_float2(sc, sc);
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 float yd[32], yo[32];
@@ -491,12 +522,27 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
                     const uint32_t off = ssd_sw128(tid, pb);
                     float f[8];
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) f[k] = fmaf(sc, yo[q * 8 + k], yd[q * 8 + k]);
+                    for (int k = 0; k < 8; k += 2) {
+                        const float2 r = __ffma2_rn(sc2, make_float2(yo[q * 8 + k], yo[q * 8 + k + 1]),
+                                                    make_float2(yd[q * 8 + k], yd[q * 8 + k + 1]));
+                        f[k] = r.x;
+                        f[k + 1] = r.y;
+                    }
                     if (has_z) {
+                        // silu(z) = z / (1 + 2^(-z log2 e)), two lanes at a time
                         float zv[8];
                         unpack16(*reinterpret_cast<const uint4*>(smem + kSsdOffXw + off), zv);
 #pragma unroll
-                        for (int k = 0; k < 8; ++k) f[k] *= silu_f32(zv[k]);
+                        for (int k = 0; k < 8; k += 2) {
+                            const float2 z2 = make_float2(zv[k], zv[k + 1]);
+                            const float2 t = __fmul2_rn(z2, make_float2(-kLog2e, -kLog2e));
+                            const float2 d = __fadd2_rn(make_float2(ex2_approx(t.x), ex2_approx(t.y)),
+                                                        make_float2(1.0f, 1.0f));
+                            const float2 g2 = __fmul2_rn(z2, make_float2(rcp_approx(d.x), rcp_approx(d.y)));
+                            const float2 r = __fmul2_rn(make_float2(f[k], f[k + 1]), g2);
+                            f[k] = r.x;
+                            f[k + 1] = r.y;
+                        }
                     }
                     *reinterpret_cast<uint4*>(smem + kSsdOffXw + off) = pack16(f);
                 }
