@@ -393,52 +393,70 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
 #pragma unroll 1
             for (int q = 0; q < kNPad / 4; ++q) {
                 const int n0 = 4 * q;
+                // The four entries run as two fp32x2 pairs (packed FMA/FMUL,
+                // rounding identical to the scalar forms).
+                const float2 a2p[2] = {make_float2(a2[0], a2[1]), make_float2(a2[2], a2[3])};
+                const float2 a2l[2] = {__fmul2_rn(a2p[0], make_float2(kLn2, kLn2)),
+                                       __fmul2_rn(a2p[1], make_float2(kLn2, kLn2))};
                 // forward: the block's 8 states of entries n0..n0+3
-                float hq[kBwdSteps][4];
-                float h[4] = {ckv[0].x, ckv[0].y, ckv[0].z, ckv[0].w};
+                float2 hq[kBwdSteps][2];
+                float2 h2[2] = {make_float2(ckv[0].x, ckv[0].y), make_float2(ckv[0].z, ckv[0].w)};
 #pragma unroll
                 for (int t = 0; t < kBwdSteps; ++t) {
                     if (t < ns) {
                         const float4 Bq = *reinterpret_cast<const float4*>(&bcf[t][n0]);
                         const float4 Cq = *reinterpret_cast<const float4*>(&bcf[t][16 + n0]);
-                        const float bq[4] = {Bq.x, Bq.y, Bq.z, Bq.w};
-                        const float cq[4] = {Cq.x, Cq.y, Cq.z, Cq.w};
+                        const float2 bq[2] = {make_float2(Bq.x, Bq.y), make_float2(Bq.z, Bq.w)};
+                        const float2 cq[2] = {make_float2(Cq.x, Cq.y), make_float2(Cq.z, Cq.w)};
                         const float du = dt[t] * uu[t];
+                        const float2 dt2 = make_float2(dt[t], dt[t]), du2 = make_float2(du, du);
+                        float2 y2 = make_float2(0.0f, 0.0f);
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const float ab = bwd_exp2<kExact>(dt[t] * a2[i]);
-                            h[i] = fmaf(ab, h[i], du * bq[i]);
-                            hq[t][i] = h[i];
-                            y[t] = fmaf(cq[i], h[i], y[t]);
+                        for (int pr = 0; pr < 2; ++pr) {
+                            const float2 x2 = __fmul2_rn(dt2, a2p[pr]);
+                            const float2 ab = make_float2(bwd_exp2<kExact>(x2.x), bwd_exp2<kExact>(x2.y));
+                            h2[pr] = __ffma2_rn(ab, h2[pr], __fmul2_rn(du2, bq[pr]));
+                            hq[t][pr] = h2[pr];
+                            y2 = __ffma2_rn(cq[pr], h2[pr], y2);
                         }
+                        y[t] += y2.x + y2.y;
                     }
                 }
                 // reverse: the adjoint of entries n0..n0+3 over the block
-                float l4[4] = {lam[0], lam[1], lam[2], lam[3]};
+                float2 l2[2] = {make_float2(lam[0], lam[1]), make_float2(lam[2], lam[3])};
+                float2 dA2[2] = {make_float2(dA_acc[0], dA_acc[1]), make_float2(dA_acc[2], dA_acc[3])};
 #pragma unroll
                 for (int t = kBwdSteps - 1; t >= 0; --t) {
                     if (t < ns) {
                         const float4 Bq = *reinterpret_cast<const float4*>(&bcf[t][n0]);
                         const float4 Cq = *reinterpret_cast<const float4*>(&bcf[t][16 + n0]);
-                        const float bq[4] = {Bq.x, Bq.y, Bq.z, Bq.w};
-                        const float cq[4] = {Cq.x, Cq.y, Cq.z, Cq.w};
+                        const float2 bq[2] = {make_float2(Bq.x, Bq.y), make_float2(Bq.z, Bq.w)};
+                        const float2 cq[2] = {make_float2(Cq.x, Cq.y), make_float2(Cq.z, Cq.w)};
                         const float du = dt[t] * uu[t];
+                        const float2 dt2 = make_float2(dt[t], dt[t]), du2 = make_float2(du, du);
+                        const float2 ndu2 = make_float2(-du, -du), dy2 = make_float2(dy[t], dy[t]);
+                        const float2 uu2 = make_float2(uu[t], uu[t]);
                         float red[8];
-                        float s_dt = 0.0f, s_b = 0.0f;
+                        float2 s_dt2 = make_float2(0.0f, 0.0f), s_b2 = make_float2(0.0f, 0.0f);
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            l4[i] = fmaf(cq[i], dy[t], l4[i]);                 // lambda_t
-                            const float ab = bwd_exp2<kExact>(dt[t] * a2[i]);
-                            const float abh = fmaf(-du, bq[i], hq[t][i]);      // Abar_t h_t-1 = h_t - b_t
-                            red[i] = l4[i] * du;                                // dB
-                            red[4 + i] = dy[t] * hq[t][i];                      // dC
-                            s_dt = fmaf(l4[i], fmaf(a2[i] * kLn2, abh, bq[i] * uu[t]), s_dt);
-                            s_b = fmaf(l4[i], bq[i], s_b);
-                            dA_acc[i] = fmaf(l4[i] * dt[t], abh, dA_acc[i]);
-                            l4[i] *= ab;                                        // to h_t-1
+                        for (int pr = 0; pr < 2; ++pr) {
+                            l2[pr] = __ffma2_rn(cq[pr], dy2, l2[pr]);                    // lambda_t
+                            const float2 x2 = __fmul2_rn(dt2, a2p[pr]);
+                            const float2 ab = make_float2(bwd_exp2<kExact>(x2.x), bwd_exp2<kExact>(x2.y));
+                            const float2 abh = __ffma2_rn(ndu2, bq[pr], hq[t][pr]);      // Abar_t h_t-1
+                            const float2 rb = __fmul2_rn(l2[pr], du2);                    // dB
+                            const float2 rc = __fmul2_rn(dy2, hq[t][pr]);                 // dC
+                            red[2 * pr] = rb.x;
+                            red[2 * pr + 1] = rb.y;
+                            red[4 + 2 * pr] = rc.x;
+                            red[5 + 2 * pr] = rc.y;
+                            s_dt2 = __ffma2_rn(l2[pr], __ffma2_rn(a2l[pr], abh, __fmul2_rn(bq[pr], uu2)), s_dt2);
+                            s_b2 = __ffma2_rn(l2[pr], bq[pr], s_b2);
+                            dA2[pr] = __ffma2_rn(__fmul2_rn(l2[pr], dt2), abh, dA2[pr]);
+                            l2[pr] = __fmul2_rn(l2[pr], ab);                              // to h_t-1
                         }
-                        ddt[t] += s_dt;
-                        dlb[t] += s_b;
+                        ddt[t] += s_dt2.x + s_dt2.y;
+                        dlb[t] += s_b2.x + s_b2.y;
                         const float tot = warp_reduce8(red, lane);
                         const int idx = lane >> 2;                              // 0..7
                         const int n = n0 + (idx & 3);
@@ -448,6 +466,11 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
                         }
                     }
                 }
+                dA_acc[0] = dA2[0].x;
+                dA_acc[1] = dA2[0].y;
+                dA_acc[2] = dA2[1].x;
+                dA_acc[3] = dA2[1].y;
+                const float l4[4] = {l2[0].x, l2[0].y, l2[1].x, l2[1].y};
 #pragma unroll
                 for (int i = 0; i < 4; ++i) lam[i] = l4[i];
                 rotate_quarter(a2);
