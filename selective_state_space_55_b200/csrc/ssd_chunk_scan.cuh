@@ -21,9 +21,9 @@
 //   y_i   = Ydiag_i + 2^(c_i) Yoff_i,  out = y silu(z)
 //   H     = 2^(c_Q) H + S               (fp32, in registers)
 //
-// Operands are bf16 in shared memory in the no-swizzle canonical layout
-// ("core matrices" of 8 rows x 16 bytes); the products accumulate in fp32 in
-// tensor memory and are read back with tcgen05.ld.  One elected thread
+// Operands are bf16 in shared memory in the tensor cores' 128-byte-swizzle
+// layout (1024-byte atoms of 8 rows x 128 bytes); the products accumulate in
+// fp32 in tensor memory and are read back with tcgen05.ld.  One elected thread
 // issues the tcgen05.mma instructions and commits them to an mbarrier that
 // the CTA waits on (bounded).  Operand tiles arrive by TMA, one box per
 // tile, and the next chunk's tiles are requested as soon as this chunk's
@@ -52,7 +52,7 @@ constexpr int kSsdOffB = 32768;      // 128 x 128 bf16: B (rows j, k = n)
 constexpr int kSsdOffX = 65536;      // 128 x 64 bf16: x (rows j, k = p)
 constexpr int kSsdOffXw = 81920;     // 128 x 64 bf16: Xw (rows j, k = p)
 constexpr int kSsdOffH = 98304;      // 128 x 64 bf16: H (rows n, k = p)
-constexpr int kSsdOffE = 114688;     // 128 fp32: e_j = c_j - log2(Delta_j)
+constexpr int kSsdOffE = 114688;     // 128 fp32: -e_j, e_j = c_j - log2(Delta_j)
 constexpr int kSsdOffMisc = 115200;  // mbarriers (+0 products 1/3, +8 product 2, +16 tiles,
                                      // +24 gate, +40 product 4), the TMEM address (+32),
                                      // warp totals (+48)
@@ -141,27 +141,6 @@ __device__ __forceinline__ void tc_fence_before() {
 
 __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-
-// 32 consecutive fp32 columns of this thread's TMEM lane; the wait for the
-// load is in the same statement, so no use of the values can precede it.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-    uint32_t r[32];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-          "=r"(r[31])
-        : "r"(taddr)
-        : "memory");
-#pragma unroll
-    for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(r[k]);
 }
 
 // 5-D tiled TMA copies of one whole operand tile.  Each map is (64 elements,
