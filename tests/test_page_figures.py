@@ -78,3 +78,20 @@ def test_configs_shapes(name):
     assert x["B"].shape == (small.batch, small.dstate, small.seqlen)
     assert x["u"].dtype == c.io_dtype and x["B"].dtype == c.bc_dtype
     assert x["A"].dtype == torch.float32 and x["A"].shape == (small.dim, small.dstate)
+
+
+def test_mamba2_layer_byte_and_flop_counts():
+    """The Mamba-2 layer's algorithmic bytes and issued tensor FLOPs on the 2.7B
+    layer shape, counted by hand: per (token, head) x, z, out (64 bf16 each) and
+    dt (one bf16); per token B and C (128 bf16 each, one group); the final fp32
+    state of every head; per 128-token chunk and head four dense products."""
+    from selective_state_space_55_b200 import roofline as R
+    batch, L, H, P, N, Q = 16, 2048, 80, 64, 128, 128
+    tokens = batch * L
+    by_hand = tokens * H * (3 * P * 2 + 2) + tokens * 2 * N * 2 + batch * H * P * N * 4
+    assert by_hand == 1_070_596_096
+    assert R.ssd_bytes(batch, L, H, P, 1, N) == by_hand
+    chunks = L // Q
+    products = Q * Q * N + Q * Q * P + N * Q * P + Q * N * P   # C B^T, Gm x, B^T Xw, C H^T
+    assert R.ssd_chunk_flops(batch, L, H, P, N, Q) == 2 * products * batch * H * chunks
+    assert R.ssd_chunk_flops(batch, L, H, P, N, Q) / (tokens * H * P) == 1280
