@@ -477,7 +477,9 @@ def ssd_chunk_scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_softplus
     x, z: (batch, L, nheads, 64) bf16; dt: (batch, L, nheads) bf16; A, D,
     dt_bias: (nheads,) fp32; B, C: (batch, L, ngroups, 128) bf16;
     initial_state: (batch, nheads, 64, 128) fp32 or None.  Returns out (like
-    x), or (out, final_state) when ``return_final_state``.
+    x), or (out, final_state) when ``return_final_state`` is set or a
+    ``final_state`` buffer is passed.  Delta must be non-negative (softplus on,
+    or dt + dt_bias >= 0 with it off).
     """
     batch, L, nheads, headdim = x.shape
     ngroups, dstate = B.shape[2], B.shape[3]

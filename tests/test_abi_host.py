@@ -277,3 +277,14 @@ def test_ssd_rejects_bad_arguments_before_launch(lib):
     assert _ssd(lib, _ssd_dims(), x=ctypes.c_void_p(0x10008)) == -3  # 16-byte rows
     assert _ssd(lib, _ssd_dims(), dt=ctypes.c_void_p(0x10001)) == -3
     assert _ssd(lib, _ssd_dims(batch=0)) == 0                         # nothing to do
+
+
+def test_ssd_binding_checks_tensors_on_the_host():
+    """The Python binding refuses host tensors and wrong shapes or dtypes before
+    calling the library (no GPU needed)."""
+    x = torch.zeros(1, 8, 2, 64, dtype=torch.bfloat16)
+    dt = torch.zeros(1, 8, 2, dtype=torch.bfloat16)
+    A = torch.zeros(2)
+    B = torch.zeros(1, 8, 1, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        ops.ssd_chunk_scan_fwd(x, dt, A, B, B)
