@@ -330,6 +330,32 @@ def cpu_baseline(w: Workload, target_s: float) -> dict:
                       "of oracle time"}
 
 
+def ssd_cpu_baseline(cfg, x: dict, target_s: float) -> dict:
+    """The float64 oracle on the host cores over the Mamba-2 layer workload:
+    batch rows in turn (all heads of a row per call), until about
+    ``target_s`` seconds of CPU work or the whole batch."""
+    from oracle import oracle
+    ref = oracle.default()
+    done, t_total, rows = 0, 0.0, 0
+    for b in range(cfg.batch):
+        sl = lambda t: None if t is None else t[b:b + 1].cpu()  # noqa: E731
+        t0 = time.perf_counter()
+        ref.ssd_scan(sl(x["x"]), sl(x["dt"]), x["A"].cpu(), sl(x["B"]), sl(x["C"]),
+                     D=None if x["D"] is None else x["D"].cpu(), z=sl(x["z"]),
+                     dt_bias=None if x["dt_bias"] is None else x["dt_bias"].cpu(),
+                     initial_state=sl(x["initial_state"]))
+        t_total += time.perf_counter() - t0
+        done += cfg.seqlen * cfg.nheads * cfg.headdim
+        rows += 1
+        if t_total >= target_s:
+            break
+    return {"value": done / t_total / 1e9, "unit": "Gelem/s", "cores": ref.num_threads(),
+            "kind": "oracle",
+            "sample": f"{rows} of {cfg.batch} batch rows of {cfg.name} ({cfg.seqlen} tokens x "
+                      f"{cfg.nheads} heads x {cfg.headdim}; {done} elements) in {t_total:.1f} s "
+                      "of oracle time"}
+
+
 # ----------------------------------------------------------------- distributed
 
 _WORLD = 1
@@ -749,6 +775,8 @@ def bench_ssd(args, rank, world, local):
                        "frac": round(tfs / peaks["bf16_tflops"], 4), "flops_per_step": flops},
             "gpu_launches": K,
             "clocks": sampler.summary(t0, t1),
+            "cpu_baseline": (None if args.no_cpu_baseline
+                             else ssd_cpu_baseline(c, x, args.cpu_seconds)),
             "partial_case": {"only": "ssd", "scan_batch": args.scan_batch,
                              "note": "measurement of the Mamba-2 layer, not the benchmark workload"},
         }
