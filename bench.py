@@ -330,6 +330,29 @@ def cpu_baseline(w: Workload, target_s: float) -> dict:
                       "of oracle time"}
 
 
+def bwd_cpu_baseline(cfg, x: dict, dout, target_s: float) -> dict:
+    """The float64 oracle's backward pass on the host over whole batch rows of
+    the workload, until about ``target_s`` seconds of CPU work."""
+    from oracle import oracle
+    ref = oracle.default()
+    done, t_total, rows = 0, 0.0, 0
+    for b in range(cfg.batch):
+        sl = lambda t: None if t is None else t[b:b + 1].cpu()  # noqa: E731
+        t0 = time.perf_counter()
+        ref.selective_scan_bwd(sl(x["u"]), sl(x["delta"]), x["A"].cpu(), sl(x["B"]), sl(x["C"]),
+                               sl(dout), D=x["D"].cpu(), z=sl(x["z"]),
+                               delta_bias=x["delta_bias"].cpu())
+        t_total += time.perf_counter() - t0
+        done += cfg.dim * cfg.seqlen
+        rows += 1
+        if t_total >= target_s:
+            break
+    return {"value": done / t_total / 1e9, "unit": "Gelem/s", "cores": 1, "kind": "oracle",
+            "sample": f"{rows} of {cfg.batch} batch rows of {cfg.name} backward ({cfg.dim} "
+                      f"channels x L={cfg.seqlen}; {done} elements) in {t_total:.1f} s of oracle "
+                      "time (the oracle's backward runs its chains in order)"}
+
+
 def ssd_cpu_baseline(cfg, x: dict, target_s: float) -> dict:
     """The float64 oracle on the host cores over the Mamba-2 layer workload:
     batch rows in turn (all heads of a row per call), until about
@@ -698,6 +721,8 @@ def bench_bwd(args, rank, world, local):
                          "frac": round(value / world / peak, 4), "traffic": None},
             "gpu_launches": K * 2,
             "clocks": sampler.summary(t0, t1),
+            "cpu_baseline": (None if args.no_cpu_baseline
+                             else bwd_cpu_baseline(c, x, dout, args.cpu_seconds)),
             "partial_case": {"only": "bwd", "scan_batch": args.scan_batch,
                              "note": "measurement of the backward pass, not the benchmark workload"},
         }
