@@ -717,8 +717,11 @@ def bench_bwd(args, rank, world, local):
                                    "bf16, gate/D/bias, checkpoint pass + adjoint)",
                        "checkpoint_bytes": ws.numel()},
             "roofline": {"bound": "alu", "pipe": f"MUFU ({mufu} per element, both launches)",
+                         "kernel": "selective_scan_bwd_kernel",
                          "achieved": round(value / world, 2), "peak": round(peak, 2), "unit": "Gelem/s",
-                         "frac": round(value / world / peak, 4), "traffic": None},
+                         "frac": round(value / world / peak, 4),
+                         "traffic": (recorded_traffic("selective_scan_bwd_kernel", sources_digest())
+                                     if c.batch == 16 else None)},
             "gpu_launches": K * 2,
             "clocks": sampler.summary(t0, t1),
             "cpu_baseline": (None if args.no_cpu_baseline
