@@ -46,6 +46,7 @@ SCAN_WORKLOAD = "mamba_2p8b_layer"
 SCAN_VARIANTS = ("euler", "zoh", "start_state")
 PROFILES = ROOT / "profiles"
 HBM_FALLBACK_GBS = 6650.0
+HBM_NOMINAL_GBS = 8000.0
 SM_MAX_MHZ_FALLBACK = 1965.0
 BF16_TFLOPS_FALLBACK = 1590.0
 
@@ -103,7 +104,7 @@ class ClockSampler:
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
                0x100: "display_clock_setting"}
 
-    def __init__(self, local_rank: int, period_s: float = 0.02):
+    def __init__(self, local_rank: int, period_s: float = 0.005):
         self.period = period_s
         self.samples: list[tuple[float, float, int]] = []
         self.max_mhz = None
@@ -295,39 +296,163 @@ def run_e2e(w: Workload, steps: int, warmup: int, rows: int = 0) -> dict:
     torch.cuda.synchronize()
     ms = max_over_ranks(s.elapsed_time(e))
     chunk_rows = rows if rows > 0 else max(1, (c.batch + 7) // 8)
-    return {"ms_total": ms, "steps": steps, "h2d": h2d, "d2h": d2h, "rows": chunk_rows}
+    pcie = pinned_copy_rates(host["u"], out_h)
+    return {"ms_total": ms, "steps": steps, "h2d": h2d, "d2h": d2h, "rows": chunk_rows,
+            "pcie": pcie}
+
+
+def pinned_copy_rates(src_h: torch.Tensor, dst_h: torch.Tensor, reps: int = 5) -> dict:
+    """Host-to-device and device-to-host copy rates (GB/s) of pinned host
+    buffers, one cudaMemcpyAsync per copy on the current stream, timed with
+    CUDA events: each direction alone, then both at once on two streams (the
+    way the host-buffer scan overlaps them)."""
+    dev_in = torch.empty(src_h.shape, dtype=src_h.dtype, device="cuda")
+    dev_out = torch.empty(dst_h.shape, dtype=dst_h.dtype, device="cuda")
+    nin = src_h.numel() * src_h.element_size()
+    nout = dst_h.numel() * dst_h.element_size()
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps * 1e-3
+
+    t_in = timed(lambda: dev_in.copy_(src_h, non_blocking=True))
+    t_out = timed(lambda: dst_h.copy_(dev_out, non_blocking=True))
+    side = torch.cuda.Stream()
+
+    def both():
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            dst_h.copy_(dev_out, non_blocking=True)
+        dev_in.copy_(src_h, non_blocking=True)
+        torch.cuda.current_stream().wait_stream(side)
+
+    t_both = timed(both)
+    return {"h2d_gbs": round(nin / t_in / 1e9, 2), "d2h_gbs": round(nout / t_out / 1e9, 2),
+            "both_directions_s": t_both, "h2d_bytes": nin, "d2h_bytes": nout,
+            "h2d_gbs_while_d2h": round(nin / t_both / 1e9, 2)}
+
+
+def _f64_block(x: dict, h0, b: int, d0: int, S: int, P: int) -> dict:
+    """Float64 host copies of one sample block of a scan workload: batch row b,
+    channels [d0, d0 + S), the first P time steps."""
+    def cut(t):
+        return None if t is None else t[b:b + 1, d0:d0 + S, :P].double().cpu().numpy().copy()
+    return dict(u=cut(x["u"]), delta=cut(x["delta"]), z=cut(x["z"]),
+                B=x["B"][b:b + 1, :, :P].double().cpu().numpy().copy(),
+                C=x["C"][b:b + 1, :, :P].double().cpu().numpy().copy(),
+                A=x["A"][d0:d0 + S].double().cpu().numpy().copy(),
+                D=None if x["D"] is None else x["D"][d0:d0 + S].double().cpu().numpy().copy(),
+                delta_bias=(None if x["delta_bias"] is None
+                            else x["delta_bias"][d0:d0 + S].double().cpu().numpy().copy()),
+                initial_state=None if h0 is None else h0[b:b + 1, d0:d0 + S].double().cpu().numpy().copy())
+
+
+def _time_oracle_scan(ref, blocks: list, threads: int, target_s: float, zoh: bool):
+    """Runs the oracle's scan over the sample blocks in turn (repeating them)
+    with ``threads`` OpenMP threads until about ``target_s`` seconds; returns
+    (elements, seconds, calls).  Inputs are float64 already, so only the
+    oracle's own work is timed."""
+    ref.set_num_threads(threads)
+    done, t_total, calls = 0, 0.0, 0
+    while True:
+        for blk in blocks:
+            t0 = time.perf_counter()
+            ref.selective_scan(blk["u"], blk["delta"], blk["A"], blk["B"], blk["C"], D=blk["D"],
+                               z=blk["z"], delta_bias=blk["delta_bias"], softplus=True, zoh=zoh,
+                               initial_state=blk["initial_state"])
+            t_total += time.perf_counter() - t0
+            done += blk["u"].size
+            calls += 1
+            if t_total >= target_s:
+                return done, t_total, calls
 
 
 def cpu_baseline(w: Workload, target_s: float) -> dict:
-    """The float64 oracle on the host cores over the same workload: batch rows
-    in turn, repeated until about ``target_s`` seconds of CPU work."""
+    """The float64 oracle on the host cores over the same workload, on all
+    cores and on one core, each for about ``target_s`` / 2 seconds.
+
+    Sample blocks are (batch row, channel block, all L steps): two batch rows
+    with all their channels for the layer shapes; for the million-token shape,
+    two blocks of 32 channels (at least two per thread) over the whole
+    sequence.  The one-core sample is one block of at most 2^21 elements.  The
+    chains are independent, so elements per second over a sample are the rate
+    over the whole workload."""
     from oracle import oracle
     ref = oracle.default()
-    x = w.x
     c = w.cfg
-    rows = []
-    for b in range(c.batch):
-        sl = lambda t: None if t is None else t[b:b + 1].cpu()  # noqa: E731
-        rows.append((sl(x["u"]), sl(x["delta"]), sl(x["z"]), x["B"][b:b + 1].cpu(),
-                     x["C"][b:b + 1].cpu(), sl(w.h0)))
-    A, D, bias = x["A"].cpu(), x["D"].cpu(), x["delta_bias"].cpu()
     zoh = w.variant == "zoh"
-    done, t_total, passes = 0, 0.0, 0
-    while True:                      # whole passes over the workload
-        for u, delta, z, B, C, h0 in rows:
+    all_threads = ref.num_threads()
+    L = c.seqlen
+    S_all = min(c.dim, max((1 << 25) // L, 2 * all_threads))
+    S_one = max(1, min(c.dim, (1 << 21) // L))
+    half = target_s / 2
+    # two blocks: batch rows 0 and 1 (or two channel blocks of row 0)
+    second = (1, 0) if c.batch > 1 else (0, S_all if 2 * S_all <= c.dim else 0)
+    blocks_all = [_f64_block(w.x, w.h0, 0, 0, S_all, L),
+                  _f64_block(w.x, w.h0, second[0], second[1], S_all, L)]
+    blocks_one = [_f64_block(w.x, w.h0, 0, 0, S_one, L)]
+    n_all, t_all, k_all = _time_oracle_scan(ref, blocks_all, all_threads, half, zoh)
+    n_one, t_one, k_one = _time_oracle_scan(ref, blocks_one, 1, half, zoh)
+    ref.set_num_threads(all_threads)
+    v_all, v_one = n_all / t_all / 1e9, n_one / t_one / 1e9
+    return {"value": v_all, "unit": "Gelem/s", "cores": all_threads, "kind": "oracle",
+            "sample": f"{k_all} oracle calls over blocks of {c.name} (batch row x {S_all} "
+                      f"channels x all L={L} steps; {n_all} elements) in {t_all:.1f} s on "
+                      f"{all_threads} threads",
+            "value_cores_all": v_all, "cores_all": all_threads,
+            "value_cores_1": v_one, "cores_1": 1,
+            "sample_cores_1": f"{k_one} oracle calls over {S_one} channels x L={L} of batch row 0 "
+                              f"({n_one} elements) in {t_one:.1f} s on 1 thread",
+            "host_cpu_count": os.cpu_count()}
+
+
+def decode_cpu_baseline(w: Workload, target_s: float) -> dict | None:
+    """The float64 update oracle on one token step of the decode workload:
+    updates of one layer's state (batch 128 x 4096 x 16) repeated, on all
+    cores and on one core (a 1/16 slice of the batch, scaled), each for about
+    ``target_s`` / 2 seconds; reported per 48-layer token step."""
+    if not w.layers:
+        return None
+    from oracle import oracle
+    ref = oracle.default()
+    d = w.dcfg
+    lay, tok = w.layers[0], w.toks[0]
+    f = lambda t: t.double().cpu().numpy().copy()  # noqa: E731
+    args = dict(state=f(lay["state"]), x=f(tok["x"]), dt=f(tok["dt"]), A=f(lay["A"]), B=f(tok["B"]),
+                C=f(tok["C"]), D=f(lay["D"]), z=f(tok["z"]), dt_bias=f(lay["dt_bias"]))
+    rows1 = max(1, d.batch // 16)
+    one = {k: (v[:rows1].copy() if k in ("state", "x", "dt", "B", "C", "z") else v)
+           for k, v in args.items()}
+
+    def timed(a, threads):
+        ref.set_num_threads(threads)
+        n, t_total = 0, 0.0
+        while t_total < target_s / 2:
             t0 = time.perf_counter()
-            ref.selective_scan(u, delta, A, B, C, D=D, z=z, delta_bias=bias, softplus=True,
-                               zoh=zoh, initial_state=h0)
+            ref.selective_state_update(a["state"], a["x"], a["dt"], a["A"], a["B"], a["C"],
+                                       D=a["D"], z=a["z"], dt_bias=a["dt_bias"])
             t_total += time.perf_counter() - t0
-            done += c.dim * c.seqlen
-        passes += 1
-        if t_total >= target_s:
-            break
-    return {"value": done / t_total / 1e9, "unit": "Gelem/s", "cores": ref.num_threads(),
-            "kind": "oracle",
-            "sample": f"{passes} full pass(es) over {c.name} ({c.batch} batch rows x "
-                      f"{c.dim} channels x L={c.seqlen}; {done} elements) in {t_total:.1f} s "
-                      "of oracle time"}
+            n += 1
+        return t_total / n, n
+
+    all_threads = ref.num_threads()
+    t_all, n_all = timed(args, all_threads)
+    t_one, n_one = timed(one, 1)
+    ref.set_num_threads(all_threads)
+    t_one_full = t_one * d.batch / rows1
+    return {"kind": "oracle", "unit": "us per token step",
+            "us_per_token_step_cores_all": round(t_all * d.layers * 1e6, 1), "cores_all": all_threads,
+            "us_per_token_step_cores_1": round(t_one_full * d.layers * 1e6, 1), "cores_1": 1,
+            "sample": f"{n_all} updates of one layer's state ({d.batch} x {d.dim} x {d.dstate}) "
+                      f"on {all_threads} threads, {n_one} updates of {rows1} of its batch rows on "
+                      f"1 thread (scaled by {d.batch // rows1}); a token step is {d.layers} layers"}
 
 
 def bwd_cpu_baseline(cfg, x: dict, dout, target_s: float) -> dict:
@@ -464,11 +589,16 @@ def bench_ours(args, rank, world, local):
 
     peaks = measured_peaks()
     clocks = sampler.summary(t_wall0, t_wall1)
-    mufu = R.scan_mufu_per_element(c.dstate, has_z=True, softplus=True,
-                                   zoh=args.scan_variant == "zoh",
-                                   io_bytes=c.io_dtype.itemsize)
-    peak_elems = R.mufu_peak_elements_per_s(torch.cuda.get_device_properties(local).multi_processor_count,
-                                            peaks["sm_max_mhz"], mufu) / 1e9
+    sms = torch.cuda.get_device_properties(local).multi_processor_count
+    zoh = args.scan_variant == "zoh"
+    # Peak on the method's own operation count (16 exponentials for Abar, 2
+    # for softplus, 2 for the silu gate, and 1/Delta with the zero-order hold),
+    # and on the count the bf16 kernel issues (its gate takes one tanh).
+    mufu = R.scan_mufu_method(c.dstate, has_z=True, softplus=True, zoh=zoh)
+    mufu_k = R.scan_mufu_per_element(c.dstate, has_z=True, softplus=True, zoh=zoh,
+                                     io_bytes=c.io_dtype.itemsize)
+    peak_elems = R.mufu_peak_elements_per_s(sms, peaks["sm_max_mhz"], mufu) / 1e9
+    peak_kernel = R.mufu_peak_elements_per_s(sms, peaks["sm_max_mhz"], mufu_k) / 1e9
     achieved = elems / (scan_launch_ms * 1e-3) / 1e9               # per launch, this rank
     scan_bytes = R.scan_bytes(c.batch, c.dim, c.dstate, c.seqlen, 2, 2, True, True,
                               start_state=w.h0 is not None)
@@ -480,18 +610,31 @@ def bench_ours(args, rank, world, local):
         "kernel": "selective_scan_fwd_kernel",
         "achieved": round(achieved, 2), "peak": round(peak_elems, 2), "unit": "Gelem/s",
         "frac": round(achieved / peak_elems, 4),
-        "peak_basis": f"148 SMs x 16 MUFU/clk x {peaks['sm_max_mhz']:.0f} MHz / {mufu} MUFU ops "
-                      "the kernel issues per element",
+        "peak_basis": f"{sms} SMs x 16 MUFU/clk x {peaks['sm_max_mhz']:.0f} MHz / {mufu} MUFU ops "
+                      "per element in the method (16 exp for Abar, 2 softplus, 2 silu"
+                      + (", 1 for 1/Delta" if zoh else "") + ")",
         "frac_at_measured_clock": (round(achieved / (peak_elems * clocks["sm_mhz"] / peaks["sm_max_mhz"]), 4)
                                    if clocks.get("sm_mhz") else None),
+        "kernel_basis": {"mufu_per_element": mufu_k, "peak": round(peak_kernel, 2),
+                         "frac": round(achieved / peak_kernel, 4),
+                         "note": "the MUFU ops this kernel issues (bf16 inputs: the gate is one tanh)"},
         "algorithmic_bytes_per_launch": scan_bytes,
         "hbm_gbs": round(scan_bytes / (scan_launch_ms * 1e-3) / 1e9, 1),
         "traffic": recorded_traffic("selective_scan_fwd_kernel", digest),
     }
+    state_bytes = 2 * d.batch * d.dim * d.dstate * 4
+    state_gbs = state_bytes * d.layers / (decode_ms / K * 1e-3) / 1e9
     decode_roof = {"bound": "hbm", "kernel": "state_update_bulk_kernel",
                    "achieved": round(decode_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                    "frac": round(decode_gbs / peaks["hbm_gbs"], 4),
                    "peak_source": peaks["source"],
+                   "frac_of_nominal": round(decode_gbs / HBM_NOMINAL_GBS, 4),
+                   "nominal_peak": HBM_NOMINAL_GBS,
+                   "state_traffic": {"bytes_per_layer": state_bytes, "achieved": round(state_gbs, 1),
+                                     "frac_of_measured": round(state_gbs / peaks["hbm_gbs"], 4),
+                                     "frac_of_nominal": round(state_gbs / HBM_NOMINAL_GBS, 4),
+                                     "target": "state traffic at >= 75% of HBM peak; reported against "
+                                               "both the measured copy peak and the nominal 8 TB/s"},
                    "algorithmic_bytes_per_launch": upd_bytes,
                    "traffic": recorded_traffic("state_update_bulk_kernel", digest)}
     decode = {
@@ -513,9 +656,21 @@ def bench_ours(args, rank, world, local):
     e2e = None
     if not args.no_e2e and args.only != "decode":
         r = run_e2e(w, max(1, min(K, args.e2e_steps)), 2, args.e2e_rows)
-        e2e = {"value": round(job_gelem_per_s(world, elems, r["steps"], r["ms_total"]), 3),
+        e2e_value = job_gelem_per_s(world, elems, r["steps"], r["ms_total"])
+        pc = r["pcie"]
+        # Both directions run at once in the host-buffer pipeline, so the copy
+        # bound of a step is the slower direction at the rates measured alone.
+        copy_s = max(r["h2d"] / (pc["h2d_gbs"] * 1e9), r["d2h"] / (pc["d2h_gbs"] * 1e9))
+        pcie_bound = world * elems / copy_s / 1e9
+        e2e = {"value": round(e2e_value, 3),
                "unit": "Gelem/s", "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
                "steps": r["steps"],
+               "pcie": {"h2d_gbs": pc["h2d_gbs"], "d2h_gbs": pc["d2h_gbs"],
+                        "h2d_gbs_while_d2h": pc["h2d_gbs_while_d2h"],
+                        "copy_bound_gelem_s": round(pcie_bound, 3),
+                        "frac_of_copy_bound": round(e2e_value / pcie_bound, 4),
+                        "method": "pinned cudaMemcpyAsync of the u tensor (h2d) and the out "
+                                  "tensor (d2h), CUDA events, same run"},
                "path": "mamba_selective_scan_fwd_host: pinned host u/delta/z/B/C/A/D/bias -> "
                        f"device in chunks of {r['rows']} batch rows, scans overlapped with the "
                        "copies in and out -> out/last_state in pinned host memory"}
@@ -523,6 +678,8 @@ def bench_ours(args, rank, world, local):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.only != "decode":
         cpu = cpu_baseline(w, args.cpu_seconds)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.only != "scan":
+        decode["cpu_baseline"] = decode_cpu_baseline(w, args.cpu_seconds / 2)
 
     if rank == 0:
         line = {
@@ -780,8 +937,9 @@ def bench_ssd(args, rank, world, local):
     peaks = measured_peaks()
     nbytes = R.ssd_bytes(c.batch, c.seqlen, c.nheads, c.headdim, c.ngroups, c.dstate, c.has_z)
     flops = R.ssd_chunk_flops(c.batch, c.seqlen, c.nheads, c.headdim, c.dstate)
+    issued = R.ssd_issued_flops(c.batch, c.seqlen, c.nheads, c.headdim, c.dstate)
     gbs = nbytes / (ms * 1e-3) / 1e9
-    tfs = flops / (ms * 1e-3) / 1e12
+    tfs = issued / (ms * 1e-3) / 1e12
     traffic = recorded_traffic("ssd_chunk_scan_kernel", sources_digest())
     value = world * c.elements / (ms * 1e-3) / 1e9
     if rank == 0:
@@ -800,7 +958,9 @@ def bench_ssd(args, rank, world, local):
                          "traffic": traffic if c.batch == 16 else None,
                          "bytes_per_step": nbytes},
             "tensor": {"issued_tflops": round(tfs, 1), "peak": peaks["bf16_tflops"],
-                       "frac": round(tfs / peaks["bf16_tflops"], 4), "flops_per_step": flops},
+                       "frac": round(tfs / peaks["bf16_tflops"], 4), "issued_flops_per_step": issued,
+                       "algorithmic_flops_per_step": flops,
+                       "algorithmic_tflops": round(flops / (ms * 1e-3) / 1e12, 1)},
             "gpu_launches": K,
             "clocks": sampler.summary(t0, t1),
             "cpu_baseline": (None if args.no_cpu_baseline

@@ -200,6 +200,12 @@ MAMBA_API size_t mamba_selective_scan_workspace_bytes(const mamba_dims_t *dims);
  *   dims->workspace    required (see mamba_selective_scan_workspace_bytes)
  * seqlen == 0 writes no output; last_state (if given) is set to zero.
  * Returns MAMBA_ERR_WORKSPACE if the workspace is missing or too small.
+ * Sources: the recurrence h_t = Abar h_{t-1} + Bbar x_t, y_t = C h_t with
+ * Abar = exp(Delta A), "超越注意力：探索Mamba与状态空间模型", section
+ * 状态空间模型基础; Delta = softplus(. + b) and B, C per token, the same page,
+ * section 选择性状态空间模型, and Bbar x = Delta B u as in its section
+ * 代码实现概览; the scan that keeps the state on chip and writes only the
+ * outputs, "Mamba 与状态空间模型", section 在芯片上扫过去.
  */
 MAMBA_API mamba_status_t mamba_selective_scan_fwd(const void *u, const void *delta, const float *A,
                                                   const void *B, const void *C, const float *D,
@@ -291,8 +297,10 @@ MAMBA_API mamba_status_t mamba_selective_scan_fwd_host(
  *    131,000 (batch x channel) chains, which includes the Mamba-2.8B layer
  *    shape (81,920 chains).
  *  - The first call on each device looks up the array's device address with
- *    cudaGetSymbolAddress, with that device current.  Make that first call
- *    before any stream capture.
+ *    cudaGetSymbolAddress, with that device current, and keeps it for the
+ *    life of the process.  Make that first call before any stream capture.
+ *    The kept address does not survive cudaDeviceReset: after resetting a
+ *    device, do not call this entry point on it again in the same process.
  *  - Every call, on every stream, shares the one array per device.  Each call
  *    clears the part that must start at zero, but calls whose executions
  *    overlap on the GPU race on the array: run them in one stream or otherwise
@@ -320,6 +328,11 @@ MAMBA_API mamba_status_t mamba_selective_scan_fwd_noalloc(
  * Paths: for dstate == 16, dim % 8 == 0 and 16-byte aligned buffers the state
  * streams through shared memory by bulk TMA (MAMBA_FLAG_NO_TMA turns that
  * off); otherwise plain vectorised loads (dstate == 16) or a scalar path.
+ * Sources: one step of the recurrence of "超越注意力：探索Mamba与状态空间模型",
+ * sections 状态空间模型基础 and 选择性状态空间模型, applied to a stored state;
+ * "Mamba: Linear-Time Sequence Modeling with Selective State Spaces", table
+ * 复杂度对比 (constant time and memory per generated token); "Mamba 与状态空间模型",
+ * section 固定大小的状态 (the fixed-size state is all that generation keeps).
  */
 MAMBA_API mamba_status_t mamba_selective_state_update(float *state, const void *x, const void *dt,
                                                       const float *A, const void *B, const void *C,
@@ -448,8 +461,11 @@ MAMBA_API mamba_status_t mamba_causal_conv1d_update(void *conv_state, const void
  * ngroups not dividing nheads) before anything is launched.  x, z, out, B and
  * C must be 16-byte aligned, the fp32 arrays 4-byte aligned and dt 2-byte
  * aligned (MAMBA_ERR_ALIGN).  Products run on the tensor cores with bf16
- * operands (the intra-chunk matrix and the state copy used for the output
- * are rounded to bf16) and fp32 accumulation; the carried state stays fp32.
+ * operands and fp32 accumulation.  The operands the kernel computes (the
+ * masked intra-chunk matrix, the weighted input and the copy of the entering
+ * state) are each carried as a bf16 hi/lo pair (about 16 significant bits),
+ * so the carried state stays fp32-accurate and the only bf16-level rounding
+ * of the output is its own.
  * Asynchronous on `stream`; allocates nothing; a device-side wait that gives
  * up is reported by mamba_device_status() as MAMBA_ERR_TIMEOUT.
  */

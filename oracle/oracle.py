@@ -115,9 +115,16 @@ class Oracle:
             i64, i64, i64, i64, i64, i64, dp, dp, dp, dp, dp, dp, dp, dp, ci, dp, dp, dp]
         self._lib.oracle_num_threads.restype = ctypes.c_int
         self._lib.oracle_num_threads.argtypes = []
+        self._lib.oracle_set_num_threads.restype = None
+        self._lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
 
     def num_threads(self) -> int:
         return int(self._lib.oracle_num_threads())
+
+    def set_num_threads(self, n: int) -> None:
+        """Threads of the oracle's later parallel loops (timing only; results
+        do not depend on it)."""
+        self._lib.oracle_set_num_threads(int(n))
 
     def selective_scan(self, u, delta, A, B, C, D=None, z=None, delta_bias=None,
                        softplus=True, zoh=False, initial_state=None):

@@ -124,6 +124,19 @@ int oracle_num_threads(void)
 #endif
 }
 
+/* Threads of later parallel loops (n >= 1), for timing the oracle on one core
+ * and on all of them.  The results do not depend on it: every parallel loop
+ * runs independent chains (the backward pass runs sequentially). */
+void oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n >= 1)
+        omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
 int oracle_selective_scan_ex_f64(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
                                  const double *u, const double *delta, const double *A,
                                  const double *B, const double *C, const double *D,

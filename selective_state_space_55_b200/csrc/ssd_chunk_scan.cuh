@@ -10,26 +10,39 @@
 // One CTA of 128 threads owns one (batch, head) chain and walks its chunks
 // of Q = 128 tokens in order.  Per chunk, with c_i the running log2-decay
 // (c_i = log2(e) A_h sum_{r<=i} Delta_r inside the chunk) and H the state
-// entering the chunk (fp32, one TMEM lane / thread per state index n):
+// entering the chunk (fp32, thread n holds row n of H^T):
 //
-//   G     = C B^T                       (Q x Q,  K = dstate)        MMA 1
 //   Yoff  = C H^T                       (Q x P,  K = dstate)        MMA 3
 //   S^T   = B^T Xw, Xw_j = 2^(c_Q - c_j) Delta_j x_j   (N x P, K = Q) MMA 4
+//   G     = C B^T                       (Q x Q,  K = dstate)        MMA 1
 //   Gm_ij = G_ij 2^(c_i - c_j) Delta_j  for j <= i, else 0,
 //           plus D_h on the diagonal    (CUDA cores)
 //   Ydiag = Gm X  (= intra-chunk part + D_h x)  (Q x P, K = Q)      MMA 2
 //   y_i   = Ydiag_i + 2^(c_i) Yoff_i,  out = y silu(z)
 //   H     = 2^(c_Q) H + S               (fp32, in registers)
 //
-// Operands are bf16 in shared memory in the tensor cores' 128-byte-swizzle
-// layout (1024-byte atoms of 8 rows x 128 bytes); the products accumulate in
-// fp32 in tensor memory and are read back with tcgen05.ld.  One elected thread
-// issues the tcgen05.mma instructions and commits them to an mbarrier that
-// the CTA waits on (bounded).  Operand tiles arrive by TMA, one box per
-// tile, and the next chunk's tiles are requested as soon as this chunk's
-// products are done with each buffer.  Delta_j enters only through
-// e_j = c_j - log2(Delta_j), so that 2^(c_i - e_j) = 2^(c_i - c_j) Delta_j
-// and padded tokens (Delta = 0, e = +inf) drop out by themselves.
+// Precision.  The tensor cores multiply bf16 operands.  C, B and x are bf16
+// inputs and enter exactly; the three operands the kernel computes (H, Xw
+// and Gm) would lose their low bits if rounded to bf16 once, and an output
+// that cancels across many terms would then carry an error near 2^-9 times
+// the sum of the terms' magnitudes.  Each of them is therefore split as
+// v = hi + lo with hi = bf16(v) and lo = bf16(v - hi), and its product is
+// issued twice into the same fp32 accumulator; the pair carries v to about
+// 2^-17 relative, so the only rounding left at the bf16 level is the one of
+// the output itself.
+//
+// Operands in shared memory are in the tensor cores' 128-byte-swizzle layout
+// (1024-byte atoms of 8 rows x 128 bytes).  Gm is formed row by row (thread i
+// holds row i) and written straight into tensor memory, from where MMA 2
+// reads it as its A operand; this keeps the 2 x 32 KB of Gm out of shared
+// memory, which then holds C, B, x and one 32 KB buffer that takes H's hi/lo
+// pair for MMA 3 and then Xw's for MMA 4, so two CTAs still fit on an SM.
+// One elected thread issues the tcgen05.mma instructions and commits them to
+// mbarriers that the CTA waits on (bounded).  Operand tiles arrive by TMA,
+// one box per tile, each requested as soon as its buffer is free.  Delta_j
+// enters only through e_j = c_j - log2(Delta_j), so that
+// 2^(c_i - e_j) = 2^(c_i - c_j) Delta_j and padded tokens (Delta = 0,
+// e = +inf) drop out by themselves.
 #pragma once
 
 #include "ssm_device.cuh"
@@ -40,24 +53,50 @@ constexpr int kSsdP = 64;          // head dimension
 constexpr int kSsdN = 128;         // state size
 constexpr int kSsdQ = 128;         // chunk length
 constexpr int kSsdThreads = 128;   // one thread per TMEM lane
-constexpr int kSsdTmemCols = 256;  // G [0,128) (then Ydiag [0,64)), Yoff [128,192), S [192,256)
+constexpr int kSsdTmemCols = 256;
 
-// Shared-memory map (bytes).  sC holds C and later Gm.  Every operand tile is
-// 128 rows in the 128-byte-swizzle layout of the tensor cores: each group of
-// 64 columns ("half") is 128 rows of 128 bytes, 8 rows to a 1024-byte atom,
-// and the 16-byte chunk c of row r sits at chunk position c ^ (r % 8); halves
-// are 16 KB apart.  ssd_sw128 gives the byte offset.
-constexpr int kSsdOffC = 0;          // 128 x 128 bf16: C (rows i, k = n), then Gm (rows i, k = j)
-constexpr int kSsdOffB = 32768;      // 128 x 128 bf16: B (rows j, k = n)
+// Tensor-memory columns (fp32 unless packed).  G fills [0, 128) until the
+// masked matrix has been formed from it; Gm's lo half (bf16 pairs, K = j)
+// then takes [0, 64) and MMA 2 writes Ydiag to [64, 128).  S fills
+// [192, 256) until the state update has read it; Gm's hi half then takes it.
+constexpr uint32_t kTmG = 0;
+constexpr uint32_t kTmGmLo = 0;
+constexpr uint32_t kTmYdiag = 64;
+constexpr uint32_t kTmYoff = 128;
+constexpr uint32_t kTmS = 192;
+constexpr uint32_t kTmGmHi = 192;
+
+// Shared-memory map (bytes).  Every operand tile is 128 rows in the
+// 128-byte-swizzle layout of the tensor cores: each group of 64 columns
+// ("half") is 128 rows of 128 bytes, 8 rows to a 1024-byte atom, and the
+// 16-byte chunk c of row r sits at chunk position c ^ (r % 8); halves are
+// 16 KB apart.  ssd_sw128 gives the byte offset.
+constexpr int kSsdOffC = 0;          // 128 x 128 bf16: C (rows i, k = n)
+constexpr int kSsdOffB = 32768;      // 128 x 128 bf16: B (rows j, k = n); once MMA 1 and 4
+                                     // are done, its first half takes the gate tile z and
+                                     // then the output tile (rows i, 64 columns p)
 constexpr int kSsdOffX = 65536;      // 128 x 64 bf16: x (rows j, k = p)
-constexpr int kSsdOffXw = 81920;     // 128 x 64 bf16: Xw (rows j, k = p)
-constexpr int kSsdOffH = 98304;      // 128 x 64 bf16: H (rows n, k = p)
+constexpr int kSsdOffHX = 81920;     // hi at +0, lo at +16384, each 128 x 64 bf16:
+                                     // H (rows n, k = p) for MMA 3, then Xw (rows j, k = p)
 constexpr int kSsdOffE = 114688;     // 128 fp32: -e_j, e_j = c_j - log2(Delta_j)
-constexpr int kSsdOffMisc = 115200;  // mbarriers (+0 products 1/3, +8 product 2, +16 tiles,
-                                     // +24 gate, +40 product 4), the TMEM address (+32),
-                                     // warp totals (+48)
-constexpr int kSsdSmemBytes = 115264;
-constexpr uint32_t kSsdTileBytes = 2 * 32768 + 16384;   // C, B and x of one chunk
+constexpr int kSsdOffBar = 115200;   // 8 mbarriers (see SsdBar)
+constexpr int kSsdOffSlot = 115264;  // TMEM base address written by tcgen05.alloc
+constexpr int kSsdOffTot = 115280;   // 4 fp32 warp totals of the decay prefix sum
+constexpr int kSsdSmemBytes = 115328;
+constexpr uint32_t kSsdLoBytes = 16384;   // offset of the lo half in the HX buffer
+
+// mbarrier indices; each completes at most once per chunk.
+enum SsdBar : int {
+    kBarC = 0,      // C tile landed
+    kBarB = 1,      // B tile landed
+    kBarX = 2,      // x tile landed
+    kBarZ = 3,      // gate tile landed
+    kBarYoff = 4,   // MMA 3 done
+    kBarS = 5,      // MMA 4 done
+    kBarG = 6,      // MMA 1 done
+    kBarYd = 7,     // MMA 2 done
+    kSsdBars = 8
+};
 
 struct SsdParams {
     const __nv_bfloat16* x;      // (batch, L, nheads, 64)
@@ -108,6 +147,7 @@ __device__ __forceinline__ uint32_t ssd_sw128(int row, int chunk) {
                       (((chunk & 7) ^ (row & 7)) << 4));
 }
 
+// D (+)= A B with A and B in shared memory.
 __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                           uint32_t idesc, uint32_t accumulate) {
     asm volatile(
@@ -115,6 +155,18 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
         ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// D (+)= A B with A in tensor memory (row m in lane m, K-major, two bf16 per
+// 32-bit column, the lower K index in the low half) and B in shared memory.
+__device__ __forceinline__ void umma_bf16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 
@@ -184,6 +236,22 @@ __device__ __forceinline__ void tmem_ld32x2(uint32_t ta, uint32_t tb, float (&a)
     }
 }
 
+// 16 consecutive 32-bit columns of this thread's TMEM lane from registers.
+// Complete (visible to the tensor cores after a fence and barrier) once
+// tmem_wait_st returns.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+          "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]),
+          "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 // 1/x on the MUFU pipe (rcp.approx, flush-to-zero); 0 for x = +inf.
 __device__ __forceinline__ float rcp_approx(float x) {
     float y;
@@ -191,19 +259,41 @@ __device__ __forceinline__ float rcp_approx(float x) {
     return y;
 }
 
-// The state H of this thread's row n as bf16 into sH (row n, 64 columns p).
+// a ~ hi + lo and b likewise: hi = bf16(v), lo = bf16(v - hi), each pair
+// packed into one word with a in the low half.  v - hi is exact in fp32
+// (hi holds v's leading 8 significant bits), so only lo's own rounding is
+// lost: |v - hi - lo| <= 2^-9 |v - hi| <= 2^-17 |v| or so.
+__device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t& hi, uint32_t& lo) {
+    hi = pack_bf16x2(a, b);
+    lo = pack_bf16x2(a - __uint_as_float(hi << 16), b - __uint_as_float(hi & 0xffff0000u));
+}
+
+// Eight fp32 values as 16-byte hi and lo chunks.
+__device__ __forceinline__ void split16(const float (&f)[8], uint4& hi, uint4& lo) {
+    split_bf16x2(f[0], f[1], hi.x, lo.x);
+    split_bf16x2(f[2], f[3], hi.y, lo.y);
+    split_bf16x2(f[4], f[5], hi.z, lo.z);
+    split_bf16x2(f[6], f[7], hi.w, lo.w);
+}
+
+// The state H of this thread's row n as its bf16 hi/lo pair into the HX
+// buffer (row n, 64 columns p per half).
 __device__ __forceinline__ void ssd_store_state(unsigned char* smem, int n, const float (&H)[kSsdP]) {
 #pragma unroll
     for (int q = 0; q < kSsdP / 8; ++q) {
         float f[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) f[k] = H[q * 8 + k];
-        *reinterpret_cast<uint4*>(smem + kSsdOffH + ssd_sw128(n, q)) = pack16(f);
+        uint4 hi, lo;
+        split16(f, hi, lo);
+        const uint32_t off = ssd_sw128(n, q);
+        *reinterpret_cast<uint4*>(smem + kSsdOffHX + off) = hi;
+        *reinterpret_cast<uint4*>(smem + kSsdOffHX + kSsdLoBytes + off) = lo;
     }
 }
 
-// Wait for one commit of the tensor-core work; true on every thread if any
-// thread's bounded wait gave up.
+// Wait for one completion of an mbarrier; true on every thread if any
+// thread's bounded wait gave up.  Also a CTA-wide barrier.
 __device__ __forceinline__ bool ssd_wait_failed(uint32_t bar, uint32_t parity) {
     const bool ok = mbar_wait_bounded(bar, parity);
     const bool failed = __syncthreads_or(!ok) != 0;
@@ -227,24 +317,21 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
     const int64_t L = p.seqlen;
     const uint32_t s0 = smem_u32(smem);
     float* sE = reinterpret_cast<float*>(smem + kSsdOffE);
-    float* sTot = reinterpret_cast<float*>(smem + kSsdOffMisc + 48);
-    const uint32_t bar1 = s0 + kSsdOffMisc, bar2 = bar1 + 8, bar_ld = bar1 + 16, bar_z = bar1 + 24;
-    const uint32_t bar_s = bar1 + 40;
-    const uint32_t* tslot = reinterpret_cast<const uint32_t*>(smem + kSsdOffMisc + 32);
+    float* sTot = reinterpret_cast<float*>(smem + kSsdOffTot);
+    const uint32_t bar0 = s0 + kSsdOffBar;
+    auto bar = [bar0](int k) -> uint32_t { return bar0 + 8u * (uint32_t)k; };
+    const uint32_t* tslot = reinterpret_cast<const uint32_t*>(smem + kSsdOffSlot);
     const bool has_z = p.z != nullptr;
 
-    if (warp == 0) tmem_alloc(s0 + kSsdOffMisc + 32, kSsdTmemCols);
+    if (warp == 0) tmem_alloc(s0 + kSsdOffSlot, kSsdTmemCols);
     if (tid == 0) {
         prefetch_tensormap(&tm_x);
         prefetch_tensormap(&tm_z);
         prefetch_tensormap(&tm_B);
         prefetch_tensormap(&tm_C);
         prefetch_tensormap(&tm_out);
-        mbar_init(bar1, 1);
-        mbar_init(bar2, 1);
-        mbar_init(bar_ld, 1);
-        mbar_init(bar_z, 1);
-        mbar_init(bar_s, 1);
+#pragma unroll
+        for (int k = 0; k < kSsdBars; ++k) mbar_init(bar(k), 1);
         fence_mbar_init();
     }
     tc_fence_before();
@@ -257,15 +344,27 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
     const float Dh = p.D ? p.D[h] : 0.0f;
     const float bias = p.dt_bias ? p.dt_bias[h] : 0.0f;
 
-    // Thread n holds row n of the state: H[p] = state[p][n], in fp32.
+    // Thread n holds row n of H^T: H[q] = state[q][n], in fp32.
     float H[kSsdP];
     const size_t hoff = (size_t)chain * kSsdP * kSsdN + tid;
 #pragma unroll
     for (int q = 0; q < kSsdP; ++q) H[q] = p.h0 ? p.h0[hoff + (size_t)q * kSsdN] : 0.0f;
     ssd_store_state(smem, tid, H);
+    fence_proxy_async_smem();
 
     const int64_t nchunks = (L + kSsdQ - 1) / kSsdQ;
+    // Every thread tracks, per mbarrier, whether a completion is outstanding
+    // (`pend`) and the parity of the next one (`phase`); the issuing thread's
+    // copy tells a failed CTA what it must still wait for before it leaves.
+    uint32_t pend = 0, phase = 0;
     bool failed = false;
+    auto issued = [&](int k) { pend |= 1u << k; };
+    auto wait_on = [&](int k) -> bool {
+        if (ssd_wait_failed(bar(k), (phase >> k) & 1u)) return true;
+        pend &= ~(1u << k);
+        phase ^= 1u << k;
+        return false;
+    };
     // K-major operand, K step k of 16 columns: 32 bytes along the swizzled
     // 128-byte rows, the second 64 columns one half (16 KB) further.
     auto kmaj = [](int k) -> uint32_t { return (uint32_t)((k >> 2) * 16384 + (k & 3) * 32); };
@@ -275,23 +374,48 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
     };
     float dt_next = load_dt(tid);
 
-    // Tiles of chunk c + 1 are requested while chunk c still computes: B once
-    // MMA 1 and 4 are done with it, C and x once MMA 2 is.  All three complete
-    // on bar_ld, whose expected byte count is set with the first of them.
-    if (tid == 0 && nchunks > 0) {
-        mbar_arrive_expect_tx(bar_ld, kSsdTileBytes);
-        tma_load_tile(s0 + kSsdOffB, &tm_B, 0, g, b, bar_ld);
-        tma_load_tile(s0 + kSsdOffC, &tm_C, 0, g, b, bar_ld);
-        tma_load_tile(s0 + kSsdOffX, &tm_x, 0, h, b, bar_ld);
+    if (nchunks > 0) {
+        if (tid == 0) {
+            mbar_arrive_expect_tx(bar(kBarC), 32768);
+            tma_load_tile(s0 + kSsdOffC, &tm_C, 0, g, b, bar(kBarC));
+            mbar_arrive_expect_tx(bar(kBarB), 32768);
+            tma_load_tile(s0 + kSsdOffB, &tm_B, 0, g, b, bar(kBarB));
+            mbar_arrive_expect_tx(bar(kBarX), 16384);
+            tma_load_tile(s0 + kSsdOffX, &tm_x, 0, h, b, bar(kBarX));
+        }
+        issued(kBarC);
+        issued(kBarB);
+        issued(kBarX);
     }
+
+    constexpr uint32_t id_g = umma_idesc_bf16(128, 128, false, false);
+    constexpr uint32_t id_off = umma_idesc_bf16(128, 64, false, true);
+    constexpr uint32_t id_s = umma_idesc_bf16(128, 64, true, true);
+    constexpr uint32_t id_y = umma_idesc_bf16(128, 64, false, true);
 
     for (int64_t c = 0; c < nchunks; ++c) {
         const int l0 = (int)(c * kSsdQ);
-        const uint32_t parity = (uint32_t)(c & 1);
-
         const bool more = c + 1 < nchunks;
 
-        // ---- Delta, the running log2-decay c_i and e_i = c_i - log2(Delta_i).
+        // ---- C landed (the barrier also publishes the entering state's hi/lo
+        // pair): MMA 3, Yoff = C (H_hi + H_lo)^T.
+        if (wait_on(kBarC)) { failed = true; break; }
+        if (tid == 0) {
+#pragma unroll
+            for (int k = 0; k < kSsdN / 16; ++k)
+                umma_bf16(tmem + kTmYoff, umma_sdesc_sw128(s0 + kSsdOffC + kmaj(k), 16, 1024),
+                          umma_sdesc_sw128(s0 + kSsdOffHX + k * 2048, 16384, 1024), id_off, k);
+#pragma unroll
+            for (int k = 0; k < kSsdN / 16; ++k)
+                umma_bf16(tmem + kTmYoff, umma_sdesc_sw128(s0 + kSsdOffC + kmaj(k), 16, 1024),
+                          umma_sdesc_sw128(s0 + kSsdOffHX + kSsdLoBytes + k * 2048, 16384, 1024),
+                          id_off, 1);
+            umma_commit(bar(kBarYoff));
+        }
+        issued(kBarYoff);
+
+        // ---- Delta, the running log2-decay c_i and e_i = c_i - log2(Delta_i),
+        // while MMA 3 runs.
         float delta = 0.0f;
         if (l0 + tid < L) {
             const float sarg = dt_next + bias;
@@ -312,15 +436,11 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
         const float cQ = (sTot[0] + sTot[1]) + (sTot[2] + sTot[3]);
         const float e_own = ci - lg2_approx(delta);   // +inf for Delta = 0
         sE[tid] = -e_own;                              // stored negated: c_i - e_j is an add
-        // The previous chunk's output store must have read the staging tile
-        // (rewritten by the Xw pass below).
-        if (tid == 0) bulk_wait_read<0>();
-        if (ssd_wait_failed(bar_ld, parity)) {   // tiles landed; sE published
-            failed = true;
-            break;
-        }
 
-        // ---- Xw_j = 2^(c_Q - e_j) x_j = 2^(c_Q - c_j) Delta_j x_j (row j = tid).
+        // ---- x landed and MMA 3 is done with the HX buffer: Xw_j hi/lo
+        // (row j = tid), Xw_j = 2^(c_Q - e_j) x_j = 2^(c_Q - c_j) Delta_j x_j.
+        if (wait_on(kBarX)) { failed = true; break; }
+        if (wait_on(kBarYoff)) { failed = true; break; }
         {
             const float w = ex2_approx(cQ - e_own);
             const float2 w2 = make_float2(w, w);
@@ -335,50 +455,45 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
                     f[k] = r.x;
                     f[k + 1] = r.y;
                 }
-                *reinterpret_cast<uint4*>(smem + kSsdOffXw + off) = pack16(f);
+                uint4 hi, lo;
+                split16(f, hi, lo);
+                *reinterpret_cast<uint4*>(smem + kSsdOffHX + off) = hi;
+                *reinterpret_cast<uint4*>(smem + kSsdOffHX + kSsdLoBytes + off) = lo;
             }
         }
         fence_proxy_async_smem();
-        __syncthreads();
 
-        // ---- MMA 4 (S^T = B^T Xw), committed alone, then 3 (Yoff = C H^T) and
-        // 1 (G = C B^T).
+        // ---- B landed (the barrier also publishes Xw and e): MMA 4,
+        // S^T = B^T (Xw_hi + Xw_lo), committed alone, then MMA 1, G = C B^T.
+        if (wait_on(kBarB)) { failed = true; break; }
         if (tid == 0) {
-            tc_fence_after();
-            constexpr uint32_t id_g = umma_idesc_bf16(128, 128, false, false);
-            constexpr uint32_t id_off = umma_idesc_bf16(128, 64, false, true);
-            constexpr uint32_t id_s = umma_idesc_bf16(128, 64, true, true);
 #pragma unroll
             for (int k = 0; k < kSsdQ / 16; ++k)
-                umma_bf16(tmem + 192, umma_sdesc_sw128(s0 + kSsdOffB + k * 2048, 16384, 1024),
-                          umma_sdesc_sw128(s0 + kSsdOffXw + k * 2048, 16384, 1024), id_s, k);
-            umma_commit(bar_s);
+                umma_bf16(tmem + kTmS, umma_sdesc_sw128(s0 + kSsdOffB + k * 2048, 16384, 1024),
+                          umma_sdesc_sw128(s0 + kSsdOffHX + k * 2048, 16384, 1024), id_s, k);
+#pragma unroll
+            for (int k = 0; k < kSsdQ / 16; ++k)
+                umma_bf16(tmem + kTmS, umma_sdesc_sw128(s0 + kSsdOffB + k * 2048, 16384, 1024),
+                          umma_sdesc_sw128(s0 + kSsdOffHX + kSsdLoBytes + k * 2048, 16384, 1024),
+                          id_s, 1);
+            umma_commit(bar(kBarS));
 #pragma unroll
             for (int k = 0; k < kSsdN / 16; ++k)
-                umma_bf16(tmem + 128, umma_sdesc_sw128(s0 + kSsdOffC + kmaj(k), 16, 1024),
-                          umma_sdesc_sw128(s0 + kSsdOffH + k * 2048, 16384, 1024), id_off, k);
-#pragma unroll
-            for (int k = 0; k < kSsdN / 16; ++k)
-                umma_bf16(tmem, umma_sdesc_sw128(s0 + kSsdOffC + kmaj(k), 16, 1024),
+                umma_bf16(tmem + kTmG, umma_sdesc_sw128(s0 + kSsdOffC + kmaj(k), 16, 1024),
                           umma_sdesc_sw128(s0 + kSsdOffB + kmaj(k), 16, 1024), id_g, k);
-            umma_commit(bar1);
+            umma_commit(bar(kBarG));
         }
-        if (ssd_wait_failed(bar_s, parity)) {
-            failed = true;
-            break;
-        }
-        // ---- the gate tile z (128 x 64) by TMA into the Xw buffer, which MMA 4
-        // no longer reads; it lands while the masked matrix and MMA 2 run.
-        if (tid == 0 && has_z) {
-            mbar_arrive_expect_tx(bar_z, 16384);
-            tma_load_tile(s0 + kSsdOffXw, &tm_z, l0, h, b, bar_z);
-        }
-        // ---- state: H = 2^(c_Q) H + S (row n = tid), in registers while MMA 3
-        // and 1 run; its bf16 copy for the next chunk's MMA 3 waits for them.
+        issued(kBarS);
+        issued(kBarG);
+
+        // ---- state: H = 2^(c_Q) H + S (row n = tid), in registers while MMA 1
+        // runs; its hi/lo pair goes to the HX buffer, which MMA 4 no longer reads,
+        // for the next chunk's MMA 3.
+        if (wait_on(kBarS)) { failed = true; break; }
         {
             const float dq = ex2_approx(cQ);
             float s_lo[32], s_hi[32];
-            tmem_ld32x2(tlane + 192, tlane + 224, s_lo, s_hi);
+            tmem_ld32x2(tlane + kTmS, tlane + kTmS + 32, s_lo, s_hi);
             const float2 dq2 = make_float2(dq, dq);
 #pragma unroll
             for (int k = 0; k < 32; k += 2) {
@@ -391,99 +506,105 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
                 H[33 + k] = hi.y;
             }
         }
-        if (ssd_wait_failed(bar1, parity)) {
-            failed = true;
-            break;
-        }
-
-        // ---- next chunk's B (MMA 1 and 4 are done with it); the state's bf16 copy.
-        if (tid == 0 && more) {
-            mbar_arrive_expect_tx(bar_ld, kSsdTileBytes);
-            tma_load_tile(s0 + kSsdOffB, &tm_B, l0 + kSsdQ, g, b, bar_ld);
-        }
         ssd_store_state(smem, tid, H);
+        fence_proxy_async_smem();
 
-        const float2 ci2 = make_float2(ci, ci);
-        // ---- Gm_ij = G_ij 2^(c_i - e_j) for j <= i (row i = tid), over C's tile.
-        // Warp w holds rows [32w, 32w + 32): quarters of columns below w are
-        // entirely at or below the diagonal, quarter w straddles it, and the
-        // quarters above are zero (no TMEM read, no exponentials).  Quarters
-        // are read from TMEM two at a time.
-#pragma unroll
-        for (int pair = 0; pair < 2; ++pair) {
-            const int qa = 2 * pair, qb = 2 * pair + 1;
-            if (qa > warp) {
-                const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-                for (int q = 0; q < 8; ++q)
-                    *reinterpret_cast<uint4*>(smem + kSsdOffC + ssd_sw128(tid, qa * 4 + q)) = zero;
-                continue;
+        // ---- MMA 1 done: C and B are free.  Next chunk's C; this chunk's gate
+        // tile into B's first half.
+        if (wait_on(kBarG)) { failed = true; break; }
+        if (tid == 0) {
+            if (more) {
+                mbar_arrive_expect_tx(bar(kBarC), 32768);
+                tma_load_tile(s0 + kSsdOffC, &tm_C, l0 + kSsdQ, g, b, bar(kBarC));
             }
-            float gv[2][32];
-            tmem_ld32x2(tlane + qa * 32, tlane + qb * 32, gv[0], gv[1]);
+            if (has_z) {
+                mbar_arrive_expect_tx(bar(kBarZ), 16384);
+                tma_load_tile(s0 + kSsdOffB, &tm_z, l0, h, b, bar(kBarZ));
+            }
+        }
+        if (more) issued(kBarC);
+        if (has_z) issued(kBarZ);
+
+        // ---- Gm_ij = G_ij 2^(c_i - e_j) for j <= i (row i = tid), as hi/lo
+        // pairs into tensor memory.  Warp w holds rows [32w, 32w + 32): quarters
+        // of columns below w are entirely at or below the diagonal, quarter w
+        // straddles it, and the quarters above are zero (no TMEM read, no
+        // exponentials).  G is read one column half at a time; the half's lo
+        // words land in columns whose G values this lane has already read.
+        {
+            const float2 ci2 = make_float2(ci, ci);
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                const int quarter = qa + half;
-                if (quarter > warp) {
-                    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+            for (int hf = 0; hf < 2; ++hf) {
+                const int qa = 2 * hf;
+                float gv[2][32];
+                if (qa <= warp) tmem_ld32x2(tlane + kTmG + qa * 32, tlane + kTmG + qa * 32 + 32,
+                                            gv[0], gv[1]);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        *reinterpret_cast<uint4*>(smem + kSsdOffC + ssd_sw128(tid, quarter * 4 + q)) = zero;
-                    continue;
-                }
-                const bool diag = quarter == warp;   // D_h x_i enters as Gm_ii += D_h
+                for (int s = 0; s < 2; ++s) {
+                    const int quarter = qa + s;
+                    uint32_t hi[16], lo[16];
+                    if (quarter > warp) {
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int j0 = quarter * 32 + q * 8;
-                    const float4 e0 = *reinterpret_cast<const float4*>(sE + j0);
-                    const float4 e1 = *reinterpret_cast<const float4*>(sE + j0 + 4);
-                    const float2 ne[4] = {make_float2(e0.x, e0.y), make_float2(e0.z, e0.w),
-                                          make_float2(e1.x, e1.y), make_float2(e1.z, e1.w)};
-                    float f[8];
+                        for (int k = 0; k < 16; ++k) hi[k] = lo[k] = 0u;
+                    } else {
+                        const bool diag = quarter == warp;   // D_h x_i enters as Gm_ii += D_h
 #pragma unroll
-                    for (int k = 0; k < 8; k += 2) {
-                        const float2 arg = __fadd2_rn(ci2, ne[k / 2]);
-                        const float2 v = __fmul2_rn(
-                            make_float2(gv[half][q * 8 + k], gv[half][q * 8 + k + 1]),
-                            make_float2(ex2_approx(arg.x), ex2_approx(arg.y)));
-                        f[k] = v.x;
-                        f[k + 1] = v.y;
+                        for (int q = 0; q < 4; ++q) {
+                            const int j0 = quarter * 32 + q * 8;
+                            const float4 e0 = *reinterpret_cast<const float4*>(sE + j0);
+                            const float4 e1 = *reinterpret_cast<const float4*>(sE + j0 + 4);
+                            const float2 ne[4] = {make_float2(e0.x, e0.y), make_float2(e0.z, e0.w),
+                                                  make_float2(e1.x, e1.y), make_float2(e1.z, e1.w)};
+                            float f[8];
+#pragma unroll
+                            for (int k = 0; k < 8; k += 2) {
+                                const float2 arg = __fadd2_rn(ci2, ne[k / 2]);
+                                const float2 v = __fmul2_rn(
+                                    make_float2(gv[s][q * 8 + k], gv[s][q * 8 + k + 1]),
+                                    make_float2(ex2_approx(arg.x), ex2_approx(arg.y)));
+                                f[k] = v.x;
+                                f[k + 1] = v.y;
+                            }
+                            if (diag) {
+#pragma unroll
+                                for (int k = 0; k < 8; ++k)
+                                    f[k] = j0 + k < tid ? f[k] : (j0 + k == tid ? f[k] + Dh : 0.0f);
+                            }
+#pragma unroll
+                            for (int k = 0; k < 4; ++k)
+                                split_bf16x2(f[2 * k], f[2 * k + 1], hi[q * 4 + k], lo[q * 4 + k]);
+                        }
                     }
-                    if (diag) {
-#pragma unroll
-                        for (int k = 0; k < 8; ++k)
-                            f[k] = j0 + k < tid ? f[k] : (j0 + k == tid ? f[k] + Dh : 0.0f);
-                    }
-                    *reinterpret_cast<uint4*>(smem + kSsdOffC + ssd_sw128(tid, j0 / 8)) = pack16(f);
+                    tmem_st16(tlane + kTmGmHi + quarter * 16, hi);
+                    tmem_st16(tlane + kTmGmLo + quarter * 16, lo);
                 }
             }
         }
-        fence_proxy_async_smem();
+        tmem_wait_st();
         tc_fence_before();
         __syncthreads();
 
-        // ---- MMA 2: Ydiag = Gm X into columns [0, 64).
+        // ---- MMA 2: Ydiag = (Gm_hi + Gm_lo) X, A from tensor memory.
         if (tid == 0) {
             tc_fence_after();
-            constexpr uint32_t id_y = umma_idesc_bf16(128, 64, false, true);
 #pragma unroll
             for (int k = 0; k < kSsdQ / 16; ++k)
-                umma_bf16(tmem, umma_sdesc_sw128(s0 + kSsdOffC + kmaj(k), 16, 1024),
-                          umma_sdesc_sw128(s0 + kSsdOffX + k * 2048, 16384, 1024), id_y, k);
-            umma_commit(bar2);
+                umma_bf16_ta(tmem + kTmYdiag, tmem + kTmGmHi + 8 * k,
+                             umma_sdesc_sw128(s0 + kSsdOffX + k * 2048, 16384, 1024), id_y, k);
+#pragma unroll
+            for (int k = 0; k < kSsdQ / 16; ++k)
+                umma_bf16_ta(tmem + kTmYdiag, tmem + kTmGmLo + 8 * k,
+                             umma_sdesc_sw128(s0 + kSsdOffX + k * 2048, 16384, 1024), id_y, 1);
+            umma_commit(bar(kBarYd));
         }
-        if (ssd_wait_failed(bar2, parity)) {
-            failed = true;
-            break;
+        issued(kBarYd);
+        if (wait_on(kBarYd)) { failed = true; break; }
+        if (tid == 0 && more) {   // x is no longer read
+            mbar_arrive_expect_tx(bar(kBarX), 16384);
+            tma_load_tile(s0 + kSsdOffX, &tm_x, l0 + kSsdQ, h, b, bar(kBarX));
         }
-        if (tid == 0 && more) {   // Gm and x are no longer read
-            tma_load_tile(s0 + kSsdOffC, &tm_C, l0 + kSsdQ, g, b, bar_ld);
-            tma_load_tile(s0 + kSsdOffX, &tm_x, l0 + kSsdQ, h, b, bar_ld);
-        }
-        if (has_z && ssd_wait_failed(bar_z, parity)) {
-            failed = true;
-            break;
-        }
+        if (more) issued(kBarX);
+        if (has_z && wait_on(kBarZ)) { failed = true; break; }
 
         // ---- y_i = Ydiag_i + 2^(c_i) Yoff_i (D x_i is inside Ydiag), gated (row
         // i = tid), written as bf16 over the gate tile, then stored by TMA (rows
@@ -494,7 +615,7 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 float yd[32], yo[32];
-                tmem_ld32x2(tlane + half * 32, tlane + 128 + half * 32, yd, yo);
+                tmem_ld32x2(tlane + kTmYdiag + half * 32, tlane + kTmYoff + half * 32, yd, yo);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     const int pb = half * 4 + q;
@@ -510,7 +631,7 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
                     if (has_z) {
                         // silu(z) = z / (1 + 2^(-z log2 e)), two lanes at a time
                         float zv[8];
-                        unpack16(*reinterpret_cast<const uint4*>(smem + kSsdOffXw + off), zv);
+                        unpack16(*reinterpret_cast<const uint4*>(smem + kSsdOffB + off), zv);
 #pragma unroll
                         for (int k = 0; k < 8; k += 2) {
                             const float2 z2 = make_float2(zv[k], zv[k + 1]);
@@ -523,24 +644,40 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
                             f[k + 1] = r.y;
                         }
                     }
-                    *reinterpret_cast<uint4*>(smem + kSsdOffXw + off) = pack16(f);
+                    *reinterpret_cast<uint4*>(smem + kSsdOffB + off) = pack16(f);
                 }
             }
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        __syncthreads();   // the output tile is complete; the next chunk rewrites the rest
+        __syncthreads();   // the output tile is complete
         if (tid == 0) {
-            tma_store_tile(&tm_out, s0 + kSsdOffXw, l0, h, b);
+            tma_store_tile(&tm_out, s0 + kSsdOffB, l0, h, b);
             bulk_commit();
+            if (more) {    // the store has read the tile: the next chunk's B may land there
+                bulk_wait_read<0>();
+                mbar_arrive_expect_tx(bar(kBarB), 32768);
+                tma_load_tile(s0 + kSsdOffB, &tm_B, l0 + kSsdQ, g, b, bar(kBarB));
+            }
         }
+        if (more) issued(kBarB);
     }
 
     if (!failed && p.hT) {
 #pragma unroll
         for (int q = 0; q < kSsdP; ++q) p.hT[hoff + (size_t)q * kSsdN] = H[q];
     }
-    if (tid == 0) bulk_wait<0>();   // output stores done before the CTA's shared memory goes
+    if (tid == 0) {
+        bulk_wait<0>();   // output stores done before the CTA's shared memory goes
+        // After a timeout, wait (bounded) for every copy and product still in
+        // flight, so that none lands in shared or tensor memory after the CTA
+        // has released them.
+        if (failed) {
+#pragma unroll 1
+            for (int k = 0; k < kSsdBars; ++k)
+                if ((pend >> k) & 1u) (void)mbar_wait_bounded(bar(k), (phase >> k) & 1u);
+        }
+    }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {

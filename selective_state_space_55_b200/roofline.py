@@ -40,6 +40,16 @@ def scan_mufu_per_element(dstate: int = 16, has_z: bool = True, softplus: bool =
             + (ZOH_MUFU if zoh else 0))
 
 
+def scan_mufu_method(dstate: int = 16, has_z: bool = True, softplus: bool = True,
+                     zoh: bool = False) -> int:
+    """MUFU operations per element that the method itself needs, independent
+    of how a kernel evaluates them: one exponential per state entry for Abar,
+    softplus as an exponential and a logarithm, the silu gate as an
+    exponential and a reciprocal, and 1/Delta with the zero-order hold."""
+    return (dstate * EXP_PER_STATE + (SOFTPLUS_MUFU if softplus else 0)
+            + (SILU_MUFU if has_z else 0) + (ZOH_MUFU if zoh else 0))
+
+
 def scan_bytes(batch: int, dim: int, dstate: int, seqlen: int, io_bytes: int = 2,
                bc_bytes: int = 2, has_z: bool = True, last_state: bool = False,
                start_state: bool = False) -> int:
@@ -107,4 +117,15 @@ def ssd_chunk_flops(batch: int, seqlen: int, nheads: int, headdim: int = 64,
     last chunk is padded)."""
     chunks = -(-seqlen // chunk)
     per = 2 * (chunk * chunk * dstate + chunk * chunk * headdim + 2 * dstate * chunk * headdim)
+    return batch * nheads * chunks * per
+
+
+def ssd_issued_flops(batch: int, seqlen: int, nheads: int, headdim: int = 64,
+                     dstate: int = 128, chunk: int = 128) -> int:
+    """Tensor-core FLOPs the Mamba-2 layer kernel issues per pass.  The three
+    operands it computes (the masked matrix, the weighted input and the state
+    copy) enter as bf16 hi/lo pairs, so the three products that take them are
+    issued twice; C B^T, whose operands are inputs, once."""
+    chunks = -(-seqlen // chunk)
+    per = 2 * (chunk * chunk * dstate + 2 * (chunk * chunk * headdim + 2 * dstate * chunk * headdim))
     return batch * nheads * chunks * per

@@ -39,17 +39,16 @@ def tol_for(dtype) -> float:
     return FP32_TOL if dtype == torch.float32 else BF16_TOL
 
 
-# Products on the tensor cores round a computed operand (the masked intra-chunk
-# matrix, the state copy, the weighted input) to bf16 before it is multiplied,
-# so an output that cancels across many terms can carry an error near
-# 2^-9 x (sum of the terms' magnitudes), far above 2^-9 x |output|.  Those
-# paths are held to a componentwise bound instead: the same recurrence run on
-# the absolute values of the inputs gives, per element, the sum of the
-# magnitudes of every term that reaches it, and the error must stay below
-# SCALED_TOL times that sum.  One bf16 rounding of an operand (2^-9) plus the
-# rounding of the output (2^-9) give at most 2^-8 of it; SCALED_TOL = 2^-7
-# leaves a factor of two.
-SCALED_TOL = 2.0 ** -7
+# A second, componentwise bound for the Mamba-2 layer on the tensor cores: the
+# same recurrence run on the absolute values of the inputs gives, per element,
+# the sum of the magnitudes of every term that reaches it, and the error must
+# stay below SCALED_TOL times that sum.  The kernel carries each operand it
+# computes (the masked intra-chunk matrix, the state copy, the weighted input)
+# as a bf16 hi/lo pair, good to about 2^-17, so the bf16 rounding of the output
+# (2^-9 of |output|, which the sum bounds) is the only rounding at that level;
+# SCALED_TOL = 2^-8 leaves a factor of two.  The layer's tests apply it beside
+# the max_rel_err gate above (2e-2 for bf16 inputs with the fp32 state).
+SCALED_TOL = 2.0 ** -8
 
 
 def max_scaled_err(got, want, scale) -> float:

@@ -1,6 +1,11 @@
 """Mamba-2 layer (scalar A per head) on the tensor cores: CUDA path through the C
-ABI vs the float64 oracle's recurrence, under the componentwise bound of
-``parity.SCALED_TOL`` (error at most 2^-7 of the summed term magnitudes).
+ABI vs the float64 oracle's recurrence.  Every case must meet both gates: the
+max relative error of ``parity.max_rel_err`` at most ``BF16_TOL`` (2e-2, bf16
+inputs with the fp32 state) on the output and on the final state, and the
+componentwise bound of ``parity.SCALED_TOL`` (error at most 2^-8 of the summed
+term magnitudes).  The final state, which the kernel keeps in fp32 and builds
+from hi/lo operand pairs, is further held to 1e-3 (``FINAL_STATE_TOL``): a
+single bf16 rounding of the weighted input would leave it near 1.5e-2.
 
 Cases: the small three-chunk workload (ragged last chunk, two groups, start
 state), every optional input off in turn, lengths at and around the chunk
@@ -13,13 +18,14 @@ import pytest
 import torch
 
 from oracle import oracle
-from parity import SCALED_TOL, max_scaled_err
+from parity import BF16_TOL, SCALED_TOL, max_rel_err, max_scaled_err
 from selective_state_space_55_b200 import ops
 from selective_state_space_55_b200.inputs import SSD_CONFIGS, make_ssd_inputs
 
 pytestmark = pytest.mark.gpu
 
 DEV = "cuda"
+FINAL_STATE_TOL = 1e-3
 
 
 @pytest.fixture(scope="module")
@@ -70,7 +76,9 @@ def check(ref, p, softplus=True, what=""):
     s_out, s_final = magnitude(ref, p, softplus)
     e_out, e_fin = max_scaled_err(out, o_out, s_out), max_scaled_err(final, o_final, s_final)
     assert e_out <= SCALED_TOL and e_fin <= SCALED_TOL, (what, e_out, e_fin)
-    return e_out, e_fin
+    r_out, r_fin = max_rel_err(out, o_out), max_rel_err(final, o_final)
+    assert r_out <= BF16_TOL and r_fin <= FINAL_STATE_TOL, (what, r_out, r_fin)
+    return r_out, r_fin
 
 
 def small(**kw):
@@ -139,6 +147,8 @@ def test_split_equals_whole(ref):
     assert max_scaled_err(final2, final.cpu(), s_final) <= SCALED_TOL
     assert max_scaled_err(joined, o_out, s_out) <= SCALED_TOL
     assert max_scaled_err(final2, o_final, s_final) <= SCALED_TOL
+    assert max_rel_err(joined, o_out) <= BF16_TOL
+    assert max_rel_err(final2, o_final) <= FINAL_STATE_TOL
 
 
 def test_empty_sequence_keeps_state():
@@ -179,6 +189,9 @@ def test_mamba2_layer_sampled_chains(ref):
         e_out = max_scaled_err(out[b:b + 1, :, h:h + 1], o_out, s_out)
         e_fin = max_scaled_err(final[b:b + 1, h:h + 1], o_final, s_final)
         assert e_out <= SCALED_TOL and e_fin <= SCALED_TOL, ((b, h), e_out, e_fin)
+        r_out = max_rel_err(out[b:b + 1, :, h:h + 1], o_out)
+        r_fin = max_rel_err(final[b:b + 1, h:h + 1], o_final)
+        assert r_out <= BF16_TOL and r_fin <= FINAL_STATE_TOL, ((b, h), r_out, r_fin)
 
 
 def test_rejects_unsupported_shape():

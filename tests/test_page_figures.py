@@ -84,7 +84,8 @@ def test_mamba2_layer_byte_and_flop_counts():
     """The Mamba-2 layer's algorithmic bytes and issued tensor FLOPs on the 2.7B
     layer shape, counted by hand: per (token, head) x, z, out (64 bf16 each) and
     dt (one bf16); per token B and C (128 bf16 each, one group); the final fp32
-    state of every head; per 128-token chunk and head four dense products."""
+    state of every head; per 128-token chunk and head four dense products, three
+    of them issued twice (hi and lo halves of a computed operand)."""
     from selective_state_space_55_b200 import roofline as R
     batch, L, H, P, N, Q = 16, 2048, 80, 64, 128, 128
     tokens = batch * L
@@ -95,3 +96,7 @@ def test_mamba2_layer_byte_and_flop_counts():
     products = Q * Q * N + Q * Q * P + N * Q * P + Q * N * P   # C B^T, Gm x, B^T Xw, C H^T
     assert R.ssd_chunk_flops(batch, L, H, P, N, Q) == 2 * products * batch * H * chunks
     assert R.ssd_chunk_flops(batch, L, H, P, N, Q) / (tokens * H * P) == 1280
+    # issued: the products of Gm x, B^T Xw and C H^T twice (hi and lo operands)
+    issued = Q * Q * N + 2 * (Q * Q * P + N * Q * P + Q * N * P)
+    assert R.ssd_issued_flops(batch, L, H, P, N, Q) == 2 * issued * batch * H * chunks
+    assert R.ssd_issued_flops(batch, L, H, P, N, Q) / (tokens * H * P) == 2048

@@ -86,12 +86,14 @@ def test_noalloc_matches_workspace_entry_point(name):
 def test_noalloc_refuses_problems_beyond_its_scratch():
     # Chained segments keep 64 bytes of carry per chain: 64 x 4096 chains need
     # 16 MiB, twice what the array holds.  The call must refuse before it
-    # touches any buffer, so these placeholder pointers are never used.
+    # touches any buffer, so these placeholder pointers are never used; u and
+    # delta are NULL, so that even a call that got past the size check would
+    # stop at the argument check (MAMBA_ERR_INVALID_ARG) before any launch.
     batch, dim, L = 64, 4096, 4096
     assert ops.scan_workspace_bytes(batch, dim, 16, L, num_chunks=2) > SCRATCH_BYTES
     dims = ops.make_scan_dims(batch, dim, 16, L, torch.bfloat16, torch.bfloat16, 2, 0)
     fake = ctypes.c_void_p(0x10000)
-    rc = noalloc_fn()(fake, fake, fake, fake, fake, None, None, None, 1, fake, None,
+    rc = noalloc_fn()(None, None, fake, fake, fake, None, None, None, 1, fake, None,
                       ctypes.byref(dims), None)
     assert rc == MAMBA_ERR_TOO_LARGE
     assert ops.status_string(rc) == "MAMBA_ERR_TOO_LARGE"
