@@ -7,18 +7,20 @@
 // (the tensor cores' work), and only the (headdim x dstate) state crosses
 // from one chunk to the next.
 //
-// One CTA of 128 threads owns one (batch, head) chain and walks its chunks
-// of Q = 128 tokens in order.  Per chunk, with c_i the running log2-decay
-// (c_i = log2(e) A_h sum_{r<=i} Delta_r inside the chunk) and H the state
-// entering the chunk (fp32, thread n holds row n of H^T):
+// One CTA of 256 threads owns one (batch, head) chain and walks its chunks
+// of Q = 128 tokens in order; two threads serve each of the 128 TMEM lanes,
+// each with half of the head dimension.  Per chunk, with c_i the running
+// log2-decay (c_i = log2(e) A_h sum_{r<=i} Delta_r inside the chunk) and H the
+// state entering the chunk (fp32 in registers, lane n holds row n of H^T):
 //
-//   Yoff  = C H^T                       (Q x P,  K = dstate)        MMA 3
+//   Y     = C H^T                       (Q x P,  K = dstate)        MMA 3
 //   S^T   = B^T Xw, Xw_j = 2^(c_Q - c_j) Delta_j x_j   (N x P, K = Q) MMA 4
 //   G     = C B^T                       (Q x Q,  K = dstate)        MMA 1
 //   Gm_ij = G_ij 2^(c_i - c_j) Delta_j  for j <= i, else 0,
 //           plus D_h on the diagonal    (CUDA cores)
-//   Ydiag = Gm X  (= intra-chunk part + D_h x)  (Q x P, K = Q)      MMA 2
-//   y_i   = Ydiag_i + 2^(c_i) Yoff_i,  out = y silu(z)
+//   Y_i  <- 2^(c_i) Y_i                 (CUDA cores, in tensor memory)
+//   Y    += Gm X  (intra-chunk part + D_h x)  (Q x P, K = Q)        MMA 2
+//   out   = Y silu(z)
 //   H     = 2^(c_Q) H + S               (fp32, in registers)
 //
 // Precision.  The tensor cores multiply bf16 operands.  C, B and x are bf16
@@ -52,17 +54,17 @@ namespace mamba {
 constexpr int kSsdP = 64;          // head dimension
 constexpr int kSsdN = 128;         // state size
 constexpr int kSsdQ = 128;         // chunk length
-constexpr int kSsdThreads = 128;   // one thread per TMEM lane
+constexpr int kSsdThreads = 256;   // two threads per TMEM lane
 constexpr int kSsdTmemCols = 256;
 
 // Tensor-memory columns (fp32 unless packed).  G fills [0, 128) until the
 // masked matrix has been formed from it; Gm's lo half (bf16 pairs, K = j)
-// then takes [0, 64) and MMA 2 writes Ydiag to [64, 128).  S fills
-// [192, 256) until the state update has read it; Gm's hi half then takes it.
+// then takes [0, 64).  S fills [192, 256) until the state update has read it;
+// Gm's hi half then takes it.  Y holds C H^T, is scaled in place by 2^(c_i)
+// per row, and MMA 2 accumulates Gm X onto it: the output before the gate.
 constexpr uint32_t kTmG = 0;
 constexpr uint32_t kTmGmLo = 0;
-constexpr uint32_t kTmYdiag = 64;
-constexpr uint32_t kTmYoff = 128;
+constexpr uint32_t kTmY = 128;
 constexpr uint32_t kTmS = 192;
 constexpr uint32_t kTmGmHi = 192;
 
@@ -81,7 +83,7 @@ constexpr int kSsdOffHX = 81920;     // hi at +0, lo at +16384, each 128 x 64 bf
 constexpr int kSsdOffE = 114688;     // 128 fp32: -e_j, e_j = c_j - log2(Delta_j)
 constexpr int kSsdOffBar = 115200;   // 8 mbarriers (see SsdBar)
 constexpr int kSsdOffSlot = 115264;  // TMEM base address written by tcgen05.alloc
-constexpr int kSsdOffTot = 115280;   // 4 fp32 warp totals of the decay prefix sum
+constexpr int kSsdOffTot = 115280;   // 2 x 4 fp32 warp totals of the decay prefix sum
 constexpr int kSsdSmemBytes = 115328;
 constexpr uint32_t kSsdLoBytes = 16384;   // offset of the lo half in the HX buffer
 
@@ -217,25 +219,6 @@ __device__ __forceinline__ void tma_store_tile(const CUtensorMap* map, uint32_t 
         : "memory");
 }
 
-// Two 32-column loads of this thread's TMEM lane and one wait: both arrays
-// are valid when the statement ends.
-__device__ __forceinline__ void tmem_ld32x2(uint32_t ta, uint32_t tb, float (&a)[32],
-                                            float (&b)[32]) {
-    uint32_t ra[32], rb[32];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%64];\n\t"
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
-        : "=r"(ra[0]), "=r"(ra[1]), "=r"(ra[2]), "=r"(ra[3]), "=r"(ra[4]), "=r"(ra[5]), "=r"(ra[6]), "=r"(ra[7]), "=r"(ra[8]), "=r"(ra[9]), "=r"(ra[10]), "=r"(ra[11]), "=r"(ra[12]), "=r"(ra[13]), "=r"(ra[14]), "=r"(ra[15]), "=r"(ra[16]), "=r"(ra[17]), "=r"(ra[18]), "=r"(ra[19]), "=r"(ra[20]), "=r"(ra[21]), "=r"(ra[22]), "=r"(ra[23]), "=r"(ra[24]), "=r"(ra[25]), "=r"(ra[26]), "=r"(ra[27]), "=r"(ra[28]), "=r"(ra[29]), "=r"(ra[30]), "=r"(ra[31]), "=r"(rb[0]), "=r"(rb[1]), "=r"(rb[2]), "=r"(rb[3]), "=r"(rb[4]), "=r"(rb[5]), "=r"(rb[6]), "=r"(rb[7]), "=r"(rb[8]), "=r"(rb[9]), "=r"(rb[10]), "=r"(rb[11]), "=r"(rb[12]), "=r"(rb[13]), "=r"(rb[14]), "=r"(rb[15]), "=r"(rb[16]), "=r"(rb[17]), "=r"(rb[18]), "=r"(rb[19]), "=r"(rb[20]), "=r"(rb[21]), "=r"(rb[22]), "=r"(rb[23]), "=r"(rb[24]), "=r"(rb[25]), "=r"(rb[26]), "=r"(rb[27]), "=r"(rb[28]), "=r"(rb[29]), "=r"(rb[30]), "=r"(rb[31])
-        : "r"(ta), "r"(tb)
-        : "memory");
-#pragma unroll
-    for (int k = 0; k < 32; ++k) {
-        a[k] = __uint_as_float(ra[k]);
-        b[k] = __uint_as_float(rb[k]);
-    }
-}
-
 // 16 consecutive 32-bit columns of this thread's TMEM lane from registers.
 // Complete (visible to the tensor cores after a fence and barrier) once
 // tmem_wait_st returns.
@@ -276,31 +259,63 @@ __device__ __forceinline__ void split16(const float (&f)[8], uint4& hi, uint4& l
     split_bf16x2(f[6], f[7], hi.w, lo.w);
 }
 
-// The state H of this thread's row n as its bf16 hi/lo pair into the HX
-// buffer (row n, 64 columns p per half).
-__device__ __forceinline__ void ssd_store_state(unsigned char* smem, int n, const float (&H)[kSsdP]) {
+// This thread's half of row n of H^T (columns p = 32 hp .. 32 hp + 31) as
+// its bf16 hi/lo pair into the HX buffer.
+__device__ __forceinline__ void ssd_store_state(unsigned char* smem, int n, int hp,
+                                                const float (&H)[kSsdP / 2]) {
 #pragma unroll
-    for (int q = 0; q < kSsdP / 8; ++q) {
+    for (int q = 0; q < kSsdP / 16; ++q) {
         float f[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) f[k] = H[q * 8 + k];
         uint4 hi, lo;
         split16(f, hi, lo);
-        const uint32_t off = ssd_sw128(n, q);
+        const uint32_t off = ssd_sw128(n, 4 * hp + q);
         *reinterpret_cast<uint4*>(smem + kSsdOffHX + off) = hi;
         *reinterpret_cast<uint4*>(smem + kSsdOffHX + kSsdLoBytes + off) = lo;
     }
 }
 
+// One 32-column load of this thread's TMEM lane; valid when it returns.
+__device__ __forceinline__ void tmem_ld32(uint32_t ta, float (&a)[32]) {
+    uint32_t ra[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(ra[0]), "=r"(ra[1]), "=r"(ra[2]), "=r"(ra[3]), "=r"(ra[4]), "=r"(ra[5]), "=r"(ra[6]), "=r"(ra[7]), "=r"(ra[8]), "=r"(ra[9]), "=r"(ra[10]), "=r"(ra[11]), "=r"(ra[12]), "=r"(ra[13]), "=r"(ra[14]), "=r"(ra[15]), "=r"(ra[16]), "=r"(ra[17]), "=r"(ra[18]), "=r"(ra[19]), "=r"(ra[20]), "=r"(ra[21]), "=r"(ra[22]), "=r"(ra[23]), "=r"(ra[24]), "=r"(ra[25]), "=r"(ra[26]), "=r"(ra[27]), "=r"(ra[28]), "=r"(ra[29]), "=r"(ra[30]), "=r"(ra[31])
+        : "r"(ta)
+        : "memory");
+#pragma unroll
+    for (int k = 0; k < 32; ++k) a[k] = __uint_as_float(ra[k]);
+}
+
+// 32 consecutive columns of this thread's TMEM lane from fp32 registers.
+__device__ __forceinline__ void tmem_st32f(uint32_t taddr, const float (&a)[32]) {
+    uint32_t lo[16], hi[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        lo[k] = __float_as_uint(a[k]);
+        hi[k] = __float_as_uint(a[16 + k]);
+    }
+    tmem_st16(taddr, lo);
+    tmem_st16(taddr + 16, hi);
+}
+
 // Wait for one completion of an mbarrier; true on every thread if any
-// thread's bounded wait gave up.  Also a CTA-wide barrier.
+// thread's bounded wait gave up.  Also a CTA-wide barrier, which orders this
+// thread's earlier tensor-memory accesses before the other threads' later ones.
 __device__ __forceinline__ bool ssd_wait_failed(uint32_t bar, uint32_t parity) {
     const bool ok = mbar_wait_bounded(bar, parity);
+    tc_fence_before();
     const bool failed = __syncthreads_or(!ok) != 0;
     tc_fence_after();
     return failed;
 }
 
+// Two threads serve each TMEM lane (row) r: threads r and r + 128 ("halves"
+// hp = 0, 1), each with half of the head dimension (columns 32 hp .. 32 hp +
+// 31 of x, Xw, H, y) and every other column quarter of the masked matrix.
+// Tensor memory is accessed by warp w in lanes 32 (w % 4) .. + 31.
 __global__ void __launch_bounds__(kSsdThreads, 2)
     ssd_chunk_scan_kernel(const __grid_constant__ SsdParams p,
                           const __grid_constant__ CUtensorMap tm_x,
@@ -310,14 +325,17 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
                           const __grid_constant__ CUtensorMap tm_out) {
     extern __shared__ __align__(1024) unsigned char smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int chain = blockIdx.x;                           // b * nheads + h
+    const int r = tid & (kSsdQ - 1);      // row: token i / j, or state index n
+    const int hp = tid >> 7;              // which half of the head dimension
+    const int wq = warp & 3;              // TMEM lane quarter of this warp
+    const int chain = blockIdx.x;         // b * nheads + h
     const int h = chain % p.nheads;
     const int b = chain / p.nheads;
     const int g = h / (p.nheads / p.ngroups);
     const int64_t L = p.seqlen;
     const uint32_t s0 = smem_u32(smem);
     float* sE = reinterpret_cast<float*>(smem + kSsdOffE);
-    float* sTot = reinterpret_cast<float*>(smem + kSsdOffTot);
+    float* sTot = reinterpret_cast<float*>(smem + kSsdOffTot) + 4 * hp;
     const uint32_t bar0 = s0 + kSsdOffBar;
     auto bar = [bar0](int k) -> uint32_t { return bar0 + 8u * (uint32_t)k; };
     const uint32_t* tslot = reinterpret_cast<const uint32_t*>(smem + kSsdOffSlot);
@@ -338,18 +356,18 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tslot;
-    const uint32_t tlane = tmem + ((uint32_t)(warp * 32) << 16);   // this warp's 32 lanes
+    const uint32_t tlane = tmem + ((uint32_t)(wq * 32) << 16);   // this warp's 32 lanes
 
     const float A2 = p.A[h] * kLog2e;
     const float Dh = p.D ? p.D[h] : 0.0f;
     const float bias = p.dt_bias ? p.dt_bias[h] : 0.0f;
 
-    // Thread n holds row n of H^T: H[q] = state[q][n], in fp32.
-    float H[kSsdP];
-    const size_t hoff = (size_t)chain * kSsdP * kSsdN + tid;
+    // This thread holds H[q] = state[32 hp + q][r], in fp32.
+    float H[kSsdP / 2];
+    const size_t hoff = ((size_t)chain * kSsdP + 32 * hp) * kSsdN + r;
 #pragma unroll
-    for (int q = 0; q < kSsdP; ++q) H[q] = p.h0 ? p.h0[hoff + (size_t)q * kSsdN] : 0.0f;
-    ssd_store_state(smem, tid, H);
+    for (int q = 0; q < kSsdP / 2; ++q) H[q] = p.h0 ? p.h0[hoff + (size_t)q * kSsdN] : 0.0f;
+    ssd_store_state(smem, r, hp, H);
     fence_proxy_async_smem();
 
     const int64_t nchunks = (L + kSsdQ - 1) / kSsdQ;
@@ -368,11 +386,12 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
     // K-major operand, K step k of 16 columns: 32 bytes along the swizzled
     // 128-byte rows, the second 64 columns one half (16 KB) further.
     auto kmaj = [](int k) -> uint32_t { return (uint32_t)((k >> 2) * 16384 + (k & 3) * 32); };
-    // dt of this thread's token in the next chunk, loaded one chunk ahead.
+    // dt of this row's token in the next chunk, loaded one chunk ahead (both
+    // halves of a row load and compute the same values).
     auto load_dt = [&](int64_t l) -> float {
         return l < L ? __bfloat162float(p.dt[((int64_t)b * L + l) * p.nheads + h]) : 0.0f;
     };
-    float dt_next = load_dt(tid);
+    float dt_next = load_dt(r);
 
     if (nchunks > 0) {
         if (tid == 0) {
@@ -398,16 +417,16 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
         const bool more = c + 1 < nchunks;
 
         // ---- C landed (the barrier also publishes the entering state's hi/lo
-        // pair): MMA 3, Yoff = C (H_hi + H_lo)^T.
+        // pair): MMA 3, Y = C (H_hi + H_lo)^T.
         if (wait_on(kBarC)) { failed = true; break; }
         if (tid == 0) {
 #pragma unroll
             for (int k = 0; k < kSsdN / 16; ++k)
-                umma_bf16(tmem + kTmYoff, umma_sdesc_sw128(s0 + kSsdOffC + kmaj(k), 16, 1024),
+                umma_bf16(tmem + kTmY, umma_sdesc_sw128(s0 + kSsdOffC + kmaj(k), 16, 1024),
                           umma_sdesc_sw128(s0 + kSsdOffHX + k * 2048, 16384, 1024), id_off, k);
 #pragma unroll
             for (int k = 0; k < kSsdN / 16; ++k)
-                umma_bf16(tmem + kTmYoff, umma_sdesc_sw128(s0 + kSsdOffC + kmaj(k), 16, 1024),
+                umma_bf16(tmem + kTmY, umma_sdesc_sw128(s0 + kSsdOffC + kmaj(k), 16, 1024),
                           umma_sdesc_sw128(s0 + kSsdOffHX + kSsdLoBytes + k * 2048, 16384, 1024),
                           id_off, 1);
             umma_commit(bar(kBarYoff));
@@ -417,43 +436,44 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
         // ---- Delta, the running log2-decay c_i and e_i = c_i - log2(Delta_i),
         // while MMA 3 runs.
         float delta = 0.0f;
-        if (l0 + tid < L) {
+        if (l0 + r < L) {
             const float sarg = dt_next + bias;
             delta = p.softplus ? softplus_f32(sarg) : sarg;
         }
-        dt_next = load_dt((int64_t)l0 + kSsdQ + tid);
+        dt_next = load_dt((int64_t)l0 + kSsdQ + r);
         float a = delta * A2;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const float v = __shfl_up_sync(0xffffffffu, a, o);
             if (lane >= o) a += v;
         }
-        if (lane == 31) sTot[warp] = a;
+        if (lane == 31) sTot[wq] = a;
         __syncthreads();
         float pre = 0.0f;
-        for (int w = 0; w < warp; ++w) pre += sTot[w];
+        for (int w = 0; w < wq; ++w) pre += sTot[w];
         const float ci = a + pre;
         const float cQ = (sTot[0] + sTot[1]) + (sTot[2] + sTot[3]);
         const float e_own = ci - lg2_approx(delta);   // +inf for Delta = 0
-        sE[tid] = -e_own;                              // stored negated: c_i - e_j is an add
+        if (hp == 0) sE[r] = -e_own;                   // stored negated: c_i - e_j is an add
 
         // ---- x landed and MMA 3 is done with the HX buffer: Xw_j hi/lo
-        // (row j = tid), Xw_j = 2^(c_Q - e_j) x_j = 2^(c_Q - c_j) Delta_j x_j.
+        // (row j = r, this half's columns), Xw_j = 2^(c_Q - e_j) x_j; and
+        // Y_i = 2^(c_i) Y_i in place, onto which MMA 2 will accumulate.
         if (wait_on(kBarX)) { failed = true; break; }
         if (wait_on(kBarYoff)) { failed = true; break; }
         {
             const float w = ex2_approx(cQ - e_own);
             const float2 w2 = make_float2(w, w);
 #pragma unroll
-            for (int pb = 0; pb < kSsdP / 8; ++pb) {
-                const uint32_t off = ssd_sw128(tid, pb);
+            for (int q = 0; q < 4; ++q) {
+                const uint32_t off = ssd_sw128(r, 4 * hp + q);
                 float f[8];
                 unpack16(*reinterpret_cast<const uint4*>(smem + kSsdOffX + off), f);
 #pragma unroll
                 for (int k = 0; k < 8; k += 2) {
-                    const float2 r = __fmul2_rn(make_float2(f[k], f[k + 1]), w2);
-                    f[k] = r.x;
-                    f[k + 1] = r.y;
+                    const float2 v = __fmul2_rn(make_float2(f[k], f[k + 1]), w2);
+                    f[k] = v.x;
+                    f[k + 1] = v.y;
                 }
                 uint4 hi, lo;
                 split16(f, hi, lo);
@@ -462,6 +482,19 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
             }
         }
         fence_proxy_async_smem();
+        {
+            const float sc = ex2_approx(ci);
+            const float2 sc2 = make_float2(sc, sc);
+            float y[32];
+            tmem_ld32(tlane + kTmY + 32 * hp, y);
+#pragma unroll
+            for (int k = 0; k < 32; k += 2) {
+                const float2 v = __fmul2_rn(make_float2(y[k], y[k + 1]), sc2);
+                y[k] = v.x;
+                y[k + 1] = v.y;
+            }
+            tmem_st32f(tlane + kTmY + 32 * hp, y);
+        }
 
         // ---- B landed (the barrier also publishes Xw and e): MMA 4,
         // S^T = B^T (Xw_hi + Xw_lo), committed alone, then MMA 1, G = C B^T.
@@ -486,27 +519,23 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
         issued(kBarS);
         issued(kBarG);
 
-        // ---- state: H = 2^(c_Q) H + S (row n = tid), in registers while MMA 1
-        // runs; its hi/lo pair goes to the HX buffer, which MMA 4 no longer reads,
-        // for the next chunk's MMA 3.
+        // ---- state: H = 2^(c_Q) H + S (row n = r, this half's columns), in
+        // registers while MMA 1 runs; its hi/lo pair goes to the HX buffer,
+        // which MMA 4 no longer reads, for the next chunk's MMA 3.
         if (wait_on(kBarS)) { failed = true; break; }
         {
             const float dq = ex2_approx(cQ);
-            float s_lo[32], s_hi[32];
-            tmem_ld32x2(tlane + kTmS, tlane + kTmS + 32, s_lo, s_hi);
+            float sv[32];
+            tmem_ld32(tlane + kTmS + 32 * hp, sv);
             const float2 dq2 = make_float2(dq, dq);
 #pragma unroll
             for (int k = 0; k < 32; k += 2) {
-                const float2 lo = __ffma2_rn(dq2, make_float2(H[k], H[k + 1]), make_float2(s_lo[k], s_lo[k + 1]));
-                const float2 hi = __ffma2_rn(dq2, make_float2(H[32 + k], H[33 + k]),
-                                             make_float2(s_hi[k], s_hi[k + 1]));
-                H[k] = lo.x;
-                H[k + 1] = lo.y;
-                H[32 + k] = hi.x;
-                H[33 + k] = hi.y;
+                const float2 v = __ffma2_rn(dq2, make_float2(H[k], H[k + 1]), make_float2(sv[k], sv[k + 1]));
+                H[k] = v.x;
+                H[k + 1] = v.y;
             }
         }
-        ssd_store_state(smem, tid, H);
+        ssd_store_state(smem, r, hp, H);
         fence_proxy_async_smem();
 
         // ---- MMA 1 done: C and B are free.  Next chunk's C; this chunk's gate
@@ -525,75 +554,74 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
         if (more) issued(kBarC);
         if (has_z) issued(kBarZ);
 
-        // ---- Gm_ij = G_ij 2^(c_i - e_j) for j <= i (row i = tid), as hi/lo
-        // pairs into tensor memory.  Warp w holds rows [32w, 32w + 32): quarters
-        // of columns below w are entirely at or below the diagonal, quarter w
-        // straddles it, and the quarters above are zero (no TMEM read, no
-        // exponentials).  G is read one column half at a time; the half's lo
-        // words land in columns whose G values this lane has already read.
+        // ---- Gm_ij = G_ij 2^(c_i - e_j) for j <= i (row i = r), as hi/lo pairs
+        // into tensor memory.  Rows [32 wq, 32 wq + 32) need column quarters
+        // 0 .. wq (quarter wq straddles the diagonal); the quarters above are
+        // zero.  This half takes quarters hp and hp + 2, so no warp forms more
+        // than two.  The hi words go to the S columns at once; the lo words
+        // overwrite G's first half, so they wait until both halves have read G.
+        uint32_t keep_lo[2][16];
         {
             const float2 ci2 = make_float2(ci, ci);
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                const int qa = 2 * hf;
-                float gv[2][32];
-                if (qa <= warp) tmem_ld32x2(tlane + kTmG + qa * 32, tlane + kTmG + qa * 32 + 32,
-                                            gv[0], gv[1]);
+            for (int s = 0; s < 2; ++s) {
+                const int quarter = hp + 2 * s;
+                uint32_t hi[16];
+                if (quarter > wq) {
 #pragma unroll
-                for (int s = 0; s < 2; ++s) {
-                    const int quarter = qa + s;
-                    uint32_t hi[16], lo[16];
-                    if (quarter > warp) {
+                    for (int k = 0; k < 16; ++k) hi[k] = keep_lo[s][k] = 0u;
+                } else {
+                    float gv[32];
+                    tmem_ld32(tlane + kTmG + 32 * quarter, gv);
+                    const bool diag = quarter == wq;   // D_h x_i enters as Gm_ii += D_h
 #pragma unroll
-                        for (int k = 0; k < 16; ++k) hi[k] = lo[k] = 0u;
-                    } else {
-                        const bool diag = quarter == warp;   // D_h x_i enters as Gm_ii += D_h
+                    for (int q = 0; q < 4; ++q) {
+                        const int j0 = quarter * 32 + q * 8;
+                        const float4 e0 = *reinterpret_cast<const float4*>(sE + j0);
+                        const float4 e1 = *reinterpret_cast<const float4*>(sE + j0 + 4);
+                        const float2 ne[4] = {make_float2(e0.x, e0.y), make_float2(e0.z, e0.w),
+                                              make_float2(e1.x, e1.y), make_float2(e1.z, e1.w)};
+                        float f[8];
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const int j0 = quarter * 32 + q * 8;
-                            const float4 e0 = *reinterpret_cast<const float4*>(sE + j0);
-                            const float4 e1 = *reinterpret_cast<const float4*>(sE + j0 + 4);
-                            const float2 ne[4] = {make_float2(e0.x, e0.y), make_float2(e0.z, e0.w),
-                                                  make_float2(e1.x, e1.y), make_float2(e1.z, e1.w)};
-                            float f[8];
-#pragma unroll
-                            for (int k = 0; k < 8; k += 2) {
-                                const float2 arg = __fadd2_rn(ci2, ne[k / 2]);
-                                const float2 v = __fmul2_rn(
-                                    make_float2(gv[s][q * 8 + k], gv[s][q * 8 + k + 1]),
-                                    make_float2(ex2_approx(arg.x), ex2_approx(arg.y)));
-                                f[k] = v.x;
-                                f[k + 1] = v.y;
-                            }
-                            if (diag) {
-#pragma unroll
-                                for (int k = 0; k < 8; ++k)
-                                    f[k] = j0 + k < tid ? f[k] : (j0 + k == tid ? f[k] + Dh : 0.0f);
-                            }
-#pragma unroll
-                            for (int k = 0; k < 4; ++k)
-                                split_bf16x2(f[2 * k], f[2 * k + 1], hi[q * 4 + k], lo[q * 4 + k]);
+                        for (int k = 0; k < 8; k += 2) {
+                            const float2 arg = __fadd2_rn(ci2, ne[k / 2]);
+                            const float2 v = __fmul2_rn(make_float2(gv[q * 8 + k], gv[q * 8 + k + 1]),
+                                                        make_float2(ex2_approx(arg.x), ex2_approx(arg.y)));
+                            f[k] = v.x;
+                            f[k + 1] = v.y;
                         }
+                        if (diag) {
+#pragma unroll
+                            for (int k = 0; k < 8; ++k)
+                                f[k] = j0 + k < r ? f[k] : (j0 + k == r ? f[k] + Dh : 0.0f);
+                        }
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            split_bf16x2(f[2 * k], f[2 * k + 1], hi[q * 4 + k], keep_lo[s][q * 4 + k]);
                     }
-                    tmem_st16(tlane + kTmGmHi + quarter * 16, hi);
-                    tmem_st16(tlane + kTmGmLo + quarter * 16, lo);
                 }
+                tmem_st16(tlane + kTmGmHi + 16 * quarter, hi);
             }
         }
+        tc_fence_before();
+        __syncthreads();   // every G column has been read
+        tc_fence_after();
+#pragma unroll
+        for (int s = 0; s < 2; ++s) tmem_st16(tlane + kTmGmLo + 16 * (hp + 2 * s), keep_lo[s]);
         tmem_wait_st();
         tc_fence_before();
         __syncthreads();
 
-        // ---- MMA 2: Ydiag = (Gm_hi + Gm_lo) X, A from tensor memory.
+        // ---- MMA 2: Y += (Gm_hi + Gm_lo) X, A from tensor memory.
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
             for (int k = 0; k < kSsdQ / 16; ++k)
-                umma_bf16_ta(tmem + kTmYdiag, tmem + kTmGmHi + 8 * k,
-                             umma_sdesc_sw128(s0 + kSsdOffX + k * 2048, 16384, 1024), id_y, k);
+                umma_bf16_ta(tmem + kTmY, tmem + kTmGmHi + 8 * k,
+                             umma_sdesc_sw128(s0 + kSsdOffX + k * 2048, 16384, 1024), id_y, 1);
 #pragma unroll
             for (int k = 0; k < kSsdQ / 16; ++k)
-                umma_bf16_ta(tmem + kTmYdiag, tmem + kTmGmLo + 8 * k,
+                umma_bf16_ta(tmem + kTmY, tmem + kTmGmLo + 8 * k,
                              umma_sdesc_sw128(s0 + kSsdOffX + k * 2048, 16384, 1024), id_y, 1);
             umma_commit(bar(kBarYd));
         }
@@ -606,46 +634,34 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
         if (more) issued(kBarX);
         if (has_z && wait_on(kBarZ)) { failed = true; break; }
 
-        // ---- y_i = Ydiag_i + 2^(c_i) Yoff_i (D x_i is inside Ydiag), gated (row
-        // i = tid), written as bf16 over the gate tile, then stored by TMA (rows
-        // past the end dropped).
+        // ---- y_i = Y_i (row i = r, this half's columns), gated, written as
+        // bf16 over the gate tile, then stored by TMA (rows past the end dropped).
         {
-            const float sc = ex2_approx(ci);
-            const float2 sc2 = make_float2(sc, sc);
+            float y[32];
+            tmem_ld32(tlane + kTmY + 32 * hp, y);
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                float yd[32], yo[32];
-                tmem_ld32x2(tlane + kTmYdiag + half * 32, tlane + kTmYoff + half * 32, yd, yo);
+            for (int q = 0; q < 4; ++q) {
+                const uint32_t off = ssd_sw128(r, 4 * hp + q);
+                float f[8];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int pb = half * 4 + q;
-                    const uint32_t off = ssd_sw128(tid, pb);
-                    float f[8];
+                for (int k = 0; k < 8; ++k) f[k] = y[q * 8 + k];
+                if (has_z) {
+                    // silu(z) = z / (1 + 2^(-z log2 e)), two lanes at a time
+                    float zv[8];
+                    unpack16(*reinterpret_cast<const uint4*>(smem + kSsdOffB + off), zv);
 #pragma unroll
                     for (int k = 0; k < 8; k += 2) {
-                        const float2 r = __ffma2_rn(sc2, make_float2(yo[q * 8 + k], yo[q * 8 + k + 1]),
-                                                    make_float2(yd[q * 8 + k], yd[q * 8 + k + 1]));
-                        f[k] = r.x;
-                        f[k + 1] = r.y;
+                        const float2 z2 = make_float2(zv[k], zv[k + 1]);
+                        const float2 t = __fmul2_rn(z2, make_float2(-kLog2e, -kLog2e));
+                        const float2 d = __fadd2_rn(make_float2(ex2_approx(t.x), ex2_approx(t.y)),
+                                                    make_float2(1.0f, 1.0f));
+                        const float2 g2 = __fmul2_rn(z2, make_float2(rcp_approx(d.x), rcp_approx(d.y)));
+                        const float2 v = __fmul2_rn(make_float2(f[k], f[k + 1]), g2);
+                        f[k] = v.x;
+                        f[k + 1] = v.y;
                     }
-                    if (has_z) {
-                        // silu(z) = z / (1 + 2^(-z log2 e)), two lanes at a time
-                        float zv[8];
-                        unpack16(*reinterpret_cast<const uint4*>(smem + kSsdOffB + off), zv);
-#pragma unroll
-                        for (int k = 0; k < 8; k += 2) {
-                            const float2 z2 = make_float2(zv[k], zv[k + 1]);
-                            const float2 t = __fmul2_rn(z2, make_float2(-kLog2e, -kLog2e));
-                            const float2 d = __fadd2_rn(make_float2(ex2_approx(t.x), ex2_approx(t.y)),
-                                                        make_float2(1.0f, 1.0f));
-                            const float2 g2 = __fmul2_rn(z2, make_float2(rcp_approx(d.x), rcp_approx(d.y)));
-                            const float2 r = __fmul2_rn(make_float2(f[k], f[k + 1]), g2);
-                            f[k] = r.x;
-                            f[k + 1] = r.y;
-                        }
-                    }
-                    *reinterpret_cast<uint4*>(smem + kSsdOffB + off) = pack16(f);
                 }
+                *reinterpret_cast<uint4*>(smem + kSsdOffB + off) = pack16(f);
             }
         }
         fence_proxy_async_smem();
@@ -665,7 +681,7 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
 
     if (!failed && p.hT) {
 #pragma unroll
-        for (int q = 0; q < kSsdP; ++q) p.hT[hoff + (size_t)q * kSsdN] = H[q];
+        for (int q = 0; q < kSsdP / 2; ++q) p.hT[hoff + (size_t)q * kSsdN] = H[q];
     }
     if (tid == 0) {
         bulk_wait<0>();   // output stores done before the CTA's shared memory goes
