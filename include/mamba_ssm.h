@@ -88,7 +88,8 @@ typedef enum {
 /* Flags (mamba_dims_t.flags). */
 #define MAMBA_FLAG_NO_TMA 0x1          /* plain loads instead of TMA (scan tiles; the
                                           * update's bulk streaming path) */
-#define MAMBA_FLAG_PARALLEL_CHUNKS 0x2 /* with num_chunks >= 1: parallel (recompute) mode */
+#define MAMBA_FLAG_PARALLEL_CHUNKS 0x2 /* with num_chunks >= 1: parallel mode (segments at
+                                          * once, carry scan, correction) */
 /* Test only: in mode 0, segments never hand their state on, so every wait for
  * a predecessor runs out (after ~0.3 s) and the call reports MAMBA_ERR_TIMEOUT
  * through mamba_device_status().  Outputs are then undefined. */
@@ -149,22 +150,30 @@ typedef struct {
  *   mode 0 (chained): one launch.  Segment k of a group starts from the state
  *     segment k-1 left in the workspace; no work is repeated.  Used when there
  *     are enough groups to occupy the GPU; nchunks only balances the load.
- *   mode 1 (parallel): two launches, for few channels and long sequences.
- *     Pass A runs segments 0..nchunks-2 at once: segment 0 writes its outputs
- *     and end state, the others only their end state from a zero start and
- *     the sum of Delta.  Pass B runs segments 1..nchunks-1 at once, each
- *     folding the earlier segments' (exp(A sum Delta), end state) pairs into
- *     its true start state before recomputing its outputs.
+ *   mode 1 (parallel): three launches, for few channels and long sequences.
+ *     1. Every segment runs at once from a zero start (segment 0 from the
+ *        start state), writes its outputs and keeps its end state and its
+ *        sum of Delta (units_pass_a items).
+ *     2. One warp per chain scans the segments' (exp(A sum Delta), end state)
+ *        pairs with warp shuffles (the associative combine of the parallel
+ *        scan): each segment's true start state, and last_state.
+ *     3. Each later segment adds its start state's contribution,
+ *        C_t . (exp(A S_t) h_in) with S_t the sum of Delta since the segment
+ *        began, to its outputs (units_pass_b items, one per chain and
+ *        segment), stopping where exp(A S_t) has underflowed in fp32 for
+ *        every state entry (when Delta >= 0 throughout, i.e. softplus on).
+ *     Nothing is computed twice; the correction costs as much per step as
+ *     the scan but covers only the steps over which the start state matters.
  */
 typedef struct {
     int32_t nchunks;           /* segments per sequence */
     int32_t tile_len;          /* time steps staged per pipeline stage */
     int64_t chunk_len;         /* time steps per segment (multiple of tile_len) */
     int64_t groups;            /* batch * ceil(dim / 32) */
-    int64_t units_pass_a;      /* work items of the first launch */
-    int64_t units_pass_b;      /* work items of the second launch (0 in mode 0) */
+    int64_t units_pass_a;      /* work items of the first launch (group x segment) */
+    int64_t units_pass_b;      /* correction items, chain x later segment (0 in mode 0) */
     int32_t warps_per_cta;
-    int32_t launches;          /* kernel launches per call (plus one memset) */
+    int32_t launches;          /* kernel launches per call (plus one memset): 1 or 3 */
     int32_t tma_capable;       /* strides allow TMA staging */
     int32_t mode;              /* 0 chained, 1 parallel */
     int32_t channels_per_lane; /* 1 or 2: a group is 32 x this many channels */

@@ -13,6 +13,7 @@
 #include "conv1d.cuh"
 #include "scan_backward.cuh"
 #include "ssd_chunk_scan.cuh"
+#include "scan_carry.cuh"
 
 namespace mamba {
 
@@ -136,6 +137,44 @@ cudaError_t dispatch_scan(const ScanParams& prm, const CUtensorMap* maps, int cp
                : dispatch_scan_cpl<IoT, 1, false>(prm, maps, has_z, sp, want_warps, dev, sms, stream);
 }
 
+// Correction pass of the parallel mode: a persistent grid of warps that pull
+// (chain, segment) items from a counter; items are few and uneven in length
+// (each stops where its start state has decayed below fp32's range).
+template <typename IoT, typename BcT, bool kHasZ, bool kSoftplus>
+cudaError_t launch_correct(const CorrectParams& q, int dev, int sms, cudaStream_t stream) {
+    static int resident[kMaxDevices] = {0};
+    auto kernel = scan_correct_kernel<IoT, BcT, kHasZ, kSoftplus>;
+    int per_sm = (dev >= 0 && dev < kMaxDevices) ? resident[dev] : 0;
+    if (per_sm <= 0) {
+        const cudaError_t e =
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kCorrectWarps * 32, 0);
+        if (e != cudaSuccess) return e;
+        if (per_sm <= 0) return cudaErrorInvalidConfiguration;
+        if (dev >= 0 && dev < kMaxDevices) resident[dev] = per_sm;
+    }
+    const int64_t need = (q.items + kCorrectWarps - 1) / kCorrectWarps;
+    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>((int64_t)per_sm * sms, need));
+    kernel<<<(unsigned)grid, kCorrectWarps * 32, 0, stream>>>(q);
+    return cudaGetLastError();
+}
+
+template <typename IoT>
+cudaError_t dispatch_correct(const CorrectParams& q, bool has_z, bool sp, int dev, int sms,
+                             cudaStream_t stream) {
+    if (q.bc_bf16) {
+        if (has_z)
+            return sp ? launch_correct<IoT, __nv_bfloat16, true, true>(q, dev, sms, stream)
+                      : launch_correct<IoT, __nv_bfloat16, true, false>(q, dev, sms, stream);
+        return sp ? launch_correct<IoT, __nv_bfloat16, false, true>(q, dev, sms, stream)
+                  : launch_correct<IoT, __nv_bfloat16, false, false>(q, dev, sms, stream);
+    }
+    if (has_z)
+        return sp ? launch_correct<IoT, float, true, true>(q, dev, sms, stream)
+                  : launch_correct<IoT, float, true, false>(q, dev, sms, stream);
+    return sp ? launch_correct<IoT, float, false, true>(q, dev, sms, stream)
+              : launch_correct<IoT, float, false, false>(q, dev, sms, stream);
+}
+
 template <typename IoT, typename BcT, bool kHasZ, bool kZoh>
 cudaError_t launch_update_bulk(const UpdateParams& prm, int dev, int sms, bool pdl,
                                cudaStream_t stream) {
@@ -223,8 +262,8 @@ cudaError_t dispatch_update(const UpdateParams& prm, bool bc_bf16, bool fast, bo
 struct ScanWorkspace {
     size_t zeroed;      // prefix cleared before every call: counters and flags
     size_t carry;       // chained mode: [chains][16] fp32
-    size_t ws_h;        // parallel mode: [K-1][chains][16] fp32
-    size_t ws_sdt;      // parallel mode: [K-1][chains] fp32
+    size_t ws_h;        // parallel mode: [K][chains][16] fp32
+    size_t ws_sdt;      // parallel mode: [K][chains] fp32
     size_t total;
 };
 
@@ -239,9 +278,9 @@ ScanWorkspace scan_workspace_layout(const mamba_dims_t* dims, int64_t groups, in
     }
     if (mode == 1) {
         w.ws_h = off;
-        off += align256((size_t)(K - 1) * chains * kNPad * sizeof(float));
+        off += align256((size_t)K * chains * kNPad * sizeof(float));
         w.ws_sdt = off;
-        off += align256((size_t)(K - 1) * chains * sizeof(float));
+        off += align256((size_t)K * chains * sizeof(float));
     }
     w.total = off;
     return w;
@@ -254,8 +293,9 @@ ScanWorkspace scan_workspace_layout(const mamba_dims_t* dims, int64_t groups, in
 //    (even load across SMs), segments at least 256 steps long.  At most G
 //    warps run, so a warp rarely picks up a segment whose predecessor has not
 //    finished.
-//  - G < W/4: parallel mode, K-1 = W/G segments per pass (every resident
-//    warp busy), segments at least 16 tiles and 512 steps long.
+//  - G < W/4: parallel mode, K = W/G segments (one segment per resident
+//    warp, so the first launch ends in one wave), segments at least 16 tiles
+//    and 512 steps long.
 //  - num_chunks >= 1 forces K; MAMBA_FLAG_PARALLEL_CHUNKS forces the parallel
 //    mode for a forced K.
 mamba_status_t plan_scan(const mamba_dims_t* dims, int sm_count, mamba_scan_plan_t* plan) {
@@ -297,7 +337,7 @@ mamba_status_t plan_scan(const mamba_dims_t* dims, int sm_count, mamba_scan_plan
         } else {
             mode = 1;
             K = std::max<int64_t>(
-                1, std::min<int64_t>(W / groups + 1, L / std::max<int64_t>(16 * T, 512)));
+                1, std::min<int64_t>(W / groups, L / std::max<int64_t>(16 * T, 512)));
         }
     }
     int64_t seg_len = L;
@@ -310,15 +350,17 @@ mamba_status_t plan_scan(const mamba_dims_t* dims, int sm_count, mamba_scan_plan
         seg_len = L;
         mode = 0;
     }
-    const int64_t items = mode == 0 ? groups * K : groups * (K - 1);
-    if (items >= ((int64_t)1 << 31)) return MAMBA_ERR_UNSUPPORTED;
+    const int64_t items = groups * K;
+    const int64_t chains = dims->batch * dims->dim;
+    const int64_t fixes = mode == 0 ? 0 : chains * (K - 1);
+    if (items >= ((int64_t)1 << 31) || fixes >= ((int64_t)1 << 31)) return MAMBA_ERR_UNSUPPORTED;
     plan->nchunks = (int32_t)K;
     plan->chunk_len = seg_len;
     plan->mode = mode;
     plan->units_pass_a = items;
-    plan->units_pass_b = mode == 0 ? 0 : items;
+    plan->units_pass_b = fixes;
     plan->max_warps = mode == 0 && K > 1 ? std::min<int64_t>(groups, W) : std::min<int64_t>(items, W);
-    plan->launches = (groups > 0 && L > 0) ? (mode == 0 ? 1 : 2) : 0;
+    plan->launches = (groups > 0 && L > 0) ? (mode == 0 ? 1 : 3) : 0;
     plan->workspace_bytes =
         (groups > 0 && L > 0) ? scan_workspace_layout(dims, groups, K, mode).total : 0;
     return MAMBA_OK;
@@ -514,8 +556,52 @@ mamba_status_t scan_fwd_internal(const void* u, const void* delta, const float* 
     if (plan.mode == 0) {
         e = run(kModeChained, counters, plan.units_pass_a);
     } else {
-        e = run(kModePassA, counters, plan.units_pass_a);
-        if (e == cudaSuccess) e = run(kModePassB, counters + 1, plan.units_pass_b);
+        // segments from their own start, then the carry over segments, then
+        // the start states' contributions to the outputs
+        e = run(kModeSegments, counters, plan.units_pass_a);
+        if (e == cudaSuccess) {
+            CarryParams cp{};
+            cp.A = A;
+            cp.ws_h = prm.ws_h;
+            cp.ws_sdt = prm.ws_sdt;
+            cp.last_state = last_state;
+            cp.chains = chains;
+            cp.dim = dims->dim;
+            cp.nseg = plan.nchunks;
+            cp.dstate = (int)dims->dstate;
+            const unsigned grid = (unsigned)((chains + kCarryWarps - 1) / kCarryWarps);
+            if (dims->io_dtype == MAMBA_F32)
+                scan_carry_kernel<true><<<grid, kCarryWarps * 32, 0, stream>>>(cp);
+            else
+                scan_carry_kernel<false><<<grid, kCarryWarps * 32, 0, stream>>>(cp);
+            e = cudaGetLastError();
+        }
+        if (e == cudaSuccess && plan.units_pass_b > 0) {
+            CorrectParams q{};
+            q.delta = delta;
+            q.z = z;
+            q.C = C;
+            q.A = A;
+            q.delta_bias = delta_bias;
+            q.out = out;
+            q.ws_h = prm.ws_h;
+            q.counter = counters + 1;
+            q.batch = dims->batch;
+            q.dim = dims->dim;
+            q.seqlen = dims->seqlen;
+            q.chains = chains;
+            q.seg_len = plan.chunk_len;
+            q.items = plan.units_pass_b;
+            q.nseg = plan.nchunks;
+            q.dstate = (int)dims->dstate;
+            q.bc_bf16 = dims->bc_dtype == MAMBA_BF16;
+            q.vec_io = ((dims->seqlen * io_es) % 16 == 0) && aligned(delta, 16) && aligned(out, 16) &&
+                       (!z || aligned(z, 16));
+            q.vec_c = ((dims->seqlen * bc_es) % 16 == 0) && aligned(C, 16);
+            e = dims->io_dtype == MAMBA_BF16
+                    ? dispatch_correct<__nv_bfloat16>(q, has_z, sp, dev, sms, stream)
+                    : dispatch_correct<float>(q, has_z, sp, dev, sms, stream);
+        }
     }
     return e == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
 }

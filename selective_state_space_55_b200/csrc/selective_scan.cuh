@@ -23,16 +23,20 @@
 //    the wait is free.  The handoff is a release/acquire flag per group; the
 //    wait is bounded and reports MAMBA_ERR_TIMEOUT through the device status
 //    word instead of hanging.  No work is repeated.
-//  * parallel (modes 1, 2; few channels, very long sequences): pass A runs
-//    segments 0..K-2 independently: segment 0 writes its outputs and end state,
-//    segments k >= 1 only their end state from a zero start and the sum of
-//    Delta.  Pass B runs segments 1..K-1: each folds the earlier segments'
-//    (exp(A sum Delta), end state) pairs into its true start state, then
-//    recomputes its outputs.  The fold applies the associative combine
-//    (P1, h1) then (P2, h2) -> (P1 P2, P2 h1 + h2) of the parallel scan
-//    ("Mamba: Linear-Time Sequence Modeling with Selective State Spaces",
-//    section 硬件效率; "Mamba 与状态空间模型", section 在芯片上扫过去).
-//
+//  * parallel (mode 1; few channels, very long sequences): every segment k
+//    runs at once from a zero start (segment 0 from the given start state),
+//    writes its outputs and keeps its end state and sum of Delta.  Two small
+//    kernels (scan_carry.cuh) then finish the job: a warp-shuffle associative
+//    scan over the segments of the pairs (exp(A sum Delta), end state), with
+//    (P1, h1) then (P2, h2) -> (P1 P2, P2 h1 + h2), gives each segment its true
+//    start state h_in ("Mamba: Linear-Time Sequence Modeling with Selective
+//    State Spaces", section 硬件效率; "Mamba 与状态空间模型", section
+//    在芯片上扫过去), and a correction pass adds to segment k's outputs what
+//    h_in contributes, C_t exp(A S_t) h_in with S_t the sum of Delta since the
+//    segment's start.  That term needs no recurrence, so it runs with lanes
+//    over time and stops where exp(A S_t) has underflowed for every state
+//    entry; nothing of the segment is computed twice.
+
 // Staging.  Per warp, a two-stage ring in shared memory holds tiles of
 // T = 32 bytes / sizeof(io) time steps of the warp's channel rows of u, delta
 // and z (TMA 3-D tiles with 32-byte swizzle, so each lane's 16-byte reads of
@@ -80,7 +84,7 @@ struct ScanLayout {
 constexpr size_t kWsCounters = 0;          // uint32 [2] dequeue counters
 constexpr size_t kWsFlags = 256;           // uint32 [groups] finished segments per group
 
-enum ScanMode { kModeChained = 0, kModePassA = 1, kModePassB = 2 };
+enum ScanMode { kModeChained = 0, kModeSegments = 1 };
 
 struct ScanParams {
     const void* u;
@@ -96,8 +100,8 @@ struct ScanParams {
     unsigned int* counter;   // dequeue counter of this launch
     unsigned int* flags;     // [groups] (chained mode)
     float* carry;            // [chains][16] (chained mode)
-    float* ws_h;             // [K-1][chains][16] (parallel mode)
-    float* ws_sdt;           // [K-1][chains]     (parallel mode)
+    float* ws_h;             // [K][chains][16] end states (parallel mode)
+    float* ws_sdt;           // [K][chains]     sums of Delta (parallel mode)
     int64_t batch, dim, seqlen;
     int64_t groups_per_batch, groups, chains;
     int64_t seg_len;
@@ -267,7 +271,8 @@ __device__ __forceinline__ void scan_step(const float* bc_row, const float (&dt)
 // all V steps are formed first: their softplus chains are independent of the
 // state, so computing them together lets their latency overlap.  The vectors
 // stay packed and are unpacked element by element to save registers.
-template <typename IoT, int kCpl, bool kHasZ, bool kSoftplus, bool kZoh, bool kOut, bool kCkpt>
+template <typename IoT, int kCpl, bool kHasZ, bool kSoftplus, bool kZoh, bool kOut, bool kCkpt,
+          bool kSum>
 __device__ __forceinline__ void compute_tile(const uint8_t* st, const float* bcf, int lane,
                                              int nsteps, LaneChains<kCpl>& lc,
                                              IoT* const (&out_row)[kCpl], bool vec_out,
@@ -329,9 +334,8 @@ __device__ __forceinline__ void compute_tile(const uint8_t* st, const float* bcf
                             pk[c].put(j, yo);
                         else if (out_row[c] != nullptr)
                             DType<IoT>::store(out_row[c] + base + j, yo);
-                    } else {
-                        kahan_add(sdt[c], sdt_c[c], dt[c]);
                     }
+                    if (kSum) kahan_add(sdt[c], sdt_c[c], dt[c]);
                 }
             }
         }
@@ -427,7 +431,8 @@ struct TmaMaps {
 // counts the tiles this warp has consumed (it fixes each tile's stage and
 // mbarrier parity across items).  Returns false if a staged tile never
 // arrived (the warp has then waited, bounded, for its copies in flight).
-template <typename IoT, int kCpl, bool kHasZ, bool kSoftplus, bool kZoh, bool kOut, bool kCkpt>
+template <typename IoT, int kCpl, bool kHasZ, bool kSoftplus, bool kZoh, bool kOut, bool kCkpt,
+          bool kSum>
 __device__ __forceinline__ bool run_segment(const ScanParams& p, const TmaMaps& maps, uint8_t* wsm,
                                             int lane, int64_t b, int64_t d0, int64_t t_begin,
                                             int64_t t_end, LaneChains<kCpl>& lc,
@@ -498,7 +503,7 @@ __device__ __forceinline__ bool run_segment(const ScanParams& p, const TmaMaps& 
             cks[c] = (kCkpt && ckpt_row[c]) ? ckpt_row[c] + ((t0 - t_begin) / kCkptSteps) * kNPad
                                             : nullptr;
         }
-        compute_tile<IoT, kCpl, kHasZ, kSoftplus, kZoh, kOut, kCkpt>(
+        compute_tile<IoT, kCpl, kHasZ, kSoftplus, kZoh, kOut, kCkpt, kSum>(
             st, bcf, lane, nsteps, lc, rows, p.vec_out != 0, sdt, sdt_c, cks);
         __syncwarp();
         if (p.use_tma && lane == 0 && i + kScanStages < ntiles) issue(i + kScanStages);
@@ -554,7 +559,7 @@ __global__ void __launch_bounds__(kScanWarps * 32, ScanLayout<kCpl>::kMinBlocks 
         if ((int64_t)item >= p.items) break;
 
         const int64_t g = item % p.groups;
-        const int64_t k = (p.mode == kModePassB ? 1 : 0) + item / p.groups;
+        const int64_t k = item / p.groups;
         const int64_t b = g / p.groups_per_batch;
         const int64_t d0 = (g % p.groups_per_batch) * Lay::kRows;
         const int64_t t_begin = k * p.seg_len;
@@ -577,7 +582,7 @@ __global__ void __launch_bounds__(kScanWarps * 32, ScanLayout<kCpl>::kMinBlocks 
                 const float a1 = in1 ? p.A[d * p.dstate + n + 1] : 0.0f;
                 lc.a2[c][pi] = make_float2(a0 * kLog2e, a1 * kLog2e);
                 if (kZoh) lc.inva[c][pi] = make_float2(in0 ? 1.0f / a0 : 0.0f, in1 ? 1.0f / a1 : 0.0f);
-                // Segment 0 starts from the given state (chained mode and pass A).
+                // Segment 0 starts from the given state (both modes).
                 const float* h0 = (k == 0 && p.h0 != nullptr) ? p.h0 + chain[c] * p.dstate : nullptr;
                 lc.h[c][pi] = make_float2((h0 != nullptr && in0) ? h0[n] : 0.0f,
                                           (h0 != nullptr && in1) ? h0[n + 1] : 0.0f);
@@ -608,25 +613,6 @@ __global__ void __launch_bounds__(kScanWarps * 32, ScanLayout<kCpl>::kMinBlocks 
 #pragma unroll
             for (int c = 0; c < kCpl; ++c)
                 if (valid[c]) load16(p.carry + chain[c] * kNPad, lc.h[c]);
-        } else if (p.mode == kModePassB) {
-            // True start state of segment k: fold the end states of 0..k-1.
-#pragma unroll
-            for (int c = 0; c < kCpl; ++c) {
-                if (!valid[c]) continue;
-                load16(p.ws_h + chain[c] * kNPad, lc.h[c]);
-                for (int64_t j = 1; j < k; ++j) {
-                    const float sj = __ldcg(p.ws_sdt + j * p.chains + chain[c]);
-                    const float2 s2 = make_float2(sj, sj);
-                    float2 hj[kNPad / 2];
-                    load16(p.ws_h + (j * p.chains + chain[c]) * kNPad, hj);
-#pragma unroll
-                    for (int pi = 0; pi < kNPad / 2; ++pi) {
-                        const float2 decay =
-                            exp2_pair<sizeof(IoT) == 4>(__fmul2_rn(lc.a2[c][pi], s2));
-                        lc.h[c][pi] = __ffma2_rn(decay, lc.h[c][pi], hj[pi]);
-                    }
-                }
-            }
         }
 
         IoT* out_row[kCpl];
@@ -643,13 +629,13 @@ __global__ void __launch_bounds__(kScanWarps * 32, ScanLayout<kCpl>::kMinBlocks 
         }
         bool ok;
         if (p.ckpt != nullptr)           // checkpoint pass of the backward: states only
-            ok = run_segment<IoT, kCpl, kHasZ, kSoftplus, kZoh, false, true>(
+            ok = run_segment<IoT, kCpl, kHasZ, kSoftplus, kZoh, false, true, false>(
                 p, maps, wsm, lane, b, d0, t_begin, t_end, lc, out_row, seq, sdt, ckpt_row);
-        else if (p.mode == kModePassA && k > 0)
-            ok = run_segment<IoT, kCpl, kHasZ, kSoftplus, kZoh, false, false>(
+        else if (p.mode == kModeSegments)
+            ok = run_segment<IoT, kCpl, kHasZ, kSoftplus, kZoh, true, false, true>(
                 p, maps, wsm, lane, b, d0, t_begin, t_end, lc, out_row, seq, sdt, ckpt_row);
         else
-            ok = run_segment<IoT, kCpl, kHasZ, kSoftplus, kZoh, true, false>(
+            ok = run_segment<IoT, kCpl, kHasZ, kSoftplus, kZoh, true, false, false>(
                 p, maps, wsm, lane, b, d0, t_begin, t_end, lc, out_row, seq, sdt, ckpt_row);
         if (!ok) break;
 
@@ -664,15 +650,15 @@ __global__ void __launch_bounds__(kScanWarps * 32, ScanLayout<kCpl>::kMinBlocks 
                 if (lane == 0 && !p.withhold_handoff)
                     st_release_gpu(p.flags + g, (unsigned int)(k + 1));
             }
-        } else if (p.mode == kModePassA) {
+        } else {   // parallel mode: the segment's end state from its own start, and its sum of Delta
 #pragma unroll
             for (int c = 0; c < kCpl; ++c) {
                 if (!valid[c]) continue;
                 store16(p.ws_h + (k * p.chains + chain[c]) * kNPad, lc.h[c]);
-                if (k >= 1) __stcg(p.ws_sdt + k * p.chains + chain[c], sdt[c]);
+                __stcg(p.ws_sdt + k * p.chains + chain[c], sdt[c]);
             }
         }
-        if (last_seg && p.mode != kModePassA && p.last_state != nullptr) {
+        if (last_seg && p.mode == kModeChained && p.last_state != nullptr) {
 #pragma unroll
             for (int c = 0; c < kCpl; ++c) {
                 if (!valid[c]) continue;

@@ -197,18 +197,21 @@ def test_plan_layer_shapes(lib):
 
 
 def test_plan_parallel_for_the_million_token_sequence(lib):
+    # few channel groups: every segment runs at once from its own start (one
+    # segment per resident warp), then the carry scan and the correction pass
     c = SCAN_CONFIGS["long_dna_1m"]
     p = ops.scan_plan(c.batch, c.dim, c.dstate, c.seqlen, c.io_dtype, c.bc_dtype, sm_count=148)
     K = p["nchunks"]
-    assert p["mode"] == 1 and p["launches"] == 2 and p["channels_per_lane"] == 1
+    assert p["mode"] == 1 and p["launches"] == 3 and p["channels_per_lane"] == 1
     assert p["groups"] == 1536 // 32
-    assert K - 1 == (148 * 16) // p["groups"]           # one item per resident warp and pass
+    assert K == (148 * 16) // p["groups"]                 # one segment per resident warp
+    assert p["units_pass_a"] == p["groups"] * K <= 148 * 16
     assert p["chunk_len"] % p["tile_len"] == 0
     assert (K - 1) * p["chunk_len"] < c.seqlen <= K * p["chunk_len"]
-    assert p["units_pass_a"] == p["units_pass_b"] == p["groups"] * (K - 1)
     chains = c.batch * c.dim
-    expect = 256 + 256 + ((K - 1) * chains * 64 + 255) // 256 * 256 + \
-        ((K - 1) * chains * 4 + 255) // 256 * 256
+    assert p["units_pass_b"] == chains * (K - 1)           # one correction item per later segment
+    expect = 256 + 256 + (K * chains * 64 + 255) // 256 * 256 + \
+        (K * chains * 4 + 255) // 256 * 256
     assert p["workspace_bytes"] == expect
     assert p["workspace_bytes"] <= 8 << 20
 
