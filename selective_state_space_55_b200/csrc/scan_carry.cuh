@@ -22,10 +22,11 @@
 //    recurrence, so one warp walks a segment with its lanes over consecutive
 //    time steps: Delta, its running sum S_t (warp-shuffle prefix sum), 16
 //    exponentials and a dot product per step.  Where Delta >= 0 throughout
-//    (softplus on) S_t never decreases, so once max_n(A_n) S_t < -127 every
-//    P_t,n is below 2^-127 for the rest of the segment, which ex2.approx.ftz
-//    returns as 0; the walk stops there and the outputs are exactly those of
-//    walking on.  Segments whose decay is slow are corrected to their end.
+//    (softplus on) S_t never decreases, so once A_n S_t < -127 the term of
+//    state entry n is below 2^-127 for the rest of the segment, which
+//    ex2.approx.ftz returns as 0: the entry drops out of the walk, and the walk
+//    stops when none is left.  The outputs are exactly those of walking on to
+//    the segment's end, which is where a segment with slow decay stops anyway.
 #pragma once
 
 #include "ssm_device.cuh"
@@ -148,14 +149,12 @@ __global__ void __launch_bounds__(kCorrectWarps * 32)
         const int64_t t_end = min(t_begin + p.seg_len, p.seqlen);
 
         float hin[kNPad], a2[kNPad];
-        float a2max = -INFINITY;
         const float* hs = p.ws_h + ((k - 1) * p.chains + chain) * kNPad;
 #pragma unroll
         for (int n = 0; n < kNPad; ++n) {
             const bool in = n < p.dstate;
             hin[n] = in ? __ldcg(hs + n) : 0.0f;
             a2[n] = in ? p.A[d * p.dstate + n] * kLog2e : 0.0f;
-            if (in) a2max = fmaxf(a2max, a2[n]);
         }
         const float bias = p.delta_bias ? p.delta_bias[d] : 0.0f;
         const IoT* drow = delta + chain * p.seqlen;
@@ -166,8 +165,14 @@ __global__ void __launch_bounds__(kCorrectWarps * 32)
         bool monotone = true;     // Delta >= 0 at every step so far
 
         for (int64_t t0 = t_begin; t0 < t_end; t0 += 32 * V) {
-            // Every remaining exp(A_n S_t) is below 2^-127, i.e. 0 after ex2.approx.ftz.
-            if (monotone && a2max < 0.0f && a2max * S_run < kUnderflowLog2) break;
+            // State entries whose exp(A_n S_t) is below 2^-127 for the rest of
+            // the segment (0 after ex2.approx.ftz) drop out; none left, done.
+            uint32_t active = 0;
+#pragma unroll
+            for (int n = 0; n < kNPad; ++n)
+                if (n < p.dstate && !(monotone && a2[n] < 0.0f && a2[n] * S_run < kUnderflowLog2))
+                    active |= 1u << n;
+            if (active == 0) break;
             const int64_t ts = t0 + (int64_t)lane * V;
             const int valid = (int)max((int64_t)0, min((int64_t)V, t_end - ts));
             float dl[V];
@@ -203,7 +208,7 @@ __global__ void __launch_bounds__(kCorrectWarps * 32)
             for (int j = 0; j < V; ++j) corr[j] = 0.0f;
 #pragma unroll
             for (int n = 0; n < kNPad; ++n) {
-                if (n >= p.dstate) break;
+                if (!((active >> n) & 1u)) continue;   // uniform across the warp
                 float cv[V];
                 load_run<BcT, V>(crow + n * p.seqlen, ts, valid, p.vec_c != 0, cv);
 #pragma unroll
