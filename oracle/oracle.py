@@ -17,9 +17,9 @@ term is the zero-order-hold one, expm1(Delta_t A_d,n) / A_d,n * B_t,n * u_t
 (Delta_t B_t,n u_t where A_d,n = 0), i.e. Bbar = (Delta A)^-1 (exp(Delta A) - I)
 Delta B for the diagonal A.
 
-The backward pass of the (Euler) scan is the adjoint recurrence in reverse
-time; ``selective_scan_bwd`` returns the gradients of a linear functional of
-out and last_state.
+The backward pass of the scan (Euler or zero-order-hold input term) is the
+adjoint recurrence in reverse time; ``selective_scan_bwd`` returns the
+gradients of a linear functional of out and last_state.
 
 ``ssd_scan`` is the Mamba-2 layer ("Mamba 与状态空间模型", section
 "Mamba-2：两种算法"): A is a scalar per head, the state of a head is a
@@ -100,9 +100,9 @@ class Oracle:
         self._lib.oracle_selective_state_update_ex_f64.restype = ctypes.c_int
         self._lib.oracle_selective_state_update_ex_f64.argtypes = [
             i64, i64, i64, dp, dp, dp, dp, dp, dp, dp, dp, dp, ci, ci, dp, dp]
-        self._lib.oracle_selective_scan_bwd_f64.restype = ctypes.c_int
-        self._lib.oracle_selective_scan_bwd_f64.argtypes = [
-            i64, i64, i64, i64, dp, dp, dp, dp, dp, dp, dp, dp, ci, dp, dp, dp,
+        self._lib.oracle_selective_scan_bwd_ex_f64.restype = ctypes.c_int
+        self._lib.oracle_selective_scan_bwd_ex_f64.argtypes = [
+            i64, i64, i64, i64, dp, dp, dp, dp, dp, dp, dp, dp, ci, ci, dp, dp, dp,
             dp, dp, dp, dp, dp, dp, dp, dp, dp]
         self._lib.oracle_causal_conv1d_f64.restype = ctypes.c_int
         self._lib.oracle_causal_conv1d_f64.argtypes = [
@@ -179,10 +179,11 @@ class Oracle:
         return new_state, out
 
     def selective_scan_bwd(self, u, delta, A, B, C, dout, D=None, z=None, delta_bias=None,
-                           softplus=True, initial_state=None, dlast_state=None):
+                           softplus=True, initial_state=None, dlast_state=None, zoh=False):
         """Gradients of sum(dout * out) + sum(dlast_state * last_state) of the
-        (Euler) scan, as a dict of float64 arrays: du, ddelta, dA, dB, dC, and
-        dD, dz, ddelta_bias, dinitial_state for the optional inputs given."""
+        scan (Euler input term, or zero-order hold with ``zoh``), as a dict of
+        float64 arrays: du, ddelta, dA, dB, dC, and dD, dz, ddelta_bias,
+        dinitial_state for the optional inputs given."""
         u, delta, A, B, C, dout = map(_f64, (u, delta, A, B, C, dout))
         D, z, delta_bias = map(_f64, (D, z, delta_bias))
         initial_state, dlast_state = _f64(initial_state), _f64(dlast_state)
@@ -200,14 +201,15 @@ class Oracle:
             g["ddelta_bias"] = np.empty_like(delta_bias)
         if initial_state is not None:
             g["dinitial_state"] = np.empty_like(initial_state)
-        rc = self._lib.oracle_selective_scan_bwd_f64(
+        rc = self._lib.oracle_selective_scan_bwd_ex_f64(
             batch, dim, dstate, seqlen, _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
-            _ptr(z), _ptr(delta_bias), int(bool(softplus)), _ptr(initial_state), _ptr(dout),
+            _ptr(z), _ptr(delta_bias), int(bool(softplus)), int(bool(zoh)), _ptr(initial_state),
+            _ptr(dout),
             _ptr(dlast_state), _ptr(g["du"]), _ptr(g["ddelta"]), _ptr(g["dA"]), _ptr(g["dB"]),
             _ptr(g["dC"]), _ptr(g.get("dD")), _ptr(g.get("dz")), _ptr(g.get("ddelta_bias")),
             _ptr(g.get("dinitial_state")))
         if rc != 0:
-            raise ValueError(f"oracle_selective_scan_bwd_f64 returned {rc}")
+            raise ValueError(f"oracle_selective_scan_bwd_ex_f64 returned {rc}")
         return g
 
     def causal_conv1d(self, x, weight, bias=None, initial_conv_state=None, silu=True):

@@ -330,18 +330,40 @@ static double oracle_softplus_grad(double s)
     return 1.0 / (1.0 + exp(-s));
 }
 
+/* Derivative of the zero-order-hold gain g(dt, a) = expm1(dt a) / a with
+ * respect to a: (x e^x - expm1(x)) / a^2 with x = dt a, i.e.
+ * dt^2 (x e^x - expm1(x)) / x^2.  Near x = 0 the difference cancels, so there
+ * the series dt^2 (1/2 + x/3 + x^2/8 + x^3/30 + x^4/144) (coefficients
+ * (k + 1) / (k + 2)!) is used; its limit at a = 0 is dt^2 / 2.  (With respect
+ * to dt the gain's derivative is exp(dt a) = Abar.) */
+static double oracle_zoh_gain_da(double dt, double a)
+{
+    double x = dt * a;
+    if (fabs(x) < 1e-3)
+        return dt * dt * (0.5 + x * (1.0 / 3.0 + x * (1.0 / 8.0 + x * (1.0 / 30.0 + x / 144.0))));
+    return (x * exp(x) - expm1(x)) / (a * a);
+}
+
 /* Gradients of sum_t dout_t out_t + sum_n dlast_n last_state_n with respect to
- * every input of oracle_selective_scan_ex_f64 (Euler input term).  Gradient
- * outputs for NULL inputs may be NULL; all others are overwritten.  Returns
- * -1 on a bad size, -2 if the scratch cannot be allocated. */
-int oracle_selective_scan_bwd_f64(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
-                                  const double *u, const double *delta, const double *A,
-                                  const double *B, const double *C, const double *D,
-                                  const double *z, const double *delta_bias, int softplus,
-                                  const double *initial_state, const double *dout,
-                                  const double *dlast_state, double *du, double *ddelta,
-                                  double *dA, double *dB, double *dC, double *dD, double *dz,
-                                  double *ddelta_bias, double *dinitial_state)
+ * every input of oracle_selective_scan_ex_f64, with the Euler input term
+ * (zoh = 0) or the zero-order-hold one (zoh = 1).  With the input gain
+ * g = Delta (Euler) or expm1(Delta a) / a (zero-order hold), one step is
+ * h_t = Abar h_t-1 + g B_t u_t, and its adjoint, with lambda = dLoss/dh_t:
+ *   dB += lambda g u,   du += lambda g B,
+ *   dDelta += lambda (dg/dDelta B u + a Abar h_t-1),   dg/dDelta = 1 or Abar,
+ *   dA += lambda (Delta Abar h_t-1 + dg/da B u),       dg/da = 0 or
+ *         oracle_zoh_gain_da,
+ *   lambda_t-1 = Abar lambda.
+ * Gradient outputs for NULL inputs may be NULL; all others are overwritten.
+ * Returns -1 on a bad size, -2 if the scratch cannot be allocated. */
+int oracle_selective_scan_bwd_ex_f64(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
+                                     const double *u, const double *delta, const double *A,
+                                     const double *B, const double *C, const double *D,
+                                     const double *z, const double *delta_bias, int softplus,
+                                     int zoh, const double *initial_state, const double *dout,
+                                     const double *dlast_state, double *du, double *ddelta,
+                                     double *dA, double *dB, double *dC, double *dD, double *dz,
+                                     double *ddelta_bias, double *dinitial_state)
 {
     if (batch < 0 || dim < 0 || seqlen < 0 || dstate < 1 || dstate > ORACLE_MAX_DSTATE)
         return -1;
@@ -382,7 +404,8 @@ int oracle_selective_scan_bwd_f64(int64_t batch, int64_t dim, int64_t dstate, in
             double y = 0.0;
             for (int64_t n = 0; n < dstate; ++n) {
                 double a_bar = exp(dt * A[d * dstate + n]);
-                double h = a_bar * hs[t * dstate + n] + dt * B[(b * dstate + n) * seqlen + t] * u_row[t];
+                double gain_f = zoh ? oracle_zoh_gain(dt, A[d * dstate + n]) : dt;
+                double h = a_bar * hs[t * dstate + n] + gain_f * B[(b * dstate + n) * seqlen + t] * u_row[t];
                 hs[(t + 1) * dstate + n] = h;
                 y += C[(b * dstate + n) * seqlen + t] * h;
             }
@@ -413,12 +436,15 @@ int oracle_selective_scan_bwd_f64(int64_t batch, int64_t dim, int64_t dstate, in
                 double a_dn = A[d * dstate + n];
                 double a_bar = exp(dt * a_dn);
                 double h_prev = hs[t * dstate + n];
+                double gain = zoh ? oracle_zoh_gain(dt, a_dn) : dt;
+                double gain_dt = zoh ? a_bar : 1.0;
+                double gain_da = zoh ? oracle_zoh_gain_da(dt, a_dn) : 0.0;
                 lam[n] += c_tn * dy;
                 dC[(b * dstate + n) * seqlen + t] += dy * hs[(t + 1) * dstate + n];
-                dB[(b * dstate + n) * seqlen + t] += lam[n] * dt * x;
-                ddt += lam[n] * (b_tn * x + a_dn * a_bar * h_prev);
-                dA[d * dstate + n] += lam[n] * dt * a_bar * h_prev;
-                dut += lam[n] * dt * b_tn;
+                dB[(b * dstate + n) * seqlen + t] += lam[n] * gain * x;
+                ddt += lam[n] * (gain_dt * b_tn * x + a_dn * a_bar * h_prev);
+                dA[d * dstate + n] += lam[n] * (dt * a_bar * h_prev + gain_da * b_tn * x);
+                dut += lam[n] * gain * b_tn;
                 lam[n] *= a_bar;
             }
             du[chain * seqlen + t] = dut;
@@ -436,6 +462,22 @@ int oracle_selective_scan_bwd_f64(int64_t batch, int64_t dim, int64_t dstate, in
     free(dts);
     free(ys);
     return 0;
+}
+
+/* The Euler-term backward (oracle_selective_scan_bwd_ex_f64 with zoh = 0). */
+int oracle_selective_scan_bwd_f64(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
+                                  const double *u, const double *delta, const double *A,
+                                  const double *B, const double *C, const double *D,
+                                  const double *z, const double *delta_bias, int softplus,
+                                  const double *initial_state, const double *dout,
+                                  const double *dlast_state, double *du, double *ddelta,
+                                  double *dA, double *dB, double *dC, double *dD, double *dz,
+                                  double *ddelta_bias, double *dinitial_state)
+{
+    return oracle_selective_scan_bwd_ex_f64(batch, dim, dstate, seqlen, u, delta, A, B, C, D, z,
+                                            delta_bias, softplus, 0, initial_state, dout,
+                                            dlast_state, du, ddelta, dA, dB, dC, dD, dz,
+                                            ddelta_bias, dinitial_state);
 }
 
 /*

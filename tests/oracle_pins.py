@@ -578,11 +578,12 @@ def _bwd_problem(seed, gated=True):
     return p, dout, dlast
 
 
-def _fd_check(o, p, dout, dlast, softplus, what):
+def _fd_check(o, p, dout, dlast, softplus, what, zoh=False):
     def loss(q):
         out, last = o.selective_scan(q["u"], q["delta"], q["A"], q["B"], q["C"], D=q.get("D"),
                                      z=q.get("z"), delta_bias=q.get("delta_bias"),
-                                     softplus=softplus, initial_state=q.get("initial_state"))
+                                     softplus=softplus, initial_state=q.get("initial_state"),
+                                     zoh=zoh)
         val = float(np.sum(dout * out))
         if dlast is not None:
             val += float(np.sum(dlast * last))
@@ -590,7 +591,7 @@ def _fd_check(o, p, dout, dlast, softplus, what):
 
     g = o.selective_scan_bwd(p["u"], p["delta"], p["A"], p["B"], p["C"], dout, D=p.get("D"),
                              z=p.get("z"), delta_bias=p.get("delta_bias"), softplus=softplus,
-                             initial_state=p.get("initial_state"), dlast_state=dlast)
+                             initial_state=p.get("initial_state"), dlast_state=dlast, zoh=zoh)
     names = {"u": "du", "delta": "ddelta", "A": "dA", "B": "dB", "C": "dC", "D": "dD",
              "z": "dz", "delta_bias": "ddelta_bias", "initial_state": "dinitial_state"}
     for key, gname in names.items():
@@ -621,6 +622,25 @@ def pin_bwd_finite_differences_plain(o):
     """The same without gate, D, bias, start state or last-state term, softplus off."""
     p, dout, dlast = _bwd_problem(52, gated=False)
     _fd_check(o, p, dout, dlast, False, "plain backward")
+
+
+def pin_bwd_zoh_finite_differences(o):
+    """Zero-order-hold input term ("超越注意力：探索Mamba与状态空间模型", section
+    状态空间模型基础: Bbar = (Delta A)^-1 (exp(Delta A) - I) Delta B): every gradient,
+    gated, softplus on, with a start state and a last-state term, against central
+    differences of the zero-order-hold forward.  One entry of A is set to 0
+    (the gain's limit Delta) and one to -5e-4 (the series branch of dg/dA)."""
+    p, dout, dlast = _bwd_problem(53, gated=True)
+    p["A"][0, 0] = 0.0
+    p["A"][1, 1] = -5e-4
+    _fd_check(o, p, dout, dlast, True, "zero-order-hold backward", zoh=True)
+
+
+def pin_bwd_zoh_plain_finite_differences(o):
+    """The zero-order-hold backward without gate, D, bias, start state or
+    last-state term, softplus off (Delta may then be negative)."""
+    p, dout, dlast = _bwd_problem(54, gated=False)
+    _fd_check(o, p, dout, dlast, False, "plain zero-order-hold backward", zoh=True)
 
 
 # --- Mamba-2 layer (scalar A per head) ------------------------------------------------------
@@ -757,6 +777,8 @@ PINS = {
     "conv_updates_equal_prefill": pin_conv_updates_equal_prefill,
     "bwd_finite_differences_gated": pin_bwd_finite_differences_gated,
     "bwd_finite_differences_plain": pin_bwd_finite_differences_plain,
+    "bwd_zoh_finite_differences": pin_bwd_zoh_finite_differences,
+    "bwd_zoh_plain_finite_differences": pin_bwd_zoh_plain_finite_differences,
     "ssd_lower_triangular_matrix": pin_ssd_lower_triangular_matrix,
     "ssd_is_tied_diagonal_scan": pin_ssd_is_tied_diagonal_scan,
     "ssd_split_equals_whole": pin_ssd_split_equals_whole,

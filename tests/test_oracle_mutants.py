@@ -84,15 +84,27 @@ MUTANTS = [
     # backward pass
     ("bwd_lambda_not_propagated", "lam[n] *= a_bar;", "lam[n] *= 1.0;"),
     ("bwd_dC_uses_previous_state", "+= dy * hs[(t + 1) * dstate + n];", "+= dy * hs[t * dstate + n];"),
-    ("bwd_dA_missing_delta", "dA[d * dstate + n] += lam[n] * dt * a_bar * h_prev;",
-     "dA[d * dstate + n] += lam[n] * a_bar * h_prev;"),
+    ("bwd_dA_missing_delta", "dA[d * dstate + n] += lam[n] * (dt * a_bar * h_prev",
+     "dA[d * dstate + n] += lam[n] * (a_bar * h_prev"),
     ("bwd_softplus_grad_skipped", "double ds = softplus ? ddt * oracle_softplus_grad(s) : ddt;",
      "double ds = ddt;"),
     ("bwd_silu_grad_is_sigmoid", "return sg * (1.0 + z * (1.0 - sg));", "return sg;"),
-    ("bwd_ddelta_A_term_sign", "ddt += lam[n] * (b_tn * x + a_dn * a_bar * h_prev);",
-     "ddt += lam[n] * (b_tn * x - a_dn * a_bar * h_prev);"),
+    ("bwd_ddelta_A_term_sign", "ddt += lam[n] * (gain_dt * b_tn * x + a_dn * a_bar * h_prev);",
+     "ddt += lam[n] * (gain_dt * b_tn * x - a_dn * a_bar * h_prev);"),
     ("bwd_du_missing_D", "double dut = D ? dy * D[d] : 0.0;", "double dut = 0.0;"),
-    ("bwd_dB_missing_u", "+= lam[n] * dt * x;", "+= lam[n] * dt;"),
+    ("bwd_dB_missing_u", "+= lam[n] * gain * x;", "+= lam[n] * gain;"),
+    # backward pass with the zero-order hold
+    ("bwd_zoh_forward_is_euler", "double gain_f = zoh ? oracle_zoh_gain(dt, A[d * dstate + n]) : dt;",
+     "double gain_f = dt;"),
+    ("bwd_zoh_gain_is_euler", "double gain = zoh ? oracle_zoh_gain(dt, a_dn) : dt;\n                double gain_dt",
+     "double gain = dt;\n                double gain_dt"),
+    ("bwd_zoh_gain_dt_is_one", "double gain_dt = zoh ? a_bar : 1.0;", "double gain_dt = 1.0;"),
+    ("bwd_zoh_gain_da_dropped", "double gain_da = zoh ? oracle_zoh_gain_da(dt, a_dn) : 0.0;",
+     "double gain_da = 0.0;"),
+    ("bwd_zoh_gain_da_sign", "return (x * exp(x) - expm1(x)) / (a * a);",
+     "return (expm1(x) - x * exp(x)) / (a * a);"),
+    ("bwd_zoh_gain_da_series_term", "(0.5 + x * (1.0 / 3.0 + x", "(0.5 + x * (1.0 / 2.0 + x"),
+    ("bwd_zoh_du_uses_delta", "dut += lam[n] * gain * b_tn;", "dut += lam[n] * dt * b_tn;"),
     ("bwd_dlast_ignored", "lam[n] = dlast_state ? dlast_state[chain * dstate + n] : 0.0;",
      "lam[n] = 0.0;"),
     ("bwd_readout_grad_ungated", "dy = g * oracle_silu(zt);", "dy = g;"),
