@@ -355,7 +355,8 @@ MAMBA_API mamba_status_t mamba_selective_state_update(float *state, const void *
  *
  * Gradients of a scalar loss, given dout = dLoss/dout (and optionally
  * dlast_state = dLoss/dlast_state), with respect to every input of
- * mamba_selective_scan_fwd_with_state, Euler input term.  As in the pages'
+ * mamba_selective_scan_fwd_with_state, with the Euler input term or, with
+ * MAMBA_FLAG_ZOH in dims->flags, the zero-order-hold one.  As in the pages'
  * description of the hardware-aware scan ("Mamba 与状态空间模型", section
  * 在芯片上扫过去), the per-step states are not stored by the forward: a
  * checkpoint pass keeps the state every 8 steps in the workspace, and the
@@ -365,6 +366,11 @@ MAMBA_API mamba_status_t mamba_selective_state_update(float *state, const void *
  *   dC_t,n = dy_t h_t,n;  dB_t,n = lambda_t,n Delta_t u_t
  *   dDelta_t = sum_n lambda_t,n (B_t,n u_t + A_n Abar_t,n h_t-1,n)  (then * softplus')
  *   dA_n = sum_t lambda_t,n Delta_t Abar_t,n h_t-1,n;  du_t = D dy_t + Delta_t sum_n lambda_t,n B_t,n
+ * With the zero-order hold the input gain g = expm1(Delta A) / A replaces Delta
+ * in the input term ("超越注意力：探索Mamba与状态空间模型", section 状态空间模型基础):
+ * dB = lambda g u, du = D dy + sum_n lambda g B, dDelta gains Abar B u in place
+ * of B u (dg/dDelta = Abar) and dA gains lambda dg/dA B u with
+ * dg/dA = (Delta Abar - g) / A (its series near Delta A = 0, limit Delta^2 / 2).
  * Inputs (device): the forward's inputs (u, delta, A, B, C, D, z, delta_bias,
  *   softplus, initial_state: same shapes, dtypes and NULL rules), dout
  *   (batch, dim, seqlen) io_dtype, dlast_state (batch, dim, dstate) fp32 or NULL.
@@ -378,9 +384,9 @@ MAMBA_API mamba_status_t mamba_selective_state_update(float *state, const void *
  * dims->workspace: at least mamba_selective_scan_bwd_workspace_bytes(dims)
  *   bytes, 256-byte aligned (64 bytes per chain and 8 steps for the
  *   checkpoints, plus the segment handoffs).
- * MAMBA_FLAG_ZOH is not supported here (MAMBA_ERR_UNSUPPORTED).  Segments of a
- * sequence are processed one after another (chained), so sequences much longer
- * than the batch x channel count can keep busy run with little parallelism.
+ * Segments of a sequence are processed one after another (chained), so
+ * sequences much longer than the batch x channel count can keep busy run with
+ * little parallelism.
  */
 MAMBA_API size_t mamba_selective_scan_bwd_workspace_bytes(const mamba_dims_t *dims);
 

@@ -13,7 +13,17 @@
 //   dh_-1      = Abar_0 lambda_0
 //
 // with dy = dout silu(z), dz = dout y silu'(z) and the softplus derivative
-// sigmoid(delta + bias) applied to dDelta.
+// sigmoid(delta + bias) applied to dDelta.  With the zero-order-hold input
+// term ("超越注意力：探索Mamba与状态空间模型", section 状态空间模型基础) the step is
+// h_t = Abar_t h_t-1 + g_t B_t u_t with the gain g = expm1(Delta A) / A =
+// Delta phi(Delta A) instead of Delta; then
+//
+//   dB_t,n     = lambda_t,n g_t,n u_t,   du_t = D dy_t + Delta_t sum_n lambda phi B
+//   dDelta_t   = sum_n lambda_t,n (Abar_t,n B_t,n u_t + A_n Abar_t,n h_t-1,n)
+//   dA_n      += lambda_t,n (Delta_t Abar_t,n h_t-1,n + dg/dA B_t,n u_t)
+//
+// with dg/dA = Delta (Abar - phi) / A, or its series Delta^2 (1/2 + x/3 + x^2/8
+// + ...) (x = Delta A) where the difference would cancel.
 //
 // Layout of the work.  A first launch (the forward kernel in its checkpoint
 // mode) stores the state before every block of kCkptSteps = 8 steps.  Then one
@@ -160,9 +170,12 @@ struct BwdStage {
     uint4 ck[32][4];
 };
 
+// Per warp: two stages, the B/C table of one block, and 1 / A of the lanes'
+// 16 state entries in quarters (zero-order hold).
 template <typename IoT, typename BcT>
 __host__ __device__ constexpr int bwd_warp_smem() {
-    return 2 * (int)sizeof(BwdStage<IoT, BcT>) + kBwdSteps * 32 * (int)sizeof(float);
+    return 2 * (int)sizeof(BwdStage<IoT, BcT>) + kBwdSteps * 32 * (int)sizeof(float) +
+           (kNPad / 4) * 32 * (int)sizeof(float4);
 }
 
 template <int kVecs>
@@ -201,7 +214,25 @@ __device__ __forceinline__ float bwd_exp2(float x) {
     return kExact ? exp2_near_one_exact(x) : ex2_approx(x);
 }
 
-template <typename IoT, typename BcT, bool kHasZ>
+// dg/dA / Delta^2 = (x e^x - expm1(x)) / x^2 for x = Delta A, as its series
+// sum_k x^k (k + 1) / (k + 2)! written in x2 = x log2(e) (coefficients
+// ln2^k (k + 1) / (k + 2)!), nine terms: truncation below 2e-9 relative for
+// |x2| < kDgdaSmall.  Beyond it the closed form Delta (Abar - phi) / A loses
+// at most a few units of 1e-6 to cancellation.
+constexpr float kDgdaSmall = 0.75f;
+
+__device__ __forceinline__ float2 zoh_dgda_series2(float2 x2) {
+    constexpr float c[9] = {0.5f, 0.23104906018664842f, 0.060056626739775174f,
+                            0.011100821732964315f, 0.0016030215179380792f,
+                            0.0001904794020918349f, 1.925441299172701e-05f,
+                            1.694748200451093e-06f, 1.3215486790144306e-07f};
+    float2 r = make_float2(c[8], c[8]);
+#pragma unroll
+    for (int k = 7; k >= 0; --k) r = __ffma2_rn(x2, r, make_float2(c[k], c[k]));
+    return r;
+}
+
+template <typename IoT, typename BcT, bool kHasZ, bool kZoh>
 __global__ void __launch_bounds__(kBwdWarps * 32)
     selective_scan_bwd_kernel(const __grid_constant__ BwdParams p) {
     constexpr bool kExact = sizeof(IoT) == 4;
@@ -213,6 +244,8 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
     uint8_t* wbase = bwd_smem + warp * bwd_warp_smem<IoT, BcT>();
     Stage* stages = reinterpret_cast<Stage*>(wbase);
     float (*bcf)[32] = reinterpret_cast<float (*)[32]>(wbase + 2 * sizeof(Stage));
+    float4 (*inva4)[32] = reinterpret_cast<float4 (*)[32]>(
+        wbase + 2 * sizeof(Stage) + kBwdSteps * 32 * sizeof(float));
 
     for (;;) {
         unsigned int item = 0;
@@ -234,6 +267,19 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
 #pragma unroll
         for (int n = 0; n < kNPad; ++n)
             a2[n] = (valid && n < p.dstate) ? p.A[d * p.dstate + n] * kLog2e : 0.0f;
+        if (kZoh) {   // 1 / A_n, as the forward holds it (read back one quarter at a time)
+#pragma unroll
+            for (int q = 0; q < kNPad / 4; ++q) {
+                float v[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int n = 4 * q + i;
+                    const float a = (valid && n < p.dstate) ? p.A[d * p.dstate + n] : 0.0f;
+                    v[i] = (valid && n < p.dstate) ? 1.0f / a : 0.0f;
+                }
+                inva4[q][lane] = make_float4(v[0], v[1], v[2], v[3]);
+            }
+        }
         const float bias = (valid && p.delta_bias != nullptr) ? p.delta_bias[d] : 0.0f;
         const float Dd = (valid && p.D != nullptr) ? p.D[d] : 0.0f;
 
@@ -396,6 +442,21 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
                 // The four entries run as two fp32x2 pairs (packed FMA/FMUL,
                 // rounding identical to the scalar forms).
                 const float2 a2p[2] = {make_float2(a2[0], a2[1]), make_float2(a2[2], a2[3])};
+                float2 iv[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
+                if (kZoh) {
+                    const float4 v = inva4[q][lane];
+                    iv[0] = make_float2(v.x, v.y);
+                    iv[1] = make_float2(v.z, v.w);
+                }
+                // phi(Delta A) of the zero-order hold, as the forward forms it:
+                // its series near 0, else (Abar - 1) / (Delta A).
+                auto zoh_phi2 = [&](float2 x2, float2 ab, float rdt, int pr) -> float2 {
+                    const float2 big = __fmul2_rn(__fadd2_rn(ab, make_float2(-1.0f, -1.0f)),
+                                                  __fmul2_rn(make_float2(rdt, rdt), iv[pr]));
+                    const float2 ser = zoh_phi_series2(x2);
+                    return make_float2(fabsf(x2.x) < kZohSmall ? ser.x : big.x,
+                                       fabsf(x2.y) < kZohSmall ? ser.y : big.y);
+                };
                 const float2 a2l[2] = {__fmul2_rn(a2p[0], make_float2(kLn2, kLn2)),
                                        __fmul2_rn(a2p[1], make_float2(kLn2, kLn2))};
                 // forward: the block's 8 states of entries n0..n0+3
@@ -410,12 +471,15 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
                         const float2 cq[2] = {make_float2(Cq.x, Cq.y), make_float2(Cq.z, Cq.w)};
                         const float du = dt[t] * uu[t];
                         const float2 dt2 = make_float2(dt[t], dt[t]), du2 = make_float2(du, du);
+                        const float rdt = kZoh ? __fdividef(1.0f, dt[t]) : 0.0f;
                         float2 y2 = make_float2(0.0f, 0.0f);
 #pragma unroll
                         for (int pr = 0; pr < 2; ++pr) {
                             const float2 x2 = __fmul2_rn(dt2, a2p[pr]);
                             const float2 ab = make_float2(bwd_exp2<kExact>(x2.x), bwd_exp2<kExact>(x2.y));
-                            h2[pr] = __ffma2_rn(ab, h2[pr], __fmul2_rn(du2, bq[pr]));
+                            float2 in = __fmul2_rn(du2, bq[pr]);
+                            if (kZoh) in = __fmul2_rn(in, zoh_phi2(x2, ab, rdt, pr));
+                            h2[pr] = __ffma2_rn(ab, h2[pr], in);
                             hq[t][pr] = h2[pr];
                             y2 = __ffma2_rn(cq[pr], h2[pr], y2);
                         }
@@ -436,6 +500,7 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
                         const float2 dt2 = make_float2(dt[t], dt[t]), du2 = make_float2(du, du);
                         const float2 ndu2 = make_float2(-du, -du), dy2 = make_float2(dy[t], dy[t]);
                         const float2 uu2 = make_float2(uu[t], uu[t]);
+                        const float rdt = kZoh ? __fdividef(1.0f, dt[t]) : 0.0f;
                         float red[8];
                         float2 s_dt2 = make_float2(0.0f, 0.0f), s_b2 = make_float2(0.0f, 0.0f);
 #pragma unroll
@@ -443,16 +508,34 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
                             l2[pr] = __ffma2_rn(cq[pr], dy2, l2[pr]);                    // lambda_t
                             const float2 x2 = __fmul2_rn(dt2, a2p[pr]);
                             const float2 ab = make_float2(bwd_exp2<kExact>(x2.x), bwd_exp2<kExact>(x2.y));
-                            const float2 abh = __ffma2_rn(ndu2, bq[pr], hq[t][pr]);      // Abar_t h_t-1
-                            const float2 rb = __fmul2_rn(l2[pr], du2);                    // dB
                             const float2 rc = __fmul2_rn(dy2, hq[t][pr]);                 // dC
-                            red[2 * pr] = rb.x;
-                            red[2 * pr + 1] = rb.y;
+                            if (!kZoh) {
+                                const float2 abh = __ffma2_rn(ndu2, bq[pr], hq[t][pr]);  // Abar_t h_t-1
+                                const float2 rb = __fmul2_rn(l2[pr], du2);                // dB
+                                red[2 * pr] = rb.x;
+                                red[2 * pr + 1] = rb.y;
+                                s_dt2 = __ffma2_rn(l2[pr], __ffma2_rn(a2l[pr], abh, __fmul2_rn(bq[pr], uu2)), s_dt2);
+                                s_b2 = __ffma2_rn(l2[pr], bq[pr], s_b2);
+                                dA2[pr] = __ffma2_rn(__fmul2_rn(l2[pr], dt2), abh, dA2[pr]);
+                            } else {
+                                const float2 phi = zoh_phi2(x2, ab, rdt, pr);
+                                const float2 bu = __fmul2_rn(bq[pr], uu2);                // B u
+                                const float2 in = __fmul2_rn(__fmul2_rn(du2, bq[pr]), phi);
+                                const float2 abh = __fadd2_rn(hq[t][pr], make_float2(-in.x, -in.y));
+                                const float2 rb = __fmul2_rn(l2[pr], __fmul2_rn(du2, phi));  // dB
+                                red[2 * pr] = rb.x;
+                                red[2 * pr + 1] = rb.y;
+                                s_dt2 = __ffma2_rn(l2[pr], __ffma2_rn(a2l[pr], abh, __fmul2_rn(ab, bu)), s_dt2);
+                                s_b2 = __ffma2_rn(l2[pr], __fmul2_rn(phi, bq[pr]), s_b2);
+                                // dg/dA: Delta^2 times its series near 0, else Delta (Abar - phi) / A
+                                const float2 ser = __fmul2_rn(__fmul2_rn(dt2, dt2), zoh_dgda_series2(x2));
+                                const float2 big = __fmul2_rn(dt2, __fmul2_rn(__fadd2_rn(ab, make_float2(-phi.x, -phi.y)), iv[pr]));
+                                const float2 dgda = make_float2(fabsf(x2.x) < kDgdaSmall ? ser.x : big.x,
+                                                                fabsf(x2.y) < kDgdaSmall ? ser.y : big.y);
+                                dA2[pr] = __ffma2_rn(l2[pr], __ffma2_rn(dt2, abh, __fmul2_rn(dgda, bu)), dA2[pr]);
+                            }
                             red[4 + 2 * pr] = rc.x;
                             red[5 + 2 * pr] = rc.y;
-                            s_dt2 = __ffma2_rn(l2[pr], __ffma2_rn(a2l[pr], abh, __fmul2_rn(bq[pr], uu2)), s_dt2);
-                            s_b2 = __ffma2_rn(l2[pr], bq[pr], s_b2);
-                            dA2[pr] = __ffma2_rn(__fmul2_rn(l2[pr], dt2), abh, dA2[pr]);
                             l2[pr] = __fmul2_rn(l2[pr], ab);                              // to h_t-1
                         }
                         ddt[t] += s_dt2.x + s_dt2.y;

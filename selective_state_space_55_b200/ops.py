@@ -361,15 +361,19 @@ def scan_bwd_workspace_bytes(batch, dim, dstate, seqlen, io_dtype=torch.bfloat16
 
 def selective_scan_bwd(u, delta, A, B, C, dout, D=None, z=None, delta_bias=None, softplus=True,
                        initial_state=None, dlast_state=None, flags=0, workspace=None,
-                       stream=None):
+                       stream=None, zoh=False):
     """Gradients of the scan through ``mamba_selective_scan_bwd``.
 
-    Same inputs as ``selective_scan_fwd`` (Euler term) plus dout (batch, dim, L)
-    in u's dtype and dlast_state (batch, dim, N) fp32 or None.  Returns a dict:
-    du, ddelta (and dz when z is given) in u's dtype; dA, dB, dC (and dD,
-    ddelta_bias, dinitial_state for the optional inputs given) in fp32.
+    Same inputs as ``selective_scan_fwd`` plus dout (batch, dim, L) in u's
+    dtype and dlast_state (batch, dim, N) fp32 or None; ``zoh`` sets
+    MAMBA_FLAG_ZOH (the zero-order-hold input term, as in the forward).
+    Returns a dict: du, ddelta (and dz when z is given) in u's dtype; dA, dB,
+    dC (and dD, ddelta_bias, dinitial_state for the optional inputs given) in
+    fp32.
     """
     batch, dim, L = u.shape
+    if zoh:
+        flags |= MAMBA_FLAG_ZOH
     N = A.shape[1]
     io, bc = u.dtype, B.dtype
     dev = u.device

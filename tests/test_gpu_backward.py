@@ -2,7 +2,8 @@
 the float64 oracle's adjoint, which finite differences of the forward oracle
 pin.  fp32 and bf16, with and without gate / D / bias / softplus / start
 state / last-state gradient, state sizes below 16, ragged lengths and channel
-counts, and sequences cut into many chained segments."""
+counts, sequences cut into many chained segments, and all of it again with
+the zero-order-hold input term."""
 import pytest
 import torch
 
@@ -35,16 +36,17 @@ def problem(batch, dim, L, dtype=torch.float32, N=16, seed=0, gated=True):
     return x
 
 
-def check(ref, x, tol, softplus=True, **kw):
+def check(ref, x, tol, softplus=True, zoh=False, **kw):
     g = ops.selective_scan_bwd(x["u"], x["delta"], x["A"], x["B"], x["C"], x["dout"], D=x["D"],
                                z=x["z"], delta_bias=x["delta_bias"], softplus=softplus,
-                               initial_state=x["h0"], dlast_state=x["dlast"], **kw)
+                               initial_state=x["h0"], dlast_state=x["dlast"], zoh=zoh, **kw)
     torch.cuda.synchronize()
     assert ops.device_status() == 0
     c = lambda t: None if t is None else t.cpu()  # noqa: E731
     o = ref.selective_scan_bwd(c(x["u"]), c(x["delta"]), c(x["A"]), c(x["B"]), c(x["C"]),
                                c(x["dout"]), D=c(x["D"]), z=c(x["z"]), delta_bias=c(x["delta_bias"]),
-                               softplus=softplus, initial_state=c(x["h0"]), dlast_state=c(x["dlast"]))
+                               softplus=softplus, initial_state=c(x["h0"]), dlast_state=c(x["dlast"]),
+                               zoh=zoh)
     assert set(g) == set(o), (set(g), set(o))
     errs = {k: max_rel_err(g[k], o[k]) for k in o}
     bad = {k: e for k, e in errs.items() if e > tol}
@@ -95,8 +97,39 @@ def test_unaligned_rows_take_scalar_path(ref):
     check(ref, problem(2, 36, 301, seed=23), FP32_TOL)
 
 
-def test_zoh_is_rejected():
-    x = problem(1, 32, 64, seed=24)
-    with pytest.raises(ops.MambaError, match="UNSUPPORTED"):
-        ops.selective_scan_bwd(x["u"], x["delta"], x["A"], x["B"], x["C"], x["dout"],
-                               flags=ops.MAMBA_FLAG_ZOH)
+# ---- zero-order-hold input term (MAMBA_FLAG_ZOH)
+
+def test_zoh_fp32_all_gradients(ref):
+    check(ref, problem(2, 70, 300, seed=31), FP32_TOL, zoh=True)
+
+
+def test_zoh_fp32_plain(ref):
+    x = problem(2, 40, 200, seed=32, gated=False)
+    x["delta"] = x["delta"].abs() * 0.1
+    check(ref, x, FP32_TOL, softplus=False, zoh=True)
+
+
+def test_zoh_small_and_zero_A(ref):
+    """Entries of A at 0 (the gain's limit Delta) and near 0, where dg/dA takes
+    its series; others across the closed form's range."""
+    x = problem(2, 64, 256, seed=33)
+    A = x["A"].clone()
+    A[:, 0] = 0.0
+    A[:, 1] = -1e-3
+    A[:, 2] = -0.05
+    A[:, 3] = -0.6
+    x["A"] = A
+    check(ref, x, FP32_TOL, zoh=True)
+
+
+@pytest.mark.parametrize("N", [1, 5, 16])
+def test_zoh_state_sizes(ref, N):
+    check(ref, problem(1, 33, 130, N=N, seed=34 + N), FP32_TOL, zoh=True)
+
+
+def test_zoh_many_segments(ref):
+    check(ref, problem(1, 64, 4096, seed=35), FP32_TOL, zoh=True)
+
+
+def test_zoh_bf16_layer_recipe(ref):
+    check(ref, problem(2, 256, 2048, dtype=torch.bfloat16, seed=36), BF16_TOL, zoh=True)
