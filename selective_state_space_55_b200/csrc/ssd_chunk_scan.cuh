@@ -56,17 +56,17 @@ constexpr int kSsdN = 128;         // state size
 constexpr int kSsdQ = 128;         // chunk length
 constexpr int kSsdThreads = 256;   // two threads per TMEM lane
 constexpr int kSsdTmemCols = 256;
+constexpr int kSsdStoreThread = 32;   // issues the output stores (not thread 0, which issues the products)
 
-// Tensor-memory columns (fp32 unless packed).  G fills [0, 128) until the
-// masked matrix has been formed from it; Gm's lo half (bf16 pairs, K = j)
-// then takes [0, 64).  S fills [192, 256) until the state update has read it;
-// Gm's hi half then takes it.  Y holds C H^T, is scaled in place by 2^(c_i)
-// per row, and MMA 2 accumulates Gm X onto it: the output before the gate.
+// Tensor-memory columns (fp32).  G fills [0, 128) until the masked matrix has
+// been formed from it; quarter q of Gm (columns j = 32 q .. 32 q + 31, bf16
+// pairs) then takes G's own quarter: its lo words in 32 q .. 32 q + 15, its
+// hi words in 32 q + 16 .. 32 q + 31.  Y holds C H^T, is scaled in place by
+// 2^(c_i) per row, and MMA 2 accumulates Gm X onto it: the output before the
+// gate.  S is the chunk's state product.
 constexpr uint32_t kTmG = 0;
-constexpr uint32_t kTmGmLo = 0;
 constexpr uint32_t kTmY = 128;
 constexpr uint32_t kTmS = 192;
-constexpr uint32_t kTmGmHi = 192;
 
 // Shared-memory map (bytes).  Every operand tile is 128 rows in the
 // 128-byte-swizzle layout of the tensor cores: each group of 64 columns
@@ -75,9 +75,9 @@ constexpr uint32_t kTmGmHi = 192;
 // 16 KB apart.  ssd_sw128 gives the byte offset.
 constexpr int kSsdOffC = 0;          // 128 x 128 bf16: C (rows i, k = n)
 constexpr int kSsdOffB = 32768;      // 128 x 128 bf16: B (rows j, k = n); once MMA 1 and 4
-                                     // are done, its first half takes the gate tile z and
-                                     // then the output tile (rows i, 64 columns p)
-constexpr int kSsdOffX = 65536;      // 128 x 64 bf16: x (rows j, k = p)
+                                     // are done, its first half takes the gate tile z
+constexpr int kSsdOffX = 65536;      // 128 x 64 bf16: x (rows j, k = p); once MMA 2 is
+                                     // done, the output tile (rows i, 64 columns p)
 constexpr int kSsdOffHX = 81920;     // hi at +0, lo at +16384, each 128 x 64 bf16:
                                      // H (rows n, k = p) for MMA 3, then Xw (rows j, k = p)
 constexpr int kSsdOffE = 114688;     // 128 fp32: -e_j, e_j = c_j - log2(Delta_j)
@@ -301,17 +301,6 @@ __device__ __forceinline__ void tmem_st32f(uint32_t taddr, const float (&a)[32])
     tmem_st16(taddr + 16, hi);
 }
 
-// Wait for one completion of an mbarrier; true on every thread if any
-// thread's bounded wait gave up.  Also a CTA-wide barrier, which orders this
-// thread's earlier tensor-memory accesses before the other threads' later ones.
-__device__ __forceinline__ bool ssd_wait_failed(uint32_t bar, uint32_t parity) {
-    const bool ok = mbar_wait_bounded(bar, parity);
-    tc_fence_before();
-    const bool failed = __syncthreads_or(!ok) != 0;
-    tc_fence_after();
-    return failed;
-}
-
 // Two threads serve each TMEM lane (row) r: threads r and r + 128 ("halves"
 // hp = 0, 1), each with half of the head dimension (columns 32 hp .. 32 hp +
 // 31 of x, Xw, H, y) and every other column quarter of the masked matrix.
@@ -371,17 +360,29 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
     fence_proxy_async_smem();
 
     const int64_t nchunks = (L + kSsdQ - 1) / kSsdQ;
-    // Every thread tracks, per mbarrier, whether a completion is outstanding
-    // (`pend`) and the parity of the next one (`phase`); the issuing thread's
-    // copy tells a failed CTA what it must still wait for before it leaves.
-    uint32_t pend = 0, phase = 0;
-    bool failed = false;
-    auto issued = [&](int k) { pend |= 1u << k; };
-    auto wait_on = [&](int k) -> bool {
-        if (ssd_wait_failed(bar(k), (phase >> k) & 1u)) return true;
-        pend &= ~(1u << k);
-        phase ^= 1u << k;
-        return false;
+    // Each mbarrier completes once per chunk, so the parity of chunk c's
+    // completion is c & 1.  Threads wait (bounded) on the barriers whose data
+    // they read; a CTA-wide barrier sits only where threads hand each other
+    // data (4 per chunk), and it also spreads a failed wait to every thread.
+    // Thread 0 issues every copy and product and tracks which completions are
+    // outstanding (`pend`) and their parity (`par`, that of the chunk whose
+    // data they carry): a failed CTA waits for them before it leaves.
+    uint32_t pend = 0, par = 0;
+    bool failed = false, lost = false;   // lost: this thread's own wait gave up
+    auto issued = [&](int k, int64_t chunk) {
+        pend |= 1u << k;
+        par = (par & ~(1u << k)) | ((uint32_t)(chunk & 1) << k);
+    };
+    auto poll = [&](int k, int64_t c) {
+        if (!mbar_wait_bounded(bar(k), (uint32_t)(c & 1))) lost = true;
+        else if (tid == 0) pend &= ~(1u << k);
+        tc_fence_after();
+    };
+    auto sync_failed = [&]() -> bool {   // CTA barrier; true on every thread if any wait gave up
+        tc_fence_before();
+        const bool f = __syncthreads_or(lost) != 0;
+        tc_fence_after();
+        return f;
     };
     // K-major operand, K step k of 16 columns: 32 bytes along the swizzled
     // 128-byte rows, the second 64 columns one half (16 KB) further.
@@ -393,19 +394,18 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
     };
     float dt_next = load_dt(r);
 
-    if (nchunks > 0) {
-        if (tid == 0) {
-            mbar_arrive_expect_tx(bar(kBarC), 32768);
-            tma_load_tile(s0 + kSsdOffC, &tm_C, 0, g, b, bar(kBarC));
-            mbar_arrive_expect_tx(bar(kBarB), 32768);
-            tma_load_tile(s0 + kSsdOffB, &tm_B, 0, g, b, bar(kBarB));
-            mbar_arrive_expect_tx(bar(kBarX), 16384);
-            tma_load_tile(s0 + kSsdOffX, &tm_x, 0, h, b, bar(kBarX));
-        }
-        issued(kBarC);
-        issued(kBarB);
-        issued(kBarX);
+    if (nchunks > 0 && tid == 0) {
+        mbar_arrive_expect_tx(bar(kBarC), 32768);
+        tma_load_tile(s0 + kSsdOffC, &tm_C, 0, g, b, bar(kBarC));
+        mbar_arrive_expect_tx(bar(kBarB), 32768);
+        tma_load_tile(s0 + kSsdOffB, &tm_B, 0, g, b, bar(kBarB));
+        mbar_arrive_expect_tx(bar(kBarX), 16384);
+        tma_load_tile(s0 + kSsdOffX, &tm_x, 0, h, b, bar(kBarX));
+        issued(kBarC, 0);
+        issued(kBarB, 0);
+        issued(kBarX, 0);
     }
+    __syncthreads();   // the start state's hi/lo pair is in HX
 
     constexpr uint32_t id_g = umma_idesc_bf16(128, 128, false, false);
     constexpr uint32_t id_off = umma_idesc_bf16(128, 64, false, true);
@@ -416,10 +416,11 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
         const int l0 = (int)(c * kSsdQ);
         const bool more = c + 1 < nchunks;
 
-        // ---- C landed (the barrier also publishes the entering state's hi/lo
-        // pair): MMA 3, Y = C (H_hi + H_lo)^T.
-        if (wait_on(kBarC)) { failed = true; break; }
+        // ---- C landed: MMA 3, Y = C (H_hi + H_lo)^T (HX holds the entering
+        // state's pair, published by the previous chunk's last barrier).
         if (tid == 0) {
+            poll(kBarC, c);
+            tc_fence_after();
 #pragma unroll
             for (int k = 0; k < kSsdN / 16; ++k)
                 umma_bf16(tmem + kTmY, umma_sdesc_sw128(s0 + kSsdOffC + kmaj(k), 16, 1024),
@@ -430,8 +431,8 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
                           umma_sdesc_sw128(s0 + kSsdOffHX + kSsdLoBytes + k * 2048, 16384, 1024),
                           id_off, 1);
             umma_commit(bar(kBarYoff));
+            issued(kBarYoff, c);
         }
-        issued(kBarYoff);
 
         // ---- Delta, the running log2-decay c_i and e_i = c_i - log2(Delta_i),
         // while MMA 3 runs.
@@ -448,7 +449,7 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
             if (lane >= o) a += v;
         }
         if (lane == 31) sTot[wq] = a;
-        __syncthreads();
+        __syncthreads();                                                 // barrier 1
         float pre = 0.0f;
         for (int w = 0; w < wq; ++w) pre += sTot[w];
         const float ci = a + pre;
@@ -459,8 +460,8 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
         // ---- x landed and MMA 3 is done with the HX buffer: Xw_j hi/lo
         // (row j = r, this half's columns), Xw_j = 2^(c_Q - e_j) x_j; and
         // Y_i = 2^(c_i) Y_i in place, onto which MMA 2 will accumulate.
-        if (wait_on(kBarX)) { failed = true; break; }
-        if (wait_on(kBarYoff)) { failed = true; break; }
+        poll(kBarX, c);
+        poll(kBarYoff, c);
         {
             const float w = ex2_approx(cQ - e_own);
             const float2 w2 = make_float2(w, w);
@@ -495,11 +496,13 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
             }
             tmem_st32f(tlane + kTmY + 32 * hp, y);
         }
+        tmem_wait_st();
 
-        // ---- B landed (the barrier also publishes Xw and e): MMA 4,
-        // S^T = B^T (Xw_hi + Xw_lo), committed alone, then MMA 1, G = C B^T.
-        if (wait_on(kBarB)) { failed = true; break; }
+        // ---- every Xw row and e are written: MMA 4, S^T = B^T (Xw_hi + Xw_lo),
+        // committed alone, then MMA 1, G = C B^T.
+        if (sync_failed()) { failed = true; break; }                    // barrier 2
         if (tid == 0) {
+            poll(kBarB, c);
 #pragma unroll
             for (int k = 0; k < kSsdQ / 16; ++k)
                 umma_bf16(tmem + kTmS, umma_sdesc_sw128(s0 + kSsdOffB + k * 2048, 16384, 1024),
@@ -515,14 +518,14 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
                 umma_bf16(tmem + kTmG, umma_sdesc_sw128(s0 + kSsdOffC + kmaj(k), 16, 1024),
                           umma_sdesc_sw128(s0 + kSsdOffB + kmaj(k), 16, 1024), id_g, k);
             umma_commit(bar(kBarG));
+            issued(kBarS, c);
+            issued(kBarG, c);
         }
-        issued(kBarS);
-        issued(kBarG);
 
         // ---- state: H = 2^(c_Q) H + S (row n = r, this half's columns), in
         // registers while MMA 1 runs; its hi/lo pair goes to the HX buffer,
         // which MMA 4 no longer reads, for the next chunk's MMA 3.
-        if (wait_on(kBarS)) { failed = true; break; }
+        poll(kBarS, c);
         {
             const float dq = ex2_approx(cQ);
             float sv[32];
@@ -540,36 +543,36 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
 
         // ---- MMA 1 done: C and B are free.  Next chunk's C; this chunk's gate
         // tile into B's first half.
-        if (wait_on(kBarG)) { failed = true; break; }
+        poll(kBarG, c);
         if (tid == 0) {
             if (more) {
                 mbar_arrive_expect_tx(bar(kBarC), 32768);
                 tma_load_tile(s0 + kSsdOffC, &tm_C, l0 + kSsdQ, g, b, bar(kBarC));
+                issued(kBarC, c + 1);
             }
             if (has_z) {
                 mbar_arrive_expect_tx(bar(kBarZ), 16384);
                 tma_load_tile(s0 + kSsdOffB, &tm_z, l0, h, b, bar(kBarZ));
+                issued(kBarZ, c);
             }
         }
-        if (more) issued(kBarC);
-        if (has_z) issued(kBarZ);
 
         // ---- Gm_ij = G_ij 2^(c_i - e_j) for j <= i (row i = r), as hi/lo pairs
-        // into tensor memory.  Rows [32 wq, 32 wq + 32) need column quarters
-        // 0 .. wq (quarter wq straddles the diagonal); the quarters above are
-        // zero.  This half takes quarters hp and hp + 2, so no warp forms more
-        // than two.  The hi words go to the S columns at once; the lo words
-        // overwrite G's first half, so they wait until both halves have read G.
-        uint32_t keep_lo[2][16];
+        // written over the G columns they come from.  Rows [32 wq, 32 wq + 32)
+        // need column quarters 0 .. wq (quarter wq straddles the diagonal); the
+        // quarters above are zero.  This half takes quarters hp and hp + 2, so
+        // no warp forms more than two; quarter q's lo words go to its own
+        // columns 32 q .. 32 q + 15 and its hi words to 32 q + 16 .. 32 q + 31,
+        // which this thread has read already and no other thread touches.
         {
             const float2 ci2 = make_float2(ci, ci);
 #pragma unroll
             for (int s = 0; s < 2; ++s) {
                 const int quarter = hp + 2 * s;
-                uint32_t hi[16];
+                uint32_t hi[16], lo[16];
                 if (quarter > wq) {
 #pragma unroll
-                    for (int k = 0; k < 16; ++k) hi[k] = keep_lo[s][k] = 0u;
+                    for (int k = 0; k < 16; ++k) hi[k] = lo[k] = 0u;
                 } else {
                     float gv[32];
                     tmem_ld32(tlane + kTmG + 32 * quarter, gv);
@@ -597,45 +600,37 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
                         }
 #pragma unroll
                         for (int k = 0; k < 4; ++k)
-                            split_bf16x2(f[2 * k], f[2 * k + 1], hi[q * 4 + k], keep_lo[s][q * 4 + k]);
+                            split_bf16x2(f[2 * k], f[2 * k + 1], hi[q * 4 + k], lo[q * 4 + k]);
                     }
                 }
-                tmem_st16(tlane + kTmGmHi + 16 * quarter, hi);
+                tmem_st16(tlane + kTmG + 32 * quarter, lo);
+                tmem_st16(tlane + kTmG + 32 * quarter + 16, hi);
             }
         }
-        tc_fence_before();
-        __syncthreads();   // every G column has been read
-        tc_fence_after();
-#pragma unroll
-        for (int s = 0; s < 2; ++s) tmem_st16(tlane + kTmGmLo + 16 * (hp + 2 * s), keep_lo[s]);
         tmem_wait_st();
-        tc_fence_before();
-        __syncthreads();
 
-        // ---- MMA 2: Y += (Gm_hi + Gm_lo) X, A from tensor memory.
+        // ---- every Gm row and the rescaled Y are in place: MMA 2,
+        // Y += (Gm_hi + Gm_lo) X, A from tensor memory (K step k: columns
+        // 16 k .. 16 k + 15 of quarter k / 2).
+        if (sync_failed()) { failed = true; break; }                    // barrier 3
         if (tid == 0) {
-            tc_fence_after();
 #pragma unroll
             for (int k = 0; k < kSsdQ / 16; ++k)
-                umma_bf16_ta(tmem + kTmY, tmem + kTmGmHi + 8 * k,
+                umma_bf16_ta(tmem + kTmY, tmem + kTmG + 32 * (k >> 1) + 16 + 8 * (k & 1),
                              umma_sdesc_sw128(s0 + kSsdOffX + k * 2048, 16384, 1024), id_y, 1);
 #pragma unroll
             for (int k = 0; k < kSsdQ / 16; ++k)
-                umma_bf16_ta(tmem + kTmY, tmem + kTmGmLo + 8 * k,
+                umma_bf16_ta(tmem + kTmY, tmem + kTmG + 32 * (k >> 1) + 8 * (k & 1),
                              umma_sdesc_sw128(s0 + kSsdOffX + k * 2048, 16384, 1024), id_y, 1);
             umma_commit(bar(kBarYd));
+            issued(kBarYd, c);
         }
-        issued(kBarYd);
-        if (wait_on(kBarYd)) { failed = true; break; }
-        if (tid == 0 && more) {   // x is no longer read
-            mbar_arrive_expect_tx(bar(kBarX), 16384);
-            tma_load_tile(s0 + kSsdOffX, &tm_x, l0 + kSsdQ, h, b, bar(kBarX));
-        }
-        if (more) issued(kBarX);
-        if (has_z && wait_on(kBarZ)) { failed = true; break; }
+        poll(kBarYd, c);
+        if (has_z) poll(kBarZ, c);
 
         // ---- y_i = Y_i (row i = r, this half's columns), gated, written as
-        // bf16 over the gate tile, then stored by TMA (rows past the end dropped).
+        // bf16 over the x tile (no longer read), then stored by TMA (rows past
+        // the end dropped).
         {
             float y[32];
             tmem_ld32(tlane + kTmY + 32 * hp, y);
@@ -661,37 +656,44 @@ __global__ void __launch_bounds__(kSsdThreads, 2)
                         f[k + 1] = v.y;
                     }
                 }
-                *reinterpret_cast<uint4*>(smem + kSsdOffB + off) = pack16(f);
+                *reinterpret_cast<uint4*>(smem + kSsdOffX + off) = pack16(f);
             }
         }
         fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();   // the output tile is complete
-        if (tid == 0) {
-            tma_store_tile(&tm_out, s0 + kSsdOffB, l0, h, b);
+        if (sync_failed()) { failed = true; break; }                    // barrier 4
+        // The gate tile is consumed: thread 0 requests the next chunk's B and
+        // moves on.  Thread kSsdStoreThread stores the output tile and, once
+        // the store has read it, requests the next chunk's x into it.
+        if (tid == 0 && more) {
+            mbar_arrive_expect_tx(bar(kBarB), 32768);
+            tma_load_tile(s0 + kSsdOffB, &tm_B, l0 + kSsdQ, g, b, bar(kBarB));
+            issued(kBarB, c + 1);
+        }
+        if (tid == kSsdStoreThread) {
+            tma_store_tile(&tm_out, s0 + kSsdOffX, l0, h, b);
             bulk_commit();
-            if (more) {    // the store has read the tile: the next chunk's B may land there
+            if (more) {
                 bulk_wait_read<0>();
-                mbar_arrive_expect_tx(bar(kBarB), 32768);
-                tma_load_tile(s0 + kSsdOffB, &tm_B, l0 + kSsdQ, g, b, bar(kBarB));
+                mbar_arrive_expect_tx(bar(kBarX), 16384);
+                tma_load_tile(s0 + kSsdOffX, &tm_x, l0 + kSsdQ, h, b, bar(kBarX));
             }
         }
-        if (more) issued(kBarB);
+        if (tid == 0 && more) issued(kBarX, c + 1);
     }
 
     if (!failed && p.hT) {
 #pragma unroll
         for (int q = 0; q < kSsdP / 2; ++q) p.hT[hoff + (size_t)q * kSsdN] = H[q];
     }
+    if (tid == kSsdStoreThread) bulk_wait<0>();   // output stores done before shared memory goes
     if (tid == 0) {
-        bulk_wait<0>();   // output stores done before the CTA's shared memory goes
         // After a timeout, wait (bounded) for every copy and product still in
         // flight, so that none lands in shared or tensor memory after the CTA
         // has released them.
         if (failed) {
 #pragma unroll 1
             for (int k = 0; k < kSsdBars; ++k)
-                if ((pend >> k) & 1u) (void)mbar_wait_bounded(bar(k), (phase >> k) & 1u);
+                if ((pend >> k) & 1u) (void)mbar_wait_bounded(bar(k), (par >> k) & 1u);
         }
     }
     tc_fence_before();
