@@ -749,8 +749,10 @@ def bench_conv(args, rank, world, local):
         ops.causal_conv1d_fwd(x, w, bias=bias, out=out, final_conv_state=fin)
 
     def decode():
+        # each layer has its own conv state: dependent launches (MAMBA_FLAG_PDL)
         for ly in lay:
-            ops.causal_conv1d_update(ly["st"], ly["x"], ly["w"], bias=ly["b"], out=ly["out"])
+            ops.causal_conv1d_update(ly["st"], ly["x"], ly["w"], bias=ly["b"], out=ly["out"],
+                                     flags=ops.MAMBA_FLAG_PDL)
 
     decode()
     torch.cuda.synchronize()

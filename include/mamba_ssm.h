@@ -425,7 +425,14 @@ MAMBA_API mamba_status_t mamba_selective_scan_bwd(
  *                       by one with x appended, then used for the sum
  *   x, out              (batch, dim), io_dtype
  * dims: batch, dim, seqlen (prefill) and io_dtype are read; dstate, bc_dtype
- * and the workspace are ignored.  width must be 1..MAMBA_MAX_CONV_WIDTH
+ * and the workspace are ignored.  For the update, dims->flags may hold
+ * MAMBA_FLAG_PDL: with width 4 and conv_state, x and out aligned to their
+ * vectors, the update is then launched as a programmatic dependent launch that
+ * may start while the previous kernel on the stream finishes; it reads its own
+ * conv_state first and waits for that kernel before it reads x or writes
+ * anything.  Set it only when the previous kernel neither reads nor writes this
+ * call's conv_state (consecutive layers of a decode step); results are then
+ * identical with and without it.  width must be 1..MAMBA_MAX_CONV_WIDTH
  * (MAMBA_ERR_UNSUPPORTED otherwise).  Both calls are asynchronous on `stream`
  * and allocate nothing.
  */

@@ -269,15 +269,25 @@ __device__ __forceinline__ void store_vec(IoT* dst, const float (&v)[kC]) {
     }
 }
 
-template <typename IoT, int kC>
+// kPdl: launched as a programmatic dependent launch.  The next launch on the
+// stream may start at once; this one reads its own conv state, then waits for
+// the previous launch to complete before it reads x and writes anything (the
+// caller guarantees that the previous launch neither reads nor writes this
+// call's state).
+template <typename IoT, int kC, bool kPdl>
 __global__ void __launch_bounds__(kConvThreads)
     causal_conv1d_update_w4xn_kernel(const __grid_constant__ ConvParams p) {
+    if (kPdl) grid_launch_dependents();
     const int64_t c0 = kC * ((int64_t)blockIdx.x * kConvThreads + threadIdx.x);
-    if (c0 >= p.chains) return;
+    if (c0 >= p.chains) {
+        if (kPdl) grid_dependency_wait();
+        return;
+    }
     IoT* st = static_cast<IoT*>(p.state) + c0 * 4;
     const IoT* xs = static_cast<const IoT*>(p.x) + c0;
     IoT* os = static_cast<IoT*>(p.out) + c0;
     if (c0 + kC > p.chains) {                           // tail, one chain at a time
+        if (kPdl) grid_dependency_wait();
         for (int64_t c = c0; c < p.chains; ++c) {
             IoT* sc = st + (c - c0) * 4;
             const float cur[4] = {DType<IoT>::load(sc + 1), DType<IoT>::load(sc + 2),
@@ -295,6 +305,7 @@ __global__ void __launch_bounds__(kConvThreads)
 #pragma unroll
         for (int j = 0; j < 4; ++j) old[4 * c + j] = v[j];
     }
+    if (kPdl) grid_dependency_wait();
     load_vec<IoT, kC>(xs, xin);
     float o[kC];
 #pragma unroll

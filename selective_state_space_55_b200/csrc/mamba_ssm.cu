@@ -1092,12 +1092,30 @@ MAMBA_API mamba_status_t mamba_causal_conv1d_update(void* conv_state, const void
                       aligned(out, kC * es) && aligned(weight, 16);
     const bool w4 = width == 4 && aligned(conv_state, 4 * es) && aligned(weight, 16);
     const unsigned int grid = blocks_for(w4xn ? (chains + kC - 1) / kC : chains);
-    if (dims->io_dtype == MAMBA_BF16) {
-        if (w4xn) causal_conv1d_update_w4xn_kernel<__nv_bfloat16, kC><<<grid, kConvThreads, 0, stream>>>(prm);
+    // MAMBA_FLAG_PDL: the vector path as a programmatic dependent launch (the
+    // other paths ignore the flag).
+    const bool pdl = w4xn && (dims->flags & MAMBA_FLAG_PDL) != 0;
+    if (pdl) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(grid);
+        cfg.blockDim = dim3(kConvThreads);
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        const cudaError_t e =
+            dims->io_dtype == MAMBA_BF16
+                ? cudaLaunchKernelEx(&cfg, causal_conv1d_update_w4xn_kernel<__nv_bfloat16, kC, true>, prm)
+                : cudaLaunchKernelEx(&cfg, causal_conv1d_update_w4xn_kernel<float, kC, true>, prm);
+        if (e != cudaSuccess) return MAMBA_ERR_CUDA;
+    } else if (dims->io_dtype == MAMBA_BF16) {
+        if (w4xn) causal_conv1d_update_w4xn_kernel<__nv_bfloat16, kC, false><<<grid, kConvThreads, 0, stream>>>(prm);
         else if (w4) causal_conv1d_update_w4_kernel<__nv_bfloat16><<<grid, kConvThreads, 0, stream>>>(prm);
         else causal_conv1d_update_kernel<__nv_bfloat16><<<grid, kConvThreads, 0, stream>>>(prm);
     } else {
-        if (w4xn) causal_conv1d_update_w4xn_kernel<float, kC><<<grid, kConvThreads, 0, stream>>>(prm);
+        if (w4xn) causal_conv1d_update_w4xn_kernel<float, kC, false><<<grid, kConvThreads, 0, stream>>>(prm);
         else if (w4) causal_conv1d_update_w4_kernel<float><<<grid, kConvThreads, 0, stream>>>(prm);
         else causal_conv1d_update_kernel<float><<<grid, kConvThreads, 0, stream>>>(prm);
     }

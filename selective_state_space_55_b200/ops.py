@@ -452,9 +452,12 @@ def causal_conv1d_fwd(x, weight, bias=None, initial_conv_state=None, silu=True, 
     return out
 
 
-def causal_conv1d_update(conv_state, x, weight, bias=None, silu=True, out=None, stream=None):
+def causal_conv1d_update(conv_state, x, weight, bias=None, silu=True, out=None, stream=None,
+                         flags=0):
     """One token of the short convolution through ``mamba_causal_conv1d_update``;
-    ``conv_state`` (batch, dim, W) is shifted in place.  Returns ``out`` (batch, dim)."""
+    ``conv_state`` (batch, dim, W) is shifted in place.  ``flags`` may hold
+    MAMBA_FLAG_PDL (dependent launch; the previous kernel on the stream must
+    not touch this conv state).  Returns ``out`` (batch, dim)."""
     batch, dim, W = conv_state.shape
     io = x.dtype
     _check_cuda("conv_state", conv_state, (io,), (batch, dim, W))
@@ -465,6 +468,7 @@ def causal_conv1d_update(conv_state, x, weight, bias=None, silu=True, out=None, 
         out = torch.empty_like(x)
     _check_cuda("out", out, (io,), (batch, dim))
     dims = _conv_dims(batch, dim, 0, io)
+    dims.flags = flags
     rc = library().mamba_causal_conv1d_update(
         _ptr(conv_state), _ptr(x), _ptr(weight), _ptr(bias), W, int(bool(silu)), _ptr(out),
         ctypes.byref(dims), _stream_handle(stream))

@@ -165,3 +165,43 @@ def test_update_one_chain_per_thread_path(ref):
     o_st, o_out = ref.causal_conv1d_update(c(init), c(xt), c(w), bias=c(bias))
     assert max_rel_err(st, o_st) == 0.0
     assert max_rel_err(out, o_out) <= tol_for(torch.bfloat16)
+
+
+def test_update_dependent_launch_is_bitwise_identical():
+    """MAMBA_FLAG_PDL on the W = 4 decode update (each layer's launch may start
+    while the previous layer's finishes; the layers' conv states are distinct):
+    the same states and outputs bit for bit as plain launches, over 48 layers x
+    3 tokens inside a CUDA graph."""
+    g = torch.Generator(device=DEV)
+    g.manual_seed(91)
+    L, batch, dim = 48, 8, 512
+    base = [torch.randn(batch, dim, 4, generator=g, device=DEV).to(torch.bfloat16) for _ in range(L)]
+    xs = [[torch.randn(batch, dim, generator=g, device=DEV).to(torch.bfloat16) for _ in range(L)]
+          for _ in range(3)]
+    ws = [torch.randn(dim, 4, generator=g, device=DEV) for _ in range(L)]
+    bs = [torch.randn(dim, generator=g, device=DEV) for _ in range(L)]
+    results = []
+    for flags in (0, ops.MAMBA_FLAG_PDL):
+        states = [b.clone() for b in base]
+        outs = [[torch.empty_like(x) for x in row] for row in xs]
+        graphs = []
+        for t in range(3):
+            keep = [st.clone() for st in states]
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                for i in range(L):
+                    ops.causal_conv1d_update(states[i], xs[t][i], ws[i], bias=bs[i],
+                                             out=outs[t][i], flags=flags)
+            for st, k in zip(states, keep):
+                st.copy_(k)
+            graphs.append(graph)
+        for graph in graphs:
+            graph.replay()
+        torch.cuda.synchronize()
+        results.append((states, outs))
+    (s0, o0), (s1, o1) = results
+    for a, b in zip(s0, s1):
+        assert torch.equal(a, b)
+    for ra, rb in zip(o0, o1):
+        for a, b in zip(ra, rb):
+            assert torch.equal(a, b)
