@@ -178,7 +178,7 @@ class Workload:
 
     def __init__(self, rank: int, scan_batch: int | None = None, decode_layers: int | None = None,
                  only: str | None = None, scan_workload: str = SCAN_WORKLOAD,
-                 scan_variant: str = "euler"):
+                 scan_variant: str = "euler", scan_seqlen: int | None = None):
         from selective_state_space_55_b200 import inputs as I
         from selective_state_space_55_b200 import ops
 
@@ -188,6 +188,8 @@ class Workload:
         self.cfg = I.SCAN_CONFIGS[scan_workload]
         if scan_batch:
             self.cfg = self.cfg.resized(batch=scan_batch)
+        if scan_seqlen:
+            self.cfg = self.cfg.resized(seqlen=scan_seqlen)
         self.dcfg = I.DECODE_CONFIG
         if decode_layers:
             self.dcfg = I.DecodeConfig(self.dcfg.name, self.dcfg.batch, self.dcfg.dim,
@@ -546,10 +548,10 @@ def bench_ours(args, rank, world, local):
         cuda_build.build()
     barrier()
     torch.cuda.set_device(local)
-    partial = (args.only is not None or args.scan_batch or args.decode_layers
+    partial = (args.only is not None or args.scan_batch or args.decode_layers or args.scan_seqlen
                or args.scan_workload != SCAN_WORKLOAD or args.scan_variant != "euler")
     w = Workload(rank, args.scan_batch, args.decode_layers, args.only, args.scan_workload,
-                 args.scan_variant)
+                 args.scan_variant, args.scan_seqlen)
     c, d = w.cfg, w.dcfg
     w.capture_decode()
     for _ in range(args.warmup):
@@ -710,6 +712,7 @@ def bench_ours(args, rank, world, local):
         }
         if partial:
             line["partial_case"] = {"only": args.only, "scan_batch": args.scan_batch,
+                                    "scan_seqlen": args.scan_seqlen,
                                     "decode_layers": args.decode_layers,
                                     "scan_workload": args.scan_workload,
                                     "scan_variant": args.scan_variant,
@@ -1039,6 +1042,8 @@ def main():
                          "bwd: the backward pass; ssd: the Mamba-2 layer")
     ap.add_argument("--scan-batch", type=int, default=None,
                     help="profiling case: smaller scan batch")
+    ap.add_argument("--scan-seqlen", type=int, default=None,
+                    help="profiling case: shorter scan sequence")
     ap.add_argument("--decode-layers", type=int, default=None,
                     help="profiling case: fewer decode layers")
     ap.add_argument("--scan-workload", default=SCAN_WORKLOAD,

@@ -145,6 +145,27 @@ def test_parallel_matches_single_pass_closely(ref):
     assert max_rel_err(b, a) <= 1e-5 and max_rel_err(lb, la) <= 1e-5
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_parallel_correction_without_early_stop(ref, dtype):
+    """The parallel mode's correction walks a segment only while some
+    exp(A_n S_t) is above fp32's range; with a state entry at A = 0 it never
+    decays, so every segment is corrected to its end."""
+    x = layer_inputs(2, 48, 3000, dtype=dtype, seed=43)
+    A = x["A"].clone()
+    A[:, 3] = 0.0
+    x["A"] = A
+    check(ref, x, tol_for(dtype), num_chunks=5, flags=PAR)
+
+
+def test_parallel_correction_with_negative_delta(ref):
+    """Softplus off with delta + bias of both signs: the running sum of Delta
+    is not monotone, so the correction may not stop early."""
+    x = layer_inputs(1, 64, 2048, dtype=torch.float32, seed=44)
+    x["delta"] = (x["delta"] * 0.02).contiguous()
+    x["delta_bias"] = torch.full_like(x["delta_bias"], 0.005)
+    check(ref, x, FP32_TOL, softplus=False, num_chunks=6, flags=PAR)
+
+
 def test_many_groups_many_segments(ref):
     """More work items than resident warps, in both modes."""
     x = layer_inputs(4, 2048, 1024, seed=31)
