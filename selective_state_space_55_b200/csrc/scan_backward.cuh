@@ -32,12 +32,20 @@
 // run in reverse order: a segment starts from the lambda the later segment
 // left in an L2-resident carry buffer (release/acquire flag, bounded wait).
 // Within a block, for each quarter of the state (4 of the 16 entries) the lane
-// recomputes the block's 8 states from the checkpoint into registers, then
-// runs the adjoint backwards over them; Abar is computed again on the way
-// back rather than kept, and Abar_t h_t-1 is taken as h_t - Delta_t B_t u_t.  dB and dC sum over the channels of a batch row: the
-// warp reduces its 32 channels with shuffles (8 values per lane and step) and
-// one lane per value adds the sum to global memory atomically.  dA, dD and
-// the bias gradient are summed per lane over the segment and added once.
+// recomputes the block's 8 states and their Abar from the checkpoint into
+// registers, then runs the adjoint backwards over them, taking Abar_t h_t-1
+// as h_t - Delta_t B_t u_t.  The lane's per-entry values (A log2 e, lambda,
+// the running dA sum) wait in shared memory while other quarters run, so the
+// quarter loop indexes registers statically and is emitted once.  A block
+// shorter than 8 steps (the sequence's last) runs as a whole block whose
+// missing steps have Delta = 0, u = dout = 0 and B = C = 0: they leave the
+// state and lambda unchanged and contribute nothing.
+//
+// dB and dC sum over the channels of a batch row.  Per quarter and block each
+// lane writes its 64 partials (8 steps x 4 entries x dB, dC) as one row of a
+// per-warp table in shared memory; then each lane adds one pair of columns
+// over the 32 rows and adds the two sums to global memory atomically.  dA, dD
+// and the bias gradient are summed per lane over the segment and added once.
 #pragma once
 
 #include "selective_scan.cuh"
@@ -120,28 +128,6 @@ __device__ __forceinline__ void store_block(T* row, int64_t t0, int n, bool vec,
         if (i < n) DType<T>::store(row + t0 + i, v[i]);
 }
 
-// Sum of v[j] over the warp's 32 lanes for j < 8.  Three halving exchanges
-// leave lane l with the partial sum of value (l >> 2) over 8 lanes; two
-// butterflies complete it on all four lanes of the quad.
-__device__ __forceinline__ float warp_reduce8(float (&v)[8], int lane) {
-#pragma unroll
-    for (int lvl = 0; lvl < 3; ++lvl) {
-        const int off = 16 >> lvl;               // 16, 8, 4
-        const int half = 4 >> lvl;               // values kept: 4, 2, 1
-        const bool upper = (lane & off) != 0;
-#pragma unroll
-        for (int i = 0; i < half; ++i) {
-            const float send = upper ? v[i] : v[i + half];
-            const float keep = upper ? v[i + half] : v[i];
-            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-        }
-    }
-    float r = v[0];
-    r += __shfl_xor_sync(0xffffffffu, r, 2);
-    r += __shfl_xor_sync(0xffffffffu, r, 1);
-    return r;                                    // total of value (lane >> 2)
-}
-
 // 16-byte asynchronous copy global -> shared (L2 only), and its groups.
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)),
@@ -170,12 +156,20 @@ struct BwdStage {
     uint4 ck[32][4];
 };
 
-// Per warp: two stages, the B/C table of one block, and 1 / A of the lanes'
-// 16 state entries in quarters (zero-order hold).
+// Per warp: two stages, the B/C table of one block, the lanes' per-entry
+// values in quarters (A log2(e), lambda, the dA sum and, for the zero-order
+// hold, 1 / A), and the dB/dC partials of one quarter of one block.  Each lane
+// reads and writes only its own column of the per-entry values.
+constexpr int kEntA2 = 0, kEntLam = 1, kEntDA = 2, kEntInvA = 3, kEntRows = 4;
+// One lane's row of partials: 8 steps x (4 dB + 4 dC), padded to 68 floats so
+// that the lanes' 16-byte stores of one step fall in distinct banks.
+constexpr int kRedStride = 2 * 4 * kBwdSteps + 4;
+
 template <typename IoT, typename BcT>
 __host__ __device__ constexpr int bwd_warp_smem() {
     return 2 * (int)sizeof(BwdStage<IoT, BcT>) + kBwdSteps * 32 * (int)sizeof(float) +
-           (kNPad / 4) * 32 * (int)sizeof(float4);
+           kEntRows * (kNPad / 4) * 32 * (int)sizeof(float4) +
+           32 * kRedStride * (int)sizeof(float);
 }
 
 template <int kVecs>
@@ -191,17 +185,6 @@ __device__ __forceinline__ void unpack_rows(const uint4 (&r)[kVecs], float (&v)[
     }
 }
 
-// Move entries 4..15 down by four and 0..3 to the top (four calls restore the order).
-__device__ __forceinline__ void rotate_quarter(float (&v)[kNPad]) {
-    const float t0 = v[0], t1 = v[1], t2 = v[2], t3 = v[3];
-#pragma unroll
-    for (int i = 0; i < kNPad - 4; ++i) v[i] = v[i + 4];
-    v[kNPad - 4] = t0;
-    v[kNPad - 3] = t1;
-    v[kNPad - 2] = t2;
-    v[kNPad - 1] = t3;
-}
-
 __device__ __forceinline__ float sigmoid_f32(float x) {
     return __fdividef(1.0f, 1.0f + ex2_approx(-x * kLog2e));
 }
@@ -210,8 +193,9 @@ __device__ __forceinline__ float sigmoid_f32(float x) {
 // for bf16 inputs, the unbiased forms for fp32), so that the recomputed states
 // follow the forward's arithmetic.
 template <bool kExact>
-__device__ __forceinline__ float bwd_exp2(float x) {
-    return kExact ? exp2_near_one_exact(x) : ex2_approx(x);
+__device__ __forceinline__ float2 bwd_exp2x2(float2 x) {
+    if constexpr (kExact) return exp2_near_one_exact2(x);
+    return make_float2(ex2_approx(x.x), ex2_approx(x.y));
 }
 
 // dg/dA / Delta^2 = (x e^x - expm1(x)) / x^2 for x = Delta A, as its series
@@ -244,8 +228,16 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
     uint8_t* wbase = bwd_smem + warp * bwd_warp_smem<IoT, BcT>();
     Stage* stages = reinterpret_cast<Stage*>(wbase);
     float (*bcf)[32] = reinterpret_cast<float (*)[32]>(wbase + 2 * sizeof(Stage));
-    float4 (*inva4)[32] = reinterpret_cast<float4 (*)[32]>(
+    float4 (*ent)[kNPad / 4][32] = reinterpret_cast<float4 (*)[kNPad / 4][32]>(
         wbase + 2 * sizeof(Stage) + kBwdSteps * 32 * sizeof(float));
+    float (*rbuf)[kRedStride] = reinterpret_cast<float (*)[kRedStride]>(
+        wbase + 2 * sizeof(Stage) + kBwdSteps * 32 * sizeof(float) +
+        kEntRows * (kNPad / 4) * 32 * sizeof(float4));
+    // The partial this lane sums in the reduction of a quarter: dB (lanes
+    // 0..15) or dC (16..31), step (lane & 15) / 2, entries 2 (lane & 1) + 0, 1.
+    const int red_kind = lane >> 4;
+    const int red_t = (lane & 15) >> 1;
+    const int red_n = (lane & 1) * 2;
 
     for (;;) {
         unsigned int item = 0;
@@ -263,32 +255,37 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
         const int64_t t_begin = k * p.seg_len;
         const int64_t t_end = min(t_begin + p.seg_len, p.seqlen);
 
-        float a2[kNPad];
+        // per-entry values of the lane's channel, one float4 per quarter
 #pragma unroll
-        for (int n = 0; n < kNPad; ++n)
-            a2[n] = (valid && n < p.dstate) ? p.A[d * p.dstate + n] * kLog2e : 0.0f;
-        if (kZoh) {   // 1 / A_n, as the forward holds it (read back one quarter at a time)
+        for (int q = 0; q < kNPad / 4; ++q) {
+            float a2v[4], iva[4];
 #pragma unroll
-            for (int q = 0; q < kNPad / 4; ++q) {
-                float v[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int n = 4 * q + i;
-                    const float a = (valid && n < p.dstate) ? p.A[d * p.dstate + n] : 0.0f;
-                    v[i] = (valid && n < p.dstate) ? 1.0f / a : 0.0f;
-                }
-                inva4[q][lane] = make_float4(v[0], v[1], v[2], v[3]);
+            for (int i = 0; i < 4; ++i) {
+                const int n = 4 * q + i;
+                const bool on = valid && n < p.dstate;
+                const float a = on ? p.A[d * p.dstate + n] : 0.0f;
+                a2v[i] = a * kLog2e;
+                iva[i] = on ? 1.0f / a : 0.0f;       // 1 / A_n, as the forward holds it
             }
+            ent[kEntA2][q][lane] = make_float4(a2v[0], a2v[1], a2v[2], a2v[3]);
+            if (kZoh) ent[kEntInvA][q][lane] = make_float4(iva[0], iva[1], iva[2], iva[3]);
+            ent[kEntDA][q][lane] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
         }
         const float bias = (valid && p.delta_bias != nullptr) ? p.delta_bias[d] : 0.0f;
         const float Dd = (valid && p.D != nullptr) ? p.D[d] : 0.0f;
 
-        float lam[kNPad];
         if (kr == 0) {
 #pragma unroll
-            for (int n = 0; n < kNPad; ++n)
-                lam[n] = (valid && p.dlast != nullptr && n < p.dstate)
-                             ? p.dlast[chain * p.dstate + n] : 0.0f;
+            for (int q = 0; q < kNPad / 4; ++q) {
+                float l[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int n = 4 * q + i;
+                    l[i] = (valid && p.dlast != nullptr && n < p.dstate)
+                               ? p.dlast[chain * p.dstate + n] : 0.0f;
+                }
+                ent[kEntLam][q][lane] = make_float4(l[0], l[1], l[2], l[3]);
+            }
         } else {
             bool ok = true;
             if (lane == 0) {
@@ -310,14 +307,11 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
             float2 c2[kNPad / 2];
             load16(p.carry + chain * kNPad, c2);
 #pragma unroll
-            for (int i = 0; i < kNPad / 2; ++i) {
-                lam[2 * i] = valid ? c2[i].x : 0.0f;
-                lam[2 * i + 1] = valid ? c2[i].y : 0.0f;
-            }
+            for (int q = 0; q < kNPad / 4; ++q)
+                ent[kEntLam][q][lane] = valid ? make_float4(c2[2 * q].x, c2[2 * q].y,
+                                                            c2[2 * q + 1].x, c2[2 * q + 1].y)
+                                              : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
         }
-        float dA_acc[kNPad];
-#pragma unroll
-        for (int n = 0; n < kNPad; ++n) dA_acc[n] = 0.0f;
         float dD_acc = 0.0f, dbias_acc = 0.0f;
 
         const IoT* urow = static_cast<const IoT*>(p.u) + chain * p.seqlen;
@@ -370,34 +364,24 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
             }
             const bool staged = pipe && ns == kBwdSteps;
             const Stage& S = stages[j & 1];
-            // ---- inputs of this block: the lane's own channel, and the B/C table
+            const float4* ck4 = reinterpret_cast<const float4*>(
+                p.ckpt + (chain * p.ckpt_tiles + t0 / kBwdSteps) * kNPad);
+            // ---- inputs of this block: the lane's own channel, and the B/C table.
+            // Steps past the end of a short block read as zero.
             float uu[kBwdSteps], dt[kBwdSteps], dy[kBwdSteps], aux[kBwdSteps];
-            float4 ckv[4];
             if (valid && staged) {
                 unpack_rows<kIoVecs>(S.io[0][lane], uu);
                 unpack_rows<kIoVecs>(S.io[1][lane], dt);   // delta, turned into Delta below
                 unpack_rows<kIoVecs>(S.io[3][lane], dy);   // dout, turned into dy below
                 if (kHasZ) unpack_rows<kIoVecs>(S.io[2][lane], aux);
-#pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    const uint4 r = S.ck[lane][v];
-                    ckv[v] = make_float4(__uint_as_float(r.x), __uint_as_float(r.y),
-                                         __uint_as_float(r.z), __uint_as_float(r.w));
-                }
             } else if (valid) {
                 load_block(urow, t0, ns, vec, uu);
                 load_block(drow, t0, ns, vec, dt);
                 load_block(grow, t0, ns, vec, dy);
                 if (kHasZ) load_block(zrow, t0, ns, vec, aux);
-                const float4* ck4 = reinterpret_cast<const float4*>(
-                    p.ckpt + (chain * p.ckpt_tiles + t0 / kBwdSteps) * kNPad);
-#pragma unroll
-                for (int v = 0; v < 4; ++v) ckv[v] = __ldcg(ck4 + v);
             } else {
 #pragma unroll
                 for (int i = 0; i < kBwdSteps; ++i) uu[i] = dt[i] = dy[i] = aux[i] = 0.0f;
-#pragma unroll
-                for (int v = 0; v < 4; ++v) ckv[v] = make_float4(0.f, 0.f, 0.f, 0.f);
             }
             {
                 float row[kBwdSteps];
@@ -414,37 +398,42 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
                 for (int i = 0; i < kBwdSteps; ++i) bcf[i][lane] = row[i];
                 __syncwarp();
             }
-            // Delta, the softplus derivative (kept in dt / sp), dy and the gate factor.
-            float sp[kBwdSteps];
+            // Delta, dy and the gate factor.  Delta is zero past the block's
+            // end, so that those steps leave the state and lambda as they are
+            // (Abar = 1, no input).
 #pragma unroll
             for (int i = 0; i < kBwdSteps; ++i) {
                 const float s = dt[i] + bias;
-                dt[i] = p.softplus ? (kExact ? softplus_f32(s) : softplus_lg2(s)) : s;
-                sp[i] = p.softplus ? sigmoid_f32(s) : 1.0f;
+                const float dlt = p.softplus ? (kExact ? softplus_f32(s) : softplus_lg2(s)) : s;
+                dt[i] = (valid && i < ns) ? dlt : 0.0f;
                 if (kHasZ) {
                     const float zv = aux[i];
                     const float sg = sigmoid_f32(zv);
-                    const float g = dy[i];
-                    dy[i] = g * zv * sg;                              // dout * silu(z)
-                    aux[i] = g * sg * fmaf(zv, 1.0f - sg, 1.0f);      // dout * silu'(z)
+                    const float gd = dy[i];
+                    dy[i] = gd * zv * sg;                              // dout * silu(z)
+                    aux[i] = gd * sg * fmaf(zv, 1.0f - sg, 1.0f);      // dout * silu'(z)
                 }
             }
-            float y[kBwdSteps], ddt[kBwdSteps], dlb[kBwdSteps];
+            // Sums over the 16 entries, kept as pairs: y (the forward's readout),
+            // the Delta adjoint and sum_n lambda B (phi B for the zero-order hold).
+            float2 y2[kBwdSteps], dd2[kBwdSteps], db2[kBwdSteps];
 #pragma unroll
-            for (int i = 0; i < kBwdSteps; ++i) y[i] = ddt[i] = dlb[i] = 0.0f;
+            for (int i = 0; i < kBwdSteps; ++i)
+                y2[i] = dd2[i] = db2[i] = make_float2(0.0f, 0.0f);
 
-            // One state quarter per pass; the per-entry arrays (a2, lam, dA_acc)
-            // and the checkpoint rotate by one quarter after each pass, so the
-            // loop body indexes them statically and is emitted once.
+            // One state quarter per pass (the loop body is emitted once).
 #pragma unroll 1
             for (int q = 0; q < kNPad / 4; ++q) {
                 const int n0 = 4 * q;
                 // The four entries run as two fp32x2 pairs (packed FMA/FMUL,
                 // rounding identical to the scalar forms).
-                const float2 a2p[2] = {make_float2(a2[0], a2[1]), make_float2(a2[2], a2[3])};
+                const float4 a4 = ent[kEntA2][q][lane];
+                const float2 a2p[2] = {make_float2(a4.x, a4.y), make_float2(a4.z, a4.w)};
+                const float2 a2l[2] = {__fmul2_rn(a2p[0], make_float2(kLn2, kLn2)),
+                                       __fmul2_rn(a2p[1], make_float2(kLn2, kLn2))};
                 float2 iv[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
                 if (kZoh) {
-                    const float4 v = inva4[q][lane];
+                    const float4 v = ent[kEntInvA][q][lane];
                     iv[0] = make_float2(v.x, v.y);
                     iv[1] = make_float2(v.z, v.w);
                 }
@@ -457,127 +446,144 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
                     return make_float2(fabsf(x2.x) < kZohSmall ? ser.x : big.x,
                                        fabsf(x2.y) < kZohSmall ? ser.y : big.y);
                 };
-                const float2 a2l[2] = {__fmul2_rn(a2p[0], make_float2(kLn2, kLn2)),
-                                       __fmul2_rn(a2p[1], make_float2(kLn2, kLn2))};
-                // forward: the block's 8 states of entries n0..n0+3
-                float2 hq[kBwdSteps][2];
-                float2 h2[2] = {make_float2(ckv[0].x, ckv[0].y), make_float2(ckv[0].z, ckv[0].w)};
+                float4 c4 = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                if (staged) {
+                    if (valid) {
+                        const uint4 r = S.ck[lane][q];
+                        c4 = make_float4(__uint_as_float(r.x), __uint_as_float(r.y),
+                                         __uint_as_float(r.z), __uint_as_float(r.w));
+                    }
+                } else if (valid) {
+                    c4 = __ldcg(ck4 + q);
+                }
+                // forward: the block's 8 states of entries n0..n0+3, and Abar
+                // (kept for the way back)
+                float2 hq[kBwdSteps][2], abq[kBwdSteps][2];
+                float2 h2[2] = {make_float2(c4.x, c4.y), make_float2(c4.z, c4.w)};
 #pragma unroll
                 for (int t = 0; t < kBwdSteps; ++t) {
-                    if (t < ns) {
-                        const float4 Bq = *reinterpret_cast<const float4*>(&bcf[t][n0]);
-                        const float4 Cq = *reinterpret_cast<const float4*>(&bcf[t][16 + n0]);
-                        const float2 bq[2] = {make_float2(Bq.x, Bq.y), make_float2(Bq.z, Bq.w)};
-                        const float2 cq[2] = {make_float2(Cq.x, Cq.y), make_float2(Cq.z, Cq.w)};
-                        const float du = dt[t] * uu[t];
-                        const float2 dt2 = make_float2(dt[t], dt[t]), du2 = make_float2(du, du);
-                        const float rdt = kZoh ? __fdividef(1.0f, dt[t]) : 0.0f;
-                        float2 y2 = make_float2(0.0f, 0.0f);
+                    const float4 Bq = *reinterpret_cast<const float4*>(&bcf[t][n0]);
+                    const float4 Cq = *reinterpret_cast<const float4*>(&bcf[t][16 + n0]);
+                    const float2 bq[2] = {make_float2(Bq.x, Bq.y), make_float2(Bq.z, Bq.w)};
+                    const float2 cq[2] = {make_float2(Cq.x, Cq.y), make_float2(Cq.z, Cq.w)};
+                    const float du = dt[t] * uu[t];
+                    const float2 dt2 = make_float2(dt[t], dt[t]), du2 = make_float2(du, du);
+                    const float rdt = kZoh ? __fdividef(1.0f, dt[t]) : 0.0f;
 #pragma unroll
-                        for (int pr = 0; pr < 2; ++pr) {
-                            const float2 x2 = __fmul2_rn(dt2, a2p[pr]);
-                            const float2 ab = make_float2(bwd_exp2<kExact>(x2.x), bwd_exp2<kExact>(x2.y));
-                            float2 in = __fmul2_rn(du2, bq[pr]);
-                            if (kZoh) in = __fmul2_rn(in, zoh_phi2(x2, ab, rdt, pr));
-                            h2[pr] = __ffma2_rn(ab, h2[pr], in);
-                            hq[t][pr] = h2[pr];
-                            y2 = __ffma2_rn(cq[pr], h2[pr], y2);
-                        }
-                        y[t] += y2.x + y2.y;
+                    for (int pr = 0; pr < 2; ++pr) {
+                        const float2 x2 = __fmul2_rn(dt2, a2p[pr]);
+                        const float2 ab = bwd_exp2x2<kExact>(x2);
+                        float2 in = __fmul2_rn(du2, bq[pr]);
+                        if (kZoh) in = __fmul2_rn(in, zoh_phi2(x2, ab, rdt, pr));
+                        h2[pr] = __ffma2_rn(ab, h2[pr], in);
+                        hq[t][pr] = h2[pr];
+                        abq[t][pr] = ab;
+                        y2[t] = __ffma2_rn(cq[pr], h2[pr], y2[t]);
                     }
                 }
                 // reverse: the adjoint of entries n0..n0+3 over the block
-                float2 l2[2] = {make_float2(lam[0], lam[1]), make_float2(lam[2], lam[3])};
-                float2 dA2[2] = {make_float2(dA_acc[0], dA_acc[1]), make_float2(dA_acc[2], dA_acc[3])};
+                const float4 l4 = ent[kEntLam][q][lane];
+                const float4 g4 = ent[kEntDA][q][lane];
+                float2 l2[2] = {make_float2(l4.x, l4.y), make_float2(l4.z, l4.w)};
+                float2 dA2[2] = {make_float2(g4.x, g4.y), make_float2(g4.z, g4.w)};
 #pragma unroll
                 for (int t = kBwdSteps - 1; t >= 0; --t) {
-                    if (t < ns) {
-                        const float4 Bq = *reinterpret_cast<const float4*>(&bcf[t][n0]);
-                        const float4 Cq = *reinterpret_cast<const float4*>(&bcf[t][16 + n0]);
-                        const float2 bq[2] = {make_float2(Bq.x, Bq.y), make_float2(Bq.z, Bq.w)};
-                        const float2 cq[2] = {make_float2(Cq.x, Cq.y), make_float2(Cq.z, Cq.w)};
-                        const float du = dt[t] * uu[t];
-                        const float2 dt2 = make_float2(dt[t], dt[t]), du2 = make_float2(du, du);
-                        const float2 ndu2 = make_float2(-du, -du), dy2 = make_float2(dy[t], dy[t]);
-                        const float2 uu2 = make_float2(uu[t], uu[t]);
-                        const float rdt = kZoh ? __fdividef(1.0f, dt[t]) : 0.0f;
-                        float red[8];
-                        float2 s_dt2 = make_float2(0.0f, 0.0f), s_b2 = make_float2(0.0f, 0.0f);
+                    const float4 Bq = *reinterpret_cast<const float4*>(&bcf[t][n0]);
+                    const float4 Cq = *reinterpret_cast<const float4*>(&bcf[t][16 + n0]);
+                    const float2 bq[2] = {make_float2(Bq.x, Bq.y), make_float2(Bq.z, Bq.w)};
+                    const float2 cq[2] = {make_float2(Cq.x, Cq.y), make_float2(Cq.z, Cq.w)};
+                    const float du = dt[t] * uu[t];
+                    const float2 dt2 = make_float2(dt[t], dt[t]), du2 = make_float2(du, du);
+                    const float2 ndu2 = make_float2(-du, -du), dy2 = make_float2(dy[t], dy[t]);
+                    const float2 uu2 = make_float2(uu[t], uu[t]);
+                    const float rdt = kZoh ? __fdividef(1.0f, dt[t]) : 0.0f;
+                    float2 rb[2], rc[2];
 #pragma unroll
-                        for (int pr = 0; pr < 2; ++pr) {
-                            l2[pr] = __ffma2_rn(cq[pr], dy2, l2[pr]);                    // lambda_t
+                    for (int pr = 0; pr < 2; ++pr) {
+                        l2[pr] = __ffma2_rn(cq[pr], dy2, l2[pr]);                    // lambda_t
+                        const float2 ab = abq[t][pr];
+                        rc[pr] = __fmul2_rn(dy2, hq[t][pr]);                          // dC
+                        if (!kZoh) {
+                            const float2 abh = __ffma2_rn(ndu2, bq[pr], hq[t][pr]);  // Abar_t h_t-1
+                            rb[pr] = __fmul2_rn(l2[pr], du2);                         // dB
+                            dd2[t] = __ffma2_rn(l2[pr], __ffma2_rn(a2l[pr], abh, __fmul2_rn(bq[pr], uu2)), dd2[t]);
+                            db2[t] = __ffma2_rn(l2[pr], bq[pr], db2[t]);
+                            dA2[pr] = __ffma2_rn(__fmul2_rn(l2[pr], dt2), abh, dA2[pr]);
+                        } else {
                             const float2 x2 = __fmul2_rn(dt2, a2p[pr]);
-                            const float2 ab = make_float2(bwd_exp2<kExact>(x2.x), bwd_exp2<kExact>(x2.y));
-                            const float2 rc = __fmul2_rn(dy2, hq[t][pr]);                 // dC
-                            if (!kZoh) {
-                                const float2 abh = __ffma2_rn(ndu2, bq[pr], hq[t][pr]);  // Abar_t h_t-1
-                                const float2 rb = __fmul2_rn(l2[pr], du2);                // dB
-                                red[2 * pr] = rb.x;
-                                red[2 * pr + 1] = rb.y;
-                                s_dt2 = __ffma2_rn(l2[pr], __ffma2_rn(a2l[pr], abh, __fmul2_rn(bq[pr], uu2)), s_dt2);
-                                s_b2 = __ffma2_rn(l2[pr], bq[pr], s_b2);
-                                dA2[pr] = __ffma2_rn(__fmul2_rn(l2[pr], dt2), abh, dA2[pr]);
-                            } else {
-                                const float2 phi = zoh_phi2(x2, ab, rdt, pr);
-                                const float2 bu = __fmul2_rn(bq[pr], uu2);                // B u
-                                const float2 in = __fmul2_rn(__fmul2_rn(du2, bq[pr]), phi);
-                                const float2 abh = __fadd2_rn(hq[t][pr], make_float2(-in.x, -in.y));
-                                const float2 rb = __fmul2_rn(l2[pr], __fmul2_rn(du2, phi));  // dB
-                                red[2 * pr] = rb.x;
-                                red[2 * pr + 1] = rb.y;
-                                s_dt2 = __ffma2_rn(l2[pr], __ffma2_rn(a2l[pr], abh, __fmul2_rn(ab, bu)), s_dt2);
-                                s_b2 = __ffma2_rn(l2[pr], __fmul2_rn(phi, bq[pr]), s_b2);
-                                // dg/dA: Delta^2 times its series near 0, else Delta (Abar - phi) / A
-                                const float2 ser = __fmul2_rn(__fmul2_rn(dt2, dt2), zoh_dgda_series2(x2));
-                                const float2 big = __fmul2_rn(dt2, __fmul2_rn(__fadd2_rn(ab, make_float2(-phi.x, -phi.y)), iv[pr]));
-                                const float2 dgda = make_float2(fabsf(x2.x) < kDgdaSmall ? ser.x : big.x,
-                                                                fabsf(x2.y) < kDgdaSmall ? ser.y : big.y);
-                                dA2[pr] = __ffma2_rn(l2[pr], __ffma2_rn(dt2, abh, __fmul2_rn(dgda, bu)), dA2[pr]);
-                            }
-                            red[4 + 2 * pr] = rc.x;
-                            red[5 + 2 * pr] = rc.y;
-                            l2[pr] = __fmul2_rn(l2[pr], ab);                              // to h_t-1
+                            const float2 phi = zoh_phi2(x2, ab, rdt, pr);
+                            const float2 bu = __fmul2_rn(bq[pr], uu2);                // B u
+                            const float2 in = __fmul2_rn(__fmul2_rn(du2, bq[pr]), phi);
+                            const float2 abh = __fadd2_rn(hq[t][pr], make_float2(-in.x, -in.y));
+                            rb[pr] = __fmul2_rn(l2[pr], __fmul2_rn(du2, phi));        // dB
+                            dd2[t] = __ffma2_rn(l2[pr], __ffma2_rn(a2l[pr], abh, __fmul2_rn(ab, bu)), dd2[t]);
+                            db2[t] = __ffma2_rn(l2[pr], __fmul2_rn(phi, bq[pr]), db2[t]);
+                            // dg/dA: Delta^2 times its series near 0, else Delta (Abar - phi) / A
+                            const float2 ser = __fmul2_rn(__fmul2_rn(dt2, dt2), zoh_dgda_series2(x2));
+                            const float2 big = __fmul2_rn(dt2, __fmul2_rn(__fadd2_rn(ab, make_float2(-phi.x, -phi.y)), iv[pr]));
+                            const float2 dgda = make_float2(fabsf(x2.x) < kDgdaSmall ? ser.x : big.x,
+                                                            fabsf(x2.y) < kDgdaSmall ? ser.y : big.y);
+                            dA2[pr] = __ffma2_rn(l2[pr], __ffma2_rn(dt2, abh, __fmul2_rn(dgda, bu)), dA2[pr]);
                         }
-                        ddt[t] += s_dt2.x + s_dt2.y;
-                        dlb[t] += s_b2.x + s_b2.y;
-                        const float tot = warp_reduce8(red, lane);
-                        const int idx = lane >> 2;                              // 0..7
-                        const int n = n0 + (idx & 3);
-                        if ((lane & 3) == 0 && n < p.dstate) {
-                            float* dst = (idx < 4 ? p.dB : p.dC) + (b * p.dstate + n) * p.seqlen + t0 + t;
-                            atomicAdd(dst, tot);
-                        }
+                        l2[pr] = __fmul2_rn(l2[pr], ab);                              // to h_t-1
                     }
+                    *reinterpret_cast<float4*>(&rbuf[lane][4 * t]) =
+                        make_float4(rb[0].x, rb[0].y, rb[1].x, rb[1].y);
+                    *reinterpret_cast<float4*>(&rbuf[lane][4 * kBwdSteps + 4 * t]) =
+                        make_float4(rc[0].x, rc[0].y, rc[1].x, rc[1].y);
                 }
-                dA_acc[0] = dA2[0].x;
-                dA_acc[1] = dA2[0].y;
-                dA_acc[2] = dA2[1].x;
-                dA_acc[3] = dA2[1].y;
-                const float l4[4] = {l2[0].x, l2[0].y, l2[1].x, l2[1].y};
+                ent[kEntLam][q][lane] = make_float4(l2[0].x, l2[0].y, l2[1].x, l2[1].y);
+                ent[kEntDA][q][lane] = make_float4(dA2[0].x, dA2[0].y, dA2[1].x, dA2[1].y);
+                // dB and dC sum over the warp's 32 channels: each lane adds one
+                // pair of the 64 partials over the 32 rows and adds the pair to
+                // global memory.
+                __syncwarp();
+                float2 acc[4];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) lam[i] = l4[i];
-                rotate_quarter(a2);
-                rotate_quarter(lam);
-                rotate_quarter(dA_acc);
-                const float4 c0 = ckv[0];
-                ckv[0] = ckv[1];
-                ckv[1] = ckv[2];
-                ckv[2] = ckv[3];
-                ckv[3] = c0;
+                for (int i = 0; i < 4; ++i) acc[i] = make_float2(0.0f, 0.0f);
+#pragma unroll
+                for (int src = 0; src < 32; ++src)
+                    acc[src & 3] = __fadd2_rn(acc[src & 3],
+                                              *reinterpret_cast<const float2*>(&rbuf[src][2 * lane]));
+                const float2 tot = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+                __syncwarp();
+                const int n = n0 + red_n;
+                if (red_t < ns && n < p.dstate) {
+                    float* dst = (red_kind ? p.dC : p.dB) + (b * p.dstate + n) * p.seqlen + t0 + red_t;
+                    atomicAdd(dst, tot.x);
+                    if (n + 1 < p.dstate) atomicAdd(dst + p.seqlen, tot.y);
+                }
             }
-            // per-step outputs of the block
+            // per-step outputs of the block; the softplus derivative
+            // sigmoid(delta + bias) from delta read again
+            float sp[kBwdSteps];
+            if (p.softplus) {
+                if (valid && staged) {
+                    unpack_rows<kIoVecs>(S.io[1][lane], sp);
+                } else if (valid) {
+                    load_block(drow, t0, ns, vec, sp);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < kBwdSteps; ++i) sp[i] = 0.0f;
+                }
+#pragma unroll
+                for (int i = 0; i < kBwdSteps; ++i) sp[i] = sigmoid_f32(sp[i] + bias);
+            } else {
+#pragma unroll
+                for (int i = 0; i < kBwdSteps; ++i) sp[i] = 1.0f;
+            }
             float o_du[kBwdSteps], o_dd[kBwdSteps], o_dz[kBwdSteps];
 #pragma unroll
             for (int t = 0; t < kBwdSteps; ++t) {
                 const bool in = t < ns;
-                o_du[t] = fmaf(Dd, dy[t], dt[t] * dlb[t]);
-                const float ds = ddt[t] * sp[t];
+                o_du[t] = fmaf(Dd, dy[t], dt[t] * (db2[t].x + db2[t].y));
+                const float ds = (dd2[t].x + dd2[t].y) * sp[t];
                 o_dd[t] = ds;
                 if (in) {
                     dbias_acc += ds;
                     dD_acc = fmaf(dy[t], uu[t], dD_acc);
                 }
-                o_dz[t] = kHasZ ? aux[t] * fmaf(Dd, uu[t], y[t]) : 0.0f;
+                o_dz[t] = kHasZ ? aux[t] * fmaf(Dd, uu[t], y2[t].x + y2[t].y) : 0.0f;
             }
             __syncwarp();
             if (valid) {
@@ -589,6 +595,14 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
         }
 
         // hand lambda to the earlier segment, or it is the start state's gradient
+        float lam[kNPad], dA_acc[kNPad];
+#pragma unroll
+        for (int q = 0; q < kNPad / 4; ++q) {
+            const float4 l4 = ent[kEntLam][q][lane];
+            const float4 g4 = ent[kEntDA][q][lane];
+            lam[4 * q] = l4.x; lam[4 * q + 1] = l4.y; lam[4 * q + 2] = l4.z; lam[4 * q + 3] = l4.w;
+            dA_acc[4 * q] = g4.x; dA_acc[4 * q + 1] = g4.y; dA_acc[4 * q + 2] = g4.z; dA_acc[4 * q + 3] = g4.w;
+        }
         if (k > 0) {
             float2 c2[kNPad / 2];
 #pragma unroll

@@ -149,7 +149,8 @@ def test_backward_rejects_bad_arguments(lib):
     assert call(None) == -1
     assert call(_dims(dstate=17)) == -2
     zoh = _dims(); zoh.flags = ops.MAMBA_FLAG_ZOH
-    assert call(zoh) == -2                             # zero-order hold: forward only
+    assert call(zoh, u=None) == -1 and call(zoh, A=None) == -1   # the zero-order hold is
+    assert call(zoh, u=ctypes.c_void_p(0x10001)) == -3           # checked like Euler
     assert call(d, u=None) == -1 and call(d, dout=None) == -1 and call(d, du=None) == -1
     assert call(d, A=None) == -1 and call(d, dA=None) == -1
     assert call(d, u=ctypes.c_void_p(0x10001)) == -3
