@@ -43,7 +43,7 @@ import torch  # noqa: E402
 METRIC = ("selective-scan Gelem/s (B·D·L) and % of roofline; "
           "decode-step µs at batch 128")
 SCAN_WORKLOAD = "mamba_2p8b_layer"
-SCAN_VARIANTS = ("euler", "zoh", "start_state")
+SCAN_VARIANTS = ("euler", "zoh", "start_state", "bld")
 PROFILES = ROOT / "profiles"
 HBM_FALLBACK_GBS = 6650.0
 HBM_NOMINAL_GBS = 8000.0
@@ -196,6 +196,12 @@ class Workload:
                                        self.dcfg.dstate, decode_layers, self.dcfg.steps)
         c = self.cfg
         self.x = I.make_scan_inputs(c, "cuda", seed=rank_seed(rank))
+        self.flags = 0
+        if scan_variant == "bld":   # the same inputs in the (batch, seqlen, dim) layout
+            for k in ("u", "delta", "z"):
+                if self.x[k] is not None:
+                    self.x[k] = self.x[k].transpose(1, 2).contiguous()
+            self.flags = ops.MAMBA_FLAG_LAYOUT_BLD
         self.out = torch.empty_like(self.x["u"])
         self.last = torch.empty((c.batch, c.dim, c.dstate), dtype=torch.float32, device="cuda")
         self.h0 = None
@@ -203,10 +209,12 @@ class Workload:
             g = torch.Generator(device="cuda")
             g.manual_seed(rank_seed(rank) + 7)
             self.h0 = torch.randn((c.batch, c.dim, c.dstate), generator=g, device="cuda")
-        ws = ops.scan_workspace_bytes(c.batch, c.dim, c.dstate, c.seqlen, c.io_dtype, c.bc_dtype)
+        ws = ops.scan_workspace_bytes(c.batch, c.dim, c.dstate, c.seqlen, c.io_dtype, c.bc_dtype,
+                                      flags=self.flags)
         self.ws = torch.empty(ws, dtype=torch.uint8, device="cuda") if ws else None
         self.plan = ops.scan_plan(c.batch, c.dim, c.dstate, c.seqlen, c.io_dtype, c.bc_dtype,
-                                  sm_count=torch.cuda.get_device_properties(0).multi_processor_count)
+                                  sm_count=torch.cuda.get_device_properties(0).multi_processor_count,
+                                  flags=self.flags)
         d = self.dcfg
         nl = 0 if only == "scan" else d.layers
         self.layers = [I.make_decode_layer(d, "cuda", seed=2000 + 100 * rank + i) for i in range(nl)]
@@ -215,7 +223,7 @@ class Workload:
         self.graph = None
 
     def scan_kwargs(self) -> dict:
-        return {"zoh": self.variant == "zoh", "initial_state": self.h0}
+        return {"zoh": self.variant == "zoh", "initial_state": self.h0, "flags": self.flags}
 
     def scan(self):
         if self.only == "decode":
@@ -272,7 +280,7 @@ def run_e2e(w: Workload, steps: int, warmup: int, rows: int = 0) -> dict:
     out_h = torch.empty(w.out.shape, dtype=w.out.dtype, pin_memory=True)
     last_h = torch.empty(w.last.shape, dtype=w.last.dtype, pin_memory=True)
     zoh = w.variant == "zoh"
-    flags = ops.MAMBA_FLAG_ZOH if zoh else 0
+    flags = (ops.MAMBA_FLAG_ZOH if zoh else 0) | w.flags
     need = ops.scan_host_workspace_bytes(c.batch, c.dim, c.dstate, c.seqlen, c.io_dtype,
                                          c.bc_dtype, rows=rows, flags=flags)
     ws = torch.empty(max(need, 1), dtype=torch.uint8, device="cuda")
@@ -284,7 +292,7 @@ def run_e2e(w: Workload, steps: int, warmup: int, rows: int = 0) -> dict:
         ops.selective_scan_fwd_host(host["u"], host["delta"], host["A"], host["B"], host["C"],
                                     D=host["D"], z=host["z"], delta_bias=host["delta_bias"],
                                     softplus=True, out=out_h, last_state=last_h, rows=rows,
-                                    workspace=ws, initial_state=h0_h, zoh=zoh)
+                                    workspace=ws, initial_state=h0_h, zoh=zoh, flags=w.flags)
 
     for _ in range(warmup):
         step()
@@ -678,7 +686,8 @@ def bench_ours(args, rank, world, local):
                        "copies in and out -> out/last_state in pinned host memory"}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.only != "decode":
+    if (rank == 0 and world == 1 and not args.no_cpu_baseline and args.only != "decode"
+            and w.variant != "bld"):   # the oracle's blocks read (batch, dim, seqlen) rows
         cpu = cpu_baseline(w, args.cpu_seconds)
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.only != "scan":
         decode["cpu_baseline"] = decode_cpu_baseline(w, args.cpu_seconds / 2)

@@ -107,6 +107,16 @@ typedef enum {
  * different layers; then results are identical with and without the flag.
  * Paths other than the streaming one ignore it. */
 #define MAMBA_FLAG_PDL 0x10
+/* Scan forward only (mamba_selective_scan_fwd, _with_state, _noalloc and the
+ * host-buffer call): u, delta, z and out are (batch, seqlen, dim), dim fastest,
+ * the activation layout of the sample module in "超越注意力：探索Mamba与状态空间
+ * 模型", section 代码实现概览; B and C stay (batch, dstate, seqlen) and the
+ * states (batch, dim, dstate).  Tiles of (steps x 32 channels) are staged by
+ * TMA (dim * element size a multiple of 16 bytes, 16-byte aligned pointers;
+ * otherwise plain loads) and transposed on chip; outputs are stored one step
+ * at a time.  Such calls always run in mode 0: MAMBA_FLAG_PARALLEL_CHUNKS with
+ * it returns MAMBA_ERR_UNSUPPORTED, and so does the backward. */
+#define MAMBA_FLAG_LAYOUT_BLD 0x20
 
 #define MAMBA_MAX_DSTATE 16
 
@@ -200,7 +210,8 @@ MAMBA_API size_t mamba_selective_scan_workspace_bytes(const mamba_dims_t *dims);
 
 /*
  * Selective scan forward.
- *   u, delta, z, out   (batch, dim, seqlen), io_dtype; z may be NULL (no gate)
+ *   u, delta, z, out   (batch, dim, seqlen), io_dtype; z may be NULL (no gate);
+ *                      (batch, seqlen, dim) with MAMBA_FLAG_LAYOUT_BLD
  *   A                  (dim, dstate) fp32
  *   B, C               (batch, dstate, seqlen), bc_dtype, shared by all channels
  *   D, delta_bias      (dim,) fp32; may be NULL (treated as 0)
@@ -356,7 +367,9 @@ MAMBA_API mamba_status_t mamba_selective_state_update(float *state, const void *
  * Gradients of a scalar loss, given dout = dLoss/dout (and optionally
  * dlast_state = dLoss/dlast_state), with respect to every input of
  * mamba_selective_scan_fwd_with_state, with the Euler input term or, with
- * MAMBA_FLAG_ZOH in dims->flags, the zero-order-hold one.  As in the pages'
+ * MAMBA_FLAG_ZOH in dims->flags, the zero-order-hold one (inputs in the
+ * (batch, dim, seqlen) layout: MAMBA_FLAG_LAYOUT_BLD returns
+ * MAMBA_ERR_UNSUPPORTED).  As in the pages'
  * description of the hardware-aware scan ("Mamba 与状态空间模型", section
  * 在芯片上扫过去), the per-step states are not stored by the forward: a
  * checkpoint pass keeps the state every 8 steps in the workspace, and the

@@ -93,13 +93,13 @@ cudaError_t ensure_smem_attr(Kernel kernel, int bytes, bool* done_per_device, in
     return e;
 }
 
-template <typename IoT, int kCpl, bool kHasZ, bool kSoftplus, bool kZoh>
+template <typename IoT, int kCpl, bool kHasZ, bool kSoftplus, bool kZoh, bool kBld>
 cudaError_t launch_scan(const ScanParams& prm, const CUtensorMap* maps, int64_t want_warps,
                         int dev, int sms, cudaStream_t stream) {
     using Lay = ScanLayout<kCpl>;
     static bool attr_done[kMaxDevices] = {false};
     static int resident[kMaxDevices] = {0};
-    auto kernel = selective_scan_fwd_kernel<IoT, kCpl, kHasZ, kSoftplus, kZoh>;
+    auto kernel = selective_scan_fwd_kernel<IoT, kCpl, kHasZ, kSoftplus, kZoh, kBld>;
     cudaError_t e = ensure_smem_attr(kernel, Lay::kCtaSmem, attr_done, dev);
     if (e != cudaSuccess) return e;
     int per_sm = (dev >= 0 && dev < kMaxDevices) ? resident[dev] : 0;
@@ -118,23 +118,27 @@ cudaError_t launch_scan(const ScanParams& prm, const CUtensorMap* maps, int64_t 
     return cudaGetLastError();
 }
 
-template <typename IoT, int kCpl, bool kZoh>
+template <typename IoT, int kCpl, bool kZoh, bool kBld>
 cudaError_t dispatch_scan_cpl(const ScanParams& prm, const CUtensorMap* maps, bool has_z, bool sp,
                               int64_t want_warps, int dev, int sms, cudaStream_t stream) {
     if (has_z)
-        return sp ? launch_scan<IoT, kCpl, true, true, kZoh>(prm, maps, want_warps, dev, sms, stream)
-                  : launch_scan<IoT, kCpl, true, false, kZoh>(prm, maps, want_warps, dev, sms, stream);
-    return sp ? launch_scan<IoT, kCpl, false, true, kZoh>(prm, maps, want_warps, dev, sms, stream)
-              : launch_scan<IoT, kCpl, false, false, kZoh>(prm, maps, want_warps, dev, sms, stream);
+        return sp ? launch_scan<IoT, kCpl, true, true, kZoh, kBld>(prm, maps, want_warps, dev, sms, stream)
+                  : launch_scan<IoT, kCpl, true, false, kZoh, kBld>(prm, maps, want_warps, dev, sms, stream);
+    return sp ? launch_scan<IoT, kCpl, false, true, kZoh, kBld>(prm, maps, want_warps, dev, sms, stream)
+              : launch_scan<IoT, kCpl, false, false, kZoh, kBld>(prm, maps, want_warps, dev, sms, stream);
 }
 
+// Kernel instance for (channels per lane, zero-order hold, activation layout).
 template <typename IoT>
 cudaError_t dispatch_scan(const ScanParams& prm, const CUtensorMap* maps, int cpl, bool has_z,
                           bool sp, bool zoh, int64_t want_warps, int dev, int sms,
                           cudaStream_t stream) {
     if (cpl != 1) return cudaErrorInvalidValue;
-    return zoh ? dispatch_scan_cpl<IoT, 1, true>(prm, maps, has_z, sp, want_warps, dev, sms, stream)
-               : dispatch_scan_cpl<IoT, 1, false>(prm, maps, has_z, sp, want_warps, dev, sms, stream);
+    if (prm.bld)
+        return zoh ? dispatch_scan_cpl<IoT, 1, true, true>(prm, maps, has_z, sp, want_warps, dev, sms, stream)
+                   : dispatch_scan_cpl<IoT, 1, false, true>(prm, maps, has_z, sp, want_warps, dev, sms, stream);
+    return zoh ? dispatch_scan_cpl<IoT, 1, true, false>(prm, maps, has_z, sp, want_warps, dev, sms, stream)
+               : dispatch_scan_cpl<IoT, 1, false, false>(prm, maps, has_z, sp, want_warps, dev, sms, stream);
 }
 
 // Correction pass of the parallel mode: a persistent grid of warps that pull
@@ -298,10 +302,15 @@ ScanWorkspace scan_workspace_layout(const mamba_dims_t* dims, int64_t groups, in
 //    and 512 steps long.
 //  - num_chunks >= 1 forces K; MAMBA_FLAG_PARALLEL_CHUNKS forces the parallel
 //    mode for a forced K.
+//  - Activations in the (batch, seqlen, dim) layout always run chained (the
+//    correction pass reads rows along time).
 mamba_status_t plan_scan(const mamba_dims_t* dims, int sm_count, mamba_scan_plan_t* plan) {
     mamba_status_t st = check_dims(dims, true);
     if (st != MAMBA_OK) return st;
     if (plan == nullptr || sm_count <= 0) return MAMBA_ERR_INVALID_ARG;
+    const bool bld = (dims->flags & MAMBA_FLAG_LAYOUT_BLD) != 0;
+    if (bld && dims->num_chunks >= 1 && (dims->flags & MAMBA_FLAG_PARALLEL_CHUNKS))
+        return MAMBA_ERR_UNSUPPORTED;
     *plan = mamba_scan_plan_t{};
     const int io_es = dtype_bytes(dims->io_dtype);
     const int bc_es = dtype_bytes(dims->bc_dtype);
@@ -323,7 +332,8 @@ mamba_status_t plan_scan(const mamba_dims_t* dims, int sm_count, mamba_scan_plan
     plan->groups = groups;
     plan->warps_per_cta = kScanWarps;
     plan->channels_per_lane = cpl;
-    plan->tma_capable = (L > 0 && (L * io_es) % 16 == 0 && (L * bc_es) % 16 == 0) ? 1 : 0;
+    const int64_t act_row = bld ? dims->dim : L;   // elements of an activation row
+    plan->tma_capable = (L > 0 && (act_row * io_es) % 16 == 0 && (L * bc_es) % 16 == 0) ? 1 : 0;
 
     int64_t K = 1;
     int mode = 0;
@@ -331,7 +341,7 @@ mamba_status_t plan_scan(const mamba_dims_t* dims, int sm_count, mamba_scan_plan
         K = dims->num_chunks;
         mode = (dims->flags & MAMBA_FLAG_PARALLEL_CHUNKS) ? 1 : 0;
     } else if (groups > 0 && L > 0) {
-        if (4 * groups >= W) {
+        if (4 * groups >= W || bld) {
             const int64_t want = (8 * W + groups - 1) / groups;
             K = std::max<int64_t>(1, std::min<int64_t>(want, L / 256));
         } else {
@@ -423,6 +433,8 @@ mamba_status_t scan_fwd_internal(const void* u, const void* delta, const float* 
                                  int64_t ckpt_tiles) {
     mamba_status_t st = check_dims(dims, true);
     if (st != MAMBA_OK) return st;
+    const bool bld = (dims->flags & MAMBA_FLAG_LAYOUT_BLD) != 0;
+    if (bld && ckpt != nullptr) return MAMBA_ERR_UNSUPPORTED;
     // Empty problems first: tensors without elements may have null pointers.
     const int64_t chains = dims->batch * dims->dim;
     if (chains == 0) return MAMBA_OK;
@@ -491,7 +503,9 @@ mamba_status_t scan_fwd_internal(const void* u, const void* delta, const float* 
     prm.dstate = (int)dims->dstate;
     prm.nseg = plan.nchunks;
     prm.bc_bf16 = dims->bc_dtype == MAMBA_BF16;
-    prm.vec_out = out != nullptr && ((dims->seqlen * io_es) % 16 == 0) && aligned(out, 16);
+    prm.bld = bld ? 1 : 0;
+    prm.out_step = bld ? dims->dim : 1;
+    prm.vec_out = !bld && out != nullptr && ((dims->seqlen * io_es) % 16 == 0) && aligned(out, 16);
     // A predecessor segment legitimately takes well under 64 us per step even
     // on a crowded GPU; wait that long (at least ~1 s) before reporting a stall.
     prm.withhold_handoff = (dims->flags & MAMBA_FLAG_TEST_WITHHOLD_HANDOFF) ? 1 : 0;
@@ -520,12 +534,13 @@ mamba_status_t scan_fwd_internal(const void* u, const void* delta, const float* 
         const uint64_t Dm = (uint64_t)dims->dim, Bt = (uint64_t)dims->batch;
         const uint64_t N = (uint64_t)dims->dstate;
         const uint32_t rows = 32u * (uint32_t)plan.channels_per_lane;
-        bool ok = encode_map_3d(&maps[0], u, io_es, L, Dm, Bt, T, rows,
-                                CU_TENSOR_MAP_SWIZZLE_32B) &&
-                  encode_map_3d(&maps[1], delta, io_es, L, Dm, Bt, T, rows,
-                                CU_TENSOR_MAP_SWIZZLE_32B) &&
-                  encode_map_3d(&maps[2], z ? z : u, io_es, L, Dm, Bt, T, rows,
-                                CU_TENSOR_MAP_SWIZZLE_32B) &&
+        // (rows x T) tiles of (batch, dim, seqlen) rows with 32-byte swizzle, or
+        // dense (T x rows) tiles of (batch, seqlen, dim) that the kernel transposes
+        auto act = [&](CUtensorMap* m, const void* base) {
+            return bld ? encode_map_3d(m, base, io_es, Dm, L, Bt, rows, T, CU_TENSOR_MAP_SWIZZLE_NONE)
+                       : encode_map_3d(m, base, io_es, L, Dm, Bt, T, rows, CU_TENSOR_MAP_SWIZZLE_32B);
+        };
+        bool ok = act(&maps[0], u) && act(&maps[1], delta) && act(&maps[2], z ? z : u) &&
                   encode_map_3d(&maps[3], B, bc_es, L, N, Bt, T, (uint32_t)N,
                                 CU_TENSOR_MAP_SWIZZLE_NONE) &&
                   encode_map_3d(&maps[4], C, bc_es, L, N, Bt, T, (uint32_t)N,
@@ -1355,6 +1370,7 @@ MAMBA_API mamba_status_t mamba_selective_scan_bwd(
     float* dinitial_state, const mamba_dims_t* dims, cudaStream_t stream) {
     mamba_status_t st = check_dims(dims, true);
     if (st != MAMBA_OK) return st;
+    if (dims->flags & MAMBA_FLAG_LAYOUT_BLD) return MAMBA_ERR_UNSUPPORTED;
     const int64_t chains = dims->batch * dims->dim;
     if (chains == 0) return MAMBA_OK;
     const int64_t L = dims->seqlen, N = dims->dstate;

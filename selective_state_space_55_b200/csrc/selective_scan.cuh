@@ -45,7 +45,10 @@
 // Once a tile lands the warp converts B and C to an fp32 table
 // bcf[t][B0..15 C0..15] that every lane reads with broadcast 16-byte loads.
 // Without TMA (odd strides or MAMBA_FLAG_NO_TMA) plain loads fill the same
-// tiles.
+// tiles.  Activations in the (batch, seqlen, dim) layout arrive as (steps x
+// channels) tiles, which the warp transposes in place once they land; their
+// outputs are stored one step at a time (32 lanes write 32 consecutive
+// channels of a step).
 #pragma once
 
 #include "ssm_device.cuh"
@@ -117,6 +120,8 @@ struct ScanParams {
     const float* h0;         // (batch, dim, dstate) start state of segment 0, or null (zero)
     float* ckpt;             // backward's checkpoint pass: [chains][ckpt_tiles][16], or null
     int64_t ckpt_tiles;      // ceil(seqlen / kCkptSteps)
+    int bld;                 // u, delta, z, out are (batch, seqlen, dim) (the kBld instances)
+    int64_t out_step;        // elements between consecutive steps of one channel's output
 };
 
 
@@ -272,10 +277,11 @@ __device__ __forceinline__ void scan_step(const float* bc_row, const float (&dt)
 // state, so computing them together lets their latency overlap.  The vectors
 // stay packed and are unpacked element by element to save registers.
 template <typename IoT, int kCpl, bool kHasZ, bool kSoftplus, bool kZoh, bool kOut, bool kCkpt,
-          bool kSum>
+          bool kSum, bool kBld>
 __device__ __forceinline__ void compute_tile(const uint8_t* st, const float* bcf, int lane,
                                              int nsteps, LaneChains<kCpl>& lc,
                                              IoT* const (&out_row)[kCpl], bool vec_out,
+                                             int64_t out_step,
                                              float (&sdt)[kCpl], float (&sdt_c)[kCpl],
                                              float* const (&ck)[kCpl]) {
     using Lay = ScanLayout<kCpl>;
@@ -333,7 +339,8 @@ __device__ __forceinline__ void compute_tile(const uint8_t* st, const float* bcf
                         if (whole[c])
                             pk[c].put(j, yo);
                         else if (out_row[c] != nullptr)
-                            DType<IoT>::store(out_row[c] + base + j, yo);
+                            DType<IoT>::store(kBld ? out_row[c] + (int64_t)(base + j) * out_step
+                                                   : out_row[c] + base + j, yo);
                     }
                     if (kSum) kahan_add(sdt[c], sdt_c[c], dt[c]);
                 }
@@ -378,9 +385,54 @@ __device__ __forceinline__ void convert_bc(const uint8_t* st, float* bcf, int la
     }
 }
 
+// Activations in the (batch, seqlen, dim) layout arrive from TMA as dense
+// (steps x channels) tiles: element (t, r) at byte (t * kRows + r) * size.
+// This rearranges such a tile in place into the swizzled (channels x steps)
+// tile that compute_tile reads.  Lane (q = lane & 15, h = lane >> 4) moves the
+// channel pairs (2p, 2p + 1), p = q + 16 i, over the steps [h V, h V + V) (V =
+// one 16-byte vector of a row): it reads all of them, the warp synchronises,
+// then it writes them.  The caller synchronises the warp afterwards.
+template <typename IoT, int kCpl>
+__device__ __forceinline__ void transpose_bld_tile(uint8_t* tile, int lane) {
+    constexpr int ES = (int)sizeof(IoT);
+    constexpr int V = 16 / ES;                 // steps per lane
+    constexpr int kRows = 32 * kCpl;
+    const int h = lane >> 4;
+    uint4 row0[kCpl], row1[kCpl];
+#pragma unroll
+    for (int i = 0; i < kCpl; ++i) {
+        const int pr = (lane & 15) + 16 * i;
+        if constexpr (ES == 2) {
+            uint32_t w[V];
+#pragma unroll
+            for (int j = 0; j < V; ++j)
+                w[j] = *reinterpret_cast<const uint32_t*>(tile + ((h * V + j) * kRows + 2 * pr) * ES);
+            // channel 2p is the low half of each word, channel 2p + 1 the high half
+            row0[i] = make_uint4(__byte_perm(w[0], w[1], 0x5410), __byte_perm(w[2], w[3], 0x5410),
+                                 __byte_perm(w[4], w[5], 0x5410), __byte_perm(w[6], w[7], 0x5410));
+            row1[i] = make_uint4(__byte_perm(w[0], w[1], 0x7632), __byte_perm(w[2], w[3], 0x7632),
+                                 __byte_perm(w[4], w[5], 0x7632), __byte_perm(w[6], w[7], 0x7632));
+        } else {
+            uint2 w[V];
+#pragma unroll
+            for (int j = 0; j < V; ++j)
+                w[j] = *reinterpret_cast<const uint2*>(tile + ((h * V + j) * kRows + 2 * pr) * ES);
+            row0[i] = make_uint4(w[0].x, w[1].x, w[2].x, w[3].x);
+            row1[i] = make_uint4(w[0].y, w[1].y, w[2].y, w[3].y);
+        }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < kCpl; ++i) {
+        const int pr = (lane & 15) + 16 * i;
+        *reinterpret_cast<uint4*>(tile + swz32(2 * pr, 16u * h)) = row0[i];
+        *reinterpret_cast<uint4*>(tile + swz32(2 * pr + 1, 16u * h)) = row1[i];
+    }
+}
+
 // Fill one stage with plain loads (any stride or alignment).  Rows beyond
 // dim and steps beyond seqlen read as zero, as TMA's out-of-bounds fill does.
-template <typename IoT, int kCpl, bool kNeedZ, bool kNeedC>
+template <typename IoT, int kCpl, bool kNeedZ, bool kNeedC, bool kBld>
 __device__ __forceinline__ void portable_stage(const ScanParams& p, uint8_t* st, float* bcf,
                                                int lane, int64_t b, int64_t d0, int64_t t0) {
     using Lay = ScanLayout<kCpl>;
@@ -390,12 +442,13 @@ __device__ __forceinline__ void portable_stage(const ScanParams& p, uint8_t* st,
     const IoT* dl = static_cast<const IoT*>(p.delta);
     const IoT* zz = static_cast<const IoT*>(p.z);
     for (int idx = lane; idx < Lay::kRows * T; idx += 32) {
-        const int r = idx / T;
-        const int j = idx % T;
+        // consecutive lanes walk the layout's contiguous index
+        const int r = kBld ? idx % Lay::kRows : idx / T;
+        const int j = kBld ? idx / Lay::kRows : idx % T;
         const int64_t d = d0 + r;
         const int64_t t = t0 + j;
         const bool in = d < p.dim && t < p.seqlen;
-        const int64_t off = (b * p.dim + d) * p.seqlen + t;
+        const int64_t off = kBld ? (b * p.seqlen + t) * p.dim + d : (b * p.dim + d) * p.seqlen + t;
         const uint32_t so = swz32(r, j * ES);
         const IoT zero = IoT(0.0f);
         *reinterpret_cast<IoT*>(st + Lay::kOffU + so) = in ? u[off] : zero;
@@ -432,7 +485,7 @@ struct TmaMaps {
 // mbarrier parity across items).  Returns false if a staged tile never
 // arrived (the warp has then waited, bounded, for its copies in flight).
 template <typename IoT, int kCpl, bool kHasZ, bool kSoftplus, bool kZoh, bool kOut, bool kCkpt,
-          bool kSum>
+          bool kSum, bool kBld>
 __device__ __forceinline__ bool run_segment(const ScanParams& p, const TmaMaps& maps, uint8_t* wsm,
                                             int lane, int64_t b, int64_t d0, int64_t t_begin,
                                             int64_t t_end, LaneChains<kCpl>& lc,
@@ -459,9 +512,11 @@ __device__ __forceinline__ bool run_segment(const ScanParams& p, const TmaMaps& 
         const uint32_t bar = smem_u32(&bars[s]);
         fence_proxy_async_smem();
         mbar_arrive_expect_tx(bar, stage_tx);
-        tma_load_3d(smem_u32(st + Lay::kOffU), maps.u, t0, (int)d0, (int)b, bar);
-        tma_load_3d(smem_u32(st + Lay::kOffDelta), maps.delta, t0, (int)d0, (int)b, bar);
-        if (kNeedZ) tma_load_3d(smem_u32(st + Lay::kOffZ), maps.z, t0, (int)d0, (int)b, bar);
+        // activation maps run over (seqlen, dim, batch), or (dim, seqlen, batch)
+        const int x0 = kBld ? (int)d0 : t0, x1 = kBld ? t0 : (int)d0;
+        tma_load_3d(smem_u32(st + Lay::kOffU), maps.u, x0, x1, (int)b, bar);
+        tma_load_3d(smem_u32(st + Lay::kOffDelta), maps.delta, x0, x1, (int)b, bar);
+        if (kNeedZ) tma_load_3d(smem_u32(st + Lay::kOffZ), maps.z, x0, x1, (int)b, bar);
         tma_load_3d(smem_u32(st + Lay::kOffB), maps.B, t0, 0, (int)b, bar);
         if (kOut) tma_load_3d(smem_u32(st + Lay::kOffC), maps.C, t0, 0, (int)b, bar);
     };
@@ -490,21 +545,26 @@ __device__ __forceinline__ bool run_segment(const ScanParams& p, const TmaMaps& 
                 __syncwarp();
                 return false;
             }
+            if constexpr (kBld) {
+                transpose_bld_tile<IoT, kCpl>(st + Lay::kOffU, lane);
+                transpose_bld_tile<IoT, kCpl>(st + Lay::kOffDelta, lane);
+                if (kNeedZ) transpose_bld_tile<IoT, kCpl>(st + Lay::kOffZ, lane);
+            }
             convert_bc<kCpl, T, kOut>(st, bcf, lane, p.dstate, p.bc_bf16 != 0);
         } else {
-            portable_stage<IoT, kCpl, kNeedZ, kOut>(p, st, bcf, lane, b, d0, t0);
+            portable_stage<IoT, kCpl, kNeedZ, kOut, kBld>(p, st, bcf, lane, b, d0, t0);
         }
         __syncwarp();
         IoT* rows[kCpl];
         float* cks[kCpl];
 #pragma unroll
         for (int c = 0; c < kCpl; ++c) {
-            rows[c] = out_row[c] ? out_row[c] + (t0 - t_begin) : nullptr;
+            rows[c] = out_row[c] ? out_row[c] + (t0 - t_begin) * (kBld ? p.out_step : 1) : nullptr;
             cks[c] = (kCkpt && ckpt_row[c]) ? ckpt_row[c] + ((t0 - t_begin) / kCkptSteps) * kNPad
                                             : nullptr;
         }
-        compute_tile<IoT, kCpl, kHasZ, kSoftplus, kZoh, kOut, kCkpt, kSum>(
-            st, bcf, lane, nsteps, lc, rows, p.vec_out != 0, sdt, sdt_c, cks);
+        compute_tile<IoT, kCpl, kHasZ, kSoftplus, kZoh, kOut, kCkpt, kSum, kBld>(
+            st, bcf, lane, nsteps, lc, rows, p.vec_out != 0, p.out_step, sdt, sdt_c, cks);
         __syncwarp();
         if (p.use_tma && lane == 0 && i + kScanStages < ntiles) issue(i + kScanStages);
     }
@@ -524,7 +584,7 @@ __device__ __forceinline__ void st_release_gpu(unsigned int* p, unsigned int v) 
 
 // kZoh keeps 1 / A in 16 more registers per channel, so its instances are
 // compiled for one CTA per SM fewer.
-template <typename IoT, int kCpl, bool kHasZ, bool kSoftplus, bool kZoh>
+template <typename IoT, int kCpl, bool kHasZ, bool kSoftplus, bool kZoh, bool kBld>
 __global__ void __launch_bounds__(kScanWarps * 32, ScanLayout<kCpl>::kMinBlocks - (kZoh ? 1 : 0))
     selective_scan_fwd_kernel(const __grid_constant__ ScanParams p,
                               const __grid_constant__ CUtensorMap tm_u,
@@ -620,23 +680,28 @@ __global__ void __launch_bounds__(kScanWarps * 32, ScanLayout<kCpl>::kMinBlocks 
         float sdt[kCpl];
 #pragma unroll
         for (int c = 0; c < kCpl; ++c) {
-            out_row[c] = (valid[c] && p.out != nullptr)
-                             ? static_cast<IoT*>(p.out) + chain[c] * p.seqlen + t_begin : nullptr;
+            const int64_t obase = kBld ? (b * p.seqlen + t_begin) * p.dim + (chain[c] - b * p.dim)
+                                        : chain[c] * p.seqlen + t_begin;
+            out_row[c] = (valid[c] && p.out != nullptr) ? static_cast<IoT*>(p.out) + obase : nullptr;
             ckpt_row[c] = (valid[c] && p.ckpt != nullptr)
                               ? p.ckpt + (chain[c] * p.ckpt_tiles + t_begin / kCkptSteps) * kNPad
                               : nullptr;
             sdt[c] = 0.0f;
         }
         bool ok;
-        if (p.ckpt != nullptr)           // checkpoint pass of the backward: states only
-            ok = run_segment<IoT, kCpl, kHasZ, kSoftplus, kZoh, false, true, false>(
+        if constexpr (kBld) {            // chained mode only, with outputs
+            ok = run_segment<IoT, kCpl, kHasZ, kSoftplus, kZoh, true, false, false, true>(
                 p, maps, wsm, lane, b, d0, t_begin, t_end, lc, out_row, seq, sdt, ckpt_row);
-        else if (p.mode == kModeSegments)
-            ok = run_segment<IoT, kCpl, kHasZ, kSoftplus, kZoh, true, false, true>(
+        } else if (p.ckpt != nullptr) {  // checkpoint pass of the backward: states only
+            ok = run_segment<IoT, kCpl, kHasZ, kSoftplus, kZoh, false, true, false, false>(
                 p, maps, wsm, lane, b, d0, t_begin, t_end, lc, out_row, seq, sdt, ckpt_row);
-        else
-            ok = run_segment<IoT, kCpl, kHasZ, kSoftplus, kZoh, true, false, false>(
+        } else if (p.mode == kModeSegments) {
+            ok = run_segment<IoT, kCpl, kHasZ, kSoftplus, kZoh, true, false, true, false>(
                 p, maps, wsm, lane, b, d0, t_begin, t_end, lc, out_row, seq, sdt, ckpt_row);
+        } else {
+            ok = run_segment<IoT, kCpl, kHasZ, kSoftplus, kZoh, true, false, false, false>(
+                p, maps, wsm, lane, b, d0, t_begin, t_end, lc, out_row, seq, sdt, ckpt_row);
+        }
         if (!ok) break;
 
         const bool last_seg = k == p.nseg - 1;

@@ -29,6 +29,7 @@ MAMBA_FLAG_PARALLEL_CHUNKS = 0x2
 MAMBA_FLAG_TEST_WITHHOLD_HANDOFF = 0x4
 MAMBA_FLAG_ZOH = 0x8
 MAMBA_FLAG_PDL = 0x10
+MAMBA_FLAG_LAYOUT_BLD = 0x20
 
 _DTYPE_CODE = {torch.float32: MAMBA_F32, torch.bfloat16: MAMBA_BF16}
 
@@ -168,6 +169,26 @@ def _stream_handle(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(s.cuda_stream)
 
 
+def _layout_flags(layout, flags):
+    """Flags with MAMBA_FLAG_LAYOUT_BLD set for ``layout="bld"``, and whether it is set."""
+    if layout not in ("bdl", "bld"):
+        raise ValueError(f"layout must be 'bdl' or 'bld', not {layout!r}")
+    if layout == "bld":
+        flags |= MAMBA_FLAG_LAYOUT_BLD
+    return flags, bool(flags & MAMBA_FLAG_LAYOUT_BLD)
+
+
+def _scan_sizes(u, bld):
+    """(batch, dim, L) of the activations u."""
+    if u.dim() != 3:
+        raise ValueError(f"u must have 3 dimensions, got shape {tuple(u.shape)}")
+    if bld:
+        batch, L, dim = u.shape
+    else:
+        batch, dim, L = u.shape
+    return batch, dim, L
+
+
 def make_scan_dims(batch, dim, dstate, seqlen, io_dtype, bc_dtype, num_chunks=0, flags=0,
                    workspace=None) -> MambaDims:
     return MambaDims(batch=batch, dim=dim, dstate=dstate, seqlen=seqlen,
@@ -200,23 +221,27 @@ def scan_workspace_bytes(batch, dim, dstate, seqlen, io_dtype=torch.bfloat16,
 
 def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
                        out=None, last_state=None, return_last_state=False, num_chunks=0,
-                       flags=0, workspace=None, stream=None, initial_state=None, zoh=False):
+                       flags=0, workspace=None, stream=None, initial_state=None, zoh=False,
+                       layout="bdl"):
     """Selective scan forward through ``mamba_selective_scan_fwd`` (or
     ``mamba_selective_scan_fwd_with_state`` when ``initial_state`` is given).
 
-    u, delta, z: (batch, dim, L) fp32 or bf16 (one dtype); B, C: (batch, N, L)
+    u, delta, z: (batch, dim, L) fp32 or bf16 (one dtype), or (batch, L, dim)
+    with ``layout="bld"`` (MAMBA_FLAG_LAYOUT_BLD); B, C: (batch, N, L)
     fp32 or bf16; A: (dim, N) fp32; D, delta_bias: (dim,) fp32 or None;
     initial_state: (batch, dim, N) fp32 start state or None (zero).  ``zoh``
     sets MAMBA_FLAG_ZOH (zero-order-hold input term).
-    Returns ``out`` (batch, dim, L) in u's dtype, and the fp32 last state
+    Returns ``out`` (u's shape and dtype), and the fp32 last state
     (batch, dim, N) too when ``return_last_state`` or ``last_state`` is given.
     """
-    batch, dim, L = u.shape
+    flags, bld = _layout_flags(layout, flags)
+    batch, dim, L = _scan_sizes(u, bld)
+    act = (batch, L, dim) if bld else (batch, dim, L)
     N = A.shape[1]
     io, bc = u.dtype, B.dtype
-    _check_cuda("u", u, (torch.float32, torch.bfloat16), (batch, dim, L))
-    _check_cuda("delta", delta, (io,), (batch, dim, L))
-    _check_cuda("z", z, (io,), (batch, dim, L))
+    _check_cuda("u", u, (torch.float32, torch.bfloat16), act)
+    _check_cuda("delta", delta, (io,), act)
+    _check_cuda("z", z, (io,), act)
     _check_cuda("A", A, (torch.float32,), (dim, N))
     _check_cuda("B", B, (torch.float32, torch.bfloat16), (batch, N, L))
     _check_cuda("C", C, (bc,), (batch, N, L))
@@ -224,7 +249,7 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softp
     _check_cuda("delta_bias", delta_bias, (torch.float32,), (dim,))
     if out is None:
         out = torch.empty_like(u)
-    _check_cuda("out", out, (io,), (batch, dim, L))
+    _check_cuda("out", out, (io,), act)
     if last_state is None and return_last_state:
         last_state = torch.empty((batch, dim, N), dtype=torch.float32, device=u.device)
     _check_cuda("last_state", last_state, (torch.float32,), (batch, dim, N))
@@ -268,7 +293,7 @@ def scan_host_workspace_bytes(batch, dim, dstate, seqlen, io_dtype=torch.bfloat1
 def selective_scan_fwd_host(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
                             out=None, last_state=None, return_last_state=False, rows=0,
                             num_chunks=0, flags=0, workspace=None, stream=None,
-                            initial_state=None, zoh=False, device=None):
+                            initial_state=None, zoh=False, device=None, layout="bdl"):
     """Selective scan over HOST tensors through ``mamba_selective_scan_fwd_host``.
 
     Every tensor argument is a contiguous CPU tensor (page-locked for the copies
@@ -278,14 +303,16 @@ def selective_scan_fwd_host(u, delta, A, B, C, D=None, z=None, delta_bias=None, 
     (allocated on ``device``, default the current CUDA device, when None).
     The call returns once the work is enqueued on ``stream``; synchronise it
     before reading ``out`` / ``last_state``.  Returns ``out`` (and the last
-    state, as ``selective_scan_fwd`` does).
+    state, as ``selective_scan_fwd`` does).  ``layout`` as for ``selective_scan_fwd``.
     """
-    batch, dim, L = u.shape
+    flags, bld = _layout_flags(layout, flags)
+    batch, dim, L = _scan_sizes(u, bld)
+    act = (batch, L, dim) if bld else (batch, dim, L)
     N = A.shape[1]
     io, bc = u.dtype, B.dtype
-    _check_host("u", u, (torch.float32, torch.bfloat16), (batch, dim, L))
-    _check_host("delta", delta, (io,), (batch, dim, L))
-    _check_host("z", z, (io,), (batch, dim, L))
+    _check_host("u", u, (torch.float32, torch.bfloat16), act)
+    _check_host("delta", delta, (io,), act)
+    _check_host("z", z, (io,), act)
     _check_host("A", A, (torch.float32,), (dim, N))
     _check_host("B", B, (torch.float32, torch.bfloat16), (batch, N, L))
     _check_host("C", C, (bc,), (batch, N, L))
@@ -295,7 +322,7 @@ def selective_scan_fwd_host(u, delta, A, B, C, D=None, z=None, delta_bias=None, 
     pin = torch.cuda.is_available()
     if out is None:
         out = torch.empty(u.shape, dtype=io, pin_memory=pin)
-    _check_host("out", out, (io,), (batch, dim, L))
+    _check_host("out", out, (io,), act)
     if last_state is None and return_last_state:
         last_state = torch.empty((batch, dim, N), dtype=torch.float32, pin_memory=pin)
     _check_host("last_state", last_state, (torch.float32,), (batch, dim, N))

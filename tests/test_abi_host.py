@@ -292,3 +292,46 @@ def test_ssd_binding_checks_tensors_on_the_host():
     B = torch.zeros(1, 8, 1, 128, dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="CUDA"):
         ops.ssd_chunk_scan_fwd(x, dt, A, B, B)
+
+
+def test_plan_bld_layout(lib):
+    """Activations in (batch, seqlen, dim): always chained, TMA when a row of
+    channels is a multiple of 16 bytes (and B/C rows are), and the parallel
+    mode refused when forced."""
+    BLD = ops.MAMBA_FLAG_LAYOUT_BLD
+    c = SCAN_CONFIGS["long_dna_1m"]
+    p = ops.scan_plan(c.batch, c.dim, c.dstate, c.seqlen, c.io_dtype, c.bc_dtype, flags=BLD)
+    assert p["mode"] == 0 and p["launches"] == 1 and p["units_pass_b"] == 0
+    assert p["nchunks"] == min((8 * 148 * 16 + p["groups"] - 1) // p["groups"], c.seqlen // 256)
+    # TMA needs dim * size (not seqlen * size) to be a multiple of 16 bytes; B/C
+    # rows (seqlen * size) still do
+    assert ops.scan_plan(1, 40, 16, 40, torch.bfloat16, torch.bfloat16, flags=BLD)["tma_capable"] == 1
+    assert ops.scan_plan(1, 36, 16, 40, torch.bfloat16, torch.bfloat16, flags=BLD)["tma_capable"] == 0
+    assert ops.scan_plan(1, 40, 16, 37, torch.bfloat16, torch.bfloat16, flags=BLD)["tma_capable"] == 0
+    assert ops.scan_plan(1, 40, 16, 40, torch.float32, torch.float32, flags=BLD)["tma_capable"] == 1
+    assert ops.scan_plan(1, 38, 16, 40, torch.float32, torch.float32, flags=BLD)["tma_capable"] == 0
+    dims = _dims(seqlen=1024)
+    dims.num_chunks = 4
+    dims.flags = BLD | ops.MAMBA_FLAG_PARALLEL_CHUNKS
+    plan = ops.ScanPlan()
+    assert lib.mamba_selective_scan_plan(ctypes.byref(dims), 148, ctypes.byref(plan)) == -2
+    dims.flags = BLD
+    assert lib.mamba_selective_scan_plan(ctypes.byref(dims), 148, ctypes.byref(plan)) == 0
+
+
+def test_backward_refuses_bld_layout(lib):
+    d = _dims()
+    d.flags = ops.MAMBA_FLAG_LAYOUT_BLD
+    rc = lib.mamba_selective_scan_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, 1, None,
+                                      FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None,
+                                      None, ctypes.byref(d), None)
+    assert rc == -2
+
+
+def test_binding_layout_argument():
+    with pytest.raises(ValueError):
+        ops._layout_flags("bdl_", 0)
+    assert ops._layout_flags("bld", ops.MAMBA_FLAG_ZOH) == (ops.MAMBA_FLAG_ZOH | ops.MAMBA_FLAG_LAYOUT_BLD, True)
+    assert ops._layout_flags("bdl", 0) == (0, False)
+    u = torch.empty(2, 7, 5)
+    assert ops._scan_sizes(u, True) == (2, 5, 7) and ops._scan_sizes(u, False) == (2, 7, 5)
