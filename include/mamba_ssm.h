@@ -117,6 +117,10 @@ typedef enum {
  * at a time.  Such calls always run in mode 0: MAMBA_FLAG_PARALLEL_CHUNKS with
  * it returns MAMBA_ERR_UNSUPPORTED, and so does the backward. */
 #define MAMBA_FLAG_LAYOUT_BLD 0x20
+/* Scan forward: keep one lane per channel where the plan would give each
+ * channel two lanes (plan.lanes_per_channel; see mamba_scan_plan_t).  For
+ * tests and measurements; results agree to rounding either way. */
+#define MAMBA_FLAG_ONE_LANE_PER_CHANNEL 0x40
 
 #define MAMBA_MAX_DSTATE 16
 
@@ -153,8 +157,9 @@ typedef struct {
 
 /*
  * How a scan call will run (host-side planning; no CUDA call is made).
- * The channels form groups of 32 or 64 (one warp each, with one or two
- * channels per lane); the sequence is cut into
+ * The channels form groups of 32 (one warp each, one channel per lane), or of
+ * 16 with two lanes per channel when 32-channel groups would leave resident
+ * warps idle in mode 0; the sequence is cut into
  * nchunks segments of chunk_len steps (the last may be shorter).  A persistent
  * grid of warps pulls (segment, group) work items from a counter.
  *   mode 0 (chained): one launch.  Segment k of a group starts from the state
@@ -179,7 +184,7 @@ typedef struct {
     int32_t nchunks;           /* segments per sequence */
     int32_t tile_len;          /* time steps staged per pipeline stage */
     int64_t chunk_len;         /* time steps per segment (multiple of tile_len) */
-    int64_t groups;            /* batch * ceil(dim / 32) */
+    int64_t groups;            /* batch * ceil(dim / (32 / lanes_per_channel)) */
     int64_t units_pass_a;      /* work items of the first launch (group x segment) */
     int64_t units_pass_b;      /* correction items, chain x later segment (0 in mode 0) */
     int32_t warps_per_cta;
@@ -187,7 +192,10 @@ typedef struct {
     int32_t tma_capable;       /* strides allow TMA staging */
     int32_t mode;              /* 0 chained, 1 parallel */
     int32_t channels_per_lane; /* 1 or 2: a group is 32 x this many channels */
-    int32_t reserved;
+    int32_t lanes_per_channel; /* 1, or 2 when a group is 16 channels whose 16 state
+                                * entries are split over two lanes (mode 0 with fewer
+                                * 32-channel groups than resident warps, Euler input
+                                * term, (batch, dim, seqlen) layout) */
     int64_t max_warps;         /* warps the persistent grid uses at most */
     size_t workspace_bytes;
 } mamba_scan_plan_t;

@@ -14,6 +14,7 @@
 #include "scan_backward.cuh"
 #include "ssd_chunk_scan.cuh"
 #include "scan_carry.cuh"
+#include "scan_split.cuh"
 
 namespace mamba {
 
@@ -126,6 +127,41 @@ cudaError_t dispatch_scan_cpl(const ScanParams& prm, const CUtensorMap* maps, bo
                   : launch_scan<IoT, kCpl, true, false, kZoh, kBld>(prm, maps, want_warps, dev, sms, stream);
     return sp ? launch_scan<IoT, kCpl, false, true, kZoh, kBld>(prm, maps, want_warps, dev, sms, stream)
               : launch_scan<IoT, kCpl, false, false, kZoh, kBld>(prm, maps, want_warps, dev, sms, stream);
+}
+
+template <typename IoT, bool kHasZ, bool kSoftplus>
+cudaError_t launch_scan_split(const ScanParams& prm, const CUtensorMap* maps, int64_t want_warps,
+                              int dev, int sms, cudaStream_t stream) {
+    using Lay = SplitLayout;
+    static bool attr_done[kMaxDevices] = {false};
+    static int resident[kMaxDevices] = {0};
+    auto kernel = selective_scan_fwd_split_kernel<IoT, kHasZ, kSoftplus>;
+    cudaError_t e = ensure_smem_attr(kernel, Lay::kCtaSmem, attr_done, dev);
+    if (e != cudaSuccess) return e;
+    int per_sm = (dev >= 0 && dev < kMaxDevices) ? resident[dev] : 0;
+    if (per_sm <= 0) {
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kScanWarps * 32,
+                                                          Lay::kCtaSmem);
+        if (e != cudaSuccess) return e;
+        if (per_sm <= 0) return cudaErrorInvalidConfiguration;
+        if (dev >= 0 && dev < kMaxDevices) resident[dev] = per_sm;
+    }
+    const int64_t want = (want_warps + kScanWarps - 1) / kScanWarps;
+    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)per_sm * sms));
+    kernel<<<(unsigned)grid, kScanWarps * 32, Lay::kCtaSmem, stream>>>(prm, maps[0], maps[1],
+                                                                         maps[2], maps[3], maps[4]);
+    return cudaGetLastError();
+}
+
+// Two lanes per channel (chained mode, Euler, (batch, dim, seqlen)).
+template <typename IoT>
+cudaError_t dispatch_scan_split(const ScanParams& prm, const CUtensorMap* maps, bool has_z, bool sp,
+                                int64_t want_warps, int dev, int sms, cudaStream_t stream) {
+    if (has_z)
+        return sp ? launch_scan_split<IoT, true, true>(prm, maps, want_warps, dev, sms, stream)
+                  : launch_scan_split<IoT, true, false>(prm, maps, want_warps, dev, sms, stream);
+    return sp ? launch_scan_split<IoT, false, true>(prm, maps, want_warps, dev, sms, stream)
+              : launch_scan_split<IoT, false, false>(prm, maps, want_warps, dev, sms, stream);
 }
 
 // Kernel instance for (channels per lane, zero-order hold, activation layout).
@@ -291,7 +327,7 @@ ScanWorkspace scan_workspace_layout(const mamba_dims_t* dims, int64_t groups, in
 }
 
 // Planning rules (pure host logic, see mamba_selective_scan_plan).
-//  - One channel per lane (32-channel groups).
+//  - One channel per lane (32-channel groups), or two (see the last rule).
 //  - W = resident warps on the GPU (16 per SM), G = channel groups.
 //  - G >= W/4: chained mode, K segments so that G*K is about 8 W work items
 //    (even load across SMs), segments at least 256 steps long.  At most G
@@ -304,6 +340,10 @@ ScanWorkspace scan_workspace_layout(const mamba_dims_t* dims, int64_t groups, in
 //    mode for a forced K.
 //  - Activations in the (batch, seqlen, dim) layout always run chained (the
 //    correction pass reads rows along time).
+//  - Chained with G < W (groups of 32 that leave resident warps idle), Euler,
+//    (batch, dim, seqlen): two lanes per channel, groups of 16 (2 G warps);
+//    K is then chosen for those groups.  MAMBA_FLAG_ONE_LANE_PER_CHANNEL
+//    keeps one lane.
 mamba_status_t plan_scan(const mamba_dims_t* dims, int sm_count, mamba_scan_plan_t* plan) {
     mamba_status_t st = check_dims(dims, true);
     if (st != MAMBA_OK) return st;
@@ -350,29 +390,49 @@ mamba_status_t plan_scan(const mamba_dims_t* dims, int sm_count, mamba_scan_plan
                 1, std::min<int64_t>(W / groups, L / std::max<int64_t>(16 * T, 512)));
         }
     }
+    auto segments = [&](int64_t& k, int64_t& len) {
+        len = L;
+        if (k > 1 && L > 0) {
+            len = ((L + k - 1) / k + T - 1) / T * T;
+            k = (L + len - 1) / len;
+        }
+        if (k <= 1) {
+            k = 1;
+            len = L;
+        }
+    };
     int64_t seg_len = L;
-    if (K > 1 && L > 0) {
-        seg_len = ((L + K - 1) / K + T - 1) / T * T;
-        K = (L + seg_len - 1) / seg_len;
+    segments(K, seg_len);
+    if (K == 1) mode = 0;
+    // Two lanes per channel: chained, groups of 32 fewer than resident warps.
+    int lanes = 1;
+    int64_t groups_run = groups;
+    if (mode == 0 && groups > 0 && L > 0 && groups < W && !bld &&
+        !(dims->flags & MAMBA_FLAG_ZOH) && !(dims->flags & MAMBA_FLAG_ONE_LANE_PER_CHANNEL)) {
+        lanes = 2;
+        groups_run = dims->batch * ((dims->dim + 15) / 16);
+        if (dims->num_chunks < 1) {
+            K = std::max<int64_t>(1, std::min<int64_t>((8 * W + groups_run - 1) / groups_run,
+                                                       L / 256));
+            segments(K, seg_len);
+        }
     }
-    if (K <= 1) {
-        K = 1;
-        seg_len = L;
-        mode = 0;
-    }
-    const int64_t items = groups * K;
+    const int64_t items = groups_run * K;
     const int64_t chains = dims->batch * dims->dim;
     const int64_t fixes = mode == 0 ? 0 : chains * (K - 1);
     if (items >= ((int64_t)1 << 31) || fixes >= ((int64_t)1 << 31)) return MAMBA_ERR_UNSUPPORTED;
+    plan->groups = groups_run;
+    plan->lanes_per_channel = lanes;
     plan->nchunks = (int32_t)K;
     plan->chunk_len = seg_len;
     plan->mode = mode;
     plan->units_pass_a = items;
     plan->units_pass_b = fixes;
-    plan->max_warps = mode == 0 && K > 1 ? std::min<int64_t>(groups, W) : std::min<int64_t>(items, W);
+    plan->max_warps = mode == 0 && K > 1 ? std::min<int64_t>(groups_run, W)
+                                         : std::min<int64_t>(items, W);
     plan->launches = (groups > 0 && L > 0) ? (mode == 0 ? 1 : 3) : 0;
     plan->workspace_bytes =
-        (groups > 0 && L > 0) ? scan_workspace_layout(dims, groups, K, mode).total : 0;
+        (groups > 0 && L > 0) ? scan_workspace_layout(dims, groups_run, K, mode).total : 0;
     return MAMBA_OK;
 }
 
@@ -473,10 +533,13 @@ mamba_status_t scan_fwd_internal(const void* u, const void* delta, const float* 
     const int sms = current_sm_count(&dev);
     if (sms <= 0) return MAMBA_ERR_CUDA;
     mamba_scan_plan_t plan;
-    st = plan_scan(dims, sms, &plan);
+    mamba_dims_t pd = *dims;
+    if (ckpt != nullptr) pd.flags |= MAMBA_FLAG_ONE_LANE_PER_CHANNEL;   // checkpoints: one lane
+    st = plan_scan(&pd, sms, &plan);
     if (st != MAMBA_OK) return st;
     if (dims->workspace == nullptr || dims->workspace_bytes < plan.workspace_bytes)
         return MAMBA_ERR_WORKSPACE;
+    const int64_t group_rows = 32 / plan.lanes_per_channel;
     if (!aligned(dims->workspace, 256)) return MAMBA_ERR_ALIGN;
 
     ScanParams prm{};
@@ -496,7 +559,7 @@ mamba_status_t scan_fwd_internal(const void* u, const void* delta, const float* 
     prm.batch = dims->batch;
     prm.dim = dims->dim;
     prm.seqlen = dims->seqlen;
-    prm.groups_per_batch = (dims->dim + 32 * plan.channels_per_lane - 1) / (32 * plan.channels_per_lane);
+    prm.groups_per_batch = (dims->dim + group_rows - 1) / group_rows;
     prm.groups = plan.groups;
     prm.chains = chains;
     prm.seg_len = plan.chunk_len;
@@ -515,7 +578,7 @@ mamba_status_t scan_fwd_internal(const void* u, const void* delta, const float* 
             : (unsigned int)std::min<int64_t>(std::max<int64_t>(plan.chunk_len * 64, 1 << 20),
                                               (int64_t)1 << 31);
     uint8_t* ws = static_cast<uint8_t*>(dims->workspace);
-    const ScanWorkspace lay = scan_workspace_layout(dims, plan.groups, plan.nchunks, plan.mode);
+    const ScanWorkspace lay = scan_workspace_layout(&pd, plan.groups, plan.nchunks, plan.mode);
     unsigned int* counters = reinterpret_cast<unsigned int*>(ws + kWsCounters);
     prm.flags = reinterpret_cast<unsigned int*>(ws + kWsFlags);
     if (lay.carry) prm.carry = reinterpret_cast<float*>(ws + lay.carry);
@@ -533,7 +596,7 @@ mamba_status_t scan_fwd_internal(const void* u, const void* delta, const float* 
         const uint64_t L = (uint64_t)dims->seqlen;
         const uint64_t Dm = (uint64_t)dims->dim, Bt = (uint64_t)dims->batch;
         const uint64_t N = (uint64_t)dims->dstate;
-        const uint32_t rows = 32u * (uint32_t)plan.channels_per_lane;
+        const uint32_t rows = (uint32_t)group_rows;
         // (rows x T) tiles of (batch, dim, seqlen) rows with 32-byte swizzle, or
         // dense (T x rows) tiles of (batch, seqlen, dim) that the kernel transposes
         auto act = [&](CUtensorMap* m, const void* base) {
@@ -561,6 +624,12 @@ mamba_status_t scan_fwd_internal(const void* u, const void* delta, const float* 
         prm.counter = counter;
         prm.items = items;
         if (items == 0) return cudaSuccess;
+        if (plan.lanes_per_channel == 2)
+            return dims->io_dtype == MAMBA_BF16
+                       ? dispatch_scan_split<__nv_bfloat16>(prm, maps, has_z, sp, plan.max_warps,
+                                                            dev, sms, stream)
+                       : dispatch_scan_split<float>(prm, maps, has_z, sp, plan.max_warps, dev,
+                                                    sms, stream);
         return dims->io_dtype == MAMBA_BF16
                    ? dispatch_scan<__nv_bfloat16>(prm, maps, plan.channels_per_lane, has_z, sp,
                                                   zoh, plan.max_warps, dev, sms, stream)
@@ -1421,7 +1490,7 @@ MAMBA_API mamba_status_t mamba_selective_scan_bwd(
     // 1. checkpoint pass: the forward, chained in w.K segments, states only
     mamba_dims_t fd = *dims;
     fd.num_chunks = (int32_t)w.K;
-    fd.flags = dims->flags & (MAMBA_FLAG_NO_TMA | MAMBA_FLAG_ZOH);
+    fd.flags = (dims->flags & (MAMBA_FLAG_NO_TMA | MAMBA_FLAG_ZOH)) | MAMBA_FLAG_ONE_LANE_PER_CHANNEL;
     fd.workspace = ws;
     fd.workspace_bytes = w.fwd_bytes;
     float* ckpt = reinterpret_cast<float*>(ws + w.ckpt);

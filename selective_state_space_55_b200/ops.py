@@ -30,6 +30,7 @@ MAMBA_FLAG_TEST_WITHHOLD_HANDOFF = 0x4
 MAMBA_FLAG_ZOH = 0x8
 MAMBA_FLAG_PDL = 0x10
 MAMBA_FLAG_LAYOUT_BLD = 0x20
+MAMBA_FLAG_ONE_LANE_PER_CHANNEL = 0x40
 
 _DTYPE_CODE = {torch.float32: MAMBA_F32, torch.bfloat16: MAMBA_BF16}
 
@@ -59,12 +60,12 @@ class ScanPlan(ctypes.Structure):
         ("units_pass_a", ctypes.c_int64), ("units_pass_b", ctypes.c_int64),
         ("warps_per_cta", ctypes.c_int32), ("launches", ctypes.c_int32),
         ("tma_capable", ctypes.c_int32), ("mode", ctypes.c_int32),
-        ("channels_per_lane", ctypes.c_int32), ("reserved", ctypes.c_int32),
+        ("channels_per_lane", ctypes.c_int32), ("lanes_per_channel", ctypes.c_int32),
         ("max_warps", ctypes.c_int64), ("workspace_bytes", ctypes.c_size_t),
     ]
 
     def as_dict(self) -> dict:
-        return {name: getattr(self, name) for name, _ in self._fields_ if name != "reserved"}
+        return {name: getattr(self, name) for name, _ in self._fields_}
 
 
 class MambaError(RuntimeError):

@@ -189,12 +189,34 @@ def test_plan_layer_shapes(lib):
     chains = c.batch * c.dim
     flags = (p["groups"] * 4 + 255) // 256 * 256
     assert p["workspace_bytes"] == 256 + flags + chains * 64
-    # 1.4B layer: 1024 groups, chained the same way with one warp per group
+    assert p["lanes_per_channel"] == 1
+    # 1.4B layer: 1024 groups of 32 would leave half the 2368 warp slots idle,
+    # so each channel gets two lanes: 2048 groups of 16, one warp each
     c = SCAN_CONFIGS["mamba_1p4b_layer"]
     p = ops.scan_plan(c.batch, c.dim, c.dstate, c.seqlen, c.io_dtype, c.bc_dtype)
-    assert p["mode"] == 0 and p["channels_per_lane"] == 1 and p["groups"] == 1024
-    assert p["nchunks"] == 8 and p["max_warps"] == 1024
-    assert p["workspace_bytes"] == 256 + 4096 + 8 * 4096 * 64
+    assert p["mode"] == 0 and p["lanes_per_channel"] == 2 and p["groups"] == 2048
+    assert p["nchunks"] == 8 and p["max_warps"] == 2048
+    assert p["workspace_bytes"] == 256 + 8192 + 8 * 4096 * 64
+    q = ops.scan_plan(c.batch, c.dim, c.dstate, c.seqlen, c.io_dtype, c.bc_dtype,
+                      flags=ops.MAMBA_FLAG_ONE_LANE_PER_CHANNEL)
+    assert q["lanes_per_channel"] == 1 and q["groups"] == 1024 and q["max_warps"] == 1024
+    assert q["workspace_bytes"] == 256 + 4096 + 8 * 4096 * 64
+
+
+def test_plan_two_lanes_per_channel_rules(lib):
+    bf = torch.bfloat16
+    two = lambda *a, **k: ops.scan_plan(*a, **k)["lanes_per_channel"] == 2  # noqa: E731
+    assert two(8, 4096, 16, 2048, bf, bf)                    # chained, 1024 < 2368 groups
+    assert not two(16, 5120, 16, 2048, bf, bf)               # 2560 groups fill the GPU
+    assert not two(8, 4096, 16, 2048, bf, bf, flags=ops.MAMBA_FLAG_ZOH)
+    assert not two(8, 4096, 16, 2048, bf, bf, flags=ops.MAMBA_FLAG_LAYOUT_BLD)
+    assert not two(1, 1536, 16, 1 << 20, bf, bf)             # parallel mode
+    assert two(1, 64, 16, 100, bf, bf)                       # one short segment, chained
+    assert two(2, 100, 16, 512, torch.float32, torch.float32)
+    p = ops.scan_plan(3, 40, 16, 4096, bf, bf, num_chunks=4)
+    assert p["lanes_per_channel"] == 2 and p["groups"] == 3 * 3 and p["nchunks"] == 4
+    p = ops.scan_plan(3, 40, 16, 4096, bf, bf, num_chunks=4, flags=ops.MAMBA_FLAG_PARALLEL_CHUNKS)
+    assert p["lanes_per_channel"] == 1 and p["mode"] == 1
 
 
 def test_plan_parallel_for_the_million_token_sequence(lib):

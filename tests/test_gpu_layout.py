@@ -22,6 +22,7 @@ pytestmark = pytest.mark.gpu
 
 DEV = "cuda"
 ACT = ("u", "delta", "z")
+ONE = ops.MAMBA_FLAG_ONE_LANE_PER_CHANNEL
 
 
 @pytest.fixture(scope="module")
@@ -60,10 +61,11 @@ def oracle_scan(ref, x, **kw):
 
 
 def check(ref, x, tol, zoh=False, h0=None, flags=0):
-    """Bitwise against the (batch, dim, seqlen) call in one segment (chained
-    segments reproduce it bit for bit), and within tol of the oracle."""
+    """Bitwise against the (batch, dim, seqlen) call with one lane per channel
+    (the kernel this layout runs) in one segment (chained segments reproduce it
+    bit for bit), and within tol of the oracle."""
     out_b, last_b = scan(x, "bld", zoh=zoh, initial_state=h0, flags=flags)
-    out_d, last_d = scan(x, "bdl", zoh=zoh, initial_state=h0, num_chunks=1)
+    out_d, last_d = scan(x, "bdl", zoh=zoh, initial_state=h0, num_chunks=1, flags=ONE)
     assert torch.equal(out_b, out_d)
     assert torch.equal(last_b, last_d)
     o_out, o_last = oracle_scan(ref, x, zoh=zoh, initial_state=None if h0 is None else h0.cpu())
@@ -142,7 +144,7 @@ def test_full_2p8b_layer_bitwise():
     c = I.SCAN_CONFIGS["mamba_2p8b_layer"]
     x = I.make_scan_inputs(c, DEV, seed=1)
     a = scan(x, "bld")
-    b = scan(x, "bdl")
+    b = scan(x, "bdl", flags=ONE)
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
 
 
