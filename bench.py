@@ -615,9 +615,18 @@ def bench_ours(args, rank, world, local):
     upd_bytes = R.update_bytes(d.batch, d.dim, d.dstate, 2, 2, True)
     decode_gbs = upd_bytes * d.layers / (decode_ms / K * 1e-3) / 1e9
     digest = sources_digest()
+    # Which kernel the plan runs, and its DRAM traffic where the record was
+    # captured on this very workload (two lanes per channel on the 1.4B layer,
+    # one lane on the 2.8B layer).
+    scan_kernel = ("selective_scan_fwd_split_kernel" if w.plan.get("lanes_per_channel") == 2
+                   else "selective_scan_fwd_kernel")
+    recorded_on = {"selective_scan_fwd_kernel": ("mamba_2p8b_layer", 16),
+                   "selective_scan_fwd_split_kernel": ("mamba_1p4b_layer", 8)}
+    same_case = ((c.name, c.batch) == recorded_on[scan_kernel] and args.scan_variant == "euler"
+                 and not args.scan_seqlen)
     scan_roof = {
         "bound": "alu", "pipe": f"MUFU (16 ops/clk/SM; {mufu} per element)",
-        "kernel": "selective_scan_fwd_kernel",
+        "kernel": scan_kernel,
         "achieved": round(achieved, 2), "peak": round(peak_elems, 2), "unit": "Gelem/s",
         "frac": round(achieved / peak_elems, 4),
         "peak_basis": f"{sms} SMs x 16 MUFU/clk x {peaks['sm_max_mhz']:.0f} MHz / {mufu} MUFU ops "
@@ -630,7 +639,7 @@ def bench_ours(args, rank, world, local):
                          "note": "the MUFU ops this kernel issues (bf16 inputs: the gate is one tanh)"},
         "algorithmic_bytes_per_launch": scan_bytes,
         "hbm_gbs": round(scan_bytes / (scan_launch_ms * 1e-3) / 1e9, 1),
-        "traffic": recorded_traffic("selective_scan_fwd_kernel", digest),
+        "traffic": recorded_traffic(scan_kernel, digest) if same_case else None,
     }
     state_bytes = 2 * d.batch * d.dim * d.dstate * 4
     state_gbs = state_bytes * d.layers / (decode_ms / K * 1e-3) / 1e9
