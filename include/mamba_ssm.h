@@ -121,6 +121,13 @@ typedef enum {
  * channel two lanes (plan.lanes_per_channel; see mamba_scan_plan_t).  For
  * tests and measurements; results agree to rounding either way. */
 #define MAMBA_FLAG_ONE_LANE_PER_CHANNEL 0x40
+/* Scan, parallel mode: run it as one launch in which each segment looks back
+ * at the earlier segments of its channel group and corrects its own outputs
+ * (plan.mode 2), instead of three launches (segments, a warp-shuffle scan of
+ * the segments' carries, a correction pass; plan.mode 1).  Results agree to
+ * rounding.  Not the default: the one-launch form measured slower (the
+ * correction shares the scan kernel's registers). */
+#define MAMBA_FLAG_PARALLEL_ONE_LAUNCH 0x80
 
 #define MAMBA_MAX_DSTATE 16
 
@@ -179,6 +186,13 @@ typedef struct {
  *        every state entry (when Delta >= 0 throughout, i.e. softplus on).
  *     Nothing is computed twice; the correction costs as much per step as
  *     the scan but covers only the steps over which the start state matters.
+ *   mode 2 (parallel, with MAMBA_FLAG_PARALLEL_ONE_LAUNCH): the same work in one launch.
+ *     After step 1 each segment publishes its end state and sum of Delta,
+ *     waits (bounded) for the earlier segments of its channel group to have
+ *     published theirs (a decoupled look-back: segments are taken in order,
+ *     so the earlier ones always run), folds them into its own start state,
+ *     and corrects its own outputs (units_pass_b corrections, inside the
+ *     launch).
  */
 typedef struct {
     int32_t nchunks;           /* segments per sequence */
@@ -190,7 +204,7 @@ typedef struct {
     int32_t warps_per_cta;
     int32_t launches;          /* kernel launches per call (plus one memset): 1 or 3 */
     int32_t tma_capable;       /* strides allow TMA staging */
-    int32_t mode;              /* 0 chained, 1 parallel */
+    int32_t mode;              /* 0 chained, 1 parallel (three launches), 2 parallel (one launch) */
     int32_t channels_per_lane; /* 1 or 2: a group is 32 x this many channels */
     int32_t lanes_per_channel; /* 1, or 2 when a group is 16 channels whose 16 state
                                 * entries are split over two lanes (mode 0 with fewer

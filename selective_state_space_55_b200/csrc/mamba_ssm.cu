@@ -94,13 +94,13 @@ cudaError_t ensure_smem_attr(Kernel kernel, int bytes, bool* done_per_device, in
     return e;
 }
 
-template <typename IoT, int kCpl, bool kHasZ, bool kSoftplus, bool kZoh, bool kBld>
+template <typename IoT, int kCpl, bool kHasZ, bool kSoftplus, bool kZoh, bool kBld, bool kLookback>
 cudaError_t launch_scan(const ScanParams& prm, const CUtensorMap* maps, int64_t want_warps,
                         int dev, int sms, cudaStream_t stream) {
     using Lay = ScanLayout<kCpl>;
     static bool attr_done[kMaxDevices] = {false};
     static int resident[kMaxDevices] = {0};
-    auto kernel = selective_scan_fwd_kernel<IoT, kCpl, kHasZ, kSoftplus, kZoh, kBld>;
+    auto kernel = selective_scan_fwd_kernel<IoT, kCpl, kHasZ, kSoftplus, kZoh, kBld, kLookback>;
     cudaError_t e = ensure_smem_attr(kernel, Lay::kCtaSmem, attr_done, dev);
     if (e != cudaSuccess) return e;
     int per_sm = (dev >= 0 && dev < kMaxDevices) ? resident[dev] : 0;
@@ -119,14 +119,14 @@ cudaError_t launch_scan(const ScanParams& prm, const CUtensorMap* maps, int64_t 
     return cudaGetLastError();
 }
 
-template <typename IoT, int kCpl, bool kZoh, bool kBld>
+template <typename IoT, int kCpl, bool kZoh, bool kBld, bool kLookback>
 cudaError_t dispatch_scan_cpl(const ScanParams& prm, const CUtensorMap* maps, bool has_z, bool sp,
                               int64_t want_warps, int dev, int sms, cudaStream_t stream) {
     if (has_z)
-        return sp ? launch_scan<IoT, kCpl, true, true, kZoh, kBld>(prm, maps, want_warps, dev, sms, stream)
-                  : launch_scan<IoT, kCpl, true, false, kZoh, kBld>(prm, maps, want_warps, dev, sms, stream);
-    return sp ? launch_scan<IoT, kCpl, false, true, kZoh, kBld>(prm, maps, want_warps, dev, sms, stream)
-              : launch_scan<IoT, kCpl, false, false, kZoh, kBld>(prm, maps, want_warps, dev, sms, stream);
+        return sp ? launch_scan<IoT, kCpl, true, true, kZoh, kBld, kLookback>(prm, maps, want_warps, dev, sms, stream)
+                  : launch_scan<IoT, kCpl, true, false, kZoh, kBld, kLookback>(prm, maps, want_warps, dev, sms, stream);
+    return sp ? launch_scan<IoT, kCpl, false, true, kZoh, kBld, kLookback>(prm, maps, want_warps, dev, sms, stream)
+              : launch_scan<IoT, kCpl, false, false, kZoh, kBld, kLookback>(prm, maps, want_warps, dev, sms, stream);
 }
 
 template <typename IoT, bool kHasZ, bool kSoftplus>
@@ -164,17 +164,20 @@ cudaError_t dispatch_scan_split(const ScanParams& prm, const CUtensorMap* maps, 
               : launch_scan_split<IoT, false, false>(prm, maps, want_warps, dev, sms, stream);
 }
 
-// Kernel instance for (channels per lane, zero-order hold, activation layout).
+// Kernel instance for (channels per lane, zero-order hold, activation layout, look-back).
 template <typename IoT>
 cudaError_t dispatch_scan(const ScanParams& prm, const CUtensorMap* maps, int cpl, bool has_z,
                           bool sp, bool zoh, int64_t want_warps, int dev, int sms,
                           cudaStream_t stream) {
     if (cpl != 1) return cudaErrorInvalidValue;
     if (prm.bld)
-        return zoh ? dispatch_scan_cpl<IoT, 1, true, true>(prm, maps, has_z, sp, want_warps, dev, sms, stream)
-                   : dispatch_scan_cpl<IoT, 1, false, true>(prm, maps, has_z, sp, want_warps, dev, sms, stream);
-    return zoh ? dispatch_scan_cpl<IoT, 1, true, false>(prm, maps, has_z, sp, want_warps, dev, sms, stream)
-               : dispatch_scan_cpl<IoT, 1, false, false>(prm, maps, has_z, sp, want_warps, dev, sms, stream);
+        return zoh ? dispatch_scan_cpl<IoT, 1, true, true, false>(prm, maps, has_z, sp, want_warps, dev, sms, stream)
+                   : dispatch_scan_cpl<IoT, 1, false, true, false>(prm, maps, has_z, sp, want_warps, dev, sms, stream);
+    if (prm.mode == kModeLookback)
+        return zoh ? dispatch_scan_cpl<IoT, 1, true, false, true>(prm, maps, has_z, sp, want_warps, dev, sms, stream)
+                   : dispatch_scan_cpl<IoT, 1, false, false, true>(prm, maps, has_z, sp, want_warps, dev, sms, stream);
+    return zoh ? dispatch_scan_cpl<IoT, 1, true, false, false>(prm, maps, has_z, sp, want_warps, dev, sms, stream)
+               : dispatch_scan_cpl<IoT, 1, false, false, false>(prm, maps, has_z, sp, want_warps, dev, sms, stream);
 }
 
 // Correction pass of the parallel mode: a persistent grid of warps that pull
@@ -310,13 +313,14 @@ struct ScanWorkspace {
 ScanWorkspace scan_workspace_layout(const mamba_dims_t* dims, int64_t groups, int64_t K, int mode) {
     ScanWorkspace w{};
     const size_t chains = (size_t)dims->batch * (size_t)dims->dim;
-    w.zeroed = kWsFlags + align256((size_t)groups * sizeof(unsigned int));
+    const size_t nflags = (size_t)groups * (mode == 2 ? (size_t)K : 1);   // mode 2: one per segment
+    w.zeroed = kWsFlags + align256(nflags * sizeof(unsigned int));
     size_t off = w.zeroed;
     if (mode == 0 && K > 1) {
         w.carry = off;
         off += align256(chains * kNPad * sizeof(float));
     }
-    if (mode == 1) {
+    if (mode >= 1) {
         w.ws_h = off;
         off += align256((size_t)K * chains * kNPad * sizeof(float));
         w.ws_sdt = off;
@@ -404,6 +408,7 @@ mamba_status_t plan_scan(const mamba_dims_t* dims, int sm_count, mamba_scan_plan
     int64_t seg_len = L;
     segments(K, seg_len);
     if (K == 1) mode = 0;
+    if (mode == 1 && (dims->flags & MAMBA_FLAG_PARALLEL_ONE_LAUNCH)) mode = 2;
     // Two lanes per channel: chained, groups of 32 fewer than resident warps.
     int lanes = 1;
     int64_t groups_run = groups;
@@ -430,7 +435,7 @@ mamba_status_t plan_scan(const mamba_dims_t* dims, int sm_count, mamba_scan_plan
     plan->units_pass_b = fixes;
     plan->max_warps = mode == 0 && K > 1 ? std::min<int64_t>(groups_run, W)
                                          : std::min<int64_t>(items, W);
-    plan->launches = (groups > 0 && L > 0) ? (mode == 0 ? 1 : 3) : 0;
+    plan->launches = (groups > 0 && L > 0) ? (mode == 1 ? 3 : 1) : 0;
     plan->workspace_bytes =
         (groups > 0 && L > 0) ? scan_workspace_layout(dims, groups_run, K, mode).total : 0;
     return MAMBA_OK;
@@ -569,6 +574,9 @@ mamba_status_t scan_fwd_internal(const void* u, const void* delta, const float* 
     prm.bld = bld ? 1 : 0;
     prm.out_step = bld ? dims->dim : 1;
     prm.vec_out = !bld && out != nullptr && ((dims->seqlen * io_es) % 16 == 0) && aligned(out, 16);
+    prm.vec_io = ((dims->seqlen * io_es) % 16 == 0) && aligned(delta, 16) && out != nullptr &&
+                 aligned(out, 16) && (!z || aligned(z, 16));
+    prm.vec_c = ((dims->seqlen * bc_es) % 16 == 0) && aligned(C, 16);
     // A predecessor segment legitimately takes well under 64 us per step even
     // on a crowded GPU; wait that long (at least ~1 s) before reporting a stall.
     prm.withhold_handoff = (dims->flags & MAMBA_FLAG_TEST_WITHHOLD_HANDOFF) ? 1 : 0;
@@ -639,6 +647,9 @@ mamba_status_t scan_fwd_internal(const void* u, const void* delta, const float* 
     cudaError_t e;
     if (plan.mode == 0) {
         e = run(kModeChained, counters, plan.units_pass_a);
+    } else if (plan.mode == 2) {
+        // segments, each looking back at the earlier ones and correcting itself
+        e = run(kModeLookback, counters, plan.units_pass_a);
     } else {
         // segments from their own start, then the carry over segments, then
         // the start states' contributions to the outputs

@@ -127,16 +127,117 @@ __device__ __forceinline__ void load_run(const T* row, int64_t t, int valid, boo
     }
 }
 
+// Segment k's correction for one chain (one warp, lanes over time): adds
+// C_t . (exp(A S_t) (.) hin) (gated) to the segment's outputs, hin being the
+// segment's true start state.  Every lane holds the same hin.
 template <typename IoT, typename BcT, bool kHasZ, bool kSoftplus>
-__global__ void __launch_bounds__(kCorrectWarps * 32)
-    scan_correct_kernel(const __grid_constant__ CorrectParams p) {
+__device__ __forceinline__ void correct_chain(const CorrectParams& p, int64_t chain, int64_t k,
+                                              const float (&hin)[kNPad], int lane) {
     constexpr int V = 16 / (int)sizeof(IoT);    // steps per lane and pass
     constexpr bool kExact = sizeof(IoT) == 4;
-    const int lane = threadIdx.x & 31;
     const IoT* delta = static_cast<const IoT*>(p.delta);
     const IoT* zz = static_cast<const IoT*>(p.z);
     const BcT* Cm = static_cast<const BcT*>(p.C);
     IoT* out = static_cast<IoT*>(p.out);
+    const int64_t b = chain / p.dim, d = chain % p.dim;
+    const int64_t t_begin = k * p.seg_len;
+    const int64_t t_end = min(t_begin + p.seg_len, p.seqlen);
+    float a2[kNPad];
+#pragma unroll
+    for (int n = 0; n < kNPad; ++n) a2[n] = n < p.dstate ? p.A[d * p.dstate + n] * kLog2e : 0.0f;
+    const float bias = p.delta_bias ? p.delta_bias[d] : 0.0f;
+    const IoT* drow = delta + chain * p.seqlen;
+    const IoT* zrow = kHasZ ? zz + chain * p.seqlen : nullptr;
+    IoT* orow = out + chain * p.seqlen;
+    const BcT* crow = Cm + b * p.dstate * p.seqlen;
+    float S_run = 0.0f;       // sum of Delta before this pass's first step
+    bool monotone = true;     // Delta >= 0 at every step so far
+
+    for (int64_t t0 = t_begin; t0 < t_end; t0 += 32 * V) {
+        // State entries whose exp(A_n S_t) is below 2^-127 for the rest of
+        // the segment (0 after ex2.approx.ftz) drop out; none left, done.
+        uint32_t active = 0;
+#pragma unroll
+        for (int n = 0; n < kNPad; ++n)
+            if (n < p.dstate && !(monotone && a2[n] < 0.0f && a2[n] * S_run < kUnderflowLog2))
+                active |= 1u << n;
+        if (active == 0) break;
+        const int64_t ts = t0 + (int64_t)lane * V;
+        const int valid = (int)max((int64_t)0, min((int64_t)V, t_end - ts));
+        float dl[V];
+        load_run<IoT, V>(drow, ts, valid, p.vec_io != 0, dl);
+        float S[V];
+        float run = 0.0f;
+        bool nonneg = true;
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+            float dt = 0.0f;
+            if (j < valid) {
+                const float sarg = dl[j] + bias;
+                dt = kSoftplus ? (kExact ? softplus_f32(sarg) : softplus_lg2(sarg)) : sarg;
+            }
+            nonneg = nonneg && dt >= 0.0f;
+            run += dt;
+            S[j] = run;
+        }
+        // exclusive prefix of the lanes' totals, then this pass's total
+        float incl = run;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        const float before = S_run + (incl - run);
+        S_run += __shfl_sync(0xffffffffu, incl, 31);
+        monotone = __all_sync(0xffffffffu, monotone && nonneg) != 0;
+        if (valid == 0) continue;
+
+        float corr[V];
+#pragma unroll
+        for (int j = 0; j < V; ++j) corr[j] = 0.0f;
+#pragma unroll
+        for (int n = 0; n < kNPad; ++n) {
+            if (!((active >> n) & 1u)) continue;   // uniform across the warp
+            float cv[V];
+            load_run<BcT, V>(crow + n * p.seqlen, ts, valid, p.vec_c != 0, cv);
+#pragma unroll
+            for (int j = 0; j < V; ++j) {
+                const float x = a2[n] * (before + S[j]);
+                corr[j] = fmaf(cv[j] * ex2_approx(x), hin[n], corr[j]);
+            }
+        }
+        float o[V];
+        load_run<IoT, V>(orow, ts, valid, p.vec_io != 0, o);
+        float zv[V];
+        if (kHasZ) load_run<IoT, V>(zrow, ts, valid, p.vec_io != 0, zv);
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+            float g = corr[j];
+            if (kHasZ) g *= kExact ? silu_f32(zv[j]) : silu_tanh(zv[j]);
+            o[j] += g;
+        }
+        if (p.vec_io != 0 && valid == V) {
+            if (sizeof(IoT) == 2) {
+                float f8[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) f8[j] = o[j];
+                *reinterpret_cast<uint4*>(orow + ts) = pack16(f8);
+            } else {
+                float f4[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) f4[j] = o[j];
+                *reinterpret_cast<uint4*>(orow + ts) = pack16(f4);
+            }
+        } else {
+            for (int j = 0; j < valid; ++j) DType<IoT>::store(orow + ts + j, o[j]);
+        }
+    }
+}
+
+template <typename IoT, typename BcT, bool kHasZ, bool kSoftplus>
+__global__ void __launch_bounds__(kCorrectWarps * 32)
+    scan_correct_kernel(const __grid_constant__ CorrectParams p) {
+    const int lane = threadIdx.x & 31;
     for (;;) {
         unsigned int item = 0;
         if (lane == 0) item = atomicAdd(p.counter, 1u);
@@ -144,105 +245,11 @@ __global__ void __launch_bounds__(kCorrectWarps * 32)
         if ((int64_t)item >= p.items) break;
         const int64_t chain = item % p.chains;
         const int64_t k = 1 + item / p.chains;
-        const int64_t b = chain / p.dim, d = chain % p.dim;
-        const int64_t t_begin = k * p.seg_len;
-        const int64_t t_end = min(t_begin + p.seg_len, p.seqlen);
-
-        float hin[kNPad], a2[kNPad];
+        float hin[kNPad];
         const float* hs = p.ws_h + ((k - 1) * p.chains + chain) * kNPad;
 #pragma unroll
-        for (int n = 0; n < kNPad; ++n) {
-            const bool in = n < p.dstate;
-            hin[n] = in ? __ldcg(hs + n) : 0.0f;
-            a2[n] = in ? p.A[d * p.dstate + n] * kLog2e : 0.0f;
-        }
-        const float bias = p.delta_bias ? p.delta_bias[d] : 0.0f;
-        const IoT* drow = delta + chain * p.seqlen;
-        const IoT* zrow = kHasZ ? zz + chain * p.seqlen : nullptr;
-        IoT* orow = out + chain * p.seqlen;
-        const BcT* crow = Cm + b * p.dstate * p.seqlen;
-        float S_run = 0.0f;       // sum of Delta before this pass's first step
-        bool monotone = true;     // Delta >= 0 at every step so far
-
-        for (int64_t t0 = t_begin; t0 < t_end; t0 += 32 * V) {
-            // State entries whose exp(A_n S_t) is below 2^-127 for the rest of
-            // the segment (0 after ex2.approx.ftz) drop out; none left, done.
-            uint32_t active = 0;
-#pragma unroll
-            for (int n = 0; n < kNPad; ++n)
-                if (n < p.dstate && !(monotone && a2[n] < 0.0f && a2[n] * S_run < kUnderflowLog2))
-                    active |= 1u << n;
-            if (active == 0) break;
-            const int64_t ts = t0 + (int64_t)lane * V;
-            const int valid = (int)max((int64_t)0, min((int64_t)V, t_end - ts));
-            float dl[V];
-            load_run<IoT, V>(drow, ts, valid, p.vec_io != 0, dl);
-            float S[V];
-            float run = 0.0f;
-            bool nonneg = true;
-#pragma unroll
-            for (int j = 0; j < V; ++j) {
-                float dt = 0.0f;
-                if (j < valid) {
-                    const float sarg = dl[j] + bias;
-                    dt = kSoftplus ? (kExact ? softplus_f32(sarg) : softplus_lg2(sarg)) : sarg;
-                }
-                nonneg = nonneg && dt >= 0.0f;
-                run += dt;
-                S[j] = run;
-            }
-            // exclusive prefix of the lanes' totals, then this pass's total
-            float incl = run;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float v = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += v;
-            }
-            const float before = S_run + (incl - run);
-            S_run += __shfl_sync(0xffffffffu, incl, 31);
-            monotone = __all_sync(0xffffffffu, monotone && nonneg) != 0;
-            if (valid == 0) continue;
-
-            float corr[V];
-#pragma unroll
-            for (int j = 0; j < V; ++j) corr[j] = 0.0f;
-#pragma unroll
-            for (int n = 0; n < kNPad; ++n) {
-                if (!((active >> n) & 1u)) continue;   // uniform across the warp
-                float cv[V];
-                load_run<BcT, V>(crow + n * p.seqlen, ts, valid, p.vec_c != 0, cv);
-#pragma unroll
-                for (int j = 0; j < V; ++j) {
-                    const float x = a2[n] * (before + S[j]);
-                    corr[j] = fmaf(cv[j] * ex2_approx(x), hin[n], corr[j]);
-                }
-            }
-            float o[V];
-            load_run<IoT, V>(orow, ts, valid, p.vec_io != 0, o);
-            float zv[V];
-            if (kHasZ) load_run<IoT, V>(zrow, ts, valid, p.vec_io != 0, zv);
-#pragma unroll
-            for (int j = 0; j < V; ++j) {
-                float g = corr[j];
-                if (kHasZ) g *= kExact ? silu_f32(zv[j]) : silu_tanh(zv[j]);
-                o[j] += g;
-            }
-            if (p.vec_io != 0 && valid == V) {
-                if (sizeof(IoT) == 2) {
-                    float f8[8];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) f8[j] = o[j];
-                    *reinterpret_cast<uint4*>(orow + ts) = pack16(f8);
-                } else {
-                    float f4[4];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) f4[j] = o[j];
-                    *reinterpret_cast<uint4*>(orow + ts) = pack16(f4);
-                }
-            } else {
-                for (int j = 0; j < valid; ++j) DType<IoT>::store(orow + ts + j, o[j]);
-            }
-        }
+        for (int n = 0; n < kNPad; ++n) hin[n] = n < p.dstate ? __ldcg(hs + n) : 0.0f;
+        correct_chain<IoT, BcT, kHasZ, kSoftplus>(p, chain, k, hin, lane);
     }
 }
 

@@ -52,13 +52,13 @@
 #pragma once
 
 #include "ssm_device.cuh"
+#include "scan_carry.cuh"
 
 namespace mamba {
 
 constexpr int kScanWarps = 4;              // warps per CTA (each an independent worker)
 constexpr int kScanStages = 2;             // tiles in flight per warp
 constexpr int kRowBytes = 32;              // bytes of one channel row in a tile
-constexpr int kNPad = 16;                  // compiled state size (smaller N is zero-padded)
 constexpr int kMaxTile = kRowBytes / 2;    // time steps per tile for 2-byte inputs
 constexpr int kBcRawBytes = kNPad * kMaxTile * 4;   // 16 rows of up to 64 bytes
 constexpr int kBcfBytes = kMaxTile * 32 * 4;        // [T][32] fp32
@@ -87,7 +87,7 @@ struct ScanLayout {
 constexpr size_t kWsCounters = 0;          // uint32 [2] dequeue counters
 constexpr size_t kWsFlags = 256;           // uint32 [groups] finished segments per group
 
-enum ScanMode { kModeChained = 0, kModeSegments = 1 };
+enum ScanMode { kModeChained = 0, kModeSegments = 1, kModeLookback = 2 };
 
 struct ScanParams {
     const void* u;
@@ -122,6 +122,8 @@ struct ScanParams {
     int64_t ckpt_tiles;      // ceil(seqlen / kCkptSteps)
     int bld;                 // u, delta, z, out are (batch, seqlen, dim) (the kBld instances)
     int64_t out_step;        // elements between consecutive steps of one channel's output
+    int vec_io;              // look-back mode: 16-byte accesses of delta, z, out rows are aligned
+    int vec_c;               // look-back mode: 16-byte loads of C rows are aligned
 };
 
 
@@ -582,9 +584,108 @@ __device__ __forceinline__ void st_release_gpu(unsigned int* p, unsigned int v) 
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+// Look-back mode (one launch for the parallel mode), segment k >= 1 of group
+// g, one channel per lane: wait (bounded) until segments 0..k-1 of the group
+// have published their end states e_j (each from its own zero start; segment
+// 0 from the given start state, so e_0 is already true) and sums of Delta,
+// fold them into this segment's true start state h_in by the associative
+// combine h_j = exp(A sum Delta_j) h_j-1 + e_j, write last_state for the last
+// segment, and add h_in's contribution to the segment's outputs chain by
+// chain (the correction of scan_carry.cuh, lanes over time).  Returns false
+// after a timeout, which it records.
+template <typename IoT, bool kHasZ, bool kSoftplus>
+__device__ __forceinline__ bool lookback_segment(const ScanParams& p, int lane, int64_t g, int64_t b,
+                                                 int64_t d0, int64_t k, const float2 (&a2)[kNPad / 2],
+                                                 const float2 (&h_own)[kNPad / 2], float sdt_own,
+                                                 bool valid, int64_t chain) {
+    constexpr bool kExact = sizeof(IoT) == 4;
+    bool ok = true;
+    for (int64_t j = lane; j < k; j += 32) {        // lane j polls segment j, j + 32, ...
+        bool got = false;
+        for (uint32_t i = 0; i < p.flag_poll_limit; ++i) {
+            if (ld_acquire_gpu(p.flags + j * p.groups + g) != 0u) {
+                got = true;
+                break;
+            }
+            __nanosleep(1000);
+        }
+        ok = ok && got;
+    }
+    if (!__all_sync(0xffffffffu, ok)) {
+        if (lane == 0) record_device_error(MAMBA_ERR_TIMEOUT);
+        return false;
+    }
+    for (int64_t j = 0; j < k; ++j) (void)ld_acquire_gpu(p.flags + j * p.groups + g);
+
+    float2 hin[kNPad / 2];
+#pragma unroll
+    for (int pi = 0; pi < kNPad / 2; ++pi) hin[pi] = make_float2(0.0f, 0.0f);
+    if (valid) {
+        for (int64_t j = 0; j < k; ++j) {
+            float2 e[kNPad / 2];
+            load16(p.ws_h + (j * p.chains + chain) * kNPad, e);
+            if (j == 0) {
+#pragma unroll
+                for (int pi = 0; pi < kNPad / 2; ++pi) hin[pi] = e[pi];
+            } else {
+                const float s = __ldcg(p.ws_sdt + j * p.chains + chain);
+#pragma unroll
+                for (int pi = 0; pi < kNPad / 2; ++pi) {
+                    const float2 P = exp2_pair<kExact>(__fmul2_rn(make_float2(s, s), a2[pi]));
+                    hin[pi] = __ffma2_rn(P, hin[pi], e[pi]);
+                }
+            }
+        }
+        if (k == p.nseg - 1 && p.last_state != nullptr) {   // the chain's last state
+            float* ls = p.last_state + chain * p.dstate;
+#pragma unroll
+            for (int pi = 0; pi < kNPad / 2; ++pi) {
+                const float2 P = exp2_pair<kExact>(__fmul2_rn(make_float2(sdt_own, sdt_own), a2[pi]));
+                const float2 v = __ffma2_rn(P, hin[pi], h_own[pi]);
+                if (2 * pi < p.dstate) ls[2 * pi] = v.x;
+                if (2 * pi + 1 < p.dstate) ls[2 * pi + 1] = v.y;
+            }
+        }
+    }
+    __syncwarp();   // this warp's outputs of the segment are written
+
+    CorrectParams cp{};
+    cp.delta = p.delta;
+    cp.z = p.z;
+    cp.C = p.C;
+    cp.A = p.A;
+    cp.delta_bias = p.delta_bias;
+    cp.out = p.out;
+    cp.batch = p.batch;
+    cp.dim = p.dim;
+    cp.seqlen = p.seqlen;
+    cp.chains = p.chains;
+    cp.seg_len = p.seg_len;
+    cp.nseg = p.nseg;
+    cp.dstate = p.dstate;
+    cp.bc_bf16 = p.bc_bf16;
+    cp.vec_io = p.vec_io;
+    cp.vec_c = p.vec_c;
+    for (int c = 0; c < 32; ++c) {                  // lanes over time for each chain
+        const int64_t d = d0 + c;
+        if (d >= p.dim) break;
+        float h16[kNPad];
+#pragma unroll
+        for (int pi = 0; pi < kNPad / 2; ++pi) {
+            h16[2 * pi] = __shfl_sync(0xffffffffu, hin[pi].x, c);
+            h16[2 * pi + 1] = __shfl_sync(0xffffffffu, hin[pi].y, c);
+        }
+        if (p.bc_bf16)
+            correct_chain<IoT, __nv_bfloat16, kHasZ, kSoftplus>(cp, b * p.dim + d, k, h16, lane);
+        else
+            correct_chain<IoT, float, kHasZ, kSoftplus>(cp, b * p.dim + d, k, h16, lane);
+    }
+    return true;
+}
+
 // kZoh keeps 1 / A in 16 more registers per channel, so its instances are
 // compiled for one CTA per SM fewer.
-template <typename IoT, int kCpl, bool kHasZ, bool kSoftplus, bool kZoh, bool kBld>
+template <typename IoT, int kCpl, bool kHasZ, bool kSoftplus, bool kZoh, bool kBld, bool kLookback>
 __global__ void __launch_bounds__(kScanWarps * 32, ScanLayout<kCpl>::kMinBlocks - (kZoh ? 1 : 0))
     selective_scan_fwd_kernel(const __grid_constant__ ScanParams p,
                               const __grid_constant__ CUtensorMap tm_u,
@@ -689,7 +790,10 @@ __global__ void __launch_bounds__(kScanWarps * 32, ScanLayout<kCpl>::kMinBlocks 
             sdt[c] = 0.0f;
         }
         bool ok;
-        if constexpr (kBld) {            // chained mode only, with outputs
+        if constexpr (kLookback) {       // segments from their own start, then the look-back
+            ok = run_segment<IoT, kCpl, kHasZ, kSoftplus, kZoh, true, false, true, false>(
+                p, maps, wsm, lane, b, d0, t_begin, t_end, lc, out_row, seq, sdt, ckpt_row);
+        } else if constexpr (kBld) {     // chained mode only, with outputs
             ok = run_segment<IoT, kCpl, kHasZ, kSoftplus, kZoh, true, false, false, true>(
                 p, maps, wsm, lane, b, d0, t_begin, t_end, lc, out_row, seq, sdt, ckpt_row);
         } else if (p.ckpt != nullptr) {  // checkpoint pass of the backward: states only
@@ -722,6 +826,16 @@ __global__ void __launch_bounds__(kScanWarps * 32, ScanLayout<kCpl>::kMinBlocks 
                 store16(p.ws_h + (k * p.chains + chain[c]) * kNPad, lc.h[c]);
                 __stcg(p.ws_sdt + k * p.chains + chain[c], sdt[c]);
             }
+        }
+        if constexpr (kLookback) {
+            static_assert(kCpl == 1, "the look-back mode runs one channel per lane");
+            // publish this segment's end state and sum of Delta (stored above)
+            __threadfence();
+            __syncwarp();
+            if (lane == 0 && !p.withhold_handoff) st_release_gpu(p.flags + k * p.groups + g, 1u);
+            if (k > 0 && !lookback_segment<IoT, kHasZ, kSoftplus>(p, lane, g, b, d0, k, lc.a2[0], lc.h[0],
+                                                                  sdt[0], valid[0], chain[0]))
+                break;
         }
         if (last_seg && p.mode == kModeChained && p.last_state != nullptr) {
 #pragma unroll

@@ -17,6 +17,7 @@ namespace mamba {
 
 constexpr float kLog2e = 1.4426950408889634f;   // log2(e)
 constexpr float kLn2 = 0.6931471805599453f;     // ln(2)
+constexpr int kNPad = 16;                        // compiled state size (smaller N is zero-padded)
 
 // First device-side error since the host last read it (0 = none).  The
 // library is compiled as one translation unit, which owns this definition.

@@ -31,6 +31,7 @@ MAMBA_FLAG_ZOH = 0x8
 MAMBA_FLAG_PDL = 0x10
 MAMBA_FLAG_LAYOUT_BLD = 0x20
 MAMBA_FLAG_ONE_LANE_PER_CHANNEL = 0x40
+MAMBA_FLAG_PARALLEL_ONE_LAUNCH = 0x80
 
 _DTYPE_CODE = {torch.float32: MAMBA_F32, torch.bfloat16: MAMBA_BF16}
 

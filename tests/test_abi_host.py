@@ -222,9 +222,19 @@ def test_plan_two_lanes_per_channel_rules(lib):
 def test_plan_parallel_for_the_million_token_sequence(lib):
     # few channel groups: every segment runs at once from its own start (one
     # segment per resident warp), then the carry scan and the correction pass
+    # (mode 1), or each segment looks back at the earlier ones and corrects
+    # itself in the same launch (mode 2)
     c = SCAN_CONFIGS["long_dna_1m"]
     p = ops.scan_plan(c.batch, c.dim, c.dstate, c.seqlen, c.io_dtype, c.bc_dtype, sm_count=148)
+    p2 = ops.scan_plan(c.batch, c.dim, c.dstate, c.seqlen, c.io_dtype, c.bc_dtype, sm_count=148,
+                       flags=ops.MAMBA_FLAG_PARALLEL_ONE_LAUNCH)
     K = p["nchunks"]
+    assert p2["mode"] == 2 and p2["launches"] == 1 and p2["nchunks"] == K
+    assert p2["units_pass_a"] == p["units_pass_a"] and p2["units_pass_b"] == p["units_pass_b"]
+    chains = c.batch * c.dim
+    flags2 = (K * p["groups"] * 4 + 255) // 256 * 256
+    assert p2["workspace_bytes"] == 256 + flags2 + (K * chains * 64 + 255) // 256 * 256 + \
+        (K * chains * 4 + 255) // 256 * 256
     assert p["mode"] == 1 and p["launches"] == 3 and p["channels_per_lane"] == 1
     assert p["groups"] == 1536 // 32
     assert K == (148 * 16) // p["groups"]                 # one segment per resident warp
@@ -260,6 +270,9 @@ def test_plan_forced_chunk_counts(lib, L, K, want_k, want_len):
     q = ops.scan_plan(1, 32, 16, L, torch.bfloat16, torch.bfloat16, num_chunks=K,
                       flags=ops.MAMBA_FLAG_PARALLEL_CHUNKS)
     assert q["nchunks"] == want_k and q["mode"] == (1 if want_k > 1 else 0)
+    q = ops.scan_plan(1, 32, 16, L, torch.bfloat16, torch.bfloat16, num_chunks=K,
+                      flags=ops.MAMBA_FLAG_PARALLEL_CHUNKS | ops.MAMBA_FLAG_PARALLEL_ONE_LAUNCH)
+    assert q["nchunks"] == want_k and q["mode"] == (2 if want_k > 1 else 0)
 
 
 def test_plan_tma_capability_follows_strides(lib):

@@ -130,7 +130,7 @@ def test_few_channels_long_sequence_runs_chained(ref):
     (batch, seqlen, dim) call stays chained and matches the oracle."""
     x = layer_inputs(1, 64, 16384, seed=9)
     plan = ops.scan_plan(1, 64, 16, 16384, flags=ops.MAMBA_FLAG_LAYOUT_BLD)
-    assert plan["mode"] == 0 and ops.scan_plan(1, 64, 16, 16384)["mode"] == 1
+    assert plan["mode"] == 0 and ops.scan_plan(1, 64, 16, 16384)["mode"] != 0
     out, last = scan(x, "bld")
     o_out, o_last = oracle_scan(ref, x)
     assert max_rel_err(out, o_out) <= tol_for(torch.bfloat16)

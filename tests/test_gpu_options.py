@@ -15,6 +15,7 @@ pytestmark = pytest.mark.gpu
 
 DEV = "cuda"
 PAR = ops.MAMBA_FLAG_PARALLEL_CHUNKS
+PAR1 = ops.MAMBA_FLAG_PARALLEL_CHUNKS | ops.MAMBA_FLAG_PARALLEL_ONE_LAUNCH
 
 
 @pytest.fixture(scope="module")
@@ -76,7 +77,7 @@ def test_zoh_layer_recipe(ref, dtype, shape):
     compare(ref, x, tol_for(dtype), zoh=True)
 
 
-@pytest.mark.parametrize("flags", [0, PAR], ids=["chained", "parallel"])
+@pytest.mark.parametrize("flags", [0, PAR, PAR1], ids=["chained", "parallel", "parallel1"])
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 def test_zoh_segments_long_memory(ref, dtype, flags):
     x = layer_inputs(1, 64, 4096, dtype=dtype, seed=7)
@@ -136,8 +137,8 @@ def test_zoh_fixed_point_from_start_state():
 
 # ------------------------------------------------------------ start state
 
-@pytest.mark.parametrize("K,flags", [(0, 0), (1, 0), (3, 0), (3, PAR)],
-                         ids=["auto", "one_segment", "chained3", "parallel3"])
+@pytest.mark.parametrize("K,flags", [(0, 0), (1, 0), (3, 0), (3, PAR), (3, PAR1)],
+                         ids=["auto", "one_segment", "chained3", "parallel3", "parallel3_one_launch"])
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 def test_start_state(ref, dtype, K, flags):
     x = layer_inputs(2, 80, 1536, dtype=dtype, seed=31)

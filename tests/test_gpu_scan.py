@@ -107,10 +107,13 @@ def test_long_dna_config_full_size_sampled(ref):
 
 # ------------------------------------------------------------ segment carry
 
-PAR = ops.MAMBA_FLAG_PARALLEL_CHUNKS
+PAR = ops.MAMBA_FLAG_PARALLEL_CHUNKS                                 # three launches
+PAR1 = ops.MAMBA_FLAG_PARALLEL_CHUNKS | ops.MAMBA_FLAG_PARALLEL_ONE_LAUNCH   # one launch, look-back
+MODES = pytest.mark.parametrize("flags", [0, PAR, PAR1], ids=["chained", "parallel", "parallel1"])
+PMODES = pytest.mark.parametrize("flags", [PAR, PAR1], ids=["parallel", "parallel1"])
 
 
-@pytest.mark.parametrize("flags", [0, PAR], ids=["chained", "parallel"])
+@MODES
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 @pytest.mark.parametrize("K", [2, 3, 8])
 def test_segments_long_memory(ref, dtype, K, flags):
@@ -122,7 +125,7 @@ def test_segments_long_memory(ref, dtype, K, flags):
     assert max_rel_err(out, ref_out) <= tol_for(dtype)
 
 
-@pytest.mark.parametrize("flags", [0, PAR], ids=["chained", "parallel"])
+@MODES
 @pytest.mark.parametrize("L,K", [(100, 5), (1000, 3), (333, 4), (4096 + 40, 7)])
 def test_segments_ragged(ref, L, K, flags):
     x = layer_inputs(2, 40, L, seed=L)
@@ -138,15 +141,17 @@ def test_chained_segments_are_bitwise_single_pass():
         assert torch.equal(a, b) and torch.equal(la, lb)
 
 
-def test_parallel_matches_single_pass_closely(ref):
+@PMODES
+def test_parallel_matches_single_pass_closely(ref, flags):
     x = layer_inputs(1, 32, 8192, dtype=torch.float32, seed=5)
     a, la = run_gpu(x, num_chunks=1)
-    b, lb = run_gpu(x, num_chunks=16, flags=PAR)
+    b, lb = run_gpu(x, num_chunks=16, flags=flags)
     assert max_rel_err(b, a) <= 1e-5 and max_rel_err(lb, la) <= 1e-5
 
 
+@PMODES
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-def test_parallel_correction_without_early_stop(ref, dtype):
+def test_parallel_correction_without_early_stop(ref, dtype, flags):
     """The parallel mode's correction walks a segment only while some
     exp(A_n S_t) is above fp32's range; with a state entry at A = 0 it never
     decays, so every segment is corrected to its end."""
@@ -154,27 +159,53 @@ def test_parallel_correction_without_early_stop(ref, dtype):
     A = x["A"].clone()
     A[:, 3] = 0.0
     x["A"] = A
-    check(ref, x, tol_for(dtype), num_chunks=5, flags=PAR)
+    check(ref, x, tol_for(dtype), num_chunks=5, flags=flags)
 
 
-def test_parallel_correction_with_negative_delta(ref):
+@PMODES
+def test_parallel_correction_with_negative_delta(ref, flags):
     """Softplus off with delta + bias of both signs: the running sum of Delta
     is not monotone, so the correction may not stop early."""
     x = layer_inputs(1, 64, 2048, dtype=torch.float32, seed=44)
     x["delta"] = (x["delta"] * 0.02).contiguous()
     x["delta_bias"] = torch.full_like(x["delta_bias"], 0.005)
-    check(ref, x, FP32_TOL, softplus=False, num_chunks=6, flags=PAR)
+    check(ref, x, FP32_TOL, softplus=False, num_chunks=6, flags=flags)
 
 
 def test_many_groups_many_segments(ref):
     """More work items than resident warps, in both modes."""
     x = layer_inputs(4, 2048, 1024, seed=31)
     out, last = run_gpu(x, num_chunks=4)
-    for flags in (0, PAR):
+    for flags in (0, PAR, PAR1):
         o2, l2 = run_gpu(x, num_chunks=4, flags=flags)
         assert max_rel_err(o2, out.double()) <= BF16_TOL
     sampled = I.SCAN_CONFIGS["mamba_1p4b_layer"].resized(batch=4, dim=2048, seqlen=1024)
     sampled_check(ref, sampled, x, out, last, 16, BF16_TOL)
+
+
+def test_one_and_three_launch_parallel_modes_agree():
+    """The look-back folds the earlier segments' states one after another, the
+    three-launch form by a warp-shuffle scan: the same sums in another order."""
+    x = layer_inputs(3, 96, 6000, seed=45)
+    plan = ops.scan_plan(3, 96, 16, 6000, num_chunks=12, flags=PAR1,
+                         sm_count=torch.cuda.get_device_properties(0).multi_processor_count)
+    assert plan["mode"] == 2 and plan["launches"] == 1
+    a, la = run_gpu(x, num_chunks=12, flags=PAR1)
+    b, lb = run_gpu(x, num_chunks=12, flags=PAR)
+    assert max_rel_err(a, b) <= BF16_TOL and max_rel_err(la, lb) <= 1e-5
+
+
+def test_lookback_wait_reports_timeout():
+    """Segments that never publish: every look-back gives up (bounded), the
+    status word says MAMBA_ERR_TIMEOUT, and a normal call afterwards is fine."""
+    x = layer_inputs(1, 64, 1024, seed=34)
+    ops.selective_scan_fwd(x["u"], x["delta"], x["A"], x["B"], x["C"], num_chunks=4,
+                           flags=PAR1 | ops.MAMBA_FLAG_TEST_WITHHOLD_HANDOFF)
+    torch.cuda.synchronize()
+    assert ops.device_status() == -6
+    assert ops.device_status() == 0
+    out, last = run_gpu(x, num_chunks=4, flags=PAR1)
+    assert torch.isfinite(out.float()).all()
 
 
 # ------------------------------------------------------------ edge cases
