@@ -107,15 +107,17 @@ typedef enum {
  * different layers; then results are identical with and without the flag.
  * Paths other than the streaming one ignore it. */
 #define MAMBA_FLAG_PDL 0x10
-/* Scan forward only (mamba_selective_scan_fwd, _with_state, _noalloc and the
- * host-buffer call): u, delta, z and out are (batch, seqlen, dim), dim fastest,
+/* Scan forward (mamba_selective_scan_fwd, _with_state, _noalloc and the
+ * host-buffer call) and backward: u, delta, z and out (dout and the
+ * gradients du, ddelta, dz) are (batch, seqlen, dim), dim fastest,
  * the activation layout of the sample module in "超越注意力：探索Mamba与状态空间
  * 模型", section 代码实现概览; B and C stay (batch, dstate, seqlen) and the
  * states (batch, dim, dstate).  Tiles of (steps x 32 channels) are staged by
  * TMA (dim * element size a multiple of 16 bytes, 16-byte aligned pointers;
  * otherwise plain loads) and transposed on chip; outputs are stored one step
  * at a time.  Such calls always run in mode 0: MAMBA_FLAG_PARALLEL_CHUNKS with
- * it returns MAMBA_ERR_UNSUPPORTED, and so does the backward. */
+ * it returns MAMBA_ERR_UNSUPPORTED.  The backward stages (8 steps x 32
+ * channels) tiles by cp.async and stores its gradients one step at a time. */
 #define MAMBA_FLAG_LAYOUT_BLD 0x20
 /* Scan forward: keep one lane per channel where the plan would give each
  * channel two lanes (plan.lanes_per_channel; see mamba_scan_plan_t).  For
@@ -389,9 +391,9 @@ MAMBA_API mamba_status_t mamba_selective_state_update(float *state, const void *
  * Gradients of a scalar loss, given dout = dLoss/dout (and optionally
  * dlast_state = dLoss/dlast_state), with respect to every input of
  * mamba_selective_scan_fwd_with_state, with the Euler input term or, with
- * MAMBA_FLAG_ZOH in dims->flags, the zero-order-hold one (inputs in the
- * (batch, dim, seqlen) layout: MAMBA_FLAG_LAYOUT_BLD returns
- * MAMBA_ERR_UNSUPPORTED).  As in the pages'
+ * MAMBA_FLAG_ZOH in dims->flags, the zero-order-hold one (with
+ * MAMBA_FLAG_LAYOUT_BLD, u, delta, z, dout and du, ddelta, dz are
+ * (batch, seqlen, dim)).  As in the pages'
  * description of the hardware-aware scan ("Mamba 与状态空间模型", section
  * 在芯片上扫过去), the per-step states are not stored by the forward: a
  * checkpoint pass keeps the state every 8 steps in the workspace, and the

@@ -499,7 +499,6 @@ mamba_status_t scan_fwd_internal(const void* u, const void* delta, const float* 
     mamba_status_t st = check_dims(dims, true);
     if (st != MAMBA_OK) return st;
     const bool bld = (dims->flags & MAMBA_FLAG_LAYOUT_BLD) != 0;
-    if (bld && ckpt != nullptr) return MAMBA_ERR_UNSUPPORTED;
     // Empty problems first: tensors without elements may have null pointers.
     const int64_t chains = dims->batch * dims->dim;
     if (chains == 0) return MAMBA_OK;
@@ -1275,11 +1274,11 @@ mamba_status_t bwd_layout(const mamba_dims_t* dims, int sms, BwdWorkspace* w) {
     return MAMBA_OK;
 }
 
-template <typename IoT, typename BcT, bool kHasZ, bool kZoh>
+template <typename IoT, typename BcT, bool kHasZ, bool kZoh, bool kBld>
 cudaError_t launch_bwd(const BwdParams& prm, int dev, int sms, cudaStream_t stream) {
     static bool attr_done[kMaxDevices] = {false};
     static int resident[kMaxDevices] = {0};
-    auto kernel = selective_scan_bwd_kernel<IoT, BcT, kHasZ, kZoh>;
+    auto kernel = selective_scan_bwd_kernel<IoT, BcT, kHasZ, kZoh, kBld>;
     constexpr int smem = kBwdWarps * bwd_warp_smem<IoT, BcT>();
     cudaError_t e = ensure_smem_attr(kernel, smem, attr_done, dev);
     if (e != cudaSuccess) return e;
@@ -1297,20 +1296,24 @@ cudaError_t launch_bwd(const BwdParams& prm, int dev, int sms, cudaStream_t stre
     return cudaGetLastError();
 }
 
-template <typename IoT, bool kZoh>
+template <typename IoT, bool kZoh, bool kBld>
 cudaError_t dispatch_bwd_zoh(const BwdParams& prm, bool has_z, int dev, int sms, cudaStream_t stream) {
     if (prm.bc_bf16)
-        return has_z ? launch_bwd<IoT, __nv_bfloat16, true, kZoh>(prm, dev, sms, stream)
-                     : launch_bwd<IoT, __nv_bfloat16, false, kZoh>(prm, dev, sms, stream);
-    return has_z ? launch_bwd<IoT, float, true, kZoh>(prm, dev, sms, stream)
-                 : launch_bwd<IoT, float, false, kZoh>(prm, dev, sms, stream);
+        return has_z ? launch_bwd<IoT, __nv_bfloat16, true, kZoh, kBld>(prm, dev, sms, stream)
+                     : launch_bwd<IoT, __nv_bfloat16, false, kZoh, kBld>(prm, dev, sms, stream);
+    return has_z ? launch_bwd<IoT, float, true, kZoh, kBld>(prm, dev, sms, stream)
+                 : launch_bwd<IoT, float, false, kZoh, kBld>(prm, dev, sms, stream);
 }
 
+// Kernel instance for (zero-order hold, activation layout).
 template <typename IoT>
-cudaError_t dispatch_bwd(const BwdParams& prm, bool has_z, bool zoh, int dev, int sms,
+cudaError_t dispatch_bwd(const BwdParams& prm, bool has_z, bool zoh, bool bld, int dev, int sms,
                          cudaStream_t stream) {
-    return zoh ? dispatch_bwd_zoh<IoT, true>(prm, has_z, dev, sms, stream)
-               : dispatch_bwd_zoh<IoT, false>(prm, has_z, dev, sms, stream);
+    if (bld)
+        return zoh ? dispatch_bwd_zoh<IoT, true, true>(prm, has_z, dev, sms, stream)
+                   : dispatch_bwd_zoh<IoT, false, true>(prm, has_z, dev, sms, stream);
+    return zoh ? dispatch_bwd_zoh<IoT, true, false>(prm, has_z, dev, sms, stream)
+               : dispatch_bwd_zoh<IoT, false, false>(prm, has_z, dev, sms, stream);
 }
 
 cudaError_t zero_async(void* p, size_t bytes, cudaStream_t stream) {
@@ -1450,7 +1453,7 @@ MAMBA_API mamba_status_t mamba_selective_scan_bwd(
     float* dinitial_state, const mamba_dims_t* dims, cudaStream_t stream) {
     mamba_status_t st = check_dims(dims, true);
     if (st != MAMBA_OK) return st;
-    if (dims->flags & MAMBA_FLAG_LAYOUT_BLD) return MAMBA_ERR_UNSUPPORTED;
+    const bool bld = (dims->flags & MAMBA_FLAG_LAYOUT_BLD) != 0;
     const int64_t chains = dims->batch * dims->dim;
     if (chains == 0) return MAMBA_OK;
     const int64_t L = dims->seqlen, N = dims->dstate;
@@ -1501,7 +1504,8 @@ MAMBA_API mamba_status_t mamba_selective_scan_bwd(
     // 1. checkpoint pass: the forward, chained in w.K segments, states only
     mamba_dims_t fd = *dims;
     fd.num_chunks = (int32_t)w.K;
-    fd.flags = (dims->flags & (MAMBA_FLAG_NO_TMA | MAMBA_FLAG_ZOH)) | MAMBA_FLAG_ONE_LANE_PER_CHANNEL;
+    fd.flags = (dims->flags & (MAMBA_FLAG_NO_TMA | MAMBA_FLAG_ZOH | MAMBA_FLAG_LAYOUT_BLD)) |
+               MAMBA_FLAG_ONE_LANE_PER_CHANNEL;
     fd.workspace = ws;
     fd.workspace_bytes = w.fwd_bytes;
     float* ckpt = reinterpret_cast<float*>(ws + w.ckpt);
@@ -1551,13 +1555,14 @@ MAMBA_API mamba_status_t mamba_selective_scan_bwd(
     for (const void* q : io_ptrs)
         if (q && !aligned(q, 16)) vec = false;
     prm.vec_ok = vec ? 1 : 0;
+    prm.bld = bld ? 1 : 0;
     prm.bc_vec = ((L * bc_es) % 16 == 0 && aligned(B, 16) && aligned(C, 16)) ? 1 : 0;
     prm.flag_poll_limit =
         (unsigned int)std::min<int64_t>(std::max<int64_t>(w.seg_len * 256, 1 << 20), (int64_t)1 << 31);
     const bool zoh = (dims->flags & MAMBA_FLAG_ZOH) != 0;
     e = dims->io_dtype == MAMBA_BF16
-            ? dispatch_bwd<__nv_bfloat16>(prm, z != nullptr, zoh, dev, sms, stream)
-            : dispatch_bwd<float>(prm, z != nullptr, zoh, dev, sms, stream);
+            ? dispatch_bwd<__nv_bfloat16>(prm, z != nullptr, zoh, bld, dev, sms, stream)
+            : dispatch_bwd<float>(prm, z != nullptr, zoh, bld, dev, sms, stream);
     return e == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
 }
 

@@ -85,6 +85,7 @@ struct BwdParams {
     int softplus;
     int bc_bf16;
     int vec_ok;                // u, delta, z, dout, du, ddelta, dz all 16-byte aligned
+    int bld;                   // those are (batch, seqlen, dim) (the kBld instances)
     int bc_vec;                // B and C rows 16-byte aligned
     unsigned int flag_poll_limit;
 };
@@ -126,6 +127,23 @@ __device__ __forceinline__ void store_block(T* row, int64_t t0, int n, bool vec,
 #pragma unroll
     for (int i = 0; i < kBwdSteps; ++i)
         if (i < n) DType<T>::store(row + t0 + i, v[i]);
+}
+
+// kBwdSteps elements of one channel of a (batch, seqlen, dim) tensor, `step`
+// elements apart (zero past `n`), and the matching stores.
+template <typename T>
+__device__ __forceinline__ void load_block_strided(const T* row, int64_t t0, int n, int64_t step,
+                                                   float (&v)[kBwdSteps]) {
+#pragma unroll
+    for (int i = 0; i < kBwdSteps; ++i) v[i] = i < n ? DType<T>::load(row + (t0 + i) * step) : 0.0f;
+}
+
+template <typename T>
+__device__ __forceinline__ void store_block_strided(T* row, int64_t t0, int n, int64_t step,
+                                                    const float (&v)[kBwdSteps]) {
+#pragma unroll
+    for (int i = 0; i < kBwdSteps; ++i)
+        if (i < n) DType<T>::store(row + (t0 + i) * step, v[i]);
 }
 
 // 16-byte asynchronous copy global -> shared (L2 only), and its groups.
@@ -185,6 +203,16 @@ __device__ __forceinline__ void unpack_rows(const uint4 (&r)[kVecs], float (&v)[
     }
 }
 
+// Column `lane` of a staged (8 steps x 32 channels) tile of a (batch,
+// seqlen, dim) tensor: this lane's channel over the block's steps.
+template <typename T, int kVecs>
+__device__ __forceinline__ void unpack_col(const uint4 (&tile)[32][kVecs], int lane,
+                                           float (&v)[kBwdSteps]) {
+    const T* t = reinterpret_cast<const T*>(&tile[0][0]);
+#pragma unroll
+    for (int i = 0; i < kBwdSteps; ++i) v[i] = DType<T>::load(t + i * 32 + lane);
+}
+
 __device__ __forceinline__ float sigmoid_f32(float x) {
     return __fdividef(1.0f, 1.0f + ex2_approx(-x * kLog2e));
 }
@@ -216,7 +244,7 @@ __device__ __forceinline__ float2 zoh_dgda_series2(float2 x2) {
     return r;
 }
 
-template <typename IoT, typename BcT, bool kHasZ, bool kZoh>
+template <typename IoT, typename BcT, bool kHasZ, bool kZoh, bool kBld>
 __global__ void __launch_bounds__(kBwdWarps * 32)
     selective_scan_bwd_kernel(const __grid_constant__ BwdParams p) {
     constexpr bool kExact = sizeof(IoT) == 4;
@@ -314,24 +342,50 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
         }
         float dD_acc = 0.0f, dbias_acc = 0.0f;
 
-        const IoT* urow = static_cast<const IoT*>(p.u) + chain * p.seqlen;
-        const IoT* drow = static_cast<const IoT*>(p.delta) + chain * p.seqlen;
-        const IoT* zrow = kHasZ ? static_cast<const IoT*>(p.z) + chain * p.seqlen : nullptr;
-        const IoT* grow = static_cast<const IoT*>(p.dout) + chain * p.seqlen;
-        const bool vec = p.vec_ok && (p.seqlen * (int64_t)sizeof(IoT)) % 16 == 0 && valid;
+        // This lane's channel of u, delta, z, dout and the gradients: step t at
+        // row[t] ((batch, dim, seqlen)), or at row[t * dim] ((batch, seqlen, dim)).
+        const int64_t io_base = kBld ? b * p.seqlen * p.dim + (valid ? d : 0) : chain * p.seqlen;
+        const int64_t io_step = kBld ? p.dim : 1;
+        const IoT* urow = static_cast<const IoT*>(p.u) + io_base;
+        const IoT* drow = static_cast<const IoT*>(p.delta) + io_base;
+        const IoT* zrow = kHasZ ? static_cast<const IoT*>(p.z) + io_base : nullptr;
+        const IoT* grow = static_cast<const IoT*>(p.dout) + io_base;
+        const bool vec = !kBld && p.vec_ok && (p.seqlen * (int64_t)sizeof(IoT)) % 16 == 0 && valid;
         const int nblk = (int)((t_end - t_begin + kBwdSteps - 1) / kBwdSteps);
         const int nbc = lane & 15;
         const BcT* bcrow = static_cast<const BcT*>(lane < 16 ? p.B : p.C) +
                            (b * p.dstate + (nbc < p.dstate ? nbc : 0)) * p.seqlen;
         // Blocks are staged one ahead by cp.async when every row is 16-byte
-        // aligned; a block shorter than 8 steps (the sequence's last) is read
-        // directly.
-        const bool pipe = p.vec_ok && p.bc_vec && (p.seqlen * (int64_t)sizeof(IoT)) % 16 == 0;
+        // aligned (with (batch, seqlen, dim): a row of channels, and the
+        // group's 32 channels all present); a block shorter than 8 steps (the
+        // sequence's last) is read directly.
+        const bool pipe = p.vec_ok && p.bc_vec &&
+                          (kBld ? (p.dim * (int64_t)sizeof(IoT)) % 16 == 0 && d0 + 32 <= p.dim
+                                : (p.seqlen * (int64_t)sizeof(IoT)) % 16 == 0);
         auto issue = [&](int jj) {
             const int64_t tt = t_begin + (int64_t)jj * kBwdSteps;
             if (pipe && t_end - tt >= kBwdSteps) {
                 Stage& S = stages[jj & 1];
-                if (valid) {
+                if constexpr (kBld) {
+                    // each tensor's (8 steps x 32 channels) tile, row r = step:
+                    // lane l copies the 16-byte chunk(s) (l & 3) of row l >> 2
+                    constexpr int kChunks = (int)sizeof(IoT) / 2;   // 1 (bf16) or 2 (fp32)
+                    const int r = lane >> 2;
+                    const int64_t roff = (b * p.seqlen + tt + r) * p.dim + d0;
+#pragma unroll
+                    for (int v = 0; v < kChunks; ++v) {
+                        const int ci = (lane & 3) * kChunks + v;
+                        const int64_t src = roff + ci * (16 / (int)sizeof(IoT));
+                        const int dst = r * 32 * (int)sizeof(IoT) + ci * 16;
+                        cp_async16(reinterpret_cast<uint8_t*>(&S.io[0][0][0]) + dst, static_cast<const IoT*>(p.u) + src);
+                        cp_async16(reinterpret_cast<uint8_t*>(&S.io[1][0][0]) + dst, static_cast<const IoT*>(p.delta) + src);
+                        if (kHasZ) cp_async16(reinterpret_cast<uint8_t*>(&S.io[2][0][0]) + dst, static_cast<const IoT*>(p.z) + src);
+                        cp_async16(reinterpret_cast<uint8_t*>(&S.io[3][0][0]) + dst, static_cast<const IoT*>(p.dout) + src);
+                    }
+                    const float* ckq = p.ckpt + (chain * p.ckpt_tiles + tt / kBwdSteps) * kNPad;
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) cp_async16(&S.ck[lane][v], ckq + 4 * v);
+                } else if (valid) {
 #pragma unroll
                     for (int v = 0; v < kIoVecs; ++v) {
                         cp_async16(&S.io[0][lane][v], urow + tt + v * (16 / (int)sizeof(IoT)));
@@ -362,6 +416,9 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
             } else {
                 cp_async_wait<0>();
             }
+            // A lane reads a column of a (batch, seqlen, dim) tile whose rows
+            // other lanes copied: their copies must have landed.
+            if constexpr (kBld) __syncwarp();
             const bool staged = pipe && ns == kBwdSteps;
             const Stage& S = stages[j & 1];
             const float4* ck4 = reinterpret_cast<const float4*>(
@@ -370,15 +427,29 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
             // Steps past the end of a short block read as zero.
             float uu[kBwdSteps], dt[kBwdSteps], dy[kBwdSteps], aux[kBwdSteps];
             if (valid && staged) {
-                unpack_rows<kIoVecs>(S.io[0][lane], uu);
-                unpack_rows<kIoVecs>(S.io[1][lane], dt);   // delta, turned into Delta below
-                unpack_rows<kIoVecs>(S.io[3][lane], dy);   // dout, turned into dy below
-                if (kHasZ) unpack_rows<kIoVecs>(S.io[2][lane], aux);
+                if constexpr (kBld) {
+                    unpack_col<IoT, kIoVecs>(S.io[0], lane, uu);
+                    unpack_col<IoT, kIoVecs>(S.io[1], lane, dt);
+                    unpack_col<IoT, kIoVecs>(S.io[3], lane, dy);
+                    if (kHasZ) unpack_col<IoT, kIoVecs>(S.io[2], lane, aux);
+                } else {
+                    unpack_rows<kIoVecs>(S.io[0][lane], uu);
+                    unpack_rows<kIoVecs>(S.io[1][lane], dt);   // delta, turned into Delta below
+                    unpack_rows<kIoVecs>(S.io[3][lane], dy);   // dout, turned into dy below
+                    if (kHasZ) unpack_rows<kIoVecs>(S.io[2][lane], aux);
+                }
             } else if (valid) {
-                load_block(urow, t0, ns, vec, uu);
-                load_block(drow, t0, ns, vec, dt);
-                load_block(grow, t0, ns, vec, dy);
-                if (kHasZ) load_block(zrow, t0, ns, vec, aux);
+                if constexpr (kBld) {
+                    load_block_strided(urow, t0, ns, io_step, uu);
+                    load_block_strided(drow, t0, ns, io_step, dt);
+                    load_block_strided(grow, t0, ns, io_step, dy);
+                    if (kHasZ) load_block_strided(zrow, t0, ns, io_step, aux);
+                } else {
+                    load_block(urow, t0, ns, vec, uu);
+                    load_block(drow, t0, ns, vec, dt);
+                    load_block(grow, t0, ns, vec, dy);
+                    if (kHasZ) load_block(zrow, t0, ns, vec, aux);
+                }
             } else {
 #pragma unroll
                 for (int i = 0; i < kBwdSteps; ++i) uu[i] = dt[i] = dy[i] = aux[i] = 0.0f;
@@ -559,9 +630,11 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
             float sp[kBwdSteps];
             if (p.softplus) {
                 if (valid && staged) {
-                    unpack_rows<kIoVecs>(S.io[1][lane], sp);
+                    if constexpr (kBld) unpack_col<IoT, kIoVecs>(S.io[1], lane, sp);
+                    else unpack_rows<kIoVecs>(S.io[1][lane], sp);
                 } else if (valid) {
-                    load_block(drow, t0, ns, vec, sp);
+                    if constexpr (kBld) load_block_strided(drow, t0, ns, io_step, sp);
+                    else load_block(drow, t0, ns, vec, sp);
                 } else {
 #pragma unroll
                     for (int i = 0; i < kBwdSteps; ++i) sp[i] = 0.0f;
@@ -587,10 +660,17 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
             }
             __syncwarp();
             if (valid) {
-                store_block(static_cast<IoT*>(p.du) + chain * p.seqlen, t0, ns, vec, o_du);
-                store_block(static_cast<IoT*>(p.ddelta) + chain * p.seqlen, t0, ns, vec, o_dd);
-                if (kHasZ && p.dz != nullptr)
-                    store_block(static_cast<IoT*>(p.dz) + chain * p.seqlen, t0, ns, vec, o_dz);
+                if constexpr (kBld) {   // 32 lanes write 32 consecutive channels of a step
+                    store_block_strided(static_cast<IoT*>(p.du) + io_base, t0, ns, io_step, o_du);
+                    store_block_strided(static_cast<IoT*>(p.ddelta) + io_base, t0, ns, io_step, o_dd);
+                    if (kHasZ && p.dz != nullptr)
+                        store_block_strided(static_cast<IoT*>(p.dz) + io_base, t0, ns, io_step, o_dz);
+                } else {
+                    store_block(static_cast<IoT*>(p.du) + chain * p.seqlen, t0, ns, vec, o_du);
+                    store_block(static_cast<IoT*>(p.ddelta) + chain * p.seqlen, t0, ns, vec, o_dd);
+                    if (kHasZ && p.dz != nullptr)
+                        store_block(static_cast<IoT*>(p.dz) + chain * p.seqlen, t0, ns, vec, o_dz);
+                }
             }
         }
 

@@ -793,9 +793,13 @@ __global__ void __launch_bounds__(kScanWarps * 32, ScanLayout<kCpl>::kMinBlocks 
         if constexpr (kLookback) {       // segments from their own start, then the look-back
             ok = run_segment<IoT, kCpl, kHasZ, kSoftplus, kZoh, true, false, true, false>(
                 p, maps, wsm, lane, b, d0, t_begin, t_end, lc, out_row, seq, sdt, ckpt_row);
-        } else if constexpr (kBld) {     // chained mode only, with outputs
-            ok = run_segment<IoT, kCpl, kHasZ, kSoftplus, kZoh, true, false, false, true>(
-                p, maps, wsm, lane, b, d0, t_begin, t_end, lc, out_row, seq, sdt, ckpt_row);
+        } else if constexpr (kBld) {     // chained mode only: outputs, or the backward's checkpoints
+            if (p.ckpt != nullptr)
+                ok = run_segment<IoT, kCpl, kHasZ, kSoftplus, kZoh, false, true, false, true>(
+                    p, maps, wsm, lane, b, d0, t_begin, t_end, lc, out_row, seq, sdt, ckpt_row);
+            else
+                ok = run_segment<IoT, kCpl, kHasZ, kSoftplus, kZoh, true, false, false, true>(
+                    p, maps, wsm, lane, b, d0, t_begin, t_end, lc, out_row, seq, sdt, ckpt_row);
         } else if (p.ckpt != nullptr) {  // checkpoint pass of the backward: states only
             ok = run_segment<IoT, kCpl, kHasZ, kSoftplus, kZoh, false, true, false, false>(
                 p, maps, wsm, lane, b, d0, t_begin, t_end, lc, out_row, seq, sdt, ckpt_row);

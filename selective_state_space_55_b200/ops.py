@@ -390,25 +390,28 @@ def scan_bwd_workspace_bytes(batch, dim, dstate, seqlen, io_dtype=torch.bfloat16
 
 def selective_scan_bwd(u, delta, A, B, C, dout, D=None, z=None, delta_bias=None, softplus=True,
                        initial_state=None, dlast_state=None, flags=0, workspace=None,
-                       stream=None, zoh=False):
+                       stream=None, zoh=False, layout="bdl"):
     """Gradients of the scan through ``mamba_selective_scan_bwd``.
 
-    Same inputs as ``selective_scan_fwd`` plus dout (batch, dim, L) in u's
-    dtype and dlast_state (batch, dim, N) fp32 or None; ``zoh`` sets
-    MAMBA_FLAG_ZOH (the zero-order-hold input term, as in the forward).
-    Returns a dict: du, ddelta (and dz when z is given) in u's dtype; dA, dB,
-    dC (and dD, ddelta_bias, dinitial_state for the optional inputs given) in
-    fp32.
+    Same inputs as ``selective_scan_fwd`` plus dout (u's shape and dtype) and
+    dlast_state (batch, dim, N) fp32 or None; ``zoh`` sets MAMBA_FLAG_ZOH (the
+    zero-order-hold input term, as in the forward) and ``layout="bld"``
+    MAMBA_FLAG_LAYOUT_BLD (u, delta, z, dout and their gradients in
+    (batch, L, dim)).  Returns a dict: du, ddelta (and dz when z is given) in
+    u's shape and dtype; dA, dB, dC (and dD, ddelta_bias, dinitial_state for
+    the optional inputs given) in fp32.
     """
-    batch, dim, L = u.shape
+    flags, bld = _layout_flags(layout, flags)
+    batch, dim, L = _scan_sizes(u, bld)
+    act = (batch, L, dim) if bld else (batch, dim, L)
     if zoh:
         flags |= MAMBA_FLAG_ZOH
     N = A.shape[1]
     io, bc = u.dtype, B.dtype
     dev = u.device
-    _check_cuda("u", u, (torch.float32, torch.bfloat16), (batch, dim, L))
+    _check_cuda("u", u, (torch.float32, torch.bfloat16), act)
     for name, t in (("delta", delta), ("z", z), ("dout", dout)):
-        _check_cuda(name, t, (io,), (batch, dim, L))
+        _check_cuda(name, t, (io,), act)
     _check_cuda("A", A, (torch.float32,), (dim, N))
     _check_cuda("B", B, (torch.float32, torch.bfloat16), (batch, N, L))
     _check_cuda("C", C, (bc,), (batch, N, L))

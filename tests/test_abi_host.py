@@ -354,13 +354,14 @@ def test_plan_bld_layout(lib):
     assert lib.mamba_selective_scan_plan(ctypes.byref(dims), 148, ctypes.byref(plan)) == 0
 
 
-def test_backward_refuses_bld_layout(lib):
+def test_backward_checks_bld_layout_like_the_standard_one(lib):
     d = _dims()
     d.flags = ops.MAMBA_FLAG_LAYOUT_BLD
-    rc = lib.mamba_selective_scan_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, 1, None,
-                                      FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None,
-                                      None, ctypes.byref(d), None)
-    assert rc == -2
+    call = lambda u=FAKE, dout=FAKE: lib.mamba_selective_scan_bwd(  # noqa: E731
+        u, FAKE, FAKE, FAKE, FAKE, None, None, None, 1, None, dout, None, FAKE, FAKE, FAKE, FAKE,
+        FAKE, None, None, None, None, ctypes.byref(d), None)
+    assert call(u=None) == -1 and call(dout=None) == -1
+    assert call(u=ctypes.c_void_p(0x10001)) == -3
 
 
 def test_binding_layout_argument():

@@ -5,7 +5,7 @@
 The kernel runs the same per-channel arithmetic in either layout, so its
 outputs must equal the (batch, dim, seqlen) call's bit for bit once transposed;
 the float64 oracle (which takes (batch, dim, seqlen)) checks the values on
-top, on inputs transposed on the host.  Cases cover the TMA tiles and the
+top, on inputs transposed on the host; the backward likewise.  Cases cover the TMA tiles and the
 plain-load path (dim * element size not a multiple of 16 bytes, or
 MAMBA_FLAG_NO_TMA), a channel count that leaves a partial group, a ragged
 last tile, the optional inputs, the zero-order hold, a start state, and the
@@ -162,11 +162,64 @@ def test_host_buffer_call():
     assert torch.equal(last, dev_last.cpu())
 
 
-def test_parallel_chunks_and_backward_are_refused():
+def test_parallel_chunks_are_refused():
     x = layer_inputs(1, 64, 1024, seed=2)
     with pytest.raises(ops.MambaError):
         scan(x, "bld", num_chunks=4, flags=ops.MAMBA_FLAG_PARALLEL_CHUNKS)
-    dout = torch.ones_like(x["u"])
-    with pytest.raises(ops.MambaError):
-        ops.selective_scan_bwd(x["u"], x["delta"], x["A"], x["B"], x["C"], dout,
-                               flags=ops.MAMBA_FLAG_LAYOUT_BLD)
+
+
+# ------------------------------------------------------------ backward
+
+def backward(x, dout, layout, zoh=False, h0=None, dlast=None):
+    args = {k: (to_bld(x[k]) if layout == "bld" else x[k]) for k in ACT}
+    g = ops.selective_scan_bwd(args["u"], args["delta"], x["A"], x["B"], x["C"],
+                               to_bld(dout) if layout == "bld" else dout, D=x["D"], z=args["z"],
+                               delta_bias=x["delta_bias"], initial_state=h0, dlast_state=dlast,
+                               zoh=zoh, layout=layout)
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    if layout == "bld":
+        for k in ("du", "ddelta", "dz"):
+            if k in g:
+                g[k] = g[k].transpose(1, 2)
+    return g
+
+
+@pytest.mark.parametrize("dtype,shape,zoh", [
+    (torch.bfloat16, (2, 256, 1000), False),   # staged tiles, ragged last block
+    (torch.float32, (2, 96, 512), False),
+    (torch.bfloat16, (3, 200, 777), False),    # a partial last group: read directly
+    (torch.bfloat16, (2, 100, 300), False),    # 200-byte rows of channels: read directly
+    (torch.bfloat16, (2, 128, 640), True),
+])
+def test_backward_matches_standard_layout(dtype, shape, zoh):
+    """Per-chain gradients (du, ddelta, dz) are the same arithmetic in either
+    layout and equal bit for bit; the gradients summed over chains (dA, dB,
+    dC, dD, the bias) are added atomically in no fixed order and agree to
+    rounding."""
+    x = layer_inputs(*shape, dtype=dtype, seed=21)
+    g = torch.Generator(device=DEV)
+    g.manual_seed(22)
+    dout = torch.randn(*shape, generator=g, device=DEV).to(dtype)
+    h0 = torch.randn(shape[0], shape[1], 16, generator=g, device=DEV)
+    dlast = torch.randn(shape[0], shape[1], 16, generator=g, device=DEV)
+    a = backward(x, dout, "bld", zoh=zoh, h0=h0, dlast=dlast)
+    b = backward(x, dout, "bdl", zoh=zoh, h0=h0, dlast=dlast)
+    assert set(a) == set(b)
+    for k in ("du", "ddelta", "dz", "dinitial_state"):
+        assert torch.equal(a[k], b[k]), k
+    for k in ("dA", "dB", "dC", "dD", "ddelta_bias"):
+        assert max_rel_err(a[k], b[k]) <= 1e-5, k
+
+
+def test_backward_against_oracle(ref):
+    x = layer_inputs(2, 64, 300, dtype=torch.float32, seed=23)
+    g = torch.Generator(device=DEV)
+    g.manual_seed(24)
+    dout = torch.randn(2, 64, 300, generator=g, device=DEV)
+    got = backward(x, dout, "bld")
+    c = lambda t: None if t is None else t.cpu()  # noqa: E731
+    o = ref.selective_scan_bwd(c(x["u"]), c(x["delta"]), c(x["A"]), c(x["B"]), c(x["C"]), dout.cpu(),
+                               D=c(x["D"]), z=c(x["z"]), delta_bias=c(x["delta_bias"]))
+    for k in o:
+        assert max_rel_err(got[k], o[k]) <= FP32_TOL, k
