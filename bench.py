@@ -833,7 +833,12 @@ def bench_conv(args, rank, world, local):
 
 def bench_bwd(args, rank, world, local):
     """Measurement case: the backward pass of the scan (checkpoint pass + adjoint)
-    on the Mamba-2.8B layer shape, gate, D and bias on, dout random."""
+    on the Mamba-2.8B layer shape, gate, D and bias on, dout random; with
+    ``--scan-variant bld`` the activations and their gradients are
+    (batch, seqlen, dim)."""
+    if args.scan_variant not in ("euler", "bld"):
+        raise SystemExit("--only bwd takes --scan-variant euler or bld")
+    bld = args.scan_variant == "bld"
     global _WORLD
     _WORLD = world
     from selective_state_space_55_b200 import build as cuda_build
@@ -854,10 +859,15 @@ def bench_bwd(args, rank, world, local):
     dout = torch.randn(c.batch, c.dim, c.seqlen, generator=g, device="cuda").to(c.io_dtype)
     ws = torch.empty(ops.scan_bwd_workspace_bytes(c.batch, c.dim, c.dstate, c.seqlen, c.io_dtype,
                                                   c.bc_dtype), dtype=torch.uint8, device="cuda")
+    act = {k: x[k] for k in ("u", "delta", "z")}
+    if bld:   # the same values in the (batch, seqlen, dim) layout
+        act = {k: (None if v is None else v.transpose(1, 2).contiguous()) for k, v in act.items()}
+        dout = dout.transpose(1, 2).contiguous()
 
     def step():
-        return ops.selective_scan_bwd(x["u"], x["delta"], x["A"], x["B"], x["C"], dout, D=x["D"],
-                                      z=x["z"], delta_bias=x["delta_bias"], workspace=ws)
+        return ops.selective_scan_bwd(act["u"], act["delta"], x["A"], x["B"], x["C"], dout, D=x["D"],
+                                      z=act["z"], delta_bias=x["delta_bias"], workspace=ws,
+                                      layout="bld" if bld else "bdl")
 
     for _ in range(args.warmup):
         step()
@@ -899,6 +909,7 @@ def bench_bwd(args, rank, world, local):
             "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded)",
             "config": {"workload": f"{c.name} backward ({c.batch}x{c.dim}, N={c.dstate}, L={c.seqlen}, "
                                    "bf16, gate/D/bias, checkpoint pass + adjoint)",
+                       "activations": "(batch, seqlen, dim)" if bld else "(batch, dim, seqlen)",
                        "checkpoint_bytes": ws.numel()},
             "roofline": {"bound": "alu", "pipe": f"MUFU ({mufu} per element, both launches)",
                          "kernel": "selective_scan_bwd_kernel",
@@ -907,12 +918,12 @@ def bench_bwd(args, rank, world, local):
                          "peak_56_op_basis": round(peak_twice, 2),
                          "frac_56_op_basis": round(value / world / peak_twice, 4),
                          "traffic": (recorded_traffic("selective_scan_bwd_kernel", sources_digest())
-                                     if c.batch == 16 else None)},
+                                     if c.batch == 16 and not bld else None)},
             "gpu_launches": K * 2,
             "clocks": sampler.summary(t0, t1),
-            "cpu_baseline": (None if args.no_cpu_baseline
+            "cpu_baseline": (None if args.no_cpu_baseline or bld
                              else bwd_cpu_baseline(c, x, dout, args.cpu_seconds)),
-            "partial_case": {"only": "bwd", "scan_batch": args.scan_batch,
+            "partial_case": {"only": "bwd", "scan_batch": args.scan_batch, "scan_variant": args.scan_variant,
                              "note": "measurement of the backward pass, not the benchmark workload"},
         }
         print(json.dumps(line), flush=True)

@@ -140,16 +140,16 @@ cudaError_t launch_scan_split(const ScanParams& prm, const CUtensorMap* maps, in
     if (e != cudaSuccess) return e;
     int per_sm = (dev >= 0 && dev < kMaxDevices) ? resident[dev] : 0;
     if (per_sm <= 0) {
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kScanWarps * 32,
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, Lay::kWarps * 32,
                                                           Lay::kCtaSmem);
         if (e != cudaSuccess) return e;
         if (per_sm <= 0) return cudaErrorInvalidConfiguration;
         if (dev >= 0 && dev < kMaxDevices) resident[dev] = per_sm;
     }
-    const int64_t want = (want_warps + kScanWarps - 1) / kScanWarps;
+    const int64_t want = (want_warps + Lay::kWarps - 1) / Lay::kWarps;
     const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)per_sm * sms));
-    kernel<<<(unsigned)grid, kScanWarps * 32, Lay::kCtaSmem, stream>>>(prm, maps[0], maps[1],
-                                                                         maps[2], maps[3], maps[4]);
+    kernel<<<(unsigned)grid, Lay::kWarps * 32, Lay::kCtaSmem, stream>>>(prm, maps[0], maps[1],
+                                                                          maps[2], maps[3], maps[4]);
     return cudaGetLastError();
 }
 
@@ -433,8 +433,11 @@ mamba_status_t plan_scan(const mamba_dims_t* dims, int sm_count, mamba_scan_plan
     plan->mode = mode;
     plan->units_pass_a = items;
     plan->units_pass_b = fixes;
-    plan->max_warps = mode == 0 && K > 1 ? std::min<int64_t>(groups_run, W)
-                                         : std::min<int64_t>(items, W);
+    // Warps the persistent grid holds at once (the two-lane kernel runs
+    // fewer per SM: SplitLayout::kWarpsPerSm).
+    const int64_t W_run = lanes == 2 ? (int64_t)sm_count * SplitLayout::kWarpsPerSm : W;
+    plan->max_warps = mode == 0 && K > 1 ? std::min<int64_t>(groups_run, W_run)
+                                         : std::min<int64_t>(items, W_run);
     plan->launches = (groups > 0 && L > 0) ? (mode == 1 ? 3 : 1) : 0;
     plan->workspace_bytes =
         (groups > 0 && L > 0) ? scan_workspace_layout(dims, groups_run, K, mode).total : 0;

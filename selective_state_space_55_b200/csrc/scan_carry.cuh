@@ -127,10 +127,59 @@ __device__ __forceinline__ void load_run(const T* row, int64_t t, int valid, boo
     }
 }
 
+// The same V values, kept as raw words (V * size / 4 of them) so that a pass
+// can have every load in flight before it uses any: one or two 16-byte loads
+// when `vec`, else element by element (0 past `valid`).
+template <typename T, int V>
+struct RawRun {
+    static constexpr int kWords = V * (int)sizeof(T) / 4;
+    uint32_t w[kWords];
+};
+
+template <typename T, int V>
+__device__ __forceinline__ void load_raw(const T* row, int64_t t, int valid, bool vec,
+                                         RawRun<T, V>& r) {
+    constexpr int kWords = RawRun<T, V>::kWords;
+    if (kWords % 4 == 0 && vec && valid == V) {
+#pragma unroll
+        for (int q = 0; q < kWords / 4; ++q) {
+            const uint4 v = __ldcs(reinterpret_cast<const uint4*>(row + t) + q);
+            r.w[4 * q] = v.x; r.w[4 * q + 1] = v.y; r.w[4 * q + 2] = v.z; r.w[4 * q + 3] = v.w;
+        }
+    } else if constexpr (sizeof(T) == 2) {
+        const unsigned short* h = reinterpret_cast<const unsigned short*>(row + t);
+#pragma unroll
+        for (int i = 0; i < kWords; ++i) {
+            const uint32_t lo = 2 * i < valid ? h[2 * i] : 0u;
+            const uint32_t hi = 2 * i + 1 < valid ? h[2 * i + 1] : 0u;
+            r.w[i] = lo | (hi << 16);
+        }
+    } else {
+        const uint32_t* f = reinterpret_cast<const uint32_t*>(row + t);
+#pragma unroll
+        for (int i = 0; i < kWords; ++i) r.w[i] = i < valid ? f[i] : 0u;
+    }
+}
+
+// Value j of a raw run, as fp32.
+template <typename T, int V>
+__device__ __forceinline__ float raw_elem(const RawRun<T, V>& r, int j) {
+    if constexpr (sizeof(T) == 2) {
+        const uint32_t w = r.w[j >> 1];
+        return __uint_as_float((j & 1) ? (w & 0xffff0000u) : (w << 16));
+    } else {
+        return __uint_as_float(r.w[j]);
+    }
+}
+
 // Segment k's correction for one chain (one warp, lanes over time): adds
 // C_t . (exp(A S_t) (.) hin) (gated) to the segment's outputs, hin being the
-// segment's true start state.  Every lane holds the same hin.
-template <typename IoT, typename BcT, bool kHasZ, bool kSoftplus>
+// segment's true start state.  Every lane holds the same hin.  With kAhead a
+// pass issues all its loads (delta, out, z and the C rows of the live state
+// entries) before it uses any, so their latencies overlap; without it (the
+// look-back inside the scan kernel, short of registers) each C row is loaded
+// where its entry is taken.
+template <typename IoT, typename BcT, bool kHasZ, bool kSoftplus, bool kAhead = false>
 __device__ __forceinline__ void correct_chain(const CorrectParams& p, int64_t chain, int64_t k,
                                               const float (&hin)[kNPad], int lane) {
     constexpr int V = 16 / (int)sizeof(IoT);    // steps per lane and pass
@@ -164,8 +213,28 @@ __device__ __forceinline__ void correct_chain(const CorrectParams& p, int64_t ch
         if (active == 0) break;
         const int64_t ts = t0 + (int64_t)lane * V;
         const int valid = (int)max((int64_t)0, min((int64_t)V, t_end - ts));
+        RawRun<BcT, V> craw[kAhead ? kNPad : 1];
+        RawRun<IoT, V> oraw, zraw;
         float dl[V];
-        load_run<IoT, V>(drow, ts, valid, p.vec_io != 0, dl);
+        if constexpr (kAhead) {
+            RawRun<IoT, V> draw;
+            load_raw<IoT, V>(drow, ts, valid, p.vec_io != 0, draw);
+#pragma unroll
+            for (int n = 0; n < kNPad; ++n) {
+                if ((active >> n) & 1u) {
+                    load_raw<BcT, V>(crow + n * p.seqlen, ts, valid, p.vec_c != 0, craw[n]);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < RawRun<BcT, V>::kWords; ++i) craw[n].w[i] = 0u;
+                }
+            }
+            load_raw<IoT, V>(orow, ts, valid, p.vec_io != 0, oraw);
+            if (kHasZ) load_raw<IoT, V>(zrow, ts, valid, p.vec_io != 0, zraw);
+#pragma unroll
+            for (int j = 0; j < V; ++j) dl[j] = raw_elem<IoT, V>(draw, j);
+        } else {
+            load_run<IoT, V>(drow, ts, valid, p.vec_io != 0, dl);
+        }
         float S[V];
         float run = 0.0f;
         bool nonneg = true;
@@ -199,7 +268,12 @@ __device__ __forceinline__ void correct_chain(const CorrectParams& p, int64_t ch
         for (int n = 0; n < kNPad; ++n) {
             if (!((active >> n) & 1u)) continue;   // uniform across the warp
             float cv[V];
-            load_run<BcT, V>(crow + n * p.seqlen, ts, valid, p.vec_c != 0, cv);
+            if constexpr (kAhead) {
+#pragma unroll
+                for (int j = 0; j < V; ++j) cv[j] = raw_elem<BcT, V>(craw[n], j);
+            } else {
+                load_run<BcT, V>(crow + n * p.seqlen, ts, valid, p.vec_c != 0, cv);
+            }
 #pragma unroll
             for (int j = 0; j < V; ++j) {
                 const float x = a2[n] * (before + S[j]);
@@ -207,9 +281,17 @@ __device__ __forceinline__ void correct_chain(const CorrectParams& p, int64_t ch
             }
         }
         float o[V];
-        load_run<IoT, V>(orow, ts, valid, p.vec_io != 0, o);
         float zv[V];
-        if (kHasZ) load_run<IoT, V>(zrow, ts, valid, p.vec_io != 0, zv);
+        if constexpr (kAhead) {
+#pragma unroll
+            for (int j = 0; j < V; ++j) {
+                o[j] = raw_elem<IoT, V>(oraw, j);
+                if (kHasZ) zv[j] = raw_elem<IoT, V>(zraw, j);
+            }
+        } else {
+            load_run<IoT, V>(orow, ts, valid, p.vec_io != 0, o);
+            if (kHasZ) load_run<IoT, V>(zrow, ts, valid, p.vec_io != 0, zv);
+        }
 #pragma unroll
         for (int j = 0; j < V; ++j) {
             float g = corr[j];
@@ -235,7 +317,10 @@ __device__ __forceinline__ void correct_chain(const CorrectParams& p, int64_t ch
 }
 
 template <typename IoT, typename BcT, bool kHasZ, bool kSoftplus>
-__global__ void __launch_bounds__(kCorrectWarps * 32)
+// Two CTAs (16 warps) per SM: the pass's loads all in flight take registers,
+// and capping them at 128 keeps the 16 warps (measured faster than 8 warps at
+// 168 registers).
+__global__ void __launch_bounds__(kCorrectWarps * 32, 2)
     scan_correct_kernel(const __grid_constant__ CorrectParams p) {
     const int lane = threadIdx.x & 31;
     for (;;) {
@@ -249,7 +334,7 @@ __global__ void __launch_bounds__(kCorrectWarps * 32)
         const float* hs = p.ws_h + ((k - 1) * p.chains + chain) * kNPad;
 #pragma unroll
         for (int n = 0; n < kNPad; ++n) hin[n] = n < p.dstate ? __ldcg(hs + n) : 0.0f;
-        correct_chain<IoT, BcT, kHasZ, kSoftplus>(p, chain, k, hin, lane);
+        correct_chain<IoT, BcT, kHasZ, kSoftplus, true>(p, chain, k, hin, lane);
     }
 }
 

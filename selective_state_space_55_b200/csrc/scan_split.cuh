@@ -42,9 +42,13 @@ struct SplitLayout {
     static constexpr int kOffBcf = kScanStages * kStage;
     static constexpr int kOffBar = kOffBcf + kBcfBytes;
     static constexpr int kWarpSmem = ((kOffBar + 64 + 255) / 256) * 256;
-    static constexpr int kCtaSmem = kScanWarps * kWarpSmem + 1024;   // + base alignment slack
-    static constexpr int kMinBlocks = 4;                             // CTAs per SM
-    static constexpr int kWarpsPerSm = kScanWarps * kMinBlocks;
+    static constexpr int kWarps = 4;                                 // warps per CTA
+    static constexpr int kCtaSmem = kWarps * kWarpSmem + 1024;       // + base alignment slack
+    // Three CTAs per SM, so up to 168 registers: on 8 x 4096 channels (2048
+    // warps) measured 1.2% faster than four CTAs at 128 registers, although
+    // fewer warps are resident at once.
+    static constexpr int kMinBlocks = 3;                             // CTAs per SM
+    static constexpr int kWarpsPerSm = kWarps * kMinBlocks;
     static_assert(3 * kIoTile <= kOffB, "activation tiles overlap the B rows");
     static_assert(kStage % 256 == 0 && kWarpSmem % 256 == 0, "32-byte swizzle needs 256-byte tiles");
 };
@@ -313,7 +317,7 @@ __device__ __forceinline__ bool run_segment_split(const ScanParams& p, const Tma
 }
 
 template <typename IoT, bool kHasZ, bool kSoftplus>
-__global__ void __launch_bounds__(kScanWarps * 32, SplitLayout::kMinBlocks)
+__global__ void __launch_bounds__(SplitLayout::kWarps * 32, SplitLayout::kMinBlocks)
     selective_scan_fwd_split_kernel(const __grid_constant__ ScanParams p,
                                     const __grid_constant__ CUtensorMap tm_u,
                                     const __grid_constant__ CUtensorMap tm_delta,

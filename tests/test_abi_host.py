@@ -191,11 +191,12 @@ def test_plan_layer_shapes(lib):
     assert p["workspace_bytes"] == 256 + flags + chains * 64
     assert p["lanes_per_channel"] == 1
     # 1.4B layer: 1024 groups of 32 would leave half the 2368 warp slots idle,
-    # so each channel gets two lanes: 2048 groups of 16, one warp each
+    # so each channel gets two lanes: 2048 groups of 16, one warp each, of
+    # which the two-lane kernel (12 warps per SM) holds 1776 at once
     c = SCAN_CONFIGS["mamba_1p4b_layer"]
     p = ops.scan_plan(c.batch, c.dim, c.dstate, c.seqlen, c.io_dtype, c.bc_dtype)
     assert p["mode"] == 0 and p["lanes_per_channel"] == 2 and p["groups"] == 2048
-    assert p["nchunks"] == 8 and p["max_warps"] == 2048
+    assert p["nchunks"] == 8 and p["max_warps"] == 148 * 12
     assert p["workspace_bytes"] == 256 + 8192 + 8 * 4096 * 64
     q = ops.scan_plan(c.batch, c.dim, c.dstate, c.seqlen, c.io_dtype, c.bc_dtype,
                       flags=ops.MAMBA_FLAG_ONE_LANE_PER_CHANNEL)
