@@ -3,7 +3,9 @@ the float64 oracle's adjoint, which finite differences of the forward oracle
 pin.  fp32 and bf16, with and without gate / D / bias / softplus / start
 state / last-state gradient, state sizes below 16, ragged lengths and channel
 counts, sequences cut into many chained segments, and all of it again with
-the zero-order-hold input term."""
+the zero-order-hold input term.  At the benchmark's full size (the 2.8B layer
+shape): sampled chains and channels against the oracle, and the two
+activation layouts against each other."""
 import pytest
 import torch
 
@@ -133,3 +135,66 @@ def test_zoh_many_segments(ref):
 
 def test_zoh_bf16_layer_recipe(ref):
     check(ref, problem(2, 256, 2048, dtype=torch.bfloat16, seed=36), BF16_TOL, zoh=True)
+
+
+# ------------------------------------------------------------ full size
+
+def full_size_backward(layout="bdl"):
+    """The backward's benchmark workload: the 2.8B layer shape (16 x 5120
+    channels x 2048 steps, bf16), gate, D and bias on, dout random."""
+    cfg = I.SCAN_CONFIGS["mamba_2p8b_layer"]
+    x = I.make_scan_inputs(cfg, DEV, seed=0)
+    g = torch.Generator(device=DEV)
+    g.manual_seed(13)
+    dout = torch.randn(cfg.batch, cfg.dim, cfg.seqlen, generator=g, device=DEV).to(cfg.io_dtype)
+    act = {k: x[k] for k in ("u", "delta", "z")}
+    dy = dout
+    if layout == "bld":
+        act = {k: v.transpose(1, 2).contiguous() for k, v in act.items()}
+        dy = dout.transpose(1, 2).contiguous()
+    grads = ops.selective_scan_bwd(act["u"], act["delta"], x["A"], x["B"], x["C"], dy, D=x["D"],
+                                   z=act["z"], delta_bias=x["delta_bias"], layout=layout)
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    if layout == "bld":
+        for k in ("du", "ddelta", "dz"):
+            grads[k] = grads[k].transpose(1, 2)
+    return cfg, x, dout, grads
+
+
+def test_full_size_sampled_chains_and_channels(ref):
+    """du, delta's gradient and dz of a chain depend only on that chain and
+    its batch row's B and C, so sampled chains are checked against the oracle
+    run on each alone; dA, dD and the bias gradient of a channel sum over the
+    batch rows, so sampled channels are checked against the oracle run on that
+    channel over all 16 rows.  (dB and dC sum over all 5120 channels; the
+    smaller cases above check them.)"""
+    cfg, x, dout, g = full_size_backward()
+    for row in I.gather_chains(x, I.sample_chains(cfg.batch, cfg.dim, 8, seed=5)):
+        b, d = row["b"], row["d"]
+        o = ref.selective_scan_bwd(row["u"], row["delta"], row["A"], row["B"], row["C"],
+                                   dout[b:b + 1, d:d + 1].cpu(), D=row["D"], z=row["z"],
+                                   delta_bias=row["delta_bias"])
+        for k in ("du", "ddelta", "dz"):
+            e = max_rel_err(g[k][b:b + 1, d:d + 1], o[k])
+            assert e <= BF16_TOL, f"chain ({b},{d}) {k} error {e:.3e}"
+    for d in (0, 2047, cfg.dim - 1):
+        c = lambda t: t[:, d:d + 1].cpu()  # noqa: E731
+        o = ref.selective_scan_bwd(c(x["u"]), c(x["delta"]), x["A"][d:d + 1].cpu(), x["B"].cpu(),
+                                   x["C"].cpu(), c(dout), D=x["D"][d:d + 1].cpu(), z=c(x["z"]),
+                                   delta_bias=x["delta_bias"][d:d + 1].cpu())
+        assert max_rel_err(g["dA"][d:d + 1], o["dA"]) <= BF16_TOL, f"channel {d} dA"
+        assert max_rel_err(g["dD"][d:d + 1], o["dD"]) <= BF16_TOL, f"channel {d} dD"
+        assert max_rel_err(g["ddelta_bias"][d:d + 1], o["ddelta_bias"]) <= BF16_TOL, f"channel {d} bias"
+
+
+def test_full_size_layouts_agree():
+    """The same workload with activations in (batch, seqlen, dim): the
+    per-chain gradients equal the (batch, dim, seqlen) call's bit for bit; the
+    sums over chains (atomics in no fixed order) agree to rounding."""
+    a = full_size_backward("bdl")[3]
+    b = full_size_backward("bld")[3]
+    for k in ("du", "ddelta", "dz"):
+        assert torch.equal(a[k], b[k]), k
+    for k in ("dA", "dB", "dC", "dD", "ddelta_bias"):
+        assert max_rel_err(a[k], b[k]) <= 1e-4, k
