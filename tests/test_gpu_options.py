@@ -2,7 +2,8 @@
 a given start state (mamba_selective_scan_fwd_with_state).  CUDA path through
 the C ABI vs the float64 oracle, plus closed forms the pages fix: the Theorem-1
 gate is exact under the zero-order hold, and a constant input has the fixed
-point -B u / A whatever Delta does."""
+point -B u / A whatever Delta does.  Both options also at the 2.8B layer
+shape, on sampled chains."""
 import pytest
 import torch
 
@@ -248,3 +249,28 @@ def test_zoh_updates_continue_zoh_scan():
     assert ops.device_status() == 0
     assert max_rel_err(torch.stack(outs, dim=-1), out.double()) <= FP32_TOL
     assert max_rel_err(state, last.double()) <= FP32_TOL
+
+
+# ------------------------------------------------------------ full size
+
+@pytest.mark.parametrize("variant", ["zoh", "start_state"])
+def test_full_size_sampled_chains(ref, variant):
+    """The benchmark's variant workloads at the 2.8B layer shape (16 x 5120 x
+    2048, bf16): the zero-order hold, and a given N(0, 1) start state.  Sampled
+    chains against the oracle run on each chain alone (with its start state)."""
+    cfg = I.SCAN_CONFIGS["mamba_2p8b_layer"]
+    x = I.make_scan_inputs(cfg, DEV, seed=0)
+    zoh = variant == "zoh"
+    h0 = start_state(cfg.batch, cfg.dim, cfg.dstate, seed=7) if variant == "start_state" else None
+    out, last = gpu_scan(x, zoh=zoh, initial_state=h0)
+    for row in I.gather_chains(x, I.sample_chains(cfg.batch, cfg.dim, 16, seed=4)):
+        b, d = row["b"], row["d"]
+        o_out, o_last = ref.selective_scan(row["u"], row["delta"], row["A"], row["B"], row["C"],
+                                           D=row["D"], z=row["z"], delta_bias=row["delta_bias"],
+                                           zoh=zoh,
+                                           initial_state=None if h0 is None
+                                           else h0[b:b + 1, d:d + 1].cpu())
+        e = max_rel_err(out[b:b + 1, d:d + 1], o_out)
+        assert e <= BF16_TOL, f"chain ({b},{d}) out error {e:.3e}"
+        e = max_rel_err(last[b:b + 1, d:d + 1], o_last)
+        assert e <= BF16_TOL, f"chain ({b},{d}) last_state error {e:.3e}"
