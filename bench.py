@@ -835,10 +835,12 @@ def bench_bwd(args, rank, world, local):
     """Measurement case: the backward pass of the scan (checkpoint pass + adjoint)
     on the Mamba-2.8B layer shape, gate, D and bias on, dout random; with
     ``--scan-variant bld`` the activations and their gradients are
-    (batch, seqlen, dim)."""
-    if args.scan_variant not in ("euler", "bld"):
-        raise SystemExit("--only bwd takes --scan-variant euler or bld")
+    (batch, seqlen, dim), with ``--scan-variant zoh`` the input term is the
+    zero-order hold's."""
+    if args.scan_variant not in ("euler", "bld", "zoh"):
+        raise SystemExit("--only bwd takes --scan-variant euler, bld or zoh")
     bld = args.scan_variant == "bld"
+    zoh = args.scan_variant == "zoh"
     global _WORLD
     _WORLD = world
     from selective_state_space_55_b200 import build as cuda_build
@@ -867,7 +869,7 @@ def bench_bwd(args, rank, world, local):
     def step():
         return ops.selective_scan_bwd(act["u"], act["delta"], x["A"], x["B"], x["C"], dout, D=x["D"],
                                       z=act["z"], delta_bias=x["delta_bias"], workspace=ws,
-                                      layout="bld" if bld else "bdl")
+                                      layout="bld" if bld else "bdl", zoh=zoh)
 
     for _ in range(args.warmup):
         step()
@@ -894,8 +896,10 @@ def bench_bwd(args, rank, world, local):
     # states are recomputed and kept for the way back), the softplus again (2),
     # its derivative sigmoid (2) and the gate's sigmoid (2).
     mufu = (16 + 2) + (16 + 2 + 2 + 2)
+    if zoh:   # the gain's 1 / Delta, once per step in each launch
+        mufu += 2
     # An adjoint that forms Abar a second time on the way back issues 16 more;
-    # the fraction on that 56-op basis is reported beside this one.
+    # the fraction on that basis is reported beside this one.
     mufu_twice = mufu + 16
     sms = torch.cuda.get_device_properties(local).multi_processor_count
     peak = R.mufu_peak_elements_per_s(sms, peaks["sm_max_mhz"], mufu) / 1e9
@@ -909,19 +913,20 @@ def bench_bwd(args, rank, world, local):
             "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded)",
             "config": {"workload": f"{c.name} backward ({c.batch}x{c.dim}, N={c.dstate}, L={c.seqlen}, "
                                    "bf16, gate/D/bias, checkpoint pass + adjoint)",
+                       "input_term": "zero-order hold" if zoh else "Euler",
                        "activations": "(batch, seqlen, dim)" if bld else "(batch, dim, seqlen)",
                        "checkpoint_bytes": ws.numel()},
             "roofline": {"bound": "alu", "pipe": f"MUFU ({mufu} per element, both launches)",
                          "kernel": "selective_scan_bwd_kernel",
                          "achieved": round(value / world, 2), "peak": round(peak, 2), "unit": "Gelem/s",
                          "frac": round(value / world / peak, 4),
-                         "peak_56_op_basis": round(peak_twice, 2),
-                         "frac_56_op_basis": round(value / world / peak_twice, 4),
+                         f"peak_{mufu_twice}_op_basis": round(peak_twice, 2),
+                         f"frac_{mufu_twice}_op_basis": round(value / world / peak_twice, 4),
                          "traffic": (recorded_traffic("selective_scan_bwd_kernel", sources_digest())
-                                     if c.batch == 16 and not bld else None)},
+                                     if c.batch == 16 and not bld and not zoh else None)},
             "gpu_launches": K * 2,
             "clocks": sampler.summary(t0, t1),
-            "cpu_baseline": (None if args.no_cpu_baseline or bld
+            "cpu_baseline": (None if args.no_cpu_baseline or bld or zoh
                              else bwd_cpu_baseline(c, x, dout, args.cpu_seconds)),
             "partial_case": {"only": "bwd", "scan_batch": args.scan_batch, "scan_variant": args.scan_variant,
                              "note": "measurement of the backward pass, not the benchmark workload"},
