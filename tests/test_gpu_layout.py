@@ -170,12 +170,12 @@ def test_parallel_chunks_are_refused():
 
 # ------------------------------------------------------------ backward
 
-def backward(x, dout, layout, zoh=False, h0=None, dlast=None):
+def backward(x, dout, layout, zoh=False, h0=None, dlast=None, softplus=True):
     args = {k: (to_bld(x[k]) if layout == "bld" else x[k]) for k in ACT}
     g = ops.selective_scan_bwd(args["u"], args["delta"], x["A"], x["B"], x["C"],
                                to_bld(dout) if layout == "bld" else dout, D=x["D"], z=args["z"],
                                delta_bias=x["delta_bias"], initial_state=h0, dlast_state=dlast,
-                               zoh=zoh, layout=layout)
+                               zoh=zoh, layout=layout, softplus=softplus)
     torch.cuda.synchronize()
     assert ops.device_status() == 0
     if layout == "bld":
@@ -212,14 +212,31 @@ def test_backward_matches_standard_layout(dtype, shape, zoh):
         assert max_rel_err(a[k], b[k]) <= 1e-5, k
 
 
-def test_backward_against_oracle(ref):
-    x = layer_inputs(2, 64, 300, dtype=torch.float32, seed=23)
+@pytest.mark.parametrize("case", ["layer", "N4", "softplus_off", "plain", "zoh_start_state"])
+def test_backward_against_oracle(ref, case):
+    """fp32 inputs in (batch, seqlen, dim): every gradient against the
+    oracle (which takes (batch, dim, seqlen)), over the options: a state of 4
+    entries, softplus off (delta kept positive), no gate, D or bias, and the
+    zero-order hold from a start state with a last-state gradient."""
+    N = 4 if case == "N4" else 16
+    x = layer_inputs(2, 64, 300, dtype=torch.float32, seed=23, N=N)
+    softplus = case != "softplus_off"
+    if not softplus:
+        x["delta"] = x["delta"].abs() * 0.05
+        x["delta_bias"] = torch.full_like(x["delta_bias"], 0.01)
+    if case == "plain":
+        x["z"] = x["D"] = x["delta_bias"] = None
     g = torch.Generator(device=DEV)
     g.manual_seed(24)
     dout = torch.randn(2, 64, 300, generator=g, device=DEV)
-    got = backward(x, dout, "bld")
+    zoh = case == "zoh_start_state"
+    h0 = torch.randn(2, 64, N, generator=g, device=DEV) if zoh else None
+    dlast = torch.randn(2, 64, N, generator=g, device=DEV) if zoh else None
+    got = backward(x, dout, "bld", zoh=zoh, h0=h0, dlast=dlast, softplus=softplus)
     c = lambda t: None if t is None else t.cpu()  # noqa: E731
     o = ref.selective_scan_bwd(c(x["u"]), c(x["delta"]), c(x["A"]), c(x["B"]), c(x["C"]), dout.cpu(),
-                               D=c(x["D"]), z=c(x["z"]), delta_bias=c(x["delta_bias"]))
+                               D=c(x["D"]), z=c(x["z"]), delta_bias=c(x["delta_bias"]),
+                               softplus=softplus, initial_state=c(h0), dlast_state=c(dlast), zoh=zoh)
+    assert set(got) == set(o), (set(got), set(o))
     for k in o:
         assert max_rel_err(got[k], o[k]) <= FP32_TOL, k
