@@ -372,3 +372,18 @@ def test_binding_layout_argument():
     assert ops._layout_flags("bdl", 0) == (0, False)
     u = torch.empty(2, 7, 5)
     assert ops._scan_sizes(u, True) == (2, 5, 7) and ops._scan_sizes(u, False) == (2, 7, 5)
+
+
+def test_no_cpu_fallback(tmp_path, lib):
+    """A missing library is an error, and host tensors are refused rather
+    than computed on the CPU."""
+    with pytest.raises(RuntimeError, match="no CPU fallback"):
+        ops.library(tmp_path / "absent.so")
+    c = SCAN_CONFIGS["tiny_fp32"]
+    u = torch.zeros(c.batch, c.dim, c.seqlen)
+    A = -torch.ones(c.dim, c.dstate)
+    B = torch.zeros(c.batch, c.dstate, c.seqlen)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        ops.selective_scan_fwd(u, u, A, B, B)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        ops.selective_scan_bwd(u, u, A, B, B, u)
