@@ -417,7 +417,11 @@ mamba_status_t plan_scan(const mamba_dims_t* dims, int sm_count, mamba_scan_plan
         lanes = 2;
         groups_run = dims->batch * ((dims->dim + 15) / 16);
         if (dims->num_chunks < 1) {
-            K = std::max<int64_t>(1, std::min<int64_t>((8 * W + groups_run - 1) / groups_run,
+            // About 4 segments per resident warp of the two-lane kernel (8 x 4096
+            // x 2048: K = 4, measured faster than 8 or 12; 6 leaves a short
+            // last segment).
+            const int64_t W2 = (int64_t)sm_count * SplitLayout::kWarpsPerSm;
+            K = std::max<int64_t>(1, std::min<int64_t>((4 * W2 + groups_run - 1) / groups_run,
                                                        L / 256));
             segments(K, seg_len);
         }

@@ -196,7 +196,7 @@ def test_plan_layer_shapes(lib):
     c = SCAN_CONFIGS["mamba_1p4b_layer"]
     p = ops.scan_plan(c.batch, c.dim, c.dstate, c.seqlen, c.io_dtype, c.bc_dtype)
     assert p["mode"] == 0 and p["lanes_per_channel"] == 2 and p["groups"] == 2048
-    assert p["nchunks"] == 8 and p["max_warps"] == 148 * 12
+    assert p["nchunks"] == 4 and p["max_warps"] == 148 * 12
     assert p["workspace_bytes"] == 256 + 8192 + 8 * 4096 * 64
     q = ops.scan_plan(c.batch, c.dim, c.dstate, c.seqlen, c.io_dtype, c.bc_dtype,
                       flags=ops.MAMBA_FLAG_ONE_LANE_PER_CHANNEL)
